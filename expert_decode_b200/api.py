@@ -1,0 +1,174 @@
+"""ctypes binding of the C ABI in include/expert_decode.h.
+
+Argument marshalling only: each wrapper checks that the torch tensors have the
+layout the ABI documents, passes their device pointers and sizes, and raises
+EPError when the library returns a status other than EP_OK.  Outputs that the
+caller does not pass are allocated with torch (device memory is plumbing).
+The library must be present: there is no fallback of any kind.
+"""
+import ctypes
+import os
+import threading
+
+import torch
+
+EP_OK, EP_EINVAL, EP_EDIM, EP_EBADID, EP_ENOMEM, EP_ECUDA, EP_ETIMEOUT = range(7)
+EP_BF16, EP_F32 = 0, 1
+EP_MAX_BANDS = 64
+_DISPATCH = {"auto": 0, "streaming": 1, "tensor": 2}
+_NAMES = {0: "EP_OK", 1: "EP_EINVAL", 2: "EP_EDIM", 3: "EP_EBADID", 4: "EP_ENOMEM",
+          5: "EP_ECUDA", 6: "EP_ETIMEOUT"}
+
+library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib",
+                            "libexpert_decode.so")
+
+
+class EPError(RuntimeError):
+    def __init__(self, code, message):
+        super().__init__(f"{_NAMES.get(code, code)}: {message}")
+        self.code = code
+
+
+class Plan(ctypes.Structure):
+    _fields_ = [("num_experts", ctypes.c_int32), ("bands", ctypes.c_int32),
+                ("band_start", ctypes.c_int32 * (EP_MAX_BANDS + 1))]
+
+    def starts(self):
+        return [self.band_start[r] for r in range(self.bands + 1)]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def library():
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(library_path):
+                raise RuntimeError(f"CUDA library {library_path} is missing: build it with "
+                                   "`python -c 'import __graft_entry__ as g; g.build()'`")
+            lib = ctypes.CDLL(library_path)
+            P, I64, I32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+            lib.ep_plan.argtypes = [I32, I32, ctypes.POINTER(Plan)]
+            lib.moe_route.argtypes = [P, ctypes.c_int, I64, I64, P, P, I64, I32, P, P, P]
+            lib.moe_ffn_workspace_size.argtypes = [I64, I64, I64, I32, I64, I64]
+            lib.moe_ffn_workspace_size.restype = SZ
+            lib.moe_ffn_forward.argtypes = [P, ctypes.c_int, I64, I64, P, P, I32, P, P, P, I64,
+                                            I64, P, P, P, I64, ctypes.POINTER(Plan), P, P, SZ, P]
+            lib.ep_set_dispatch.argtypes = [ctypes.c_int]
+            lib.ep_check_status.argtypes = [P]
+            lib.ep_last_error.restype = ctypes.c_char_p
+            lib.ep_last_launch_count.restype = I32
+            for fn in ("ep_plan", "moe_route", "moe_ffn_forward", "ep_set_dispatch",
+                       "ep_check_status"):
+                getattr(lib, fn).restype = ctypes.c_int
+            _lib = lib
+        return _lib
+
+
+def _check(rc):
+    if rc != EP_OK:
+        raise EPError(rc, library().ep_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype(x):
+    if x.dtype == torch.bfloat16:
+        return EP_BF16
+    if x.dtype == torch.float32:
+        return EP_F32
+    raise TypeError(f"activations must be bf16 or fp32, got {x.dtype}")
+
+
+def _dense(t, name, dtype=None, ndim=None):
+    if t is None:
+        return
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (row-major)")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions")
+
+
+def ep_plan(num_experts, bands):
+    plan = Plan()
+    _check(library().ep_plan(int(num_experts), int(bands), ctypes.byref(plan)))
+    return plan
+
+
+def moe_route(x, w_router, bias, top_k, ids=None, weights=None, stream=None):
+    """ids [T, top_k] int32 and weights [T, top_k] fp32 of the replicated router."""
+    _dense(x, "x", ndim=2)
+    _dense(w_router, "w_router", torch.bfloat16, 2)
+    _dense(bias, "bias", torch.float32, 1)
+    T, H = x.shape
+    E = w_router.shape[0]
+    if ids is None:
+        ids = torch.empty((T, top_k), dtype=torch.int32, device=x.device)
+    if weights is None:
+        weights = torch.empty((T, top_k), dtype=torch.float32, device=x.device)
+    _dense(ids, "ids", torch.int32)
+    _dense(weights, "weights", torch.float32)
+    _check(library().moe_route(_ptr(x), _dtype(x), T, H, _ptr(w_router), _ptr(bias), E,
+                               int(top_k), _ptr(ids), _ptr(weights), _stream(stream)))
+    return ids, weights
+
+
+def moe_ffn_workspace_size(T, H, E, top_k, I, I_s):
+    return int(library().moe_ffn_workspace_size(int(T), int(H), int(E), int(top_k), int(I),
+                                                int(I_s)))
+
+
+def moe_ffn_forward(x, ids, weights, w_gate, w_up, w_down, shared, plan, y=None,
+                    workspace=None, stream=None):
+    """y [T, H] fp32 of the routed MoE FFN; shared = (ws_gate, ws_up, ws_down) or None."""
+    _dense(x, "x", ndim=2)
+    _dense(ids, "ids", torch.int32, 2)
+    _dense(weights, "weights", torch.float32, 2)
+    for name, t in (("w_gate", w_gate), ("w_up", w_up), ("w_down", w_down)):
+        _dense(t, name, torch.bfloat16, 3)
+    T, H = x.shape
+    top_k = ids.shape[1]
+    E, I = w_gate.shape[0], w_gate.shape[1]
+    if shared is not None:
+        ws_gate, ws_up, ws_down = shared
+        for name, t in (("ws_gate", ws_gate), ("ws_up", ws_up), ("ws_down", ws_down)):
+            _dense(t, name, torch.bfloat16, 2)
+        I_s = ws_gate.shape[0]
+    else:
+        ws_gate = ws_up = ws_down = None
+        I_s = 0
+    if y is None:
+        y = torch.empty((T, H), dtype=torch.float32, device=x.device)
+    _dense(y, "y", torch.float32, 2)
+    need = moe_ffn_workspace_size(T, H, E, top_k, I, I_s)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    _check(library().moe_ffn_forward(
+        _ptr(x), _dtype(x), T, H, _ptr(ids), _ptr(weights), top_k, _ptr(w_gate), _ptr(w_up),
+        _ptr(w_down), E, I, _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), I_s, ctypes.byref(plan),
+        _ptr(y), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return y
+
+
+def ep_check_status(stream=None):
+    _check(library().ep_check_status(_stream(stream)))
+
+
+def ep_set_dispatch(mode):
+    _check(library().ep_set_dispatch(_DISPATCH[mode]))
+
+
+def ep_last_launch_count():
+    return int(library().ep_last_launch_count())

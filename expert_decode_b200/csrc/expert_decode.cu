@@ -1,0 +1,406 @@
+// expert_decode.cu -- the C ABI (include/expert_decode.h): host-side
+// validation, the workspace layout, path dispatch and kernel launches.
+// Every kernel of the library is compiled into this one translation unit.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/expert_decode.h"
+#include "common.cuh"
+#include "router.cuh"
+#include "streaming.cuh"
+#include "grouped.cuh"
+
+namespace {
+
+thread_local char t_error[512] = "";
+thread_local int32_t t_launches = 0;
+std::atomic<int> g_dispatch{EP_DISPATCH_AUTO};
+
+ep_status fail(ep_status s, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(t_error, sizeof t_error, fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+ep_status ok() {
+    t_error[0] = '\0';
+    return EP_OK;
+}
+
+#define EP_CUDA_CHECK(call)                                                                    \
+    do {                                                                                       \
+        cudaError_t err_ = (call);                                                             \
+        if (err_ != cudaSuccess)                                                               \
+            return fail(EP_ECUDA, "%s failed: %s", #call, cudaGetErrorString(err_));           \
+    } while (0)
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+struct DeviceInfo {
+    bool ready = false;
+    int sm_count = 0;
+    int smem_optin = 0;
+};
+
+constexpr int kMaxDevices = 64;
+std::mutex g_device_mu;
+DeviceInfo g_devices[kMaxDevices];
+
+// Per device, once: SM count, shared-memory limit, kernel attributes.
+ep_status device_info(const DeviceInfo **out) {
+    int dev = 0;
+    EP_CUDA_CHECK(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices)
+        return fail(EP_ECUDA, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_device_mu);
+    DeviceInfo &d = g_devices[dev];
+    if (!d.ready) {
+        int major = 0;
+        EP_CUDA_CHECK(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+        if (major != 10)
+            return fail(EP_ECUDA, "device %d has compute capability %d.x; this library is built "
+                                  "for sm_100a (B200)", dev, major);
+        EP_CUDA_CHECK(cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev));
+        EP_CUDA_CHECK(
+            cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
+        const int m = d.smem_optin;
+        EP_CUDA_CHECK(cudaFuncSetAttribute(epk::router_topk_kernel<false>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, m));
+        EP_CUDA_CHECK(cudaFuncSetAttribute(epk::router_topk_kernel<true>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, m));
+        EP_CUDA_CHECK(cudaFuncSetAttribute(epk::stream_gate_up_kernel<false>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, m));
+        EP_CUDA_CHECK(cudaFuncSetAttribute(epk::stream_gate_up_kernel<true>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, m));
+        EP_CUDA_CHECK(cudaFuncSetAttribute(epk::stream_down_fold_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, m));
+        ep_status s = epk::grouped_set_attributes(m);
+        if (s != EP_OK)
+            return fail(s, "setting the grouped GEMM kernel attributes failed");
+        d.ready = true;
+    }
+    *out = &d;
+    return EP_OK;
+}
+
+constexpr int64_t kMaxT = 65536;
+constexpr int64_t kMaxPairs = 1 << 20;
+constexpr int64_t kMaxH = 16384;
+constexpr int64_t kMaxE = 1024;
+constexpr int64_t kMaxI = 16384;
+constexpr int kMaxTopK = 16;
+// Shared memory the streaming kernels may take, leaving the rest of the
+// SM's unified L1 for the activations they read through the cache.
+constexpr size_t kStreamSmemBudget = 200 * 1024;
+
+size_t align256(size_t v) { return (v + 255) / 256 * 256; }
+
+// ---------------------------------------------------------- workspace layout
+struct Workspace {
+    // streaming path (T <= 8)
+    size_t h_routed = 0, h_shared = 0;
+    // tensor path
+    epk::GroupedWorkspace grouped;
+    size_t total = 0;
+};
+
+Workspace workspace_layout(int64_t T, int64_t H, int64_t E, int64_t k, int64_t I, int64_t I_s) {
+    Workspace w;
+    size_t o = 0;
+    if (T <= epk::kStreamMaxT) {
+        w.h_routed = o;
+        o = align256(o + (size_t)T * k * I * 4);
+        w.h_shared = o;
+        o = align256(o + (size_t)T * I_s * 4);
+    }
+    w.grouped = epk::grouped_workspace_layout(o, T, H, E, k, I, I_s);
+    o = align256(w.grouped.end);
+    w.total = o;
+    return w;
+}
+
+// --------------------------------------------------------- streaming path fit
+struct StreamingPlan {
+    bool fits = false;
+    int gu_slots = 0, down_slots = 0, down_grid = 0, down_rows_max = 0;
+    size_t gu_smem = 0, down_smem = 0;
+};
+
+StreamingPlan streaming_fit(const DeviceInfo &d, int64_t T, int64_t H, int xb, int64_t k,
+                            int64_t I, int64_t I_s) {
+    StreamingPlan p;
+    if (T < 1 || T > epk::kStreamMaxT || k > epk::kStreamMaxK)
+        return p;
+    const size_t budget = std::min<size_t>(kStreamSmemBudget, (size_t)d.smem_optin);
+    int slots = epk::kGUMaxSlots;
+    while (slots >= 2 && epk::gate_up_smem_layout((int)T, (int)H, xb, slots).total > budget)
+        --slots;
+    if (slots < 2)
+        return p;
+    p.gu_slots = slots;
+    p.gu_smem = epk::gate_up_smem_layout((int)T, (int)H, xb, slots).total;
+    const int64_t I_max = std::max(I, I_s);
+    p.down_grid = (int)std::max<int64_t>(1, std::min<int64_t>(d.sm_count, H / 8));
+    p.down_rows_max = (int)((H + p.down_grid - 1) / p.down_grid);
+    slots = epk::kDownMaxSlots;
+    while (slots >= 2 &&
+           epk::down_smem_layout((int)I_max, slots, p.down_rows_max).total > budget)
+        --slots;
+    if (slots < 2)
+        return p;
+    p.down_slots = slots;
+    p.down_smem = epk::down_smem_layout((int)I_max, slots, p.down_rows_max).total;
+    p.fits = true;
+    return p;
+}
+
+}  // namespace
+
+// =========================================================================== ABI
+
+extern "C" ep_status ep_plan(int32_t num_experts, int32_t bands, ep_plan_t *out) {
+    if (out == nullptr)
+        return fail(EP_EINVAL, "ep_plan: out is NULL");
+    if (num_experts < 1)
+        return fail(EP_EINVAL, "ep_plan: num_experts = %d < 1", num_experts);
+    if (bands < 1 || bands > num_experts || bands > EP_MAX_BANDS)
+        return fail(EP_EINVAL, "ep_plan: bands = %d must be in [1, min(num_experts = %d, %d)]",
+                    bands, num_experts, EP_MAX_BANDS);
+    ep_plan_t p;
+    memset(&p, 0, sizeof p);
+    p.num_experts = num_experts;
+    p.bands = bands;
+    const int32_t base = num_experts / bands, extra = num_experts % bands;
+    p.band_start[0] = 0;
+    for (int32_t r = 0; r < bands; ++r)
+        p.band_start[r + 1] = p.band_start[r] + base + (r < extra ? 1 : 0);
+    *out = p;
+    return ok();
+}
+
+extern "C" ep_status ep_set_dispatch(ep_dispatch mode) {
+    if (mode != EP_DISPATCH_AUTO && mode != EP_DISPATCH_STREAMING && mode != EP_DISPATCH_TENSOR)
+        return fail(EP_EINVAL, "ep_set_dispatch: unknown mode %d", (int)mode);
+    g_dispatch.store((int)mode);
+    return ok();
+}
+
+extern "C" const char *ep_last_error(void) { return t_error; }
+
+extern "C" int32_t ep_last_launch_count(void) { return t_launches; }
+
+extern "C" ep_status ep_check_status(void *stream) {
+    EP_CUDA_CHECK(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+    unsigned int v = 0, zero = 0;
+    EP_CUDA_CHECK(cudaMemcpyFromSymbol(&v, epk::g_status, sizeof v));
+    EP_CUDA_CHECK(cudaMemcpyToSymbol(epk::g_status, &zero, sizeof zero));
+    if (v & epk::kStatusTimeout)
+        return fail(EP_ETIMEOUT, "a device-side wait ran out of time");
+    if (v & epk::kStatusBadId)
+        return fail(EP_EBADID, "an expert id outside [0, E) was skipped on the device");
+    return ok();
+}
+
+extern "C" ep_status moe_route(const void *x, ep_dtype x_dtype, int64_t T, int64_t H,
+                               const void *w_router, const float *bias, int64_t E,
+                               int32_t top_k, int32_t *ids, float *weights, void *stream) {
+    if (x_dtype != EP_BF16 && x_dtype != EP_F32)
+        return fail(EP_EINVAL, "moe_route: unknown x dtype %d", (int)x_dtype);
+    if (T < 0 || T > kMaxT)
+        return fail(EP_EINVAL, "moe_route: T = %lld outside [0, %lld]", (long long)T,
+                    (long long)kMaxT);
+    if (H < 8 || H > kMaxH || H % 8 != 0)
+        return fail(EP_EINVAL, "moe_route: H = %lld must be a multiple of 8 in [8, %lld]",
+                    (long long)H, (long long)kMaxH);
+    if (E < 1 || E > kMaxE)
+        return fail(EP_EINVAL, "moe_route: E = %lld outside [1, %lld]", (long long)E,
+                    (long long)kMaxE);
+    if (top_k < 1 || top_k > kMaxTopK || top_k > E)
+        return fail(EP_EINVAL, "moe_route: top_k = %d outside [1, min(E, %d)]", top_k, kMaxTopK);
+    if (T == 0) {
+        t_launches = 0;
+        return ok();
+    }
+    if (x == nullptr || w_router == nullptr || ids == nullptr || weights == nullptr)
+        return fail(EP_EINVAL, "moe_route: NULL x, w_router, ids or weights");
+    if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(ids, 4) || !aligned(weights, 4) ||
+        (bias != nullptr && !aligned(bias, 4)))
+        return fail(EP_EINVAL, "moe_route: misaligned pointer (x, w_router need 16 bytes)");
+    const DeviceInfo *d = nullptr;
+    ep_status s = device_info(&d);
+    if (s != EP_OK)
+        return s;
+    const int xb = x_dtype == EP_F32 ? 4 : 2;
+    const int tb_max =
+        (int)std::max<int64_t>(1, std::min<int64_t>(epk::kRouterMaxTB, epk::kRouterXBudget / (H * xb)));
+    const epk::RouterSmem L = epk::router_smem_layout(tb_max, (int)H, xb, (int)E);
+    if ((int)L.total > d->smem_optin)
+        return fail(EP_EINVAL, "moe_route: H = %lld, E = %lld need %u bytes of shared memory",
+                    (long long)H, (long long)E, L.total);
+    const int64_t nblk = (T + tb_max - 1) / tb_max;
+    const dim3 grid((unsigned)(nblk * epk::kRouterCluster));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (x_dtype == EP_F32)
+        epk::router_topk_kernel<true><<<grid, epk::kRouterThreads, L.total, st>>>(
+            x, T, (int)H, static_cast<const uint16_t *>(w_router), bias, (int)E, top_k, tb_max,
+            ids, weights);
+    else
+        epk::router_topk_kernel<false><<<grid, epk::kRouterThreads, L.total, st>>>(
+            x, T, (int)H, static_cast<const uint16_t *>(w_router), bias, (int)E, top_k, tb_max,
+            ids, weights);
+    EP_CUDA_CHECK(cudaGetLastError());
+    t_launches = 1;
+    return ok();
+}
+
+extern "C" size_t moe_ffn_workspace_size(int64_t T, int64_t H, int64_t E, int32_t top_k,
+                                         int64_t I, int64_t I_s) {
+    if (T <= 0 || H <= 0 || E <= 0 || top_k <= 0 || I <= 0 || I_s < 0)
+        return 0;
+    return workspace_layout(T, H, E, top_k, I, I_s).total;
+}
+
+extern "C" ep_status moe_ffn_forward(const void *x, ep_dtype x_dtype, int64_t T, int64_t H,
+                                     const int32_t *ids, const float *weights, int32_t top_k,
+                                     const void *w_gate, const void *w_up, const void *w_down,
+                                     int64_t E, int64_t I, const void *ws_gate,
+                                     const void *ws_up, const void *ws_down, int64_t I_s,
+                                     const ep_plan_t *plan, float *y, void *workspace,
+                                     size_t workspace_bytes, void *stream) {
+    // ---- validation: nothing is launched and nothing written on failure
+    if (plan == nullptr)
+        return fail(EP_EINVAL, "moe_ffn_forward: plan is NULL");
+    if (plan->num_experts != E)
+        return fail(EP_EDIM, "moe_ffn_forward: plan covers %d experts, E = %lld",
+                    plan->num_experts, (long long)E);
+    if (plan->bands < 1 || plan->bands > EP_MAX_BANDS || plan->bands > E ||
+        plan->band_start[0] != 0 || plan->band_start[plan->bands] != E)
+        return fail(EP_EINVAL, "moe_ffn_forward: plan is not a partition of [0, E)");
+    for (int r = 0; r < plan->bands; ++r)
+        if (plan->band_start[r + 1] <= plan->band_start[r])
+            return fail(EP_EINVAL, "moe_ffn_forward: band %d of the plan is empty or reversed", r);
+    if (x_dtype != EP_BF16 && x_dtype != EP_F32)
+        return fail(EP_EINVAL, "moe_ffn_forward: unknown x dtype %d", (int)x_dtype);
+    if (T < 0 || T > kMaxT || T * (int64_t)std::max(top_k, 1) > kMaxPairs)
+        return fail(EP_EINVAL, "moe_ffn_forward: T = %lld out of range", (long long)T);
+    if (H < 8 || H > kMaxH || H % 8 != 0)
+        return fail(EP_EINVAL, "moe_ffn_forward: H = %lld must be a multiple of 8 in [8, %lld]",
+                    (long long)H, (long long)kMaxH);
+    if (E < 1 || E > kMaxE)
+        return fail(EP_EINVAL, "moe_ffn_forward: E = %lld outside [1, %lld]", (long long)E,
+                    (long long)kMaxE);
+    if (top_k < 1 || top_k > kMaxTopK || top_k > E)
+        return fail(EP_EINVAL, "moe_ffn_forward: top_k = %d outside [1, min(E, %d)]", top_k,
+                    kMaxTopK);
+    if (I < 8 || I > kMaxI || I % 8 != 0)
+        return fail(EP_EINVAL, "moe_ffn_forward: I = %lld must be a multiple of 8 in [8, %lld]",
+                    (long long)I, (long long)kMaxI);
+    if (I_s != 0 && (I_s < 8 || I_s > kMaxI || I_s % 8 != 0))
+        return fail(EP_EINVAL, "moe_ffn_forward: I_s = %lld must be 0 or a multiple of 8 in "
+                               "[8, %lld]", (long long)I_s, (long long)kMaxI);
+    if (T == 0) {
+        t_launches = 0;
+        return ok();
+    }
+    if (x == nullptr || ids == nullptr || weights == nullptr || w_gate == nullptr ||
+        w_up == nullptr || w_down == nullptr || y == nullptr)
+        return fail(EP_EINVAL, "moe_ffn_forward: a required pointer is NULL");
+    if ((I_s > 0) != (ws_gate != nullptr) || (I_s > 0) != (ws_up != nullptr) ||
+        (I_s > 0) != (ws_down != nullptr))
+        return fail(EP_EINVAL, "moe_ffn_forward: shared-expert pointers must all be set iff "
+                               "I_s > 0");
+    const void *al16[] = {x, w_gate, w_up, w_down, y, ws_gate, ws_up, ws_down};
+    for (const void *p : al16)
+        if (p != nullptr && !aligned(p, 16))
+            return fail(EP_EINVAL, "moe_ffn_forward: a tensor is not 16-byte aligned");
+    if (!aligned(ids, 4) || !aligned(weights, 4))
+        return fail(EP_EINVAL, "moe_ffn_forward: ids / weights not 4-byte aligned");
+    const Workspace W = workspace_layout(T, H, E, top_k, I, I_s);
+    if (workspace == nullptr || workspace_bytes < W.total)
+        return fail(EP_ENOMEM, "moe_ffn_forward: workspace of %zu bytes, %zu needed",
+                    workspace_bytes, W.total);
+    if (!aligned(workspace, 256))
+        return fail(EP_EINVAL, "moe_ffn_forward: workspace not 256-byte aligned");
+    const DeviceInfo *d = nullptr;
+    ep_status s = device_info(&d);
+    if (s != EP_OK)
+        return s;
+
+    const int xb = x_dtype == EP_F32 ? 4 : 2;
+    const StreamingPlan sp = streaming_fit(*d, T, H, xb, top_k, I, I_s);
+    const int mode = g_dispatch.load();
+    bool use_streaming;
+    if (mode == EP_DISPATCH_STREAMING) {
+        if (!sp.fits)
+            return fail(EP_EINVAL, "moe_ffn_forward: the streaming path does not fit these sizes");
+        use_streaming = true;
+    } else if (mode == EP_DISPATCH_TENSOR) {
+        use_streaming = false;
+    } else {
+        use_streaming = sp.fits;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+
+    if (use_streaming) {
+        epk::StreamGateUpArgs ga;
+        ga.x = x;
+        ga.T = (int)T; ga.H = (int)H; ga.E = (int)E; ga.I = (int)I; ga.I_s = (int)I_s;
+        ga.top_k = top_k; ga.n_slots = sp.gu_slots;
+        ga.w_gate = static_cast<const uint16_t *>(w_gate);
+        ga.w_up = static_cast<const uint16_t *>(w_up);
+        ga.ws_gate = static_cast<const uint16_t *>(ws_gate);
+        ga.ws_up = static_cast<const uint16_t *>(ws_up);
+        ga.ids = ids;
+        ga.weights = weights;
+        ga.h_routed = reinterpret_cast<float *>(ws + W.h_routed);
+        ga.h_shared = reinterpret_cast<float *>(ws + W.h_shared);
+        const dim3 gu_grid((unsigned)d->sm_count);
+        if (x_dtype == EP_F32)
+            epk::stream_gate_up_kernel<true><<<gu_grid, epk::kGUThreads, sp.gu_smem, st>>>(ga);
+        else
+            epk::stream_gate_up_kernel<false><<<gu_grid, epk::kGUThreads, sp.gu_smem, st>>>(ga);
+        EP_CUDA_CHECK(cudaGetLastError());
+
+        epk::StreamDownArgs da;
+        da.T = (int)T; da.H = (int)H; da.E = (int)E; da.I = (int)I; da.I_s = (int)I_s;
+        da.top_k = top_k; da.n_slots = sp.down_slots; da.rows_max = sp.down_rows_max;
+        da.w_down = static_cast<const uint16_t *>(w_down);
+        da.ws_down = static_cast<const uint16_t *>(ws_down);
+        da.ids = ids;
+        da.weights = weights;
+        da.h_routed = ga.h_routed;
+        da.h_shared = ga.h_shared;
+        da.y = y;
+        epk::stream_down_fold_kernel<<<sp.down_grid, epk::kDownThreads, sp.down_smem, st>>>(da);
+        EP_CUDA_CHECK(cudaGetLastError());
+        t_launches = 2;
+        return ok();
+    }
+
+    epk::GroupedArgs g;
+    g.x = x; g.x_f32 = x_dtype == EP_F32;
+    g.T = T; g.H = H; g.E = E; g.I = I; g.I_s = I_s; g.top_k = top_k;
+    g.ids = ids; g.weights = weights;
+    g.w_gate = w_gate; g.w_up = w_up; g.w_down = w_down;
+    g.ws_gate = ws_gate; g.ws_up = ws_up; g.ws_down = ws_down;
+    g.y = y;
+    g.sm_count = d->sm_count;
+    g.smem_optin = d->smem_optin;
+    int launches = 0;
+    char why[256] = "";
+    s = epk::grouped_forward(g, W.grouped, ws, st, &launches, why, sizeof why);
+    if (s != EP_OK)
+        return fail(s, "moe_ffn_forward: %s", why);
+    t_launches = launches;
+    return ok();
+}

@@ -1,0 +1,177 @@
+/*
+ * expert_decode.h -- C ABI of the B200 (sm_100a) routed MoE FFN with an
+ * expert-parallel band decomposition.
+ *
+ * The operation.  A replicated router picks the same top-k experts for every
+ * rank; the experts are split into contiguous bands, one band per rank, and
+ * each band's SwiGLU experts contribute an [H] partial that is summed in rank
+ * order (fak note "GLM-5.2 multi-GPU: expert-parallel sharding + the
+ * resident-fit benchmark", section "What landed": ExpertParallelPlan, one
+ * AllReduceSum of the per-rank partials; TensorFold issue #214 "GLM-5.3-Flash
+ * on CUDA: attention on one GPU, routed experts on the Sparks", "Per MoE
+ * layer": rows, top-k ids and weights in, partials out, summed in rank
+ * order).  On one GPU the bands are a logical partition only.
+ *
+ * Conventions shared by every entry point:
+ *  - Ownership.  The caller allocates and owns every buffer, including the
+ *    workspace; the library allocates no device memory and frees nothing.
+ *  - Layout.  Device arrays are dense, row-major, and their base addresses are
+ *    16-byte aligned (the workspace 256-byte aligned).  bf16 is IEEE
+ *    bfloat16 (the upper 16 bits of a binary32).
+ *  - Streams.  `stream` is a cudaStream_t (NULL = the legacy default stream).
+ *    Calls are asynchronous on that stream and never synchronise the host,
+ *    except ep_check_status().
+ *  - Errors.  Arguments are validated on the host before anything is
+ *    launched; on any error status nothing is launched and no output is
+ *    written.  ep_last_error() gives the reason (per host thread).  Errors
+ *    found on the device (an expert id outside [0, E)) never trap and never
+ *    read out of bounds: the pick is skipped, a sticky device status word is
+ *    set, and ep_check_status() reports it.
+ *  - Thread safety.  Every function may be called from several host threads.
+ */
+#ifndef EXPERT_DECODE_H
+#define EXPERT_DECODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    EP_OK = 0,
+    EP_EINVAL = 1,    /* bad size, null or misaligned pointer, bad plan layout */
+    EP_EDIM = 2,      /* plan does not match the expert count (plan.Dim != NumExperts) */
+    EP_EBADID = 3,    /* device side: an expert id outside [0, E) was skipped */
+    EP_ENOMEM = 4,    /* the workspace is smaller than moe_ffn_workspace_size() */
+    EP_ECUDA = 5,     /* a CUDA runtime call failed; ep_last_error() has its text */
+    EP_ETIMEOUT = 6   /* device side: a bounded wait ran out */
+} ep_status;
+
+typedef enum { EP_BF16 = 0, EP_F32 = 1 } ep_dtype;
+
+#define EP_MAX_BANDS 64
+
+/*
+ * ExpertParallelPlan(numExperts, ranks): contiguous bands over [0, E), band r
+ * = [band_start[r], band_start[r+1]) (fak note "GLM-5.2 multi-GPU", "What
+ * landed").  Band sizes follow the shard rule of TensorFold issue #310
+ * ("GLM-5.3-Flash on CUDA over three ranks (--tp 3)", MiaAI-Lab's proposal,
+ * shares.py): whole experts, as even as they go, the first E % bands bands
+ * taking one more (largest remainder, ties to the lower rank).
+ */
+typedef struct {
+    int32_t num_experts;
+    int32_t bands;
+    int32_t band_start[EP_MAX_BANDS + 1];
+} ep_plan_t;
+
+/*
+ * ep_plan -- build the plan on the host.  Refused with EP_EINVAL (and *out
+ * untouched) when num_experts < 1, bands < 1, bands > num_experts (the fak
+ * note's fail-closed gate: "ranks > experts") or bands > EP_MAX_BANDS.
+ */
+ep_status ep_plan(int32_t num_experts, int32_t bands, ep_plan_t *out);
+
+/*
+ * moe_route -- the replicated router (fak note "GLM-5.2 multi-GPU", "What
+ * landed": the router runs replicated and picks the same top-k).
+ *   l[t,e] = sum_h x[t,h] * W_router[e,h] + bias[e]
+ *   p = softmax(l); S = the top_k experts by logit, ties to the lower id;
+ *   weights[t,j] = p[S_j] / sum_{e in S} p[e]
+ * ids[t,:] are written in descending weight order (equal weights: ascending
+ * id).  The selection and the weights are decided on fp64 logits: logits are
+ * first accumulated in fp32 with a proven error bound, and every expert that
+ * could be in the top-k under that bound is recomputed in fp64 before the
+ * pick, so the result equals the exact-arithmetic top-k up to fp64 rounding.
+ *
+ *   x         device, [T, H], bf16 (EP_BF16) or fp32 (EP_F32)
+ *   w_router  device, [E, H] bf16, one row per expert
+ *   bias      device, [E] fp32, or NULL for none (added to the logits)
+ *   ids       device, [T, top_k] int32 (output)
+ *   weights   device, [T, top_k] fp32 (output)
+ * Limits: 0 <= T <= 65536 (T = 0 is a no-op), 8 <= H <= 16384 with H % 8 ==
+ * 0, 1 <= E <= 1024, 1 <= top_k <= min(E, 16).
+ */
+ep_status moe_route(const void *x, ep_dtype x_dtype, int64_t T, int64_t H,
+                    const void *w_router, const float *bias, int64_t E, int32_t top_k,
+                    int32_t *ids, float *weights, void *stream);
+
+/*
+ * moe_ffn_workspace_size -- bytes of device workspace moe_ffn_forward needs
+ * for these sizes (0 when T = 0).  The workspace holds the token grouping,
+ * the grouped activations and the per-pick partial outputs; its contents on
+ * entry do not matter.
+ */
+size_t moe_ffn_workspace_size(int64_t T, int64_t H, int64_t E, int32_t top_k, int64_t I,
+                              int64_t I_s);
+
+/*
+ * moe_ffn_forward -- the routed MoE FFN with the shared expert.
+ * For every token t and pick j (e = ids[t,j], w = weights[t,j]):
+ *   f_e(x) = W_down[e] (silu(W_gate[e] x) * (W_up[e] x)),  silu(g) = g/(1+e^-g)
+ *   (expertSwiGLU, fak note "GLM-5.2 multi-GPU", "What is not yet" update)
+ *   y[t] = fold over the picks in ascending (expert id, j) of w * f_e(x[t]),
+ *          then + f_shared(x[t]) when I_s > 0.
+ * The fold runs band by band in rank order and passes its running sum from
+ * one band to the next, so it is one fixed sum order whatever the plan
+ * (TensorFold #310, maintainer's reply: every sum follows one fixed tree of
+ * slices however the slices fall over ranks): y is bit-identical for every
+ * plan and from run to run.
+ *
+ *   x        device, [T, H], bf16 or fp32
+ *   ids      device, [T, top_k] int32 expert ids (any order, repeats allowed)
+ *   weights  device, [T, top_k] fp32 routing weights
+ *   w_gate, w_up  device, [E, I, H] bf16 (row i of expert e = one unit of I)
+ *   w_down   device, [E, H, I] bf16 (row r of expert e = one output feature)
+ *   ws_gate, ws_up  device, [I_s, H] bf16; ws_down device, [H, I_s] bf16;
+ *            all three NULL when I_s = 0 (no shared expert)
+ *   plan     host, must satisfy plan->num_experts == E (else EP_EDIM) and be
+ *            a valid contiguous partition of [0, E) (else EP_EINVAL)
+ *   y        device, [T, H] fp32 (output)
+ *   workspace device, >= moe_ffn_workspace_size(T, H, E, top_k, I, I_s) bytes
+ *            (else EP_ENOMEM), 256-byte aligned
+ * Limits: 0 <= T <= 65536, T * top_k <= 2^20; 8 <= H <= 16384; 1 <= E <= 1024;
+ * 1 <= top_k <= min(E, 16); 8 <= I, I_s <= 16384 (I_s may be 0); H, I and
+ * I_s multiples of 8.
+ * Precision: bf16 products, fp32 accumulation.  Up to 8 rows the weights are
+ * streamed by a CUDA-core path that keeps the SwiGLU activations in fp32;
+ * above that, tensor-core tiles round the activations to bf16 between the
+ * two projections.
+ */
+ep_status moe_ffn_forward(const void *x, ep_dtype x_dtype, int64_t T, int64_t H,
+                          const int32_t *ids, const float *weights, int32_t top_k,
+                          const void *w_gate, const void *w_up, const void *w_down,
+                          int64_t E, int64_t I,
+                          const void *ws_gate, const void *ws_up, const void *ws_down,
+                          int64_t I_s, const ep_plan_t *plan, float *y,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Which moe_ffn_forward path runs.  EP_DISPATCH_AUTO (the default) takes the
+ * weight-streaming path for T <= 8 when its on-chip buffers fit, else the
+ * tensor-core path.  Forcing a path that does not fit the sizes makes
+ * moe_ffn_forward return EP_EINVAL.  Process-wide; meant for tests and tuning.
+ */
+typedef enum { EP_DISPATCH_AUTO = 0, EP_DISPATCH_STREAMING = 1, EP_DISPATCH_TENSOR = 2 } ep_dispatch;
+ep_status ep_set_dispatch(ep_dispatch mode);
+
+/*
+ * ep_check_status -- synchronise `stream`, then return and clear the sticky
+ * device status of the current device: EP_OK, EP_EBADID or EP_ETIMEOUT
+ * (EP_ECUDA if the synchronisation itself failed).
+ */
+ep_status ep_check_status(void *stream);
+
+/* Text of the last error on the calling host thread ("" if none). */
+const char *ep_last_error(void);
+
+/* Number of kernels the last successful call on this host thread launched. */
+int32_t ep_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXPERT_DECODE_H */

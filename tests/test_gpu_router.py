@@ -1,0 +1,84 @@
+"""moe_route on the GPU against the fp64 oracle: ids exact (barring ties within
+1e-6 of the oracle's own logits), weights within 1e-6, run-to-run identical."""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+import expert_decode_b200 as ed
+from gpu_parity import check_route, device_inputs, oracle_route
+
+pytestmark = pytest.mark.gpu
+WL = workloads.WORKLOADS
+
+
+def _route_and_check(o, wl, T, rows=None, seed=workloads.SEED_BASE, **sizes):
+    W, x = device_inputs(wl, T, seed=seed, **sizes)
+    ids, w = ed.moe_route(x, W["w_router"], W["bias"], wl.top_k)
+    ids2, w2 = ed.moe_route(x, W["w_router"], W["bias"], wl.top_k)
+    torch.cuda.synchronize()
+    assert torch.equal(ids, ids2) and torch.equal(w, w2), "router not run-to-run identical"
+    ed.ep_check_status()
+    ids_ref, w_ref, logits = oracle_route(o, x, W, wl.top_k, rows=rows)
+    if rows is not None:
+        ids, w = ids[rows], w[rows]
+    return check_route(ids, w, ids_ref, w_ref, logits)
+
+
+@pytest.mark.parametrize("T", [1, 4, 8])
+def test_router_decode(oracle_lib, T):
+    _route_and_check(oracle_lib, WL["decode"], T)
+
+
+def test_router_tiny_fp32_x(oracle_lib):
+    _route_and_check(oracle_lib, WL["tiny"], 4)
+
+
+def test_router_prefill_full(oracle_lib):
+    _route_and_check(oracle_lib, WL["prefill"], 512)
+
+
+def test_router_imbalanced_full(oracle_lib):
+    excused = _route_and_check(oracle_lib, WL["imbalanced"], 2048)
+    assert excused == 0
+
+
+def test_router_large_sampled(oracle_lib):
+    T = 4096
+    rows = np.r_[0:16, 16:T - 16:61, T - 16:T]
+    _route_and_check(oracle_lib, WL["large"], T, rows=rows)
+
+
+@pytest.mark.parametrize("T", [3, 13, 17])
+def test_router_ragged_token_blocks(oracle_lib, T):
+    _route_and_check(oracle_lib, WL["decode"], T, seed=77)
+
+
+def test_router_odd_sizes(oracle_lib):
+    wl = workloads.Workload("odd", (5,), 200, 37, 5, 16, 0, "bf16", "zipf1.1", (1,))
+    _route_and_check(oracle_lib, wl, 11, seed=5)
+
+
+def test_router_max_experts_and_top_k(oracle_lib):
+    wl = workloads.Workload("wide", (3,), 512, 1024, 16, 16, 0, "bf16", "none", (1,))
+    _route_and_check(oracle_lib, wl, 3, seed=9)
+
+
+def test_router_all_equal_logits():
+    """Zero router weights: every logit ties; ids 0..k-1, weights 1/k (the
+    candidate set exceeds the parallel budget, so the streaming fallback runs)."""
+    E, H, k, T = 128, 256, 8, 3
+    x = torch.randn(T, H, device="cuda").to(torch.bfloat16)
+    w = torch.zeros(E, H, device="cuda", dtype=torch.bfloat16)
+    ids, wts = ed.moe_route(x, w, None, k)
+    torch.cuda.synchronize()
+    assert ids.cpu().tolist() == [list(range(k))] * T
+    assert torch.all(wts.cpu() == 1.0 / k)
+
+
+def test_router_empty_is_a_no_op():
+    x = torch.empty((0, 256), device="cuda", dtype=torch.bfloat16)
+    w = torch.randn(16, 256, device="cuda").to(torch.bfloat16)
+    ids = torch.full((0, 4), -7, dtype=torch.int32, device="cuda")
+    ed.moe_route(x, w, None, 4, ids=ids)
+    assert ed.ep_last_launch_count() == 0

@@ -1,0 +1,124 @@
+"""The weight-streaming path (T <= 8) of moe_ffn_forward against the fp64 oracle,
+with the bit-identity the method promises: across runs and across band counts."""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+import expert_decode_b200 as ed
+from gpu_parity import check_y, device_inputs, gpu_ffn, oracle_ffn, oracle_route
+
+pytestmark = pytest.mark.gpu
+WL = workloads.WORKLOADS
+
+
+@pytest.fixture(autouse=True)
+def streaming_dispatch():
+    ed.ep_set_dispatch("streaming")
+    yield
+    ed.ep_set_dispatch("auto")
+
+
+def _routed(o, wl, T, seed=workloads.SEED_BASE, batch=0, **sizes):
+    W, x = device_inputs(wl, T, seed=seed, batch=batch, **sizes)
+    ids_ref, w_ref, _ = oracle_route(o, x, W, wl.top_k)
+    ids = torch.from_numpy(ids_ref).cuda()
+    w = torch.from_numpy(w_ref.astype(np.float32)).cuda()
+    return W, x, ids, w
+
+
+def test_tiny_all_band_counts(oracle_lib):
+    wl = WL["tiny"]
+    W, x, ids, w = _routed(oracle_lib, wl, 4)
+    ys = {}
+    for R in wl.bands + (8, 16):
+        ys[R] = gpu_ffn(x, ids, w, W, ed.ep_plan(wl.E, R))
+        ed.ep_check_status()
+        ref = oracle_ffn(oracle_lib, x, ids, w, W, bands=oracle_lib.expert_parallel_plan(wl.E, R))
+        check_y(ys[R], ref, what=f"tiny bands={R}")
+    mono = oracle_ffn(oracle_lib, x, ids, w, W)
+    check_y(ys[1], mono, rel_tol=1e-4, what="tiny vs monolith")
+    for R, y in ys.items():
+        assert torch.equal(y, ys[1]), f"bands={R} differs from bands=1"
+
+
+@pytest.mark.parametrize("T", [1, 4, 8])
+def test_decode_full_size(oracle_lib, T):
+    wl = WL["decode"]
+    W, x, ids, w = _routed(oracle_lib, wl, T)
+    plan = ed.ep_plan(wl.E, 8)
+    y = gpu_ffn(x, ids, w, W, plan)
+    ed.ep_check_status()
+    check_y(y, oracle_ffn(oracle_lib, x, ids, w, W), rel_tol=1e-4, what=f"decode T={T}")
+    check_y(y, oracle_ffn(oracle_lib, x, ids, w, W, bands=plan.starts()),
+            what=f"decode T={T} vs EP(8)")
+    for R in (1, 2, 4):
+        assert torch.equal(gpu_ffn(x, ids, w, W, ed.ep_plan(wl.E, R)), y)
+    assert torch.equal(gpu_ffn(x, ids, w, W, plan), y), "not run-to-run identical"
+
+
+def test_decode_end_to_end_with_gpu_router(oracle_lib):
+    wl = WL["decode"]
+    W, x = device_inputs(wl, 8, batch=3)
+    ids, w = ed.moe_route(x, W["w_router"], W["bias"], wl.top_k)
+    y = gpu_ffn(x, ids, w, W, ed.ep_plan(wl.E, 8))
+    ids_ref, w_ref, _ = oracle_route(oracle_lib, x, W, wl.top_k)
+    assert np.array_equal(ids.cpu().numpy(), ids_ref)
+    check_y(y, oracle_ffn(oracle_lib, x, ids_ref, w_ref, W), rel_tol=1e-4, what="decode e2e")
+
+
+def test_odd_sizes_and_max_pairs(oracle_lib):
+    wl = workloads.Workload("odd", (8,), 200, 23, 16, 72, 40, "bf16", "none", (1,))
+    W, x, ids, w = _routed(oracle_lib, wl, 8, seed=21)
+    y = gpu_ffn(x, ids, w, W, ed.ep_plan(wl.E, 5))
+    check_y(y, oracle_ffn(oracle_lib, x, ids, w, W), rel_tol=1e-4, what="odd sizes, 128 picks")
+
+
+def test_no_shared_expert(oracle_lib):
+    wl = WL["imbalanced"]
+    W, x, ids, w = _routed(oracle_lib, wl, 5, H=512, I=64, seed=4)
+    assert W["ws_gate"] is None
+    y = gpu_ffn(x, ids, w, W, ed.ep_plan(wl.E, 4))
+    y1 = gpu_ffn(x, ids, w, W, ed.ep_plan(wl.E, 1))
+    assert torch.equal(y, y1)
+    assert int(ids.max()) < 16
+    check_y(y, oracle_ffn(oracle_lib, x, ids, w, W), rel_tol=1e-4, what="imbalanced, small")
+
+
+def test_repeated_expert_in_one_token(oracle_lib):
+    wl = WL["tiny"]
+    W, x, ids, w = _routed(oracle_lib, wl, 4, seed=8)
+    ids[1, 2] = ids[1, 0]          # token 1 picks one expert twice
+    ids[3, :] = ids[3, 1]          # token 3 picks one expert four times
+    y = gpu_ffn(x, ids, w, W, ed.ep_plan(wl.E, 2))
+    check_y(y, oracle_ffn(oracle_lib, x, ids, w, W), rel_tol=1e-4, what="repeated picks")
+
+
+def test_bad_ids_are_skipped_and_reported(oracle_lib):
+    wl = WL["tiny"]
+    W, x, ids, w = _routed(oracle_lib, wl, 4, seed=12)
+    ed.ep_check_status()
+    bad = ids.clone()
+    bad[0, 1] = -1
+    bad[2, 3] = wl.E
+    y = gpu_ffn(x, bad, w, W, ed.ep_plan(wl.E, 1))
+    with pytest.raises(ed.EPError) as ei:
+        ed.ep_check_status()
+    assert ei.value.code == ed.EP_EBADID
+    ed.ep_check_status()  # cleared
+    # the skipped picks contribute nothing: same as a valid pick with weight 0
+    ref_ids, ref_w = ids.clone(), w.clone()
+    ref_w[0, 1] = 0.0
+    ref_w[2, 3] = 0.0
+    check_y(y, oracle_ffn(oracle_lib, x, ref_ids, ref_w, W), rel_tol=1e-4, what="bad ids")
+
+
+def test_empty_batch_is_a_no_op():
+    wl = WL["tiny"]
+    W, _ = device_inputs(wl, 1)
+    x = torch.empty((0, wl.H), device="cuda", dtype=torch.float32)
+    ids = torch.empty((0, wl.top_k), device="cuda", dtype=torch.int32)
+    w = torch.empty((0, wl.top_k), device="cuda", dtype=torch.float32)
+    y = gpu_ffn(x, ids, w, W, ed.ep_plan(wl.E, 1))
+    assert y.shape == (0, wl.H)
+    assert ed.ep_last_launch_count() == 0
