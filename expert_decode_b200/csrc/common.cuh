@@ -40,6 +40,9 @@ __device__ __forceinline__ uint16_t f32_to_bf16_rne(float f) {
     return (uint16_t)(u >> 16);
 }
 
+// silu(g) = g / (1 + e^-g), the SwiGLU gate activation.
+__device__ __forceinline__ float silu_f32(float g) { return g / (1.0f + expf(-g)); }
+
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return (uint32_t)__cvta_generic_to_shared(p);
 }

@@ -1,0 +1,818 @@
+// grouped.cuh -- the tensor-core path of the routed MoE FFN (more than 8 rows).
+//
+//  1. group_plan    (one CTA): the picks grouped by expert with a warp-level
+//                   histogram (__match_any_sync) and prefix scans; a stable
+//                   scatter keeps each expert's rows in (token, slot) order.
+//                   This is the batched expert dispatch of the fak note
+//                   "GLM-5.2 multi-GPU" (hostBatchedGLMExperts: run each
+//                   expert once over the rows that picked it).
+//  2. gather_rows:  the picked activation rows, expert by expert, as bf16,
+//                   followed by every token's row for the shared expert.
+//  3. grouped GEMM, gate/up: per (expert, 64 units of I, up to 256 rows) tile
+//                   one 128-row tcgen05 MMA stack whose A tile interleaves 16
+//                   W_gate rows and 16 W_up rows (the fused gate/up row of
+//                   TensorFold #593's packGateUp), so that a warp's lanes l and
+//                   l + 16 hold g and u of the same unit; the epilogue forms
+//                   h = silu(g) * u and rounds it to bf16.
+//  4. grouped GEMM, down: per (expert, 128 output features, up to 256 rows)
+//                   tile; the epilogue scales by the routing weight and writes
+//                   each pick's fp32 contribution to its (token, slot) row.
+//  5. combine:      y[t] = fold of the contributions in ascending (expert id,
+//                   slot) -- the band partials in rank order with the carry
+//                   passed along, one fixed order whatever the plan -- then
+//                   plus the shared expert's output.
+//
+// The GEMMs are persistent and warp specialised: warp 0 issues TMA loads
+// (cp.async.bulk.tensor, 128-byte swizzle, no multicast) into a 4-stage
+// shared-memory ring, warp 1 issues tcgen05.mma with the fp32 accumulator in
+// tensor memory (two accumulators, so the epilogue of one tile overlaps the
+// MMAs of the next), and warps 2..5 drain the accumulator with tcgen05.ld.
+// Weights sit on the MMA's M side (128 rows) and the expert's tokens on the
+// N side (16..256), so a tile is never padded to 128 tokens.
+#pragma once
+
+#include <cudaTypedefs.h>
+#include <cstdio>
+
+#include "common.cuh"
+
+namespace epk {
+
+constexpr int kGemmBM = 128;
+constexpr int kGemmBN = 256;
+constexpr int kGemmBK = 64;
+constexpr int kGemmStages = 4;
+constexpr int kGemmThreads = 192;
+constexpr int kGateUpRows = 64;  // units of I per gate/up tile (64 gate + 64 up rows)
+constexpr int kBoxRowsA = 16;    // gate/up A tile is loaded 16 rows at a time
+constexpr int kBoxRowsB = 32;
+constexpr uint32_t kTileABytes = kGemmBM * kGemmBK * 2;
+constexpr uint32_t kTileBBytes = kGemmBN * kGemmBK * 2;
+constexpr uint32_t kStageBytes = kTileABytes + kTileBBytes;
+constexpr int kTmemCols = 2 * kGemmBN;
+constexpr int kPlanThreads = 1024;
+constexpr int kPlanWarps = kPlanThreads / 32;
+constexpr int kMaxGroups = 1025;
+
+struct GroupedWorkspace {
+    size_t group_offset = 0, perm_pair = 0, units_gu = 0, units_dn = 0;
+    size_t x_perm = 0, h_perm = 0, h_shared = 0, c = 0, s = 0;
+    size_t end = 0;
+};
+
+inline size_t g_align256(size_t v) { return (v + 255) / 256 * 256; }
+
+inline GroupedWorkspace grouped_workspace_layout(size_t base, int64_t T, int64_t H, int64_t E,
+                                                 int64_t k, int64_t I, int64_t I_s) {
+    GroupedWorkspace w;
+    const size_t P = (size_t)T * k;
+    size_t o = g_align256(base);
+    w.group_offset = o; o = g_align256(o + (size_t)(E + 2) * 4);
+    w.perm_pair = o;    o = g_align256(o + P * 4);
+    w.units_gu = o;     o = g_align256(o + (size_t)(E + 2) * 4);
+    w.units_dn = o;     o = g_align256(o + (size_t)(E + 2) * 4);
+    w.x_perm = o;       o = g_align256(o + (P + (size_t)T) * H * 2);
+    w.h_perm = o;       o = g_align256(o + P * I * 2);
+    w.h_shared = o;     o = g_align256(o + (size_t)T * I_s * 2);
+    w.c = o;            o = g_align256(o + P * H * 4);
+    w.s = o;            o = g_align256(o + (size_t)T * H * 4);
+    w.end = o;
+    return w;
+}
+
+// ------------------------------------------------------------- block scans
+// Exclusive scan of up to 2 * blockDim.x values held two per thread
+// (elements 2 tid, 2 tid + 1); returns the total.  blockDim.x == 1024.
+__device__ int block_exclusive_scan2(int &v0, int &v1, int *warp_sums) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int local = v0 + v1;
+    int incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off)
+            incl += n;
+    }
+    if (lane == 31)
+        warp_sums[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int s = lane < (int)(blockDim.x >> 5) ? warp_sums[lane] : 0;
+        int inc = s;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, inc, off);
+            if (lane >= off)
+                inc += n;
+        }
+        warp_sums[32 + lane] = inc - s;   // exclusive prefix of the warp totals
+        if (lane == 31)
+            warp_sums[64] = inc;
+    }
+    __syncthreads();
+    const int excl = warp_sums[32 + warp] + incl - local;
+    const int total = warp_sums[64];
+    v1 = excl + v0;
+    v0 = excl;
+    __syncthreads();
+    return total;
+}
+
+// ------------------------------------------------------------- group plan
+struct PlanArgs {
+    const int32_t *ids;
+    int64_t T, P;
+    int top_k, E, H, I, I_s;
+    int32_t *group_offset;  // [E + 2]: routed row offsets, [E] = valid picks, [E+1] = P
+    int32_t *perm_pair;     // [P]: permuted row -> pick index t * top_k + j
+    int32_t *units_gu;      // [G + 1] exclusive prefix of gate/up tiles per group
+    int32_t *units_dn;      // [G + 1] same for the down projection
+};
+
+__global__ void __launch_bounds__(kPlanThreads, 1) group_plan_kernel(const PlanArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    int *cnt = reinterpret_cast<int *>(smem);            // [kPlanWarps][E]
+    int *total = cnt + kPlanWarps * a.E;                 // [E]
+    int *goff = total + a.E;                             // [E]
+    int *wsum = goff + a.E;                              // [65]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int E = a.E;
+    const int64_t P = a.P;
+    const int64_t per_warp = (((P + kPlanWarps - 1) / kPlanWarps) + 31) / 32 * 32;
+    const int64_t p_lo = (int64_t)warp * per_warp;
+    const int64_t p_hi = min(P, p_lo + per_warp);
+
+    for (int i = tid; i < kPlanWarps * E; i += kPlanThreads)
+        cnt[i] = 0;
+    __syncthreads();
+    // pass 1: per-warp histogram of the picks, in pick order
+    for (int64_t base = p_lo; base < p_hi; base += 32) {
+        const int64_t p = base + lane;
+        int e = -1;
+        bool valid = false;
+        if (p < p_hi) {
+            e = a.ids[p];
+            valid = e >= 0 && e < E;
+            if (!valid)
+                flag_status(kStatusBadId);
+        }
+        const int key = valid ? e : -(lane + 2);
+        const uint32_t m = __match_any_sync(0xffffffffu, key);
+        if (valid && lane == __ffs(m) - 1)
+            cnt[warp * E + e] += __popc(m);
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += kPlanThreads) {
+        int run = 0;
+        for (int w = 0; w < kPlanWarps; ++w) {
+            const int c = cnt[w * E + e];
+            cnt[w * E + e] = run;
+            run += c;
+        }
+        total[e] = run;
+    }
+    __syncthreads();
+    // exclusive scan of the per-expert totals (E <= 1024 <= 2 * threads)
+    {
+        int v0 = 2 * tid < E ? total[2 * tid] : 0;
+        int v1 = 2 * tid + 1 < E ? total[2 * tid + 1] : 0;
+        const int all = block_exclusive_scan2(v0, v1, wsum);
+        if (2 * tid < E)
+            goff[2 * tid] = v0;
+        if (2 * tid + 1 < E)
+            goff[2 * tid + 1] = v1;
+        if (tid == 0) {
+            a.group_offset[E] = all;
+            a.group_offset[E + 1] = (int)P;
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += kPlanThreads) {
+        a.group_offset[e] = goff[e];
+        for (int w = 0; w < kPlanWarps; ++w)
+            cnt[w * E + e] += goff[e];
+    }
+    __syncthreads();
+    // pass 2: stable scatter, same order as pass 1
+    for (int64_t base = p_lo; base < p_hi; base += 32) {
+        const int64_t p = base + lane;
+        int e = -1;
+        bool valid = false;
+        if (p < p_hi) {
+            e = a.ids[p];
+            valid = e >= 0 && e < E;
+        }
+        const int key = valid ? e : -(lane + 2);
+        const uint32_t m = __match_any_sync(0xffffffffu, key);
+        int pos = 0;
+        if (valid)
+            pos = cnt[warp * E + e] + __popc(m & ((1u << lane) - 1u));
+        __syncwarp();
+        if (valid) {
+            a.perm_pair[pos] = (int32_t)p;
+            if (lane == __ffs(m) - 1)
+                cnt[warp * E + e] += __popc(m);
+        }
+        __syncwarp();
+    }
+    // tiles per group: routed groups, then the shared expert (all T rows)
+    const int G = E + (a.I_s > 0 ? 1 : 0);
+    {
+        int gu[2], dn[2];
+        for (int q = 0; q < 2; ++q) {
+            const int g = 2 * tid + q;
+            gu[q] = dn[q] = 0;
+            if (g < G) {
+                const int64_t rows = g < E ? total[g] : a.T;
+                const int nb = (int)((rows + kGemmBN - 1) / kGemmBN);
+                const int m_rows = g < E ? a.I : a.I_s;
+                gu[q] = nb * ((m_rows + kGateUpRows - 1) / kGateUpRows);
+                dn[q] = nb * ((a.H + kGemmBM - 1) / kGemmBM);
+            }
+        }
+        const int all_gu = block_exclusive_scan2(gu[0], gu[1], wsum);
+        const int all_dn = block_exclusive_scan2(dn[0], dn[1], wsum);
+        for (int q = 0; q < 2; ++q) {
+            const int g = 2 * tid + q;
+            if (g < G) {
+                a.units_gu[g] = gu[q];
+                a.units_dn[g] = dn[q];
+            }
+        }
+        if (tid == 0) {
+            a.units_gu[G] = all_gu;
+            a.units_dn[G] = all_dn;
+        }
+    }
+}
+
+// ----------------------------------------------------------- row gather
+__global__ void __launch_bounds__(256) gather_rows_kernel(const void *__restrict__ x, int x_f32,
+                                                          int64_t T, int H, int top_k, int64_t P,
+                                                          int E, int with_shared,
+                                                          const int32_t *__restrict__ group_offset,
+                                                          const int32_t *__restrict__ perm_pair,
+                                                          uint16_t *__restrict__ x_perm) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warp_global = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int64_t n_valid = group_offset[E];
+    const int64_t rows = n_valid + (with_shared ? T : 0);
+    const int nck = H >> 3;
+    for (int64_t r = warp_global; r < rows; r += nwarps) {
+        int64_t t, dst;
+        if (r < n_valid) {
+            t = perm_pair[r] / top_k;
+            dst = r;
+        } else {
+            t = r - n_valid;
+            dst = P + t;
+        }
+        uint4 *out = reinterpret_cast<uint4 *>(x_perm + (size_t)dst * H);
+        if (x_f32) {
+            const float4 *in = reinterpret_cast<const float4 *>(
+                reinterpret_cast<const float *>(x) + (size_t)t * H);
+            for (int c = lane; c < nck; c += 32) {
+                const float4 a = in[2 * c], b = in[2 * c + 1];
+                uint4 v;
+                v.x = (uint32_t)f32_to_bf16_rne(a.x) | ((uint32_t)f32_to_bf16_rne(a.y) << 16);
+                v.y = (uint32_t)f32_to_bf16_rne(a.z) | ((uint32_t)f32_to_bf16_rne(a.w) << 16);
+                v.z = (uint32_t)f32_to_bf16_rne(b.x) | ((uint32_t)f32_to_bf16_rne(b.y) << 16);
+                v.w = (uint32_t)f32_to_bf16_rne(b.z) | ((uint32_t)f32_to_bf16_rne(b.w) << 16);
+                out[c] = v;
+            }
+        } else {
+            const uint4 *in = reinterpret_cast<const uint4 *>(
+                reinterpret_cast<const uint16_t *>(x) + (size_t)t * H);
+            for (int c = lane; c < nck; c += 32)
+                out[c] = in[c];
+        }
+    }
+}
+
+// ------------------------------------------------------------ grouped GEMM
+struct GemmMaps {
+    CUtensorMap a, a2;               // routed weights (gate/up: W_gate, W_up; down: W_down)
+    CUtensorMap a_shared, a2_shared; // shared expert weights
+    CUtensorMap b, b_shared;         // activations (routed rows, shared rows)
+};
+
+struct GemmParams {
+    int E, G;
+    int64_t T, P;
+    int top_k;
+    int m_routed, m_shared;   // rows of the weight matrices: gate/up I, I_s; down H, H
+    int k_routed, k_shared;   // reduction length: gate/up H, H; down I, I_s
+    const int32_t *group_offset, *units, *perm_pair;
+    const float *weights;
+    uint16_t *h_out, *h_shared_out;   // gate/up outputs
+    int I, I_s;
+    float *c_out, *s_out;             // down outputs
+    int H;
+};
+
+struct GemmSmem {
+    static constexpr uint32_t stages = 0;
+    static constexpr uint32_t bars = kGemmStages * kStageBytes;
+    static constexpr uint32_t misc = bars + 256;
+    static constexpr uint32_t units = misc + 64;
+    static constexpr uint32_t offsets = units + kMaxGroups * 4 + 4;
+    static constexpr uint32_t total = offsets + (kMaxGroups + 2) * 4;
+    static constexpr uint32_t alloc = total + 1024;  // room to align the base to 1024
+};
+
+template <bool GATE_UP>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + GemmSmem::bars);
+    uint64_t *empty = full + kGemmStages;
+    uint64_t *tfull = empty + kGemmStages;
+    uint64_t *tempty = tfull + 2;
+    uint64_t *drain = tempty + 2;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + GemmSmem::misc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + GemmSmem::misc + 8);
+    int *units = reinterpret_cast<int *>(smem + GemmSmem::units);
+    int *offsets = reinterpret_cast<int *>(smem + GemmSmem::offsets);
+
+    const int warp = (int)(threadIdx.x >> 5);
+    const int lane = (int)lane_id();
+    const int G = p.G;
+
+    if (warp == 0 && lane == 0) {
+        for (int s = 0; s < kGemmStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 4);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tensormap(&maps.a);
+        prefetch_tensormap(&maps.b);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, kTmemCols);
+        tmem_relinquish();
+    }
+    for (int i = threadIdx.x; i <= G; i += blockDim.x)
+        units[i] = p.units[i];
+    for (int i = threadIdx.x; i < p.E + 2; i += blockDim.x)
+        offsets[i] = p.group_offset[i];
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_holder;
+    const int total_units = units[G];
+
+    // unit -> (group, m block, n block); m-major inside a group so that
+    // consecutive units reuse the same weight tile from L2.
+    auto decode = [&](int u, int &g, int &mb, int &nb, int &rows, int &n_blocks) {
+        int lo = 0, hi = G - 1;
+        while (lo < hi) {  // largest g with units[g] <= u
+            const int mid = (lo + hi + 1) >> 1;
+            if (units[mid] <= u)
+                lo = mid;
+            else
+                hi = mid - 1;
+        }
+        g = lo;
+        rows = g < p.E ? offsets[g + 1] - offsets[g] : (int)p.T;
+        n_blocks = (rows + kGemmBN - 1) / kGemmBN;
+        const int local = u - units[g];
+        mb = local / n_blocks;
+        nb = local - mb * n_blocks;
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer
+        if (elect_one()) {
+            const uint64_t pol_w = policy_evict_first();
+            const uint64_t pol_x = policy_evict_last();
+            uint32_t stage = 0, phase = 0;
+            int issued = 0;
+            bool stop = false;
+            for (int u = blockIdx.x; u < total_units && !stop; u += gridDim.x) {
+                int g, mb, nb, rows, n_blocks;
+                decode(u, g, mb, nb, rows, n_blocks);
+                const bool shared = g >= p.E;
+                const int K = shared ? p.k_shared : p.k_routed;
+                const int n0 = nb * kGemmBN;
+                const int n_valid = min(kGemmBN, rows - n0);
+                const int n_loads = (n_valid + kBoxRowsB - 1) / kBoxRowsB;
+                int brow;
+                if (GATE_UP)
+                    brow = (shared ? (int)p.P : offsets[g]) + n0;
+                else
+                    brow = (shared ? 0 : offsets[g]) + n0;
+                const CUtensorMap *bmap = (!GATE_UP && shared) ? &maps.b_shared : &maps.b;
+                const int kblocks = (K + kGemmBK - 1) / kGemmBK;
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+                        stop = true;
+                        break;
+                    }
+                    uint8_t *sa = smem + stage * kStageBytes;
+                    uint8_t *sb = sa + kTileABytes;
+                    mbar_arrive_expect_tx(&full[stage],
+                                          kTileABytes + (uint32_t)n_loads * kBoxRowsB * kGemmBK * 2);
+                    const int k0 = kb * kGemmBK;
+                    if (GATE_UP) {
+                        for (int j = 0; j < kGemmBM / kBoxRowsA; ++j) {
+                            const bool up = j & 1;
+                            const int row = mb * kGateUpRows + (j >> 1) * kBoxRowsA;
+                            uint8_t *dst = sa + j * kBoxRowsA * kGemmBK * 2;
+                            if (shared)
+                                tma_load_2d(dst, up ? &maps.a2_shared : &maps.a_shared, k0, row,
+                                            &full[stage], pol_w);
+                            else
+                                tma_load_3d(dst, up ? &maps.a2 : &maps.a, k0, row, g,
+                                            &full[stage], pol_w);
+                        }
+                    } else {
+                        if (shared)
+                            tma_load_2d(sa, &maps.a_shared, k0, mb * kGemmBM, &full[stage], pol_w);
+                        else
+                            tma_load_3d(sa, &maps.a, k0, mb * kGemmBM, g, &full[stage], pol_w);
+                    }
+                    for (int q = 0; q < n_loads; ++q)
+                        tma_load_2d(sb + q * kBoxRowsB * kGemmBK * 2, bmap, k0, brow + q * kBoxRowsB,
+                                    &full[stage], pol_x);
+                    ++issued;
+                    if (++stage == kGemmStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // no copy may still be landing in shared memory when the CTA exits
+            for (int n = issued > kGemmStages ? issued - kGemmStages : 0; n < issued; ++n)
+                mbar_wait(&full[n % kGemmStages], (uint32_t)(n / kGemmStages) & 1u, nullptr);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer
+        if (elect_one()) {
+            uint32_t stage = 0, phase = 0;
+            uint32_t acc = 0, acc_phase = 0;
+            bool stop = false;
+            for (int u = blockIdx.x; u < total_units && !stop; u += gridDim.x) {
+                int g, mb, nb, rows, n_blocks;
+                decode(u, g, mb, nb, rows, n_blocks);
+                const bool shared = g >= p.E;
+                const int K = shared ? p.k_shared : p.k_routed;
+                const int n_valid = min(kGemmBN, rows - nb * kGemmBN);
+                const uint32_t n_mma = (uint32_t)((n_valid + 15) / 16 * 16);
+                const uint32_t idesc = idesc_bf16_f32(kGemmBM, n_mma);
+                if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag))
+                    break;
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem_base + acc * kGemmBN;
+                const int kblocks = (K + kGemmBK - 1) / kGemmBK;
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, abort_flag)) {
+                        stop = true;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t a_addr = smem_u32(smem + stage * kStageBytes);
+                    const uint32_t b_addr = a_addr + kTileABytes;
+#pragma unroll
+                    for (int kk = 0; kk < kGemmBK / 16; ++kk)
+                        umma_bf16(d_tmem, smem_desc_sw128_kmajor(a_addr + kk * 32),
+                                  smem_desc_sw128_kmajor(b_addr + kk * 32), idesc,
+                                  (kb > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(&empty[stage]);  // frees the slot once these MMAs are done
+                    if (++stage == kGemmStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (stop)
+                    break;
+                umma_commit(&tfull[acc]);
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+            // every MMA issued by this thread has completed before TMEM is freed
+            umma_commit(drain);
+            mbar_wait(drain, 0, nullptr);
+        }
+    } else {
+        // ------------------------------------------------------ epilogue
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        uint32_t acc = 0, acc_phase = 0;
+        for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
+            int g, mb, nb, rows, n_blocks;
+            decode(u, g, mb, nb, rows, n_blocks);
+            const bool shared = g >= p.E;
+            const int n0 = nb * kGemmBN;
+            const int n_valid = min(kGemmBN, rows - n0);
+            if (!mbar_wait(&tfull[acc], acc_phase, abort_flag))
+                break;
+            tc_fence_after_sync();
+            const uint32_t t_row = tmem_base + ((uint32_t)(32 * q) << 16) + acc * kGemmBN;
+            for (int c0 = 0; c0 < n_valid; c0 += 32) {
+                uint32_t v[32];
+                tmem_load_32cols(t_row + (uint32_t)c0, v);
+                tmem_load_wait();
+                if (GATE_UP) {
+                    // lanes 0..15 hold gate rows, 16..31 the up rows of the same units
+                    const int M = shared ? p.I_s : p.I;
+                    const int unit = mb * kGateUpRows + 16 * q + (lane & 15);
+                    const bool is_gate = lane < 16;
+                    uint16_t *hrow_base = shared ? p.h_shared_out : p.h_out;
+                    const int ld = shared ? p.I_s : p.I;
+                    const int64_t row0 = (shared ? 0 : offsets[g]) + n0 + c0;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float mine = __uint_as_float(v[j]);
+                        const float other = __shfl_xor_sync(0xffffffffu, mine, 16);
+                        // lanes 0..15 finish columns 0..15, lanes 16..31 columns 16..31
+                        if ((j < 16) == is_gate) {
+                            const float gv = is_gate ? mine : other;
+                            const float uv = is_gate ? other : mine;
+                            const int col = c0 + j;
+                            if (col < n_valid && unit < M)
+                                hrow_base[(size_t)(row0 + j) * ld + unit] =
+                                    f32_to_bf16_rne(silu_f32(gv) * uv);
+                        }
+                    }
+                } else {
+                    const int row = mb * kGemmBM + 32 * q + lane;
+                    if (row < p.H) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int col = c0 + j;
+                            if (col < n_valid) {
+                                const float d = __uint_as_float(v[j]);
+                                if (shared) {
+                                    p.s_out[(size_t)(n0 + col) * p.H + row] = d;
+                                } else {
+                                    const int pick = p.perm_pair[offsets[g] + n0 + col];
+                                    p.c_out[(size_t)pick * p.H + row] = p.weights[pick] * d;
+                                }
+                            }
+                        }
+                    }
+                }
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&tempty[acc]);
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------- combine
+// y[t] = contributions of t's picks folded in ascending (expert id, slot),
+// then + the shared expert's output.  Skipped (invalid) picks add nothing.
+__global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ c,
+                                                      const float *__restrict__ s,
+                                                      const int32_t *__restrict__ ids, int64_t T,
+                                                      int H, int top_k, int E,
+                                                      float *__restrict__ y) {
+    __shared__ int order[16];
+    __shared__ int n_valid;
+    const int64_t t = blockIdx.x;
+    if (threadIdx.x == 0) {
+        int n = 0;
+        for (int j = 0; j < top_k; ++j) {
+            const int e = ids[t * top_k + j];
+            if (e < 0 || e >= E)
+                continue;
+            int pos = n++;
+            while (pos > 0 && ids[t * top_k + order[pos - 1]] > e) {
+                order[pos] = order[pos - 1];
+                --pos;
+            }
+            order[pos] = j;
+        }
+        n_valid = n;
+    }
+    __syncthreads();
+    const int h4 = blockIdx.y * blockDim.x + threadIdx.x;  // float4 column
+    if (h4 * 4 >= H)
+        return;
+    const int n = n_valid;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int q = 0; q < n; ++q) {
+        const float4 v =
+            reinterpret_cast<const float4 *>(c + ((size_t)t * top_k + order[q]) * H)[h4];
+        if (q == 0) {
+            acc = v;
+        } else {
+            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+        }
+    }
+    if (s != nullptr) {
+        const float4 v = reinterpret_cast<const float4 *>(s + (size_t)t * H)[h4];
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    reinterpret_cast<float4 *>(y + (size_t)t * H)[h4] = acc;
+}
+
+// ================================================================== host side
+struct GroupedArgs {
+    const void *x;
+    bool x_f32;
+    int64_t T, H, E, I, I_s;
+    int top_k;
+    const int32_t *ids;
+    const float *weights;
+    const void *w_gate, *w_up, *w_down, *ws_gate, *ws_up, *ws_down;
+    float *y;
+    int sm_count, smem_optin;
+};
+
+inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        cudaDriverEntryPointQueryResult q;
+        void *p = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
+                                             cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// bf16 tensor map: dims innermost first; box (64 elements of K) x box_rows (x 1).
+inline bool make_map(CUtensorMap *m, const void *base, int rank, const uint64_t *dims,
+                     const uint64_t *strides_bytes, uint32_t box_rows) {
+    auto enc = tensor_map_encoder();
+    if (enc == nullptr)
+        return false;
+    cuuint64_t gdim[3], gstride[2];
+    cuuint32_t box[3], estride[3] = {1, 1, 1};
+    for (int i = 0; i < rank; ++i)
+        gdim[i] = dims[i];
+    for (int i = 0; i < rank - 1; ++i)
+        gstride[i] = strides_bytes[i];
+    box[0] = kGemmBK;
+    box[1] = box_rows;
+    box[2] = 1;
+    const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank,
+                           const_cast<void *>(base), gdim, gstride, box, estride,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+inline bool map_2d(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows,
+                   uint32_t box_rows) {
+    const uint64_t dims[2] = {cols, rows};
+    const uint64_t strides[1] = {cols * 2};
+    return make_map(m, base, 2, dims, strides, box_rows);
+}
+
+inline bool map_3d(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint64_t mats,
+                   uint32_t box_rows) {
+    const uint64_t dims[3] = {cols, rows, mats};
+    const uint64_t strides[2] = {cols * 2, cols * rows * 2};
+    return make_map(m, base, 3, dims, strides, box_rows);
+}
+
+inline size_t plan_smem_bytes(int64_t E) { return (size_t)(kPlanWarps * E + 2 * E + 65) * 4; }
+
+inline ep_status grouped_set_attributes(int smem_optin) {
+    if (cudaFuncSetAttribute(group_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem_optin) != cudaSuccess)
+        return EP_ECUDA;
+    if (cudaFuncSetAttribute(grouped_gemm_kernel<true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem_optin) != cudaSuccess)
+        return EP_ECUDA;
+    if (cudaFuncSetAttribute(grouped_gemm_kernel<false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem_optin) != cudaSuccess)
+        return EP_ECUDA;
+    return EP_OK;
+}
+
+inline ep_status grouped_forward(const GroupedArgs &g, const GroupedWorkspace &W, uint8_t *ws,
+                                 cudaStream_t st, int *launches, char *why, size_t why_len) {
+    *launches = 0;
+    const int64_t T = g.T, H = g.H, E = g.E, I = g.I, I_s = g.I_s;
+    const int k = g.top_k;
+    const int64_t P = T * k;
+    const int G = (int)E + (I_s > 0 ? 1 : 0);
+    if (GemmSmem::alloc > (uint32_t)g.smem_optin || plan_smem_bytes(E) > (size_t)g.smem_optin) {
+        snprintf(why, why_len, "not enough shared memory per block for the tensor path");
+        return EP_EINVAL;
+    }
+    if (tensor_map_encoder() == nullptr) {
+        snprintf(why, why_len, "cuTensorMapEncodeTiled is not available from the driver");
+        return EP_ECUDA;
+    }
+    int32_t *group_offset = reinterpret_cast<int32_t *>(ws + W.group_offset);
+    int32_t *perm_pair = reinterpret_cast<int32_t *>(ws + W.perm_pair);
+    int32_t *units_gu = reinterpret_cast<int32_t *>(ws + W.units_gu);
+    int32_t *units_dn = reinterpret_cast<int32_t *>(ws + W.units_dn);
+    uint16_t *x_perm = reinterpret_cast<uint16_t *>(ws + W.x_perm);
+    uint16_t *h_perm = reinterpret_cast<uint16_t *>(ws + W.h_perm);
+    uint16_t *h_shared = reinterpret_cast<uint16_t *>(ws + W.h_shared);
+    float *c = reinterpret_cast<float *>(ws + W.c);
+    float *s = reinterpret_cast<float *>(ws + W.s);
+
+    // 1. plan
+    PlanArgs pa;
+    pa.ids = g.ids; pa.T = T; pa.P = P; pa.top_k = k; pa.E = (int)E; pa.H = (int)H;
+    pa.I = (int)I; pa.I_s = (int)I_s;
+    pa.group_offset = group_offset; pa.perm_pair = perm_pair;
+    pa.units_gu = units_gu; pa.units_dn = units_dn;
+    group_plan_kernel<<<1, kPlanThreads, plan_smem_bytes(E), st>>>(pa);
+    if (cudaGetLastError() != cudaSuccess) {
+        snprintf(why, why_len, "group_plan launch failed");
+        return EP_ECUDA;
+    }
+    // 2. gather
+    {
+        const int64_t rows = P + (I_s > 0 ? T : 0);
+        const int64_t blocks = std::min<int64_t>((rows + 7) / 8, (int64_t)g.sm_count * 8);
+        gather_rows_kernel<<<(unsigned)std::max<int64_t>(blocks, 1), 256, 0, st>>>(
+            g.x, g.x_f32 ? 1 : 0, T, (int)H, k, P, (int)E, I_s > 0 ? 1 : 0, group_offset,
+            perm_pair, x_perm);
+        if (cudaGetLastError() != cudaSuccess) {
+            snprintf(why, why_len, "gather_rows launch failed");
+            return EP_ECUDA;
+        }
+    }
+    // 3. gate/up
+    GemmMaps gm;
+    memset(&gm, 0, sizeof gm);
+    bool okm = map_3d(&gm.a, g.w_gate, H, I, E, kBoxRowsA) &&
+               map_3d(&gm.a2, g.w_up, H, I, E, kBoxRowsA) &&
+               map_2d(&gm.b, x_perm, H, P + T, kBoxRowsB);
+    if (I_s > 0)
+        okm = okm && map_2d(&gm.a_shared, g.ws_gate, H, I_s, kBoxRowsA) &&
+              map_2d(&gm.a2_shared, g.ws_up, H, I_s, kBoxRowsA);
+    if (!okm) {
+        snprintf(why, why_len, "encoding a gate/up tensor map failed");
+        return EP_ECUDA;
+    }
+    GemmParams gp;
+    memset(&gp, 0, sizeof gp);
+    gp.E = (int)E; gp.G = G; gp.T = T; gp.P = P; gp.top_k = k;
+    gp.m_routed = (int)I; gp.m_shared = (int)I_s; gp.k_routed = (int)H; gp.k_shared = (int)H;
+    gp.group_offset = group_offset; gp.units = units_gu; gp.perm_pair = perm_pair;
+    gp.weights = g.weights;
+    gp.h_out = h_perm; gp.h_shared_out = h_shared; gp.I = (int)I; gp.I_s = (int)I_s;
+    gp.c_out = c; gp.s_out = s; gp.H = (int)H;
+    grouped_gemm_kernel<true><<<g.sm_count, kGemmThreads, GemmSmem::alloc, st>>>(gm, gp);
+    if (cudaGetLastError() != cudaSuccess) {
+        snprintf(why, why_len, "gate/up GEMM launch failed");
+        return EP_ECUDA;
+    }
+    // 4. down
+    memset(&gm, 0, sizeof gm);
+    okm = map_3d(&gm.a, g.w_down, I, H, E, kGemmBM) && map_2d(&gm.b, h_perm, I, std::max<int64_t>(P, 1), kBoxRowsB);
+    if (I_s > 0)
+        okm = okm && map_2d(&gm.a_shared, g.ws_down, I_s, H, kGemmBM) &&
+              map_2d(&gm.b_shared, h_shared, I_s, T, kBoxRowsB);
+    if (!okm) {
+        snprintf(why, why_len, "encoding a down tensor map failed");
+        return EP_ECUDA;
+    }
+    gp.m_routed = (int)H; gp.m_shared = (int)H; gp.k_routed = (int)I; gp.k_shared = (int)I_s;
+    gp.units = units_dn;
+    grouped_gemm_kernel<false><<<g.sm_count, kGemmThreads, GemmSmem::alloc, st>>>(gm, gp);
+    if (cudaGetLastError() != cudaSuccess) {
+        snprintf(why, why_len, "down GEMM launch failed");
+        return EP_ECUDA;
+    }
+    // 5. combine
+    {
+        const dim3 grid((unsigned)T, (unsigned)((H / 4 + 255) / 256));
+        combine_kernel<<<grid, 256, 0, st>>>(c, I_s > 0 ? s : nullptr, g.ids, T, (int)H, k,
+                                             (int)E, g.y);
+        if (cudaGetLastError() != cudaSuccess) {
+            snprintf(why, why_len, "combine launch failed");
+            return EP_ECUDA;
+        }
+    }
+    *launches = 5;
+    return EP_OK;
+}
+
+}  // namespace epk

@@ -1,0 +1,131 @@
+"""The tensor-core path (tcgen05 grouped GEMMs) of moe_ffn_forward against the fp64
+oracle: small cases that span several tiles with ragged tails, element by
+element; the full-size workloads on rows the oracle computes one by one; and
+the bit-identity across runs and band counts at every size."""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+import expert_decode_b200 as ed
+from gpu_parity import check_y, device_inputs, gpu_ffn, oracle_ffn, oracle_route
+
+pytestmark = pytest.mark.gpu
+WL = workloads.WORKLOADS
+
+
+@pytest.fixture(autouse=True)
+def tensor_dispatch():
+    ed.ep_set_dispatch("tensor")
+    yield
+    ed.ep_set_dispatch("auto")
+
+
+def _routed(o, wl, T, seed=workloads.SEED_BASE, batch=0, rows=None, **sizes):
+    W, x = device_inputs(wl, T, seed=seed, batch=batch, **sizes)
+    ids, w = ed.moe_route(x, W["w_router"], W["bias"], wl.top_k)
+    torch.cuda.synchronize()
+    ids_ref, w_ref, _ = oracle_route(o, x, W, wl.top_k, rows=rows)
+    got = ids.cpu().numpy() if rows is None else ids.cpu().numpy()[rows]
+    assert np.array_equal(got, ids_ref)
+    return W, x, ids, w
+
+
+def test_tiny_tensor_path_all_bands(oracle_lib):
+    wl = WL["tiny"]
+    W, x, ids, w = _routed(oracle_lib, wl, 24)
+    ys = [gpu_ffn(x, ids, w, W, ed.ep_plan(wl.E, R)) for R in (1, 2, 4, 8)]
+    ed.ep_check_status()
+    assert ed.ep_last_launch_count() == 5
+    for y in ys[1:]:
+        assert torch.equal(y, ys[0])
+    check_y(ys[0], oracle_ffn(oracle_lib, x, ids, w, W), what="tiny T=24 tensor")
+    check_y(ys[0], oracle_ffn(oracle_lib, x, ids, w, W, bands=oracle_lib.expert_parallel_plan(16, 4)),
+            what="tiny T=24 tensor vs EP(4)")
+
+
+@pytest.mark.parametrize("T", [1, 8, 33, 300])
+def test_ragged_multi_tile(oracle_lib, T):
+    """H, I, I_s not multiples of the tile; groups of every size incl. > 256 rows."""
+    wl = workloads.Workload("ragged", (T,), 200, 12, 6, 136, 72, "bf16", "none", (3,))
+    W, x, ids, w = _routed(oracle_lib, wl, T, seed=31)
+    y = gpu_ffn(x, ids, w, W, ed.ep_plan(wl.E, 3))
+    ed.ep_check_status()
+    check_y(y, oracle_ffn(oracle_lib, x, ids, w, W), what=f"ragged T={T}")
+
+
+def test_fp32_activations(oracle_lib):
+    wl = workloads.Workload("f32", (40,), 256, 16, 4, 128, 128, "f32", "none", (2,))
+    W, x, ids, w = _routed(oracle_lib, wl, 40, seed=3)
+    y = gpu_ffn(x, ids, w, W, ed.ep_plan(wl.E, 2))
+    check_y(y, oracle_ffn(oracle_lib, x, ids, w, W), what="fp32 x tensor")
+
+
+def test_hot_expert_many_tiles(oracle_lib):
+    """One expert takes every token's first pick: > 256 rows, several N tiles."""
+    wl = workloads.Workload("hot", (600,), 256, 8, 2, 192, 0, "bf16", "none", (2,))
+    W, x = device_inputs(wl, 600, seed=6)
+    ids = torch.stack([torch.zeros(600, dtype=torch.int32),
+                       torch.arange(600, dtype=torch.int32) % 7 + 1], 1).cuda()
+    w = torch.full((600, 2), 0.5, device="cuda")
+    y = gpu_ffn(x, ids, w, W, ed.ep_plan(wl.E, 2))
+    rows = np.r_[0:8, 250:262, 590:600]
+    ref = oracle_ffn(oracle_lib, x, ids, w, W, rows=rows)
+    check_y(y[rows], ref, what="hot expert")
+
+
+def test_tensor_matches_streaming_within_tolerance(oracle_lib):
+    wl = WL["decode"]
+    W, x, ids, w = _routed(oracle_lib, wl, 8, batch=2)
+    plan = ed.ep_plan(wl.E, 8)
+    y_t = gpu_ffn(x, ids, w, W, plan)
+    ed.ep_set_dispatch("streaming")
+    y_s = gpu_ffn(x, ids, w, W, plan)
+    ed.ep_set_dispatch("tensor")
+    ref = oracle_ffn(oracle_lib, x, ids, w, W)
+    check_y(y_t, ref, what="decode T=8 tensor")
+    check_y(y_s, ref, rel_tol=1e-4, what="decode T=8 streaming")
+
+
+def test_repeated_and_bad_ids(oracle_lib):
+    wl = WL["tiny"]
+    W, x, ids, w = _routed(oracle_lib, wl, 20, seed=14)
+    ed.ep_check_status()
+    ids = ids.clone()
+    ids[2, 1] = ids[2, 0]
+    ids[5, 3] = -3
+    y = gpu_ffn(x, ids, w, W, ed.ep_plan(wl.E, 4))
+    with pytest.raises(ed.EPError):
+        ed.ep_check_status()
+    ref_ids, ref_w = ids.clone(), w.clone()
+    ref_ids[5, 3] = 0
+    ref_w[5, 3] = 0.0
+    check_y(y, oracle_ffn(oracle_lib, x, ref_ids, ref_w, W), what="repeated / bad ids")
+
+
+# ------------------------------------------------------------ full-size workloads
+def _full(o, name, rows, bands):
+    wl = WL[name]
+    T = wl.T[0]
+    W, x, ids, w = _routed(o, wl, T, rows=rows)
+    ys = [gpu_ffn(x, ids, w, W, ed.ep_plan(wl.E, R)) for R in bands]
+    ed.ep_check_status()
+    for y in ys[1:]:
+        assert torch.equal(y, ys[0]), "band counts differ"
+    assert torch.equal(gpu_ffn(x, ids, w, W, ed.ep_plan(wl.E, bands[0])), ys[0]), "runs differ"
+    ref = oracle_ffn(o, x, ids, w, W, rows=rows)
+    check_y(ys[0][rows], ref, what=f"{name} sampled rows")
+    return W, x, ids, w, ys[0]
+
+
+def test_prefill_full_size(oracle_lib):
+    _full(oracle_lib, "prefill", np.array([0, 1, 255, 511]), (4, 1, 2, 8))
+
+
+def test_imbalanced_full_size(oracle_lib):
+    W, x, ids, w, y = _full(oracle_lib, "imbalanced", np.r_[0:6, 1000:1004, 2042:2048], (4, 1))
+    assert int(ids.max()) < 16, "bias +8 on experts 0..15 must put every pick in band 0"
+
+
+def test_large_full_size(oracle_lib):
+    _full(oracle_lib, "large", np.array([0, 2047, 4095]), (8, 1))
