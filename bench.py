@@ -1,0 +1,517 @@
+#!/usr/bin/env python
+"""Throughput of the routed MoE FFN on B200: tokens/s, with the dominant
+kernel's fraction of its roofline.
+
+A step is one pass of the whole hot path (router, top-k, experts, fixed-order
+combine) over the workload's batches; the default workload is decode: three
+calls at T = 1, 4 and 8 rows (13 tokens), H=4096, E=128, top_k=8, I=1536, one
+shared expert, plan of 8 bands.  Inputs are seeded synthetic tensors resident
+in HBM; 16 distinct x batches per row count cycle so that routing varies; the
+L2 cache is flushed (a 512 MiB write) before every step, outside the timed
+events.  `value` = tokens / device time (CUDA events around each step, max over
+ranks); `e2e` repeats the measurement through the public API with the inputs
+copied from pinned host memory and y copied back inside the timed region.
+
+  python bench.py [--gpus N --steps K --warmup W] [--config decode|prefill|...]
+  python bench.py --impl reference ...   # the fp64 CPU oracle on the host cores
+
+With N > 1 (torchrun) every rank runs an independent replica on its own GPU:
+the tokens of a MoE layer are independent problems, so the ranks share no data
+and the reported throughput is the sum over ranks (weak scaling).
+"""
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "routed MoE FFN tokens/s; decode HBM GB/s and prefill TFLOPS as % of B200 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+N_BATCHES = 16
+FLUSH_BYTES = 512 << 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--config", choices=tuple(workloads.WORKLOADS), default="decode")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=500)
+    return ap.parse_args()
+
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        uuid = str(torch.cuda.get_device_properties(device).uuid)
+        self.gpu = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        self.out = os.path.join("/tmp", f"clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.out, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu, "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in open(self.out):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[3:7]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        os.unlink(self.out)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ workload
+class Layer:
+    """One MoE layer's weights on the device plus per-row-count buffers."""
+
+    def __init__(self, wl, device, seed):
+        import expert_decode_b200 as ed
+        self.ed = ed
+        self.wl = wl
+        self.W = workloads.make_weights(wl, device=device, seed=workloads.SEED_BASE)
+        self.shared = (None if self.W["ws_gate"] is None
+                       else (self.W["ws_gate"], self.W["ws_up"], self.W["ws_down"]))
+        self.plan = ed.ep_plan(wl.E, wl.bands[0])
+        self.xs = {T: [workloads.make_x(wl, T, device=device, seed=seed, batch=b + 100 * T)
+                       for b in range(N_BATCHES if T <= 8 else 2)] for T in wl.T}
+        self.ids = {T: torch.empty((T, wl.top_k), dtype=torch.int32, device=device)
+                    for T in wl.T}
+        self.wts = {T: torch.empty((T, wl.top_k), dtype=torch.float32, device=device)
+                    for T in wl.T}
+        self.y = {T: torch.empty((T, wl.H), dtype=torch.float32, device=device) for T in wl.T}
+        ws = max(ed.moe_ffn_workspace_size(T, wl.H, wl.E, wl.top_k, wl.I, wl.I_s)
+                 for T in wl.T)
+        self.workspace = torch.empty(ws, dtype=torch.uint8, device=device)
+        self.launches = 0
+
+    def call(self, T, b, x=None):
+        ed = self.ed
+        x = self.xs[T][b % len(self.xs[T])] if x is None else x
+        ed.moe_route(x, self.W["w_router"], self.W["bias"], self.wl.top_k, ids=self.ids[T],
+                     weights=self.wts[T])
+        self.launches += ed.ep_last_launch_count()
+
+    def ffn(self, T, b, x=None, y=None):
+        ed = self.ed
+        x = self.xs[T][b % len(self.xs[T])] if x is None else x
+        ed.moe_ffn_forward(x, self.ids[T], self.wts[T], self.W["w_gate"], self.W["w_up"],
+                           self.W["w_down"], self.shared, self.plan,
+                           y=self.y[T] if y is None else y, workspace=self.workspace)
+        self.launches += ed.ep_last_launch_count()
+
+    def distinct_experts(self, T, b):
+        self.call(T, b)
+        torch.cuda.synchronize()
+        return int(torch.unique(self.ids[T]).numel())
+
+
+# ---------------------------------------------------------------- bytes/flops
+def kernel_cost(wl, T, n_distinct, tensor_path):
+    """Algorithmic bytes / flops of the dominant kernel (gate/up) of one call,
+    and of the whole call.  Weights: only the picked experts plus the shared
+    one, each read once; activations at their stored widths."""
+    H, I, I_s, k = wl.H, wl.I, wl.I_s, wl.top_k
+    xb = 4 if wl.x_dtype == "f32" else 2
+    n_exp = n_distinct + (1 if I_s else 0)
+    w_gu = (n_distinct * 2 * H * I + (2 * H * I_s if I_s else 0)) * 2
+    w_dn = (n_distinct * H * I + (H * I_s if I_s else 0)) * 2
+    P = T * k
+    flops_gu = 2 * (P * 2 * H * I + (T * 2 * H * I_s if I_s else 0))
+    flops_dn = 2 * (P * H * I + (T * H * I_s if I_s else 0))
+    if tensor_path:
+        gu_bytes = w_gu + (P + (T if I_s else 0)) * H * 2 + (P * I + T * I_s) * 2
+    else:
+        gu_bytes = w_gu + T * H * xb
+    call_bytes = (wl.E * H * 2 + T * H * xb + T * k * 8) + w_gu + w_dn + T * H * 4
+    call_flops = 2 * T * H * wl.E + flops_gu + flops_dn
+    return {"gu_bytes": gu_bytes, "gu_flops": flops_gu, "call_bytes": call_bytes,
+            "call_flops": call_flops, "n_experts": n_exp}
+
+
+def source_digest():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "expert_decode_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(f"{kernel}:{workload}")
+    if not e or e.get("source_digest") != source_digest():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------- CPU legs
+def oracle_sample(layer, rows_per_T, threads, batches=1):
+    """Time the fp64 oracle on a bounded sample: route + monolith FFN of the
+    given rows of the first `batches` batches of each row count.  Returns
+    tokens, seconds (the host copies of the weights are not timed)."""
+    import oracle
+    o = oracle.load()
+    W = layer.W
+    wl = layer.wl
+    bias = None if W["bias"] is None else W["bias"].cpu().numpy()
+    wr = workloads.bits(W["w_router"])
+    sh = None if layer.shared is None else tuple(workloads.bits(t) for t in layer.shared)
+    tokens, seconds = 0, 0.0
+    for T, nrows, b in [(T, n, b) for T, n in rows_per_T.items() for b in range(batches)]:
+        x = layer.xs[T][b % len(layer.xs[T])][:nrows]
+        xh = workloads.bits(x)
+        t0 = time.perf_counter()
+        ids, w, _ = o.route(xh, wr, bias, wl.top_k, threads=min(threads, nrows))
+        seconds += time.perf_counter() - t0
+        used = sorted(set(int(e) for e in ids.ravel()))
+        mats = tuple({e: workloads.bits(W[k][e]) for e in used}
+                     for k in ("w_gate", "w_up", "w_down"))
+        t0 = time.perf_counter()
+        o.moe_ffn_monolith(xh, ids, w, *mats, wl.E, shared=sh, threads=min(threads, nrows))
+        seconds += time.perf_counter() - t0
+        tokens += nrows
+    return tokens, seconds
+
+
+def run_reference(args, wl):
+    """The oracle arm: the fp64 CPU oracle, as it stands, on this host's cores.
+
+    A token of the workload costs its routing plus top_k + 1 expert
+    evaluations (routed picks and the shared expert).  Each step makes one
+    oracle call over `cores` (token, expert) evaluations, which the oracle
+    runs in parallel (OpenMP over its rows); each evaluation counts as
+    1 / (top_k + 1) of a token, and routing is timed when a token is first
+    met.  That bounds a step to about one expert evaluation of wall time, so
+    that K + W steps finish within a few minutes."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    torch.cuda.set_device(0)
+    o = oracle.load()
+    layer = Layer(wl, "cuda:0", workloads.SEED_BASE)
+    cores = os.cpu_count() or 1
+    W = layer.W
+    T0 = wl.T[-1]
+    x = layer.xs[T0][0]
+    xh = workloads.bits(x)
+    bias = None if W["bias"] is None else W["bias"].cpu().numpy()
+    wr = workloads.bits(W["w_router"])
+    ids, w, _ = o.route(xh, wr, bias, wl.top_k, threads=min(cores, T0))
+    # the evaluations of the batch: (token, expert slot); the shared expert is
+    # appended to the expert table as entry E so one call can mix both kinds
+    evals = [(t, int(ids[t, j]), float(w[t, j])) for t in range(T0) for j in range(wl.top_k)]
+    if layer.shared is not None:
+        evals += [(t, wl.E, 1.0) for t in range(T0)]
+    per_token = wl.top_k + (1 if layer.shared is not None else 0)
+    used = sorted(set(e for _, e, _ in evals if e < wl.E))
+    tables = []
+    for kname, sname in (("w_gate", "ws_gate"), ("w_up", "ws_up"), ("w_down", "ws_down")):
+        t = {e: workloads.bits(W[kname][e]) for e in used}
+        if layer.shared is not None:
+            t[wl.E] = workloads.bits(W[sname])
+        tables.append(t)
+    n = min(cores, len(evals))
+    total_tok, total_s = 0.0, 0.0
+    seen = set()
+    for i in range(args.warmup + args.steps):
+        batch = [evals[(i * n + q) % len(evals)] for q in range(n)]
+        rows = np.array([t for t, _, _ in batch])
+        new = sorted(set(rows.tolist()) - seen)
+        t0 = time.perf_counter()
+        if new:
+            o.route(xh[new], wr, bias, wl.top_k, threads=min(cores, len(new)))
+        o.moe_ffn_monolith(xh[rows], np.array([[e] for _, e, _ in batch], dtype=np.int32),
+                           np.array([[wt] for _, _, wt in batch]), *tables, wl.E + 1,
+                           threads=n)
+        sec = time.perf_counter() - t0
+        seen.update(new)
+        if len(seen) == T0:
+            seen = set()
+        if i >= args.warmup:
+            total_tok += n / per_token
+            total_s += sec
+    value = total_tok / total_s
+    sample = (f"each step: {n} (token, expert) evaluations of the T={T0} batch in one oracle "
+              f"call (OpenMP over rows), routing when a token is first met; a token = "
+              f"{per_token} evaluations")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total_s / max(args.steps, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.description, "bands": wl.bands[0]},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": n, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# -------------------------------------------------------------------- our arm
+def run_ours(args, wl):
+    import expert_decode_b200 as ed
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+    peaks, peak_src = read_peaks()
+    layer = Layer(wl, device, workloads.SEED_BASE + 7919 * rank)
+    Ts = wl.T
+    tensor_path = {T: T > 8 for T in Ts}
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    # per (T, batch): distinct experts picked (fixed for a given batch)
+    n_batches = {T: len(layer.xs[T]) for T in Ts}
+    distinct = {(T, b): layer.distinct_experts(T, b) for T in Ts for b in range(n_batches[T])}
+    dom = "gate/up GEMM (tcgen05)" if any(tensor_path.values()) else "stream_gate_up"
+    dom_index = {T: (2 if tensor_path[T] else 0) for T in Ts}   # kernel j of the ffn call
+
+    def step(i, prof=None):
+        for T in Ts:
+            layer.call(T, i)
+            if prof is not None:
+                ed.ep_profile_events(prof[T])
+            layer.ffn(T, i)
+            if prof is not None:
+                ed.ep_profile_events(None)
+
+    for i in range(args.warmup):
+        flush.zero_()
+        step(i)
+    torch.cuda.synchronize()
+    ed.ep_check_status()
+
+    K = args.steps
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    nk = 10
+    prof = [{T: [torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)] for T in Ts}
+            for _ in range(K)]
+    for p in prof:
+        for evs in p.values():
+            for e in evs:
+                e.record()
+    torch.cuda.synchronize()
+    layer.launches = 0
+    sampler = ClockSampler(device) if rank == 0 else None
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    t_wall = time.perf_counter()
+    for i in range(K):
+        flush.zero_()
+        ev_s[i].record()
+        step(args.warmup + i, prof[i])
+        ev_e[i].record()
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter() - t_wall
+    clocks = sampler.stop() if sampler else None
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ed.ep_check_status()
+    launches = layer.launches
+
+    step_ms = [ev_s[i].elapsed_time(ev_e[i]) for i in range(K)]
+    dev_s = sum(step_ms) / 1e3
+    tokens_rank = K * sum(Ts)
+    # dominant kernel: summed algorithmic bytes over summed durations
+    dom_bytes = dom_flops = dom_s = 0.0
+    step_bytes = step_flops = 0.0
+    per_T = {}
+    for T in Ts:
+        j = dom_index[T]
+        durs, byts, fl = [], 0.0, 0.0
+        for i in range(K):
+            b = args.warmup + i
+            c = kernel_cost(wl, T, distinct[(T, b % n_batches[T])], tensor_path[T])
+            durs.append(prof[i][T][2 * j].elapsed_time(prof[i][T][2 * j + 1]) / 1e3)
+            byts += c["gu_bytes"]
+            fl += c["gu_flops"]
+            step_bytes += c["call_bytes"]
+            step_flops += c["call_flops"]
+        dom_bytes += byts
+        dom_flops += fl
+        dom_s += sum(durs)
+        per_T[f"T={T}"] = {"dominant_kernel_us": 1e6 * sum(durs) / K,
+                           "dominant_kernel_GBps": byts / sum(durs) / 1e9}
+
+    if dist is not None:
+        t = torch.tensor([dev_s], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dev_s_max = float(t.item())
+    else:
+        dev_s_max = dev_s
+    value = tokens_rank * world / dev_s_max
+
+    # roofline of the dominant kernel
+    t_hbm = dom_bytes / (peaks["hbm_gbs"] * 1e9)
+    # the kernel is timed inside a long run of steps: the sustained GEMM peak
+    peak_tf = peaks["bf16_tflops_sustained"]
+    t_tc = dom_flops / (peak_tf * 1e12)
+    if t_hbm >= t_tc:
+        roof = {"bound": "hbm", "achieved": dom_bytes / dom_s / 1e9, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": dom_flops / dom_s / 1e12, "peak": peak_tf,
+                "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    kname = "grouped_gemm_kernel<true>" if any(tensor_path.values()) else "stream_gate_up_kernel"
+    roof["traffic"] = traffic_for(kname, wl.name)
+    roof["kernel"] = kname
+    roof["peak_source"] = peak_src
+
+    # e2e: inputs from pinned host memory, y back to pinned host, in the region
+    e2e = None
+    if args.e2e_steps > 0:
+        KE = min(args.e2e_steps, K)
+        hx = {T: [x.cpu().pin_memory() for x in layer.xs[T]] for T in Ts}
+        dx = {T: torch.empty_like(layer.xs[T][0]) for T in Ts}
+        hy = {T: torch.empty((T, wl.H), dtype=torch.float32).pin_memory() for T in Ts}
+        es = torch.cuda.Event(enable_timing=True)
+        ee = torch.cuda.Event(enable_timing=True)
+        h2d = sum(hx[T][0].numel() * hx[T][0].element_size() for T in Ts)
+        d2h = sum(hy[T].numel() * 4 for T in Ts)
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        es.record()
+        for i in range(KE):
+            for T in Ts:
+                b = i % len(hx[T])
+                dx[T].copy_(hx[T][b], non_blocking=True)
+                layer.call(T, 0, x=dx[T])
+                layer.ffn(T, 0, x=dx[T])
+                hy[T].copy_(layer.y[T], non_blocking=True)
+        ee.record()
+        torch.cuda.synchronize()
+        e2e_s = es.elapsed_time(ee) / 1e3
+        if dist is not None:
+            t = torch.tensor([e2e_s], device=device, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_s = float(t.item())
+        e2e = {"value": KE * sum(Ts) * world / e2e_s, "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": KE,
+               "l2": "not flushed"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = os.cpu_count() or 1
+        rows = {T: min(T, 8) for T in Ts}
+        tok, sec = oracle_sample(layer, rows, threads, batches=2)
+        cpu = {"value": tok / sec, "unit": "tokens/s", "cores": min(threads, max(rows.values())),
+               "kind": "oracle",
+               "sample": "first 2 batches of each row count ("
+                         + ", ".join(f"{n} of T={T}" for T, n in rows.items())
+                         + "), fp64 route + monolith FFN, OpenMP over tokens"}
+
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": 1e3 * dev_s_max / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.description, "bands": wl.bands[0],
+                   "l2": "flushed before every step (512 MiB write)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "batches": "16 distinct x batches per row count, cycled"},
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "detail": {"per_T": per_T, "wall_s": t_wall,
+                   "step_hbm_GBps": step_bytes / dev_s / 1e9,
+                   "step_hbm_frac": step_bytes / dev_s / 1e9 / peaks["hbm_gbs"],
+                   "step_tflops": step_flops / dev_s / 1e12,
+                   "dominant_kernel": dom},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    wl = workloads.WORKLOADS[args.config]
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    main()

@@ -60,6 +60,8 @@ def library():
             lib.ep_check_status.argtypes = [P]
             lib.ep_last_error.restype = ctypes.c_char_p
             lib.ep_last_launch_count.restype = I32
+            lib.ep_profile_events.argtypes = [P, I32]
+            lib.ep_profile_events.restype = ctypes.c_int
             for fn in ("ep_plan", "moe_route", "moe_ffn_forward", "ep_set_dispatch",
                        "ep_check_status"):
                 getattr(lib, fn).restype = ctypes.c_int
@@ -172,3 +174,19 @@ def ep_set_dispatch(mode):
 
 def ep_last_launch_count():
     return int(library().ep_last_launch_count())
+
+
+_profile_keep = threading.local()
+
+
+def ep_profile_events(events):
+    """Bracket each kernel of later calls (this thread) with these torch.cuda.Events:
+    kernel j between events[2j] and events[2j+1].  None stops.  Each event must
+    have been recorded once so that its CUDA handle exists."""
+    if events is None:
+        _profile_keep.arr = None
+        _check(library().ep_profile_events(None, 0))
+        return
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _profile_keep.arr = arr
+    _check(library().ep_profile_events(ctypes.cast(arr, ctypes.c_void_p), len(events)))

@@ -21,6 +21,22 @@ namespace {
 
 thread_local char t_error[512] = "";
 thread_local int32_t t_launches = 0;
+thread_local void *const *t_prof_events = nullptr;
+thread_local int32_t t_prof_n = 0;
+
+// Per-kernel timing hook (ep_profile_events): events around launch j.
+struct KernelBracket {
+    cudaStream_t st;
+    int j;
+    KernelBracket(cudaStream_t s, int index) : st(s), j(index) {
+        if (t_prof_events != nullptr && 2 * j + 1 < t_prof_n)
+            cudaEventRecord(static_cast<cudaEvent_t>(t_prof_events[2 * j]), st);
+    }
+    ~KernelBracket() {
+        if (t_prof_events != nullptr && 2 * j + 1 < t_prof_n)
+            cudaEventRecord(static_cast<cudaEvent_t>(t_prof_events[2 * j + 1]), st);
+    }
+};
 std::atomic<int> g_dispatch{EP_DISPATCH_AUTO};
 
 ep_status fail(ep_status s, const char *fmt, ...) {
@@ -198,6 +214,14 @@ extern "C" const char *ep_last_error(void) { return t_error; }
 
 extern "C" int32_t ep_last_launch_count(void) { return t_launches; }
 
+extern "C" ep_status ep_profile_events(void *const *events, int32_t n_events) {
+    if (n_events < 0)
+        return fail(EP_EINVAL, "ep_profile_events: n_events = %d < 0", n_events);
+    t_prof_events = n_events > 0 ? events : nullptr;
+    t_prof_n = events != nullptr ? n_events : 0;
+    return ok();
+}
+
 extern "C" ep_status ep_check_status(void *stream) {
     EP_CUDA_CHECK(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
     unsigned int v = 0, zero = 0;
@@ -249,6 +273,7 @@ extern "C" ep_status moe_route(const void *x, ep_dtype x_dtype, int64_t T, int64
     const int64_t nblk = (T + tb_max - 1) / tb_max;
     const dim3 grid((unsigned)(nblk * epk::kRouterCluster));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    KernelBracket kb0(st, 0);
     if (x_dtype == EP_F32)
         epk::router_topk_kernel<true><<<grid, epk::kRouterThreads, L.total, st>>>(
             x, T, (int)H, static_cast<const uint16_t *>(w_router), bias, (int)E, top_k, tb_max,
@@ -365,10 +390,13 @@ extern "C" ep_status moe_ffn_forward(const void *x, ep_dtype x_dtype, int64_t T,
         ga.h_routed = reinterpret_cast<float *>(ws + W.h_routed);
         ga.h_shared = reinterpret_cast<float *>(ws + W.h_shared);
         const dim3 gu_grid((unsigned)d->sm_count);
+        {
+        KernelBracket kb0(st, 0);
         if (x_dtype == EP_F32)
             epk::stream_gate_up_kernel<true><<<gu_grid, epk::kGUThreads, sp.gu_smem, st>>>(ga);
         else
             epk::stream_gate_up_kernel<false><<<gu_grid, epk::kGUThreads, sp.gu_smem, st>>>(ga);
+        }
         EP_CUDA_CHECK(cudaGetLastError());
 
         epk::StreamDownArgs da;
@@ -381,7 +409,10 @@ extern "C" ep_status moe_ffn_forward(const void *x, ep_dtype x_dtype, int64_t T,
         da.h_routed = ga.h_routed;
         da.h_shared = ga.h_shared;
         da.y = y;
-        epk::stream_down_fold_kernel<<<sp.down_grid, epk::kDownThreads, sp.down_smem, st>>>(da);
+        {
+            KernelBracket kb1(st, 1);
+            epk::stream_down_fold_kernel<<<sp.down_grid, epk::kDownThreads, sp.down_smem, st>>>(da);
+        }
         EP_CUDA_CHECK(cudaGetLastError());
         t_launches = 2;
         return ok();
@@ -398,7 +429,8 @@ extern "C" ep_status moe_ffn_forward(const void *x, ep_dtype x_dtype, int64_t T,
     g.smem_optin = d->smem_optin;
     int launches = 0;
     char why[256] = "";
-    s = epk::grouped_forward(g, W.grouped, ws, st, &launches, why, sizeof why);
+    s = epk::grouped_forward(g, W.grouped, ws, st, &launches, why, sizeof why,
+                             t_prof_events, t_prof_n);
     if (s != EP_OK)
         return fail(s, "moe_ffn_forward: %s", why);
     t_launches = launches;

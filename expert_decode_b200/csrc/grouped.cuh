@@ -710,8 +710,15 @@ inline ep_status grouped_set_attributes(int smem_optin) {
     return EP_OK;
 }
 
+// Records events[2j] / events[2j+1] around kernel j when a timing hook is set.
+inline void bracket_event(void *const *events, int n, int idx, cudaStream_t st) {
+    if (events != nullptr && idx < n && (idx | 1) < n)
+        cudaEventRecord(static_cast<cudaEvent_t>(events[idx]), st);
+}
+
 inline ep_status grouped_forward(const GroupedArgs &g, const GroupedWorkspace &W, uint8_t *ws,
-                                 cudaStream_t st, int *launches, char *why, size_t why_len) {
+                                 cudaStream_t st, int *launches, char *why, size_t why_len,
+                                 void *const *ev, int n_ev) {
     *launches = 0;
     const int64_t T = g.T, H = g.H, E = g.E, I = g.I, I_s = g.I_s;
     const int k = g.top_k;
@@ -741,7 +748,9 @@ inline ep_status grouped_forward(const GroupedArgs &g, const GroupedWorkspace &W
     pa.I = (int)I; pa.I_s = (int)I_s;
     pa.group_offset = group_offset; pa.perm_pair = perm_pair;
     pa.units_gu = units_gu; pa.units_dn = units_dn;
+    bracket_event(ev, n_ev, 0, st);
     group_plan_kernel<<<1, kPlanThreads, plan_smem_bytes(E), st>>>(pa);
+    bracket_event(ev, n_ev, 1, st);
     if (cudaGetLastError() != cudaSuccess) {
         snprintf(why, why_len, "group_plan launch failed");
         return EP_ECUDA;
@@ -750,9 +759,11 @@ inline ep_status grouped_forward(const GroupedArgs &g, const GroupedWorkspace &W
     {
         const int64_t rows = P + (I_s > 0 ? T : 0);
         const int64_t blocks = std::min<int64_t>((rows + 7) / 8, (int64_t)g.sm_count * 8);
+        bracket_event(ev, n_ev, 2, st);
         gather_rows_kernel<<<(unsigned)std::max<int64_t>(blocks, 1), 256, 0, st>>>(
             g.x, g.x_f32 ? 1 : 0, T, (int)H, k, P, (int)E, I_s > 0 ? 1 : 0, group_offset,
             perm_pair, x_perm);
+        bracket_event(ev, n_ev, 3, st);
         if (cudaGetLastError() != cudaSuccess) {
             snprintf(why, why_len, "gather_rows launch failed");
             return EP_ECUDA;
@@ -779,7 +790,9 @@ inline ep_status grouped_forward(const GroupedArgs &g, const GroupedWorkspace &W
     gp.weights = g.weights;
     gp.h_out = h_perm; gp.h_shared_out = h_shared; gp.I = (int)I; gp.I_s = (int)I_s;
     gp.c_out = c; gp.s_out = s; gp.H = (int)H;
+    bracket_event(ev, n_ev, 4, st);
     grouped_gemm_kernel<true><<<g.sm_count, kGemmThreads, GemmSmem::alloc, st>>>(gm, gp);
+    bracket_event(ev, n_ev, 5, st);
     if (cudaGetLastError() != cudaSuccess) {
         snprintf(why, why_len, "gate/up GEMM launch failed");
         return EP_ECUDA;
@@ -796,7 +809,9 @@ inline ep_status grouped_forward(const GroupedArgs &g, const GroupedWorkspace &W
     }
     gp.m_routed = (int)H; gp.m_shared = (int)H; gp.k_routed = (int)I; gp.k_shared = (int)I_s;
     gp.units = units_dn;
+    bracket_event(ev, n_ev, 6, st);
     grouped_gemm_kernel<false><<<g.sm_count, kGemmThreads, GemmSmem::alloc, st>>>(gm, gp);
+    bracket_event(ev, n_ev, 7, st);
     if (cudaGetLastError() != cudaSuccess) {
         snprintf(why, why_len, "down GEMM launch failed");
         return EP_ECUDA;
@@ -804,8 +819,10 @@ inline ep_status grouped_forward(const GroupedArgs &g, const GroupedWorkspace &W
     // 5. combine
     {
         const dim3 grid((unsigned)T, (unsigned)((H / 4 + 255) / 256));
+        bracket_event(ev, n_ev, 8, st);
         combine_kernel<<<grid, 256, 0, st>>>(c, I_s > 0 ? s : nullptr, g.ids, T, (int)H, k,
                                              (int)E, g.y);
+        bracket_event(ev, n_ev, 9, st);
         if (cudaGetLastError() != cudaSuccess) {
             snprintf(why, why_len, "combine launch failed");
             return EP_ECUDA;

@@ -170,6 +170,18 @@ const char *ep_last_error(void);
 /* Number of kernels the last successful call on this host thread launched. */
 int32_t ep_last_launch_count(void);
 
+/*
+ * ep_profile_events -- per-kernel timing aid.  While `events` is not NULL,
+ * every kernel that a later moe_route / moe_ffn_forward call on this host
+ * thread launches is bracketed on the call's stream by
+ * cudaEventRecord(events[2j]) and cudaEventRecord(events[2j+1]), j counting
+ * the kernels of that one call (kernels past n_events / 2 are not bracketed).
+ * `events` are cudaEvent_t handles the caller created and owns; the array is
+ * read at each call, so the caller may change its contents between calls.
+ * Pass NULL (or n_events = 0) to stop.  EP_EINVAL for n_events < 0.
+ */
+ep_status ep_profile_events(void *const *events, int32_t n_events);
+
 #ifdef __cplusplus
 }
 #endif
