@@ -52,6 +52,10 @@ def parse_args():
     ap.add_argument("--config", choices=tuple(workloads.WORKLOADS), default="decode")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=500)
+    ap.add_argument("--experts", type=int, default=0,
+                    help="profiling only: fewer experts (same H, I, top_k) to keep an ncu "
+                         "capture to a few GB on the device")
+    ap.add_argument("--flush-mib", type=int, default=FLUSH_BYTES >> 20)
     return ap.parse_args()
 
 
@@ -329,7 +333,7 @@ def run_ours(args, wl):
     layer = Layer(wl, device, workloads.SEED_BASE + 7919 * rank)
     Ts = wl.T
     tensor_path = {T: T > 8 for T in Ts}
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    flush = torch.empty(args.flush_mib << 20, dtype=torch.uint8, device=device)
 
     # per (T, batch): distinct experts picked (fixed for a given batch)
     n_batches = {T: len(layer.xs[T]) for T in Ts}
@@ -355,14 +359,6 @@ def run_ours(args, wl):
     K = args.steps
     ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    nk = 10
-    prof = [{T: [torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)] for T in Ts}
-            for _ in range(K)]
-    for p in prof:
-        for evs in p.values():
-            for e in evs:
-                e.record()
-    torch.cuda.synchronize()
     layer.launches = 0
     sampler = ClockSampler(device) if rank == 0 else None
     if dist is not None:
@@ -374,7 +370,7 @@ def run_ours(args, wl):
     for i in range(K):
         flush.zero_()
         ev_s[i].record()
-        step(args.warmup + i, prof[i])
+        step(args.warmup + i)
         ev_e[i].record()
     torch.cuda.synchronize()
     t_wall = time.perf_counter() - t_wall
@@ -384,6 +380,22 @@ def run_ours(args, wl):
     torch.cuda.synchronize()
     ed.ep_check_status()
     launches = layer.launches
+
+    # second pass of K steps, each kernel bracketed by its own events, for the
+    # dominant kernel's duration (events between launches stop the early
+    # launch of the next kernel, so the throughput above is taken without them)
+    nk = 10
+    prof = [{T: [torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)] for T in Ts}
+            for _ in range(K)]
+    for p in prof:
+        for evs in p.values():
+            for e in evs:
+                e.record()
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.zero_()
+        step(args.warmup + i, prof[i])
+    torch.cuda.synchronize()
 
     step_ms = [ev_s[i].elapsed_time(ev_e[i]) for i in range(K)]
     dev_s = sum(step_ms) / 1e3
@@ -489,7 +501,9 @@ def run_ours(args, wl):
         "config": {"workload": wl.description, "bands": wl.bands[0],
                    "l2": "flushed before every step (512 MiB write)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "batches": "16 distinct x batches per row count, cycled"},
+                   "batches": "16 distinct x batches per row count, cycled",
+                   "roofline_timing": "dominant kernel timed in a second pass of K steps "
+                                      "with events around each kernel"},
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": e2e,
@@ -507,6 +521,10 @@ def run_ours(args, wl):
 def main():
     args = parse_args()
     wl = workloads.WORKLOADS[args.config]
+    if args.experts:
+        import dataclasses
+        wl = dataclasses.replace(wl, E=args.experts, bands=(min(wl.bands[0], args.experts),),
+                                 description=wl.description + f" (E reduced to {args.experts})")
     if args.impl == "reference":
         run_reference(args, wl)
     else:

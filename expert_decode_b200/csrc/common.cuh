@@ -40,6 +40,20 @@ __device__ __forceinline__ uint16_t f32_to_bf16_rne(float f) {
     return (uint16_t)(u >> 16);
 }
 
+// Packed fp32 pairs: d = a * b + c per component (sm_100 packed FMA).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    unsigned long long ra = *reinterpret_cast<unsigned long long *>(&a);
+    unsigned long long rb = *reinterpret_cast<unsigned long long *>(&b);
+    unsigned long long rc = *reinterpret_cast<unsigned long long *>(&c);
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(rc) : "l"(ra), "l"(rb));
+    return *reinterpret_cast<float2 *>(&rc);
+}
+
+// The two bf16 of a 32-bit word as an fp32 pair (low half first).
+__device__ __forceinline__ float2 bf16x2_to_f2(uint32_t v) {
+    return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+}
+
 // silu(g) = g / (1 + e^-g), the SwiGLU gate activation.
 __device__ __forceinline__ float silu_f32(float g) { return g / (1.0f + expf(-g)); }
 
@@ -276,6 +290,31 @@ __device__ __forceinline__ uint32_t map_shared_rank(const void *p, uint32_t rank
 }
 __device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ void st_cluster_f64(uint32_t addr, double v) {
+    asm volatile("st.shared::cluster.f64 [%0], %1;" ::"r"(addr), "d"(v) : "memory");
+}
+__device__ __forceinline__ int ld_cluster_s32(uint32_t addr) {
+    int v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+// --------------------------------------------------------- named barriers
+// bar.sync / bar.red on barrier `id` (1..15) among `n` threads (multiple of 32).
+__device__ __forceinline__ void named_sync(uint32_t id, uint32_t n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ int named_count(uint32_t id, uint32_t n, bool pred) {
+    int r;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.u32 p, %3, 0;\n\t"
+        "bar.red.popc.u32 %0, %1, %2, p;\n\t}"
+        : "=r"(r)
+        : "r"(id), "r"(n), "r"((uint32_t)pred)
+        : "memory");
+    return r;
 }
 
 // ------------------------------------------------------------- global loads

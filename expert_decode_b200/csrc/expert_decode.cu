@@ -9,6 +9,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <cstdlib>
 #include <mutex>
 
 #include "../../include/expert_decode.h"
@@ -61,6 +62,33 @@ ep_status ok() {
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// Programmatic dependent launch: the kernel may start while the previous
+// kernel on the stream is still running; it reads that kernel's outputs only
+// after griddepcontrol.wait.  EXPERT_DECODE_NO_PDL=1 turns it off.
+bool pdl_enabled() {
+    static const bool on = [] {
+        const char *v = getenv("EXPERT_DECODE_NO_PDL");
+        return !(v != nullptr && v[0] == '1');
+    }();
+    return on;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                   Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 struct DeviceInfo {
     bool ready = false;
     int sm_count = 0;
@@ -93,9 +121,11 @@ ep_status device_info(const DeviceInfo **out) {
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, m));
         EP_CUDA_CHECK(cudaFuncSetAttribute(epk::router_topk_kernel<true>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, m));
-        EP_CUDA_CHECK(cudaFuncSetAttribute(epk::stream_gate_up_kernel<false>,
+        EP_CUDA_CHECK(cudaFuncSetAttribute(epk::stream_gate_up_kernel<false, false>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, m));
-        EP_CUDA_CHECK(cudaFuncSetAttribute(epk::stream_gate_up_kernel<true>,
+        EP_CUDA_CHECK(cudaFuncSetAttribute(epk::stream_gate_up_kernel<false, true>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, m));
+        EP_CUDA_CHECK(cudaFuncSetAttribute(epk::stream_gate_up_kernel<true, true>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, m));
         EP_CUDA_CHECK(cudaFuncSetAttribute(epk::stream_down_fold_kernel,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, m));
@@ -147,6 +177,7 @@ Workspace workspace_layout(int64_t T, int64_t H, int64_t E, int64_t k, int64_t I
 // --------------------------------------------------------- streaming path fit
 struct StreamingPlan {
     bool fits = false;
+    bool xs_f32 = false;  // gate/up keeps x as fp32 in shared memory
     int gu_slots = 0, down_slots = 0, down_grid = 0, down_rows_max = 0;
     size_t gu_smem = 0, down_smem = 0;
 };
@@ -157,24 +188,28 @@ StreamingPlan streaming_fit(const DeviceInfo &d, int64_t T, int64_t H, int xb, i
     if (T < 1 || T > epk::kStreamMaxT || k > epk::kStreamMaxK)
         return p;
     const size_t budget = std::min<size_t>(kStreamSmemBudget, (size_t)d.smem_optin);
+    // fp32 activations in shared memory skip the per-use unpacking; bf16 x
+    // is widened when it takes at most 64 KB
+    p.xs_f32 = xb == 4 || T * H * 4 <= 64 * 1024;
+    const int xsb = p.xs_f32 ? 4 : 2;
     int slots = epk::kGUMaxSlots;
-    while (slots >= 2 && epk::gate_up_smem_layout((int)T, (int)H, xb, slots).total > budget)
+    while (slots >= 2 && epk::gate_up_smem_layout((int)T, (int)H, xsb, slots).total > budget)
         --slots;
     if (slots < 2)
         return p;
     p.gu_slots = slots;
-    p.gu_smem = epk::gate_up_smem_layout((int)T, (int)H, xb, slots).total;
+    p.gu_smem = epk::gate_up_smem_layout((int)T, (int)H, xsb, slots).total;
     const int64_t I_max = std::max(I, I_s);
     p.down_grid = (int)std::max<int64_t>(1, std::min<int64_t>(d.sm_count, H / 8));
     p.down_rows_max = (int)((H + p.down_grid - 1) / p.down_grid);
     slots = epk::kDownMaxSlots;
     while (slots >= 2 &&
-           epk::down_smem_layout((int)I_max, slots, p.down_rows_max).total > budget)
+           epk::down_smem_layout((int)T, (int)I_max, slots, p.down_rows_max).total > budget)
         --slots;
     if (slots < 2)
         return p;
     p.down_slots = slots;
-    p.down_smem = epk::down_smem_layout((int)I_max, slots, p.down_rows_max).total;
+    p.down_smem = epk::down_smem_layout((int)T, (int)I_max, slots, p.down_rows_max).total;
     p.fits = true;
     return p;
 }
@@ -265,24 +300,25 @@ extern "C" ep_status moe_route(const void *x, ep_dtype x_dtype, int64_t T, int64
         return s;
     const int xb = x_dtype == EP_F32 ? 4 : 2;
     const int tb_max =
-        (int)std::max<int64_t>(1, std::min<int64_t>(epk::kRouterMaxTB, epk::kRouterXBudget / (H * xb)));
-    const epk::RouterSmem L = epk::router_smem_layout(tb_max, (int)H, xb, (int)E);
+        (int)std::max<int64_t>(1, std::min<int64_t>(epk::kRouterMaxTB, epk::kRouterXBudget / (H * 4)));
+    const epk::RouterSmem L = epk::router_smem_layout(tb_max, (int)H, (int)E);
     if ((int)L.total > d->smem_optin)
         return fail(EP_EINVAL, "moe_route: H = %lld, E = %lld need %u bytes of shared memory",
                     (long long)H, (long long)E, L.total);
     const int64_t nblk = (T + tb_max - 1) / tb_max;
     const dim3 grid((unsigned)(nblk * epk::kRouterCluster));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    KernelBracket kb0(st, 0);
-    if (x_dtype == EP_F32)
-        epk::router_topk_kernel<true><<<grid, epk::kRouterThreads, L.total, st>>>(
-            x, T, (int)H, static_cast<const uint16_t *>(w_router), bias, (int)E, top_k, tb_max,
-            ids, weights);
-    else
-        epk::router_topk_kernel<false><<<grid, epk::kRouterThreads, L.total, st>>>(
-            x, T, (int)H, static_cast<const uint16_t *>(w_router), bias, (int)E, top_k, tb_max,
-            ids, weights);
-    EP_CUDA_CHECK(cudaGetLastError());
+    {
+        KernelBracket kb0(st, 0);
+        const uint16_t *wr = static_cast<const uint16_t *>(w_router);
+        if (x_dtype == EP_F32)
+            EP_CUDA_CHECK(launch(epk::router_topk_kernel<true>, grid, epk::kRouterThreads, L.total,
+                                 st, x, T, (int)H, wr, bias, (int)E, top_k, tb_max, ids, weights));
+        else
+            EP_CUDA_CHECK(launch(epk::router_topk_kernel<false>, grid, epk::kRouterThreads,
+                                 L.total, st, x, T, (int)H, wr, bias, (int)E, top_k, tb_max, ids,
+                                 weights));
+    }
     t_launches = 1;
     return ok();
 }
@@ -391,13 +427,17 @@ extern "C" ep_status moe_ffn_forward(const void *x, ep_dtype x_dtype, int64_t T,
         ga.h_shared = reinterpret_cast<float *>(ws + W.h_shared);
         const dim3 gu_grid((unsigned)d->sm_count);
         {
-        KernelBracket kb0(st, 0);
-        if (x_dtype == EP_F32)
-            epk::stream_gate_up_kernel<true><<<gu_grid, epk::kGUThreads, sp.gu_smem, st>>>(ga);
-        else
-            epk::stream_gate_up_kernel<false><<<gu_grid, epk::kGUThreads, sp.gu_smem, st>>>(ga);
+            KernelBracket kb0(st, 0);
+            if (x_dtype == EP_F32)
+                EP_CUDA_CHECK(launch(epk::stream_gate_up_kernel<true, true>, gu_grid,
+                                     epk::kGUThreads, sp.gu_smem, st, ga));
+            else if (sp.xs_f32)
+                EP_CUDA_CHECK(launch(epk::stream_gate_up_kernel<false, true>, gu_grid,
+                                     epk::kGUThreads, sp.gu_smem, st, ga));
+            else
+                EP_CUDA_CHECK(launch(epk::stream_gate_up_kernel<false, false>, gu_grid,
+                                     epk::kGUThreads, sp.gu_smem, st, ga));
         }
-        EP_CUDA_CHECK(cudaGetLastError());
 
         epk::StreamDownArgs da;
         da.T = (int)T; da.H = (int)H; da.E = (int)E; da.I = (int)I; da.I_s = (int)I_s;
@@ -411,9 +451,9 @@ extern "C" ep_status moe_ffn_forward(const void *x, ep_dtype x_dtype, int64_t T,
         da.y = y;
         {
             KernelBracket kb1(st, 1);
-            epk::stream_down_fold_kernel<<<sp.down_grid, epk::kDownThreads, sp.down_smem, st>>>(da);
+            EP_CUDA_CHECK(launch(epk::stream_down_fold_kernel, dim3((unsigned)sp.down_grid),
+                                 epk::kDownThreads, sp.down_smem, st, da));
         }
-        EP_CUDA_CHECK(cudaGetLastError());
         t_launches = 2;
         return ok();
     }

@@ -6,15 +6,21 @@
 // lower expert id, weights renormalised over the picked set.
 //
 // One thread-block cluster of kRouterCluster CTAs handles a block of up to
-// kRouterMaxTB tokens.  CTA r of the cluster computes the fp32 logits of its
-// slice of experts for those tokens (the x block sits in its shared memory,
-// the router rows stream from HBM with 16-byte loads), together with a
-// rigorous bound on each logit's rounding error, and stores both into the
-// shared memory of CTA 0 (distributed shared memory).  CTA 0 then finds, per
-// token, every expert that could belong to the exact top-k under those bounds,
-// recomputes exactly those logits in fp64, and makes the pick and the weights
-// from the fp64 values.  The selection and the weights are therefore those of
-// exact arithmetic up to fp64 rounding.
+// kRouterMaxTB tokens; CTA r owns a contiguous slice of the experts.
+//  1. Each CTA holds the block's activations in shared memory as fp32.
+//  2. Each warp computes, for one expert row of its CTA's slice at a time,
+//     the fp32 logits of all the block's tokens (the row streams from HBM
+//     with one round of 16-byte loads per lane) and a rigorous bound on each
+//     logit's rounding error; both go to CTA 0 through distributed shared
+//     memory.
+//  3. CTA 0 finds, per token, every expert whose exact logit could reach the
+//     k-th largest under those bounds (the candidates).
+//  4. Every CTA recomputes its own candidates' logits in fp64 and sends them
+//     back to CTA 0.
+//  5. CTA 0 picks the top_k on the fp64 logits (ties to the lower id), orders
+//     them by descending logit and renormalises the softmax over them in fp64.
+// The selection and the weights are therefore those of exact arithmetic up to
+// fp64 rounding.
 #pragma once
 
 #include "common.cuh"
@@ -27,7 +33,8 @@ constexpr int kRouterWarps = kRouterThreads / 32;
 constexpr int kRouterMaxTB = 8;        // tokens per cluster
 constexpr int kRouterMaxK = 16;
 constexpr int kRouterMaxCand = 64;     // fp64 candidates per token handled in parallel
-constexpr int kRouterXBudget = 96 * 1024;
+constexpr int kRouterXBudget = 128 * 1024;  // fp32 activations of one token block
+constexpr int kRouterRowChunks = 16;   // 16-byte chunks of a router row per lane per round
 
 struct RouterSmem {
     // byte offsets into dynamic shared memory
@@ -36,10 +43,10 @@ struct RouterSmem {
 
 __host__ __device__ inline uint32_t align_up_u32(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
-__host__ __device__ inline RouterSmem router_smem_layout(int tb_max, int H, int x_bytes, int E) {
+__host__ __device__ inline RouterSmem router_smem_layout(int tb_max, int H, int E) {
     RouterSmem s;
     uint32_t o = 0;
-    s.x = o;        o = align_up_u32(o + (uint32_t)tb_max * H * x_bytes, 16);
+    s.x = o;        o = align_up_u32(o + (uint32_t)tb_max * H * 4, 16);
     s.logit = o;    o = align_up_u32(o + (uint32_t)kRouterMaxTB * E * 4, 16);
     s.bound = o;    o = align_up_u32(o + (uint32_t)kRouterMaxTB * E * 4, 16);
     s.xnorm2 = o;   o = align_up_u32(o + kRouterMaxTB * 4, 16);
@@ -52,42 +59,43 @@ __host__ __device__ inline RouterSmem router_smem_layout(int tb_max, int H, int 
     return s;
 }
 
-// Eight activations of token row `xs_row` at 16-byte chunk c, as floats.
-template <bool XF32>
-__device__ __forceinline__ void load_x8(const uint8_t *xs_row, int c, float (&xf)[8]) {
-    if constexpr (XF32) {
-        const float4 *p = reinterpret_cast<const float4 *>(xs_row) + 2 * c;
-        float4 a = p[0], b = p[1];
-        xf[0] = a.x; xf[1] = a.y; xf[2] = a.z; xf[3] = a.w;
-        xf[4] = b.x; xf[5] = b.y; xf[6] = b.z; xf[7] = b.w;
-    } else {
-        uint4 v = reinterpret_cast<const uint4 *>(xs_row)[c];
-        xf[0] = bf16_lo(v.x); xf[1] = bf16_hi(v.x); xf[2] = bf16_lo(v.y); xf[3] = bf16_hi(v.y);
-        xf[4] = bf16_lo(v.z); xf[5] = bf16_hi(v.z); xf[6] = bf16_lo(v.w); xf[7] = bf16_hi(v.w);
-    }
-}
-
 __device__ __forceinline__ void unpack_w8(uint4 v, float (&wf)[8]) {
     wf[0] = bf16_lo(v.x); wf[1] = bf16_hi(v.x); wf[2] = bf16_lo(v.y); wf[3] = bf16_hi(v.y);
     wf[4] = bf16_lo(v.z); wf[5] = bf16_hi(v.z); wf[6] = bf16_lo(v.w); wf[7] = bf16_hi(v.w);
 }
 
-// fp64 logit of expert e for the token whose activations are at xs_row.
-template <bool XF32>
-__device__ double logit_fp64(const uint8_t *xs_row, const uint16_t *__restrict__ w_router,
+// fp64 logit of expert e for the token whose fp32 activations are at xrow.
+__device__ double logit_fp64(const float *xrow, const uint16_t *__restrict__ w_router,
                              const float *__restrict__ bias, int H, int e) {
     const int lane = (int)lane_id();
     const int nck = H >> 3;
-    const uint16_t *wrow = w_router + (size_t)e * H;
+    const uint4 *wrow = reinterpret_cast<const uint4 *>(w_router + (size_t)e * H);
     double acc = 0.0;
-    for (int c = lane; c < nck; c += 32) {
-        uint4 wv = *reinterpret_cast<const uint4 *>(wrow + (size_t)c * 8);
-        float wf[8], xf[8];
-        unpack_w8(wv, wf);
-        load_x8<XF32>(xs_row, c, xf);
+    for (int base = 0; base < nck; base += 32 * kRouterRowChunks) {
+        uint4 wv[kRouterRowChunks];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-            acc = fma((double)xf[j], (double)wf[j], acc);
+        for (int u = 0; u < kRouterRowChunks; ++u) {
+            const int c = base + lane + 32 * u;
+            wv[u] = c < nck ? wrow[c] : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < kRouterRowChunks; ++u) {
+            const int c = base + lane + 32 * u;
+            if (c < nck) {
+                float wf[8];
+                unpack_w8(wv[u], wf);
+                const float4 *xp = reinterpret_cast<const float4 *>(xrow) + 2 * c;
+                const float4 a = xp[0], b = xp[1];
+                acc = fma((double)a.x, (double)wf[0], acc);
+                acc = fma((double)a.y, (double)wf[1], acc);
+                acc = fma((double)a.z, (double)wf[2], acc);
+                acc = fma((double)a.w, (double)wf[3], acc);
+                acc = fma((double)b.x, (double)wf[4], acc);
+                acc = fma((double)b.y, (double)wf[5], acc);
+                acc = fma((double)b.z, (double)wf[6], acc);
+                acc = fma((double)b.w, (double)wf[7], acc);
+            }
+        }
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1)
@@ -97,6 +105,36 @@ __device__ double logit_fp64(const uint8_t *xs_row, const uint16_t *__restrict__
     return acc;
 }
 
+// Index of the k-th largest fp32 logit of one token (ties to the lower id),
+// computed by a warp; `chosen` keeps the picked lanes' bits.
+__device__ float kth_logit(const float *lt, int E, int top_k) {
+    const int lane = (int)lane_id();
+    const int per_lane = (E + 31) / 32;  // <= 32
+    uint32_t chosen = 0;
+    float vk = -INFINITY;
+    for (int r = 0; r < top_k; ++r) {
+        float bv = -INFINITY;
+        int be = 0x7fffffff;
+        for (int i = 0; i < per_lane; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E && !((chosen >> i) & 1u)) {
+                const float v = lt[e];
+                if (v > bv || (v == bv && e < be)) { bv = v; be = e; }
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+            if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+        }
+        if (be != 0x7fffffff && (be & 31) == lane)
+            chosen |= 1u << (be >> 5);
+        vk = bv;
+    }
+    return vk;
+}
+
 template <bool XF32>
 __global__ void __cluster_dims__(kRouterCluster, 1, 1) __launch_bounds__(kRouterThreads, 1)
 router_topk_kernel(const void *__restrict__ x, int64_t T, int H,
@@ -104,16 +142,19 @@ router_topk_kernel(const void *__restrict__ x, int64_t T, int H,
                    int top_k, int tb_max, int32_t *__restrict__ ids, float *__restrict__ weights) {
     extern __shared__ __align__(1024) uint8_t smem[];
     constexpr int XB = XF32 ? 4 : 2;
-    const RouterSmem L = router_smem_layout(tb_max, H, XB, E);
-    uint8_t *xs = smem + L.x;
+    const RouterSmem L = router_smem_layout(tb_max, H, E);
+    float *xs = reinterpret_cast<float *>(smem + L.x);            // [tb][H] fp32
     float *logit = reinterpret_cast<float *>(smem + L.logit);     // [kRouterMaxTB][E], CTA 0
     float *bound = reinterpret_cast<float *>(smem + L.bound);     // [kRouterMaxTB][E], CTA 0
     float *xnorm2 = reinterpret_cast<float *>(smem + L.xnorm2);
-    int *ncand = reinterpret_cast<int *>(smem + L.ncand);
-    int *cand = reinterpret_cast<int *>(smem + L.cand);
-    double *cval = reinterpret_cast<double *>(smem + L.cval);
+    int *ncand = reinterpret_cast<int *>(smem + L.ncand);         // CTA 0
+    int *cand = reinterpret_cast<int *>(smem + L.cand);           // CTA 0
+    double *cval = reinterpret_cast<double *>(smem + L.cval);     // CTA 0
     double *list_val = reinterpret_cast<double *>(smem + L.list_val);
     int *list_id = reinterpret_cast<int *>(smem + L.list_id);
+
+    grid_dependents_launch();
+    grid_dependency_wait();  // x may come from the previous kernel; ids / weights are read there
 
     const uint32_t rank = cluster_ctarank();
     const int64_t t0 = (int64_t)(blockIdx.x / kRouterCluster) * tb_max;
@@ -121,26 +162,49 @@ router_topk_kernel(const void *__restrict__ x, int64_t T, int H,
     const int warp = (int)(threadIdx.x >> 5);
     const int lane = (int)lane_id();
     const int nck = H >> 3;
+    const int per_cta = (E + kRouterCluster - 1) / kRouterCluster;
+    const int e_lo = (int)rank * per_cta;
+    const int e_hi = min(E, e_lo + per_cta);
 
-    // ---- phase 1: this block's activations into shared memory, ||x_t||^2
+    // ---- 1. this block's activations as fp32, ||x_t||^2
     {
         const uint4 *src = reinterpret_cast<const uint4 *>(
             reinterpret_cast<const uint8_t *>(x) + (size_t)t0 * H * XB);
-        uint4 *dst = reinterpret_cast<uint4 *>(xs);
         const int n16 = tb * H * XB / 16;
-        for (int i = threadIdx.x; i < n16; i += kRouterThreads)
-            dst[i] = src[i];
+        for (int i0 = threadIdx.x; i0 < n16; i0 += 4 * kRouterThreads) {
+            uint4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + u * kRouterThreads;
+                v[u] = i < n16 ? src[i] : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + u * kRouterThreads;
+                if (i < n16) {
+                    if constexpr (XF32) {
+                        reinterpret_cast<uint4 *>(xs)[i] = v[u];
+                    } else {
+                        float f[8];
+                        unpack_w8(v[u], f);
+                        float4 *d = reinterpret_cast<float4 *>(xs) + 2 * i;
+                        d[0] = make_float4(f[0], f[1], f[2], f[3]);
+                        d[1] = make_float4(f[4], f[5], f[6], f[7]);
+                    }
+                }
+            }
+        }
     }
     __syncthreads();
     if (warp < tb) {
-        const uint8_t *row = xs + (size_t)warp * H * XB;
+        const float4 *row = reinterpret_cast<const float4 *>(xs + (size_t)warp * H);
         float s = 0.f;
-        for (int c = lane; c < nck; c += 32) {
-            float xf[8];
-            load_x8<XF32>(row, c, xf);
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-                s = fmaf(xf[j], xf[j], s);
+        for (int c = lane; c < H / 4; c += 32) {
+            const float4 v = row[c];
+            s = fmaf(v.x, v.x, s);
+            s = fmaf(v.y, v.y, s);
+            s = fmaf(v.z, v.z, s);
+            s = fmaf(v.w, v.w, s);
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1)
@@ -150,11 +214,8 @@ router_topk_kernel(const void *__restrict__ x, int64_t T, int H,
     }
     cluster_sync();  // every CTA of the cluster is running; x block and norms visible
 
-    // ---- phase 2: fp32 logits of this CTA's experts, with error bounds
+    // ---- 2. fp32 logits of this CTA's experts, with error bounds, to CTA 0
     {
-        const int per_cta = (E + kRouterCluster - 1) / kRouterCluster;
-        const int e_lo = (int)rank * per_cta;
-        const int e_hi = min(E, e_lo + per_cta);
         const uint32_t r_logit = map_shared_rank(logit, 0);
         const uint32_t r_bound = map_shared_rank(bound, 0);
         // Each lane folds at most n_lane products with fused multiply-adds,
@@ -170,22 +231,39 @@ router_topk_kernel(const void *__restrict__ x, int64_t T, int H,
             for (int t = 0; t < kRouterMaxTB; ++t)
                 acc[t] = 0.f;
             float wsq = 0.f;
-            const uint16_t *wrow = w_router + (size_t)e * H;
-#pragma unroll 2
-            for (int c = lane; c < nck; c += 32) {
-                float wf[8];
-                unpack_w8(ld_stream_16(wrow + (size_t)c * 8), wf);
+            const uint4 *wrow = reinterpret_cast<const uint4 *>(w_router + (size_t)e * H);
+            for (int base = 0; base < nck; base += 32 * kRouterRowChunks) {
+                uint4 wv[kRouterRowChunks];
 #pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    wsq = fmaf(wf[j], wf[j], wsq);
+                for (int q = 0; q < kRouterRowChunks; ++q) {
+                    const int c = base + lane + 32 * q;
+                    wv[q] = c < nck ? ld_stream_16(wrow + c) : make_uint4(0u, 0u, 0u, 0u);
+                }
 #pragma unroll
-                for (int t = 0; t < kRouterMaxTB; ++t) {
-                    if (t < tb) {
-                        float xf[8];
-                        load_x8<XF32>(xs + (size_t)t * H * XB, c, xf);
+                for (int q = 0; q < kRouterRowChunks; ++q) {
+                    const int c = base + lane + 32 * q;
+                    if (c < nck) {
+                        float wf[8];
+                        unpack_w8(wv[q], wf);
 #pragma unroll
                         for (int j = 0; j < 8; ++j)
-                            acc[t] = fmaf(xf[j], wf[j], acc[t]);
+                            wsq = fmaf(wf[j], wf[j], wsq);
+#pragma unroll
+                        for (int t = 0; t < kRouterMaxTB; ++t) {
+                            if (t < tb) {
+                                const float4 *xp =
+                                    reinterpret_cast<const float4 *>(xs + (size_t)t * H) + 2 * c;
+                                const float4 a = xp[0], b = xp[1];
+                                acc[t] = fmaf(a.x, wf[0], acc[t]);
+                                acc[t] = fmaf(a.y, wf[1], acc[t]);
+                                acc[t] = fmaf(a.z, wf[2], acc[t]);
+                                acc[t] = fmaf(a.w, wf[3], acc[t]);
+                                acc[t] = fmaf(b.x, wf[4], acc[t]);
+                                acc[t] = fmaf(b.y, wf[5], acc[t]);
+                                acc[t] = fmaf(b.z, wf[6], acc[t]);
+                                acc[t] = fmaf(b.w, wf[7], acc[t]);
+                            }
+                        }
                     }
                 }
             }
@@ -210,37 +288,13 @@ router_topk_kernel(const void *__restrict__ x, int64_t T, int H,
         }
     }
     cluster_sync();  // all logits and bounds are in CTA 0
-    if (rank != 0)
-        return;
 
-    // ---- phase 3 (CTA 0): candidates per token
-    if (warp < tb) {
+    // ---- 3. CTA 0: candidates per token
+    if (rank == 0 && warp < tb) {
         const int t = warp;
         const float *lt = logit + t * E;
         const float *bt = bound + t * E;
-        const int per_lane = (E + 31) / 32;  // <= 32
-        uint32_t chosen = 0;
-        float vk = -INFINITY;
-        for (int r = 0; r < top_k; ++r) {
-            float bv = -INFINITY;
-            int be = 0x7fffffff;
-            for (int i = 0; i < per_lane; ++i) {
-                const int e = lane + 32 * i;
-                if (e < E && !((chosen >> i) & 1u)) {
-                    const float v = lt[e];
-                    if (v > bv || (v == bv && e < be)) { bv = v; be = e; }
-                }
-            }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-                const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-                if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
-            }
-            if (be != 0x7fffffff && (be & 31) == lane)
-                chosen |= 1u << (be >> 5);
-            vk = bv;
-        }
+        const float vk = kth_logit(lt, E, top_k);
         float dmax = 0.f;
         for (int e = lane; e < E; e += 32)
             dmax = fmaxf(dmax, bt[e]);
@@ -250,7 +304,7 @@ router_topk_kernel(const void *__restrict__ x, int64_t T, int H,
         // every expert whose exact logit could reach the k-th one
         const double thr = (double)vk - 2.0 * (double)dmax * 1.0001;
         int count = 0;
-        for (int i = 0; i < per_lane; ++i) {
+        for (int i = 0; i < (E + 31) / 32; ++i) {
             const int e = lane + 32 * i;
             const bool c = e < E && (double)lt[e] >= thr;
             const uint32_t m = __ballot_sync(0xffffffffu, c);
@@ -262,33 +316,54 @@ router_topk_kernel(const void *__restrict__ x, int64_t T, int H,
         if (lane == 0)
             ncand[t] = count;
     }
-    __syncthreads();
+    cluster_sync();  // candidate lists visible to every CTA
 
-    // ---- fp64 logits of the candidates, all warps in parallel
+    // ---- 4. every CTA: fp64 logits of the candidates in its expert slice
     {
-        // (token, candidate) pairs of the tokens with at most kRouterMaxCand
-        // candidates, enumerated token by token
+        // CTAs other than 0 copy CTA 0's candidate lists into their own arrays
+        const uint32_t r_ncand = map_shared_rank(ncand, 0);
+        const uint32_t r_cand = map_shared_rank(cand, 0);
+        const uint32_t r_cval = map_shared_rank(cval, 0);
+        if (rank != 0) {
+            if (threadIdx.x < (unsigned)tb)
+                ncand[threadIdx.x] = ld_cluster_s32(r_ncand + 4u * threadIdx.x);
+            for (int i = threadIdx.x; i < tb * kRouterMaxCand; i += kRouterThreads)
+                cand[i] = ld_cluster_s32(r_cand + 4u * (uint32_t)i);
+        }
+        __syncthreads();
+        int nc[kRouterMaxTB];
         int total = 0;
-        for (int t = 0; t < tb; ++t)
-            total += ncand[t] <= kRouterMaxCand ? ncand[t] : 0;
-        for (int p = warp; p < total; p += kRouterWarps) {
+#pragma unroll
+        for (int t = 0; t < kRouterMaxTB; ++t) {
+            nc[t] = 0;
+            if (t < tb)
+                nc[t] = ncand[t] <= kRouterMaxCand ? ncand[t] : 0;  // larger sets: CTA 0 fallback
+            total += nc[t];
+        }
+        // (token, candidate) pairs, token by token; the warps of the CTA that
+        // owns the expert split them by the expert's place in the slice
+        for (int p = 0; p < total; ++p) {
             int t = 0, ci = p;
-            while (true) {
-                const int c = ncand[t] <= kRouterMaxCand ? ncand[t] : 0;
-                if (ci < c)
-                    break;
-                ci -= c;
-                ++t;
+#pragma unroll
+            for (int q = 0; q < kRouterMaxTB; ++q) {
+                if (t == q && ci >= nc[q]) {
+                    ci -= nc[q];
+                    ++t;
+                }
             }
             const int e = cand[t * kRouterMaxCand + ci];
-            const double v = logit_fp64<XF32>(xs + (size_t)t * H * XB, w_router, bias, H, e);
+            if (e < e_lo || e >= e_hi || ((e - e_lo) % kRouterWarps) != warp)
+                continue;
+            const double v = logit_fp64(xs + (size_t)t * H, w_router, bias, H, e);
             if (lane == 0)
-                cval[t * kRouterMaxCand + ci] = v;
+                st_cluster_f64(r_cval + 8u * (uint32_t)(t * kRouterMaxCand + ci), v);
         }
     }
-    __syncthreads();
+    cluster_sync();  // fp64 logits are in CTA 0
+    if (rank != 0)
+        return;
 
-    // ---- pick top_k on the fp64 logits, renormalise, write
+    // ---- 5. CTA 0: pick top_k on the fp64 logits, renormalise, write
     if (warp < tb) {
         const int t = warp;
         const int nc = ncand[t];
@@ -320,8 +395,8 @@ router_topk_kernel(const void *__restrict__ x, int64_t T, int H,
             }
         } else {
             // Degenerate input (more than kRouterMaxCand experts within the
-            // bound of the k-th logit): stream every candidate through a
-            // sorted top_k list, in ascending expert id.
+            // bound of the k-th logit): stream every candidate, in ascending
+            // id, through a sorted top_k list.
             const float *lt = logit + t * E;
             float dmax = 0.f;
             for (int e = lane; e < E; e += 32)
@@ -329,38 +404,12 @@ router_topk_kernel(const void *__restrict__ x, int64_t T, int H,
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1)
                 dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, off));
-            // the k-th fp32 logit again (the candidate test of phase 3)
-            float vk = -INFINITY;
-            {
-                uint32_t chosen = 0;
-                const int per_lane = (E + 31) / 32;
-                for (int r = 0; r < top_k; ++r) {
-                    float bv = -INFINITY;
-                    int be = 0x7fffffff;
-                    for (int i = 0; i < per_lane; ++i) {
-                        const int e = lane + 32 * i;
-                        if (e < E && !((chosen >> i) & 1u)) {
-                            const float v = lt[e];
-                            if (v > bv || (v == bv && e < be)) { bv = v; be = e; }
-                        }
-                    }
-#pragma unroll
-                    for (int off = 16; off > 0; off >>= 1) {
-                        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-                        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-                        if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
-                    }
-                    if (be != 0x7fffffff && (be & 31) == lane)
-                        chosen |= 1u << (be >> 5);
-                    vk = bv;
-                }
-            }
-            const double thr = (double)vk - 2.0 * (double)dmax * 1.0001;
+            const double thr = (double)kth_logit(lt, E, top_k) - 2.0 * (double)dmax * 1.0001;
             int n = 0;
             for (int e = 0; e < E; ++e) {
                 if ((double)lt[e] < thr)
                     continue;
-                const double v = logit_fp64<XF32>(xs + (size_t)t * H * XB, w_router, bias, H, e);
+                const double v = logit_fp64(xs + (size_t)t * H, w_router, bias, H, e);
                 if (lane == 0) {
                     if (n < top_k || v > lv[top_k - 1]) {
                         int pos = n < top_k ? n : top_k - 1;
@@ -379,15 +428,13 @@ router_topk_kernel(const void *__restrict__ x, int64_t T, int H,
             }
         }
         __syncwarp();
-        if (lane == 0) {
+        if (lane < top_k) {
             const double m = lv[0];
             double s = 0.0;
             for (int j = 0; j < top_k; ++j)
                 s += exp(lv[j] - m);
-            for (int j = 0; j < top_k; ++j) {
-                ids[(t0 + t) * top_k + j] = li[j];
-                weights[(t0 + t) * top_k + j] = (float)(exp(lv[j] - m) / s);
-            }
+            ids[(t0 + t) * top_k + lane] = li[lane];
+            weights[(t0 + t) * top_k + lane] = (float)(exp(lv[lane] - m) / s);
         }
     }
 }

@@ -4,22 +4,29 @@
 // Only the picked experts' weights are read, each exactly once for all the
 // tokens that picked it, with 1-D bulk copies (cp.async.bulk) into a ring of
 // shared-memory slots that a producer warp keeps full while consumer warps
-// compute on CUDA cores.  Products are bf16 x bf16 (or fp32 x bf16) folded in
+// compute on CUDA cores with packed fp32 FMAs (fma.rn.f32x2).  Products are bf16 x bf16 (or fp32 x bf16) folded in
 // fp32; the SwiGLU activations stay fp32 between the two projections.
 //
 // Two kernels:
-//  * stream_gate_up: per (picked expert, row i of I) task, the dots of the
-//    expert's W_gate and W_up rows with the x of every token that picked it,
-//    then h = silu(g) * u (expertSwiGLU, fak note "GLM-5.2 multi-GPU: expert-
-//    parallel sharding", "What is not yet" update).
+//  * stream_gate_up: per (picked expert, unit i of I) task, the dots of the
+//    expert's W_gate row and W_up row with the x of every token that picked
+//    it, then h = silu(g) * u (expertSwiGLU, fak note "GLM-5.2 multi-GPU:
+//    expert-parallel sharding", "What is not yet" update).  Each task's
+//    inner loop is specialised on its token count (1..8).
 //  * stream_down_fold: each CTA owns a contiguous slice of the H output
-//    features and walks the picked experts in ascending (id, repeat) order,
-//    then the shared expert, folding w * (W_down h) into one fp32 running sum
-//    per (feature, token).  That walk is the bands in rank order with the
-//    carry passed along (TensorFold issue #310, maintainer's reply: one fixed
-//    sum order however the slices fall over ranks), so y does not depend on
-//    the plan; the shared expert enters after the routed sum (the GLM shared-
-//    expert wrapper of the fak note's gate table).
+//    features.  It computes the shared expert's share first, then walks the
+//    picked experts in ascending (id, repeat) order, folding w * (W_down h)
+//    into one fp32 running sum per (feature, token); y = routed + shared.
+//    The walk is the bands in rank order with the carry passed along
+//    (TensorFold issue #310, maintainer's reply: one fixed sum order however
+//    the slices fall over ranks), so y does not depend on the plan; the
+//    shared expert enters after the routed sum (the GLM shared-expert wrapper
+//    of the fak note's gate table).
+//
+// Both kernels are launched as programmatic dependents: before
+// griddepcontrol.wait they only prefetch the shared expert's weight rows
+// (which no kernel writes) into their rings; every read of x, ids, routing
+// weights or h, and every global write, comes after the wait.
 #pragma once
 
 #include "common.cuh"
@@ -29,6 +36,7 @@ namespace epk {
 constexpr int kStreamMaxT = 8;
 constexpr int kStreamMaxK = 16;
 constexpr int kStreamMaxPairs = kStreamMaxT * kStreamMaxK;
+constexpr int kChunkUnroll = 4;  // 16-byte chunks in flight per lane
 
 // The picks of up to 8 tokens grouped by expert, in fold order.  A group is
 // one (expert, repeat) pair: a token that picks the same expert twice has its
@@ -48,16 +56,16 @@ struct StreamPlan {
     int sorted_src[kStreamMaxPairs];
 };
 
-// Built by every CTA from ids (<= 128 picks): sort key (expert, repeat, token).
-// Needs blockDim.x >= kStreamMaxPairs.  Ends with __syncthreads().
+// Built from ids (<= 128 picks) by `nthr` (>= 128) threads with local ids
+// ltid, synchronised on named barrier `bar`; sort key (expert, repeat, token).
 __device__ void build_stream_plan(StreamPlan &P, const int32_t *__restrict__ ids,
-                                  const float *__restrict__ weights, int T, int k, int E) {
-    const int tid = threadIdx.x;
+                                  const float *__restrict__ weights, int T, int k, int E,
+                                  int ltid, uint32_t nthr, uint32_t bar) {
     const int np = T * k;
     int key = 0x7fffffff;
-    if (tid < np) {
-        const int e = ids[tid];
-        const int t = tid / k, j = tid - t * k;
+    if (ltid < np) {
+        const int e = ids[ltid];
+        const int t = ltid / k, j = ltid - t * k;
         if (e >= 0 && e < E) {
             int rep = 0;
             for (int q = 0; q < j; ++q)
@@ -67,19 +75,19 @@ __device__ void build_stream_plan(StreamPlan &P, const int32_t *__restrict__ ids
             flag_status(kStatusBadId);
         }
     }
-    if (tid < kStreamMaxPairs)
-        P.keys[tid] = key;
-    const int nvalid = __syncthreads_count(tid < np && key != 0x7fffffff);
-    if (tid < np && key != 0x7fffffff) {
+    if (ltid < kStreamMaxPairs)
+        P.keys[ltid] = key;
+    const int nvalid = named_count(bar, nthr, ltid < np && key != 0x7fffffff);
+    if (ltid < np && key != 0x7fffffff) {
         int r = 0;
         for (int q = 0; q < np; ++q)
             r += P.keys[q] < key;
         P.sorted_key[r] = key;
-        P.sorted_src[r] = tid;
+        P.sorted_src[r] = ltid;
     }
-    __syncthreads();
-    if (tid < 32) {
-        const int lane = tid;
+    named_sync(bar, nthr);
+    if (ltid < 32) {
+        const int lane = ltid;
         int base = 0;
         for (int r0 = 0; r0 < nvalid; r0 += 32) {
             const int r = r0 + lane;
@@ -99,50 +107,204 @@ __device__ void build_stream_plan(StreamPlan &P, const int32_t *__restrict__ ids
             P.n_pairs = nvalid;
         }
     }
-    if (tid < nvalid) {
-        const int src = P.sorted_src[tid];
+    if (ltid < nvalid) {
+        const int src = P.sorted_src[ltid];
         const int t = src / k;
-        P.pair_token[tid] = (int8_t)t;
-        P.pair_weight[tid] = weights[src];
+        P.pair_token[ltid] = (int8_t)t;
+        P.pair_weight[ltid] = weights[src];
         bool first = true;
-        for (int q = 0; q < tid; ++q)
+        for (int q = 0; q < ltid; ++q)
             first &= (P.sorted_key[q] % kStreamMaxT) != t;
-        P.pair_is_first[tid] = first;
+        P.pair_is_first[ltid] = first;
     }
-    if (tid < T) {
+    if (ltid < T) {
         bool has = false;
         for (int q = 0; q < nvalid; ++q)
-            has |= (P.sorted_key[q] % kStreamMaxT) == tid;
-        P.token_has_pick[tid] = has;
+            has |= (P.sorted_key[q] % kStreamMaxT) == ltid;
+        P.token_has_pick[ltid] = has;
     }
-    __syncthreads();
-}
-
-template <bool XF32>
-__device__ __forceinline__ void x8_from_smem(const uint8_t *xs_row, int c, float (&xf)[8]) {
-    if constexpr (XF32) {
-        const float4 *p = reinterpret_cast<const float4 *>(xs_row) + 2 * c;
-        const float4 a = p[0], b = p[1];
-        xf[0] = a.x; xf[1] = a.y; xf[2] = a.z; xf[3] = a.w;
-        xf[4] = b.x; xf[5] = b.y; xf[6] = b.z; xf[7] = b.w;
-    } else {
-        const uint4 v = reinterpret_cast<const uint4 *>(xs_row)[c];
-        xf[0] = bf16_lo(v.x); xf[1] = bf16_hi(v.x); xf[2] = bf16_lo(v.y); xf[3] = bf16_hi(v.y);
-        xf[4] = bf16_lo(v.z); xf[5] = bf16_hi(v.z); xf[6] = bf16_lo(v.w); xf[7] = bf16_hi(v.w);
-    }
-}
-
-__device__ __forceinline__ void w8_unpack(const uint4 v, float (&wf)[8]) {
-    wf[0] = bf16_lo(v.x); wf[1] = bf16_hi(v.x); wf[2] = bf16_lo(v.y); wf[3] = bf16_hi(v.y);
-    wf[4] = bf16_lo(v.z); wf[5] = bf16_hi(v.z); wf[6] = bf16_lo(v.w); wf[7] = bf16_hi(v.w);
+    named_sync(bar, nthr);
 }
 
 __host__ __device__ inline size_t align_up_sz(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// Eight bf16 weights as four fp32 pairs.
+__device__ __forceinline__ void w_pairs(const uint4 v, float2 (&wp)[4]) {
+    wp[0] = bf16x2_to_f2(v.x);
+    wp[1] = bf16x2_to_f2(v.y);
+    wp[2] = bf16x2_to_f2(v.z);
+    wp[3] = bf16x2_to_f2(v.w);
+}
+
+// Eight activations of 16-byte weight chunk c as four fp32 pairs, from a row
+// held in shared memory as fp32 (XS_F32) or bf16.
+template <bool XS_F32>
+__device__ __forceinline__ void x_pairs(const uint8_t *xrow, int c, float2 (&xp)[4]) {
+    if constexpr (XS_F32) {
+        const float4 *p = reinterpret_cast<const float4 *>(xrow) + 2 * c;
+        const float4 a = p[0], b = p[1];
+        xp[0] = make_float2(a.x, a.y);
+        xp[1] = make_float2(a.z, a.w);
+        xp[2] = make_float2(b.x, b.y);
+        xp[3] = make_float2(b.z, b.w);
+    } else {
+        const uint4 v = reinterpret_cast<const uint4 *>(xrow)[c];
+        xp[0] = bf16x2_to_f2(v.x);
+        xp[1] = bf16x2_to_f2(v.y);
+        xp[2] = bf16x2_to_f2(v.z);
+        xp[3] = bf16x2_to_f2(v.w);
+    }
+}
+
+__device__ __forceinline__ float pair_sum(float2 a, float2 b) { return (a.x + a.y) + (b.x + b.y); }
+
+// One gate/up task for TE tokens: the dots of the W_gate row and the W_up row
+// (16-byte chunks, lane-strided, four chunks in flight per lane, two packed
+// accumulators per token and row), a butterfly reduction, then lane j writes
+// h = silu(g) * u of token j.
+template <int TE, bool XS_F32>
+__device__ __forceinline__ void gate_up_task(const uint4 *__restrict__ wg,
+                                             const uint4 *__restrict__ wu, int nck,
+                                             const uint8_t *xs, size_t xrow_bytes,
+                                             const int (&tok)[kStreamMaxT], uint64_t *empty_bar,
+                                             float *__restrict__ hout, size_t hstride) {
+    const int lane = (int)lane_id();
+    float2 ag[TE][2], au[TE][2];
+#pragma unroll
+    for (int t = 0; t < TE; ++t)
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+            ag[t][b] = make_float2(0.f, 0.f);
+            au[t][b] = make_float2(0.f, 0.f);
+        }
+    const uint8_t *xr[TE];
+#pragma unroll
+    for (int t = 0; t < TE; ++t)
+        xr[t] = xs + (size_t)tok[t] * xrow_bytes;
+    const int full_end = nck - nck % (32 * kChunkUnroll);
+    int base = 0;
+    for (; base < full_end; base += 32 * kChunkUnroll) {
+        uint4 vg[kChunkUnroll], vu[kChunkUnroll];
+#pragma unroll
+        for (int q = 0; q < kChunkUnroll; ++q) {
+            vg[q] = wg[base + lane + 32 * q];
+            vu[q] = wu[base + lane + 32 * q];
+        }
+#pragma unroll
+        for (int q = 0; q < kChunkUnroll; ++q) {
+            const int c = base + lane + 32 * q;
+            float2 gp[4], up[4];
+            w_pairs(vg[q], gp);
+            w_pairs(vu[q], up);
+#pragma unroll
+            for (int t = 0; t < TE; ++t) {
+                float2 xp[4];
+                x_pairs<XS_F32>(xr[t], c, xp);
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    ag[t][q & 1] = ffma2(gp[p], xp[p], ag[t][q & 1]);
+                    au[t][q & 1] = ffma2(up[p], xp[p], au[t][q & 1]);
+                }
+            }
+        }
+    }
+    for (int c = base + lane; c < nck; c += 32) {
+        float2 gp[4], up[4];
+        w_pairs(wg[c], gp);
+        w_pairs(wu[c], up);
+#pragma unroll
+        for (int t = 0; t < TE; ++t) {
+            float2 xp[4];
+            x_pairs<XS_F32>(xr[t], c, xp);
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                ag[t][0] = ffma2(gp[p], xp[p], ag[t][0]);
+                au[t][0] = ffma2(up[p], xp[p], au[t][0]);
+            }
+        }
+    }
+    __syncwarp();
+    if (lane == 0)
+        mbar_arrive(empty_bar);  // the slot's contents are in registers now
+    float g[TE], u[TE];
+#pragma unroll
+    for (int t = 0; t < TE; ++t) {
+        g[t] = pair_sum(ag[t][0], ag[t][1]);
+        u[t] = pair_sum(au[t][0], au[t][1]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            g[t] += __shfl_xor_sync(0xffffffffu, g[t], off);
+            u[t] += __shfl_xor_sync(0xffffffffu, u[t], off);
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < TE; ++t)
+        if (lane == t)
+            hout[(size_t)t * hstride] = silu_f32(g[t]) * u[t];
+}
+
+// One down-projection row for TE tokens: the dot of a bf16 W_down row with
+// the group's fp32 activations held in shared memory.
+template <int TE>
+__device__ __forceinline__ void down_row(const uint4 *__restrict__ wrow, int nck,
+                                         const float *hg, int width, float (&acc)[TE]) {
+    const int lane = (int)lane_id();
+    float2 a[TE][2];
+#pragma unroll
+    for (int t = 0; t < TE; ++t) {
+        a[t][0] = make_float2(0.f, 0.f);
+        a[t][1] = make_float2(0.f, 0.f);
+    }
+    const int full_end = nck - nck % (32 * kChunkUnroll);
+    int base = 0;
+    for (; base < full_end; base += 32 * kChunkUnroll) {
+        uint4 v[kChunkUnroll];
+#pragma unroll
+        for (int q = 0; q < kChunkUnroll; ++q)
+            v[q] = wrow[base + lane + 32 * q];
+#pragma unroll
+        for (int q = 0; q < kChunkUnroll; ++q) {
+            const int c = base + lane + 32 * q;
+            float2 wp[4];
+            w_pairs(v[q], wp);
+#pragma unroll
+            for (int t = 0; t < TE; ++t) {
+                const float4 *hp = reinterpret_cast<const float4 *>(hg + (size_t)t * width) + 2 * c;
+                const float4 h0 = hp[0], h1 = hp[1];
+                a[t][q & 1] = ffma2(wp[0], make_float2(h0.x, h0.y), a[t][q & 1]);
+                a[t][q & 1] = ffma2(wp[1], make_float2(h0.z, h0.w), a[t][q & 1]);
+                a[t][q & 1] = ffma2(wp[2], make_float2(h1.x, h1.y), a[t][q & 1]);
+                a[t][q & 1] = ffma2(wp[3], make_float2(h1.z, h1.w), a[t][q & 1]);
+            }
+        }
+    }
+    for (int c = base + lane; c < nck; c += 32) {
+        float2 wp[4];
+        w_pairs(wrow[c], wp);
+#pragma unroll
+        for (int t = 0; t < TE; ++t) {
+            const float4 *hp = reinterpret_cast<const float4 *>(hg + (size_t)t * width) + 2 * c;
+            const float4 h0 = hp[0], h1 = hp[1];
+            a[t][0] = ffma2(wp[0], make_float2(h0.x, h0.y), a[t][0]);
+            a[t][0] = ffma2(wp[1], make_float2(h0.z, h0.w), a[t][0]);
+            a[t][0] = ffma2(wp[2], make_float2(h1.x, h1.y), a[t][0]);
+            a[t][0] = ffma2(wp[3], make_float2(h1.z, h1.w), a[t][0]);
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < TE; ++t) {
+        acc[t] = pair_sum(a[t][0], a[t][1]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+            acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
+    }
+}
+
 // ------------------------------------------------------------------ gate / up
-constexpr int kGUConsumerWarps = 4;
+constexpr int kGUConsumerWarps = 8;
 constexpr int kGUThreads = 32 * (1 + kGUConsumerWarps);
-constexpr int kGUMaxSlots = 8;
+constexpr int kGUMaxSlots = 16;
+constexpr uint32_t kGUBarPlan = 1;  // named barrier of the 256 consumer threads
 
 struct StreamGateUpArgs {
     const void *x;
@@ -158,72 +320,86 @@ struct GateUpSmem {
     size_t plan, x, slots, bars, total;
 };
 
-__host__ __device__ inline GateUpSmem gate_up_smem_layout(int T, int H, int x_bytes, int n_slots) {
+// xs_bytes: bytes per activation in shared memory (4: fp32, 2: bf16)
+__host__ __device__ inline GateUpSmem gate_up_smem_layout(int T, int H, int xs_bytes, int n_slots) {
     GateUpSmem s;
     size_t o = 0;
     s.plan = o;  o = align_up_sz(o + sizeof(StreamPlan), 128);
-    s.x = o;     o = align_up_sz(o + (size_t)T * H * x_bytes, 128);
+    s.x = o;     o = align_up_sz(o + (size_t)T * H * xs_bytes, 128);
     s.slots = o; o = align_up_sz(o + (size_t)n_slots * 4 * H, 128);
-    s.bars = o;  o = align_up_sz(o + (size_t)2 * kGUMaxSlots * 8 + 16, 128);
+    s.bars = o;  o = align_up_sz(o + (size_t)(2 * kGUMaxSlots + 2) * 8 + 16, 128);
     s.total = o;
     return s;
 }
 
-template <bool XF32>
+// XIN_F32: x is fp32 in global memory; XS_F32: x is held as fp32 in shared
+// memory (converted from bf16 when XIN_F32 is false).
+template <bool XIN_F32, bool XS_F32>
 __global__ void __launch_bounds__(kGUThreads, 1) stream_gate_up_kernel(const StreamGateUpArgs a) {
+    static_assert(XS_F32 || !XIN_F32, "fp32 activations stay fp32");
     extern __shared__ __align__(1024) uint8_t smem[];
-    constexpr int XB = XF32 ? 4 : 2;
-    const GateUpSmem L = gate_up_smem_layout(a.T, a.H, XB, a.n_slots);
+    constexpr int XSB = XS_F32 ? 4 : 2;
+    const GateUpSmem L = gate_up_smem_layout(a.T, a.H, XSB, a.n_slots);
     StreamPlan &P = *reinterpret_cast<StreamPlan *>(smem + L.plan);
     uint8_t *xs = smem + L.x;
     uint8_t *slots = smem + L.slots;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bars);
     uint64_t *empty = full + kGUMaxSlots;
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + kGUMaxSlots);
+    uint64_t *xbar = empty + kGUMaxSlots;
+    uint64_t *planbar = xbar + 1;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(planbar + 1);
     const int H = a.H, I = a.I, I_s = a.I_s, NS = a.n_slots;
     const uint32_t slot_bytes = 4u * (uint32_t)H;
+    const int warp = (int)(threadIdx.x >> 5);
+    constexpr bool kBulkX = XIN_F32 == XS_F32;  // x lands in shared memory as stored
 
-    build_stream_plan(P, a.ids, a.weights, a.T, a.top_k, a.E);
-    {
-        const uint4 *src = reinterpret_cast<const uint4 *>(a.x);
-        uint4 *dst = reinterpret_cast<uint4 *>(xs);
-        const int n16 = a.T * H * XB / 16;
-        for (int i = threadIdx.x; i < n16; i += blockDim.x)
-            dst[i] = src[i];
-    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
+        mbar_init(xbar, 1);
+        mbar_init(planbar, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
     __syncthreads();
+    grid_dependents_launch();
 
-    // tasks: the shared expert's rows first, then (group, row) in plan order
-    const int64_t total = (int64_t)I_s + (int64_t)P.n_groups * I;
-    const int64_t lo = total * blockIdx.x / gridDim.x;
-    const int64_t hi = total * (blockIdx.x + 1) / gridDim.x;
-    const int ntask = (int)(hi - lo);
-    const int warp = (int)(threadIdx.x >> 5);
-    const int lane = (int)lane_id();
+    // shared-expert rows [s_lo, s_hi) first, then routed (group, unit) tasks
+    const int64_t G = gridDim.x, c = blockIdx.x;
+    const int64_t s_lo = (int64_t)I_s * c / G, s_hi = (int64_t)I_s * (c + 1) / G;
+    const int n_shared = (int)(s_hi - s_lo);
 
     if (warp == 0) {
         if (elect_one()) {
             const uint64_t pol = policy_evict_first();
             int issued = 0;
-            for (int n = 0; n < ntask; ++n) {
+            int ntask = n_shared;        // grows once the plan is known
+            bool have_plan = false;
+            int64_t r_lo = 0;
+            for (int n = 0; n < ntask || !have_plan; ++n) {
+                if (n >= n_shared && !have_plan) {
+                    // routed tasks need the plan the consumers build
+                    if (!mbar_wait(planbar, 0, abort_flag))
+                        break;
+                    have_plan = true;
+                    const int64_t R = (int64_t)P.n_groups * I;
+                    r_lo = R * c / G;
+                    ntask = n_shared + (int)(R * (c + 1) / G - r_lo);
+                    if (n >= ntask)
+                        break;
+                }
                 const int s = n % NS;
                 if (n >= NS && !mbar_wait(&empty[s], (uint32_t)((n / NS) - 1) & 1u, abort_flag))
                     break;
-                const int64_t tau = lo + n;
                 const uint16_t *g, *u;
-                if (tau < I_s) {
-                    g = a.ws_gate + (size_t)tau * H;
-                    u = a.ws_up + (size_t)tau * H;
+                if (n < n_shared) {
+                    const int64_t row = s_lo + n;
+                    g = a.ws_gate + (size_t)row * H;
+                    u = a.ws_up + (size_t)row * H;
                 } else {
-                    const int64_t q = tau - I_s;
+                    const int64_t q = r_lo + (n - n_shared);
                     const int grp = (int)(q / I), i = (int)(q - (int64_t)grp * I);
                     const size_t row = (size_t)P.group_expert[grp] * I + i;
                     g = a.w_gate + row * H;
@@ -238,79 +414,82 @@ __global__ void __launch_bounds__(kGUThreads, 1) stream_gate_up_kernel(const Str
             // no copy may still be writing this CTA's shared memory at exit
             for (int n = issued > NS ? issued - NS : 0; n < issued; ++n)
                 mbar_wait(&full[n % NS], (uint32_t)(n / NS) & 1u, nullptr);
+            if (kBulkX)
+                mbar_wait(xbar, 0, nullptr);
         }
         return;
     }
 
-    const int c_warp = warp - 1;
+    // ---------------------------------------------------------------- consumers
+    const int ltid = (int)threadIdx.x - 32;
+    const int w = warp - 1;
+    grid_dependency_wait();  // ids, weights and x may come from the previous kernel
+    if (kBulkX) {
+        if (ltid == 0) {
+            const uint32_t xbytes = (uint32_t)(a.T * H * XSB);
+            mbar_arrive_expect_tx(xbar, xbytes);
+            bulk_g2s(xs, a.x, xbytes, xbar, policy_evict_last());
+        }
+    } else {
+        // bf16 x widened to fp32 on the way in (exact)
+        const uint4 *src = reinterpret_cast<const uint4 *>(a.x);
+        float4 *dst = reinterpret_cast<float4 *>(xs);
+        const int n16 = a.T * H / 8;
+        for (int i = ltid; i < n16; i += 32 * kGUConsumerWarps) {
+            const uint4 v = src[i];
+            dst[2 * i] = make_float4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y));
+            dst[2 * i + 1] = make_float4(bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w));
+        }
+    }
+    // (the plan's closing barrier also publishes the widened x)
+    build_stream_plan(P, a.ids, a.weights, a.T, a.top_k, a.E, ltid, 32 * kGUConsumerWarps,
+                      kGUBarPlan);
+    if (ltid == 0)
+        mbar_arrive(planbar);
+    const int64_t R = (int64_t)P.n_groups * I;
+    const int64_t r_lo = R * c / G;
+    const int ntask = n_shared + (int)(R * (c + 1) / G - r_lo);
+    if (kBulkX && !mbar_wait(xbar, 0, abort_flag))
+        return;
+
     const int nck = H >> 3;
-    for (int n = c_warp; n < ntask; n += kGUConsumerWarps) {
+    const size_t xrow_bytes = (size_t)H * XSB;
+    for (int n = w; n < ntask; n += kGUConsumerWarps) {
         const int s = n % NS;
         if (!mbar_wait(&full[s], (uint32_t)(n / NS) & 1u, abort_flag))
             break;
-        const int64_t tau = lo + n;
-        int cnt, first = 0, i;
-        bool shared_task;
-        if (tau < I_s) {
-            shared_task = true;
+        int cnt, first = 0;
+        float *hout;
+        size_t hstride;
+        bool shared_task = n < n_shared;
+        if (shared_task) {
             cnt = a.T;
-            i = (int)tau;
+            hout = a.h_shared + (s_lo + n);
+            hstride = (size_t)I_s;
         } else {
-            shared_task = false;
-            const int64_t q = tau - I_s;
+            const int64_t q = r_lo + (n - n_shared);
             const int grp = (int)(q / I);
-            i = (int)(q - (int64_t)grp * I);
+            const int i = (int)(q - (int64_t)grp * I);
             first = P.group_first[grp];
             cnt = P.group_first[grp + 1] - first;
+            hout = a.h_routed + (size_t)first * I + i;
+            hstride = (size_t)I;
         }
         int tok[kStreamMaxT];
 #pragma unroll
         for (int j = 0; j < kStreamMaxT; ++j)
             tok[j] = j < cnt ? (shared_task ? j : (int)P.pair_token[first + j]) : 0;
-        const uint4 *sg = reinterpret_cast<const uint4 *>(slots + (size_t)s * slot_bytes);
-        const uint4 *su = reinterpret_cast<const uint4 *>(slots + (size_t)s * slot_bytes + 2 * H);
-        float ga[kStreamMaxT], ua[kStreamMaxT];
-#pragma unroll
-        for (int j = 0; j < kStreamMaxT; ++j) { ga[j] = 0.f; ua[j] = 0.f; }
-        for (int c = lane; c < nck; c += 32) {
-            float gf[8], uf[8];
-            w8_unpack(sg[c], gf);
-            w8_unpack(su[c], uf);
-#pragma unroll
-            for (int j = 0; j < kStreamMaxT; ++j) {
-                if (j < cnt) {
-                    float xf[8];
-                    x8_from_smem<XF32>(xs + (size_t)tok[j] * H * XB, c, xf);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        ga[j] = fmaf(gf[q], xf[q], ga[j]);
-                        ua[j] = fmaf(uf[q], xf[q], ua[j]);
-                    }
-                }
-            }
-        }
-        __syncwarp();
-        if (lane == 0)
-            mbar_arrive(&empty[s]);  // slot contents are in registers now
-#pragma unroll
-        for (int j = 0; j < kStreamMaxT; ++j) {
-            if (j < cnt) {
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) {
-                    ga[j] += __shfl_xor_sync(0xffffffffu, ga[j], off);
-                    ua[j] += __shfl_xor_sync(0xffffffffu, ua[j], off);
-                }
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < kStreamMaxT; ++j) {
-            if (j < cnt && lane == j) {
-                const float h = silu_f32(ga[j]) * ua[j];
-                if (shared_task)
-                    a.h_shared[(size_t)j * I_s + i] = h;
-                else
-                    a.h_routed[(size_t)(first + j) * I + i] = h;
-            }
+        const uint4 *wg = reinterpret_cast<const uint4 *>(slots + (size_t)s * slot_bytes);
+        const uint4 *wu = reinterpret_cast<const uint4 *>(slots + (size_t)s * slot_bytes + 2 * H);
+        switch (cnt) {
+        case 1: gate_up_task<1, XS_F32>(wg, wu, nck, xs, xrow_bytes, tok, &empty[s], hout, hstride); break;
+        case 2: gate_up_task<2, XS_F32>(wg, wu, nck, xs, xrow_bytes, tok, &empty[s], hout, hstride); break;
+        case 3: gate_up_task<3, XS_F32>(wg, wu, nck, xs, xrow_bytes, tok, &empty[s], hout, hstride); break;
+        case 4: gate_up_task<4, XS_F32>(wg, wu, nck, xs, xrow_bytes, tok, &empty[s], hout, hstride); break;
+        case 5: gate_up_task<5, XS_F32>(wg, wu, nck, xs, xrow_bytes, tok, &empty[s], hout, hstride); break;
+        case 6: gate_up_task<6, XS_F32>(wg, wu, nck, xs, xrow_bytes, tok, &empty[s], hout, hstride); break;
+        case 7: gate_up_task<7, XS_F32>(wg, wu, nck, xs, xrow_bytes, tok, &empty[s], hout, hstride); break;
+        default: gate_up_task<8, XS_F32>(wg, wu, nck, xs, xrow_bytes, tok, &empty[s], hout, hstride); break;
         }
     }
 }
@@ -320,6 +499,7 @@ constexpr int kDownConsumerWarps = 8;
 constexpr int kDownRowsPerSlot = kDownConsumerWarps;
 constexpr int kDownThreads = 32 * (1 + kDownConsumerWarps);
 constexpr int kDownMaxSlots = 8;
+constexpr uint32_t kDownBarPlan = 1;
 
 struct StreamDownArgs {
     int T, H, E, I, I_s, top_k, n_slots, rows_max;
@@ -331,16 +511,19 @@ struct StreamDownArgs {
 };
 
 struct DownSmem {
-    size_t plan, slots, acc, bars, total;
+    size_t plan, hbuf, slots, acc, sacc, bars, total;
 };
 
-__host__ __device__ inline DownSmem down_smem_layout(int I_max, int n_slots, int rows_max) {
+// h buffers hold one group's activations: up to T rows of max(I, I_s) fp32
+__host__ __device__ inline DownSmem down_smem_layout(int T, int I_max, int n_slots, int rows_max) {
     DownSmem s;
     size_t o = 0;
     s.plan = o;  o = align_up_sz(o + sizeof(StreamPlan), 128);
+    s.hbuf = o;  o = align_up_sz(o + (size_t)2 * T * I_max * 4, 128);
     s.slots = o; o = align_up_sz(o + (size_t)n_slots * kDownRowsPerSlot * I_max * 2, 128);
     s.acc = o;   o = align_up_sz(o + (size_t)rows_max * kStreamMaxT * 4, 128);
-    s.bars = o;  o = align_up_sz(o + (size_t)2 * kDownMaxSlots * 8 + 16, 128);
+    s.sacc = o;  o = align_up_sz(o + (size_t)rows_max * kStreamMaxT * 4, 128);
+    s.bars = o;  o = align_up_sz(o + (size_t)(2 * kDownMaxSlots + 4 + 1) * 8 + 16, 128);
     s.total = o;
     return s;
 }
@@ -348,145 +531,207 @@ __host__ __device__ inline DownSmem down_smem_layout(int I_max, int n_slots, int
 __global__ void __launch_bounds__(kDownThreads, 1) stream_down_fold_kernel(const StreamDownArgs a) {
     extern __shared__ __align__(1024) uint8_t smem[];
     const int I_max = a.I > a.I_s ? a.I : a.I_s;
-    const DownSmem L = down_smem_layout(I_max, a.n_slots, a.rows_max);
+    const DownSmem L = down_smem_layout(a.T, I_max, a.n_slots, a.rows_max);
     StreamPlan &P = *reinterpret_cast<StreamPlan *>(smem + L.plan);
+    float *hbuf = reinterpret_cast<float *>(smem + L.hbuf);   // [2][T * I_max]
     uint8_t *slots = smem + L.slots;
-    float *yacc = reinterpret_cast<float *>(smem + L.acc);  // [row][token]
+    float *yacc = reinterpret_cast<float *>(smem + L.acc);    // routed fold [row][token]
+    float *sacc = reinterpret_cast<float *>(smem + L.sacc);   // shared expert [row][token]
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bars);
     uint64_t *empty = full + kDownMaxSlots;
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + kDownMaxSlots);
+    uint64_t *hfull = empty + kDownMaxSlots;                  // [2]
+    uint64_t *hempty = hfull + 2;                             // [2]
+    uint64_t *planbar = hempty + 2;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(planbar + 1);
     const int H = a.H, NS = a.n_slots;
     const size_t slot_bytes = (size_t)kDownRowsPerSlot * I_max * 2;
+    const size_t hbuf_floats = (size_t)a.T * I_max;
+    const int warp = (int)(threadIdx.x >> 5);
+    const int lane = (int)lane_id();
 
-    build_stream_plan(P, a.ids, a.weights, a.T, a.top_k, a.E);
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kDownConsumerWarps);
         }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&hfull[b], 1);
+            mbar_init(&hempty[b], kDownConsumerWarps);
+        }
+        mbar_init(planbar, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
     __syncthreads();
+    grid_dependents_launch();
 
     const int r0 = (int)((int64_t)H * blockIdx.x / gridDim.x);
     const int r1 = (int)((int64_t)H * (blockIdx.x + 1) / gridDim.x);
     const int nrows = r1 - r0;
     const int nsub = (nrows + kDownRowsPerSlot - 1) / kDownRowsPerSlot;
-    const int ngroups = P.n_groups + (a.I_s > 0 ? 1 : 0);
-    const int ntask = ngroups * nsub;
-    const int warp = (int)(threadIdx.x >> 5);
-    const int lane = (int)lane_id();
+    const int has_shared = a.I_s > 0 ? 1 : 0;
 
     if (warp == 0) {
         if (elect_one()) {
             const uint64_t pol = policy_evict_first();
-            int issued = 0;
-            for (int n = 0; n < ntask; ++n) {
-                const int s = n % NS;
-                if (n >= NS && !mbar_wait(&empty[s], (uint32_t)((n / NS) - 1) & 1u, abort_flag))
-                    break;
-                const int gi = n / nsub, q = n - gi * nsub;
-                const bool shared_task = gi >= P.n_groups;
-                const int width = shared_task ? a.I_s : a.I;
-                const uint16_t *mat = shared_task
-                                          ? a.ws_down
-                                          : a.w_down + (size_t)P.group_expert[gi] * H * a.I;
-                const int row = r0 + q * kDownRowsPerSlot;
-                const int nr = min(kDownRowsPerSlot, r1 - row);
-                const uint32_t bytes = (uint32_t)nr * (uint32_t)width * 2u;
-                mbar_arrive_expect_tx(&full[s], bytes);
-                bulk_g2s(slots + (size_t)s * slot_bytes, mat + (size_t)row * width, bytes, &full[s],
-                         pol);
-                ++issued;
+            const uint64_t pol_h = policy_evict_last();
+            int issued = 0, h_issued = 0;
+            bool waited = false;
+            int ngroups = has_shared;  // the routed groups are added once the plan is known
+            bool have_plan = false;
+            bool stop = false;
+            for (int gi = 0; (gi < ngroups || !have_plan) && !stop; ++gi) {
+                if (gi >= has_shared && !have_plan) {
+                    if (!mbar_wait(planbar, 0, abort_flag))
+                        break;
+                    have_plan = true;
+                    ngroups = has_shared + P.n_groups;
+                    if (gi >= ngroups)
+                        break;
+                }
+                const bool shared_group = gi < has_shared;
+                const int width = shared_group ? a.I_s : a.I;
+                const uint16_t *mat;
+                const float *hsrc;
+                uint32_t hbytes;
+                if (shared_group) {
+                    mat = a.ws_down;
+                    hsrc = a.h_shared;
+                    hbytes = (uint32_t)(a.T * a.I_s * 4);
+                } else {
+                    const int g = gi - has_shared;
+                    mat = a.w_down + (size_t)P.group_expert[g] * H * a.I;
+                    const int first = P.group_first[g];
+                    hsrc = a.h_routed + (size_t)first * a.I;
+                    hbytes = (uint32_t)((P.group_first[g + 1] - first) * a.I * 4);
+                }
+                for (int q = 0; q < nsub; ++q) {
+                    const int n = gi * nsub + q;
+                    const int s = n % NS;
+                    if (n >= NS && !mbar_wait(&empty[s], (uint32_t)((n / NS) - 1) & 1u, abort_flag)) {
+                        stop = true;
+                        break;
+                    }
+                    const int row = r0 + q * kDownRowsPerSlot;
+                    const int nr = min(kDownRowsPerSlot, r1 - row);
+                    const uint32_t bytes = (uint32_t)nr * (uint32_t)width * 2u;
+                    mbar_arrive_expect_tx(&full[s], bytes);
+                    bulk_g2s(slots + (size_t)s * slot_bytes, mat + (size_t)row * width, bytes,
+                             &full[s], pol);
+                    ++issued;
+                    if (q == 0) {
+                        // this group's activations (written by the previous kernel)
+                        if (!waited) {
+                            grid_dependency_wait();
+                            waited = true;
+                        }
+                        const int hb = gi & 1;
+                        if (gi >= 2 &&
+                            !mbar_wait(&hempty[hb], (uint32_t)((gi >> 1) - 1) & 1u, abort_flag)) {
+                            stop = true;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&hfull[hb], hbytes);
+                        bulk_g2s(hbuf + hb * hbuf_floats, hsrc, hbytes, &hfull[hb], pol_h);
+                        ++h_issued;
+                    }
+                }
             }
             for (int n = issued > NS ? issued - NS : 0; n < issued; ++n)
                 mbar_wait(&full[n % NS], (uint32_t)(n / NS) & 1u, nullptr);
+            for (int q = h_issued > 2 ? h_issued - 2 : 0; q < h_issued; ++q)
+                mbar_wait(&hfull[q & 1], (uint32_t)(q >> 1) & 1u, nullptr);
         }
     } else {
+        const int ltid = (int)threadIdx.x - 32;
         const int w = warp - 1;
-        for (int n = 0; n < ntask; ++n) {
-            const int s = n % NS;
-            if (!mbar_wait(&full[s], (uint32_t)(n / NS) & 1u, abort_flag))
+        grid_dependency_wait();
+        build_stream_plan(P, a.ids, a.weights, a.T, a.top_k, a.E, ltid, 32 * kDownConsumerWarps,
+                          kDownBarPlan);
+        if (ltid == 0)
+            mbar_arrive(planbar);
+        const int ngroups = has_shared + P.n_groups;
+        bool stop = false;
+        for (int gi = 0; gi < ngroups && !stop; ++gi) {
+            const bool shared_group = gi < has_shared;
+            const int width = shared_group ? a.I_s : a.I;
+            int cnt, first = 0;
+            if (shared_group) {
+                cnt = a.T;
+            } else {
+                const int g = gi - has_shared;
+                first = P.group_first[g];
+                cnt = P.group_first[g + 1] - first;
+            }
+            const int hb = gi & 1;
+            if (!mbar_wait(&hfull[hb], (uint32_t)(gi >> 1) & 1u, abort_flag))
                 break;
-            const int gi = n / nsub, q = n - gi * nsub;
-            const int rl = q * kDownRowsPerSlot + w;  // this warp's row, local to the CTA
-            if (rl < nrows) {
-                const bool shared_task = gi >= P.n_groups;
-                const int width = shared_task ? a.I_s : a.I;
-                int cnt, first = 0;
-                const float *hbase;
-                if (shared_task) {
-                    cnt = a.T;
-                    hbase = a.h_shared;
-                } else {
-                    first = P.group_first[gi];
-                    cnt = P.group_first[gi + 1] - first;
-                    hbase = a.h_routed + (size_t)first * a.I;
+            const float *hg = hbuf + hb * hbuf_floats;
+            const int nck = width >> 3;
+            for (int q = 0; q < nsub; ++q) {
+                const int n = gi * nsub + q;
+                const int s = n % NS;
+                if (!mbar_wait(&full[s], (uint32_t)(n / NS) & 1u, abort_flag)) {
+                    stop = true;
+                    break;
                 }
-                const uint4 *wrow = reinterpret_cast<const uint4 *>(
-                    slots + (size_t)s * slot_bytes + (size_t)w * width * 2);
-                float acc[kStreamMaxT];
-#pragma unroll
-                for (int j = 0; j < kStreamMaxT; ++j)
-                    acc[j] = 0.f;
-                const int nck = width >> 3;
-                for (int c = lane; c < nck; c += 32) {
-                    float wf[8];
-                    w8_unpack(wrow[c], wf);
+                const int rl = q * kDownRowsPerSlot + w;  // this warp's row, local to the CTA
+                if (rl < nrows) {
+                    const uint4 *wrow = reinterpret_cast<const uint4 *>(
+                        slots + (size_t)s * slot_bytes + (size_t)w * width * 2);
+                    float acc[kStreamMaxT];
+                    switch (cnt) {
+                    case 1: { float t1[1]; down_row<1>(wrow, nck, hg, width, t1); acc[0] = t1[0]; break; }
+                    case 2: { float t2[2]; down_row<2>(wrow, nck, hg, width, t2);
+                              for (int j = 0; j < 2; ++j) acc[j] = t2[j]; break; }
+                    case 3: { float t3[3]; down_row<3>(wrow, nck, hg, width, t3);
+                              for (int j = 0; j < 3; ++j) acc[j] = t3[j]; break; }
+                    case 4: { float t4[4]; down_row<4>(wrow, nck, hg, width, t4);
+                              for (int j = 0; j < 4; ++j) acc[j] = t4[j]; break; }
+                    case 5: { float t5[5]; down_row<5>(wrow, nck, hg, width, t5);
+                              for (int j = 0; j < 5; ++j) acc[j] = t5[j]; break; }
+                    case 6: { float t6[6]; down_row<6>(wrow, nck, hg, width, t6);
+                              for (int j = 0; j < 6; ++j) acc[j] = t6[j]; break; }
+                    case 7: { float t7[7]; down_row<7>(wrow, nck, hg, width, t7);
+                              for (int j = 0; j < 7; ++j) acc[j] = t7[j]; break; }
+                    default: { down_row<8>(wrow, nck, hg, width, acc); break; }
+                    }
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(&empty[s]);
 #pragma unroll
                     for (int j = 0; j < kStreamMaxT; ++j) {
-                        if (j < cnt) {
-                            const float4 *hp =
-                                reinterpret_cast<const float4 *>(hbase + (size_t)j * width) + 2 * c;
-                            const float4 h0 = __ldg(hp), h1 = __ldg(hp + 1);
-                            acc[j] = fmaf(wf[0], h0.x, acc[j]);
-                            acc[j] = fmaf(wf[1], h0.y, acc[j]);
-                            acc[j] = fmaf(wf[2], h0.z, acc[j]);
-                            acc[j] = fmaf(wf[3], h0.w, acc[j]);
-                            acc[j] = fmaf(wf[4], h1.x, acc[j]);
-                            acc[j] = fmaf(wf[5], h1.y, acc[j]);
-                            acc[j] = fmaf(wf[6], h1.z, acc[j]);
-                            acc[j] = fmaf(wf[7], h1.w, acc[j]);
+                        if (j < cnt && lane == j) {
+                            if (shared_group) {
+                                sacc[rl * kStreamMaxT + j] = acc[j];
+                            } else {
+                                const int p = first + j;
+                                const int t = P.pair_token[p];
+                                const float cval = P.pair_weight[p] * acc[j];
+                                float &ya = yacc[rl * kStreamMaxT + t];
+                                ya = P.pair_is_first[p] ? cval : ya + cval;
+                            }
                         }
                     }
-                }
-#pragma unroll
-                for (int j = 0; j < kStreamMaxT; ++j) {
-                    if (j < cnt) {
-#pragma unroll
-                        for (int off = 16; off > 0; off >>= 1)
-                            acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], off);
-                    }
-                }
-#pragma unroll
-                for (int j = 0; j < kStreamMaxT; ++j) {
-                    if (j < cnt && lane == j) {
-                        if (shared_task) {
-                            float &ya = yacc[rl * kStreamMaxT + j];
-                            ya = P.token_has_pick[j] ? ya + acc[j] : 0.0f + acc[j];
-                        } else {
-                            const int p = first + j;
-                            const int t = P.pair_token[p];
-                            const float c = P.pair_weight[p] * acc[j];
-                            float &ya = yacc[rl * kStreamMaxT + t];
-                            ya = P.pair_is_first[p] ? c : ya + c;
-                        }
-                    }
+                } else {
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(&empty[s]);
                 }
             }
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(&empty[s]);
+                mbar_arrive(&hempty[hb]);
         }
     }
     __syncthreads();
     if (*abort_flag)
         return;
+    // y = routed fold + shared expert; a token with no routed pick gets 0 + s
     for (int idx = threadIdx.x; idx < a.T * nrows; idx += blockDim.x) {
         const int t = idx / nrows, r = idx - t * nrows;
-        const bool any = P.token_has_pick[t] || a.I_s > 0;
-        a.y[(size_t)t * H + r0 + r] = any ? yacc[r * kStreamMaxT + t] : 0.0f;
+        const float routed = P.token_has_pick[t] ? yacc[r * kStreamMaxT + t] : 0.0f;
+        a.y[(size_t)t * H + r0 + r] = has_shared ? routed + sacc[r * kStreamMaxT + t] : routed;
     }
 }
 
