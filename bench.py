@@ -343,6 +343,8 @@ def run_ours(args, wl):
 
     def step(i, prof=None):
         for T in Ts:
+            if prof is not None:
+                ed.ep_profile_events(prof[("route", T)])
             layer.call(T, i)
             if prof is not None:
                 ed.ep_profile_events(prof[T])
@@ -385,8 +387,8 @@ def run_ours(args, wl):
     # dominant kernel's duration (events between launches stop the early
     # launch of the next kernel, so the throughput above is taken without them)
     nk = 10
-    prof = [{T: [torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)] for T in Ts}
-            for _ in range(K)]
+    prof = [{key: [torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)]
+             for key in list(Ts) + [("route", T) for T in Ts]} for _ in range(K)]
     for p in prof:
         for evs in p.values():
             for e in evs:
@@ -420,6 +422,16 @@ def run_ours(args, wl):
         dom_s += sum(durs)
         per_T[f"T={T}"] = {"dominant_kernel_us": 1e6 * sum(durs) / K,
                            "dominant_kernel_GBps": byts / sum(durs) / 1e9}
+        # mean duration of every kernel of the route and forward calls
+        names = (["plan", "gather", "gate_up", "down", "combine"] if tensor_path[T]
+                 else ["gate_up", "down_fold"])
+        kus = {}
+        for j, name in enumerate(names):
+            kus[name] = 1e3 * sum(prof[i][T][2 * j].elapsed_time(prof[i][T][2 * j + 1])
+                                  for i in range(K)) / K
+        kus["router"] = 1e3 * sum(prof[i][("route", T)][0].elapsed_time(prof[i][("route", T)][1])
+                                  for i in range(K)) / K
+        per_T[f"T={T}"]["kernels_us"] = {k: round(v, 2) for k, v in kus.items()}
 
     if dist is not None:
         t = torch.tensor([dev_s], device=device, dtype=torch.float64)

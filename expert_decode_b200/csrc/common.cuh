@@ -113,12 +113,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     if (mbar_try_wait(bar, parity))
         return true;
     const uint64_t t0 = global_timer_ns();
-    while (true) {
+    for (uint32_t spin = 1;; ++spin) {
         if (mbar_try_wait(bar, parity))
             return true;
         if (abort != nullptr && *abort)
             return false;
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
+        if ((spin & 255u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
             if (abort != nullptr)
                 *abort = 1;
             flag_status(kStatusTimeout);
@@ -277,6 +277,12 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;
     asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
     return r;
+}
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\t"

@@ -74,19 +74,36 @@ bool pdl_enabled() {
 }
 
 template <typename... KArgs, typename... Args>
-cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-                   Args... args) {
+cudaError_t launch_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                           cudaStream_t st, unsigned cluster_x, Args... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    if (pdl_enabled()) {
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    if (cluster_x > 0) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = cluster_x;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    cfg.numAttrs = n;
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                   Args... args) {
+    return launch_cluster(kernel, grid, block, smem, st, 0u, args...);
 }
 
 struct DeviceInfo {
@@ -117,9 +134,15 @@ ep_status device_info(const DeviceInfo **out) {
         EP_CUDA_CHECK(
             cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
         const int m = d.smem_optin;
-        EP_CUDA_CHECK(cudaFuncSetAttribute(epk::router_topk_kernel<false>,
+#define EPK_RT_ATTR(XF, TMV)                                                                 \
+    EP_CUDA_CHECK(cudaFuncSetAttribute(epk::router_tiled_kernel<XF, TMV>,                    \
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, m))
+        EPK_RT_ATTR(false, 1); EPK_RT_ATTR(false, 2); EPK_RT_ATTR(false, 4);
+        EPK_RT_ATTR(true, 1); EPK_RT_ATTR(true, 2); EPK_RT_ATTR(true, 4);
+#undef EPK_RT_ATTR
+        EP_CUDA_CHECK(cudaFuncSetAttribute(epk::router_fp64_kernel<false>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, m));
-        EP_CUDA_CHECK(cudaFuncSetAttribute(epk::router_topk_kernel<true>,
+        EP_CUDA_CHECK(cudaFuncSetAttribute(epk::router_fp64_kernel<true>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, m));
         EP_CUDA_CHECK(cudaFuncSetAttribute(epk::stream_gate_up_kernel<false, false>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, m));
@@ -144,6 +167,8 @@ constexpr int64_t kMaxH = 16384;
 constexpr int64_t kMaxE = 1024;
 constexpr int64_t kMaxI = 16384;
 constexpr int kMaxTopK = 16;
+// moe_route computes the logits directly in fp64 up to this many tokens
+constexpr int64_t kRouterFp64MaxT = 32;
 // Shared memory the streaming kernels may take, leaving the rest of the
 // SM's unified L1 for the activations they read through the cache.
 constexpr size_t kStreamSmemBudget = 200 * 1024;
@@ -177,6 +202,7 @@ Workspace workspace_layout(int64_t T, int64_t H, int64_t E, int64_t k, int64_t I
 // --------------------------------------------------------- streaming path fit
 struct StreamingPlan {
     bool fits = false;
+    int down_rw = 1;  // down-projection rows per consumer warp per slot
     bool xs_f32 = false;  // gate/up keeps x as fp32 in shared memory
     int gu_slots = 0, down_slots = 0, down_grid = 0, down_rows_max = 0;
     size_t gu_smem = 0, down_smem = 0;
@@ -202,14 +228,22 @@ StreamingPlan streaming_fit(const DeviceInfo &d, int64_t T, int64_t H, int xb, i
     const int64_t I_max = std::max(I, I_s);
     p.down_grid = (int)std::max<int64_t>(1, std::min<int64_t>(d.sm_count, H / 8));
     p.down_rows_max = (int)((H + p.down_grid - 1) / p.down_grid);
-    slots = epk::kDownMaxSlots;
-    while (slots >= 2 &&
-           epk::down_smem_layout((int)T, (int)I_max, slots, p.down_rows_max).total > budget)
-        --slots;
-    if (slots < 2)
+    // two rows per warp per slot when three such slots still fit
+    for (int rw = epk::kDownMaxRowsPerWarp; rw >= 1; --rw) {
+        slots = epk::kDownMaxSlots;
+        while (slots >= 2 && epk::down_smem_layout((int)T, (int)I_max, slots, p.down_rows_max,
+                                                   rw).total > budget)
+            --slots;
+        if (slots >= (rw > 1 ? 3 : 2)) {
+            p.down_rw = rw;
+            p.down_slots = slots;
+            p.down_smem =
+                epk::down_smem_layout((int)T, (int)I_max, slots, p.down_rows_max, rw).total;
+            break;
+        }
+    }
+    if (p.down_slots < 2)
         return p;
-    p.down_slots = slots;
-    p.down_smem = epk::down_smem_layout((int)T, (int)I_max, slots, p.down_rows_max).total;
     p.fits = true;
     return p;
 }
@@ -298,26 +332,45 @@ extern "C" ep_status moe_route(const void *x, ep_dtype x_dtype, int64_t T, int64
     ep_status s = device_info(&d);
     if (s != EP_OK)
         return s;
-    const int xb = x_dtype == EP_F32 ? 4 : 2;
-    const int tb_max =
-        (int)std::max<int64_t>(1, std::min<int64_t>(epk::kRouterMaxTB, epk::kRouterXBudget / (H * 4)));
-    const epk::RouterSmem L = epk::router_smem_layout(tb_max, (int)H, (int)E);
-    if ((int)L.total > d->smem_optin)
-        return fail(EP_EINVAL, "moe_route: H = %lld, E = %lld need %u bytes of shared memory",
-                    (long long)H, (long long)E, L.total);
-    const int64_t nblk = (T + tb_max - 1) / tb_max;
-    const dim3 grid((unsigned)(nblk * epk::kRouterCluster));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    {
-        KernelBracket kb0(st, 0);
-        const uint16_t *wr = static_cast<const uint16_t *>(w_router);
+    const uint16_t *wr = static_cast<const uint16_t *>(w_router);
+    KernelBracket kb0(st, 0);
+    if (T <= kRouterFp64MaxT) {
+        // small batches: logits directly in fp64
+        const int tb_max = (int)std::max<int64_t>(
+            1, std::min<int64_t>(epk::kR64MaxTB, epk::kR64XBudget / (H * 8)));
+        const epk::R64Smem L = epk::r64_smem_layout(tb_max, (int)H, (int)E);
+        if ((int)L.total > d->smem_optin)
+            return fail(EP_EINVAL, "moe_route: H = %lld, E = %lld need %u bytes of shared memory",
+                        (long long)H, (long long)E, L.total);
+        const int64_t nblk = (T + tb_max - 1) / tb_max;
+        const dim3 grid((unsigned)(nblk * epk::kRouterCluster));
         if (x_dtype == EP_F32)
-            EP_CUDA_CHECK(launch(epk::router_topk_kernel<true>, grid, epk::kRouterThreads, L.total,
+            EP_CUDA_CHECK(launch(epk::router_fp64_kernel<true>, grid, epk::kR64Threads, L.total,
                                  st, x, T, (int)H, wr, bias, (int)E, top_k, tb_max, ids, weights));
         else
-            EP_CUDA_CHECK(launch(epk::router_topk_kernel<false>, grid, epk::kRouterThreads,
-                                 L.total, st, x, T, (int)H, wr, bias, (int)E, top_k, tb_max, ids,
-                                 weights));
+            EP_CUDA_CHECK(launch(epk::router_fp64_kernel<false>, grid, epk::kR64Threads, L.total,
+                                 st, x, T, (int)H, wr, bias, (int)E, top_k, tb_max, ids, weights));
+    } else {
+        // larger batches: register-tiled fp32 logits, fp64 for the candidates
+        const int BT = epk::rt_block_tokens((int)E);
+        const epk::RtSmem L = epk::rt_smem_layout(BT, (int)E);
+        if ((int)L.total > d->smem_optin)
+            return fail(EP_EINVAL, "moe_route: E = %lld needs %u bytes of shared memory",
+                        (long long)E, L.total);
+        const unsigned C = (unsigned)((E + epk::kRtBE - 1) / epk::kRtBE);
+        const dim3 grid(C, (unsigned)((T + BT - 1) / BT));
+        cudaError_t e;
+#define EPK_RT(XF, TMV)                                                                        \
+    e = launch_cluster(epk::router_tiled_kernel<XF, TMV>, grid, epk::kRtThreads, L.total, st, C, \
+                       x, T, (int)H, wr, bias, (int)E, top_k, ids, weights)
+        if (x_dtype == EP_F32) {
+            if (BT == 32) EPK_RT(true, 4); else if (BT == 16) EPK_RT(true, 2); else EPK_RT(true, 1);
+        } else {
+            if (BT == 32) EPK_RT(false, 4); else if (BT == 16) EPK_RT(false, 2); else EPK_RT(false, 1);
+        }
+#undef EPK_RT
+        EP_CUDA_CHECK(e);
     }
     t_launches = 1;
     return ok();
@@ -442,6 +495,7 @@ extern "C" ep_status moe_ffn_forward(const void *x, ep_dtype x_dtype, int64_t T,
         epk::StreamDownArgs da;
         da.T = (int)T; da.H = (int)H; da.E = (int)E; da.I = (int)I; da.I_s = (int)I_s;
         da.top_k = top_k; da.n_slots = sp.down_slots; da.rows_max = sp.down_rows_max;
+        da.rw = sp.down_rw;
         da.w_down = static_cast<const uint16_t *>(w_down);
         da.ws_down = static_cast<const uint16_t *>(ws_down);
         da.ids = ids;

@@ -317,7 +317,9 @@ struct GemmSmem {
     static constexpr uint32_t misc = bars + 256;
     static constexpr uint32_t units = misc + 64;
     static constexpr uint32_t offsets = units + kMaxGroups * 4 + 4;
-    static constexpr uint32_t total = offsets + (kMaxGroups + 2) * 4;
+    // per epilogue warp: the tile's pick index and routing weight per column
+    static constexpr uint32_t colmeta = (offsets + (kMaxGroups + 2) * 4 + 15) / 16 * 16;
+    static constexpr uint32_t total = colmeta + 4 * kGemmBN * 8;
     static constexpr uint32_t alloc = total + 1024;  // room to align the base to 1024
 };
 
@@ -507,6 +509,8 @@ grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
     } else {
         // ------------------------------------------------------ epilogue
         const int q = warp & 3;  // TMEM lane quarter this warp may access
+        int *col_pick = reinterpret_cast<int *>(smem + GemmSmem::colmeta) + (warp - 2) * 2 * kGemmBN;
+        float *col_w = reinterpret_cast<float *>(col_pick + kGemmBN);
         uint32_t acc = 0, acc_phase = 0;
         for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
             int g, mb, nb, rows, n_blocks;
@@ -514,6 +518,16 @@ grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
             const bool shared = g >= p.E;
             const int n0 = nb * kGemmBN;
             const int n_valid = min(kGemmBN, rows - n0);
+            if (!GATE_UP && !shared) {
+                // this tile's pick index and routing weight per column, loaded by
+                // the warp's lanes in parallel while the accumulator fills
+                for (int col = lane; col < n_valid; col += 32) {
+                    const int pick = p.perm_pair[offsets[g] + n0 + col];
+                    col_pick[col] = pick;
+                    col_w[col] = p.weights[pick];
+                }
+                __syncwarp();
+            }
             if (!mbar_wait(&tfull[acc], acc_phase, abort_flag))
                 break;
             tc_fence_after_sync();
@@ -555,8 +569,8 @@ grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
                                 if (shared) {
                                     p.s_out[(size_t)(n0 + col) * p.H + row] = d;
                                 } else {
-                                    const int pick = p.perm_pair[offsets[g] + n0 + col];
-                                    p.c_out[(size_t)pick * p.H + row] = p.weights[pick] * d;
+                                    const int pick = col_pick[col];
+                                    p.c_out[(size_t)pick * p.H + row] = col_w[col] * d;
                                 }
                             }
                         }

@@ -5,22 +5,15 @@
 // the same top-k.  Softmax over the logits, top_k by logit with ties to the
 // lower expert id, weights renormalised over the picked set.
 //
-// One thread-block cluster of kRouterCluster CTAs handles a block of up to
-// kRouterMaxTB tokens; CTA r owns a contiguous slice of the experts.
-//  1. Each CTA holds the block's activations in shared memory as fp32.
-//  2. Each warp computes, for one expert row of its CTA's slice at a time,
-//     the fp32 logits of all the block's tokens (the row streams from HBM
-//     with one round of 16-byte loads per lane) and a rigorous bound on each
-//     logit's rounding error; both go to CTA 0 through distributed shared
-//     memory.
-//  3. CTA 0 finds, per token, every expert whose exact logit could reach the
-//     k-th largest under those bounds (the candidates).
-//  4. Every CTA recomputes its own candidates' logits in fp64 and sends them
-//     back to CTA 0.
-//  5. CTA 0 picks the top_k on the fp64 logits (ties to the lower id), orders
-//     them by descending logit and renormalises the softmax over them in fp64.
-// The selection and the weights are therefore those of exact arithmetic up to
-// fp64 rounding.
+// Two kernels, both launched as clusters of CTAs that split the experts and
+// meet in CTA 0's shared memory (distributed shared memory):
+//  * router_fp64_kernel (up to 32 tokens): every logit in fp64 directly.
+//  * router_tiled_kernel (more tokens): register-tiled fp32 logits with a
+//    rigorous bound on each logit's rounding error; every expert whose exact
+//    logit could reach the k-th largest under those bounds is recomputed in
+//    fp64 before the pick.
+// Either way the selection, its order and the renormalised weights are those
+// of exact arithmetic up to fp64 rounding.
 #pragma once
 
 #include "common.cuh"
@@ -28,81 +21,14 @@
 namespace epk {
 
 constexpr int kRouterCluster = 8;
-constexpr int kRouterThreads = 256;
-constexpr int kRouterWarps = kRouterThreads / 32;
-constexpr int kRouterMaxTB = 8;        // tokens per cluster
-constexpr int kRouterMaxK = 16;
 constexpr int kRouterMaxCand = 64;     // fp64 candidates per token handled in parallel
-constexpr int kRouterXBudget = 128 * 1024;  // fp32 activations of one token block
 constexpr int kRouterRowChunks = 16;   // 16-byte chunks of a router row per lane per round
 
-struct RouterSmem {
-    // byte offsets into dynamic shared memory
-    uint32_t x, logit, bound, xnorm2, ncand, cand, cval, list_val, list_id, total;
-};
-
 __host__ __device__ inline uint32_t align_up_u32(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
-
-__host__ __device__ inline RouterSmem router_smem_layout(int tb_max, int H, int E) {
-    RouterSmem s;
-    uint32_t o = 0;
-    s.x = o;        o = align_up_u32(o + (uint32_t)tb_max * H * 4, 16);
-    s.logit = o;    o = align_up_u32(o + (uint32_t)kRouterMaxTB * E * 4, 16);
-    s.bound = o;    o = align_up_u32(o + (uint32_t)kRouterMaxTB * E * 4, 16);
-    s.xnorm2 = o;   o = align_up_u32(o + kRouterMaxTB * 4, 16);
-    s.ncand = o;    o = align_up_u32(o + kRouterMaxTB * 4, 16);
-    s.cand = o;     o = align_up_u32(o + kRouterMaxTB * kRouterMaxCand * 4, 16);
-    s.cval = o;     o = align_up_u32(o + kRouterMaxTB * kRouterMaxCand * 8, 16);
-    s.list_val = o; o = align_up_u32(o + kRouterMaxTB * kRouterMaxK * 8, 16);
-    s.list_id = o;  o = align_up_u32(o + kRouterMaxTB * kRouterMaxK * 4, 16);
-    s.total = o;
-    return s;
-}
 
 __device__ __forceinline__ void unpack_w8(uint4 v, float (&wf)[8]) {
     wf[0] = bf16_lo(v.x); wf[1] = bf16_hi(v.x); wf[2] = bf16_lo(v.y); wf[3] = bf16_hi(v.y);
     wf[4] = bf16_lo(v.z); wf[5] = bf16_hi(v.z); wf[6] = bf16_lo(v.w); wf[7] = bf16_hi(v.w);
-}
-
-// fp64 logit of expert e for the token whose fp32 activations are at xrow.
-__device__ double logit_fp64(const float *xrow, const uint16_t *__restrict__ w_router,
-                             const float *__restrict__ bias, int H, int e) {
-    const int lane = (int)lane_id();
-    const int nck = H >> 3;
-    const uint4 *wrow = reinterpret_cast<const uint4 *>(w_router + (size_t)e * H);
-    double acc = 0.0;
-    for (int base = 0; base < nck; base += 32 * kRouterRowChunks) {
-        uint4 wv[kRouterRowChunks];
-#pragma unroll
-        for (int u = 0; u < kRouterRowChunks; ++u) {
-            const int c = base + lane + 32 * u;
-            wv[u] = c < nck ? wrow[c] : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int u = 0; u < kRouterRowChunks; ++u) {
-            const int c = base + lane + 32 * u;
-            if (c < nck) {
-                float wf[8];
-                unpack_w8(wv[u], wf);
-                const float4 *xp = reinterpret_cast<const float4 *>(xrow) + 2 * c;
-                const float4 a = xp[0], b = xp[1];
-                acc = fma((double)a.x, (double)wf[0], acc);
-                acc = fma((double)a.y, (double)wf[1], acc);
-                acc = fma((double)a.z, (double)wf[2], acc);
-                acc = fma((double)a.w, (double)wf[3], acc);
-                acc = fma((double)b.x, (double)wf[4], acc);
-                acc = fma((double)b.y, (double)wf[5], acc);
-                acc = fma((double)b.z, (double)wf[6], acc);
-                acc = fma((double)b.w, (double)wf[7], acc);
-            }
-        }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1)
-        acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (bias != nullptr)
-        acc += (double)bias[e];
-    return acc;
 }
 
 // Index of the k-th largest fp32 logit of one token (ties to the lower id),
@@ -135,26 +61,48 @@ __device__ float kth_logit(const float *lt, int E, int top_k) {
     return vk;
 }
 
+// ------------------------------------------------------------ fp64 router
+// For small batches the logits are computed in fp64 directly (bf16 and fp32
+// values widen to fp64 exactly; products are exact inside the fused
+// multiply-add): no error bounds, no candidate round trip, and two cluster
+// barriers.  Same cluster split of the experts as above; 16 warps per CTA,
+// one expert row per warp at a time; the activations sit in shared memory as
+// fp64.
+constexpr int kR64Threads = 512;
+constexpr int kR64Warps = kR64Threads / 32;
+constexpr int kR64MaxTB = 4;
+constexpr int kR64XBudget = 128 * 1024;
+
+struct R64Smem {
+    uint32_t x, vals, logit, total;
+};
+
+__host__ __device__ inline R64Smem r64_smem_layout(int tb_max, int H, int E) {
+    R64Smem s;
+    uint32_t o = 0;
+    const int per_cta = (E + kRouterCluster - 1) / kRouterCluster;
+    s.x = o;     o = align_up_u32(o + (uint32_t)tb_max * H * 8, 16);
+    s.vals = o;  o = align_up_u32(o + (uint32_t)kR64MaxTB * per_cta * 8, 16);
+    s.logit = o; o = align_up_u32(o + (uint32_t)kR64MaxTB * E * 8, 16);
+    s.total = o;
+    return s;
+}
+
 template <bool XF32>
-__global__ void __cluster_dims__(kRouterCluster, 1, 1) __launch_bounds__(kRouterThreads, 1)
-router_topk_kernel(const void *__restrict__ x, int64_t T, int H,
+__global__ void __cluster_dims__(kRouterCluster, 1, 1) __launch_bounds__(kR64Threads, 1)
+router_fp64_kernel(const void *__restrict__ x, int64_t T, int H,
                    const uint16_t *__restrict__ w_router, const float *__restrict__ bias, int E,
                    int top_k, int tb_max, int32_t *__restrict__ ids, float *__restrict__ weights) {
     extern __shared__ __align__(1024) uint8_t smem[];
     constexpr int XB = XF32 ? 4 : 2;
-    const RouterSmem L = router_smem_layout(tb_max, H, E);
-    float *xs = reinterpret_cast<float *>(smem + L.x);            // [tb][H] fp32
-    float *logit = reinterpret_cast<float *>(smem + L.logit);     // [kRouterMaxTB][E], CTA 0
-    float *bound = reinterpret_cast<float *>(smem + L.bound);     // [kRouterMaxTB][E], CTA 0
-    float *xnorm2 = reinterpret_cast<float *>(smem + L.xnorm2);
-    int *ncand = reinterpret_cast<int *>(smem + L.ncand);         // CTA 0
-    int *cand = reinterpret_cast<int *>(smem + L.cand);           // CTA 0
-    double *cval = reinterpret_cast<double *>(smem + L.cval);     // CTA 0
-    double *list_val = reinterpret_cast<double *>(smem + L.list_val);
-    int *list_id = reinterpret_cast<int *>(smem + L.list_id);
+    const R64Smem L = r64_smem_layout(tb_max, H, E);
+    double *xs = reinterpret_cast<double *>(smem + L.x);        // [tb][H]
+    double *vals = reinterpret_cast<double *>(smem + L.vals);   // [kR64MaxTB][per_cta]
+    double *logit = reinterpret_cast<double *>(smem + L.logit); // [kR64MaxTB][E], CTA 0
 
     grid_dependents_launch();
-    grid_dependency_wait();  // x may come from the previous kernel; ids / weights are read there
+    grid_dependency_wait();
+    cluster_arrive_relaxed();  // "this CTA runs"; waited for before the first remote store
 
     const uint32_t rank = cluster_ctarank();
     const int64_t t0 = (int64_t)(blockIdx.x / kRouterCluster) * tb_max;
@@ -166,121 +114,400 @@ router_topk_kernel(const void *__restrict__ x, int64_t T, int H,
     const int e_lo = (int)rank * per_cta;
     const int e_hi = min(E, e_lo + per_cta);
 
-    // ---- 1. this block's activations as fp32, ||x_t||^2
+    // activations of the block, widened to fp64
     {
-        const uint4 *src = reinterpret_cast<const uint4 *>(
-            reinterpret_cast<const uint8_t *>(x) + (size_t)t0 * H * XB);
-        const int n16 = tb * H * XB / 16;
-        for (int i0 = threadIdx.x; i0 < n16; i0 += 4 * kRouterThreads) {
-            uint4 v[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int i = i0 + u * kRouterThreads;
-                v[u] = i < n16 ? src[i] : make_uint4(0u, 0u, 0u, 0u);
+        const uint8_t *src = reinterpret_cast<const uint8_t *>(x) + (size_t)t0 * H * XB;
+        const int n8 = tb * H / 8;  // groups of 8 activations
+        for (int i = threadIdx.x; i < n8; i += kR64Threads) {
+            float f[8];
+            if constexpr (XF32) {
+                const float4 a = reinterpret_cast<const float4 *>(src)[2 * i];
+                const float4 b = reinterpret_cast<const float4 *>(src)[2 * i + 1];
+                f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+                f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+            } else {
+                unpack_w8(reinterpret_cast<const uint4 *>(src)[i], f);
             }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int i = i0 + u * kRouterThreads;
-                if (i < n16) {
-                    if constexpr (XF32) {
-                        reinterpret_cast<uint4 *>(xs)[i] = v[u];
-                    } else {
-                        float f[8];
-                        unpack_w8(v[u], f);
-                        float4 *d = reinterpret_cast<float4 *>(xs) + 2 * i;
-                        d[0] = make_float4(f[0], f[1], f[2], f[3]);
-                        d[1] = make_float4(f[4], f[5], f[6], f[7]);
-                    }
-                }
-            }
+            double2 *d = reinterpret_cast<double2 *>(xs) + 4 * i;
+            d[0] = make_double2(f[0], f[1]);
+            d[1] = make_double2(f[2], f[3]);
+            d[2] = make_double2(f[4], f[5]);
+            d[3] = make_double2(f[6], f[7]);
         }
     }
     __syncthreads();
-    if (warp < tb) {
-        const float4 *row = reinterpret_cast<const float4 *>(xs + (size_t)warp * H);
-        float s = 0.f;
-        for (int c = lane; c < H / 4; c += 32) {
-            const float4 v = row[c];
-            s = fmaf(v.x, v.x, s);
-            s = fmaf(v.y, v.y, s);
-            s = fmaf(v.z, v.z, s);
-            s = fmaf(v.w, v.w, s);
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
-            s += __shfl_xor_sync(0xffffffffu, s, off);
-        if (lane == 0)
-            xnorm2[warp] = s;
-    }
-    cluster_sync();  // every CTA of the cluster is running; x block and norms visible
 
-    // ---- 2. fp32 logits of this CTA's experts, with error bounds, to CTA 0
-    {
-        const uint32_t r_logit = map_shared_rank(logit, 0);
-        const uint32_t r_bound = map_shared_rank(bound, 0);
-        // Each lane folds at most n_lane products with fused multiply-adds,
-        // then five butterfly additions and the bias add: the classic bound
-        // |fl(s) - s| <= gamma_n * sum |x_h w_h| + u |l|, gamma_n = n u / (1 - n u),
-        // with sum |x_h w_h| <= ||x|| ||w|| (Cauchy-Schwarz).
-        const int n_lane = 8 * ((nck + 31) / 32) + 6;
-        const float u = 5.9604644775390625e-8f;  // 2^-24
-        const float gam = (float)n_lane * u / (1.0f - (float)n_lane * u);
-        for (int e = e_lo + warp; e < e_hi; e += kRouterWarps) {
-            float acc[kRouterMaxTB];
+    for (int e = e_lo + warp; e < e_hi; e += kR64Warps) {
+        double acc[kR64MaxTB];
 #pragma unroll
-            for (int t = 0; t < kRouterMaxTB; ++t)
-                acc[t] = 0.f;
-            float wsq = 0.f;
-            const uint4 *wrow = reinterpret_cast<const uint4 *>(w_router + (size_t)e * H);
-            for (int base = 0; base < nck; base += 32 * kRouterRowChunks) {
-                uint4 wv[kRouterRowChunks];
+        for (int t = 0; t < kR64MaxTB; ++t)
+            acc[t] = 0.0;
+        const uint4 *wrow = reinterpret_cast<const uint4 *>(w_router + (size_t)e * H);
+        for (int base = 0; base < nck; base += 32 * kRouterRowChunks) {
+            uint4 wv[kRouterRowChunks];
 #pragma unroll
-                for (int q = 0; q < kRouterRowChunks; ++q) {
-                    const int c = base + lane + 32 * q;
-                    wv[q] = c < nck ? ld_stream_16(wrow + c) : make_uint4(0u, 0u, 0u, 0u);
-                }
+            for (int q = 0; q < kRouterRowChunks; ++q) {
+                const int c = base + lane + 32 * q;
+                wv[q] = c < nck ? ld_stream_16(wrow + c) : make_uint4(0u, 0u, 0u, 0u);
+            }
 #pragma unroll
-                for (int q = 0; q < kRouterRowChunks; ++q) {
-                    const int c = base + lane + 32 * q;
-                    if (c < nck) {
-                        float wf[8];
-                        unpack_w8(wv[q], wf);
+            for (int q = 0; q < kRouterRowChunks; ++q) {
+                const int c = base + lane + 32 * q;
+                if (c < nck) {
+                    float wf[8];
+                    unpack_w8(wv[q], wf);
 #pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            wsq = fmaf(wf[j], wf[j], wsq);
+                    for (int t = 0; t < kR64MaxTB; ++t) {
+                        if (t < tb) {
+                            const double2 *xp =
+                                reinterpret_cast<const double2 *>(xs + (size_t)t * H) + 4 * c;
 #pragma unroll
-                        for (int t = 0; t < kRouterMaxTB; ++t) {
-                            if (t < tb) {
-                                const float4 *xp =
-                                    reinterpret_cast<const float4 *>(xs + (size_t)t * H) + 2 * c;
-                                const float4 a = xp[0], b = xp[1];
-                                acc[t] = fmaf(a.x, wf[0], acc[t]);
-                                acc[t] = fmaf(a.y, wf[1], acc[t]);
-                                acc[t] = fmaf(a.z, wf[2], acc[t]);
-                                acc[t] = fmaf(a.w, wf[3], acc[t]);
-                                acc[t] = fmaf(b.x, wf[4], acc[t]);
-                                acc[t] = fmaf(b.y, wf[5], acc[t]);
-                                acc[t] = fmaf(b.z, wf[6], acc[t]);
-                                acc[t] = fmaf(b.w, wf[7], acc[t]);
+                            for (int p = 0; p < 4; ++p) {
+                                const double2 xv = xp[p];
+                                acc[t] = fma(xv.x, (double)wf[2 * p], acc[t]);
+                                acc[t] = fma(xv.y, (double)wf[2 * p + 1], acc[t]);
                             }
                         }
                     }
                 }
             }
+        }
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                wsq += __shfl_xor_sync(0xffffffffu, wsq, off);
+        for (int t = 0; t < kR64MaxTB; ++t) {
+            if (t < tb) {
 #pragma unroll
-                for (int t = 0; t < kRouterMaxTB; ++t)
+                for (int off = 16; off > 0; off >>= 1)
                     acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
             }
-            const float b = bias != nullptr ? bias[e] : 0.f;
-            const float wnorm = sqrtf(wsq);
+        }
+        const double b = bias != nullptr ? (double)bias[e] : 0.0;
 #pragma unroll
-            for (int t = 0; t < kRouterMaxTB; ++t) {
-                if (t < tb && lane == t) {
-                    const float l = acc[t] + b;
-                    const float d = 1.5f * (gam * sqrtf(xnorm2[t]) * wnorm + u * fabsf(l)) + 1e-30f;
+        for (int t = 0; t < kR64MaxTB; ++t)
+            if (t < tb && lane == t)
+                vals[t * per_cta + (e - e_lo)] = acc[t] + b;
+    }
+    __syncthreads();
+    cluster_wait();  // every CTA of the cluster runs: CTA 0's shared memory may be written
+    {
+        const uint32_t r_logit = map_shared_rank(logit, 0);
+        const int n = e_hi - e_lo;
+        for (int i = threadIdx.x; i < tb * n; i += kR64Threads) {
+            const int t = i / n, j = i - t * n;
+            st_cluster_f64(r_logit + 8u * (uint32_t)(t * E + e_lo + j), vals[t * per_cta + j]);
+        }
+    }
+    cluster_sync();  // all logits are in CTA 0
+    if (rank != 0 || warp >= tb)
+        return;
+    // CTA 0, warp t: top_k by logit (ties to the lower id), softmax over them
+    const int t = warp;
+    const double *lt = logit + t * E;
+    const int per_lane = (E + 31) / 32;
+    uint32_t chosen = 0;
+    double pick_v = 0.0, top = 0.0;
+    int pick_e = 0;
+    for (int r = 0; r < top_k; ++r) {
+        double bv = -INFINITY;
+        int be = 0x7fffffff;
+        for (int i = 0; i < per_lane; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E && !((chosen >> i) & 1u)) {
+                const double v = lt[e];
+                if (v > bv || (v == bv && e < be)) { bv = v; be = e; }
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const double ov = __shfl_xor_sync(0xffffffffu, bv, off);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+            if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+        }
+        if (be != 0x7fffffff && (be & 31) == lane)
+            chosen |= 1u << (be >> 5);
+        if (r == 0)
+            top = bv;
+        if (lane == r) {
+            pick_v = bv;
+            pick_e = be;
+        }
+    }
+    double ev = lane < top_k ? exp(pick_v - top) : 0.0;
+    double s = 0.0;
+    for (int j = 0; j < top_k; ++j)
+        s += __shfl_sync(0xffffffffu, ev, j);
+    if (lane < top_k) {
+        ids[(t0 + t) * top_k + lane] = pick_e;
+        weights[(t0 + t) * top_k + lane] = (float)(ev / s);
+    }
+}
+
+// ------------------------------------------------------- tiled fp32 router
+// For larger batches the fp32 logits are a register-tiled SIMT product: a
+// cluster of ceil(E / 128) CTAs covers one block of BT tokens, CTA r the
+// experts [128 r, 128 r + 128).  Both operand tiles are widened to fp32 in
+// shared memory, 32 values of H at a time (double-buffered), and each thread
+// keeps TM tokens x 4 experts of accumulators.  Each 32-term block is summed
+// on its own and then added to the running total, which bounds the rounding
+// error by (32 + ceil(H/32) + 2) u sum|x_h w_h| + u |l|.  Candidates and their
+// fp64 refinement then follow the small-batch kernel's steps 3 to 5.
+constexpr int kRtBE = 128;
+constexpr int kRtBK = 32;
+constexpr int kRtPad = 4;
+constexpr int kRtThreads = 256;
+constexpr int kRtMaxBT = 32;
+
+__host__ __device__ inline int rt_block_tokens(int E) {
+    // the logits and bounds of the block live in CTA 0: BT * E * 8 <= 64 KB
+    return E <= 256 ? 32 : (E <= 512 ? 16 : 8);
+}
+
+struct RtSmem {
+    uint32_t xs, ws, xsq, wsq, logit, bound, ncand, cand, cval, total;
+};
+
+__host__ __device__ inline RtSmem rt_smem_layout(int BT, int E) {
+    RtSmem s;
+    uint32_t o = 0;
+    s.xs = o;    o = align_up_u32(o + 2u * BT * (kRtBK + kRtPad) * 4, 16);
+    s.ws = o;    o = align_up_u32(o + 2u * kRtBE * (kRtBK + kRtPad) * 4, 16);
+    s.xsq = o;   o = align_up_u32(o + (uint32_t)BT * 4, 16);
+    s.wsq = o;   o = align_up_u32(o + kRtBE * 4, 16);
+    s.logit = o; o = align_up_u32(o + (uint32_t)BT * E * 4, 16);
+    s.bound = o; o = align_up_u32(o + (uint32_t)BT * E * 4, 16);
+    s.ncand = o; o = align_up_u32(o + (uint32_t)BT * 4, 16);
+    s.cand = o;  o = align_up_u32(o + (uint32_t)BT * kRouterMaxCand * 4, 16);
+    s.cval = o;  o = align_up_u32(o + (uint32_t)BT * kRouterMaxCand * 8, 16);
+    s.total = o;
+    return s;
+}
+
+// fp64 logit of expert e for one token whose activations are in global memory.
+template <bool XF32>
+__device__ double logit_fp64_global(const void *xrow, const uint16_t *__restrict__ w_router,
+                                    const float *__restrict__ bias, int H, int e) {
+    const int lane = (int)lane_id();
+    const int nck = H >> 3;
+    const uint4 *wrow = reinterpret_cast<const uint4 *>(w_router + (size_t)e * H);
+    double acc0 = 0.0, acc1 = 0.0;
+    for (int c = lane; c < nck; c += 32) {
+        float wf[8], xf[8];
+        unpack_w8(wrow[c], wf);
+        if constexpr (XF32) {
+            const float4 a = reinterpret_cast<const float4 *>(xrow)[2 * c];
+            const float4 b = reinterpret_cast<const float4 *>(xrow)[2 * c + 1];
+            xf[0] = a.x; xf[1] = a.y; xf[2] = a.z; xf[3] = a.w;
+            xf[4] = b.x; xf[5] = b.y; xf[6] = b.z; xf[7] = b.w;
+        } else {
+            unpack_w8(reinterpret_cast<const uint4 *>(xrow)[c], xf);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; j += 2) {
+            acc0 = fma((double)xf[j], (double)wf[j], acc0);
+            acc1 = fma((double)xf[j + 1], (double)wf[j + 1], acc1);
+        }
+    }
+    double acc = acc0 + acc1;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (bias != nullptr)
+        acc += (double)bias[e];
+    return acc;
+}
+
+template <bool XF32, int TM>
+__global__ void __launch_bounds__(kRtThreads, 1)
+router_tiled_kernel(const void *__restrict__ x, int64_t T, int H,
+                    const uint16_t *__restrict__ w_router, const float *__restrict__ bias, int E,
+                    int top_k, int32_t *__restrict__ ids, float *__restrict__ weights) {
+    constexpr int BT = 8 * TM;             // tokens per cluster
+    constexpr int XB = XF32 ? 4 : 2;
+    constexpr int LD = kRtBK + kRtPad;     // padded row of a k-tile, in floats
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const RtSmem L = rt_smem_layout(BT, E);
+    float *xs = reinterpret_cast<float *>(smem + L.xs);       // [2][BT][LD]
+    float *ws = reinterpret_cast<float *>(smem + L.ws);       // [2][kRtBE][LD]
+    float *xsq = reinterpret_cast<float *>(smem + L.xsq);
+    float *wsq = reinterpret_cast<float *>(smem + L.wsq);
+    float *logit = reinterpret_cast<float *>(smem + L.logit); // [BT][E], CTA 0
+    float *bound = reinterpret_cast<float *>(smem + L.bound); // [BT][E], CTA 0
+    int *ncand = reinterpret_cast<int *>(smem + L.ncand);
+    int *cand = reinterpret_cast<int *>(smem + L.cand);
+    double *cval = reinterpret_cast<double *>(smem + L.cval);
+
+    grid_dependents_launch();
+    grid_dependency_wait();
+    cluster_arrive_relaxed();
+
+    const uint32_t rank = cluster_ctarank();
+    const int64_t t0 = (int64_t)blockIdx.y * BT;
+    const int tb = (T - t0 < (int64_t)BT) ? (int)(T - t0) : BT;
+    const int e0 = (int)rank * kRtBE;
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int tx = lane, ty = warp;        // experts tx + 32 j, tokens TM ty + i
+
+    // global -> registers for one k-tile: x (BT x 32) and w (128 x 32) as
+    // 16-byte chunks of 8 bf16 (x fp32: 8 floats in two chunks)
+    constexpr int XCH = BT * (kRtBK / 8);          // 8-value chunks of the x tile
+    constexpr int WCH = kRtBE * (kRtBK / 8);       // 512
+    float xr[(XCH + kRtThreads - 1) / kRtThreads][8];
+    float wr[WCH / kRtThreads][8];
+    auto fetch = [&](int k0) {
+#pragma unroll
+        for (int q = 0; q < (XCH + kRtThreads - 1) / kRtThreads; ++q) {
+            const int ch = tid + q * kRtThreads;
+            const int row = ch / (kRtBK / 8), kc = (ch % (kRtBK / 8)) * 8;
+            bool ok = ch < XCH && row < tb && k0 + kc < H;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                xr[q][j] = 0.f;
+            if (ok) {
+                const uint8_t *src = reinterpret_cast<const uint8_t *>(x) +
+                                     ((size_t)(t0 + row) * H + k0 + kc) * XB;
+                if constexpr (XF32) {
+                    const float4 a = reinterpret_cast<const float4 *>(src)[0];
+                    const float4 b = reinterpret_cast<const float4 *>(src)[1];
+                    xr[q][0] = a.x; xr[q][1] = a.y; xr[q][2] = a.z; xr[q][3] = a.w;
+                    xr[q][4] = b.x; xr[q][5] = b.y; xr[q][6] = b.z; xr[q][7] = b.w;
+                } else {
+                    unpack_w8(*reinterpret_cast<const uint4 *>(src), xr[q]);
+                }
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < WCH / kRtThreads; ++q) {
+            const int ch = tid + q * kRtThreads;
+            const int row = ch / (kRtBK / 8), kc = (ch % (kRtBK / 8)) * 8;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                wr[q][j] = 0.f;
+            if (e0 + row < E && k0 + kc < H)
+                unpack_w8(ld_stream_16(w_router + (size_t)(e0 + row) * H + k0 + kc), wr[q]);
+        }
+    };
+    auto stash = [&](int buf) {
+#pragma unroll
+        for (int q = 0; q < (XCH + kRtThreads - 1) / kRtThreads; ++q) {
+            const int ch = tid + q * kRtThreads;
+            if (ch < XCH) {
+                const int row = ch / (kRtBK / 8), kc = (ch % (kRtBK / 8)) * 8;
+                float4 *d = reinterpret_cast<float4 *>(xs + (size_t)(buf * BT + row) * LD + kc);
+                d[0] = make_float4(xr[q][0], xr[q][1], xr[q][2], xr[q][3]);
+                d[1] = make_float4(xr[q][4], xr[q][5], xr[q][6], xr[q][7]);
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < WCH / kRtThreads; ++q) {
+            const int ch = tid + q * kRtThreads;
+            const int row = ch / (kRtBK / 8), kc = (ch % (kRtBK / 8)) * 8;
+            float4 *d = reinterpret_cast<float4 *>(ws + (size_t)(buf * kRtBE + row) * LD + kc);
+            d[0] = make_float4(wr[q][0], wr[q][1], wr[q][2], wr[q][3]);
+            d[1] = make_float4(wr[q][4], wr[q][5], wr[q][6], wr[q][7]);
+        }
+    };
+
+    float acc[TM][4], xs2[TM], ws2[4];
+#pragma unroll
+    for (int i = 0; i < TM; ++i) {
+        xs2[i] = 0.f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            acc[i][j] = 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        ws2[j] = 0.f;
+    const int nkt = (H + kRtBK - 1) / kRtBK;
+    fetch(0);
+    stash(0);
+    __syncthreads();
+    for (int kt = 0; kt < nkt; ++kt) {
+        const int buf = kt & 1;
+        if (kt + 1 < nkt)
+            fetch((kt + 1) * kRtBK);
+        float blk[TM][4];
+#pragma unroll
+        for (int i = 0; i < TM; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                blk[i][j] = 0.f;
+        const float *xb = xs + (size_t)buf * BT * LD;
+        const float *wb = ws + (size_t)buf * kRtBE * LD;
+#pragma unroll
+        for (int k = 0; k < kRtBK; k += 4) {
+            float4 xv[TM], wv[4];
+#pragma unroll
+            for (int i = 0; i < TM; ++i)
+                xv[i] = *reinterpret_cast<const float4 *>(xb + (size_t)(TM * ty + i) * LD + k);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                wv[j] = *reinterpret_cast<const float4 *>(wb + (size_t)(tx + 32 * j) * LD + k);
+#pragma unroll
+            for (int i = 0; i < TM; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    blk[i][j] = fmaf(xv[i].x, wv[j].x, blk[i][j]);
+                    blk[i][j] = fmaf(xv[i].y, wv[j].y, blk[i][j]);
+                    blk[i][j] = fmaf(xv[i].z, wv[j].z, blk[i][j]);
+                    blk[i][j] = fmaf(xv[i].w, wv[j].w, blk[i][j]);
+                }
+            if (ty == 0) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    ws2[j] = fmaf(wv[j].x, wv[j].x, ws2[j]);
+                    ws2[j] = fmaf(wv[j].y, wv[j].y, ws2[j]);
+                    ws2[j] = fmaf(wv[j].z, wv[j].z, ws2[j]);
+                    ws2[j] = fmaf(wv[j].w, wv[j].w, ws2[j]);
+                }
+            }
+            if (tx == 0) {
+#pragma unroll
+                for (int i = 0; i < TM; ++i) {
+                    xs2[i] = fmaf(xv[i].x, xv[i].x, xs2[i]);
+                    xs2[i] = fmaf(xv[i].y, xv[i].y, xs2[i]);
+                    xs2[i] = fmaf(xv[i].z, xv[i].z, xs2[i]);
+                    xs2[i] = fmaf(xv[i].w, xv[i].w, xs2[i]);
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < TM; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                acc[i][j] += blk[i][j];
+        // the other buffer was last read before the previous barrier
+        if (kt + 1 < nkt) {
+            stash(buf ^ 1);
+            __syncthreads();
+        }
+    }
+    if (ty == 0)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            wsq[tx + 32 * j] = ws2[j];
+    if (tx == 0)
+#pragma unroll
+        for (int i = 0; i < TM; ++i)
+            xsq[TM * ty + i] = xs2[i];
+    __syncthreads();
+    cluster_wait();  // every CTA runs: CTA 0's shared memory may be written
+    {
+        const uint32_t r_logit = map_shared_rank(logit, 0);
+        const uint32_t r_bound = map_shared_rank(bound, 0);
+        const float u = 5.9604644775390625e-8f;  // 2^-24
+        const float n = (float)(kRtBK + nkt + 2);
+        const float gam = n * u / (1.0f - n * u);
+#pragma unroll
+        for (int i = 0; i < TM; ++i) {
+            const int t = TM * ty + i;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int e = e0 + tx + 32 * j;
+                if (t < tb && e < E) {
+                    const float l = acc[i][j] + (bias != nullptr ? bias[e] : 0.f);
+                    const float d =
+                        1.5f * (gam * sqrtf(xsq[t]) * sqrtf(wsq[tx + 32 * j]) + u * fabsf(l)) + 1e-30f;
                     st_cluster_f32(r_logit + 4u * (uint32_t)(t * E + e), l);
                     st_cluster_f32(r_bound + 4u * (uint32_t)(t * E + e), d);
                 }
@@ -289,88 +516,76 @@ router_topk_kernel(const void *__restrict__ x, int64_t T, int H,
     }
     cluster_sync();  // all logits and bounds are in CTA 0
 
-    // ---- 3. CTA 0: candidates per token
-    if (rank == 0 && warp < tb) {
-        const int t = warp;
-        const float *lt = logit + t * E;
-        const float *bt = bound + t * E;
-        const float vk = kth_logit(lt, E, top_k);
-        float dmax = 0.f;
-        for (int e = lane; e < E; e += 32)
-            dmax = fmaxf(dmax, bt[e]);
+    // candidates per token (CTA 0): every expert whose exact logit could
+    // reach the k-th largest under the bounds
+    if (rank == 0) {
+        for (int t = warp; t < tb; t += kRtThreads / 32) {
+            const float *lt = logit + t * E;
+            const float *bt = bound + t * E;
+            const float vk = kth_logit(lt, E, top_k);
+            float dmax = 0.f;
+            for (int e = lane; e < E; e += 32)
+                dmax = fmaxf(dmax, bt[e]);
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
-            dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, off));
-        // every expert whose exact logit could reach the k-th one
-        const double thr = (double)vk - 2.0 * (double)dmax * 1.0001;
-        int count = 0;
-        for (int i = 0; i < (E + 31) / 32; ++i) {
-            const int e = lane + 32 * i;
-            const bool c = e < E && (double)lt[e] >= thr;
-            const uint32_t m = __ballot_sync(0xffffffffu, c);
-            const int pos = count + __popc(m & ((1u << lane) - 1u));
-            if (c && pos < kRouterMaxCand)
-                cand[t * kRouterMaxCand + pos] = e;
-            count += __popc(m);
+            for (int off = 16; off > 0; off >>= 1)
+                dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, off));
+            const double thr = (double)vk - 2.0 * (double)dmax * 1.0001;
+            int count = 0;
+            for (int i = 0; i < (E + 31) / 32; ++i) {
+                const int e = lane + 32 * i;
+                const bool c = e < E && (double)lt[e] >= thr;
+                const uint32_t m = __ballot_sync(0xffffffffu, c);
+                const int pos = count + __popc(m & ((1u << lane) - 1u));
+                if (c && pos < kRouterMaxCand)
+                    cand[t * kRouterMaxCand + pos] = e;
+                count += __popc(m);
+            }
+            if (lane == 0)
+                ncand[t] = count;
         }
-        if (lane == 0)
-            ncand[t] = count;
     }
     cluster_sync();  // candidate lists visible to every CTA
 
-    // ---- 4. every CTA: fp64 logits of the candidates in its expert slice
+    // every CTA: fp64 logits of the candidates in its expert slice
     {
-        // CTAs other than 0 copy CTA 0's candidate lists into their own arrays
         const uint32_t r_ncand = map_shared_rank(ncand, 0);
         const uint32_t r_cand = map_shared_rank(cand, 0);
         const uint32_t r_cval = map_shared_rank(cval, 0);
         if (rank != 0) {
-            if (threadIdx.x < (unsigned)tb)
-                ncand[threadIdx.x] = ld_cluster_s32(r_ncand + 4u * threadIdx.x);
-            for (int i = threadIdx.x; i < tb * kRouterMaxCand; i += kRouterThreads)
+            if (tid < tb)
+                ncand[tid] = ld_cluster_s32(r_ncand + 4u * tid);
+            for (int i = tid; i < tb * kRouterMaxCand; i += kRtThreads)
                 cand[i] = ld_cluster_s32(r_cand + 4u * (uint32_t)i);
         }
         __syncthreads();
-        int nc[kRouterMaxTB];
-        int total = 0;
-#pragma unroll
-        for (int t = 0; t < kRouterMaxTB; ++t) {
-            nc[t] = 0;
-            if (t < tb)
-                nc[t] = ncand[t] <= kRouterMaxCand ? ncand[t] : 0;  // larger sets: CTA 0 fallback
-            total += nc[t];
-        }
-        // (token, candidate) pairs, token by token; the warps of the CTA that
-        // owns the expert split them by the expert's place in the slice
-        for (int p = 0; p < total; ++p) {
-            int t = 0, ci = p;
-#pragma unroll
-            for (int q = 0; q < kRouterMaxTB; ++q) {
-                if (t == q && ci >= nc[q]) {
-                    ci -= nc[q];
-                    ++t;
-                }
+        // (token, candidate) pairs whose expert this CTA owns, one per warp
+        int mine = 0;
+        for (int t = 0; t < tb; ++t) {
+            const int nc = ncand[t] <= kRouterMaxCand ? ncand[t] : 0;
+            for (int ci = 0; ci < nc; ++ci) {
+                const int e = cand[t * kRouterMaxCand + ci];
+                if (e < e0 || e >= e0 + kRtBE)
+                    continue;
+                if ((mine++ % (kRtThreads / 32)) != warp)
+                    continue;
+                const uint8_t *xrow = reinterpret_cast<const uint8_t *>(x) + (size_t)(t0 + t) * H * XB;
+                const double v = logit_fp64_global<XF32>(xrow, w_router, bias, H, e);
+                if (lane == 0)
+                    st_cluster_f64(r_cval + 8u * (uint32_t)(t * kRouterMaxCand + ci), v);
             }
-            const int e = cand[t * kRouterMaxCand + ci];
-            if (e < e_lo || e >= e_hi || ((e - e_lo) % kRouterWarps) != warp)
-                continue;
-            const double v = logit_fp64(xs + (size_t)t * H, w_router, bias, H, e);
-            if (lane == 0)
-                st_cluster_f64(r_cval + 8u * (uint32_t)(t * kRouterMaxCand + ci), v);
         }
     }
     cluster_sync();  // fp64 logits are in CTA 0
     if (rank != 0)
         return;
 
-    // ---- 5. CTA 0: pick top_k on the fp64 logits, renormalise, write
-    if (warp < tb) {
-        const int t = warp;
+    // CTA 0: pick top_k on the fp64 logits, renormalise, write
+    for (int t = warp; t < tb; t += kRtThreads / 32) {
         const int nc = ncand[t];
-        double *lv = list_val + t * kRouterMaxK;
-        int *li = list_id + t * kRouterMaxK;
+        double bv_list = 0.0, top = 0.0;
+        int be_list = 0;
         if (nc <= kRouterMaxCand) {
-            uint32_t chosen = 0;  // bit i: candidate lane + 32 i taken (nc <= 64)
+            uint32_t chosen = 0;
             for (int r = 0; r < top_k; ++r) {
                 double bv = -INFINITY;
                 int be = 0x7fffffff, bi = -1;
@@ -391,12 +606,16 @@ router_topk_kernel(const void *__restrict__ x, int64_t T, int H,
                 }
                 if (bi >= 0 && (bi & 31) == lane)
                     chosen |= 1u << (bi >> 5);
-                if (lane == 0) { lv[r] = bv; li[r] = be; }
+                if (r == 0)
+                    top = bv;
+                if (lane == r) {
+                    bv_list = bv;
+                    be_list = be;
+                }
             }
         } else {
-            // Degenerate input (more than kRouterMaxCand experts within the
-            // bound of the k-th logit): stream every candidate, in ascending
-            // id, through a sorted top_k list.
+            // degenerate input: every candidate in ascending id through a
+            // sorted top_k list kept in registers of lanes 0..top_k-1
             const float *lt = logit + t * E;
             float dmax = 0.f;
             for (int e = lane; e < E; e += 32)
@@ -405,36 +624,35 @@ router_topk_kernel(const void *__restrict__ x, int64_t T, int H,
             for (int off = 16; off > 0; off >>= 1)
                 dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, off));
             const double thr = (double)kth_logit(lt, E, top_k) - 2.0 * (double)dmax * 1.0001;
-            int n = 0;
+            const uint8_t *xrow = reinterpret_cast<const uint8_t *>(x) + (size_t)(t0 + t) * H * XB;
+            double lv = -INFINITY;  // lane j holds the j-th best so far
+            int li = 0x7fffffff;
             for (int e = 0; e < E; ++e) {
                 if ((double)lt[e] < thr)
                     continue;
-                const double v = logit_fp64(xs + (size_t)t * H, w_router, bias, H, e);
-                if (lane == 0) {
-                    if (n < top_k || v > lv[top_k - 1]) {
-                        int pos = n < top_k ? n : top_k - 1;
-                        while (pos > 0 && v > lv[pos - 1]) {  // equal values keep the lower id first
-                            lv[pos] = lv[pos - 1];
-                            li[pos] = li[pos - 1];
-                            --pos;
-                        }
-                        lv[pos] = v;
-                        li[pos] = e;
-                        if (n < top_k)
-                            ++n;
-                    }
+                const double v = logit_fp64_global<XF32>(xrow, w_router, bias, H, e);
+                // insert: lanes whose value ranks below v shift down by one
+                const bool below = !(lv > v || (lv == v && li < e));
+                const uint32_t m = __ballot_sync(0xffffffffu, below && lane < top_k);
+                const int pos = m ? __ffs(m) - 1 : top_k;
+                const double pv = __shfl_up_sync(0xffffffffu, lv, 1);
+                const int pi = __shfl_up_sync(0xffffffffu, li, 1);
+                if (lane < top_k && pos < top_k) {
+                    if (lane == pos) { lv = v; li = e; }
+                    else if (lane > pos) { lv = pv; li = pi; }
                 }
-                __syncwarp();
             }
+            top = __shfl_sync(0xffffffffu, lv, 0);
+            bv_list = lv;
+            be_list = li;
         }
-        __syncwarp();
+        const double ev = lane < top_k ? exp(bv_list - top) : 0.0;
+        double ssum = 0.0;
+        for (int j = 0; j < top_k; ++j)
+            ssum += __shfl_sync(0xffffffffu, ev, j);
         if (lane < top_k) {
-            const double m = lv[0];
-            double s = 0.0;
-            for (int j = 0; j < top_k; ++j)
-                s += exp(lv[j] - m);
-            ids[(t0 + t) * top_k + lane] = li[lane];
-            weights[(t0 + t) * top_k + lane] = (float)(exp(lv[lane] - m) / s);
+            ids[(t0 + t) * top_k + lane] = be_list;
+            weights[(t0 + t) * top_k + lane] = (float)(ev / ssum);
         }
     }
 }

@@ -243,61 +243,79 @@ __device__ __forceinline__ void gate_up_task(const uint4 *__restrict__ wg,
             hout[(size_t)t * hstride] = silu_f32(g[t]) * u[t];
 }
 
-// One down-projection row for TE tokens: the dot of a bf16 W_down row with
-// the group's fp32 activations held in shared memory.
-template <int TE>
-__device__ __forceinline__ void down_row(const uint4 *__restrict__ wrow, int nck,
-                                         const float *hg, int width, float (&acc)[TE]) {
+// RW down-projection rows for TE tokens: the dots of bf16 W_down rows with the
+// group's fp32 activations in shared memory; each activation chunk is loaded
+// once for all RW rows.
+template <int TE, int RW>
+__device__ __forceinline__ void down_rows(const uint4 *__restrict__ w0, size_t row_stride16,
+                                          int nck, const float *hg, int width,
+                                          float (&acc)[RW][TE]) {
     const int lane = (int)lane_id();
-    float2 a[TE][2];
+    float2 a[RW][TE][2];
 #pragma unroll
-    for (int t = 0; t < TE; ++t) {
-        a[t][0] = make_float2(0.f, 0.f);
-        a[t][1] = make_float2(0.f, 0.f);
-    }
+    for (int r = 0; r < RW; ++r)
+#pragma unroll
+        for (int t = 0; t < TE; ++t) {
+            a[r][t][0] = make_float2(0.f, 0.f);
+            a[r][t][1] = make_float2(0.f, 0.f);
+        }
     const int full_end = nck - nck % (32 * kChunkUnroll);
     int base = 0;
     for (; base < full_end; base += 32 * kChunkUnroll) {
-        uint4 v[kChunkUnroll];
+        uint4 v[RW][kChunkUnroll];
 #pragma unroll
-        for (int q = 0; q < kChunkUnroll; ++q)
-            v[q] = wrow[base + lane + 32 * q];
+        for (int r = 0; r < RW; ++r)
+#pragma unroll
+            for (int q = 0; q < kChunkUnroll; ++q)
+                v[r][q] = w0[r * row_stride16 + base + lane + 32 * q];
 #pragma unroll
         for (int q = 0; q < kChunkUnroll; ++q) {
             const int c = base + lane + 32 * q;
-            float2 wp[4];
-            w_pairs(v[q], wp);
+            float2 wp[RW][4];
+#pragma unroll
+            for (int r = 0; r < RW; ++r)
+                w_pairs(v[r][q], wp[r]);
 #pragma unroll
             for (int t = 0; t < TE; ++t) {
                 const float4 *hp = reinterpret_cast<const float4 *>(hg + (size_t)t * width) + 2 * c;
                 const float4 h0 = hp[0], h1 = hp[1];
-                a[t][q & 1] = ffma2(wp[0], make_float2(h0.x, h0.y), a[t][q & 1]);
-                a[t][q & 1] = ffma2(wp[1], make_float2(h0.z, h0.w), a[t][q & 1]);
-                a[t][q & 1] = ffma2(wp[2], make_float2(h1.x, h1.y), a[t][q & 1]);
-                a[t][q & 1] = ffma2(wp[3], make_float2(h1.z, h1.w), a[t][q & 1]);
+                const float2 hx[4] = {make_float2(h0.x, h0.y), make_float2(h0.z, h0.w),
+                                      make_float2(h1.x, h1.y), make_float2(h1.z, h1.w)};
+#pragma unroll
+                for (int r = 0; r < RW; ++r)
+#pragma unroll
+                    for (int p = 0; p < 4; ++p)
+                        a[r][t][q & 1] = ffma2(wp[r][p], hx[p], a[r][t][q & 1]);
             }
         }
     }
     for (int c = base + lane; c < nck; c += 32) {
-        float2 wp[4];
-        w_pairs(wrow[c], wp);
+        float2 wp[RW][4];
+#pragma unroll
+        for (int r = 0; r < RW; ++r)
+            w_pairs(w0[r * row_stride16 + c], wp[r]);
 #pragma unroll
         for (int t = 0; t < TE; ++t) {
             const float4 *hp = reinterpret_cast<const float4 *>(hg + (size_t)t * width) + 2 * c;
             const float4 h0 = hp[0], h1 = hp[1];
-            a[t][0] = ffma2(wp[0], make_float2(h0.x, h0.y), a[t][0]);
-            a[t][0] = ffma2(wp[1], make_float2(h0.z, h0.w), a[t][0]);
-            a[t][0] = ffma2(wp[2], make_float2(h1.x, h1.y), a[t][0]);
-            a[t][0] = ffma2(wp[3], make_float2(h1.z, h1.w), a[t][0]);
+            const float2 hx[4] = {make_float2(h0.x, h0.y), make_float2(h0.z, h0.w),
+                                  make_float2(h1.x, h1.y), make_float2(h1.z, h1.w)};
+#pragma unroll
+            for (int r = 0; r < RW; ++r)
+#pragma unroll
+                for (int p = 0; p < 4; ++p)
+                    a[r][t][0] = ffma2(wp[r][p], hx[p], a[r][t][0]);
         }
     }
 #pragma unroll
-    for (int t = 0; t < TE; ++t) {
-        acc[t] = pair_sum(a[t][0], a[t][1]);
+    for (int r = 0; r < RW; ++r)
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
-            acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
-    }
+        for (int t = 0; t < TE; ++t) {
+            acc[r][t] = pair_sum(a[r][t][0], a[r][t][1]);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1)
+                acc[r][t] += __shfl_xor_sync(0xffffffffu, acc[r][t], off);
+        }
 }
 
 // ------------------------------------------------------------------ gate / up
@@ -496,13 +514,14 @@ __global__ void __launch_bounds__(kGUThreads, 1) stream_gate_up_kernel(const Str
 
 // ------------------------------------------------------------- down + fold
 constexpr int kDownConsumerWarps = 8;
-constexpr int kDownRowsPerSlot = kDownConsumerWarps;
+constexpr int kDownMaxRowsPerWarp = 2;
 constexpr int kDownThreads = 32 * (1 + kDownConsumerWarps);
 constexpr int kDownMaxSlots = 8;
 constexpr uint32_t kDownBarPlan = 1;
 
 struct StreamDownArgs {
     int T, H, E, I, I_s, top_k, n_slots, rows_max;
+    int rw;  // rows per consumer warp per slot (1 or 2)
     const uint16_t *w_down, *ws_down;
     const int32_t *ids;
     const float *weights;
@@ -515,12 +534,13 @@ struct DownSmem {
 };
 
 // h buffers hold one group's activations: up to T rows of max(I, I_s) fp32
-__host__ __device__ inline DownSmem down_smem_layout(int T, int I_max, int n_slots, int rows_max) {
+__host__ __device__ inline DownSmem down_smem_layout(int T, int I_max, int n_slots, int rows_max,
+                                                    int rw) {
     DownSmem s;
     size_t o = 0;
     s.plan = o;  o = align_up_sz(o + sizeof(StreamPlan), 128);
     s.hbuf = o;  o = align_up_sz(o + (size_t)2 * T * I_max * 4, 128);
-    s.slots = o; o = align_up_sz(o + (size_t)n_slots * kDownRowsPerSlot * I_max * 2, 128);
+    s.slots = o; o = align_up_sz(o + (size_t)n_slots * kDownConsumerWarps * rw * I_max * 2, 128);
     s.acc = o;   o = align_up_sz(o + (size_t)rows_max * kStreamMaxT * 4, 128);
     s.sacc = o;  o = align_up_sz(o + (size_t)rows_max * kStreamMaxT * 4, 128);
     s.bars = o;  o = align_up_sz(o + (size_t)(2 * kDownMaxSlots + 4 + 1) * 8 + 16, 128);
@@ -531,7 +551,7 @@ __host__ __device__ inline DownSmem down_smem_layout(int T, int I_max, int n_slo
 __global__ void __launch_bounds__(kDownThreads, 1) stream_down_fold_kernel(const StreamDownArgs a) {
     extern __shared__ __align__(1024) uint8_t smem[];
     const int I_max = a.I > a.I_s ? a.I : a.I_s;
-    const DownSmem L = down_smem_layout(a.T, I_max, a.n_slots, a.rows_max);
+    const DownSmem L = down_smem_layout(a.T, I_max, a.n_slots, a.rows_max, a.rw);
     StreamPlan &P = *reinterpret_cast<StreamPlan *>(smem + L.plan);
     float *hbuf = reinterpret_cast<float *>(smem + L.hbuf);   // [2][T * I_max]
     uint8_t *slots = smem + L.slots;
@@ -544,7 +564,8 @@ __global__ void __launch_bounds__(kDownThreads, 1) stream_down_fold_kernel(const
     uint64_t *planbar = hempty + 2;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(planbar + 1);
     const int H = a.H, NS = a.n_slots;
-    const size_t slot_bytes = (size_t)kDownRowsPerSlot * I_max * 2;
+    const int rows_per_slot = kDownConsumerWarps * a.rw;
+    const size_t slot_bytes = (size_t)rows_per_slot * I_max * 2;
     const size_t hbuf_floats = (size_t)a.T * I_max;
     const int warp = (int)(threadIdx.x >> 5);
     const int lane = (int)lane_id();
@@ -568,7 +589,7 @@ __global__ void __launch_bounds__(kDownThreads, 1) stream_down_fold_kernel(const
     const int r0 = (int)((int64_t)H * blockIdx.x / gridDim.x);
     const int r1 = (int)((int64_t)H * (blockIdx.x + 1) / gridDim.x);
     const int nrows = r1 - r0;
-    const int nsub = (nrows + kDownRowsPerSlot - 1) / kDownRowsPerSlot;
+    const int nsub = (nrows + rows_per_slot - 1) / rows_per_slot;
     const int has_shared = a.I_s > 0 ? 1 : 0;
 
     if (warp == 0) {
@@ -612,14 +633,17 @@ __global__ void __launch_bounds__(kDownThreads, 1) stream_down_fold_kernel(const
                         stop = true;
                         break;
                     }
-                    const int row = r0 + q * kDownRowsPerSlot;
-                    const int nr = min(kDownRowsPerSlot, r1 - row);
+                    const int row = r0 + q * rows_per_slot;
+                    const int nr = min(rows_per_slot, r1 - row);
                     const uint32_t bytes = (uint32_t)nr * (uint32_t)width * 2u;
                     mbar_arrive_expect_tx(&full[s], bytes);
                     bulk_g2s(slots + (size_t)s * slot_bytes, mat + (size_t)row * width, bytes,
                              &full[s], pol);
                     ++issued;
-                    if (q == 0) {
+                    // the first group's weights are prefetched into the empty
+                    // ring before its activations can be waited for
+                    const int q_h = gi == 0 ? min(nsub, NS) - 1 : 0;
+                    if (q == q_h) {
                         // this group's activations (written by the previous kernel)
                         if (!waited) {
                             grid_dependency_wait();
@@ -645,11 +669,14 @@ __global__ void __launch_bounds__(kDownThreads, 1) stream_down_fold_kernel(const
     } else {
         const int ltid = (int)threadIdx.x - 32;
         const int w = warp - 1;
-        grid_dependency_wait();
+        // The only kernel that can still be running is this call's gate/up
+        // kernel, which writes h alone: ids and weights may be read before
+        // griddepcontrol.wait, so the plan is built while it finishes.
         build_stream_plan(P, a.ids, a.weights, a.T, a.top_k, a.E, ltid, 32 * kDownConsumerWarps,
                           kDownBarPlan);
         if (ltid == 0)
             mbar_arrive(planbar);
+        grid_dependency_wait();
         const int ngroups = has_shared + P.n_groups;
         bool stop = false;
         for (int gi = 0; gi < ngroups && !stop; ++gi) {
@@ -675,41 +702,56 @@ __global__ void __launch_bounds__(kDownThreads, 1) stream_down_fold_kernel(const
                     stop = true;
                     break;
                 }
-                const int rl = q * kDownRowsPerSlot + w;  // this warp's row, local to the CTA
-                if (rl < nrows) {
+                // this warp's rows of the slot, local to the CTA: rl0, rl0 + 8
+                const int rl0 = q * rows_per_slot + w;
+                const int nmine = rl0 >= nrows ? 0 : (a.rw == 2 && rl0 + kDownConsumerWarps < nrows ? 2 : 1);
+                if (nmine > 0) {
                     const uint4 *wrow = reinterpret_cast<const uint4 *>(
                         slots + (size_t)s * slot_bytes + (size_t)w * width * 2);
-                    float acc[kStreamMaxT];
+                    const size_t stride16 = (size_t)kDownConsumerWarps * width / 8;
+                    float acc[kDownMaxRowsPerWarp][kStreamMaxT];
+#define EPK_DOWN_CASE(TE)                                                              \
+    case TE: {                                                                         \
+        if (nmine == 2) {                                                              \
+            float r2[2][TE];                                                           \
+            down_rows<TE, 2>(wrow, stride16, nck, hg, width, r2);                      \
+            for (int j = 0; j < TE; ++j) { acc[0][j] = r2[0][j]; acc[1][j] = r2[1][j]; } \
+        } else {                                                                       \
+            float r1[1][TE];                                                           \
+            down_rows<TE, 1>(wrow, stride16, nck, hg, width, r1);                      \
+            for (int j = 0; j < TE; ++j) acc[0][j] = r1[0][j];                         \
+        }                                                                              \
+        break;                                                                         \
+    }
                     switch (cnt) {
-                    case 1: { float t1[1]; down_row<1>(wrow, nck, hg, width, t1); acc[0] = t1[0]; break; }
-                    case 2: { float t2[2]; down_row<2>(wrow, nck, hg, width, t2);
-                              for (int j = 0; j < 2; ++j) acc[j] = t2[j]; break; }
-                    case 3: { float t3[3]; down_row<3>(wrow, nck, hg, width, t3);
-                              for (int j = 0; j < 3; ++j) acc[j] = t3[j]; break; }
-                    case 4: { float t4[4]; down_row<4>(wrow, nck, hg, width, t4);
-                              for (int j = 0; j < 4; ++j) acc[j] = t4[j]; break; }
-                    case 5: { float t5[5]; down_row<5>(wrow, nck, hg, width, t5);
-                              for (int j = 0; j < 5; ++j) acc[j] = t5[j]; break; }
-                    case 6: { float t6[6]; down_row<6>(wrow, nck, hg, width, t6);
-                              for (int j = 0; j < 6; ++j) acc[j] = t6[j]; break; }
-                    case 7: { float t7[7]; down_row<7>(wrow, nck, hg, width, t7);
-                              for (int j = 0; j < 7; ++j) acc[j] = t7[j]; break; }
-                    default: { down_row<8>(wrow, nck, hg, width, acc); break; }
+                        EPK_DOWN_CASE(1)
+                        EPK_DOWN_CASE(2)
+                        EPK_DOWN_CASE(3)
+                        EPK_DOWN_CASE(4)
+                        EPK_DOWN_CASE(5)
+                        EPK_DOWN_CASE(6)
+                        EPK_DOWN_CASE(7)
+                        default:
+                        EPK_DOWN_CASE(8)
                     }
+#undef EPK_DOWN_CASE
                     __syncwarp();
                     if (lane == 0)
                         mbar_arrive(&empty[s]);
+                    for (int r = 0; r < nmine; ++r) {
+                        const int rl = rl0 + r * kDownConsumerWarps;
 #pragma unroll
-                    for (int j = 0; j < kStreamMaxT; ++j) {
-                        if (j < cnt && lane == j) {
-                            if (shared_group) {
-                                sacc[rl * kStreamMaxT + j] = acc[j];
-                            } else {
-                                const int p = first + j;
-                                const int t = P.pair_token[p];
-                                const float cval = P.pair_weight[p] * acc[j];
-                                float &ya = yacc[rl * kStreamMaxT + t];
-                                ya = P.pair_is_first[p] ? cval : ya + cval;
+                        for (int j = 0; j < kStreamMaxT; ++j) {
+                            if (j < cnt && lane == j) {
+                                if (shared_group) {
+                                    sacc[rl * kStreamMaxT + j] = acc[r][j];
+                                } else {
+                                    const int p = first + j;
+                                    const int t = P.pair_token[p];
+                                    const float cval = P.pair_weight[p] * acc[r][j];
+                                    float &ya = yacc[rl * kStreamMaxT + t];
+                                    ya = P.pair_is_first[p] ? cval : ya + cval;
+                                }
                             }
                         }
                     }

@@ -82,3 +82,27 @@ def test_router_empty_is_a_no_op():
     ids = torch.full((0, 4), -7, dtype=torch.int32, device="cuda")
     ed.moe_route(x, w, None, 4, ids=ids)
     assert ed.ep_last_launch_count() == 0
+
+
+# ---------------------------------------------------- tiled path (T > 32 tokens)
+@pytest.mark.parametrize("E,T,k", [(37, 45, 5), (300, 70, 8), (1024, 41, 16), (64, 33, 4)])
+def test_router_tiled_odd_shapes(oracle_lib, E, T, k):
+    """Clusters of 1, 3 and 8 CTAs, ragged token blocks of 32 / 16 / 8."""
+    wl = workloads.Workload("tiled", (T,), 328, E, k, 16, 0, "bf16", "zipf1.1", (1,))
+    _route_and_check(oracle_lib, wl, T, seed=E + T)
+
+
+def test_router_tiled_fp32_activations(oracle_lib):
+    wl = workloads.Workload("tiled32", (40,), 256, 16, 4, 16, 0, "f32", "none", (1,))
+    _route_and_check(oracle_lib, wl, 40, seed=2)
+
+
+def test_router_tiled_all_equal_logits():
+    """Every logit ties: more candidates than the parallel budget (fallback list)."""
+    E, H, k, T = 128, 256, 8, 40
+    x = torch.randn(T, H, device="cuda").to(torch.bfloat16)
+    w = torch.zeros(E, H, device="cuda", dtype=torch.bfloat16)
+    ids, wts = ed.moe_route(x, w, None, k)
+    torch.cuda.synchronize()
+    assert ids.cpu().tolist() == [list(range(k))] * T
+    assert torch.all(wts.cpu() == 1.0 / k)
