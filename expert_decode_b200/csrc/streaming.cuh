@@ -522,6 +522,7 @@ constexpr uint32_t kDownBarPlan = 1;
 struct StreamDownArgs {
     int T, H, E, I, I_s, top_k, n_slots, rows_max;
     int rw;  // rows per consumer warp per slot (1 or 2)
+    int n_h;  // h buffers (1, or 2 so that the next group's h lands during this one)
     const uint16_t *w_down, *ws_down;
     const int32_t *ids;
     const float *weights;
@@ -533,49 +534,233 @@ struct DownSmem {
     size_t plan, hbuf, slots, acc, sacc, bars, total;
 };
 
-// h buffers hold one group's activations: up to T rows of max(I, I_s) fp32
+// An h buffer holds a group's activations: up to T rows of max(I, I_s) fp32.
 __host__ __device__ inline DownSmem down_smem_layout(int T, int I_max, int n_slots, int rows_max,
-                                                    int rw) {
+                                                    int rw, int n_h) {
     DownSmem s;
     size_t o = 0;
     s.plan = o;  o = align_up_sz(o + sizeof(StreamPlan), 128);
-    s.hbuf = o;  o = align_up_sz(o + (size_t)2 * T * I_max * 4, 128);
+    s.hbuf = o;  o = align_up_sz(o + (size_t)n_h * T * I_max * 4, 128);
     s.slots = o; o = align_up_sz(o + (size_t)n_slots * kDownConsumerWarps * rw * I_max * 2, 128);
     s.acc = o;   o = align_up_sz(o + (size_t)rows_max * kStreamMaxT * 4, 128);
     s.sacc = o;  o = align_up_sz(o + (size_t)rows_max * kStreamMaxT * 4, 128);
-    s.bars = o;  o = align_up_sz(o + (size_t)(2 * kDownMaxSlots + 4 + 1) * 8 + 16, 128);
+    s.bars = o;  o = align_up_sz(o + (size_t)(2 * kDownMaxSlots + 5) * 8 + 16, 128);
     s.total = o;
     return s;
+}
+
+// What a consumer warp needs to walk one group's slots.
+struct DownGroup {
+    const StreamPlan *P;
+    uint8_t *slots;
+    size_t slot_bytes;
+    uint64_t *full, *empty, *hempty;
+    volatile int *abort_flag;
+    float *yacc, *sacc;
+    const float *hg;
+    int NS, nsub, rows_per_slot, nrows, w, gi, width, cnt, first, rw;
+    bool shared_group;
+};
+
+// The values of one row for the group's tokens (lane j holds token j's)
+// folded into the per-(row, token) accumulators.
+template <int TE>
+__device__ __forceinline__ void fold_row(const DownGroup &g, int rl, const float (&v)[TE]) {
+    const int lane = (int)lane_id();
+#pragma unroll
+    for (int j = 0; j < TE; ++j) {
+        if (lane == j) {
+            if (g.shared_group) {
+                g.sacc[rl * kStreamMaxT + j] = v[j];
+            } else {
+                const int p = g.first + j;
+                const int t = g.P->pair_token[p];
+                const float cval = g.P->pair_weight[p] * v[j];
+                float &ya = g.yacc[rl * kStreamMaxT + t];
+                ya = g.P->pair_is_first[p] ? cval : ya + cval;
+            }
+        }
+    }
+}
+
+// One row for TE tokens whose activations sit in registers: lane l holds
+// chunks c = l + 32 i (i < NCL) of every token.
+template <int TE, int NCL>
+__device__ __forceinline__ void down_row_reg(const uint4 *__restrict__ wrow,
+                                             const float2 (&hr)[TE][NCL][4], float (&acc)[TE]) {
+    const int lane = (int)lane_id();
+    float2 a[TE][2];
+#pragma unroll
+    for (int t = 0; t < TE; ++t) {
+        a[t][0] = make_float2(0.f, 0.f);
+        a[t][1] = make_float2(0.f, 0.f);
+    }
+#pragma unroll
+    for (int i = 0; i < NCL; ++i) {
+        float2 wp[4];
+        w_pairs(wrow[lane + 32 * i], wp);
+#pragma unroll
+        for (int t = 0; t < TE; ++t)
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+                a[t][i & 1] = ffma2(wp[p], hr[t][i][p], a[t][i & 1]);
+    }
+#pragma unroll
+    for (int t = 0; t < TE; ++t) {
+        acc[t] = pair_sum(a[t][0], a[t][1]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+            acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
+    }
+}
+
+// A group of TE (1, or 2 when NCL <= 6) tokens with width = 256 NCL: each warp
+// copies its slice of h into registers once, then walks the group's slots.
+// The h buffer is freed only after the group's last slot: an arrive does not
+// wait for shared-memory loads still in flight, and the next group's h is
+// written by a bulk copy (the async proxy), so freeing it right after the
+// loads let that copy overwrite values not yet read.  Returns false when a
+// wait gave up.
+template <int TE, int NCL>
+__device__ bool down_group_reg(const DownGroup &g) {
+    const int lane = (int)lane_id();
+    float2 hr[TE][NCL][4];
+#pragma unroll
+    for (int t = 0; t < TE; ++t)
+#pragma unroll
+        for (int i = 0; i < NCL; ++i) {
+            const float4 *hp =
+                reinterpret_cast<const float4 *>(g.hg + (size_t)t * g.width) + 2 * (lane + 32 * i);
+            const float4 h0 = hp[0], h1 = hp[1];
+            hr[t][i][0] = make_float2(h0.x, h0.y);
+            hr[t][i][1] = make_float2(h0.z, h0.w);
+            hr[t][i][2] = make_float2(h1.x, h1.y);
+            hr[t][i][3] = make_float2(h1.z, h1.w);
+        }
+    const size_t stride16 = (size_t)kDownConsumerWarps * g.width / 8;
+    for (int q = 0; q < g.nsub; ++q) {
+        const int n = g.gi * g.nsub + q;
+        const int s = n % g.NS;
+        if (!mbar_wait(&g.full[s], (uint32_t)(n / g.NS) & 1u, g.abort_flag))
+            return false;
+        const int rl0 = q * g.rows_per_slot + g.w;
+        const int nmine =
+            rl0 >= g.nrows ? 0 : (g.rw == 2 && rl0 + kDownConsumerWarps < g.nrows ? 2 : 1);
+        const uint4 *wrow =
+            reinterpret_cast<const uint4 *>(g.slots + (size_t)s * g.slot_bytes + (size_t)g.w * g.width * 2);
+        float acc0[TE], acc1[TE];
+        if (nmine >= 1)
+            down_row_reg<TE, NCL>(wrow, hr, acc0);
+        if (nmine == 2)
+            down_row_reg<TE, NCL>(wrow + stride16, hr, acc1);
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(&g.empty[s]);
+        if (nmine >= 1)
+            fold_row<TE>(g, rl0, acc0);
+        if (nmine == 2)
+            fold_row<TE>(g, rl0 + kDownConsumerWarps, acc1);
+    }
+    __syncwarp();
+    if (lane == 0)
+        mbar_arrive(g.hempty);
+    return true;
+}
+
+// Any other group: h is read from shared memory for every row; the h
+// buffer is freed after the group's last slot.
+template <int TE>
+__device__ bool down_group_smem(const DownGroup &g) {
+    const int lane = (int)lane_id();
+    const int nck = g.width >> 3;
+    const size_t stride16 = (size_t)kDownConsumerWarps * g.width / 8;
+    bool ok = true;
+    for (int q = 0; q < g.nsub; ++q) {
+        const int n = g.gi * g.nsub + q;
+        const int s = n % g.NS;
+        if (!mbar_wait(&g.full[s], (uint32_t)(n / g.NS) & 1u, g.abort_flag)) {
+            ok = false;
+            break;
+        }
+        const int rl0 = q * g.rows_per_slot + g.w;
+        const int nmine =
+            rl0 >= g.nrows ? 0 : (g.rw == 2 && rl0 + kDownConsumerWarps < g.nrows ? 2 : 1);
+        const uint4 *wrow =
+            reinterpret_cast<const uint4 *>(g.slots + (size_t)s * g.slot_bytes + (size_t)g.w * g.width * 2);
+        if (nmine == 2) {
+            float acc[2][TE];
+            down_rows<TE, 2>(wrow, stride16, nck, g.hg, g.width, acc);
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&g.empty[s]);
+            fold_row<TE>(g, rl0, acc[0]);
+            fold_row<TE>(g, rl0 + kDownConsumerWarps, acc[1]);
+        } else if (nmine == 1) {
+            float acc[1][TE];
+            down_rows<TE, 1>(wrow, stride16, nck, g.hg, g.width, acc);
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&g.empty[s]);
+            fold_row<TE>(g, rl0, acc[0]);
+        } else {
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&g.empty[s]);
+        }
+    }
+    __syncwarp();
+    if (lane == 0)
+        mbar_arrive(g.hempty);
+    return ok;
+}
+
+__device__ __forceinline__ bool down_group(const DownGroup &g) {
+    // small groups keep h in registers, the rest read it from shared memory
+    const int ncl = (g.width % 256 == 0) ? g.width / 256 : 0;
+    if (g.cnt == 1 && (ncl == 4 || ncl == 6 || ncl == 8))
+        return ncl == 4 ? down_group_reg<1, 4>(g)
+                        : (ncl == 6 ? down_group_reg<1, 6>(g) : down_group_reg<1, 8>(g));
+    if (g.cnt == 2 && (ncl == 4 || ncl == 6))
+        return ncl == 4 ? down_group_reg<2, 4>(g) : down_group_reg<2, 6>(g);
+    switch (g.cnt) {
+    case 1: return down_group_smem<1>(g);
+    case 2: return down_group_smem<2>(g);
+    case 3: return down_group_smem<3>(g);
+    case 4: return down_group_smem<4>(g);
+    case 5: return down_group_smem<5>(g);
+    case 6: return down_group_smem<6>(g);
+    case 7: return down_group_smem<7>(g);
+    default: return down_group_smem<8>(g);
+    }
 }
 
 __global__ void __launch_bounds__(kDownThreads, 1) stream_down_fold_kernel(const StreamDownArgs a) {
     extern __shared__ __align__(1024) uint8_t smem[];
     const int I_max = a.I > a.I_s ? a.I : a.I_s;
-    const DownSmem L = down_smem_layout(a.T, I_max, a.n_slots, a.rows_max, a.rw);
+    const DownSmem L = down_smem_layout(a.T, I_max, a.n_slots, a.rows_max, a.rw, a.n_h);
     StreamPlan &P = *reinterpret_cast<StreamPlan *>(smem + L.plan);
-    float *hbuf = reinterpret_cast<float *>(smem + L.hbuf);   // [2][T * I_max]
+    float *hbuf = reinterpret_cast<float *>(smem + L.hbuf);   // [n_h][T * I_max]
     uint8_t *slots = smem + L.slots;
     float *yacc = reinterpret_cast<float *>(smem + L.acc);    // routed fold [row][token]
     float *sacc = reinterpret_cast<float *>(smem + L.sacc);   // shared expert [row][token]
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bars);
     uint64_t *empty = full + kDownMaxSlots;
-    uint64_t *hfull = empty + kDownMaxSlots;                  // [2]
-    uint64_t *hempty = hfull + 2;                             // [2]
+    uint64_t *hfull = empty + kDownMaxSlots;   // [2]
+    uint64_t *hempty = hfull + 2;              // [2]
     uint64_t *planbar = hempty + 2;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(planbar + 1);
-    const int H = a.H, NS = a.n_slots;
+    const int H = a.H, NS = a.n_slots, NH = a.n_h;
+    const size_t h_elems = (size_t)a.T * I_max;
     const int rows_per_slot = kDownConsumerWarps * a.rw;
     const size_t slot_bytes = (size_t)rows_per_slot * I_max * 2;
-    const size_t hbuf_floats = (size_t)a.T * I_max;
     const int warp = (int)(threadIdx.x >> 5);
-    const int lane = (int)lane_id();
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kDownConsumerWarps);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < NH; ++b) {
             mbar_init(&hfull[b], 1);
             mbar_init(&hempty[b], kDownConsumerWarps);
         }
@@ -626,6 +811,9 @@ __global__ void __launch_bounds__(kDownThreads, 1) stream_down_fold_kernel(const
                     hsrc = a.h_routed + (size_t)first * a.I;
                     hbytes = (uint32_t)((P.group_first[g + 1] - first) * a.I * 4);
                 }
+                // the first group's weights are prefetched into the empty ring
+                // before its activations can be waited for
+                const int q_h = gi == 0 ? min(nsub, NS) - 1 : 0;
                 for (int q = 0; q < nsub; ++q) {
                     const int n = gi * nsub + q;
                     const int s = n % NS;
@@ -640,35 +828,32 @@ __global__ void __launch_bounds__(kDownThreads, 1) stream_down_fold_kernel(const
                     bulk_g2s(slots + (size_t)s * slot_bytes, mat + (size_t)row * width, bytes,
                              &full[s], pol);
                     ++issued;
-                    // the first group's weights are prefetched into the empty
-                    // ring before its activations can be waited for
-                    const int q_h = gi == 0 ? min(nsub, NS) - 1 : 0;
                     if (q == q_h) {
                         // this group's activations (written by the previous kernel)
                         if (!waited) {
                             grid_dependency_wait();
                             waited = true;
                         }
-                        const int hb = gi & 1;
-                        if (gi >= 2 &&
-                            !mbar_wait(&hempty[hb], (uint32_t)((gi >> 1) - 1) & 1u, abort_flag)) {
+                        // group gi uses buffer gi % NH, free once group gi - NH is done
+                        const int hb = gi % NH;
+                        if (gi >= NH &&
+                            !mbar_wait(&hempty[hb], (uint32_t)(gi / NH - 1) & 1u, abort_flag)) {
                             stop = true;
                             break;
                         }
                         mbar_arrive_expect_tx(&hfull[hb], hbytes);
-                        bulk_g2s(hbuf + hb * hbuf_floats, hsrc, hbytes, &hfull[hb], pol_h);
+                        bulk_g2s(hbuf + (size_t)hb * h_elems, hsrc, hbytes, &hfull[hb], pol_h);
                         ++h_issued;
                     }
                 }
             }
             for (int n = issued > NS ? issued - NS : 0; n < issued; ++n)
                 mbar_wait(&full[n % NS], (uint32_t)(n / NS) & 1u, nullptr);
-            for (int q = h_issued > 2 ? h_issued - 2 : 0; q < h_issued; ++q)
-                mbar_wait(&hfull[q & 1], (uint32_t)(q >> 1) & 1u, nullptr);
+            for (int n = h_issued > NH ? h_issued - NH : 0; n < h_issued; ++n)
+                mbar_wait(&hfull[n % NH], (uint32_t)(n / NH) & 1u, nullptr);
         }
     } else {
         const int ltid = (int)threadIdx.x - 32;
-        const int w = warp - 1;
         // The only kernel that can still be running is this call's gate/up
         // kernel, which writes h alone: ids and weights may be read before
         // griddepcontrol.wait, so the plan is built while it finishes.
@@ -677,93 +862,40 @@ __global__ void __launch_bounds__(kDownThreads, 1) stream_down_fold_kernel(const
         if (ltid == 0)
             mbar_arrive(planbar);
         grid_dependency_wait();
+        DownGroup g;
+        g.P = &P;
+        g.slots = slots;
+        g.slot_bytes = slot_bytes;
+        g.full = full;
+        g.empty = empty;
+        g.abort_flag = abort_flag;
+        g.yacc = yacc;
+        g.sacc = sacc;
+        g.NS = NS;
+        g.nsub = nsub;
+        g.rows_per_slot = rows_per_slot;
+        g.nrows = nrows;
+        g.w = warp - 1;
+        g.rw = a.rw;
         const int ngroups = has_shared + P.n_groups;
-        bool stop = false;
-        for (int gi = 0; gi < ngroups && !stop; ++gi) {
-            const bool shared_group = gi < has_shared;
-            const int width = shared_group ? a.I_s : a.I;
-            int cnt, first = 0;
-            if (shared_group) {
-                cnt = a.T;
+        for (int gi = 0; gi < ngroups; ++gi) {
+            g.gi = gi;
+            g.shared_group = gi < has_shared;
+            g.width = g.shared_group ? a.I_s : a.I;
+            if (g.shared_group) {
+                g.cnt = a.T;
+                g.first = 0;
             } else {
-                const int g = gi - has_shared;
-                first = P.group_first[g];
-                cnt = P.group_first[g + 1] - first;
+                const int grp = gi - has_shared;
+                g.first = P.group_first[grp];
+                g.cnt = P.group_first[grp + 1] - g.first;
             }
-            const int hb = gi & 1;
-            if (!mbar_wait(&hfull[hb], (uint32_t)(gi >> 1) & 1u, abort_flag))
+            g.hg = hbuf + (size_t)(gi % NH) * h_elems;
+            g.hempty = &hempty[gi % NH];
+            if (!mbar_wait(&hfull[gi % NH], (uint32_t)(gi / NH) & 1u, abort_flag))
                 break;
-            const float *hg = hbuf + hb * hbuf_floats;
-            const int nck = width >> 3;
-            for (int q = 0; q < nsub; ++q) {
-                const int n = gi * nsub + q;
-                const int s = n % NS;
-                if (!mbar_wait(&full[s], (uint32_t)(n / NS) & 1u, abort_flag)) {
-                    stop = true;
-                    break;
-                }
-                // this warp's rows of the slot, local to the CTA: rl0, rl0 + 8
-                const int rl0 = q * rows_per_slot + w;
-                const int nmine = rl0 >= nrows ? 0 : (a.rw == 2 && rl0 + kDownConsumerWarps < nrows ? 2 : 1);
-                if (nmine > 0) {
-                    const uint4 *wrow = reinterpret_cast<const uint4 *>(
-                        slots + (size_t)s * slot_bytes + (size_t)w * width * 2);
-                    const size_t stride16 = (size_t)kDownConsumerWarps * width / 8;
-                    float acc[kDownMaxRowsPerWarp][kStreamMaxT];
-#define EPK_DOWN_CASE(TE)                                                              \
-    case TE: {                                                                         \
-        if (nmine == 2) {                                                              \
-            float r2[2][TE];                                                           \
-            down_rows<TE, 2>(wrow, stride16, nck, hg, width, r2);                      \
-            for (int j = 0; j < TE; ++j) { acc[0][j] = r2[0][j]; acc[1][j] = r2[1][j]; } \
-        } else {                                                                       \
-            float r1[1][TE];                                                           \
-            down_rows<TE, 1>(wrow, stride16, nck, hg, width, r1);                      \
-            for (int j = 0; j < TE; ++j) acc[0][j] = r1[0][j];                         \
-        }                                                                              \
-        break;                                                                         \
-    }
-                    switch (cnt) {
-                        EPK_DOWN_CASE(1)
-                        EPK_DOWN_CASE(2)
-                        EPK_DOWN_CASE(3)
-                        EPK_DOWN_CASE(4)
-                        EPK_DOWN_CASE(5)
-                        EPK_DOWN_CASE(6)
-                        EPK_DOWN_CASE(7)
-                        default:
-                        EPK_DOWN_CASE(8)
-                    }
-#undef EPK_DOWN_CASE
-                    __syncwarp();
-                    if (lane == 0)
-                        mbar_arrive(&empty[s]);
-                    for (int r = 0; r < nmine; ++r) {
-                        const int rl = rl0 + r * kDownConsumerWarps;
-#pragma unroll
-                        for (int j = 0; j < kStreamMaxT; ++j) {
-                            if (j < cnt && lane == j) {
-                                if (shared_group) {
-                                    sacc[rl * kStreamMaxT + j] = acc[r][j];
-                                } else {
-                                    const int p = first + j;
-                                    const int t = P.pair_token[p];
-                                    const float cval = P.pair_weight[p] * acc[r][j];
-                                    float &ya = yacc[rl * kStreamMaxT + t];
-                                    ya = P.pair_is_first[p] ? cval : ya + cval;
-                                }
-                            }
-                        }
-                    }
-                } else {
-                    __syncwarp();
-                    if (lane == 0)
-                        mbar_arrive(&empty[s]);
-                }
-            }
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&hempty[hb]);
+            if (!down_group(g))
+                break;
         }
     }
     __syncthreads();
