@@ -56,14 +56,17 @@ def library():
             lib.moe_ffn_workspace_size.restype = SZ
             lib.moe_ffn_forward.argtypes = [P, ctypes.c_int, I64, I64, P, P, I32, P, P, P, I64,
                                             I64, P, P, P, I64, ctypes.POINTER(Plan), P, P, SZ, P]
+            lib.moe_ffn_forward_noalloc.argtypes = [P, ctypes.c_int, I64, I64, P, P, I32, P, P,
+                                                    P, I64, I64, P, P, P, I64,
+                                                    ctypes.POINTER(Plan), P, P]
             lib.ep_set_dispatch.argtypes = [ctypes.c_int]
             lib.ep_check_status.argtypes = [P]
             lib.ep_last_error.restype = ctypes.c_char_p
             lib.ep_last_launch_count.restype = I32
             lib.ep_profile_events.argtypes = [P, I32]
             lib.ep_profile_events.restype = ctypes.c_int
-            for fn in ("ep_plan", "moe_route", "moe_ffn_forward", "ep_set_dispatch",
-                       "ep_check_status"):
+            for fn in ("ep_plan", "moe_route", "moe_ffn_forward", "moe_ffn_forward_noalloc",
+                       "ep_set_dispatch", "ep_check_status"):
                 getattr(lib, fn).restype = ctypes.c_int
             _lib = lib
         return _lib
@@ -161,6 +164,34 @@ def moe_ffn_forward(x, ids, weights, w_gate, w_up, w_down, shared, plan, y=None,
         _ptr(x), _dtype(x), T, H, _ptr(ids), _ptr(weights), top_k, _ptr(w_gate), _ptr(w_up),
         _ptr(w_down), E, I, _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), I_s, ctypes.byref(plan),
         _ptr(y), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return y
+
+
+def moe_ffn_forward_noalloc(x, ids, weights, w_gate, w_up, w_down, shared, plan, y,
+                            stream=None):
+    """moe_ffn_forward into the caller's y [T, H] fp32, with the library's static
+    scratch in place of a workspace: neither this wrapper nor the library
+    allocates anything."""
+    _dense(x, "x", ndim=2)
+    _dense(ids, "ids", torch.int32, 2)
+    _dense(weights, "weights", torch.float32, 2)
+    for name, t in (("w_gate", w_gate), ("w_up", w_up), ("w_down", w_down)):
+        _dense(t, name, torch.bfloat16, 3)
+    _dense(y, "y", torch.float32, 2)
+    T, H = x.shape
+    E, I = w_gate.shape[0], w_gate.shape[1]
+    if shared is not None:
+        ws_gate, ws_up, ws_down = shared
+        for name, t in (("ws_gate", ws_gate), ("ws_up", ws_up), ("ws_down", ws_down)):
+            _dense(t, name, torch.bfloat16, 2)
+        I_s = ws_gate.shape[0]
+    else:
+        ws_gate = ws_up = ws_down = None
+        I_s = 0
+    _check(library().moe_ffn_forward_noalloc(
+        _ptr(x), _dtype(x), T, H, _ptr(ids), _ptr(weights), ids.shape[1], _ptr(w_gate),
+        _ptr(w_up), _ptr(w_down), E, I, _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), I_s,
+        ctypes.byref(plan), _ptr(y), _stream(stream)))
     return y
 
 

@@ -535,3 +535,62 @@ extern "C" ep_status moe_ffn_forward(const void *x, ep_dtype x_dtype, int64_t T,
     t_launches = launches;
     return ok();
 }
+
+// ============================================================ no-alloc variant
+// A fixed scratch area that lives in this library's own device memory (one
+// copy per device, created when the CUDA runtime loads the library's kernels
+// onto it), for callers that must not allocate.
+static __device__ __align__(256) unsigned char ep_static_scratch[EP_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+void *g_static_scratch[kMaxDevices];  // per device, guarded by g_device_mu
+
+// Address of the current device's copy of ep_static_scratch, looked up once
+// per device with that device current.
+ep_status static_scratch(void **out) {
+    int dev = 0;
+    EP_CUDA_CHECK(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices)
+        return fail(EP_ECUDA, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_device_mu);
+    if (g_static_scratch[dev] == nullptr) {
+        void *p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, ep_static_scratch);
+        if (e != cudaSuccess || p == nullptr)
+            return fail(EP_ECUDA, "moe_ffn_forward_noalloc: looking up the static scratch on "
+                                  "device %d failed: %s", dev, cudaGetErrorString(e));
+        g_static_scratch[dev] = p;
+    }
+    *out = g_static_scratch[dev];
+    return EP_OK;
+}
+
+}  // namespace
+
+extern "C" ep_status moe_ffn_forward_noalloc(const void *x, ep_dtype x_dtype, int64_t T,
+                                             int64_t H, const int32_t *ids,
+                                             const float *weights, int32_t top_k,
+                                             const void *w_gate, const void *w_up,
+                                             const void *w_down, int64_t E, int64_t I,
+                                             const void *ws_gate, const void *ws_up,
+                                             const void *ws_down, int64_t I_s,
+                                             const ep_plan_t *plan, float *y, void *stream) {
+    // sizes beyond the scratch are refused before anything else happens
+    const size_t need = moe_ffn_workspace_size(T, H, E, top_k, I, I_s);
+    if (need > (size_t)EP_STATIC_SCRATCH_BYTES)
+        return fail(EP_ENOMEM, "moe_ffn_forward_noalloc: these sizes need %zu bytes of scratch, "
+                               "more than the %zu bytes of its static scratch; call "
+                               "moe_ffn_forward with a workspace instead",
+                    need, (size_t)EP_STATIC_SCRATCH_BYTES);
+    void *scratch = nullptr;
+    const ep_status s = static_scratch(&scratch);
+    if (s != EP_OK)
+        return s;
+    // Nothing in the scratch has to start at zero: every byte that either
+    // path reads is written earlier in the same call, as with a caller's
+    // workspace.
+    return moe_ffn_forward(x, x_dtype, T, H, ids, weights, top_k, w_gate, w_up, w_down, E, I,
+                           ws_gate, ws_up, ws_down, I_s, plan, y, scratch,
+                           (size_t)EP_STATIC_SCRATCH_BYTES, stream);
+}

@@ -149,6 +149,37 @@ ep_status moe_ffn_forward(const void *x, ep_dtype x_dtype, int64_t T, int64_t H,
                           void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * moe_ffn_forward_noalloc -- moe_ffn_forward without a caller's workspace.
+ * The method has no counterpart for this: it is a library convenience.
+ * Some callers cannot hand over a workspace: a host runtime that has given
+ * all device memory to its own pool, or a latency-bound loop in which an
+ * allocation (which may synchronise the device, or fail once memory is
+ * committed) is not allowed.  This entry point allocates nothing and calls
+ * no allocating routine; instead it uses a scratch area of
+ * EP_STATIC_SCRATCH_BYTES that is part of the library's own device memory.
+ * Arguments, results, limits and precision are those of moe_ffn_forward,
+ * less `workspace` and `workspace_bytes`.
+ *   Sizes whose moe_ffn_workspace_size exceeds EP_STATIC_SCRATCH_BYTES
+ *   (4 MiB: every T <= 16 at H = 4096, E = 128, top_k = 8, I = I_s = 1536)
+ *   return EP_ENOMEM before anything is launched.
+ *   The first call on each device looks the scratch's address up (with that
+ *   device current) and may make the CUDA runtime load the library's kernels
+ *   onto the device; make that first call before any stream capture begins.
+ *   Nothing in the scratch needs to start at zero.
+ *   There is one scratch per device: calls that can be in flight at the
+ *   same time on one device (on different streams, or from different host
+ *   threads without ordering) race on it and give wrong results.  Calls
+ *   issued in order on one stream are safe.
+ */
+#define EP_STATIC_SCRATCH_BYTES (4u << 20)
+ep_status moe_ffn_forward_noalloc(const void *x, ep_dtype x_dtype, int64_t T, int64_t H,
+                                  const int32_t *ids, const float *weights, int32_t top_k,
+                                  const void *w_gate, const void *w_up, const void *w_down,
+                                  int64_t E, int64_t I,
+                                  const void *ws_gate, const void *ws_up, const void *ws_down,
+                                  int64_t I_s, const ep_plan_t *plan, float *y, void *stream);
+
+/*
  * Which moe_ffn_forward path runs.  EP_DISPATCH_AUTO (the default) takes the
  * weight-streaming path for T <= 8 when its on-chip buffers fit, else the
  * tensor-core path.  Forcing a path that does not fit the sizes makes
