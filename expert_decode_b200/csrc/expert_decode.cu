@@ -224,6 +224,10 @@ StreamingPlan streaming_fit(const DeviceInfo &d, int64_t T, int64_t H, int xb, i
         --slots;
     if (slots < 2)
         return p;
+    // each gate/up slot has a single consumer warp: 8 warps share 8 or 16
+    // slots, and fewer slots than warps leave the extra warps idle
+    if (slots >= epk::kGUConsumerWarps)
+        slots = slots / epk::kGUConsumerWarps * epk::kGUConsumerWarps;
     p.gu_slots = slots;
     p.gu_smem = epk::gate_up_smem_layout((int)T, (int)H, xsb, slots).total;
     const int64_t I_max = std::max(I, I_s);

@@ -470,9 +470,16 @@ __global__ void __launch_bounds__(kGUThreads, 1) stream_gate_up_kernel(const Str
     if (kBulkX && !mbar_wait(xbar, 0, abort_flag))
         return;
 
+    // Task n uses slot n % NS and goes to consumer warp n % A, where A
+    // divides NS: every slot then has one consumer, which waits for the
+    // slot's phases in order.  (Were a slot shared by two warps, one could
+    // wait for phase k + 1 while phase k is still in flight, and the parity
+    // test would pass at once on the stale phase.)
+    // (the host sizes NS as 2..7, 8 or 16)
+    const int A = NS < kGUConsumerWarps ? NS : kGUConsumerWarps;
     const int nck = H >> 3;
     const size_t xrow_bytes = (size_t)H * XSB;
-    for (int n = w; n < ntask; n += kGUConsumerWarps) {
+    for (int n = w; w < A && n < ntask; n += A) {
         const int s = n % NS;
         if (!mbar_wait(&full[s], (uint32_t)(n / NS) & 1u, abort_flag))
             break;

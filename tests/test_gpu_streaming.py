@@ -74,6 +74,22 @@ def test_odd_sizes_and_max_pairs(oracle_lib):
     check_y(y, oracle_ffn(oracle_lib, x, ids, w, W), rel_tol=1e-4, what="odd sizes, 128 picks")
 
 
+# Wide rows shrink the gate/up weight ring: at H = 8192 one slot (a W_gate and
+# a W_up row) takes 32 KB, so 2 (T = 8, bf16 x) or 4 (T = 2, x widened to
+# fp32) slots fit beside x, and fewer consumer warps than usual take tasks.
+# H = 6144 with fp32 x at T = 4 leaves 4 slots of 24 KB.
+@pytest.mark.parametrize("T,H,x_dtype", [(8, 8192, "bf16"), (2, 8192, "bf16"),
+                                         (4, 6144, "f32")])
+def test_wide_rows_few_gate_up_slots(oracle_lib, T, H, x_dtype):
+    wl = workloads.Workload("wide", (T,), H, 16, 4, 256, 128, x_dtype, "none", (1,))
+    W, x, ids, w = _routed(oracle_lib, wl, T, seed=31 + T)
+    y = gpu_ffn(x, ids, w, W, ed.ep_plan(wl.E, 4))
+    ed.ep_check_status()
+    check_y(y, oracle_ffn(oracle_lib, x, ids, w, W), rel_tol=1e-4,
+            what=f"wide rows T={T} H={H} {x_dtype}")
+    assert torch.equal(gpu_ffn(x, ids, w, W, ed.ep_plan(wl.E, 4)), y), "not run-to-run identical"
+
+
 def test_no_shared_expert(oracle_lib):
     wl = WL["imbalanced"]
     W, x, ids, w = _routed(oracle_lib, wl, 5, H=512, I=64, seed=4)
