@@ -369,11 +369,15 @@ def run_ours(args, wl):
     if sampler:
         sampler.start()
     t_wall = time.perf_counter()
+    # an NVTX range marks the timed launches for a profiler's launch filter
+    # (ncu --nvtx --nvtx-include timed/)
+    torch.cuda.nvtx.range_push("timed")
     for i in range(K):
         flush.zero_()
         ev_s[i].record()
         step(args.warmup + i)
         ev_e[i].record()
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     t_wall = time.perf_counter() - t_wall
     clocks = sampler.stop() if sampler else None

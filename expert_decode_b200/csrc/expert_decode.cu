@@ -140,10 +140,11 @@ ep_status device_info(const DeviceInfo **out) {
         EPK_RT_ATTR(false, 1); EPK_RT_ATTR(false, 2); EPK_RT_ATTR(false, 4);
         EPK_RT_ATTR(true, 1); EPK_RT_ATTR(true, 2); EPK_RT_ATTR(true, 4);
 #undef EPK_RT_ATTR
-        EP_CUDA_CHECK(cudaFuncSetAttribute(epk::router_fp64_kernel<false>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, m));
-        EP_CUDA_CHECK(cudaFuncSetAttribute(epk::router_fp64_kernel<true>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, m));
+#define EPK_RD_ATTR(XF, TBV)                                                                 \
+    EP_CUDA_CHECK(cudaFuncSetAttribute(epk::router_dot2_kernel<XF, TBV>,                     \
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, m))
+        EPK_RD_ATTR(false, 1); EPK_RD_ATTR(false, 2); EPK_RD_ATTR(true, 1); EPK_RD_ATTR(true, 2);
+#undef EPK_RD_ATTR
         EP_CUDA_CHECK(cudaFuncSetAttribute(epk::stream_gate_up_kernel<false, false>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, m));
         EP_CUDA_CHECK(cudaFuncSetAttribute(epk::stream_gate_up_kernel<false, true>,
@@ -167,8 +168,8 @@ constexpr int64_t kMaxH = 16384;
 constexpr int64_t kMaxE = 1024;
 constexpr int64_t kMaxI = 16384;
 constexpr int kMaxTopK = 16;
-// moe_route computes the logits directly in fp64 up to this many tokens
-constexpr int64_t kRouterFp64MaxT = 32;
+// moe_route computes every logit by Dot2 up to this many tokens
+constexpr int64_t kRouterDot2MaxT = 32;
 // Shared memory the streaming kernels may take, leaving the rest of the
 // SM's unified L1 for the activations they read through the cache.
 constexpr size_t kStreamSmemBudget = 200 * 1024;
@@ -343,24 +344,30 @@ extern "C" ep_status moe_route(const void *x, ep_dtype x_dtype, int64_t T, int64
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const uint16_t *wr = static_cast<const uint16_t *>(w_router);
     KernelBracket kb0(st, 0);
-    if (T <= kRouterFp64MaxT) {
-        // small batches: logits directly in fp64
-        const int tb_max = (int)std::max<int64_t>(
-            1, std::min<int64_t>(epk::kR64MaxTB, epk::kR64XBudget / (H * 8)));
-        const epk::R64Smem L = epk::r64_smem_layout(tb_max, (int)H, (int)E);
+    if (T <= kRouterDot2MaxT) {
+        // small batches: every logit by Dot2, one cluster per token while
+        // the clusters fit on the SMs at once, else two tokens per cluster
+        const int64_t max_clusters = std::max(1, d->sm_count / epk::kRouterCluster);
+        const int tb = T <= max_clusters ? 1 : epk::kRdMaxTB;
+        const epk::RdSmem L = epk::rd_smem_layout(tb, (int)H, (int)E);
         if ((int)L.total > d->smem_optin)
             return fail(EP_EINVAL, "moe_route: H = %lld, E = %lld need %u bytes of shared memory",
                         (long long)H, (long long)E, L.total);
-        const int64_t nblk = (T + tb_max - 1) / tb_max;
+        const int64_t nblk = (T + tb - 1) / tb;
         const dim3 grid((unsigned)(nblk * epk::kRouterCluster));
-        if (x_dtype == EP_F32)
-            EP_CUDA_CHECK(launch(epk::router_fp64_kernel<true>, grid, epk::kR64Threads, L.total,
-                                 st, x, T, (int)H, wr, bias, (int)E, top_k, tb_max, ids, weights));
-        else
-            EP_CUDA_CHECK(launch(epk::router_fp64_kernel<false>, grid, epk::kR64Threads, L.total,
-                                 st, x, T, (int)H, wr, bias, (int)E, top_k, tb_max, ids, weights));
+        cudaError_t e;
+#define EPK_RD(XF, TBV)                                                                        \
+    e = launch(epk::router_dot2_kernel<XF, TBV>, grid, epk::kRdThreads, L.total, st, x, T,      \
+               (int)H, wr, bias, (int)E, top_k, ids, weights)
+        if (x_dtype == EP_F32) {
+            if (tb == 1) EPK_RD(true, 1); else EPK_RD(true, 2);
+        } else {
+            if (tb == 1) EPK_RD(false, 1); else EPK_RD(false, 2);
+        }
+#undef EPK_RD
+        EP_CUDA_CHECK(e);
     } else {
-        // larger batches: register-tiled fp32 logits, fp64 for the candidates
+        // larger batches: register-tiled fp32 logits, Dot2 for the candidates
         const int BT = epk::rt_block_tokens((int)E);
         const epk::RtSmem L = epk::rt_smem_layout(BT, (int)E);
         if ((int)L.total > d->smem_optin)

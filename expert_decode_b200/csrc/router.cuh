@@ -7,13 +7,15 @@
 //
 // Two kernels, both launched as clusters of CTAs that split the experts and
 // meet in CTA 0's shared memory (distributed shared memory):
-//  * router_fp64_kernel (up to 32 tokens): every logit in fp64 directly.
+//  * router_dot2_kernel (up to 32 tokens): every logit as a compensated
+//    (Dot2) fp32 dot product, accurate to about 1e-9 (bound below).
 //  * router_tiled_kernel (more tokens): register-tiled fp32 logits with a
 //    rigorous bound on each logit's rounding error; every expert whose exact
-//    logit could reach the k-th largest under those bounds is recomputed in
-//    fp64 before the pick.
-// Either way the selection, its order and the renormalised weights are those
-// of exact arithmetic up to fp64 rounding.
+//    logit could reach the k-th largest under those bounds is recomputed by
+//    Dot2 before the pick.
+// Either way the selection and its order are those of exact arithmetic
+// except between logits closer than the Dot2 bound, and the weights carry
+// the error of that bound plus one fp32 rounding.
 #pragma once
 
 #include "common.cuh"
@@ -21,7 +23,7 @@
 namespace epk {
 
 constexpr int kRouterCluster = 8;
-constexpr int kRouterMaxCand = 64;     // fp64 candidates per token handled in parallel
+constexpr int kRouterMaxCand = 64;     // refined candidates per token handled in parallel
 constexpr int kRouterRowChunks = 16;   // 16-byte chunks of a router row per lane per round
 
 __host__ __device__ inline uint32_t align_up_u32(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
@@ -61,147 +63,77 @@ __device__ float kth_logit(const float *lt, int E, int top_k) {
     return vk;
 }
 
-// ------------------------------------------------------------ fp64 router
-// For small batches the logits are computed in fp64 directly (bf16 and fp32
-// values widen to fp64 exactly; products are exact inside the fused
-// multiply-add): no error bounds, no candidate round trip, and two cluster
-// barriers.  Same cluster split of the experts as above; 16 warps per CTA,
-// one expert row per warp at a time; the activations sit in shared memory as
-// fp64.
-constexpr int kR64Threads = 512;
-constexpr int kR64Warps = kR64Threads / 32;
-constexpr int kR64MaxTB = 4;
-constexpr int kR64XBudget = 128 * 1024;
+// ------------------------------------------------------ compensated logits
+// A logit is a dot product of H terms x_h w_h.  With bf16 activations every
+// product is exact in fp32 (8 + 8 significant bits); with fp32 activations
+// the rounding error of each product is recovered exactly by an FMA.  The
+// terms are summed as an unevaluated pair (s, c): s the running fp32 sum and
+// c the sum of the exact rounding errors of the additions into s (Knuth's
+// TwoSum), the compensated dot product "Dot2" of Ogita, Rump and Oishi
+// ("Accurate sum and dot product", SIAM J. Sci. Comput. 26(6), 2005).  Each
+// lane sums its terms in two packed chains and the 32 lanes are combined by
+// the same error-free step, so the pair differs from the exact dot product
+// by at most about gamma_n^2 sum_h |x_h w_h|, gamma_n = n u / (1 - n u),
+// u = 2^-24, n = H/64 + 6: about 1e-9 at H = 4096 for unit activations and
+// weights of scale 0.02.  fp64 arithmetic is not used for the sums: on this
+// part its throughput is a small fraction of fp32's.
 
-struct R64Smem {
-    uint32_t x, vals, logit, total;
-};
+// s + p as the pair (s, c): s takes the rounded sum, c the exact error.
+__device__ __forceinline__ void dot2_add(float2 &s, float2 &c, float2 p) {
+    const float2 sn = add2(s, p);
+    const float2 bb = sub2(sn, s);
+    c = add2(c, add2(sub2(s, sub2(sn, bb)), sub2(p, bb)));
+    s = sn;
+}
 
-__host__ __device__ inline R64Smem r64_smem_layout(int tb_max, int H, int E) {
-    R64Smem s;
-    uint32_t o = 0;
-    const int per_cta = (E + kRouterCluster - 1) / kRouterCluster;
-    s.x = o;     o = align_up_u32(o + (uint32_t)tb_max * H * 8, 16);
-    s.vals = o;  o = align_up_u32(o + (uint32_t)kR64MaxTB * per_cta * 8, 16);
-    s.logit = o; o = align_up_u32(o + (uint32_t)kR64MaxTB * E * 8, 16);
-    s.total = o;
+// Eight terms of one 16-byte weight chunk: wp the weights as fp32 pairs, wn
+// their negations (used only for fp32 activations), xp the activations.
+template <bool XF32>
+__device__ __forceinline__ void dot2_chunk(const float2 (&wp)[4], const float2 (&wn)[4],
+                                           const float2 (&xp)[4], float2 &s, float2 &c) {
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const float2 prod = mul2(wp[p], xp[p]);
+        if constexpr (XF32)
+            c = sub2(c, ffma2(wn[p], xp[p], prod));  // + (w x - prod), exact
+        dot2_add(s, c, prod);
+    }
+}
+
+__device__ __forceinline__ void dot2_unpack_w(uint4 v, float2 (&wp)[4], float2 (&wn)[4]) {
+    wp[0] = bf16x2_to_f2(v.x); wp[1] = bf16x2_to_f2(v.y);
+    wp[2] = bf16x2_to_f2(v.z); wp[3] = bf16x2_to_f2(v.w);
+    wn[0] = bf16x2_to_f2(v.x ^ 0x80008000u); wn[1] = bf16x2_to_f2(v.y ^ 0x80008000u);
+    wn[2] = bf16x2_to_f2(v.z ^ 0x80008000u); wn[3] = bf16x2_to_f2(v.w ^ 0x80008000u);
+}
+
+__device__ __forceinline__ float two_sum(float a, float b, float &err) {
+    const float s = __fadd_rn(a, b);
+    const float bb = __fsub_rn(s, a);
+    err = __fadd_rn(__fsub_rn(a, __fsub_rn(s, bb)), __fsub_rn(b, bb));
     return s;
 }
 
-template <bool XF32>
-__global__ void __cluster_dims__(kRouterCluster, 1, 1) __launch_bounds__(kR64Threads, 1)
-router_fp64_kernel(const void *__restrict__ x, int64_t T, int H,
-                   const uint16_t *__restrict__ w_router, const float *__restrict__ bias, int E,
-                   int top_k, int tb_max, int32_t *__restrict__ ids, float *__restrict__ weights) {
-    extern __shared__ __align__(1024) uint8_t smem[];
-    constexpr int XB = XF32 ? 4 : 2;
-    const R64Smem L = r64_smem_layout(tb_max, H, E);
-    double *xs = reinterpret_cast<double *>(smem + L.x);        // [tb][H]
-    double *vals = reinterpret_cast<double *>(smem + L.vals);   // [kR64MaxTB][per_cta]
-    double *logit = reinterpret_cast<double *>(smem + L.logit); // [kR64MaxTB][E], CTA 0
+// The warp's pairs summed into one value (identical in every lane).
+__device__ __forceinline__ double dot2_warp_total(float2 s, float2 c) {
+    float r;
+    float S = two_sum(s.x, s.y, r);
+    float C = __fadd_rn(__fadd_rn(c.x, c.y), r);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const float So = __shfl_xor_sync(0xffffffffu, S, off);
+        const float Co = __shfl_xor_sync(0xffffffffu, C, off);
+        S = two_sum(S, So, r);
+        C = __fadd_rn(__fadd_rn(C, Co), r);
+    }
+    return (double)S + (double)C;
+}
 
-    grid_dependents_launch();
-    grid_dependency_wait();
-    cluster_arrive_relaxed();  // "this CTA runs"; waited for before the first remote store
-
-    const uint32_t rank = cluster_ctarank();
-    const int64_t t0 = (int64_t)(blockIdx.x / kRouterCluster) * tb_max;
-    const int tb = (T - t0 < (int64_t)tb_max) ? (int)(T - t0) : tb_max;
-    const int warp = (int)(threadIdx.x >> 5);
+// One warp: top_k of the E logits of one token (ties to the lower id) and
+// their softmax renormalised over the picked set.
+__device__ void topk_softmax_warp(const double *lt, int E, int top_k, int32_t *ids_row,
+                                  float *w_row) {
     const int lane = (int)lane_id();
-    const int nck = H >> 3;
-    const int per_cta = (E + kRouterCluster - 1) / kRouterCluster;
-    const int e_lo = (int)rank * per_cta;
-    const int e_hi = min(E, e_lo + per_cta);
-
-    // activations of the block, widened to fp64
-    {
-        const uint8_t *src = reinterpret_cast<const uint8_t *>(x) + (size_t)t0 * H * XB;
-        const int n8 = tb * H / 8;  // groups of 8 activations
-        for (int i = threadIdx.x; i < n8; i += kR64Threads) {
-            float f[8];
-            if constexpr (XF32) {
-                const float4 a = reinterpret_cast<const float4 *>(src)[2 * i];
-                const float4 b = reinterpret_cast<const float4 *>(src)[2 * i + 1];
-                f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
-                f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
-            } else {
-                unpack_w8(reinterpret_cast<const uint4 *>(src)[i], f);
-            }
-            double2 *d = reinterpret_cast<double2 *>(xs) + 4 * i;
-            d[0] = make_double2(f[0], f[1]);
-            d[1] = make_double2(f[2], f[3]);
-            d[2] = make_double2(f[4], f[5]);
-            d[3] = make_double2(f[6], f[7]);
-        }
-    }
-    __syncthreads();
-
-    for (int e = e_lo + warp; e < e_hi; e += kR64Warps) {
-        double acc[kR64MaxTB];
-#pragma unroll
-        for (int t = 0; t < kR64MaxTB; ++t)
-            acc[t] = 0.0;
-        const uint4 *wrow = reinterpret_cast<const uint4 *>(w_router + (size_t)e * H);
-        for (int base = 0; base < nck; base += 32 * kRouterRowChunks) {
-            uint4 wv[kRouterRowChunks];
-#pragma unroll
-            for (int q = 0; q < kRouterRowChunks; ++q) {
-                const int c = base + lane + 32 * q;
-                wv[q] = c < nck ? ld_stream_16(wrow + c) : make_uint4(0u, 0u, 0u, 0u);
-            }
-#pragma unroll
-            for (int q = 0; q < kRouterRowChunks; ++q) {
-                const int c = base + lane + 32 * q;
-                if (c < nck) {
-                    float wf[8];
-                    unpack_w8(wv[q], wf);
-#pragma unroll
-                    for (int t = 0; t < kR64MaxTB; ++t) {
-                        if (t < tb) {
-                            const double2 *xp =
-                                reinterpret_cast<const double2 *>(xs + (size_t)t * H) + 4 * c;
-#pragma unroll
-                            for (int p = 0; p < 4; ++p) {
-                                const double2 xv = xp[p];
-                                acc[t] = fma(xv.x, (double)wf[2 * p], acc[t]);
-                                acc[t] = fma(xv.y, (double)wf[2 * p + 1], acc[t]);
-                            }
-                        }
-                    }
-                }
-            }
-        }
-#pragma unroll
-        for (int t = 0; t < kR64MaxTB; ++t) {
-            if (t < tb) {
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1)
-                    acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
-            }
-        }
-        const double b = bias != nullptr ? (double)bias[e] : 0.0;
-#pragma unroll
-        for (int t = 0; t < kR64MaxTB; ++t)
-            if (t < tb && lane == t)
-                vals[t * per_cta + (e - e_lo)] = acc[t] + b;
-    }
-    __syncthreads();
-    cluster_wait();  // every CTA of the cluster runs: CTA 0's shared memory may be written
-    {
-        const uint32_t r_logit = map_shared_rank(logit, 0);
-        const int n = e_hi - e_lo;
-        for (int i = threadIdx.x; i < tb * n; i += kR64Threads) {
-            const int t = i / n, j = i - t * n;
-            st_cluster_f64(r_logit + 8u * (uint32_t)(t * E + e_lo + j), vals[t * per_cta + j]);
-        }
-    }
-    cluster_sync();  // all logits are in CTA 0
-    if (rank != 0 || warp >= tb)
-        return;
-    // CTA 0, warp t: top_k by logit (ties to the lower id), softmax over them
-    const int t = warp;
-    const double *lt = logit + t * E;
     const int per_lane = (E + 31) / 32;
     uint32_t chosen = 0;
     double pick_v = 0.0, top = 0.0;
@@ -231,14 +163,160 @@ router_fp64_kernel(const void *__restrict__ x, int64_t T, int H,
             pick_e = be;
         }
     }
-    double ev = lane < top_k ? exp(pick_v - top) : 0.0;
-    double s = 0.0;
+    const double ev = lane < top_k ? exp(pick_v - top) : 0.0;
+    double sum = 0.0;
     for (int j = 0; j < top_k; ++j)
-        s += __shfl_sync(0xffffffffu, ev, j);
+        sum += __shfl_sync(0xffffffffu, ev, j);
     if (lane < top_k) {
-        ids[(t0 + t) * top_k + lane] = pick_e;
-        weights[(t0 + t) * top_k + lane] = (float)(ev / s);
+        ids_row[lane] = pick_e;
+        w_row[lane] = (float)(ev / sum);
     }
+}
+
+// ------------------------------------------------------ small-batch router
+// Up to 32 tokens: every logit by Dot2.  A cluster of 8 CTAs takes TB tokens
+// (one or two), CTA r the experts [r E/8, (r+1) E/8); 16 warps per CTA, one
+// expert row per warp at a time, each lane 16-byte chunks lane + 32 j of the
+// row.  The first chunks of each warp's first row are loaded before
+// griddepcontrol.wait (the router weights never come from the previous
+// kernel).  Logits go to CTA 0 by distributed shared memory, where one warp
+// per token picks and normalises.
+constexpr int kRdThreads = 512;
+constexpr int kRdWarps = kRdThreads / 32;
+constexpr int kRdMaxTB = 2;
+
+struct RdSmem {
+    uint32_t x, vals, logit, total;
+};
+
+__host__ __device__ inline RdSmem rd_smem_layout(int tb_max, int H, int E) {
+    RdSmem s;
+    uint32_t o = 0;
+    const int per_cta = (E + kRouterCluster - 1) / kRouterCluster;
+    s.x = o;     o = align_up_u32(o + (uint32_t)tb_max * H * 4, 16);
+    s.vals = o;  o = align_up_u32(o + (uint32_t)tb_max * per_cta * 8, 16);
+    s.logit = o; o = align_up_u32(o + (uint32_t)tb_max * E * 8, 16);
+    s.total = o;
+    return s;
+}
+
+__device__ __forceinline__ void rd_load_chunks(const uint4 *__restrict__ wrow, int base, int nck,
+                                               uint4 (&wv)[kRouterRowChunks]) {
+    const int lane = (int)lane_id();
+#pragma unroll
+    for (int q = 0; q < kRouterRowChunks; ++q) {
+        const int c = base + lane + 32 * q;
+        wv[q] = c < nck ? ld_stream_16(wrow + c) : make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+
+template <bool XF32, int TB>
+__global__ void __cluster_dims__(kRouterCluster, 1, 1) __launch_bounds__(kRdThreads, 1)
+router_dot2_kernel(const void *__restrict__ x, int64_t T, int H,
+                   const uint16_t *__restrict__ w_router, const float *__restrict__ bias, int E,
+                   int top_k, int32_t *__restrict__ ids, float *__restrict__ weights) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    constexpr int XB = XF32 ? 4 : 2;
+    const RdSmem L = rd_smem_layout(TB, H, E);
+    float *xs = reinterpret_cast<float *>(smem + L.x);          // [TB][H]
+    double *vals = reinterpret_cast<double *>(smem + L.vals);   // [TB][per_cta]
+    double *logit = reinterpret_cast<double *>(smem + L.logit); // [TB][E], CTA 0
+
+    const uint32_t rank = cluster_ctarank();
+    const int64_t t0 = (int64_t)(blockIdx.x / kRouterCluster) * TB;
+    const int tb = (T - t0 < (int64_t)TB) ? (int)(T - t0) : TB;
+    const int warp = (int)(threadIdx.x >> 5);
+    const int lane = (int)lane_id();
+    const int nck = H >> 3;
+    const int per_cta = (E + kRouterCluster - 1) / kRouterCluster;
+    const int e_lo = (int)rank * per_cta;
+    const int e_hi = min(E, e_lo + per_cta);
+    const int e_first = e_lo + warp;
+
+    uint4 wv[kRouterRowChunks];
+    if (e_first < e_hi)
+        rd_load_chunks(reinterpret_cast<const uint4 *>(w_router + (size_t)e_first * H), 0, nck, wv);
+    grid_dependents_launch();
+    grid_dependency_wait();
+    cluster_arrive_relaxed();  // "this CTA runs"; waited for before the first remote store
+
+    // activations of the block as fp32 (bf16 widens exactly)
+    {
+        const uint8_t *src = reinterpret_cast<const uint8_t *>(x) + (size_t)t0 * H * XB;
+        const int n8 = tb * H / 8;
+        for (int i = threadIdx.x; i < n8; i += kRdThreads) {
+            float4 a, b;
+            if constexpr (XF32) {
+                a = reinterpret_cast<const float4 *>(src)[2 * i];
+                b = reinterpret_cast<const float4 *>(src)[2 * i + 1];
+            } else {
+                const uint4 v = reinterpret_cast<const uint4 *>(src)[i];
+                a = make_float4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y));
+                b = make_float4(bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w));
+            }
+            reinterpret_cast<float4 *>(xs)[2 * i] = a;
+            reinterpret_cast<float4 *>(xs)[2 * i + 1] = b;
+        }
+    }
+    __syncthreads();
+
+    bool have = true;  // wv holds the first chunks of the warp's first row
+    for (int e = e_first; e < e_hi; e += kRdWarps) {
+        float2 s[TB], c[TB];
+#pragma unroll
+        for (int t = 0; t < TB; ++t) {
+            s[t] = make_float2(0.f, 0.f);
+            c[t] = make_float2(0.f, 0.f);
+        }
+        const uint4 *wrow = reinterpret_cast<const uint4 *>(w_router + (size_t)e * H);
+        for (int base = 0; base < nck; base += 32 * kRouterRowChunks) {
+            if (!have)
+                rd_load_chunks(wrow, base, nck, wv);
+            have = false;
+#pragma unroll
+            for (int q = 0; q < kRouterRowChunks; ++q) {
+                const int ch = base + lane + 32 * q;
+                if (ch < nck) {
+                    float2 wp[4], wn[4];
+                    dot2_unpack_w(wv[q], wp, wn);
+#pragma unroll
+                    for (int t = 0; t < TB; ++t) {
+                        if (t < tb) {
+                            const float4 *xp4 = reinterpret_cast<const float4 *>(xs + (size_t)t * H) + 2 * ch;
+                            const float4 a = xp4[0], b = xp4[1];
+                            const float2 xp[4] = {make_float2(a.x, a.y), make_float2(a.z, a.w),
+                                                  make_float2(b.x, b.y), make_float2(b.z, b.w)};
+                            dot2_chunk<XF32>(wp, wn, xp, s[t], c[t]);
+                        }
+                    }
+                }
+            }
+        }
+        const double b = bias != nullptr ? (double)bias[e] : 0.0;
+#pragma unroll
+        for (int t = 0; t < TB; ++t) {
+            if (t < tb) {
+                const double l = dot2_warp_total(s[t], c[t]) + b;
+                if (lane == 0)
+                    vals[t * per_cta + (e - e_lo)] = l;
+            }
+        }
+    }
+    __syncthreads();
+    cluster_wait();  // every CTA of the cluster runs: CTA 0's shared memory may be written
+    {
+        const uint32_t r_logit = map_shared_rank(logit, 0);
+        const int n = e_hi - e_lo;
+        for (int i = threadIdx.x; i < tb * n; i += kRdThreads) {
+            const int t = i / n, j = i - t * n;
+            st_cluster_f64(r_logit + 8u * (uint32_t)(t * E + e_lo + j), vals[t * per_cta + j]);
+        }
+    }
+    cluster_sync();  // all logits are in CTA 0
+    if (rank != 0 || warp >= tb)
+        return;
+    topk_softmax_warp(logit + warp * E, E, top_k, ids + (t0 + warp) * top_k,
+                      weights + (t0 + warp) * top_k);
 }
 
 // ------------------------------------------------------- tiled fp32 router
@@ -249,7 +327,7 @@ router_fp64_kernel(const void *__restrict__ x, int64_t T, int H,
 // keeps TM tokens x 4 experts of accumulators.  Each 32-term block is summed
 // on its own and then added to the running total, which bounds the rounding
 // error by (32 + ceil(H/32) + 2) u sum|x_h w_h| + u |l|.  Candidates and their
-// fp64 refinement then follow the small-batch kernel's steps 3 to 5.
+// Dot2 refinement follow.
 constexpr int kRtBE = 128;
 constexpr int kRtBK = 32;
 constexpr int kRtPad = 4;
@@ -281,35 +359,45 @@ __host__ __device__ inline RtSmem rt_smem_layout(int BT, int E) {
     return s;
 }
 
-// fp64 logit of expert e for one token whose activations are in global memory.
+// Dot2 logit of expert e for one token whose activations are in global
+// memory (one warp); eight chunks per lane are loaded before they are used.
 template <bool XF32>
-__device__ double logit_fp64_global(const void *xrow, const uint16_t *__restrict__ w_router,
+__device__ double logit_dot2_global(const void *xrow, const uint16_t *__restrict__ w_router,
                                     const float *__restrict__ bias, int H, int e) {
+    constexpr int U = 8;
     const int lane = (int)lane_id();
     const int nck = H >> 3;
     const uint4 *wrow = reinterpret_cast<const uint4 *>(w_router + (size_t)e * H);
-    double acc0 = 0.0, acc1 = 0.0;
-    for (int c = lane; c < nck; c += 32) {
-        float wf[8], xf[8];
-        unpack_w8(wrow[c], wf);
-        if constexpr (XF32) {
-            const float4 a = reinterpret_cast<const float4 *>(xrow)[2 * c];
-            const float4 b = reinterpret_cast<const float4 *>(xrow)[2 * c + 1];
-            xf[0] = a.x; xf[1] = a.y; xf[2] = a.z; xf[3] = a.w;
-            xf[4] = b.x; xf[5] = b.y; xf[6] = b.z; xf[7] = b.w;
-        } else {
-            unpack_w8(reinterpret_cast<const uint4 *>(xrow)[c], xf);
+    float2 s = make_float2(0.f, 0.f), c = make_float2(0.f, 0.f);
+    for (int base = 0; base < nck; base += 32 * U) {
+        uint4 wv[U], xv[U][XF32 ? 2 : 1];
+#pragma unroll
+        for (int q = 0; q < U; ++q) {
+            const int ch = base + lane + 32 * q;
+            const bool ok = ch < nck;
+            wv[q] = ok ? wrow[ch] : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int h = 0; h < (XF32 ? 2 : 1); ++h)
+                xv[q][h] = ok ? reinterpret_cast<const uint4 *>(xrow)[(XF32 ? 2 : 1) * ch + h]
+                              : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
-        for (int j = 0; j < 8; j += 2) {
-            acc0 = fma((double)xf[j], (double)wf[j], acc0);
-            acc1 = fma((double)xf[j + 1], (double)wf[j + 1], acc1);
+        for (int q = 0; q < U; ++q) {
+            float2 wp[4], wn[4], xp[4];
+            dot2_unpack_w(wv[q], wp, wn);
+            if constexpr (XF32) {
+                xp[0] = make_float2(__uint_as_float(xv[q][0].x), __uint_as_float(xv[q][0].y));
+                xp[1] = make_float2(__uint_as_float(xv[q][0].z), __uint_as_float(xv[q][0].w));
+                xp[2] = make_float2(__uint_as_float(xv[q][1].x), __uint_as_float(xv[q][1].y));
+                xp[3] = make_float2(__uint_as_float(xv[q][1].z), __uint_as_float(xv[q][1].w));
+            } else {
+                xp[0] = bf16x2_to_f2(xv[q][0].x); xp[1] = bf16x2_to_f2(xv[q][0].y);
+                xp[2] = bf16x2_to_f2(xv[q][0].z); xp[3] = bf16x2_to_f2(xv[q][0].w);
+            }
+            dot2_chunk<XF32>(wp, wn, xp, s, c);  // zero chunks add exact zeros
         }
     }
-    double acc = acc0 + acc1;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1)
-        acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    double acc = dot2_warp_total(s, c);
     if (bias != nullptr)
         acc += (double)bias[e];
     return acc;
@@ -546,7 +634,7 @@ router_tiled_kernel(const void *__restrict__ x, int64_t T, int H,
     }
     cluster_sync();  // candidate lists visible to every CTA
 
-    // every CTA: fp64 logits of the candidates in its expert slice
+    // every CTA: Dot2 logits of the candidates in its expert slice
     {
         const uint32_t r_ncand = map_shared_rank(ncand, 0);
         const uint32_t r_cand = map_shared_rank(cand, 0);
@@ -569,17 +657,17 @@ router_tiled_kernel(const void *__restrict__ x, int64_t T, int H,
                 if ((mine++ % (kRtThreads / 32)) != warp)
                     continue;
                 const uint8_t *xrow = reinterpret_cast<const uint8_t *>(x) + (size_t)(t0 + t) * H * XB;
-                const double v = logit_fp64_global<XF32>(xrow, w_router, bias, H, e);
+                const double v = logit_dot2_global<XF32>(xrow, w_router, bias, H, e);
                 if (lane == 0)
                     st_cluster_f64(r_cval + 8u * (uint32_t)(t * kRouterMaxCand + ci), v);
             }
         }
     }
-    cluster_sync();  // fp64 logits are in CTA 0
+    cluster_sync();  // refined logits are in CTA 0
     if (rank != 0)
         return;
 
-    // CTA 0: pick top_k on the fp64 logits, renormalise, write
+    // CTA 0: pick top_k on the refined logits, renormalise, write
     for (int t = warp; t < tb; t += kRtThreads / 32) {
         const int nc = ncand[t];
         double bv_list = 0.0, top = 0.0;
@@ -630,7 +718,7 @@ router_tiled_kernel(const void *__restrict__ x, int64_t T, int H,
             for (int e = 0; e < E; ++e) {
                 if ((double)lt[e] < thr)
                     continue;
-                const double v = logit_fp64_global<XF32>(xrow, w_router, bias, H, e);
+                const double v = logit_dot2_global<XF32>(xrow, w_router, bias, H, e);
                 // insert: lanes whose value ranks below v shift down by one
                 const bool below = !(lv > v || (lv == v && li < e));
                 const uint32_t m = __ballot_sync(0xffffffffu, below && lane < top_k);

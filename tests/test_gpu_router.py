@@ -54,6 +54,18 @@ def test_router_ragged_token_blocks(oracle_lib, T):
     _route_and_check(oracle_lib, WL["decode"], T, seed=77)
 
 
+# Up to 32 tokens every logit is a compensated (Dot2) fp32 dot product: one
+# token per cluster of 8 CTAs while the clusters fit on the SMs at once
+# (T <= 18 on 148 SMs), else two.  fp32 activations add the exact product
+# errors (TwoProd) to the compensation term.
+@pytest.mark.parametrize("T,x_dtype", [(1, "f32"), (8, "f32"), (19, "bf16"), (32, "bf16"),
+                                       (27, "f32")])
+def test_router_dot2_small_batches(oracle_lib, T, x_dtype):
+    wl = workloads.Workload("dot2", (T,), 4096, 128, 8, 16, 0, x_dtype, "zipf1.1", (1,))
+    excused = _route_and_check(oracle_lib, wl, T, seed=40 + T)
+    assert excused == 0
+
+
 def test_router_odd_sizes(oracle_lib):
     wl = workloads.Workload("odd", (5,), 200, 37, 5, 16, 0, "bf16", "zipf1.1", (1,))
     _route_and_check(oracle_lib, wl, 11, seed=5)
