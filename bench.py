@@ -56,6 +56,10 @@ def parse_args():
                     help="profiling only: fewer experts (same H, I, top_k) to keep an ncu "
                          "capture to a few GB on the device")
     ap.add_argument("--flush-mib", type=int, default=FLUSH_BYTES >> 20)
+    ap.add_argument("--router-only", action="store_true",
+                    help="profiling only: run moe_route alone on the workload's router weights, "
+                         "bias and activations (no expert weights on the device) and print its "
+                         "per-call time; no bench line")
     return ap.parse_args()
 
 
@@ -534,6 +538,34 @@ def run_ours(args, wl):
     print(json.dumps(line), flush=True)
 
 
+def run_router_only(args, wl):
+    """Profiling aid: moe_route alone, W warm-up and K timed calls per token count."""
+    import expert_decode_b200 as ed
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    w_router = workloads._bf16_normal((wl.E, wl.H), workloads.SEED_BASE + 1, device,
+                                      workloads.WEIGHT_STD)
+    bias = workloads.router_bias(wl.bias, wl.E)
+    bias = None if bias is None else bias.to(device)
+    for T in wl.T:
+        x = workloads.make_x(wl, T, device=device)
+        ids = torch.empty((T, wl.top_k), dtype=torch.int32, device=device)
+        w = torch.empty((T, wl.top_k), dtype=torch.float32, device=device)
+        for _ in range(args.warmup):
+            ed.moe_route(x, w_router, bias, wl.top_k, ids=ids, weights=w)
+        torch.cuda.synchronize()
+        ed.ep_check_status()
+        es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        es.record()
+        for _ in range(args.steps):
+            ed.moe_route(x, w_router, bias, wl.top_k, ids=ids, weights=w)
+        ee.record()
+        torch.cuda.synchronize()
+        ed.ep_check_status()
+        print(f"router {wl.name} T={T}: {es.elapsed_time(ee) * 1e3 / max(args.steps, 1):.2f} us "
+              f"per call (back to back, weights L2-resident)", flush=True)
+
+
 def main():
     args = parse_args()
     wl = workloads.WORKLOADS[args.config]
@@ -543,6 +575,8 @@ def main():
                                  description=wl.description + f" (E reduced to {args.experts})")
     if args.impl == "reference":
         run_reference(args, wl)
+    elif args.router_only:
+        run_router_only(args, wl)
     else:
         run_ours(args, wl)
 

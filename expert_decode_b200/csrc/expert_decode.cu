@@ -373,12 +373,20 @@ extern "C" ep_status moe_route(const void *x, ep_dtype x_dtype, int64_t T, int64
         if ((int)L.total > d->smem_optin)
             return fail(EP_EINVAL, "moe_route: E = %lld needs %u bytes of shared memory",
                         (long long)E, L.total);
-        const unsigned C = (unsigned)((E + epk::kRtBE - 1) / epk::kRtBE);
-        const dim3 grid(C, (unsigned)((T + BT - 1) / BT));
+        // a cluster of CE expert slices x CK slices of H (at most 8 CTAs);
+        // H is split only as far as it takes to fill about two waves of CTAs
+        const int CE = (int)((E + epk::kRtBE - 1) / epk::kRtBE);
+        const int nkt = (int)((H + epk::kRtBK - 1) / epk::kRtBK);
+        const int64_t blocks = (T + BT - 1) / BT;
+        const int64_t want = (2 * (int64_t)d->sm_count + blocks * CE - 1) / (blocks * CE);
+        const int CK = (int)std::max<int64_t>(
+            1, std::min<int64_t>(want, std::min(epk::kRouterCluster / CE, nkt)));
+        const dim3 grid((unsigned)(CE * CK), (unsigned)((T + BT - 1) / BT));
         cudaError_t e;
 #define EPK_RT(XF, TMV)                                                                        \
-    e = launch_cluster(epk::router_tiled_kernel<XF, TMV>, grid, epk::kRtThreads, L.total, st, C, \
-                       x, T, (int)H, wr, bias, (int)E, top_k, ids, weights)
+    e = launch_cluster(epk::router_tiled_kernel<XF, TMV>, grid, epk::kRtThreads, L.total, st,  \
+                       (unsigned)(CE * CK), x, T, (int)H, wr, bias, (int)E, top_k, ids, weights, \
+                       CE, CK)
         if (x_dtype == EP_F32) {
             if (BT == 32) EPK_RT(true, 4); else if (BT == 16) EPK_RT(true, 2); else EPK_RT(true, 1);
         } else {

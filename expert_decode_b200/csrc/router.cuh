@@ -320,14 +320,18 @@ router_dot2_kernel(const void *__restrict__ x, int64_t T, int H,
 }
 
 // ------------------------------------------------------- tiled fp32 router
-// For larger batches the fp32 logits are a register-tiled SIMT product: a
-// cluster of ceil(E / 128) CTAs covers one block of BT tokens, CTA r the
-// experts [128 r, 128 r + 128).  Both operand tiles are widened to fp32 in
-// shared memory, 32 values of H at a time (double-buffered), and each thread
-// keeps TM tokens x 4 experts of accumulators.  Each 32-term block is summed
-// on its own and then added to the running total, which bounds the rounding
-// error by (32 + ceil(H/32) + 2) u sum|x_h w_h| + u |l|.  Candidates and their
-// Dot2 refinement follow.
+// For larger batches the fp32 logits are a register-tiled SIMT product.  A
+// cluster of CE x CK CTAs covers one block of BT tokens: CE = ceil(E / 128)
+// expert slices times CK slices of H (CE CK <= 8).  CTA (e, k) accumulates
+// the experts [128 e, 128 e + 128) over its k-tiles of 32 values of H; both
+// operand tiles are widened to fp32 in shared memory (double-buffered), and
+// each thread keeps TM tokens x 4 experts of packed accumulators.  The CK
+// partial tiles are then added in a fixed order, each CTA taking a share of
+// the tokens.  Every 32-term block is summed on its own (two 16-term packed
+// halves) before it joins the running total, which bounds the rounding error
+// of a logit by gamma_n sum_h |x_h w_h| + u |l|, n = 32 + (k-tiles per CTA)
+// + CK + 2, with sum |x_h w_h| <= ||x|| ||w||.  Candidates and their Dot2
+// refinement follow.
 constexpr int kRtBE = 128;
 constexpr int kRtBK = 32;
 constexpr int kRtPad = 4;
@@ -340,7 +344,7 @@ __host__ __device__ inline int rt_block_tokens(int E) {
 }
 
 struct RtSmem {
-    uint32_t xs, ws, xsq, wsq, logit, bound, ncand, cand, cval, total;
+    uint32_t xs, ws, xsq, wsq, part, logit, bound, ncand, cand, cval, total;
 };
 
 __host__ __device__ inline RtSmem rt_smem_layout(int BT, int E) {
@@ -350,6 +354,7 @@ __host__ __device__ inline RtSmem rt_smem_layout(int BT, int E) {
     s.ws = o;    o = align_up_u32(o + 2u * kRtBE * (kRtBK + kRtPad) * 4, 16);
     s.xsq = o;   o = align_up_u32(o + (uint32_t)BT * 4, 16);
     s.wsq = o;   o = align_up_u32(o + kRtBE * 4, 16);
+    s.part = o;  o = align_up_u32(o + (uint32_t)BT * kRtBE * 4, 16);
     s.logit = o; o = align_up_u32(o + (uint32_t)BT * E * 4, 16);
     s.bound = o; o = align_up_u32(o + (uint32_t)BT * E * 4, 16);
     s.ncand = o; o = align_up_u32(o + (uint32_t)BT * 4, 16);
@@ -407,7 +412,8 @@ template <bool XF32, int TM>
 __global__ void __launch_bounds__(kRtThreads, 1)
 router_tiled_kernel(const void *__restrict__ x, int64_t T, int H,
                     const uint16_t *__restrict__ w_router, const float *__restrict__ bias, int E,
-                    int top_k, int32_t *__restrict__ ids, float *__restrict__ weights) {
+                    int top_k, int32_t *__restrict__ ids, float *__restrict__ weights, int CE,
+                    int CK) {
     constexpr int BT = 8 * TM;             // tokens per cluster
     constexpr int XB = XF32 ? 4 : 2;
     constexpr int LD = kRtBK + kRtPad;     // padded row of a k-tile, in floats
@@ -417,6 +423,7 @@ router_tiled_kernel(const void *__restrict__ x, int64_t T, int H,
     float *ws = reinterpret_cast<float *>(smem + L.ws);       // [2][kRtBE][LD]
     float *xsq = reinterpret_cast<float *>(smem + L.xsq);
     float *wsq = reinterpret_cast<float *>(smem + L.wsq);
+    float *part = reinterpret_cast<float *>(smem + L.part);   // [BT][kRtBE], this CTA's k-slice
     float *logit = reinterpret_cast<float *>(smem + L.logit); // [BT][E], CTA 0
     float *bound = reinterpret_cast<float *>(smem + L.bound); // [BT][E], CTA 0
     int *ncand = reinterpret_cast<int *>(smem + L.ncand);
@@ -425,12 +432,12 @@ router_tiled_kernel(const void *__restrict__ x, int64_t T, int H,
 
     grid_dependents_launch();
     grid_dependency_wait();
-    cluster_arrive_relaxed();
 
     const uint32_t rank = cluster_ctarank();
     const int64_t t0 = (int64_t)blockIdx.y * BT;
     const int tb = (T - t0 < (int64_t)BT) ? (int)(T - t0) : BT;
-    const int e0 = (int)rank * kRtBE;
+    const int e_part = (int)rank % CE, k_part = (int)rank / CE;
+    const int e0 = e_part * kRtBE;
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const int tx = lane, ty = warp;        // experts tx + 32 j, tokens TM ty + i
@@ -474,52 +481,70 @@ router_tiled_kernel(const void *__restrict__ x, int64_t T, int H,
                 unpack_w8(ld_stream_16(w_router + (size_t)(e0 + row) * H + k0 + kc), wr[q]);
         }
     };
+    // A thread stashes the same rows' chunks in every k-tile, so it also
+    // keeps their running sums of squares (for the error bound).
+    constexpr int XQ = (XCH + kRtThreads - 1) / kRtThreads;
+    constexpr int WQ = WCH / kRtThreads;
+    float2 x2[XQ], w2[WQ];
+#pragma unroll
+    for (int q = 0; q < XQ; ++q)
+        x2[q] = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int q = 0; q < WQ; ++q)
+        w2[q] = make_float2(0.f, 0.f);
     auto stash = [&](int buf) {
 #pragma unroll
-        for (int q = 0; q < (XCH + kRtThreads - 1) / kRtThreads; ++q) {
+        for (int q = 0; q < XQ; ++q) {
             const int ch = tid + q * kRtThreads;
             if (ch < XCH) {
                 const int row = ch / (kRtBK / 8), kc = (ch % (kRtBK / 8)) * 8;
                 float4 *d = reinterpret_cast<float4 *>(xs + (size_t)(buf * BT + row) * LD + kc);
                 d[0] = make_float4(xr[q][0], xr[q][1], xr[q][2], xr[q][3]);
                 d[1] = make_float4(xr[q][4], xr[q][5], xr[q][6], xr[q][7]);
+#pragma unroll
+                for (int j = 0; j < 8; j += 2)
+                    x2[q] = ffma2(make_float2(xr[q][j], xr[q][j + 1]),
+                                  make_float2(xr[q][j], xr[q][j + 1]), x2[q]);
             }
         }
 #pragma unroll
-        for (int q = 0; q < WCH / kRtThreads; ++q) {
+        for (int q = 0; q < WQ; ++q) {
             const int ch = tid + q * kRtThreads;
             const int row = ch / (kRtBK / 8), kc = (ch % (kRtBK / 8)) * 8;
             float4 *d = reinterpret_cast<float4 *>(ws + (size_t)(buf * kRtBE + row) * LD + kc);
             d[0] = make_float4(wr[q][0], wr[q][1], wr[q][2], wr[q][3]);
             d[1] = make_float4(wr[q][4], wr[q][5], wr[q][6], wr[q][7]);
+#pragma unroll
+            for (int j = 0; j < 8; j += 2)
+                w2[q] = ffma2(make_float2(wr[q][j], wr[q][j + 1]),
+                              make_float2(wr[q][j], wr[q][j + 1]), w2[q]);
         }
     };
 
-    float acc[TM][4], xs2[TM], ws2[4];
+    float acc[TM][4];
 #pragma unroll
-    for (int i = 0; i < TM; ++i) {
-        xs2[i] = 0.f;
+    for (int i = 0; i < TM; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j)
             acc[i][j] = 0.f;
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-        ws2[j] = 0.f;
     const int nkt = (H + kRtBK - 1) / kRtBK;
-    fetch(0);
-    stash(0);
+    const int kt_lo = nkt * k_part / CK, kt_hi = nkt * (k_part + 1) / CK;
+    if (kt_lo < kt_hi) {
+        fetch(kt_lo * kRtBK);
+        stash(0);
+    }
     __syncthreads();
-    for (int kt = 0; kt < nkt; ++kt) {
-        const int buf = kt & 1;
-        if (kt + 1 < nkt)
+    for (int kt = kt_lo; kt < kt_hi; ++kt) {
+        const int buf = (kt - kt_lo) & 1;
+        if (kt + 1 < kt_hi)
             fetch((kt + 1) * kRtBK);
-        float blk[TM][4];
+        // two 16-term packed halves per 32-term block
+        float2 blk[TM][4];
 #pragma unroll
         for (int i = 0; i < TM; ++i)
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-                blk[i][j] = 0.f;
+                blk[i][j] = make_float2(0.f, 0.f);
         const float *xb = xs + (size_t)buf * BT * LD;
         const float *wb = ws + (size_t)buf * kRtBE * LD;
 #pragma unroll
@@ -535,71 +560,75 @@ router_tiled_kernel(const void *__restrict__ x, int64_t T, int H,
             for (int i = 0; i < TM; ++i)
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    blk[i][j] = fmaf(xv[i].x, wv[j].x, blk[i][j]);
-                    blk[i][j] = fmaf(xv[i].y, wv[j].y, blk[i][j]);
-                    blk[i][j] = fmaf(xv[i].z, wv[j].z, blk[i][j]);
-                    blk[i][j] = fmaf(xv[i].w, wv[j].w, blk[i][j]);
+                    blk[i][j] = ffma2(make_float2(xv[i].x, xv[i].y), make_float2(wv[j].x, wv[j].y),
+                                      blk[i][j]);
+                    blk[i][j] = ffma2(make_float2(xv[i].z, xv[i].w), make_float2(wv[j].z, wv[j].w),
+                                      blk[i][j]);
                 }
-            if (ty == 0) {
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    ws2[j] = fmaf(wv[j].x, wv[j].x, ws2[j]);
-                    ws2[j] = fmaf(wv[j].y, wv[j].y, ws2[j]);
-                    ws2[j] = fmaf(wv[j].z, wv[j].z, ws2[j]);
-                    ws2[j] = fmaf(wv[j].w, wv[j].w, ws2[j]);
-                }
-            }
-            if (tx == 0) {
-#pragma unroll
-                for (int i = 0; i < TM; ++i) {
-                    xs2[i] = fmaf(xv[i].x, xv[i].x, xs2[i]);
-                    xs2[i] = fmaf(xv[i].y, xv[i].y, xs2[i]);
-                    xs2[i] = fmaf(xv[i].z, xv[i].z, xs2[i]);
-                    xs2[i] = fmaf(xv[i].w, xv[i].w, xs2[i]);
-                }
-            }
         }
 #pragma unroll
         for (int i = 0; i < TM; ++i)
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-                acc[i][j] += blk[i][j];
+                acc[i][j] += blk[i][j].x + blk[i][j].y;
         // the other buffer was last read before the previous barrier
-        if (kt + 1 < nkt) {
+        if (kt + 1 < kt_hi) {
             stash(buf ^ 1);
             __syncthreads();
         }
     }
-    if (ty == 0)
+    // this CTA's k-slice: partial sums and sums of squares
+#pragma unroll
+    for (int i = 0; i < TM; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-            wsq[tx + 32 * j] = ws2[j];
-    if (tx == 0)
+            part[(TM * ty + i) * kRtBE + tx + 32 * j] = acc[i][j];
+    // a row's chunks sit in 4 adjacent lanes (ch = 4 row + c)
 #pragma unroll
-        for (int i = 0; i < TM; ++i)
-            xsq[TM * ty + i] = xs2[i];
+    for (int q = 0; q < XQ; ++q) {
+        float v = x2[q].x + x2[q].y;
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        const int ch = tid + q * kRtThreads;
+        if (ch < XCH && (ch & 3) == 0)
+            xsq[ch >> 2] = v;
+    }
+#pragma unroll
+    for (int q = 0; q < WQ; ++q) {
+        float v = w2[q].x + w2[q].y;
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        const int ch = tid + q * kRtThreads;
+        if ((ch & 3) == 0)
+            wsq[ch >> 2] = v;
+    }
     __syncthreads();
-    cluster_wait();  // every CTA runs: CTA 0's shared memory may be written
+    cluster_sync();  // every CTA runs and has its partial tile in place
     {
+        // CTA (e, k) adds the CK partials of tokens [BT k / CK, BT (k+1) / CK)
+        // of expert slice e, in ascending k-slice order
         const uint32_t r_logit = map_shared_rank(logit, 0);
         const uint32_t r_bound = map_shared_rank(bound, 0);
         const float u = 5.9604644775390625e-8f;  // 2^-24
-        const float n = (float)(kRtBK + nkt + 2);
+        const float n = (float)(kRtBK + (nkt + CK - 1) / CK + CK + 2);
         const float gam = n * u / (1.0f - n * u);
-#pragma unroll
-        for (int i = 0; i < TM; ++i) {
-            const int t = TM * ty + i;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int e = e0 + tx + 32 * j;
-                if (t < tb && e < E) {
-                    const float l = acc[i][j] + (bias != nullptr ? bias[e] : 0.f);
-                    const float d =
-                        1.5f * (gam * sqrtf(xsq[t]) * sqrtf(wsq[tx + 32 * j]) + u * fabsf(l)) + 1e-30f;
-                    st_cluster_f32(r_logit + 4u * (uint32_t)(t * E + e), l);
-                    st_cluster_f32(r_bound + 4u * (uint32_t)(t * E + e), d);
-                }
+        const int t_lo = BT * k_part / CK, t_hi = BT * (k_part + 1) / CK;
+        for (int idx = tid; idx < (t_hi - t_lo) * kRtBE; idx += kRtThreads) {
+            const int t = t_lo + idx / kRtBE, el = idx % kRtBE;
+            const int e = e0 + el;
+            if (t >= tb || e >= E)
+                continue;
+            float sum = 0.f, x2 = 0.f, w2 = 0.f;
+            for (int j = 0; j < CK; ++j) {
+                const uint32_t r = (uint32_t)(e_part + CE * j);
+                sum += ld_cluster_f32(map_shared_rank(part + t * kRtBE + el, r));
+                x2 += ld_cluster_f32(map_shared_rank(xsq + t, r));
+                w2 += ld_cluster_f32(map_shared_rank(wsq + el, r));
             }
+            const float l = sum + (bias != nullptr ? bias[e] : 0.f);
+            const float d = 1.5f * (gam * sqrtf(x2) * sqrtf(w2) + u * fabsf(l)) + 1e-30f;
+            st_cluster_f32(r_logit + 4u * (uint32_t)(t * E + e), l);
+            st_cluster_f32(r_bound + 4u * (uint32_t)(t * E + e), d);
         }
     }
     cluster_sync();  // all logits and bounds are in CTA 0
@@ -654,7 +683,8 @@ router_tiled_kernel(const void *__restrict__ x, int64_t T, int H,
                 const int e = cand[t * kRouterMaxCand + ci];
                 if (e < e0 || e >= e0 + kRtBE)
                     continue;
-                if ((mine++ % (kRtThreads / 32)) != warp)
+                // the CK CTAs of this expert slice share its candidates
+                if ((mine++ % (CK * (kRtThreads / 32))) != warp + k_part * (kRtThreads / 32))
                     continue;
                 const uint8_t *xrow = reinterpret_cast<const uint8_t *>(x) + (size_t)(t0 + t) * H * XB;
                 const double v = logit_dot2_global<XF32>(xrow, w_router, bias, H, e);
