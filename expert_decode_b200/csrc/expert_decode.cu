@@ -204,7 +204,7 @@ Workspace workspace_layout(int64_t T, int64_t H, int64_t E, int64_t k, int64_t I
 struct StreamingPlan {
     bool fits = false;
     int down_rw = 1;  // down-projection rows per consumer warp per slot
-    int down_nh = 1;  // h buffers in the down kernel
+    size_t down_h_arena = 0;  // bytes of the down kernel's h arena
     bool xs_f32 = false;  // gate/up keeps x as fp32 in shared memory
     int gu_slots = 0, down_slots = 0, down_grid = 0, down_rows_max = 0;
     size_t gu_smem = 0, down_smem = 0;
@@ -235,10 +235,11 @@ StreamingPlan streaming_fit(const DeviceInfo &d, int64_t T, int64_t H, int xb, i
     p.down_grid = (int)std::max<int64_t>(1, std::min<int64_t>(d.sm_count, H / 8));
     p.down_rows_max = (int)((H + p.down_grid - 1) / p.down_grid);
     // two rows per warp per slot when three such slots still fit
+    const size_t h_min = (size_t)T * I_max * 4;  // one group of every token
     for (int rw = epk::kDownMaxRowsPerWarp; rw >= 1; --rw) {
         slots = epk::kDownMaxSlots;
         while (slots >= 2 && epk::down_smem_layout((int)T, (int)I_max, slots, p.down_rows_max,
-                                                   rw, 1).total > budget)
+                                                   rw, h_min).total > budget)
             --slots;
         if (slots >= (rw > 1 ? 3 : 2)) {
             p.down_rw = rw;
@@ -248,11 +249,12 @@ StreamingPlan streaming_fit(const DeviceInfo &d, int64_t T, int64_t H, int xb, i
     }
     if (p.down_slots < 2)
         return p;
-    // a second h buffer only when the weight ring keeps its shape
-    p.down_nh = epk::down_smem_layout((int)T, (int)I_max, p.down_slots, p.down_rows_max,
-                                      p.down_rw, 2).total <= budget ? 2 : 1;
+    // the h arena takes whatever the weight ring leaves of the budget
+    const size_t rest = budget - epk::down_smem_layout((int)T, (int)I_max, p.down_slots,
+                                                       p.down_rows_max, p.down_rw, 0).total;
+    p.down_h_arena = std::max(h_min, rest / 128 * 128);
     p.down_smem = epk::down_smem_layout((int)T, (int)I_max, p.down_slots, p.down_rows_max,
-                                        p.down_rw, p.down_nh).total;
+                                        p.down_rw, p.down_h_arena).total;
     p.fits = true;
     return p;
 }
@@ -519,7 +521,7 @@ extern "C" ep_status moe_ffn_forward(const void *x, ep_dtype x_dtype, int64_t T,
         da.T = (int)T; da.H = (int)H; da.E = (int)E; da.I = (int)I; da.I_s = (int)I_s;
         da.top_k = top_k; da.n_slots = sp.down_slots; da.rows_max = sp.down_rows_max;
         da.rw = sp.down_rw;
-        da.n_h = sp.down_nh;
+        da.h_arena = (int)sp.down_h_arena;
         da.w_down = static_cast<const uint16_t *>(w_down);
         da.ws_down = static_cast<const uint16_t *>(ws_down);
         da.ids = ids;

@@ -524,12 +524,13 @@ constexpr int kDownConsumerWarps = 8;
 constexpr int kDownMaxRowsPerWarp = 2;
 constexpr int kDownThreads = 32 * (1 + kDownConsumerWarps);
 constexpr int kDownMaxSlots = 8;
+constexpr int kDownHGroups = 8;  // groups whose activations may be in the arena at once
 constexpr uint32_t kDownBarPlan = 1;
 
 struct StreamDownArgs {
     int T, H, E, I, I_s, top_k, n_slots, rows_max;
     int rw;  // rows per consumer warp per slot (1 or 2)
-    int n_h;  // h buffers (1, or 2 so that the next group's h lands during this one)
+    int h_arena;  // bytes of the h arena, >= T * max(I, I_s) * 4
     const uint16_t *w_down, *ws_down;
     const int32_t *ids;
     const float *weights;
@@ -541,17 +542,22 @@ struct DownSmem {
     size_t plan, hbuf, slots, acc, sacc, bars, total;
 };
 
-// An h buffer holds a group's activations: up to T rows of max(I, I_s) fp32.
+// The h arena holds the activations of the groups in flight, each group's
+// rows (count x width fp32) contiguous at a 128-byte boundary.
 __host__ __device__ inline DownSmem down_smem_layout(int T, int I_max, int n_slots, int rows_max,
-                                                    int rw, int n_h) {
+                                                    int rw, size_t h_arena) {
     DownSmem s;
     size_t o = 0;
+    (void)T;
+    (void)I_max;
     s.plan = o;  o = align_up_sz(o + sizeof(StreamPlan), 128);
-    s.hbuf = o;  o = align_up_sz(o + (size_t)n_h * T * I_max * 4, 128);
+    s.hbuf = o;  o = align_up_sz(o + h_arena, 128);
     s.slots = o; o = align_up_sz(o + (size_t)n_slots * kDownConsumerWarps * rw * I_max * 2, 128);
     s.acc = o;   o = align_up_sz(o + (size_t)rows_max * kStreamMaxT * 4, 128);
     s.sacc = o;  o = align_up_sz(o + (size_t)rows_max * kStreamMaxT * 4, 128);
-    s.bars = o;  o = align_up_sz(o + (size_t)(2 * kDownMaxSlots + 5) * 8 + 16, 128);
+    s.bars = o;
+    o = align_up_sz(o + (size_t)(2 * kDownMaxSlots + 2 * kDownHGroups + 1) * 8 +
+                        (size_t)kDownHGroups * 4 + 16, 128);
     s.total = o;
     return s;
 }
@@ -744,20 +750,23 @@ __device__ __forceinline__ bool down_group(const DownGroup &g) {
 __global__ void __launch_bounds__(kDownThreads, 1) stream_down_fold_kernel(const StreamDownArgs a) {
     extern __shared__ __align__(1024) uint8_t smem[];
     const int I_max = a.I > a.I_s ? a.I : a.I_s;
-    const DownSmem L = down_smem_layout(a.T, I_max, a.n_slots, a.rows_max, a.rw, a.n_h);
+    const DownSmem L = down_smem_layout(a.T, I_max, a.n_slots, a.rows_max, a.rw,
+                                        (size_t)a.h_arena);
     StreamPlan &P = *reinterpret_cast<StreamPlan *>(smem + L.plan);
-    float *hbuf = reinterpret_cast<float *>(smem + L.hbuf);   // [n_h][T * I_max]
+    float *hbuf = reinterpret_cast<float *>(smem + L.hbuf);   // the h arena
     uint8_t *slots = smem + L.slots;
     float *yacc = reinterpret_cast<float *>(smem + L.acc);    // routed fold [row][token]
     float *sacc = reinterpret_cast<float *>(smem + L.sacc);   // shared expert [row][token]
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bars);
     uint64_t *empty = full + kDownMaxSlots;
-    uint64_t *hfull = empty + kDownMaxSlots;   // [2]
-    uint64_t *hempty = hfull + 2;              // [2]
-    uint64_t *planbar = hempty + 2;
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(planbar + 1);
-    const int H = a.H, NS = a.n_slots, NH = a.n_h;
-    const size_t h_elems = (size_t)a.T * I_max;
+    uint64_t *hfull = empty + kDownMaxSlots;      // [kDownHGroups]
+    uint64_t *hempty = hfull + kDownHGroups;      // [kDownHGroups]
+    uint64_t *planbar = hempty + kDownHGroups;
+    int *hoff = reinterpret_cast<int *>(planbar + 1);  // [kDownHGroups] arena offsets (floats)
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(hoff + kDownHGroups);
+    const int H = a.H, NS = a.n_slots;
+    constexpr int HK = kDownHGroups;
+    const int HA = a.h_arena / 4;  // arena capacity in floats
     const int rows_per_slot = kDownConsumerWarps * a.rw;
     const size_t slot_bytes = (size_t)rows_per_slot * I_max * 2;
     const int warp = (int)(threadIdx.x >> 5);
@@ -767,7 +776,7 @@ __global__ void __launch_bounds__(kDownThreads, 1) stream_down_fold_kernel(const
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kDownConsumerWarps);
         }
-        for (int b = 0; b < NH; ++b) {
+        for (int b = 0; b < HK; ++b) {
             mbar_init(&hfull[b], 1);
             mbar_init(&hempty[b], kDownConsumerWarps);
         }
@@ -790,6 +799,10 @@ __global__ void __launch_bounds__(kDownThreads, 1) stream_down_fold_kernel(const
             const uint64_t pol_h = policy_evict_last();
             int issued = 0, h_issued = 0;
             bool waited = false;
+            // arena ring: the live groups [g_old, h_issued) occupy [head, tail),
+            // or [head, HA) and [0, tail) once wrapped
+            int g_old = 0, head = 0, tail = 0;
+            bool wrapped = false;
             int ngroups = has_shared;  // the routed groups are added once the plan is known
             bool have_plan = false;
             bool stop = false;
@@ -841,23 +854,55 @@ __global__ void __launch_bounds__(kDownThreads, 1) stream_down_fold_kernel(const
                             grid_dependency_wait();
                             waited = true;
                         }
-                        // group gi uses buffer gi % NH, free once group gi - NH is done
-                        const int hb = gi % NH;
-                        if (gi >= NH &&
-                            !mbar_wait(&hempty[hb], (uint32_t)(gi / NH - 1) & 1u, abort_flag)) {
-                            stop = true;
-                            break;
+                        // a contiguous place in the arena, freeing the oldest
+                        // groups (in order) until one exists
+                        const int need = (int)((hbytes / 4 + 31) & ~31u);
+                        int off = -1;
+                        for (;;) {
+                            if (g_old == gi) {
+                                head = tail = 0;
+                                wrapped = false;
+                            }
+                            if (gi - g_old < HK) {
+                                if (!wrapped) {
+                                    if (tail + need <= HA) {
+                                        off = tail;
+                                    } else if (need <= head) {
+                                        off = 0;
+                                        wrapped = true;
+                                    }
+                                } else if (tail + need <= head) {
+                                    off = tail;
+                                }
+                                if (off >= 0)
+                                    break;
+                            }
+                            if (!mbar_wait(&hempty[g_old % HK], (uint32_t)(g_old / HK) & 1u,
+                                           abort_flag)) {
+                                stop = true;
+                                break;
+                            }
+                            ++g_old;
+                            if (g_old < gi) {
+                                head = hoff[g_old % HK];
+                                wrapped = head >= tail;
+                            }
                         }
+                        if (stop)
+                            break;
+                        tail = off + need;
+                        const int hb = gi % HK;
+                        hoff[hb] = off;
                         mbar_arrive_expect_tx(&hfull[hb], hbytes);
-                        bulk_g2s(hbuf + (size_t)hb * h_elems, hsrc, hbytes, &hfull[hb], pol_h);
+                        bulk_g2s(hbuf + off, hsrc, hbytes, &hfull[hb], pol_h);
                         ++h_issued;
                     }
                 }
             }
             for (int n = issued > NS ? issued - NS : 0; n < issued; ++n)
                 mbar_wait(&full[n % NS], (uint32_t)(n / NS) & 1u, nullptr);
-            for (int n = h_issued > NH ? h_issued - NH : 0; n < h_issued; ++n)
-                mbar_wait(&hfull[n % NH], (uint32_t)(n / NH) & 1u, nullptr);
+            for (int n = h_issued > HK ? h_issued - HK : 0; n < h_issued; ++n)
+                mbar_wait(&hfull[n % HK], (uint32_t)(n / HK) & 1u, nullptr);
         }
     } else {
         const int ltid = (int)threadIdx.x - 32;
@@ -897,10 +942,10 @@ __global__ void __launch_bounds__(kDownThreads, 1) stream_down_fold_kernel(const
                 g.first = P.group_first[grp];
                 g.cnt = P.group_first[grp + 1] - g.first;
             }
-            g.hg = hbuf + (size_t)(gi % NH) * h_elems;
-            g.hempty = &hempty[gi % NH];
-            if (!mbar_wait(&hfull[gi % NH], (uint32_t)(gi / NH) & 1u, abort_flag))
+            if (!mbar_wait(&hfull[gi % HK], (uint32_t)(gi / HK) & 1u, abort_flag))
                 break;
+            g.hg = hbuf + hoff[gi % HK];
+            g.hempty = &hempty[gi % HK];
             if (!down_group(g))
                 break;
         }
