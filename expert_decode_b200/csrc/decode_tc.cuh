@@ -1,0 +1,310 @@
+// decode_tc.cuh -- gate/up of the weight-streaming (decode) path on the
+// tensor cores.
+//
+// Same contraction as stream_gate_up_kernel (h = silu(W_gate x) * (W_up x)
+// for every picked expert and the shared expert; fak note "GLM-5.2
+// multi-GPU", expertSwiGLU), laid out for tcgen05: a tile is 64 units of I,
+// i.e. 128 weight rows on the MMA's M side with 16 W_gate rows and 16 W_up
+// rows interleaved (TensorFold #593's packGateUp), and all T <= 8 tokens on
+// its N side (N = 16; the tensor map zero-fills the rows after T).  Every
+// tile therefore computes every token, and the epilogue keeps the tokens
+// that picked the tile's expert, so no activation gather is needed.
+//
+// Persistent and warp specialised, one CTA per SM:
+//   warp 0     TMA producer: per 64-wide k block the A tile (8 boxes of 16
+//              weight rows, 16 KB) and the x tile (16 rows, 2 KB) into a
+//              ring of kTcStages stages, 128-byte swizzle, no multicast;
+//   warp 1     tcgen05.mma issuer (M = 128, N = 16, K = 16 per instruction),
+//              fp32 accumulators in TMEM, two of them so that the epilogue
+//              of one tile overlaps the MMAs of the next;
+//   warps 2-5  build the expert grouping from ids (the streaming plan), then
+//              drain each accumulator with tcgen05.ld: lanes l and l + 16 of a
+//              warp hold g and u of the same unit, h = silu(g) * u is written
+//              in fp32, in the layout the down kernel reads.
+// Tiles go round-robin over the CTAs: the shared expert's first, then each
+// routed group's in ascending expert id.
+#pragma once
+
+#include "common.cuh"
+#include "grouped.cuh"
+#include "streaming.cuh"
+
+namespace epk {
+
+constexpr int kTcN = 16;                                   // MMA N: tokens, zero rows after T
+constexpr int kTcStages = 10;
+constexpr int kTcThreads = 192;
+constexpr uint32_t kTcABytes = kGemmBM * kGemmBK * 2;      // 64 gate + 64 up rows, 16 KB
+constexpr uint32_t kTcBBytes = kTcN * kGemmBK * 2;         // 16 token rows, 2 KB
+constexpr uint32_t kTcStageBytes = kTcABytes + kTcBBytes;  // 18 KB, a multiple of 1024
+constexpr int kTcTmemCols = 2 * kTcN;                      // two accumulators
+constexpr uint32_t kTcBarPlan = 1;                         // named barrier of the epilogue warps
+constexpr int kTcMaxGroups = kStreamMaxPairs + 1;          // routed groups + the shared expert
+
+struct TcMaps {
+    CUtensorMap wg, wu;  // W_gate, W_up [E, I, H]: box 64 x 16 x 1
+    CUtensorMap sg, su;  // shared expert [I_s, H]: box 64 x 16
+    CUtensorMap x;       // activations [T, H]: box 64 x 16
+};
+
+struct TcArgs {
+    int T, H, E, I, I_s, top_k;
+    const int32_t *ids;
+    const float *weights;
+    float *h_routed;  // [pairs, I] in plan order
+    float *h_shared;  // [T, I_s]
+};
+
+struct TcSmem {
+    static constexpr uint32_t stages = 0;
+    static constexpr uint32_t bars = kTcStages * kTcStageBytes;
+    // full[S], empty[S], tfull[2], tempty[2], drain, planbar; tmem holder, abort flag
+    static constexpr uint32_t misc = bars + (2 * kTcStages + 6) * 8;
+    static constexpr uint32_t tile_first = misc + 16;  // [kTcMaxGroups + 1]
+    static constexpr uint32_t plan = (tile_first + (kTcMaxGroups + 1) * 4 + 127) / 128 * 128;
+    static constexpr uint32_t total = plan + (uint32_t)sizeof(StreamPlan);
+    static constexpr uint32_t alloc = total + 1024;  // room to align the base to 1024
+};
+
+__device__ __forceinline__ void tmem_load_16cols(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1)
+stream_gate_up_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + TcSmem::bars);
+    uint64_t *empty = full + kTcStages;
+    uint64_t *tfull = empty + kTcStages;
+    uint64_t *tempty = tfull + 2;
+    uint64_t *drain = tempty + 2;
+    uint64_t *planbar = drain + 1;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + TcSmem::misc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + TcSmem::misc + 8);
+    int *tile_first = reinterpret_cast<int *>(smem + TcSmem::tile_first);
+    StreamPlan &P = *reinterpret_cast<StreamPlan *>(smem + TcSmem::plan);
+
+    const int warp = (int)(threadIdx.x >> 5);
+    const int lane = (int)lane_id();
+    const int has_shared = a.I_s > 0 ? 1 : 0;
+
+    if (warp == 0 && lane == 0) {
+        for (int s = 0; s < kTcStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 4);
+        }
+        mbar_init(drain, 1);
+        mbar_init(planbar, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tensormap(&maps.wg);
+        prefetch_tensormap(&maps.wu);
+        prefetch_tensormap(&maps.x);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, kTcTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    grid_dependents_launch();
+    const uint32_t tmem_base = *tmem_holder;
+
+    // tile u -> (group index gi, first unit m0); gi = 0 is the shared expert
+    // when there is one
+    auto decode = [&](int u, int &gi, int &m0) {
+        const int G = has_shared + P.n_groups;
+        int lo = 0, hi = G - 1;
+        while (lo < hi) {  // largest gi with tile_first[gi] <= u
+            const int mid = (lo + hi + 1) >> 1;
+            if (tile_first[mid] <= u)
+                lo = mid;
+            else
+                hi = mid - 1;
+        }
+        gi = lo;
+        m0 = (u - tile_first[gi]) * kGateUpRows;
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer
+        if (elect_one()) {
+            const uint64_t pol_w = policy_evict_first();
+            const uint64_t pol_x = policy_evict_last();
+            grid_dependency_wait();  // x may come from the previous kernel
+            uint32_t stage = 0, phase = 0;
+            int issued = 0;
+            bool stop = !mbar_wait(planbar, 0, abort_flag);
+            const int total = stop ? 0 : tile_first[has_shared + P.n_groups];
+            const int kblocks = (a.H + kGemmBK - 1) / kGemmBK;
+            for (int u = blockIdx.x; u < total && !stop; u += gridDim.x) {
+                int gi, m0;
+                decode(u, gi, m0);
+                const bool shared = gi < has_shared;
+                const int e = shared ? 0 : (int)P.group_expert[gi - has_shared];
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+                        stop = true;
+                        break;
+                    }
+                    uint8_t *sa = smem + stage * kTcStageBytes;
+                    uint8_t *sb = sa + kTcABytes;
+                    mbar_arrive_expect_tx(&full[stage], kTcStageBytes);
+                    const int k0 = kb * kGemmBK;
+#pragma unroll
+                    for (int j = 0; j < kGemmBM / kBoxRowsA; ++j) {
+                        const bool up = j & 1;
+                        const int row = m0 + (j >> 1) * kBoxRowsA;
+                        uint8_t *dst = sa + j * kBoxRowsA * kGemmBK * 2;
+                        if (shared)
+                            tma_load_2d(dst, up ? &maps.su : &maps.sg, k0, row, &full[stage], pol_w);
+                        else
+                            tma_load_3d(dst, up ? &maps.wu : &maps.wg, k0, row, e, &full[stage],
+                                        pol_w);
+                    }
+                    tma_load_2d(sb, &maps.x, k0, 0, &full[stage], pol_x);
+                    ++issued;
+                    if (++stage == kTcStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // no copy may still be landing in shared memory when the CTA exits
+            for (int n = issued > kTcStages ? issued - kTcStages : 0; n < issued; ++n)
+                mbar_wait(&full[n % kTcStages], (uint32_t)(n / kTcStages) & 1u, nullptr);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer
+        if (elect_one()) {
+            uint32_t stage = 0, phase = 0;
+            uint32_t acc = 0, acc_phase = 0;
+            bool stop = !mbar_wait(planbar, 0, abort_flag);
+            const int total = stop ? 0 : tile_first[has_shared + P.n_groups];
+            const int kblocks = (a.H + kGemmBK - 1) / kGemmBK;
+            const uint32_t idesc = idesc_bf16_f32(kGemmBM, kTcN);
+            for (int u = blockIdx.x; u < total && !stop; u += gridDim.x) {
+                if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag))
+                    break;
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem_base + acc * kTcN;
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, abort_flag)) {
+                        stop = true;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t a_addr = smem_u32(smem + stage * kTcStageBytes);
+                    const uint32_t b_addr = a_addr + kTcABytes;
+#pragma unroll
+                    for (int kk = 0; kk < kGemmBK / 16; ++kk)
+                        umma_bf16(d_tmem, smem_desc_sw128_kmajor(a_addr + kk * 32),
+                                  smem_desc_sw128_kmajor(b_addr + kk * 32), idesc,
+                                  (kb > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(&empty[stage]);  // frees the stage once these MMAs are done
+                    if (++stage == kTcStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (stop)
+                    break;
+                umma_commit(&tfull[acc]);
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+            // every MMA issued by this thread has completed before TMEM is freed
+            umma_commit(drain);
+            mbar_wait(drain, 0, nullptr);
+        }
+    } else {
+        // ------------------------------------------------ plan, then epilogue
+        const int ltid = (int)threadIdx.x - 64;
+        grid_dependency_wait();  // ids and weights may come from the previous kernel
+        build_stream_plan(P, a.ids, a.weights, a.T, a.top_k, a.E, ltid, 128, kTcBarPlan);
+        if (ltid == 0) {
+            const int G = has_shared + P.n_groups;
+            int t = 0;
+            for (int gi = 0; gi < G; ++gi) {
+                tile_first[gi] = t;
+                const int width = gi < has_shared ? a.I_s : a.I;
+                t += (width + kGateUpRows - 1) / kGateUpRows;
+            }
+            tile_first[G] = t;
+            mbar_arrive(planbar);  // release: the plan and the tile table are written
+        }
+        if (mbar_wait(planbar, 0, abort_flag)) {
+            const int q = warp & 3;  // TMEM lane quarter this warp may access
+            const int total = tile_first[has_shared + P.n_groups];
+            uint32_t acc = 0, acc_phase = 0;
+            for (int u = blockIdx.x; u < total; u += gridDim.x) {
+                int gi, m0;
+                decode(u, gi, m0);
+                const bool shared = gi < has_shared;
+                if (!mbar_wait(&tfull[acc], acc_phase, abort_flag))
+                    break;
+                tc_fence_after_sync();
+                uint32_t v[16];
+                tmem_load_16cols(tmem_base + ((uint32_t)(32 * q) << 16) + acc * kTcN, v);
+                tmem_load_wait();
+                // lanes 0..15 hold gate rows, 16..31 the up rows of the same units
+                const int unit = m0 + 16 * q + (lane & 15);
+                const bool is_gate = lane < 16;
+                if (shared) {
+#pragma unroll
+                    for (int t = 0; t < kStreamMaxT; ++t) {
+                        const float other = __shfl_xor_sync(0xffffffffu, __uint_as_float(v[t]), 16);
+                        if (is_gate && t < a.T && unit < a.I_s)
+                            a.h_shared[(size_t)t * a.I_s + unit] =
+                                silu_f32(__uint_as_float(v[t])) * other;
+                    }
+                } else {
+                    const int g = gi - has_shared;
+                    const int first = P.group_first[g];
+                    const int cnt = P.group_first[g + 1] - first;
+                    for (int j = 0; j < cnt; ++j) {
+                        const int tok = P.pair_token[first + j];
+                        float mine = 0.f;
+#pragma unroll
+                        for (int t = 0; t < kStreamMaxT; ++t)
+                            mine = t == tok ? __uint_as_float(v[t]) : mine;
+                        const float other = __shfl_xor_sync(0xffffffffu, mine, 16);
+                        if (is_gate && unit < a.I)
+                            a.h_routed[(size_t)(first + j) * a.I + unit] = silu_f32(mine) * other;
+                    }
+                }
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&tempty[acc]);
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem_base, kTcTmemCols);
+    }
+}
+
+}  // namespace epk

@@ -17,6 +17,7 @@
 #include "router.cuh"
 #include "streaming.cuh"
 #include "grouped.cuh"
+#include "decode_tc.cuh"
 
 namespace {
 
@@ -153,6 +154,8 @@ ep_status device_info(const DeviceInfo **out) {
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, m));
         EP_CUDA_CHECK(cudaFuncSetAttribute(epk::stream_down_fold_kernel,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, m));
+        EP_CUDA_CHECK(cudaFuncSetAttribute(epk::stream_gate_up_tc_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, m));
         ep_status s = epk::grouped_set_attributes(m);
         if (s != EP_OK)
             return fail(s, "setting the grouped GEMM kernel attributes failed");
@@ -168,6 +171,8 @@ constexpr int64_t kMaxH = 16384;
 constexpr int64_t kMaxE = 1024;
 constexpr int64_t kMaxI = 16384;
 constexpr int kMaxTopK = 16;
+// the decode path's gate/up runs on the tensor cores from this many tokens
+constexpr int64_t kTcMinT = 2;
 // moe_route computes every logit by Dot2 up to this many tokens
 constexpr int64_t kRouterDot2MaxT = 32;
 // Shared memory the streaming kernels may take, leaving the rest of the
@@ -284,7 +289,7 @@ extern "C" ep_status ep_plan(int32_t num_experts, int32_t bands, ep_plan_t *out)
 }
 
 extern "C" ep_status ep_set_dispatch(ep_dispatch mode) {
-    if (mode != EP_DISPATCH_AUTO && mode != EP_DISPATCH_STREAMING && mode != EP_DISPATCH_TENSOR)
+    if ((int)mode < (int)EP_DISPATCH_AUTO || (int)mode > (int)EP_DISPATCH_STREAMING_SIMT)
         return fail(EP_EINVAL, "ep_set_dispatch: unknown mode %d", (int)mode);
     g_dispatch.store((int)mode);
     return ok();
@@ -478,7 +483,8 @@ extern "C" ep_status moe_ffn_forward(const void *x, ep_dtype x_dtype, int64_t T,
     const StreamingPlan sp = streaming_fit(*d, T, H, xb, top_k, I, I_s);
     const int mode = g_dispatch.load();
     bool use_streaming;
-    if (mode == EP_DISPATCH_STREAMING) {
+    if (mode == EP_DISPATCH_STREAMING || mode == EP_DISPATCH_STREAMING_TC ||
+        mode == EP_DISPATCH_STREAMING_SIMT) {
         if (!sp.fits)
             return fail(EP_EINVAL, "moe_ffn_forward: the streaming path does not fit these sizes");
         use_streaming = true;
@@ -504,7 +510,41 @@ extern "C" ep_status moe_ffn_forward(const void *x, ep_dtype x_dtype, int64_t T,
         ga.h_routed = reinterpret_cast<float *>(ws + W.h_routed);
         ga.h_shared = reinterpret_cast<float *>(ws + W.h_shared);
         const dim3 gu_grid((unsigned)d->sm_count);
-        {
+        // gate/up on the tensor cores needs bf16 activations and the tensor
+        // maps; by default it takes over from 2 tokens on
+        epk::TcMaps tm;
+        memset(&tm, 0, sizeof tm);
+        bool tc_ok = x_dtype == EP_BF16 && epk::TcSmem::alloc <= (uint32_t)d->smem_optin &&
+                     epk::tensor_map_encoder() != nullptr;
+        if (tc_ok && mode != EP_DISPATCH_STREAMING_SIMT &&
+            (mode == EP_DISPATCH_STREAMING_TC || T >= kTcMinT)) {
+            tc_ok = epk::map_3d(&tm.wg, w_gate, H, I, E, epk::kBoxRowsA) &&
+                    epk::map_3d(&tm.wu, w_up, H, I, E, epk::kBoxRowsA) &&
+                    epk::map_2d(&tm.x, x, H, T, epk::kTcN);
+            if (I_s > 0)
+                tc_ok = tc_ok && epk::map_2d(&tm.sg, ws_gate, H, I_s, epk::kBoxRowsA) &&
+                        epk::map_2d(&tm.su, ws_up, H, I_s, epk::kBoxRowsA);
+        }
+        bool use_tc;
+        if (mode == EP_DISPATCH_STREAMING_TC) {
+            if (!tc_ok)
+                return fail(EP_EINVAL, "moe_ffn_forward: tensor-core gate/up needs bf16 x");
+            use_tc = true;
+        } else {
+            use_tc = tc_ok && mode != EP_DISPATCH_STREAMING_SIMT && T >= kTcMinT;
+        }
+        if (use_tc) {
+            epk::TcArgs ta;
+            ta.T = (int)T; ta.H = (int)H; ta.E = (int)E; ta.I = (int)I; ta.I_s = (int)I_s;
+            ta.top_k = top_k;
+            ta.ids = ids;
+            ta.weights = weights;
+            ta.h_routed = ga.h_routed;
+            ta.h_shared = ga.h_shared;
+            KernelBracket kb0(st, 0);
+            EP_CUDA_CHECK(launch(epk::stream_gate_up_tc_kernel, gu_grid, epk::kTcThreads,
+                                 epk::TcSmem::alloc, st, tm, ta));
+        } else {
             KernelBracket kb0(st, 0);
             if (x_dtype == EP_F32)
                 EP_CUDA_CHECK(launch(epk::stream_gate_up_kernel<true, true>, gu_grid,

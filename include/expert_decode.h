@@ -185,7 +185,13 @@ ep_status moe_ffn_forward_noalloc(const void *x, ep_dtype x_dtype, int64_t T, in
  * tensor-core path.  Forcing a path that does not fit the sizes makes
  * moe_ffn_forward return EP_EINVAL.  Process-wide; meant for tests and tuning.
  */
-typedef enum { EP_DISPATCH_AUTO = 0, EP_DISPATCH_STREAMING = 1, EP_DISPATCH_TENSOR = 2 } ep_dispatch;
+typedef enum {
+    EP_DISPATCH_AUTO = 0,
+    EP_DISPATCH_STREAMING = 1,      /* streaming path, gate/up kernel chosen as in AUTO */
+    EP_DISPATCH_TENSOR = 2,
+    EP_DISPATCH_STREAMING_TC = 3,   /* streaming path, gate/up on the tensor cores (bf16 x) */
+    EP_DISPATCH_STREAMING_SIMT = 4  /* streaming path, gate/up on the CUDA cores */
+} ep_dispatch;
 ep_status ep_set_dispatch(ep_dispatch mode);
 
 /*

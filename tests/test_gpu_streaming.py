@@ -1,5 +1,7 @@
 """The weight-streaming path (T <= 8) of moe_ffn_forward against the fp64 oracle,
-with the bit-identity the method promises: across runs and across band counts."""
+with the bit-identity the method promises: across runs and across band counts.
+Every test runs twice: gate/up on the CUDA cores and on the tensor cores (the
+latter takes bf16 activations only)."""
 import numpy as np
 import pytest
 import torch
@@ -12,11 +14,20 @@ pytestmark = pytest.mark.gpu
 WL = workloads.WORKLOADS
 
 
-@pytest.fixture(autouse=True)
-def streaming_dispatch():
-    ed.ep_set_dispatch("streaming")
-    yield
+# the tiny workload with bf16 activations, for the tensor-core gate/up
+TINY_BF16 = workloads.Workload("tiny_bf16", (4,), 256, 16, 4, 128, 128, "bf16", "none", (1, 2, 4))
+
+
+@pytest.fixture(autouse=True, params=["streaming_simt", "streaming_tc"])
+def gate_up(request):
+    ed.ep_set_dispatch(request.param)
+    yield request.param
     ed.ep_set_dispatch("auto")
+
+
+def _activations_supported(gate_up, x_dtype):
+    if gate_up == "streaming_tc" and x_dtype != "bf16":
+        pytest.skip("the tensor-core gate/up takes bf16 activations")
 
 
 def _routed(o, wl, T, seed=workloads.SEED_BASE, batch=0, **sizes):
@@ -27,8 +38,9 @@ def _routed(o, wl, T, seed=workloads.SEED_BASE, batch=0, **sizes):
     return W, x, ids, w
 
 
-def test_tiny_all_band_counts(oracle_lib):
-    wl = WL["tiny"]
+@pytest.mark.parametrize("wl", [WL["tiny"], TINY_BF16], ids=["fp32_x", "bf16_x"])
+def test_tiny_all_band_counts(oracle_lib, gate_up, wl):
+    _activations_supported(gate_up, wl.x_dtype)
     W, x, ids, w = _routed(oracle_lib, wl, 4)
     ys = {}
     for R in wl.bands + (8, 16):
@@ -80,7 +92,8 @@ def test_odd_sizes_and_max_pairs(oracle_lib):
 # H = 6144 with fp32 x at T = 4 leaves 4 slots of 24 KB.
 @pytest.mark.parametrize("T,H,x_dtype", [(8, 8192, "bf16"), (2, 8192, "bf16"),
                                          (4, 6144, "f32")])
-def test_wide_rows_few_gate_up_slots(oracle_lib, T, H, x_dtype):
+def test_wide_rows_few_gate_up_slots(oracle_lib, gate_up, T, H, x_dtype):
+    _activations_supported(gate_up, x_dtype)
     wl = workloads.Workload("wide", (T,), H, 16, 4, 256, 128, x_dtype, "none", (1,))
     W, x, ids, w = _routed(oracle_lib, wl, T, seed=31 + T)
     y = gpu_ffn(x, ids, w, W, ed.ep_plan(wl.E, 4))
@@ -101,8 +114,9 @@ def test_no_shared_expert(oracle_lib):
     check_y(y, oracle_ffn(oracle_lib, x, ids, w, W), rel_tol=1e-4, what="imbalanced, small")
 
 
-def test_repeated_expert_in_one_token(oracle_lib):
-    wl = WL["tiny"]
+@pytest.mark.parametrize("wl", [WL["tiny"], TINY_BF16], ids=["fp32_x", "bf16_x"])
+def test_repeated_expert_in_one_token(oracle_lib, gate_up, wl):
+    _activations_supported(gate_up, wl.x_dtype)
     W, x, ids, w = _routed(oracle_lib, wl, 4, seed=8)
     ids[1, 2] = ids[1, 0]          # token 1 picks one expert twice
     ids[3, :] = ids[3, 1]          # token 3 picks one expert four times
@@ -110,8 +124,9 @@ def test_repeated_expert_in_one_token(oracle_lib):
     check_y(y, oracle_ffn(oracle_lib, x, ids, w, W), rel_tol=1e-4, what="repeated picks")
 
 
-def test_bad_ids_are_skipped_and_reported(oracle_lib):
-    wl = WL["tiny"]
+@pytest.mark.parametrize("wl", [WL["tiny"], TINY_BF16], ids=["fp32_x", "bf16_x"])
+def test_bad_ids_are_skipped_and_reported(oracle_lib, gate_up, wl):
+    _activations_supported(gate_up, wl.x_dtype)
     W, x, ids, w = _routed(oracle_lib, wl, 4, seed=12)
     ed.ep_check_status()
     bad = ids.clone()
