@@ -147,6 +147,7 @@ class Layer:
                  for T in wl.T)
         self.workspace = torch.empty(ws, dtype=torch.uint8, device=device)
         self.launches = 0
+        self.ffn_kernels = {}  # kernels of the last forward call per row count
 
     def call(self, T, b, x=None):
         ed = self.ed
@@ -161,7 +162,9 @@ class Layer:
         ed.moe_ffn_forward(x, self.ids[T], self.wts[T], self.W["w_gate"], self.W["w_up"],
                            self.W["w_down"], self.shared, self.plan,
                            y=self.y[T] if y is None else y, workspace=self.workspace)
-        self.launches += ed.ep_last_launch_count()
+        n = ed.ep_last_launch_count()
+        self.launches += n
+        self.ffn_kernels[T] = n
 
     def distinct_experts(self, T, b):
         self.call(T, b)
@@ -431,8 +434,12 @@ def run_ours(args, wl):
         per_T[f"T={T}"] = {"dominant_kernel_us": 1e6 * sum(durs) / K,
                            "dominant_kernel_GBps": byts / sum(durs) / 1e9}
         # mean duration of every kernel of the route and forward calls
-        names = (["plan", "gather", "gate_up", "down", "combine"] if tensor_path[T]
-                 else ["gate_up", "down_fold"])
+        if tensor_path[T]:
+            names = ["plan", "gather", "gate_up", "down", "combine"]
+        elif layer.ffn_kernels.get(T) == 3:
+            names = ["gate_up", "down", "fold"]
+        else:
+            names = ["gate_up", "down_fold"]
         kus = {}
         for j, name in enumerate(names):
             kus[name] = 1e3 * sum(prof[i][T][2 * j].elapsed_time(prof[i][T][2 * j + 1])

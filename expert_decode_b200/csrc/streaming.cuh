@@ -906,14 +906,14 @@ __global__ void __launch_bounds__(kDownThreads, 1) stream_down_fold_kernel(const
         }
     } else {
         const int ltid = (int)threadIdx.x - 32;
-        // The only kernel that can still be running is this call's gate/up
-        // kernel, which writes h alone: ids and weights may be read before
-        // griddepcontrol.wait, so the plan is built while it finishes.
+        // ids and weights are read only after griddepcontrol.wait: the
+        // gate/up kernel lets this one start early, possibly while the kernel
+        // that wrote the ids (the router) is still running
+        grid_dependency_wait();
         build_stream_plan(P, a.ids, a.weights, a.T, a.top_k, a.E, ltid, 32 * kDownConsumerWarps,
                           kDownBarPlan);
         if (ltid == 0)
             mbar_arrive(planbar);
-        grid_dependency_wait();
         DownGroup g;
         g.P = &P;
         g.slots = slots;

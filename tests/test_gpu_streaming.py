@@ -1,7 +1,7 @@
 """The weight-streaming path (T <= 8) of moe_ffn_forward against the fp64 oracle,
 with the bit-identity the method promises: across runs and across band counts.
-Every test runs twice: gate/up on the CUDA cores and on the tensor cores (the
-latter takes bf16 activations only)."""
+Every test runs with the gate/up projection on the CUDA cores, on the tensor
+cores (bf16 activations only), and with the default choice of kernel."""
 import numpy as np
 import pytest
 import torch
@@ -18,7 +18,11 @@ WL = workloads.WORKLOADS
 TINY_BF16 = workloads.Workload("tiny_bf16", (4,), 256, 16, 4, 128, 128, "bf16", "none", (1, 2, 4))
 
 
-@pytest.fixture(autouse=True, params=["streaming_simt", "streaming_tc"])
+# streaming_simt: gate/up on the CUDA cores; streaming_tc: gate/up on the
+# tensor cores (bf16 activations only); streaming: the default choice (tensor
+# cores from 2 tokens with bf16 activations).  The down projection and its
+# fold run on the CUDA cores in every case.
+@pytest.fixture(autouse=True, params=["streaming_simt", "streaming_tc", "streaming"])
 def gate_up(request):
     ed.ep_set_dispatch(request.param)
     yield request.param
@@ -142,6 +146,22 @@ def test_bad_ids_are_skipped_and_reported(oracle_lib, gate_up, wl):
     ref_w[0, 1] = 0.0
     ref_w[2, 3] = 0.0
     check_y(y, oracle_ffn(oracle_lib, x, ref_ids, ref_w, W), rel_tol=1e-4, what="bad ids")
+
+
+def test_all_ids_bad_without_shared_expert_gives_zero(oracle_lib, gate_up):
+    """No valid pick and no shared expert: y = 0 (nothing folds a row)."""
+    wl = workloads.Workload("noshared", (4,), 256, 16, 4, 128, 0, "bf16", "none", (1,))
+    W, x = device_inputs(wl, 4, seed=3)
+    ids = torch.full((4, wl.top_k), wl.E + 3, dtype=torch.int32, device="cuda")
+    w = torch.full((4, wl.top_k), 0.25, dtype=torch.float32, device="cuda")
+    y = torch.full((4, wl.H), float("nan"), dtype=torch.float32, device="cuda")
+    ed.moe_ffn_forward(x, ids, w, W["w_gate"], W["w_up"], W["w_down"], None,
+                       ed.ep_plan(wl.E, 1), y=y)
+    torch.cuda.synchronize()
+    with pytest.raises(ed.EPError) as ei:
+        ed.ep_check_status()
+    assert ei.value.code == ed.EP_EBADID
+    assert torch.count_nonzero(y).item() == 0
 
 
 def test_empty_batch_is_a_no_op():
