@@ -189,6 +189,83 @@ int oracle_route(const void *x, int x_is_f32, int64_t T, int64_t H,
     return status;
 }
 
+/*
+ * The GLM router variant [GATE page, a contributor's comment "What exists
+ * now": glm_route.cu, "sigmoid + bias top-k, raw-score weights"].  The page
+ * names only the three ingredients; they are read here as:
+ *   l_e = sum_h x[t,h] * W_r[e,h]          (sequential over h, no bias)
+ *   s_e = 1 / (1 + exp(-l_e))              the expert's score
+ *   k_e = s_e + b_e                        the bias moves the selection only
+ *   S   = the top_k experts by key, ties to the lower id
+ *   w_j = scale * s_{S_j}                  the raw score (normalize = 0), or
+ *   w_j = scale * s_{S_j} / sum_{e in S} s_e  (normalize = 1)
+ * ids[t, j] and weights[t, j] are written in the order of S (descending key,
+ * equal keys by ascending id).  keys and scores (optional) receive k and s,
+ * [T][E].
+ */
+int oracle_route_sigmoid(const void *x, int x_is_f32, int64_t T, int64_t H,
+                         const uint16_t *w_router, const double *bias, int64_t E,
+                         int32_t top_k, int normalize, double scale, int32_t *ids,
+                         double *weights, double *keys, double *scores, int nthreads)
+{
+    if (T < 0 || H < 1 || E < 1 || top_k < 1 || top_k > E)
+        return ORACLE_EINVAL;
+    if (T == 0)
+        return ORACLE_OK;
+    if (x == NULL || w_router == NULL || ids == NULL || weights == NULL)
+        return ORACLE_EINVAL;
+    int status = ORACLE_OK;
+#ifdef _OPENMP
+    if (nthreads < 1)
+        nthreads = 1;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+#endif
+    for (int64_t t = 0; t < T; ++t) {
+        double *sc = (double *)malloc(sizeof(double) * (size_t)E);
+        double *key = (double *)malloc(sizeof(double) * (size_t)E);
+        int32_t *order = (int32_t *)malloc(sizeof(int32_t) * (size_t)E);
+        if (sc == NULL || key == NULL || order == NULL) {
+            free(sc); free(key); free(order);
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+            status = ORACLE_EINVAL;
+            continue;
+        }
+        for (int64_t e = 0; e < E; ++e) {
+            double l = 0.0;
+            for (int64_t h = 0; h < H; ++h)
+                l += activation_value(x, x_is_f32, t * H + h) * bf16_value(w_router[e * H + h]);
+            sc[e] = 1.0 / (1.0 + exp(-l));
+            key[e] = bias != NULL ? sc[e] + bias[e] : sc[e];
+        }
+        /* full order of the experts by (key desc, id asc): insertion sort */
+        for (int64_t e = 0; e < E; ++e) {
+            int64_t pos = e;
+            while (pos > 0 && ranks_before(key[e], (int32_t)e, key[order[pos - 1]], order[pos - 1])) {
+                order[pos] = order[pos - 1];
+                --pos;
+            }
+            order[pos] = (int32_t)e;
+        }
+        double sum = 0.0;
+        for (int32_t j = 0; j < top_k; ++j)
+            sum += sc[order[j]];
+        for (int32_t j = 0; j < top_k; ++j) {
+            ids[t * top_k + j] = order[j];
+            weights[t * top_k + j] = normalize ? scale * (sc[order[j]] / sum) : scale * sc[order[j]];
+        }
+        for (int64_t e = 0; e < E; ++e) {
+            if (keys != NULL)
+                keys[t * E + e] = key[e];
+            if (scores != NULL)
+                scores[t * E + e] = sc[e];
+        }
+        free(sc); free(key); free(order);
+    }
+    return status;
+}
+
 /* ------------------------------------------------------------------------ */
 /* One SwiGLU expert.                                                         */
 /* ------------------------------------------------------------------------ */

@@ -43,12 +43,15 @@ class Oracle:
         lib = ctypes.CDLL(path)
         lib.oracle_expert_parallel_plan.argtypes = [_I64, _I64, _I32, _P]
         lib.oracle_route.argtypes = [_P, _INT, _I64, _I64, _P, _P, _I64, _I32, _P, _P, _P, _INT]
+        lib.oracle_route_sigmoid.argtypes = [_P, _INT, _I64, _I64, _P, _P, _I64, _I32, _INT,
+                                             ctypes.c_double, _P, _P, _P, _P, _INT]
         lib.oracle_expert_swiglu.argtypes = [_P, _P, _P, _P, _I64, _I64, _P]
         common = [_P, _INT, _I64, _I64, _P, _P, _I32, _P, _P, _P, _I64, _I64, _P, _P, _P, _I64]
         lib.oracle_moe_ffn_monolith.argtypes = common + [_P, _INT]
         lib.oracle_moe_ffn_expert_parallel.argtypes = common + [_P, _I32, _P, _INT]
         lib.oracle_max_threads.argtypes = []
-        for fn in ("oracle_expert_parallel_plan", "oracle_route", "oracle_expert_swiglu",
+        for fn in ("oracle_expert_parallel_plan", "oracle_route", "oracle_route_sigmoid",
+                   "oracle_expert_swiglu",
                    "oracle_moe_ffn_monolith", "oracle_moe_ffn_expert_parallel",
                    "oracle_max_threads"):
             getattr(lib, fn).restype = ctypes.c_int
@@ -87,6 +90,26 @@ class Oracle:
         if rc != OK:
             raise OracleError(rc, "route")
         return ids, weights, logits
+
+    def route_sigmoid(self, x, w_router, bias, top_k, normalize=False, scale=1.0, threads=None):
+        """The sigmoid router variant: ids, weights, keys (s + b), scores (s)."""
+        x, is_f32 = self._activations(x)
+        T, H = x.shape
+        w_router = np.ascontiguousarray(w_router, dtype=np.uint16)
+        E = w_router.shape[0]
+        assert w_router.shape == (E, H)
+        b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float64)
+        ids = np.zeros((T, top_k), dtype=np.int32)
+        weights = np.zeros((T, top_k), dtype=np.float64)
+        keys = np.zeros((T, E), dtype=np.float64)
+        scores = np.zeros((T, E), dtype=np.float64)
+        rc = self.lib.oracle_route_sigmoid(_ptr(x), is_f32, T, H, _ptr(w_router), _ptr(b), E,
+                                           int(top_k), 1 if normalize else 0, float(scale),
+                                           _ptr(ids), _ptr(weights), _ptr(keys), _ptr(scores),
+                                           self._threads(threads))
+        if rc != OK:
+            raise OracleError(rc, "route_sigmoid")
+        return ids, weights, keys, scores
 
     # -- experts ------------------------------------------------------------
     def expert_swiglu(self, xt, w_gate, w_up, w_down):

@@ -10,6 +10,10 @@ What pins what:
   router          exact rational brute force on tiny inputs; closed forms
                   (large logits, top_k = 1, ties, all-equal, Zipf skew);
                   top_k = E against torch.softmax in float64
+  sigmoid router  closed forms (golden/router_sigmoid_closed_forms.json);
+                  without a bias its picks are the softmax router's (the
+                  sigmoid is increasing); its scores against torch.sigmoid of
+                  the pinned fp64 logits
   expert          a hand-derived 2x2 SwiGLU (golden/swiglu_hand.json); E = 1,
                   top_k = 1 against a dense SwiGLU from torch.nn.functional
   fold / bands    exact IEEE folds where the order shows (golden/fold_order.json);
@@ -160,6 +164,43 @@ def _hand_expert():
             exact_bf16_bits(g["w_down"]))
 
 
+def pin_router_sigmoid_closed_forms(o):
+    g = golden("router_sigmoid_closed_forms.json")
+    for case in g["cases"]:
+        E = len(case["logits"])
+        x = np.ones((1, 1), dtype=np.float32)
+        w = exact_bf16_bits([[float(v)] for v in case["logits"]])
+        b = None if case["bias"] is None else np.array(case["bias"], dtype=np.float64)
+        ids, wts, keys, scores = o.route_sigmoid(x, w, b, case["top_k"],
+                                                 normalize=case["normalize"], scale=case["scale"])
+        assert ids[0].tolist() == case["ids"], (case["what"], ids[0])
+        ref = np.array([float(v) for v in case["weights"]])
+        assert np.allclose(wts[0], ref, rtol=1e-15, atol=1e-27), (case["what"], wts[0], ref)
+
+
+def pin_router_sigmoid_vs_softmax_and_library(o):
+    """No bias: the sigmoid router picks what the softmax router picks (the
+    sigmoid is strictly increasing), and its scores are torch.sigmoid of the
+    same fp64 logits; the raw weights are those scores, the normalised ones
+    sum to the scale."""
+    for seed in range(4):
+        x, w, _ = _tiny_router_case(20 + seed, T=5, H=24, E=10, with_bias=False)
+        k = 4
+        ids_sm, _, logits = o.route(workloads.bits(x), workloads.bits(w), None, k)
+        ids, wts, keys, scores = o.route_sigmoid(workloads.bits(x), workloads.bits(w), None, k)
+        assert np.array_equal(ids, ids_sm), (seed, ids, ids_sm)
+        ref = torch.sigmoid(torch.tensor(logits, dtype=torch.float64)).numpy()
+        assert np.allclose(scores, ref, rtol=1e-15, atol=0), seed
+        assert np.array_equal(keys, scores)
+        for t in range(x.shape[0]):
+            assert np.allclose(wts[t], ref[t][ids[t]], rtol=1e-15, atol=0)
+        ids_n, wts_n, _, _ = o.route_sigmoid(workloads.bits(x), workloads.bits(w), None, k,
+                                             normalize=True, scale=2.0)
+        assert np.array_equal(ids_n, ids)
+        assert np.allclose(wts_n.sum(axis=1), 2.0, rtol=1e-15, atol=0)
+        assert np.allclose(wts_n, 2.0 * wts / wts.sum(axis=1, keepdims=True), rtol=1e-15, atol=0)
+
+
 def pin_swiglu_hand(o):
     g, x, wg, wu, wd = _hand_expert()
     f = o.expert_swiglu(x, wg, wu, wd)
@@ -308,6 +349,8 @@ def pin_fail_closed(o):
 
 
 ALL_PINS = [pin_plan_shares, pin_plan_refused, pin_router_brute_force, pin_router_closed_forms,
-            pin_router_full_softmax, pin_router_zipf, pin_router_bias_pull, pin_swiglu_hand,
+            pin_router_full_softmax, pin_router_zipf, pin_router_bias_pull,
+            pin_router_sigmoid_closed_forms, pin_router_sigmoid_vs_softmax_and_library,
+            pin_swiglu_hand,
             pin_swiglu_routed_hand, pin_dense_swiglu_library, pin_shared_additive,
             pin_fold_order, pin_ep_invariants, pin_imbalanced, pin_fail_closed]

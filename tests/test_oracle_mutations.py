@@ -30,6 +30,18 @@ MUTATIONS = [
      "while (0) {"),
     ("shared expert dropped", "yt[h] = yt[h] + f[h];", "yt[h] = yt[h];"),
     ("routing weight dropped", "double c = w_t[j] * f[h];", "double c = f[h];"),
+    ("sigmoid sign", "sc[e] = 1.0 / (1.0 + exp(-l));", "sc[e] = 1.0 / (1.0 + exp(l));"),
+    ("sigmoid bias ignored in the selection", "key[e] = bias != NULL ? sc[e] + bias[e] : sc[e];",
+     "key[e] = sc[e];"),
+    ("sigmoid weights from the biased keys",
+     "weights[t * top_k + j] = normalize ? scale * (sc[order[j]] / sum) : scale * sc[order[j]];",
+     "weights[t * top_k + j] = normalize ? scale * (key[order[j]] / sum) : scale * key[order[j]];"),
+    ("sigmoid normalisation ignored",
+     "weights[t * top_k + j] = normalize ? scale * (sc[order[j]] / sum) : scale * sc[order[j]];",
+     "weights[t * top_k + j] = scale * sc[order[j]];"),
+    ("sigmoid scale ignored",
+     "weights[t * top_k + j] = normalize ? scale * (sc[order[j]] / sum) : scale * sc[order[j]];",
+     "weights[t * top_k + j] = normalize ? (sc[order[j]] / sum) : sc[order[j]];"),
     ("gate row index off by a transpose", "g += bf16_value(w_gate[i * H + h]) * xt[h];",
      "g += bf16_value(w_gate[(i * H + h) % (I * H)]) * xt[(h + 1) % H];"),
 ]
