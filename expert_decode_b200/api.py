@@ -52,6 +52,8 @@ def library():
             P, I64, I32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
             lib.ep_plan.argtypes = [I32, I32, ctypes.POINTER(Plan)]
             lib.moe_route.argtypes = [P, ctypes.c_int, I64, I64, P, P, I64, I32, P, P, P]
+            lib.moe_route_sigmoid.argtypes = [P, ctypes.c_int, I64, I64, P, P, I64, I32, I32,
+                                              ctypes.c_float, P, P, P]
             lib.moe_ffn_workspace_size.argtypes = [I64, I64, I64, I32, I64, I64]
             lib.moe_ffn_workspace_size.restype = SZ
             lib.moe_ffn_forward.argtypes = [P, ctypes.c_int, I64, I64, P, P, I32, P, P, P, I64,
@@ -65,7 +67,8 @@ def library():
             lib.ep_last_launch_count.restype = I32
             lib.ep_profile_events.argtypes = [P, I32]
             lib.ep_profile_events.restype = ctypes.c_int
-            for fn in ("ep_plan", "moe_route", "moe_ffn_forward", "moe_ffn_forward_noalloc",
+            for fn in ("ep_plan", "moe_route", "moe_route_sigmoid", "moe_ffn_forward",
+                       "moe_ffn_forward_noalloc",
                        "ep_set_dispatch", "ep_check_status"):
                 getattr(lib, fn).restype = ctypes.c_int
             _lib = lib
@@ -127,6 +130,26 @@ def moe_route(x, w_router, bias, top_k, ids=None, weights=None, stream=None):
     _dense(weights, "weights", torch.float32)
     _check(library().moe_route(_ptr(x), _dtype(x), T, H, _ptr(w_router), _ptr(bias), E,
                                int(top_k), _ptr(ids), _ptr(weights), _stream(stream)))
+    return ids, weights
+
+
+def moe_route_sigmoid(x, w_router, bias, top_k, normalize=False, scale=1.0, ids=None,
+                      weights=None, stream=None):
+    """ids and weights of the sigmoid router variant (bias selects only)."""
+    _dense(x, "x", ndim=2)
+    _dense(w_router, "w_router", torch.bfloat16, 2)
+    _dense(bias, "bias", torch.float32, 1)
+    T, H = x.shape
+    E = w_router.shape[0]
+    if ids is None:
+        ids = torch.empty((T, top_k), dtype=torch.int32, device=x.device)
+    if weights is None:
+        weights = torch.empty((T, top_k), dtype=torch.float32, device=x.device)
+    _dense(ids, "ids", torch.int32)
+    _dense(weights, "weights", torch.float32)
+    _check(library().moe_route_sigmoid(_ptr(x), _dtype(x), T, H, _ptr(w_router), _ptr(bias), E,
+                                       int(top_k), 1 if normalize else 0, float(scale),
+                                       _ptr(ids), _ptr(weights), _stream(stream)))
     return ids, weights
 
 

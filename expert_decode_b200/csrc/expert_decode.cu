@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -135,16 +136,27 @@ ep_status device_info(const DeviceInfo **out) {
         EP_CUDA_CHECK(
             cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
         const int m = d.smem_optin;
-#define EPK_RT_ATTR(XF, TMV)                                                                 \
-    EP_CUDA_CHECK(cudaFuncSetAttribute(epk::router_tiled_kernel<XF, TMV>,                    \
+#define EPK_RT_ATTR(XF, TMV, SG)                                                             \
+    EP_CUDA_CHECK(cudaFuncSetAttribute(epk::router_tiled_kernel<XF, TMV, SG>,                \
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, m))
-        EPK_RT_ATTR(false, 1); EPK_RT_ATTR(false, 2); EPK_RT_ATTR(false, 4);
-        EPK_RT_ATTR(true, 1); EPK_RT_ATTR(true, 2); EPK_RT_ATTR(true, 4);
+        for (int sg = 0; sg < 2; ++sg) {
+            if (sg) {
+                EPK_RT_ATTR(false, 1, true); EPK_RT_ATTR(false, 2, true); EPK_RT_ATTR(false, 4, true);
+                EPK_RT_ATTR(true, 1, true); EPK_RT_ATTR(true, 2, true); EPK_RT_ATTR(true, 4, true);
+            } else {
+                EPK_RT_ATTR(false, 1, false); EPK_RT_ATTR(false, 2, false);
+                EPK_RT_ATTR(false, 4, false); EPK_RT_ATTR(true, 1, false);
+                EPK_RT_ATTR(true, 2, false); EPK_RT_ATTR(true, 4, false);
+            }
+        }
 #undef EPK_RT_ATTR
-#define EPK_RD_ATTR(XF, TBV)                                                                 \
-    EP_CUDA_CHECK(cudaFuncSetAttribute(epk::router_dot2_kernel<XF, TBV>,                     \
+#define EPK_RD_ATTR(XF, TBV, SG)                                                             \
+    EP_CUDA_CHECK(cudaFuncSetAttribute(epk::router_dot2_kernel<XF, TBV, SG>,                 \
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, m))
-        EPK_RD_ATTR(false, 1); EPK_RD_ATTR(false, 2); EPK_RD_ATTR(true, 1); EPK_RD_ATTR(true, 2);
+        EPK_RD_ATTR(false, 1, false); EPK_RD_ATTR(false, 2, false);
+        EPK_RD_ATTR(true, 1, false); EPK_RD_ATTR(true, 2, false);
+        EPK_RD_ATTR(false, 1, true); EPK_RD_ATTR(false, 2, true);
+        EPK_RD_ATTR(true, 1, true); EPK_RD_ATTR(true, 2, true);
 #undef EPK_RD_ATTR
         EP_CUDA_CHECK(cudaFuncSetAttribute(epk::stream_gate_up_kernel<false, false>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, m));
@@ -319,31 +331,36 @@ extern "C" ep_status ep_check_status(void *stream) {
     return ok();
 }
 
-extern "C" ep_status moe_route(const void *x, ep_dtype x_dtype, int64_t T, int64_t H,
-                               const void *w_router, const float *bias, int64_t E,
-                               int32_t top_k, int32_t *ids, float *weights, void *stream) {
+namespace {
+
+// Both routers: sig selects the sigmoid variant (normalize, scale used only
+// there); `who` names the entry point in error messages.
+ep_status route_impl(const char *who, bool sig, const void *x, ep_dtype x_dtype, int64_t T,
+                     int64_t H, const void *w_router, const float *bias, int64_t E,
+                     int32_t top_k, int32_t normalize, float scale, int32_t *ids,
+                     float *weights, void *stream) {
     if (x_dtype != EP_BF16 && x_dtype != EP_F32)
-        return fail(EP_EINVAL, "moe_route: unknown x dtype %d", (int)x_dtype);
+        return fail(EP_EINVAL, "%s: unknown x dtype %d", who, (int)x_dtype);
     if (T < 0 || T > kMaxT)
-        return fail(EP_EINVAL, "moe_route: T = %lld outside [0, %lld]", (long long)T,
+        return fail(EP_EINVAL, "%s: T = %lld outside [0, %lld]", who, (long long)T,
                     (long long)kMaxT);
     if (H < 8 || H > kMaxH || H % 8 != 0)
-        return fail(EP_EINVAL, "moe_route: H = %lld must be a multiple of 8 in [8, %lld]",
+        return fail(EP_EINVAL, "%s: H = %lld must be a multiple of 8 in [8, %lld]", who,
                     (long long)H, (long long)kMaxH);
     if (E < 1 || E > kMaxE)
-        return fail(EP_EINVAL, "moe_route: E = %lld outside [1, %lld]", (long long)E,
+        return fail(EP_EINVAL, "%s: E = %lld outside [1, %lld]", who, (long long)E,
                     (long long)kMaxE);
     if (top_k < 1 || top_k > kMaxTopK || top_k > E)
-        return fail(EP_EINVAL, "moe_route: top_k = %d outside [1, min(E, %d)]", top_k, kMaxTopK);
+        return fail(EP_EINVAL, "%s: top_k = %d outside [1, min(E, %d)]", who, top_k, kMaxTopK);
     if (T == 0) {
         t_launches = 0;
         return ok();
     }
     if (x == nullptr || w_router == nullptr || ids == nullptr || weights == nullptr)
-        return fail(EP_EINVAL, "moe_route: NULL x, w_router, ids or weights");
+        return fail(EP_EINVAL, "%s: NULL x, w_router, ids or weights", who);
     if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(ids, 4) || !aligned(weights, 4) ||
         (bias != nullptr && !aligned(bias, 4)))
-        return fail(EP_EINVAL, "moe_route: misaligned pointer (x, w_router need 16 bytes)");
+        return fail(EP_EINVAL, "%s: misaligned pointer (x, w_router need 16 bytes)", who);
     const DeviceInfo *d = nullptr;
     ep_status s = device_info(&d);
     if (s != EP_OK)
@@ -358,18 +375,21 @@ extern "C" ep_status moe_route(const void *x, ep_dtype x_dtype, int64_t T, int64
         const int tb = T <= max_clusters ? 1 : epk::kRdMaxTB;
         const epk::RdSmem L = epk::rd_smem_layout(tb, (int)H, (int)E);
         if ((int)L.total > d->smem_optin)
-            return fail(EP_EINVAL, "moe_route: H = %lld, E = %lld need %u bytes of shared memory",
+            return fail(EP_EINVAL, "%s: H = %lld, E = %lld need %u bytes of shared memory", who,
                         (long long)H, (long long)E, L.total);
         const int64_t nblk = (T + tb - 1) / tb;
         const dim3 grid((unsigned)(nblk * epk::kRouterCluster));
         cudaError_t e;
-#define EPK_RD(XF, TBV)                                                                        \
-    e = launch(epk::router_dot2_kernel<XF, TBV>, grid, epk::kRdThreads, L.total, st, x, T,      \
-               (int)H, wr, bias, (int)E, top_k, ids, weights)
-        if (x_dtype == EP_F32) {
-            if (tb == 1) EPK_RD(true, 1); else EPK_RD(true, 2);
+#define EPK_RD(XF, TBV, SG)                                                                    \
+    e = launch(epk::router_dot2_kernel<XF, TBV, SG>, grid, epk::kRdThreads, L.total, st, x, T,  \
+               (int)H, wr, bias, (int)E, top_k, ids, weights, normalize, scale)
+        const bool f32 = x_dtype == EP_F32;
+        if (sig) {
+            if (f32) { if (tb == 1) EPK_RD(true, 1, true); else EPK_RD(true, 2, true); }
+            else { if (tb == 1) EPK_RD(false, 1, true); else EPK_RD(false, 2, true); }
         } else {
-            if (tb == 1) EPK_RD(false, 1); else EPK_RD(false, 2);
+            if (f32) { if (tb == 1) EPK_RD(true, 1, false); else EPK_RD(true, 2, false); }
+            else { if (tb == 1) EPK_RD(false, 1, false); else EPK_RD(false, 2, false); }
         }
 #undef EPK_RD
         EP_CUDA_CHECK(e);
@@ -378,7 +398,7 @@ extern "C" ep_status moe_route(const void *x, ep_dtype x_dtype, int64_t T, int64
         const int BT = epk::rt_block_tokens((int)E);
         const epk::RtSmem L = epk::rt_smem_layout(BT, (int)E);
         if ((int)L.total > d->smem_optin)
-            return fail(EP_EINVAL, "moe_route: E = %lld needs %u bytes of shared memory",
+            return fail(EP_EINVAL, "%s: E = %lld needs %u bytes of shared memory", who,
                         (long long)E, L.total);
         // a cluster of CE expert slices x CK slices of H (at most 8 CTAs);
         // H is split only as far as it takes to fill about two waves of CTAs
@@ -390,20 +410,47 @@ extern "C" ep_status moe_route(const void *x, ep_dtype x_dtype, int64_t T, int64
             1, std::min<int64_t>(want, std::min(epk::kRouterCluster / CE, nkt)));
         const dim3 grid((unsigned)(CE * CK), (unsigned)((T + BT - 1) / BT));
         cudaError_t e;
-#define EPK_RT(XF, TMV)                                                                        \
-    e = launch_cluster(epk::router_tiled_kernel<XF, TMV>, grid, epk::kRtThreads, L.total, st,  \
-                       (unsigned)(CE * CK), x, T, (int)H, wr, bias, (int)E, top_k, ids, weights, \
-                       CE, CK)
-        if (x_dtype == EP_F32) {
-            if (BT == 32) EPK_RT(true, 4); else if (BT == 16) EPK_RT(true, 2); else EPK_RT(true, 1);
+#define EPK_RT(XF, TMV, SG)                                                                    \
+    e = launch_cluster(epk::router_tiled_kernel<XF, TMV, SG>, grid, epk::kRtThreads, L.total,   \
+                       st, (unsigned)(CE * CK), x, T, (int)H, wr, bias, (int)E, top_k, ids,     \
+                       weights, CE, CK, normalize, scale)
+#define EPK_RT_BT(XF, SG)                                                                      \
+    do {                                                                                       \
+        if (BT == 32) EPK_RT(XF, 4, SG); else if (BT == 16) EPK_RT(XF, 2, SG);                 \
+        else EPK_RT(XF, 1, SG);                                                                \
+    } while (0)
+        if (sig) {
+            if (x_dtype == EP_F32) EPK_RT_BT(true, true); else EPK_RT_BT(false, true);
         } else {
-            if (BT == 32) EPK_RT(false, 4); else if (BT == 16) EPK_RT(false, 2); else EPK_RT(false, 1);
+            if (x_dtype == EP_F32) EPK_RT_BT(true, false); else EPK_RT_BT(false, false);
         }
+#undef EPK_RT_BT
 #undef EPK_RT
         EP_CUDA_CHECK(e);
     }
     t_launches = 1;
     return ok();
+}
+
+}  // namespace
+
+extern "C" ep_status moe_route(const void *x, ep_dtype x_dtype, int64_t T, int64_t H,
+                               const void *w_router, const float *bias, int64_t E,
+                               int32_t top_k, int32_t *ids, float *weights, void *stream) {
+    return route_impl("moe_route", false, x, x_dtype, T, H, w_router, bias, E, top_k, 0, 1.0f,
+                      ids, weights, stream);
+}
+
+extern "C" ep_status moe_route_sigmoid(const void *x, ep_dtype x_dtype, int64_t T, int64_t H,
+                                       const void *w_router, const float *bias, int64_t E,
+                                       int32_t top_k, int32_t normalize, float scale,
+                                       int32_t *ids, float *weights, void *stream) {
+    if (normalize != 0 && normalize != 1)
+        return fail(EP_EINVAL, "moe_route_sigmoid: normalize = %d must be 0 or 1", normalize);
+    if (!(scale > 0.0f) || !std::isfinite(scale))
+        return fail(EP_EINVAL, "moe_route_sigmoid: scale must be finite and positive");
+    return route_impl("moe_route_sigmoid", true, x, x_dtype, T, H, w_router, bias, E, top_k,
+                      normalize, scale, ids, weights, stream);
 }
 
 extern "C" size_t moe_ffn_workspace_size(int64_t T, int64_t H, int64_t E, int32_t top_k,

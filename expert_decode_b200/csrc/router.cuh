@@ -129,23 +129,22 @@ __device__ __forceinline__ double dot2_warp_total(float2 s, float2 c) {
     return (double)S + (double)C;
 }
 
-// One warp: top_k of the E logits of one token (ties to the lower id) and
-// their softmax renormalised over the picked set.
-__device__ void topk_softmax_warp(const double *lt, int E, int top_k, int32_t *ids_row,
-                                  float *w_row) {
+// One warp: the top_k of E values of one token by value, ties to the lower
+// id; lane r < top_k receives the r-th pick's id and value.
+__device__ void topk_select_warp(const double *v, int E, int top_k, int &pick_e, double &pick_v) {
     const int lane = (int)lane_id();
     const int per_lane = (E + 31) / 32;
     uint32_t chosen = 0;
-    double pick_v = 0.0, top = 0.0;
-    int pick_e = 0;
+    pick_v = 0.0;
+    pick_e = 0;
     for (int r = 0; r < top_k; ++r) {
         double bv = -INFINITY;
         int be = 0x7fffffff;
         for (int i = 0; i < per_lane; ++i) {
             const int e = lane + 32 * i;
             if (e < E && !((chosen >> i) & 1u)) {
-                const double v = lt[e];
-                if (v > bv || (v == bv && e < be)) { bv = v; be = e; }
+                const double x = v[e];
+                if (x > bv || (x == bv && e < be)) { bv = x; be = e; }
             }
         }
 #pragma unroll
@@ -156,13 +155,21 @@ __device__ void topk_softmax_warp(const double *lt, int E, int top_k, int32_t *i
         }
         if (be != 0x7fffffff && (be & 31) == lane)
             chosen |= 1u << (be >> 5);
-        if (r == 0)
-            top = bv;
         if (lane == r) {
             pick_v = bv;
             pick_e = be;
         }
     }
+}
+
+// Softmax router: the picks by logit, weights = softmax over the picked set.
+__device__ void topk_softmax_warp(const double *lt, int E, int top_k, int32_t *ids_row,
+                                  float *w_row) {
+    const int lane = (int)lane_id();
+    int pick_e;
+    double pick_v;
+    topk_select_warp(lt, E, top_k, pick_e, pick_v);
+    const double top = __shfl_sync(0xffffffffu, pick_v, 0);
     const double ev = lane < top_k ? exp(pick_v - top) : 0.0;
     double sum = 0.0;
     for (int j = 0; j < top_k; ++j)
@@ -172,6 +179,28 @@ __device__ void topk_softmax_warp(const double *lt, int E, int top_k, int32_t *i
         w_row[lane] = (float)(ev / sum);
     }
 }
+
+// Sigmoid router (the GLM variant: sigmoid + bias top-k, raw-score weights;
+// TensorFold #593, "What exists now", glm_route.cu): the picks by key =
+// score + bias, weights = scale * score, or scale * score / (sum of the
+// picked scores) with normalize.
+__device__ void topk_sigmoid_warp(const double *key, const double *score, int E, int top_k,
+                                  int normalize, float scale, int32_t *ids_row, float *w_row) {
+    const int lane = (int)lane_id();
+    int pick_e;
+    double pick_v;
+    topk_select_warp(key, E, top_k, pick_e, pick_v);
+    const double sc = lane < top_k ? score[pick_e] : 0.0;
+    double sum = 0.0;
+    for (int j = 0; j < top_k; ++j)
+        sum += __shfl_sync(0xffffffffu, sc, j);
+    if (lane < top_k) {
+        ids_row[lane] = pick_e;
+        w_row[lane] = (float)((double)scale * (normalize ? sc / sum : sc));
+    }
+}
+
+__device__ __forceinline__ double sigmoid_f64(double l) { return 1.0 / (1.0 + exp(-l)); }
 
 // ------------------------------------------------------ small-batch router
 // Up to 32 tokens: every logit by Dot2.  A cluster of 8 CTAs takes TB tokens
@@ -194,8 +223,10 @@ __host__ __device__ inline RdSmem rd_smem_layout(int tb_max, int H, int E) {
     uint32_t o = 0;
     const int per_cta = (E + kRouterCluster - 1) / kRouterCluster;
     s.x = o;     o = align_up_u32(o + (uint32_t)tb_max * H * 4, 16);
-    s.vals = o;  o = align_up_u32(o + (uint32_t)tb_max * per_cta * 8, 16);
-    s.logit = o; o = align_up_u32(o + (uint32_t)tb_max * E * 8, 16);
+    // [2][tb][per_cta] and [2][tb][E]: the logit (softmax) or the key and the
+    // score (sigmoid)
+    s.vals = o;  o = align_up_u32(o + 2u * tb_max * per_cta * 8, 16);
+    s.logit = o; o = align_up_u32(o + 2u * tb_max * E * 8, 16);
     s.total = o;
     return s;
 }
@@ -210,17 +241,18 @@ __device__ __forceinline__ void rd_load_chunks(const uint4 *__restrict__ wrow, i
     }
 }
 
-template <bool XF32, int TB>
+template <bool XF32, int TB, bool SIG>
 __global__ void __cluster_dims__(kRouterCluster, 1, 1) __launch_bounds__(kRdThreads, 1)
 router_dot2_kernel(const void *__restrict__ x, int64_t T, int H,
                    const uint16_t *__restrict__ w_router, const float *__restrict__ bias, int E,
-                   int top_k, int32_t *__restrict__ ids, float *__restrict__ weights) {
+                   int top_k, int32_t *__restrict__ ids, float *__restrict__ weights,
+                   int normalize, float scale) {
     extern __shared__ __align__(1024) uint8_t smem[];
     constexpr int XB = XF32 ? 4 : 2;
     const RdSmem L = rd_smem_layout(TB, H, E);
     float *xs = reinterpret_cast<float *>(smem + L.x);          // [TB][H]
-    double *vals = reinterpret_cast<double *>(smem + L.vals);   // [TB][per_cta]
-    double *logit = reinterpret_cast<double *>(smem + L.logit); // [TB][E], CTA 0
+    double *vals = reinterpret_cast<double *>(smem + L.vals);   // [2][TB][per_cta]
+    double *logit = reinterpret_cast<double *>(smem + L.logit); // [2][TB][E], CTA 0
 
     const uint32_t rank = cluster_ctarank();
     const int64_t t0 = (int64_t)(blockIdx.x / kRouterCluster) * TB;
@@ -296,9 +328,16 @@ router_dot2_kernel(const void *__restrict__ x, int64_t T, int H,
 #pragma unroll
         for (int t = 0; t < TB; ++t) {
             if (t < tb) {
-                const double l = dot2_warp_total(s[t], c[t]) + b;
-                if (lane == 0)
-                    vals[t * per_cta + (e - e_lo)] = l;
+                const double l = dot2_warp_total(s[t], c[t]);
+                if (lane == 0) {
+                    if constexpr (SIG) {
+                        const double sc = sigmoid_f64(l);
+                        vals[t * per_cta + (e - e_lo)] = sc + b;
+                        vals[(TB + t) * per_cta + (e - e_lo)] = sc;
+                    } else {
+                        vals[t * per_cta + (e - e_lo)] = l + b;
+                    }
+                }
             }
         }
     }
@@ -310,13 +349,20 @@ router_dot2_kernel(const void *__restrict__ x, int64_t T, int H,
         for (int i = threadIdx.x; i < tb * n; i += kRdThreads) {
             const int t = i / n, j = i - t * n;
             st_cluster_f64(r_logit + 8u * (uint32_t)(t * E + e_lo + j), vals[t * per_cta + j]);
+            if (SIG)
+                st_cluster_f64(r_logit + 8u * (uint32_t)((TB + t) * E + e_lo + j),
+                               vals[(TB + t) * per_cta + j]);
         }
     }
     cluster_sync();  // all logits are in CTA 0
     if (rank != 0 || warp >= tb)
         return;
-    topk_softmax_warp(logit + warp * E, E, top_k, ids + (t0 + warp) * top_k,
-                      weights + (t0 + warp) * top_k);
+    if constexpr (SIG)
+        topk_sigmoid_warp(logit + warp * E, logit + (TB + warp) * E, E, top_k, normalize, scale,
+                          ids + (t0 + warp) * top_k, weights + (t0 + warp) * top_k);
+    else
+        topk_softmax_warp(logit + warp * E, E, top_k, ids + (t0 + warp) * top_k,
+                          weights + (t0 + warp) * top_k);
 }
 
 // ------------------------------------------------------- tiled fp32 router
@@ -344,7 +390,7 @@ __host__ __device__ inline int rt_block_tokens(int E) {
 }
 
 struct RtSmem {
-    uint32_t xs, ws, xsq, wsq, part, logit, bound, ncand, cand, cval, total;
+    uint32_t xs, ws, xsq, wsq, part, logit, bound, ncand, cand, cval, cscore, total;
 };
 
 __host__ __device__ inline RtSmem rt_smem_layout(int BT, int E) {
@@ -360,6 +406,7 @@ __host__ __device__ inline RtSmem rt_smem_layout(int BT, int E) {
     s.ncand = o; o = align_up_u32(o + (uint32_t)BT * 4, 16);
     s.cand = o;  o = align_up_u32(o + (uint32_t)BT * kRouterMaxCand * 4, 16);
     s.cval = o;  o = align_up_u32(o + (uint32_t)BT * kRouterMaxCand * 8, 16);
+    s.cscore = o; o = align_up_u32(o + (uint32_t)BT * kRouterMaxCand * 8, 16);
     s.total = o;
     return s;
 }
@@ -408,12 +455,12 @@ __device__ double logit_dot2_global(const void *xrow, const uint16_t *__restrict
     return acc;
 }
 
-template <bool XF32, int TM>
+template <bool XF32, int TM, bool SIG>
 __global__ void __launch_bounds__(kRtThreads, 1)
 router_tiled_kernel(const void *__restrict__ x, int64_t T, int H,
                     const uint16_t *__restrict__ w_router, const float *__restrict__ bias, int E,
                     int top_k, int32_t *__restrict__ ids, float *__restrict__ weights, int CE,
-                    int CK) {
+                    int CK, int normalize, float scale) {
     constexpr int BT = 8 * TM;             // tokens per cluster
     constexpr int XB = XF32 ? 4 : 2;
     constexpr int LD = kRtBK + kRtPad;     // padded row of a k-tile, in floats
@@ -428,7 +475,8 @@ router_tiled_kernel(const void *__restrict__ x, int64_t T, int H,
     float *bound = reinterpret_cast<float *>(smem + L.bound); // [BT][E], CTA 0
     int *ncand = reinterpret_cast<int *>(smem + L.ncand);
     int *cand = reinterpret_cast<int *>(smem + L.cand);
-    double *cval = reinterpret_cast<double *>(smem + L.cval);
+    double *cval = reinterpret_cast<double *>(smem + L.cval);      // refined logit or key
+    double *cscore = reinterpret_cast<double *>(smem + L.cscore);  // refined score (sigmoid)
 
     grid_dependents_launch();
     grid_dependency_wait();
@@ -625,8 +673,18 @@ router_tiled_kernel(const void *__restrict__ x, int64_t T, int H,
                 x2 += ld_cluster_f32(map_shared_rank(xsq + t, r));
                 w2 += ld_cluster_f32(map_shared_rank(wsq + el, r));
             }
-            const float l = sum + (bias != nullptr ? bias[e] : 0.f);
-            const float d = 1.5f * (gam * sqrtf(x2) * sqrtf(w2) + u * fabsf(l)) + 1e-30f;
+            const float b = bias != nullptr ? bias[e] : 0.f;
+            float l, d;
+            if (SIG) {
+                // key = sigmoid(l) + b; the sigmoid's slope is at most 1/4, and
+                // 4e-7 (1 + |key|) covers its fp32 evaluation and the sum
+                const float d_l = 1.5f * (gam * sqrtf(x2) * sqrtf(w2) + u * fabsf(sum)) + 1e-30f;
+                l = 1.0f / (1.0f + expf(-sum)) + b;
+                d = 0.25f * d_l + 4e-7f * (1.0f + fabsf(l));
+            } else {
+                l = sum + b;
+                d = 1.5f * (gam * sqrtf(x2) * sqrtf(w2) + u * fabsf(l)) + 1e-30f;
+            }
             st_cluster_f32(r_logit + 4u * (uint32_t)(t * E + e), l);
             st_cluster_f32(r_bound + 4u * (uint32_t)(t * E + e), d);
         }
@@ -668,6 +726,7 @@ router_tiled_kernel(const void *__restrict__ x, int64_t T, int H,
         const uint32_t r_ncand = map_shared_rank(ncand, 0);
         const uint32_t r_cand = map_shared_rank(cand, 0);
         const uint32_t r_cval = map_shared_rank(cval, 0);
+        const uint32_t r_cscore = map_shared_rank(cscore, 0);
         if (rank != 0) {
             if (tid < tb)
                 ncand[tid] = ld_cluster_s32(r_ncand + 4u * tid);
@@ -687,9 +746,18 @@ router_tiled_kernel(const void *__restrict__ x, int64_t T, int H,
                 if ((mine++ % (CK * (kRtThreads / 32))) != warp + k_part * (kRtThreads / 32))
                     continue;
                 const uint8_t *xrow = reinterpret_cast<const uint8_t *>(x) + (size_t)(t0 + t) * H * XB;
-                const double v = logit_dot2_global<XF32>(xrow, w_router, bias, H, e);
-                if (lane == 0)
-                    st_cluster_f64(r_cval + 8u * (uint32_t)(t * kRouterMaxCand + ci), v);
+                if (SIG) {
+                    const double sc = sigmoid_f64(logit_dot2_global<XF32>(xrow, w_router, nullptr, H, e));
+                    if (lane == 0) {
+                        st_cluster_f64(r_cval + 8u * (uint32_t)(t * kRouterMaxCand + ci),
+                                       sc + (bias != nullptr ? (double)bias[e] : 0.0));
+                        st_cluster_f64(r_cscore + 8u * (uint32_t)(t * kRouterMaxCand + ci), sc);
+                    }
+                } else {
+                    const double v = logit_dot2_global<XF32>(xrow, w_router, bias, H, e);
+                    if (lane == 0)
+                        st_cluster_f64(r_cval + 8u * (uint32_t)(t * kRouterMaxCand + ci), v);
+                }
             }
         }
     }
@@ -700,7 +768,7 @@ router_tiled_kernel(const void *__restrict__ x, int64_t T, int H,
     // CTA 0: pick top_k on the refined logits, renormalise, write
     for (int t = warp; t < tb; t += kRtThreads / 32) {
         const int nc = ncand[t];
-        double bv_list = 0.0, top = 0.0;
+        double bv_list = 0.0, top = 0.0, bs_list = 0.0;  // lane r: the r-th pick's value, score
         int be_list = 0;
         if (nc <= kRouterMaxCand) {
             uint32_t chosen = 0;
@@ -729,6 +797,8 @@ router_tiled_kernel(const void *__restrict__ x, int64_t T, int H,
                 if (lane == r) {
                     bv_list = bv;
                     be_list = be;
+                    if (SIG && bi >= 0)
+                        bs_list = cscore[t * kRouterMaxCand + bi];
                 }
             }
         } else {
@@ -744,33 +814,51 @@ router_tiled_kernel(const void *__restrict__ x, int64_t T, int H,
             const double thr = (double)kth_logit(lt, E, top_k) - 2.0 * (double)dmax * 1.0001;
             const uint8_t *xrow = reinterpret_cast<const uint8_t *>(x) + (size_t)(t0 + t) * H * XB;
             double lv = -INFINITY;  // lane j holds the j-th best so far
+            double ls = 0.0;        // and its score (sigmoid)
             int li = 0x7fffffff;
             for (int e = 0; e < E; ++e) {
                 if ((double)lt[e] < thr)
                     continue;
-                const double v = logit_dot2_global<XF32>(xrow, w_router, bias, H, e);
+                double v, sc = 0.0;
+                if (SIG) {
+                    sc = sigmoid_f64(logit_dot2_global<XF32>(xrow, w_router, nullptr, H, e));
+                    v = sc + (bias != nullptr ? (double)bias[e] : 0.0);
+                } else {
+                    v = logit_dot2_global<XF32>(xrow, w_router, bias, H, e);
+                }
                 // insert: lanes whose value ranks below v shift down by one
                 const bool below = !(lv > v || (lv == v && li < e));
                 const uint32_t m = __ballot_sync(0xffffffffu, below && lane < top_k);
                 const int pos = m ? __ffs(m) - 1 : top_k;
                 const double pv = __shfl_up_sync(0xffffffffu, lv, 1);
+                const double ps = __shfl_up_sync(0xffffffffu, ls, 1);
                 const int pi = __shfl_up_sync(0xffffffffu, li, 1);
                 if (lane < top_k && pos < top_k) {
-                    if (lane == pos) { lv = v; li = e; }
-                    else if (lane > pos) { lv = pv; li = pi; }
+                    if (lane == pos) { lv = v; ls = sc; li = e; }
+                    else if (lane > pos) { lv = pv; ls = ps; li = pi; }
                 }
             }
             top = __shfl_sync(0xffffffffu, lv, 0);
             bv_list = lv;
+            bs_list = ls;
             be_list = li;
         }
-        const double ev = lane < top_k ? exp(bv_list - top) : 0.0;
-        double ssum = 0.0;
-        for (int j = 0; j < top_k; ++j)
-            ssum += __shfl_sync(0xffffffffu, ev, j);
+        double wv;
+        if (SIG) {
+            double ssum = 0.0;
+            for (int j = 0; j < top_k; ++j)
+                ssum += __shfl_sync(0xffffffffu, lane < top_k ? bs_list : 0.0, j);
+            wv = (double)scale * (normalize ? bs_list / ssum : bs_list);
+        } else {
+            const double ev = lane < top_k ? exp(bv_list - top) : 0.0;
+            double ssum = 0.0;
+            for (int j = 0; j < top_k; ++j)
+                ssum += __shfl_sync(0xffffffffu, ev, j);
+            wv = ev / ssum;
+        }
         if (lane < top_k) {
             ids[(t0 + t) * top_k + lane] = be_list;
-            weights[(t0 + t) * top_k + lane] = (float)(ev / ssum);
+            weights[(t0 + t) * top_k + lane] = (float)wv;
         }
     }
 }

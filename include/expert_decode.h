@@ -99,6 +99,26 @@ ep_status moe_route(const void *x, ep_dtype x_dtype, int64_t T, int64_t H,
                     int32_t *ids, float *weights, void *stream);
 
 /*
+ * moe_route_sigmoid -- the GLM router variant: "sigmoid + bias top-k,
+ * raw-score weights" (TensorFold #593, a contributor's comment "What exists
+ * now", glm_route.cu).  The page names the ingredients only; read as:
+ *   l_e = sum_h x[t,h] W_router[e,h]       (no bias)
+ *   s_e = 1 / (1 + exp(-l_e))              the score
+ *   S   = top_k experts by s_e + bias[e]   (the bias moves the selection only),
+ *         ties to the lower id
+ *   weights[t,j] = scale * s_{S_j}, or with normalize = 1
+ *   weights[t,j] = scale * s_{S_j} / sum over S of s
+ * ids written by descending s + bias.  Arguments, layouts, limits and errors
+ * as moe_route, plus normalize (0 or 1) and scale (finite, > 0; else
+ * EP_EINVAL).  The logits are compensated fp32 sums as in moe_route; the
+ * scores and keys are formed from them in fp64.
+ */
+ep_status moe_route_sigmoid(const void *x, ep_dtype x_dtype, int64_t T, int64_t H,
+                            const void *w_router, const float *bias, int64_t E, int32_t top_k,
+                            int32_t normalize, float scale, int32_t *ids, float *weights,
+                            void *stream);
+
+/*
  * moe_ffn_workspace_size -- bytes of device workspace moe_ffn_forward needs
  * for these sizes (0 when T = 0).  The workspace holds the token grouping,
  * the grouped activations and the per-pick partial outputs; its contents on
