@@ -376,8 +376,9 @@ router_dot2_kernel(const void *__restrict__ x, int64_t T, int H,
 // the tokens.  Every 32-term block is summed on its own (two 16-term packed
 // halves) before it joins the running total, which bounds the rounding error
 // of a logit by gamma_n sum_h |x_h w_h| + u |l|, n = 32 + (k-tiles per CTA)
-// + CK + 2, with sum |x_h w_h| <= ||x|| ||w||.  Candidates and their Dot2
-// refinement follow.
+// + CK + 2, with sum |x_h w_h| <= ||x|| ||w||.  Each token's logits and bounds
+// then go to one CTA of the cluster (token t to CTA t mod CE CK), which picks
+// its candidates, refines them by Dot2 and writes its ids and weights.
 constexpr int kRtBE = 128;
 constexpr int kRtBK = 32;
 constexpr int kRtPad = 4;
@@ -652,11 +653,14 @@ router_tiled_kernel(const void *__restrict__ x, int64_t T, int H,
     }
     __syncthreads();
     cluster_sync();  // every CTA runs and has its partial tile in place
+    // Token t of the block belongs to CTA t mod NC of the cluster (local row
+    // t / NC): its logits and bounds are delivered there, and that CTA picks
+    // its candidates, refines them and writes its ids and weights.
+    const int NC = CE * CK;
+    const int n_local = (tb - (int)rank + NC - 1) / NC;  // tokens this CTA owns
     {
         // CTA (e, k) adds the CK partials of tokens [BT k / CK, BT (k+1) / CK)
         // of expert slice e, in ascending k-slice order
-        const uint32_t r_logit = map_shared_rank(logit, 0);
-        const uint32_t r_bound = map_shared_rank(bound, 0);
         const float u = 5.9604644775390625e-8f;  // 2^-24
         const float n = (float)(kRtBK + (nkt + CK - 1) / CK + CK + 2);
         const float gam = n * u / (1.0f - n * u);
@@ -685,89 +689,73 @@ router_tiled_kernel(const void *__restrict__ x, int64_t T, int H,
                 l = sum + b;
                 d = 1.5f * (gam * sqrtf(x2) * sqrtf(w2) + u * fabsf(l)) + 1e-30f;
             }
-            st_cluster_f32(r_logit + 4u * (uint32_t)(t * E + e), l);
-            st_cluster_f32(r_bound + 4u * (uint32_t)(t * E + e), d);
+            const uint32_t owner = (uint32_t)(t % NC), row = (uint32_t)(t / NC);
+            st_cluster_f32(map_shared_rank(logit + row * E + e, owner), l);
+            st_cluster_f32(map_shared_rank(bound + row * E + e, owner), d);
         }
     }
-    cluster_sync();  // all logits and bounds are in CTA 0
+    cluster_sync();  // every token's logits and bounds are with its owner; no
+                     // shared memory of another CTA is used after this point
 
-    // candidates per token (CTA 0): every expert whose exact logit could
-    // reach the k-th largest under the bounds
-    if (rank == 0) {
-        for (int t = warp; t < tb; t += kRtThreads / 32) {
-            const float *lt = logit + t * E;
-            const float *bt = bound + t * E;
-            const float vk = kth_logit(lt, E, top_k);
-            float dmax = 0.f;
-            for (int e = lane; e < E; e += 32)
-                dmax = fmaxf(dmax, bt[e]);
+    // candidates per owned token (one warp each): every expert whose exact
+    // logit could reach the k-th largest under the bounds
+    for (int j = warp; j < n_local; j += kRtThreads / 32) {
+        const float *lt = logit + j * E;
+        const float *bt = bound + j * E;
+        const float vk = kth_logit(lt, E, top_k);
+        float dmax = 0.f;
+        for (int e = lane; e < E; e += 32)
+            dmax = fmaxf(dmax, bt[e]);
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1)
-                dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, off));
-            const double thr = (double)vk - 2.0 * (double)dmax * 1.0001;
-            int count = 0;
-            for (int i = 0; i < (E + 31) / 32; ++i) {
-                const int e = lane + 32 * i;
-                const bool c = e < E && (double)lt[e] >= thr;
-                const uint32_t m = __ballot_sync(0xffffffffu, c);
-                const int pos = count + __popc(m & ((1u << lane) - 1u));
-                if (c && pos < kRouterMaxCand)
-                    cand[t * kRouterMaxCand + pos] = e;
-                count += __popc(m);
-            }
-            if (lane == 0)
-                ncand[t] = count;
+        for (int off = 16; off > 0; off >>= 1)
+            dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, off));
+        const double thr = (double)vk - 2.0 * (double)dmax * 1.0001;
+        int count = 0;
+        for (int i = 0; i < (E + 31) / 32; ++i) {
+            const int e = lane + 32 * i;
+            const bool c = e < E && (double)lt[e] >= thr;
+            const uint32_t m = __ballot_sync(0xffffffffu, c);
+            const int pos = count + __popc(m & ((1u << lane) - 1u));
+            if (c && pos < kRouterMaxCand)
+                cand[j * kRouterMaxCand + pos] = e;
+            count += __popc(m);
         }
+        if (lane == 0)
+            ncand[j] = count;
     }
-    cluster_sync();  // candidate lists visible to every CTA
+    __syncthreads();
 
-    // every CTA: Dot2 logits of the candidates in its expert slice
+    // Dot2 logits of the owned tokens' candidates, spread over the warps
     {
-        const uint32_t r_ncand = map_shared_rank(ncand, 0);
-        const uint32_t r_cand = map_shared_rank(cand, 0);
-        const uint32_t r_cval = map_shared_rank(cval, 0);
-        const uint32_t r_cscore = map_shared_rank(cscore, 0);
-        if (rank != 0) {
-            if (tid < tb)
-                ncand[tid] = ld_cluster_s32(r_ncand + 4u * tid);
-            for (int i = tid; i < tb * kRouterMaxCand; i += kRtThreads)
-                cand[i] = ld_cluster_s32(r_cand + 4u * (uint32_t)i);
-        }
-        __syncthreads();
-        // (token, candidate) pairs whose expert this CTA owns, one per warp
         int mine = 0;
-        for (int t = 0; t < tb; ++t) {
-            const int nc = ncand[t] <= kRouterMaxCand ? ncand[t] : 0;
+        for (int j = 0; j < n_local; ++j) {
+            const int t = (int)rank + NC * j;
+            const int nc = ncand[j] <= kRouterMaxCand ? ncand[j] : 0;
+            const uint8_t *xrow = reinterpret_cast<const uint8_t *>(x) + (size_t)(t0 + t) * H * XB;
             for (int ci = 0; ci < nc; ++ci) {
-                const int e = cand[t * kRouterMaxCand + ci];
-                if (e < e0 || e >= e0 + kRtBE)
+                if ((mine++ % (kRtThreads / 32)) != warp)
                     continue;
-                // the CK CTAs of this expert slice share its candidates
-                if ((mine++ % (CK * (kRtThreads / 32))) != warp + k_part * (kRtThreads / 32))
-                    continue;
-                const uint8_t *xrow = reinterpret_cast<const uint8_t *>(x) + (size_t)(t0 + t) * H * XB;
+                const int e = cand[j * kRouterMaxCand + ci];
                 if (SIG) {
                     const double sc = sigmoid_f64(logit_dot2_global<XF32>(xrow, w_router, nullptr, H, e));
                     if (lane == 0) {
-                        st_cluster_f64(r_cval + 8u * (uint32_t)(t * kRouterMaxCand + ci),
-                                       sc + (bias != nullptr ? (double)bias[e] : 0.0));
-                        st_cluster_f64(r_cscore + 8u * (uint32_t)(t * kRouterMaxCand + ci), sc);
+                        cval[j * kRouterMaxCand + ci] = sc + (bias != nullptr ? (double)bias[e] : 0.0);
+                        cscore[j * kRouterMaxCand + ci] = sc;
                     }
                 } else {
                     const double v = logit_dot2_global<XF32>(xrow, w_router, bias, H, e);
                     if (lane == 0)
-                        st_cluster_f64(r_cval + 8u * (uint32_t)(t * kRouterMaxCand + ci), v);
+                        cval[j * kRouterMaxCand + ci] = v;
                 }
             }
         }
     }
-    cluster_sync();  // refined logits are in CTA 0
-    if (rank != 0)
-        return;
+    __syncthreads();
 
-    // CTA 0: pick top_k on the refined logits, renormalise, write
-    for (int t = warp; t < tb; t += kRtThreads / 32) {
-        const int nc = ncand[t];
+    // pick top_k on the refined values of each owned token, weigh, write
+    for (int j = warp; j < n_local; j += kRtThreads / 32) {
+        const int t = (int)rank + NC * j;
+        const int nc = ncand[j];
         double bv_list = 0.0, top = 0.0, bs_list = 0.0;  // lane r: the r-th pick's value, score
         int be_list = 0;
         if (nc <= kRouterMaxCand) {
@@ -778,8 +766,8 @@ router_tiled_kernel(const void *__restrict__ x, int64_t T, int H,
                 for (int i = 0; i < 2; ++i) {
                     const int ci = lane + 32 * i;
                     if (ci < nc && !((chosen >> i) & 1u)) {
-                        const double v = cval[t * kRouterMaxCand + ci];
-                        const int e = cand[t * kRouterMaxCand + ci];
+                        const double v = cval[j * kRouterMaxCand + ci];
+                        const int e = cand[j * kRouterMaxCand + ci];
                         if (v > bv || (v == bv && e < be)) { bv = v; be = e; bi = ci; }
                     }
                 }
@@ -798,16 +786,16 @@ router_tiled_kernel(const void *__restrict__ x, int64_t T, int H,
                     bv_list = bv;
                     be_list = be;
                     if (SIG && bi >= 0)
-                        bs_list = cscore[t * kRouterMaxCand + bi];
+                        bs_list = cscore[j * kRouterMaxCand + bi];
                 }
             }
         } else {
             // degenerate input: every candidate in ascending id through a
             // sorted top_k list kept in registers of lanes 0..top_k-1
-            const float *lt = logit + t * E;
+            const float *lt = logit + j * E;
             float dmax = 0.f;
             for (int e = lane; e < E; e += 32)
-                dmax = fmaxf(dmax, bound[t * E + e]);
+                dmax = fmaxf(dmax, bound[j * E + e]);
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1)
                 dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, off));
@@ -846,14 +834,14 @@ router_tiled_kernel(const void *__restrict__ x, int64_t T, int H,
         double wv;
         if (SIG) {
             double ssum = 0.0;
-            for (int j = 0; j < top_k; ++j)
-                ssum += __shfl_sync(0xffffffffu, lane < top_k ? bs_list : 0.0, j);
+            for (int jj = 0; jj < top_k; ++jj)
+                ssum += __shfl_sync(0xffffffffu, lane < top_k ? bs_list : 0.0, jj);
             wv = (double)scale * (normalize ? bs_list / ssum : bs_list);
         } else {
             const double ev = lane < top_k ? exp(bv_list - top) : 0.0;
             double ssum = 0.0;
-            for (int j = 0; j < top_k; ++j)
-                ssum += __shfl_sync(0xffffffffu, ev, j);
+            for (int jj = 0; jj < top_k; ++jj)
+                ssum += __shfl_sync(0xffffffffu, ev, jj);
             wv = ev / ssum;
         }
         if (lane < top_k) {
