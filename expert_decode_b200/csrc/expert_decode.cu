@@ -333,6 +333,47 @@ extern "C" ep_status ep_check_status(void *stream) {
 
 namespace {
 
+// Clusters of `csize` CTAs of `fn` with `smem` bytes that can be resident at
+// once on this device (cudaOccupancyMaxActiveClusters), cached; 0 if none.
+int max_active_clusters(const void *fn, int csize, uint32_t smem) {
+    struct Entry {
+        const void *fn;
+        int dev, csize;
+        uint32_t smem;
+        int value;
+    };
+    static std::mutex mu;
+    static Entry cache[64];
+    static int n_cache = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < n_cache; ++i)
+        if (cache[i].fn == fn && cache[i].dev == dev && cache[i].csize == csize &&
+            cache[i].smem == smem)
+            return cache[i].value;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)csize, 1, 1);
+    cfg.blockDim = dim3((unsigned)epk::kRtThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = (unsigned)csize;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();
+        n = 0;
+    }
+    if (n_cache < 64)
+        cache[n_cache++] = Entry{fn, dev, csize, smem, n};
+    return n;
+}
+
 // Both routers: sig selects the sigmoid variant (normalize, scale used only
 // there); `who` names the entry point in error messages.
 ep_status route_impl(const char *who, bool sig, const void *x, ep_dtype x_dtype, int64_t T,
@@ -400,32 +441,47 @@ ep_status route_impl(const char *who, bool sig, const void *x, ep_dtype x_dtype,
         if ((int)L.total > d->smem_optin)
             return fail(EP_EINVAL, "%s: E = %lld needs %u bytes of shared memory", who,
                         (long long)E, L.total);
-        // a cluster of CE expert slices x CK slices of H (at most 8 CTAs);
-        // H is split only as far as it takes to fill about two waves of CTAs
+        // the kernel for this activation type, block size and router
+        using TiledFn = void (*)(const void *, int64_t, int, const uint16_t *, const float *, int,
+                                 int, int32_t *, float *, int, int, int, float);
+        TiledFn fn;
+        {
+            const bool f = x_dtype == EP_F32;
+#define EPK_RT_FN(TMV)                                                                         \
+    (sig ? (f ? epk::router_tiled_kernel<true, TMV, true> : epk::router_tiled_kernel<false, TMV, true>) \
+         : (f ? epk::router_tiled_kernel<true, TMV, false> : epk::router_tiled_kernel<false, TMV, false>))
+            fn = BT == 32 ? EPK_RT_FN(4) : (BT == 16 ? EPK_RT_FN(2) : EPK_RT_FN(1));
+#undef EPK_RT_FN
+        }
+        // A cluster of CE expert slices x CK slices of H (at most 8 CTAs).
+        // Splitting H shortens every CTA's main loop but makes the clusters
+        // larger, and larger clusters fit fewer at a time on the GPCs; CK is
+        // chosen for the least (waves) x (main loop / CK + the fixed tail),
+        // the tail taken as a tenth of an unsplit main loop.
         const int CE = (int)((E + epk::kRtBE - 1) / epk::kRtBE);
         const int nkt = (int)((H + epk::kRtBK - 1) / epk::kRtBK);
         const int64_t blocks = (T + BT - 1) / BT;
-        const int64_t want = (2 * (int64_t)d->sm_count + blocks * CE - 1) / (blocks * CE);
-        const int CK = (int)std::max<int64_t>(
-            1, std::min<int64_t>(want, std::min(epk::kRouterCluster / CE, nkt)));
-        const dim3 grid((unsigned)(CE * CK), (unsigned)((T + BT - 1) / BT));
-        cudaError_t e;
-#define EPK_RT(XF, TMV, SG)                                                                    \
-    e = launch_cluster(epk::router_tiled_kernel<XF, TMV, SG>, grid, epk::kRtThreads, L.total,   \
-                       st, (unsigned)(CE * CK), x, T, (int)H, wr, bias, (int)E, top_k, ids,     \
-                       weights, CE, CK, normalize, scale)
-#define EPK_RT_BT(XF, SG)                                                                      \
-    do {                                                                                       \
-        if (BT == 32) EPK_RT(XF, 4, SG); else if (BT == 16) EPK_RT(XF, 2, SG);                 \
-        else EPK_RT(XF, 1, SG);                                                                \
-    } while (0)
-        if (sig) {
-            if (x_dtype == EP_F32) EPK_RT_BT(true, true); else EPK_RT_BT(false, true);
-        } else {
-            if (x_dtype == EP_F32) EPK_RT_BT(true, false); else EPK_RT_BT(false, false);
+        const int ck_max = std::max(1, std::min(epk::kRouterCluster / CE, nkt));
+        int CK = 1;
+        bool have = false;
+        double best = 0.0;
+        for (int ck = 1; ck <= ck_max; ++ck) {
+            const int fit = max_active_clusters(reinterpret_cast<const void *>(fn), CE * ck,
+                                                L.total);
+            if (fit < 1)
+                continue;
+            const double waves = (double)((blocks + fit - 1) / fit);
+            const double cost = waves * (1.0 / ck + 0.1);
+            if (!have || cost < best) {
+                have = true;
+                best = cost;
+                CK = ck;
+            }
         }
-#undef EPK_RT_BT
-#undef EPK_RT
+        const dim3 grid((unsigned)(CE * CK), (unsigned)blocks);
+        const cudaError_t e = launch_cluster(fn, grid, epk::kRtThreads, L.total, st,
+                                             (unsigned)(CE * CK), x, T, (int)H, wr, bias, (int)E,
+                                             top_k, ids, weights, CE, CK, normalize, scale);
         EP_CUDA_CHECK(e);
     }
     t_launches = 1;
