@@ -43,6 +43,20 @@ N_BATCHES = 16
 FLUSH_BYTES = 512 << 20
 
 
+def whole_job_throughput(tokens, seconds, dist=None, device="cpu"):
+    """Units per second of the whole job: the tokens of every rank over the
+    slowest rank's time (sum and max over the ranks of the process group;
+    this rank alone when dist is None).  Returns (throughput, max seconds)."""
+    if dist is None:
+        return tokens / seconds, seconds
+    t = torch.tensor([float(tokens), seconds], device=device, dtype=torch.float64)
+    tokens_t = t[:1].clone()
+    seconds_t = t[1:].clone()
+    dist.all_reduce(tokens_t, op=dist.ReduceOp.SUM)
+    dist.all_reduce(seconds_t, op=dist.ReduceOp.MAX)
+    return float(tokens_t.item()) / float(seconds_t.item()), float(seconds_t.item())
+
+
 def parse_args():
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -451,13 +465,7 @@ def run_ours(args, wl):
                                   for i in range(K)) / K
         per_T[f"T={T}"]["kernels_us"] = {k: round(v, 2) for k, v in kus.items()}
 
-    if dist is not None:
-        t = torch.tensor([dev_s], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        dev_s_max = float(t.item())
-    else:
-        dev_s_max = dev_s
-    value = tokens_rank * world / dev_s_max
+    value, dev_s_max = whole_job_throughput(tokens_rank, dev_s, dist, device)
 
     # roofline of the dominant kernel
     t_hbm = dom_bytes / (peaks["hbm_gbs"] * 1e9)
@@ -529,11 +537,8 @@ def run_ours(args, wl):
         ee.record()
         torch.cuda.synchronize()
         e2e_s = es.elapsed_time(ee) / 1e3
-        if dist is not None:
-            t = torch.tensor([e2e_s], device=device, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_s = float(t.item())
-        e2e = {"value": KE * sum(Ts) * world / e2e_s, "unit": "tokens/s",
+        e2e_value, e2e_s = whole_job_throughput(KE * sum(Ts), e2e_s, dist, device)
+        e2e = {"value": e2e_value, "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": KE,
                "l2": "not flushed"}
 
