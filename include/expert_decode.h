@@ -215,6 +215,14 @@ typedef enum {
 ep_status ep_set_dispatch(ep_dispatch mode);
 
 /*
+ * Launch mode.  Kernels are launched with programmatic dependent launch: a
+ * kernel may start while the previous kernel on the stream is still running
+ * and reads that kernel's outputs only after griddepcontrol.wait.  Setting
+ * the environment variable EXPERT_DECODE_NO_PDL=1 before the first call of a
+ * process launches every kernel without it (the value is read once).
+ */
+
+/*
  * ep_check_status -- synchronise `stream`, then return and clear the sticky
  * device status of the current device: EP_OK, EP_EBADID or EP_ETIMEOUT
  * (EP_ECUDA if the synchronisation itself failed).

@@ -28,7 +28,9 @@
  * order, where the shared expert enters) are the ones listed in the design
  * notes: softmax router with renormalised top-k, ties to the lower expert id,
  * picks folded in ascending (expert id, slot), the shared expert added after
- * the routed sum, routed scaling factor 1.
+ * the routed sum, routed scaling factor 1.  The GLM router variant of the
+ * tracker page (sigmoid + bias top-k, raw-score weights) is read as in
+ * oracle_route_sigmoid below.
  */
 #include <math.h>
 #include <stdint.h>
