@@ -73,6 +73,17 @@ def test_decode_full_size(oracle_lib, T):
     assert torch.equal(gpu_ffn(x, ids, w, W, plan), y), "not run-to-run identical"
 
 
+@pytest.mark.parametrize("T", [1, 8])
+def test_decode_at_the_large_sizes(oracle_lib, gate_up, T):
+    """H = 6144, E = 256, top_k = 8, I = I_s = 2048 with the Zipf bias: 96 k blocks
+    per tensor-core tile, 8-chunk rows in the down kernel's register path."""
+    wl = WL["large"]
+    W, x, ids, w = _routed(oracle_lib, wl, T, seed=51)
+    y = gpu_ffn(x, ids, w, W, ed.ep_plan(wl.E, 8))
+    ed.ep_check_status()
+    check_y(y, oracle_ffn(oracle_lib, x, ids, w, W), rel_tol=1e-4, what=f"large sizes T={T}")
+
+
 def test_decode_end_to_end_with_gpu_router(oracle_lib):
     wl = WL["decode"]
     W, x = device_inputs(wl, 8, batch=3)
