@@ -107,3 +107,36 @@ def test_workspace_size_grows_with_work():
     big = ed.moe_ffn_workspace_size(512, 4096, 128, 8, 2048, 2048)
     assert 0 < small < big
     assert ed.moe_ffn_workspace_size(0, 4096, 128, 8, 1536, 1536) == 0
+
+
+def test_sigmoid_route_fails_closed_before_any_launch():
+    lib = api.library()
+    f = _fake()
+    def route(**kw):
+        a = dict(x=f, xdt=0, T=4, H=256, w=f, b=None, E=16, k=4, norm=0, scale=1.0, ids=f, wts=f)
+        a.update(kw)
+        return lib.moe_route_sigmoid(a["x"], a["xdt"], a["T"], a["H"], a["w"], a["b"], a["E"],
+                                     a["k"], a["norm"], a["scale"], a["ids"], a["wts"], None)
+    assert route(norm=2) == ed.EP_EINVAL
+    assert route(scale=0.0) == ed.EP_EINVAL
+    assert route(scale=-1.0) == ed.EP_EINVAL
+    assert route(scale=float("nan")) == ed.EP_EINVAL
+    assert route(scale=float("inf")) == ed.EP_EINVAL
+    assert route(k=17) == ed.EP_EINVAL
+    assert route(T=65537) == ed.EP_EINVAL
+    assert route(x=None) == ed.EP_EINVAL
+    assert route(T=0) == ed.EP_OK
+    assert b"moe_route_sigmoid" in lib.ep_last_error() or lib.ep_last_error() == b""
+
+
+def test_noalloc_refuses_sizes_beyond_its_static_scratch():
+    lib = api.library()
+    f = _fake()
+    plan = ed.ep_plan(128, 8)
+    # T = 64 at H = 4096, E = 128, top_k = 8, I = I_s = 1536 needs about 16 MB
+    need = ed.moe_ffn_workspace_size(64, 4096, 128, 8, 1536, 1536)
+    assert need > (4 << 20)
+    rc = lib.moe_ffn_forward_noalloc(f, 0, 64, 4096, f, f, 8, f, f, f, 128, 1536, f, f, f, 1536,
+                                     ctypes.byref(plan), f, None)
+    assert rc == ed.EP_ENOMEM
+    assert b"static scratch" in lib.ep_last_error()
