@@ -13,6 +13,9 @@ namespace epk {
 // ---------------------------------------------------------------- status word
 enum : unsigned { kStatusBadId = 1u, kStatusTimeout = 2u };
 
+// An empty pick slot (EP_ID_NONE of the C ABI): skipped, and not reported.
+constexpr int32_t kIdNone = (int32_t)0x80000000;
+
 // One word per device (module global).  Kernels OR bits into it; the host
 // reads and clears it in ep_check_status().
 __device__ unsigned int g_status;

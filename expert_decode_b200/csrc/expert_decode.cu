@@ -19,6 +19,7 @@
 #include "streaming.cuh"
 #include "grouped.cuh"
 #include "decode_tc.cuh"
+#include "ep.cuh"
 
 namespace {
 
@@ -516,13 +517,17 @@ extern "C" size_t moe_ffn_workspace_size(int64_t T, int64_t H, int64_t E, int32_
     return workspace_layout(T, H, E, top_k, I, I_s).total;
 }
 
-extern "C" ep_status moe_ffn_forward(const void *x, ep_dtype x_dtype, int64_t T, int64_t H,
-                                     const int32_t *ids, const float *weights, int32_t top_k,
-                                     const void *w_gate, const void *w_up, const void *w_down,
-                                     int64_t E, int64_t I, const void *ws_gate,
-                                     const void *ws_up, const void *ws_down, int64_t I_s,
-                                     const ep_plan_t *plan, float *y, void *workspace,
-                                     size_t workspace_bytes, void *stream) {
+namespace {
+
+// moe_ffn_forward's body.  band_call: a band partial (moe_ffn_partial), whose
+// picks may outnumber the band's experts (they span bands), so top_k is not
+// bounded by E there.
+ep_status ffn_forward_impl(bool band_call, const void *x, ep_dtype x_dtype, int64_t T, int64_t H,
+                           const int32_t *ids, const float *weights, int32_t top_k,
+                           const void *w_gate, const void *w_up, const void *w_down, int64_t E,
+                           int64_t I, const void *ws_gate, const void *ws_up,
+                           const void *ws_down, int64_t I_s, const ep_plan_t *plan, float *y,
+                           void *workspace, size_t workspace_bytes, void *stream) {
     // ---- validation: nothing is launched and nothing written on failure
     if (plan == nullptr)
         return fail(EP_EINVAL, "moe_ffn_forward: plan is NULL");
@@ -545,7 +550,7 @@ extern "C" ep_status moe_ffn_forward(const void *x, ep_dtype x_dtype, int64_t T,
     if (E < 1 || E > kMaxE)
         return fail(EP_EINVAL, "moe_ffn_forward: E = %lld outside [1, %lld]", (long long)E,
                     (long long)kMaxE);
-    if (top_k < 1 || top_k > kMaxTopK || top_k > E)
+    if (top_k < 1 || top_k > kMaxTopK || (!band_call && top_k > E))
         return fail(EP_EINVAL, "moe_ffn_forward: top_k = %d outside [1, min(E, %d)]", top_k,
                     kMaxTopK);
     if (I < 8 || I > kMaxI || I % 8 != 0)
@@ -697,6 +702,146 @@ extern "C" ep_status moe_ffn_forward(const void *x, ep_dtype x_dtype, int64_t T,
     if (s != EP_OK)
         return fail(s, "moe_ffn_forward: %s", why);
     t_launches = launches;
+    return ok();
+}
+
+}  // namespace
+
+extern "C" ep_status moe_ffn_forward(const void *x, ep_dtype x_dtype, int64_t T, int64_t H,
+                                     const int32_t *ids, const float *weights, int32_t top_k,
+                                     const void *w_gate, const void *w_up, const void *w_down,
+                                     int64_t E, int64_t I, const void *ws_gate,
+                                     const void *ws_up, const void *ws_down, int64_t I_s,
+                                     const ep_plan_t *plan, float *y, void *workspace,
+                                     size_t workspace_bytes, void *stream) {
+    return ffn_forward_impl(false, x, x_dtype, T, H, ids, weights, top_k, w_gate, w_up, w_down,
+                            E, I, ws_gate, ws_up, ws_down, I_s, plan, y, workspace,
+                            workspace_bytes, stream);
+}
+
+// ======================================================== expert parallel
+// One rank's band partial and the rank-order combine of all partials.
+
+namespace {
+
+size_t partial_ids_offset(int64_t T, int64_t H, int64_t E_band, int64_t k, int64_t I) {
+    return align256(workspace_layout(T, H, E_band, k, I, 0).total);
+}
+
+}  // namespace
+
+extern "C" size_t moe_ffn_partial_workspace_size(int64_t T, int64_t H, int64_t E_band,
+                                                 int32_t top_k, int64_t I) {
+    if (T <= 0 || H <= 0 || E_band <= 0 || top_k <= 0 || I <= 0)
+        return 0;
+    return partial_ids_offset(T, H, E_band, top_k, I) + align256((size_t)T * top_k * 4);
+}
+
+extern "C" ep_status moe_ffn_partial(const void *x, ep_dtype x_dtype, int64_t T, int64_t H,
+                                     const int32_t *ids, const float *weights, int32_t top_k,
+                                     const void *w_gate, const void *w_up, const void *w_down,
+                                     int64_t I, const ep_plan_t *plan, int32_t rank,
+                                     float *partial, void *workspace, size_t workspace_bytes,
+                                     void *stream) {
+    if (plan == nullptr)
+        return fail(EP_EINVAL, "moe_ffn_partial: plan is NULL");
+    const int64_t E = plan->num_experts;
+    if (E < 1 || E > kMaxE || plan->bands < 1 || plan->bands > EP_MAX_BANDS ||
+        plan->bands > E || plan->band_start[0] != 0 || plan->band_start[plan->bands] != E)
+        return fail(EP_EINVAL, "moe_ffn_partial: plan is not a partition of [0, E)");
+    for (int r = 0; r < plan->bands; ++r)
+        if (plan->band_start[r + 1] <= plan->band_start[r])
+            return fail(EP_EINVAL, "moe_ffn_partial: band %d of the plan is empty or reversed", r);
+    if (rank < 0 || rank >= plan->bands)
+        return fail(EP_EINVAL, "moe_ffn_partial: rank %d outside [0, %d)", rank, plan->bands);
+    if (T < 0 || T > kMaxT || T * (int64_t)std::max(top_k, 1) > kMaxPairs)
+        return fail(EP_EINVAL, "moe_ffn_partial: T = %lld out of range", (long long)T);
+    if (top_k < 1 || top_k > kMaxTopK || top_k > E)
+        return fail(EP_EINVAL, "moe_ffn_partial: top_k = %d outside [1, min(E, %d)]", top_k,
+                    kMaxTopK);
+    if (T == 0) {
+        t_launches = 0;
+        return ok();
+    }
+    if (ids == nullptr || partial == nullptr)
+        return fail(EP_EINVAL, "moe_ffn_partial: a required pointer is NULL");
+    if (!aligned(ids, 4))
+        return fail(EP_EINVAL, "moe_ffn_partial: ids not 4-byte aligned");
+    const int32_t e_lo = plan->band_start[rank], e_hi = plan->band_start[rank + 1];
+    const int64_t E_band = e_hi - e_lo;
+    const size_t need = moe_ffn_partial_workspace_size(T, H, E_band, top_k, I);
+    if (workspace == nullptr || workspace_bytes < need || need == 0)
+        return fail(EP_ENOMEM, "moe_ffn_partial: workspace of %zu bytes, %zu needed",
+                    workspace_bytes, need);
+    if (!aligned(workspace, 256))
+        return fail(EP_EINVAL, "moe_ffn_partial: workspace not 256-byte aligned");
+    const size_t ids_off = partial_ids_offset(T, H, E_band, top_k, I);
+    int32_t *local = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) + ids_off);
+    const DeviceInfo *d = nullptr;
+    ep_status s = device_info(&d);
+    if (s != EP_OK)
+        return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t n = T * top_k;
+    {
+        const unsigned blocks = (unsigned)std::min<int64_t>((n + 255) / 256, (int64_t)d->sm_count * 4);
+        EP_CUDA_CHECK(launch(epk::ep_band_ids_kernel, dim3(blocks), 256, 0, st, ids, n, (int32_t)E,
+                             e_lo, e_hi, local));
+    }
+    // the band's picks through the single-band forward, without the shared expert
+    ep_plan_t band;
+    memset(&band, 0, sizeof band);
+    band.num_experts = (int32_t)E_band;
+    band.bands = 1;
+    band.band_start[0] = 0;
+    band.band_start[1] = (int32_t)E_band;
+    s = ffn_forward_impl(true, x, x_dtype, T, H, local, weights, top_k, w_gate, w_up, w_down,
+                         E_band, I, nullptr, nullptr, nullptr, 0, &band, partial, workspace,
+                         ids_off, stream);
+    if (s != EP_OK)
+        return s;
+    t_launches += 1;
+    return ok();
+}
+
+extern "C" ep_status moe_ep_combine(const float *partials, int64_t T, int64_t H,
+                                    const int32_t *ids, int32_t top_k, const ep_plan_t *plan,
+                                    const float *shared, float *y, void *stream) {
+    if (plan == nullptr)
+        return fail(EP_EINVAL, "moe_ep_combine: plan is NULL");
+    const int64_t E = plan->num_experts;
+    if (E < 1 || plan->bands < 1 || plan->bands > EP_MAX_BANDS || plan->bands > E ||
+        plan->band_start[0] != 0 || plan->band_start[plan->bands] != E)
+        return fail(EP_EINVAL, "moe_ep_combine: plan is not a partition of [0, E)");
+    for (int r = 0; r < plan->bands; ++r)
+        if (plan->band_start[r + 1] <= plan->band_start[r])
+            return fail(EP_EINVAL, "moe_ep_combine: band %d of the plan is empty or reversed", r);
+    if (T < 0 || T > kMaxT || H < 1 || H > kMaxH || top_k < 1 || top_k > kMaxTopK)
+        return fail(EP_EINVAL, "moe_ep_combine: T = %lld, H = %lld or top_k = %d out of range",
+                    (long long)T, (long long)H, top_k);
+    if (T == 0) {
+        t_launches = 0;
+        return ok();
+    }
+    if (partials == nullptr || ids == nullptr || y == nullptr)
+        return fail(EP_EINVAL, "moe_ep_combine: a required pointer is NULL");
+    if (!aligned(partials, 4) || !aligned(ids, 4) || !aligned(y, 4) ||
+        (shared != nullptr && !aligned(shared, 4)))
+        return fail(EP_EINVAL, "moe_ep_combine: misaligned pointer");
+    const DeviceInfo *d = nullptr;
+    const ep_status s = device_info(&d);
+    if (s != EP_OK)
+        return s;
+    epk::EpBands bands;
+    memset(&bands, 0, sizeof bands);
+    for (int r = 0; r <= plan->bands; ++r)
+        bands.start[r] = plan->band_start[r];
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const dim3 grid((unsigned)((H + epk::kEpCombineThreads - 1) / epk::kEpCombineThreads),
+                    (unsigned)T);
+    EP_CUDA_CHECK(launch(epk::ep_combine_kernel, grid, epk::kEpCombineThreads, 0, st, partials, T,
+                         (int)H, ids, top_k, (int)E, bands, plan->bands, shared, y));
+    t_launches = 1;
     return ok();
 }
 

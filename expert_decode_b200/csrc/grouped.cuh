@@ -153,7 +153,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) group_plan_kernel(const PlanA
         if (p < p_hi) {
             e = a.ids[p];
             valid = e >= 0 && e < E;
-            if (!valid)
+            if (!valid && e != kIdNone)
                 flag_status(kStatusBadId);
         }
         const int key = valid ? e : -(lane + 2);

@@ -71,7 +71,7 @@ __device__ void build_stream_plan(StreamPlan &P, const int32_t *__restrict__ ids
             for (int q = 0; q < j; ++q)
                 rep += ids[t * k + q] == e;
             key = (e * kStreamMaxK + rep) * kStreamMaxT + t;
-        } else {
+        } else if (e != kIdNone) {
             flag_status(kStatusBadId);
         }
     }

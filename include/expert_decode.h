@@ -200,6 +200,56 @@ ep_status moe_ffn_forward_noalloc(const void *x, ep_dtype x_dtype, int64_t T, in
                                   int64_t I_s, const ep_plan_t *plan, float *y, void *stream);
 
 /*
+ * EP_ID_NONE -- an empty pick slot.  A pick whose id is EP_ID_NONE is skipped
+ * by every call that takes ids and is not reported as a bad id (any other id
+ * outside [0, E) is skipped and reported).
+ */
+#define EP_ID_NONE ((int32_t)0x80000000)
+
+/*
+ * The expert-parallel form across ranks (fak note "GLM-5.2 multi-GPU", "What
+ * landed": contiguous bands of experts, every rank the partial of the picks
+ * in its band, the partials summed in rank order; TensorFold #310: one fixed
+ * order of that sum).
+ *
+ * moe_ffn_partial_workspace_size -- bytes of device workspace moe_ffn_partial
+ * needs with E_band experts in the band (0 for an empty input).
+ *
+ * moe_ffn_partial -- rank `rank`'s partial for every token:
+ *   partial[t] = fold over t's picks with expert ids in band `rank` of the
+ *                plan, in ascending (expert id, slot), starting from the first,
+ *                of weights[t,j] * f_e(x[t]);  0 when t has no pick in the band.
+ *   No shared expert (it enters after the rank-order sum, in moe_ep_combine).
+ *   The weights are band-resident: w_gate, w_up [E_band, I, H], w_down
+ *   [E_band, H, I] hold the band's experts only, expert e at index
+ *   e - plan->band_start[rank].  ids and weights as moe_ffn_forward, with the
+ *   global expert ids of the plan (ids of other bands are simply not this
+ *   rank's; ids outside [0, plan->num_experts) are skipped and reported).
+ *   partial device [T, H] fp32; workspace 256-byte aligned, at least
+ *   moe_ffn_partial_workspace_size(T, H, E_band, top_k, I) bytes.  Limits
+ *   and errors as moe_ffn_forward; rank outside [0, plan->bands) -> EP_EINVAL.
+ *
+ * moe_ep_combine -- y[t] = the partials of the bands that hold at least one of
+ *   t's valid picks, left-folded in rank order, + shared[t] (shared device
+ *   [T, H] fp32 or NULL).  A token without a valid pick gets shared[t] (or 0).
+ *   partials device [plan->bands][T][H] fp32 (rank r's partial at r); ids
+ *   device [T, top_k] int32; y device [T, H] fp32.  The result is the fp64
+ *   oracle's band form (expertParallelPartials + rank-order sum), which for
+ *   more than one band may differ in the last bits from moe_ffn_forward's one
+ *   fold with the carry passed along.
+ */
+size_t moe_ffn_partial_workspace_size(int64_t T, int64_t H, int64_t E_band, int32_t top_k,
+                                      int64_t I);
+ep_status moe_ffn_partial(const void *x, ep_dtype x_dtype, int64_t T, int64_t H,
+                          const int32_t *ids, const float *weights, int32_t top_k,
+                          const void *w_gate, const void *w_up, const void *w_down, int64_t I,
+                          const ep_plan_t *plan, int32_t rank, float *partial, void *workspace,
+                          size_t workspace_bytes, void *stream);
+ep_status moe_ep_combine(const float *partials, int64_t T, int64_t H, const int32_t *ids,
+                         int32_t top_k, const ep_plan_t *plan, const float *shared, float *y,
+                         void *stream);
+
+/*
  * Which moe_ffn_forward path runs.  EP_DISPATCH_AUTO (the default) takes the
  * weight-streaming path for T <= 8 when its on-chip buffers fit, else the
  * tensor-core path.  Forcing a path that does not fit the sizes makes
