@@ -129,6 +129,17 @@ __device__ __forceinline__ double dot2_warp_total(float2 s, float2 c) {
     return (double)S + (double)C;
 }
 
+// An fp64 value and an expert id as one unsigned key that orders by value,
+// then by lower id: the value's bits made order-preserving as an unsigned
+// integer, with the lowest 10 bits replaced by 1023 - id.  Values closer than
+// about 2^-42 of their size (far inside the Dot2 logits' error bound) are
+// thereby ordered by id, as exact ties are.  E <= 1024.
+__device__ __forceinline__ unsigned long long topk_key(double v, int e) {
+    const unsigned long long b = (unsigned long long)__double_as_longlong(v);
+    const unsigned long long ord = (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+    return (ord & ~0x3ffull) | (unsigned long long)(1023 - e);
+}
+
 // One warp: the top_k of E values of one token by value, ties to the lower
 // id; lane r < top_k receives the r-th pick's id and value.
 __device__ void topk_select_warp(const double *v, int E, int top_k, int &pick_e, double &pick_v) {
@@ -138,26 +149,25 @@ __device__ void topk_select_warp(const double *v, int E, int top_k, int &pick_e,
     pick_v = 0.0;
     pick_e = 0;
     for (int r = 0; r < top_k; ++r) {
-        double bv = -INFINITY;
-        int be = 0x7fffffff;
+        unsigned long long best = 0ull;  // below every key of a finite value
         for (int i = 0; i < per_lane; ++i) {
             const int e = lane + 32 * i;
             if (e < E && !((chosen >> i) & 1u)) {
-                const double x = v[e];
-                if (x > bv || (x == bv && e < be)) { bv = x; be = e; }
+                const unsigned long long k = topk_key(v[e], e);
+                best = k > best ? k : best;
             }
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
-            const double ov = __shfl_xor_sync(0xffffffffu, bv, off);
-            const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-            if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+            const unsigned long long o = __shfl_xor_sync(0xffffffffu, best, off);
+            best = o > best ? o : best;
         }
-        if (be != 0x7fffffff && (be & 31) == lane)
+        const int be = 1023 - (int)(best & 0x3ffull);
+        if ((be & 31) == lane)
             chosen |= 1u << (be >> 5);
         if (lane == r) {
-            pick_v = bv;
             pick_e = be;
+            pick_v = v[be];
         }
     }
 }
