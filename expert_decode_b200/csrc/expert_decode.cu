@@ -344,7 +344,7 @@ int max_active_clusters(const void *fn, int csize, uint32_t smem) {
         int value;
     };
     static std::mutex mu;
-    static Entry cache[64];
+    static Entry cache[128];
     static int n_cache = 0;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess)
@@ -370,7 +370,7 @@ int max_active_clusters(const void *fn, int csize, uint32_t smem) {
         (void)cudaGetLastError();
         n = 0;
     }
-    if (n_cache < 64)
+    if (n_cache < 128)
         cache[n_cache++] = Entry{fn, dev, csize, smem, n};
     return n;
 }
