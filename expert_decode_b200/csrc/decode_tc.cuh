@@ -4,23 +4,27 @@
 // Same contraction as stream_gate_up_kernel (h = silu(W_gate x) * (W_up x)
 // for every picked expert and the shared expert; fak note "GLM-5.2
 // multi-GPU", expertSwiGLU), laid out for tcgen05: a tile is 64 units of I,
-// i.e. 128 weight rows on the MMA's M side with 16 W_gate rows and 16 W_up
-// rows interleaved (TensorFold #593's packGateUp), and all T <= 8 tokens on
-// its N side (N = 16; the tensor map zero-fills the rows after T).  Every
+// i.e. 128 weight rows on the MMA's M side, the 64 W_gate rows over the 64
+// W_up rows of the same units (TensorFold #593's packGateUp operand), and all
+// T <= 8 tokens on its N side (N = 16; the tensor map zero-fills the rows
+// after T).  Every
 // tile therefore computes every token, and the epilogue keeps the tokens
 // that picked the tile's expert, so no activation gather is needed.
 //
 // Persistent and warp specialised, one CTA per SM:
-//   warp 0     TMA producer: per 64-wide k block the A tile (8 boxes of 16
+//   warp 0     TMA producer: per 64-wide k block the A tile (two boxes of 64
 //              weight rows, 16 KB) and the x tile (16 rows, 2 KB) into a
-//              ring of kTcStages stages, 128-byte swizzle, no multicast;
+//              ring of kTcStages stages, 128-byte swizzle, no multicast: three
+//              copy instructions per stage, as few as the operands allow;
 //   warp 1     tcgen05.mma issuer (M = 128, N = 16, K = 16 per instruction),
 //              fp32 accumulators in TMEM, two of them so that the epilogue
 //              of one tile overlaps the MMAs of the next;
 //   warps 2-5  build the expert grouping from ids (the streaming plan), then
-//              drain each accumulator with tcgen05.ld: lanes l and l + 16 of a
-//              warp hold g and u of the same unit, h = silu(g) * u is written
-//              in fp32, in the layout the down kernel reads.
+//              drain each accumulator with tcgen05.ld: the warps of TMEM
+//              quarters 2 and 3 (up rows) pass their values through shared
+//              memory to those of quarters 0 and 1 (gate rows of the same
+//              units), which write h = silu(g) * u in fp32, in the layout the
+//              down kernel reads.
 // Tiles go round-robin over the CTAs: the shared expert's first, then each
 // routed group's in ascending expert id.
 #pragma once
@@ -39,11 +43,12 @@ constexpr uint32_t kTcBBytes = kTcN * kGemmBK * 2;         // 16 token rows, 2 K
 constexpr uint32_t kTcStageBytes = kTcABytes + kTcBBytes;  // 18 KB, a multiple of 1024
 constexpr int kTcTmemCols = 2 * kTcN;                      // two accumulators
 constexpr uint32_t kTcBarPlan = 1;                         // named barrier of the epilogue warps
+constexpr uint32_t kTcBarPair = 2;                         // + pair: the two warps of one pair
 constexpr int kTcMaxGroups = kStreamMaxPairs + 1;          // routed groups + the shared expert
 
 struct TcMaps {
-    CUtensorMap wg, wu;  // W_gate, W_up [E, I, H]: box 64 x 16 x 1
-    CUtensorMap sg, su;  // shared expert [I_s, H]: box 64 x 16
+    CUtensorMap wg, wu;  // W_gate, W_up [E, I, H]: box 64 x 64 x 1
+    CUtensorMap sg, su;  // shared expert [I_s, H]: box 64 x 64
     CUtensorMap x;       // activations [T, H]: box 64 x 16
 };
 
@@ -61,7 +66,9 @@ struct TcSmem {
     // full[S], empty[S], tfull[2], tempty[2], drain, planbar; tmem holder, abort flag
     static constexpr uint32_t misc = bars + (2 * kTcStages + 6) * 8;
     static constexpr uint32_t tile_first = misc + 16;  // [kTcMaxGroups + 1]
-    static constexpr uint32_t plan = (tile_first + (kTcMaxGroups + 1) * 4 + 127) / 128 * 128;
+    // up values handed to the gate warps: [pair][accumulator][token][lane]
+    static constexpr uint32_t xchg = (tile_first + (kTcMaxGroups + 1) * 4 + 15) / 16 * 16;
+    static constexpr uint32_t plan = (xchg + 2 * 2 * kStreamMaxT * 32 * 4 + 127) / 128 * 128;
     static constexpr uint32_t total = plan + (uint32_t)sizeof(StreamPlan);
     static constexpr uint32_t alloc = total + 1024;  // room to align the base to 1024
 };
@@ -90,6 +97,7 @@ stream_gate_up_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + TcSmem::misc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + TcSmem::misc + 8);
     int *tile_first = reinterpret_cast<int *>(smem + TcSmem::tile_first);
+    float *xchg = reinterpret_cast<float *>(smem + TcSmem::xchg);
     StreamPlan &P = *reinterpret_cast<StreamPlan *>(smem + TcSmem::plan);
 
     const int warp = (int)(threadIdx.x >> 5);
@@ -164,16 +172,14 @@ stream_gate_up_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
                     uint8_t *sb = sa + kTcABytes;
                     mbar_arrive_expect_tx(&full[stage], kTcStageBytes);
                     const int k0 = kb * kGemmBK;
-#pragma unroll
-                    for (int j = 0; j < kGemmBM / kBoxRowsA; ++j) {
-                        const bool up = j & 1;
-                        const int row = m0 + (j >> 1) * kBoxRowsA;
-                        uint8_t *dst = sa + j * kBoxRowsA * kGemmBK * 2;
-                        if (shared)
-                            tma_load_2d(dst, up ? &maps.su : &maps.sg, k0, row, &full[stage], pol_w);
-                        else
-                            tma_load_3d(dst, up ? &maps.wu : &maps.wg, k0, row, e, &full[stage],
-                                        pol_w);
+                    // rows 0..63: W_gate of the tile's units, 64..127: W_up
+                    uint8_t *sa_up = sa + kGateUpRows * kGemmBK * 2;
+                    if (shared) {
+                        tma_load_2d(sa, &maps.sg, k0, m0, &full[stage], pol_w);
+                        tma_load_2d(sa_up, &maps.su, k0, m0, &full[stage], pol_w);
+                    } else {
+                        tma_load_3d(sa, &maps.wg, k0, m0, e, &full[stage], pol_w);
+                        tma_load_3d(sa_up, &maps.wu, k0, m0, e, &full[stage], pol_w);
                     }
                     tma_load_2d(sb, &maps.x, k0, 0, &full[stage], pol_x);
                     ++issued;
@@ -248,32 +254,47 @@ stream_gate_up_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
             tile_first[G] = t;
             mbar_arrive(planbar);  // release: the plan and the tile table are written
         }
-        if (mbar_wait(planbar, 0, abort_flag)) {
+        // the planning warps agree on the plan wait, so the pairs below either
+        // all enter the tile loop or none does
+        const bool planned =
+            named_count(kTcBarPlan, 128, mbar_wait(planbar, 0, abort_flag)) == 128;
+        if (planned) {
             const int q = warp & 3;  // TMEM lane quarter this warp may access
+            // quarters 0, 1: gate rows of units 0..31, 32..63; 2, 3: their up rows
+            const bool gate_warp = q < 2;
+            const int pair = q & 1;
             const int total = tile_first[has_shared + P.n_groups];
             uint32_t acc = 0, acc_phase = 0;
             for (int u = blockIdx.x; u < total; u += gridDim.x) {
                 int gi, m0;
                 decode(u, gi, m0);
                 const bool shared = gi < has_shared;
-                if (!mbar_wait(&tfull[acc], acc_phase, abort_flag))
+                // the two warps of a pair leave together or not at all
+                const bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag);
+                if (named_count(kTcBarPair + pair, 64, ok) != 64)
                     break;
                 tc_fence_after_sync();
                 uint32_t v[16];
                 tmem_load_16cols(tmem_base + ((uint32_t)(32 * q) << 16) + acc * kTcN, v);
                 tmem_load_wait();
-                // lanes 0..15 hold gate rows, 16..31 the up rows of the same units
-                const int unit = m0 + 16 * q + (lane & 15);
-                const bool is_gate = lane < 16;
-                if (shared) {
+                // [token][lane] of this pair and accumulator; a buffer is written
+                // again two tiles later, after the pair's next barrier, which the
+                // gate warp reaches only once it has read this one
+                float *xb = xchg + (pair * 2 + acc) * kStreamMaxT * 32;
+                if (!gate_warp) {
 #pragma unroll
-                    for (int t = 0; t < kStreamMaxT; ++t) {
-                        const float other = __shfl_xor_sync(0xffffffffu, __uint_as_float(v[t]), 16);
-                        if (is_gate && t < a.T && unit < a.I_s)
+                    for (int t = 0; t < kStreamMaxT; ++t)
+                        xb[t * 32 + lane] = __uint_as_float(v[t]);
+                }
+                named_sync(kTcBarPair + pair, 64);
+                const int unit = m0 + 32 * pair + lane;
+                if (gate_warp && shared) {
+#pragma unroll
+                    for (int t = 0; t < kStreamMaxT; ++t)
+                        if (t < a.T && unit < a.I_s)
                             a.h_shared[(size_t)t * a.I_s + unit] =
-                                silu_f32(__uint_as_float(v[t])) * other;
-                    }
-                } else {
+                                silu_f32(__uint_as_float(v[t])) * xb[t * 32 + lane];
+                } else if (gate_warp) {
                     const int g = gi - has_shared;
                     const int first = P.group_first[g];
                     const int cnt = P.group_first[g + 1] - first;
@@ -283,9 +304,9 @@ stream_gate_up_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
 #pragma unroll
                         for (int t = 0; t < kStreamMaxT; ++t)
                             mine = t == tok ? __uint_as_float(v[t]) : mine;
-                        const float other = __shfl_xor_sync(0xffffffffu, mine, 16);
-                        if (is_gate && unit < a.I)
-                            a.h_routed[(size_t)(first + j) * a.I + unit] = silu_f32(mine) * other;
+                        if (unit < a.I)
+                            a.h_routed[(size_t)(first + j) * a.I + unit] =
+                                silu_f32(mine) * xb[tok * 32 + lane];
                     }
                 }
                 tc_fence_before_sync();

@@ -626,12 +626,12 @@ ep_status ffn_forward_impl(bool band_call, const void *x, ep_dtype x_dtype, int6
                      epk::tensor_map_encoder() != nullptr;
         if (tc_ok && mode != EP_DISPATCH_STREAMING_SIMT &&
             (mode == EP_DISPATCH_STREAMING_TC || T >= kTcMinT)) {
-            tc_ok = epk::map_3d(&tm.wg, w_gate, H, I, E, epk::kBoxRowsA) &&
-                    epk::map_3d(&tm.wu, w_up, H, I, E, epk::kBoxRowsA) &&
+            tc_ok = epk::map_3d(&tm.wg, w_gate, H, I, E, epk::kGateUpRows) &&
+                    epk::map_3d(&tm.wu, w_up, H, I, E, epk::kGateUpRows) &&
                     epk::map_2d(&tm.x, x, H, T, epk::kTcN);
             if (I_s > 0)
-                tc_ok = tc_ok && epk::map_2d(&tm.sg, ws_gate, H, I_s, epk::kBoxRowsA) &&
-                        epk::map_2d(&tm.su, ws_up, H, I_s, epk::kBoxRowsA);
+                tc_ok = tc_ok && epk::map_2d(&tm.sg, ws_gate, H, I_s, epk::kGateUpRows) &&
+                        epk::map_2d(&tm.su, ws_up, H, I_s, epk::kGateUpRows);
         }
         bool use_tc;
         if (mode == EP_DISPATCH_STREAMING_TC) {

@@ -9,11 +9,12 @@
 //  2. gather_rows:  the picked activation rows, expert by expert, as bf16,
 //                   followed by every token's row for the shared expert.
 //  3. grouped GEMM, gate/up: per (expert, 64 units of I, up to 256 rows) tile
-//                   one 128-row tcgen05 MMA stack whose A tile interleaves 16
-//                   W_gate rows and 16 W_up rows (the fused gate/up row of
-//                   TensorFold #593's packGateUp), so that a warp's lanes l and
-//                   l + 16 hold g and u of the same unit; the epilogue forms
-//                   h = silu(g) * u and rounds it to bf16.
+//                   one 128-row tcgen05 MMA stack whose A tile stacks 64
+//                   W_gate rows over the 64 W_up rows of the same units (the
+//                   fused gate/up operand of TensorFold #593's packGateUp),
+//                   loaded as two boxes; the epilogue warp holding a unit's g
+//                   and the one holding its u swap half their columns through
+//                   shared memory, form h = silu(g) * u and round it to bf16.
 //  4. grouped GEMM, down: per (expert, 128 output features, up to 256 rows)
 //                   tile; the epilogue scales by the routing weight and writes
 //                   each pick's fp32 contribution to its (token, slot) row.
@@ -44,8 +45,11 @@ constexpr int kGemmBK = 64;
 constexpr int kGemmStages = 4;
 constexpr int kGemmThreads = 192;
 constexpr int kGateUpRows = 64;  // units of I per gate/up tile (64 gate + 64 up rows)
-constexpr int kBoxRowsA = 16;    // gate/up A tile is loaded 16 rows at a time
-constexpr int kBoxRowsB = 32;
+// The activation tile is one box per stage, of the smallest of these heights
+// (capped at the tensor's rows rounded up to 32) that covers the tile's rows:
+// one copy instruction instead of one per 32 rows.
+constexpr int kBoxLevels = 4;
+constexpr int kBoxRowsB[kBoxLevels] = {32, 64, 128, 256};
 constexpr uint32_t kTileABytes = kGemmBM * kGemmBK * 2;
 constexpr uint32_t kTileBBytes = kGemmBN * kGemmBK * 2;
 constexpr uint32_t kStageBytes = kTileABytes + kTileBBytes;
@@ -294,7 +298,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const void *__restrict
 struct GemmMaps {
     CUtensorMap a, a2;               // routed weights (gate/up: W_gate, W_up; down: W_down)
     CUtensorMap a_shared, a2_shared; // shared expert weights
-    CUtensorMap b, b_shared;         // activations (routed rows, shared rows)
+    CUtensorMap b[kBoxLevels];       // activations of the routed rows, one map per box height
+    CUtensorMap b_shared[kBoxLevels];  // the shared expert's rows (down only)
 };
 
 struct GemmParams {
@@ -309,6 +314,7 @@ struct GemmParams {
     int I, I_s;
     float *c_out, *s_out;             // down outputs
     int H;
+    int b_rows[kBoxLevels], bs_rows[kBoxLevels];  // box heights of maps.b and maps.b_shared
 };
 
 struct GemmSmem {
@@ -356,7 +362,8 @@ grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tensormap(&maps.a);
-        prefetch_tensormap(&maps.b);
+        for (int l = 0; l < kBoxLevels; ++l)
+            prefetch_tensormap(&maps.b[l]);
     }
     if (warp == 1) {
         tmem_alloc(tmem_holder, kTmemCols);
@@ -406,13 +413,18 @@ grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
                 const int K = shared ? p.k_shared : p.k_routed;
                 const int n0 = nb * kGemmBN;
                 const int n_valid = min(kGemmBN, rows - n0);
-                const int n_loads = (n_valid + kBoxRowsB - 1) / kBoxRowsB;
                 int brow;
                 if (GATE_UP)
                     brow = (shared ? (int)p.P : offsets[g]) + n0;
                 else
                     brow = (shared ? 0 : offsets[g]) + n0;
-                const CUtensorMap *bmap = (!GATE_UP && shared) ? &maps.b_shared : &maps.b;
+                const bool bs = !GATE_UP && shared;
+                const int *box_rows = bs ? p.bs_rows : p.b_rows;
+                int lvl = 0;
+                while (lvl + 1 < kBoxLevels && box_rows[lvl] < n_valid)
+                    ++lvl;
+                const CUtensorMap *bmap = bs ? &maps.b_shared[lvl] : &maps.b[lvl];
+                const uint32_t b_bytes = (uint32_t)box_rows[lvl] * kGemmBK * 2;
                 const int kblocks = (K + kGemmBK - 1) / kGemmBK;
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
@@ -421,20 +433,18 @@ grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
                     }
                     uint8_t *sa = smem + stage * kStageBytes;
                     uint8_t *sb = sa + kTileABytes;
-                    mbar_arrive_expect_tx(&full[stage],
-                                          kTileABytes + (uint32_t)n_loads * kBoxRowsB * kGemmBK * 2);
+                    mbar_arrive_expect_tx(&full[stage], kTileABytes + b_bytes);
                     const int k0 = kb * kGemmBK;
                     if (GATE_UP) {
-                        for (int j = 0; j < kGemmBM / kBoxRowsA; ++j) {
-                            const bool up = j & 1;
-                            const int row = mb * kGateUpRows + (j >> 1) * kBoxRowsA;
-                            uint8_t *dst = sa + j * kBoxRowsA * kGemmBK * 2;
-                            if (shared)
-                                tma_load_2d(dst, up ? &maps.a2_shared : &maps.a_shared, k0, row,
-                                            &full[stage], pol_w);
-                            else
-                                tma_load_3d(dst, up ? &maps.a2 : &maps.a, k0, row, g,
-                                            &full[stage], pol_w);
+                        // rows 0..63: W_gate of the tile's 64 units, 64..127: W_up
+                        const int row = mb * kGateUpRows;
+                        uint8_t *sa_up = sa + kGateUpRows * kGemmBK * 2;
+                        if (shared) {
+                            tma_load_2d(sa, &maps.a_shared, k0, row, &full[stage], pol_w);
+                            tma_load_2d(sa_up, &maps.a2_shared, k0, row, &full[stage], pol_w);
+                        } else {
+                            tma_load_3d(sa, &maps.a, k0, row, g, &full[stage], pol_w);
+                            tma_load_3d(sa_up, &maps.a2, k0, row, g, &full[stage], pol_w);
                         }
                     } else {
                         if (shared)
@@ -442,9 +452,7 @@ grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
                         else
                             tma_load_3d(sa, &maps.a, k0, mb * kGemmBM, g, &full[stage], pol_w);
                     }
-                    for (int q = 0; q < n_loads; ++q)
-                        tma_load_2d(sb + q * kBoxRowsB * kGemmBK * 2, bmap, k0, brow + q * kBoxRowsB,
-                                    &full[stage], pol_x);
+                    tma_load_2d(sb, bmap, k0, brow, &full[stage], pol_x);
                     ++issued;
                     if (++stage == kGemmStages) {
                         stage = 0;
@@ -511,6 +519,15 @@ grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         int *col_pick = reinterpret_cast<int *>(smem + GemmSmem::colmeta) + (warp - 2) * 2 * kGemmBN;
         float *col_w = reinterpret_cast<float *>(col_pick + kGemmBN);
+        // gate/up: quarters 0, 1 hold the gate rows of units 0..31, 32..63 and
+        // quarters 2, 3 the up rows of the same units; the two warps of a pair
+        // (same units) swap half their columns through the colmeta area, which
+        // gate/up does not otherwise use: xg = gate values of columns 16..31,
+        // xu = up values of columns 0..15, each [16][32 lanes]
+        const bool gate_warp = q < 2;
+        const int pair = q & 1;
+        float *xg = reinterpret_cast<float *>(smem + GemmSmem::colmeta) + pair * 2 * 16 * 32;
+        float *xu = xg + 16 * 32;
         uint32_t acc = 0, acc_phase = 0;
         for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
             int g, mb, nb, rows, n_blocks;
@@ -528,7 +545,12 @@ grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
                 }
                 __syncwarp();
             }
-            if (!mbar_wait(&tfull[acc], acc_phase, abort_flag))
+            bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag);
+            // the two warps of a pair leave together or not at all (their
+            // exchange below synchronises on a named barrier)
+            if (GATE_UP)
+                ok = named_count(1 + pair, 64, ok) == 64;
+            if (!ok)
                 break;
             tc_fence_after_sync();
             const uint32_t t_row = tmem_base + ((uint32_t)(32 * q) << 16) + acc * kGemmBN;
@@ -537,27 +559,41 @@ grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
                 tmem_load_32cols(t_row + (uint32_t)c0, v);
                 tmem_load_wait();
                 if (GATE_UP) {
-                    // lanes 0..15 hold gate rows, 16..31 the up rows of the same units
+                    // lane = unit; the gate warp finishes columns 0..15 of the
+                    // chunk, the up warp columns 16..31
                     const int M = shared ? p.I_s : p.I;
-                    const int unit = mb * kGateUpRows + 16 * q + (lane & 15);
-                    const bool is_gate = lane < 16;
+                    const int unit = mb * kGateUpRows + 32 * pair + lane;
                     uint16_t *hrow_base = shared ? p.h_shared_out : p.h_out;
                     const int ld = shared ? p.I_s : p.I;
                     const int64_t row0 = (shared ? 0 : offsets[g]) + n0 + c0;
+                    if (gate_warp) {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const float mine = __uint_as_float(v[j]);
-                        const float other = __shfl_xor_sync(0xffffffffu, mine, 16);
-                        // lanes 0..15 finish columns 0..15, lanes 16..31 columns 16..31
-                        if ((j < 16) == is_gate) {
-                            const float gv = is_gate ? mine : other;
-                            const float uv = is_gate ? other : mine;
+                        for (int j = 0; j < 16; ++j)
+                            xg[j * 32 + lane] = __uint_as_float(v[16 + j]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            xu[j * 32 + lane] = __uint_as_float(v[j]);
+                    }
+                    named_sync(1 + pair, 64);
+                    if (gate_warp) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
                             const int col = c0 + j;
                             if (col < n_valid && unit < M)
-                                hrow_base[(size_t)(row0 + j) * ld + unit] =
-                                    f32_to_bf16_rne(silu_f32(gv) * uv);
+                                hrow_base[(size_t)(row0 + j) * ld + unit] = f32_to_bf16_rne(
+                                    silu_f32(__uint_as_float(v[j])) * xu[j * 32 + lane]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int col = c0 + 16 + j;
+                            if (col < n_valid && unit < M)
+                                hrow_base[(size_t)(row0 + 16 + j) * ld + unit] = f32_to_bf16_rne(
+                                    silu_f32(xg[j * 32 + lane]) * __uint_as_float(v[16 + j]));
                         }
                     }
+                    named_sync(1 + pair, 64);  // the buffers are free for the next chunk
                 } else {
                     const int row = mb * kGemmBM + 32 * q + lane;
                     if (row < p.H) {
@@ -707,6 +743,19 @@ inline bool map_3d(CUtensorMap *m, const void *base, uint64_t cols, uint64_t row
     return make_map(m, base, 3, dims, strides, box_rows);
 }
 
+// The activation maps of every box height; a height is capped at the rows
+// rounded up to 32, so that no box is taller than the tensor needs.
+inline bool map_b_levels(CUtensorMap *maps, int *box_rows, const void *base, uint64_t cols,
+                         int64_t rows) {
+    const int64_t cap = (rows + 31) / 32 * 32;
+    for (int l = 0; l < kBoxLevels; ++l) {
+        box_rows[l] = (int)std::min<int64_t>(kBoxRowsB[l], cap);
+        if (!map_2d(&maps[l], base, cols, (uint64_t)rows, (uint32_t)box_rows[l]))
+            return false;
+    }
+    return true;
+}
+
 inline size_t plan_smem_bytes(int64_t E) { return (size_t)(kPlanWarps * E + 2 * E + 65) * 4; }
 
 inline ep_status grouped_set_attributes(int smem_optin) {
@@ -786,18 +835,18 @@ inline ep_status grouped_forward(const GroupedArgs &g, const GroupedWorkspace &W
     // 3. gate/up
     GemmMaps gm;
     memset(&gm, 0, sizeof gm);
-    bool okm = map_3d(&gm.a, g.w_gate, H, I, E, kBoxRowsA) &&
-               map_3d(&gm.a2, g.w_up, H, I, E, kBoxRowsA) &&
-               map_2d(&gm.b, x_perm, H, P + T, kBoxRowsB);
+    GemmParams gp;
+    memset(&gp, 0, sizeof gp);
+    bool okm = map_3d(&gm.a, g.w_gate, H, I, E, kGateUpRows) &&
+               map_3d(&gm.a2, g.w_up, H, I, E, kGateUpRows) &&
+               map_b_levels(gm.b, gp.b_rows, x_perm, H, P + T);
     if (I_s > 0)
-        okm = okm && map_2d(&gm.a_shared, g.ws_gate, H, I_s, kBoxRowsA) &&
-              map_2d(&gm.a2_shared, g.ws_up, H, I_s, kBoxRowsA);
+        okm = okm && map_2d(&gm.a_shared, g.ws_gate, H, I_s, kGateUpRows) &&
+              map_2d(&gm.a2_shared, g.ws_up, H, I_s, kGateUpRows);
     if (!okm) {
         snprintf(why, why_len, "encoding a gate/up tensor map failed");
         return EP_ECUDA;
     }
-    GemmParams gp;
-    memset(&gp, 0, sizeof gp);
     gp.E = (int)E; gp.G = G; gp.T = T; gp.P = P; gp.top_k = k;
     gp.m_routed = (int)I; gp.m_shared = (int)I_s; gp.k_routed = (int)H; gp.k_shared = (int)H;
     gp.group_offset = group_offset; gp.units = units_gu; gp.perm_pair = perm_pair;
@@ -813,10 +862,11 @@ inline ep_status grouped_forward(const GroupedArgs &g, const GroupedWorkspace &W
     }
     // 4. down
     memset(&gm, 0, sizeof gm);
-    okm = map_3d(&gm.a, g.w_down, I, H, E, kGemmBM) && map_2d(&gm.b, h_perm, I, std::max<int64_t>(P, 1), kBoxRowsB);
+    okm = map_3d(&gm.a, g.w_down, I, H, E, kGemmBM) &&
+          map_b_levels(gm.b, gp.b_rows, h_perm, I, std::max<int64_t>(P, 1));
     if (I_s > 0)
         okm = okm && map_2d(&gm.a_shared, g.ws_down, I_s, H, kGemmBM) &&
-              map_2d(&gm.b_shared, h_shared, I_s, T, kBoxRowsB);
+              map_b_levels(gm.b_shared, gp.bs_rows, h_shared, I_s, T);
     if (!okm) {
         snprintf(why, why_len, "encoding a down tensor map failed");
         return EP_ECUDA;
