@@ -58,7 +58,26 @@ struct TcArgs {
     const float *weights;
     float *h_routed;  // [pairs, I] in plan order
     float *h_shared;  // [T, I_s]
+    // When set, h goes out instead as bf16 hi/lo pairs for the tensor-core
+    // down projection, in hb_routed [2 * pairs + 16][I]: a group of cnt picks
+    // takes 2 cnt rows, cut into slices of up to 8 picks; a slice of n picks
+    // at row b holds hi(h) of its picks in rows b .. b+n-1 and lo(h) =
+    // h - hi(h) in rows b+n .. b+2n-1.  The shared expert's T tokens likewise
+    // in hb_shared [16][I_s] (hi in rows 0..T-1, lo in T..2T-1).
+    uint16_t *hb_routed;
+    uint16_t *hb_shared;
 };
+
+constexpr int kTcSlice = 8;  // picks per slice of the bf16 hi/lo activations
+
+// h as the two bf16 parts hi = bf16(h), lo = bf16(h - hi): together they
+// carry h to about 16 significant bits, so that a bf16 x bf16 contraction of
+// both parts loses next to nothing against fp32 h.
+__device__ __forceinline__ void store_hi_lo(uint16_t *hi_p, uint16_t *lo_p, float h) {
+    const uint16_t hi = f32_to_bf16_rne(h);
+    *hi_p = hi;
+    *lo_p = f32_to_bf16_rne(h - __uint_as_float((uint32_t)hi << 16));
+}
 
 struct TcSmem {
     static constexpr uint32_t stages = 0;
@@ -66,8 +85,9 @@ struct TcSmem {
     // full[S], empty[S], tfull[2], tempty[2], drain, planbar; tmem holder, abort flag
     static constexpr uint32_t misc = bars + (2 * kTcStages + 6) * 8;
     static constexpr uint32_t tile_first = misc + 16;  // [kTcMaxGroups + 1]
+    static constexpr uint32_t row_first = tile_first + (kTcMaxGroups + 1) * 4;  // [kTcMaxGroups]
     // up values handed to the gate warps: [pair][accumulator][token][lane]
-    static constexpr uint32_t xchg = (tile_first + (kTcMaxGroups + 1) * 4 + 15) / 16 * 16;
+    static constexpr uint32_t xchg = (row_first + kTcMaxGroups * 4 + 15) / 16 * 16;
     static constexpr uint32_t plan = (xchg + 2 * 2 * kStreamMaxT * 32 * 4 + 127) / 128 * 128;
     static constexpr uint32_t total = plan + (uint32_t)sizeof(StreamPlan);
     static constexpr uint32_t alloc = total + 1024;  // room to align the base to 1024
@@ -97,6 +117,7 @@ stream_gate_up_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + TcSmem::misc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + TcSmem::misc + 8);
     int *tile_first = reinterpret_cast<int *>(smem + TcSmem::tile_first);
+    int *row_first = reinterpret_cast<int *>(smem + TcSmem::row_first);  // per routed group
     float *xchg = reinterpret_cast<float *>(smem + TcSmem::xchg);
     StreamPlan &P = *reinterpret_cast<StreamPlan *>(smem + TcSmem::plan);
 
@@ -252,7 +273,9 @@ stream_gate_up_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
                 t += (width + kGateUpRows - 1) / kGateUpRows;
             }
             tile_first[G] = t;
-            mbar_arrive(planbar);  // release: the plan and the tile table are written
+            for (int g = 0; g < P.n_groups; ++g)
+                row_first[g] = 2 * P.group_first[g];  // 2 rows (hi, lo) per pick
+            mbar_arrive(planbar);  // release: the plan and the tile tables are written
         }
         // the planning warps agree on the plan wait, so the pairs below either
         // all enter the tile loop or none does
@@ -291,9 +314,14 @@ stream_gate_up_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
                 if (gate_warp && shared) {
 #pragma unroll
                     for (int t = 0; t < kStreamMaxT; ++t)
-                        if (t < a.T && unit < a.I_s)
-                            a.h_shared[(size_t)t * a.I_s + unit] =
-                                silu_f32(__uint_as_float(v[t])) * xb[t * 32 + lane];
+                        if (t < a.T && unit < a.I_s) {
+                            const float h = silu_f32(__uint_as_float(v[t])) * xb[t * 32 + lane];
+                            if (a.hb_shared != nullptr)
+                                store_hi_lo(a.hb_shared + (size_t)t * a.I_s + unit,
+                                            a.hb_shared + (size_t)(a.T + t) * a.I_s + unit, h);
+                            else
+                                a.h_shared[(size_t)t * a.I_s + unit] = h;
+                        }
                 } else if (gate_warp) {
                     const int g = gi - has_shared;
                     const int first = P.group_first[g];
@@ -304,9 +332,283 @@ stream_gate_up_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
 #pragma unroll
                         for (int t = 0; t < kStreamMaxT; ++t)
                             mine = t == tok ? __uint_as_float(v[t]) : mine;
-                        if (unit < a.I)
-                            a.h_routed[(size_t)(first + j) * a.I + unit] =
-                                silu_f32(mine) * xb[tok * 32 + lane];
+                        if (unit < a.I) {
+                            const float h = silu_f32(mine) * xb[tok * 32 + lane];
+                            if (a.hb_routed != nullptr) {
+                                const int j0 = j / kTcSlice * kTcSlice;
+                                const int n = min(kTcSlice, cnt - j0);
+                                const size_t b = (size_t)row_first[g] + 2 * j0;
+                                uint16_t *hb = a.hb_routed + unit;
+                                store_hi_lo(hb + (b + (j - j0)) * a.I,
+                                            hb + (b + n + (j - j0)) * a.I, h);
+                            } else {
+                                a.h_routed[(size_t)(first + j) * a.I + unit] = h;
+                            }
+                        }
+                    }
+                }
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&tempty[acc]);
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem_base, kTcTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// The down projection of the weight-streaming path on the tensor cores:
+// c[pick] = w * (W_down[e] h) for every pick, s[t] = Ws_down h_s[t] for the
+// shared expert.  A tile is 128 rows of W_down (the MMA's M side) against one
+// slice of n <= 8 picks of one expert, whose h enters as the bf16 parts hi
+// (B rows 0..n-1) and lo (rows n..2n-1) written by stream_gate_up_tc_kernel,
+// so that D[:, r] + D[:, n + r] is W_down h for pick r (the box's other rows
+// belong to the next slice and land in columns nobody reads).  Two copy instructions
+// per 64-wide k block (one 128-row weight box, one 16-row activation box).
+// The contributions are written per (token, slot) and folded afterwards by
+// combine_kernel in ascending (expert id, slot), then + s: the same fold as
+// the other paths.
+struct DtMaps {
+    CUtensorMap wd;  // W_down [E, H, I]: box 64 x 128 x 1
+    CUtensorMap sd;  // shared W_down [H, I_s]: box 64 x 128
+    CUtensorMap hr;  // routed h, bf16 hi/lo rows [2 * pairs + 16, I]: box 64 x 16
+    CUtensorMap hs;  // shared h [16, I_s] bf16: box 64 x 16
+};
+
+struct DtArgs {
+    int T, H, E, I, I_s, top_k;
+    const int32_t *ids;
+    const float *weights;
+    float *c;  // [T * top_k, H]: weighted contribution of pick t * top_k + j
+    float *s;  // [T, H]: the shared expert's output
+};
+
+struct DtSmem {
+    static constexpr uint32_t bars = kTcStages * kTcStageBytes;
+    // full[S], empty[S], tfull[2], tempty[2], drain, planbar; tmem holder, abort flag
+    static constexpr uint32_t misc = bars + (2 * kTcStages + 6) * 8;
+    static constexpr uint32_t slice_group = misc + 16;                        // [kStreamMaxPairs]
+    static constexpr uint32_t slice_j0 = slice_group + kStreamMaxPairs * 4;    // [kStreamMaxPairs]
+    static constexpr uint32_t n_slices = slice_j0 + kStreamMaxPairs * 4;
+    // a slice's first pair p0 = group_first[g] + j0 is also its first h row / 2
+    static constexpr uint32_t plan = (n_slices + 4 + 127) / 128 * 128;
+    static constexpr uint32_t total = plan + (uint32_t)sizeof(StreamPlan);
+    static constexpr uint32_t alloc = total + 1024;  // room to align the base to 1024
+};
+
+__global__ void __launch_bounds__(kTcThreads, 1)
+stream_down_tc_kernel(const __grid_constant__ DtMaps maps, const DtArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + DtSmem::bars);
+    uint64_t *empty = full + kTcStages;
+    uint64_t *tfull = empty + kTcStages;
+    uint64_t *tempty = tfull + 2;
+    uint64_t *drain = tempty + 2;
+    uint64_t *planbar = drain + 1;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + DtSmem::misc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + DtSmem::misc + 8);
+    int *slice_group = reinterpret_cast<int *>(smem + DtSmem::slice_group);
+    int *slice_j0 = reinterpret_cast<int *>(smem + DtSmem::slice_j0);
+    int *n_slices = reinterpret_cast<int *>(smem + DtSmem::n_slices);
+    StreamPlan &P = *reinterpret_cast<StreamPlan *>(smem + DtSmem::plan);
+
+    const int warp = (int)(threadIdx.x >> 5);
+    const int lane = (int)lane_id();
+    const int has_shared = a.I_s > 0 ? 1 : 0;
+    const int n_mb = (a.H + kGemmBM - 1) / kGemmBM;  // 128-row blocks of H
+
+    if (warp == 0 && lane == 0) {
+        for (int s = 0; s < kTcStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 4);
+        }
+        mbar_init(drain, 1);
+        mbar_init(planbar, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tensormap(&maps.wd);
+        prefetch_tensormap(&maps.hr);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, kTcTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    grid_dependents_launch();
+    const uint32_t tmem_base = *tmem_holder;
+
+    // tile u -> (slice si, 128-row block mb); si = 0 is the shared expert when
+    // there is one, then the routed slices in plan order
+
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer
+        if (elect_one()) {
+            const uint64_t pol_w = policy_evict_first();
+            const uint64_t pol_h = policy_evict_last();
+            grid_dependency_wait();  // h comes from the previous kernel
+            uint32_t stage = 0, phase = 0;
+            int issued = 0;
+            bool stop = !mbar_wait(planbar, 0, abort_flag);
+            const int total = stop ? 0 : (has_shared + *n_slices) * n_mb;
+            for (int u = blockIdx.x; u < total && !stop; u += gridDim.x) {
+                const int si = u / n_mb, mb = u - si * n_mb;
+                const bool shared = si < has_shared;
+                const int slice = si - has_shared;
+                const int e = shared ? 0 : (int)P.group_expert[slice_group[slice]];
+                const int kblocks = ((shared ? a.I_s : a.I) + kGemmBK - 1) / kGemmBK;
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+                        stop = true;
+                        break;
+                    }
+                    uint8_t *sa = smem + stage * kTcStageBytes;
+                    uint8_t *sb = sa + kTcABytes;
+                    mbar_arrive_expect_tx(&full[stage], kTcStageBytes);
+                    const int k0 = kb * kGemmBK;
+                    if (shared) {
+                        tma_load_2d(sa, &maps.sd, k0, mb * kGemmBM, &full[stage], pol_w);
+                        tma_load_2d(sb, &maps.hs, k0, 0, &full[stage], pol_h);
+                    } else {
+                        const int row = 2 * ((int)P.group_first[slice_group[slice]] + slice_j0[slice]);
+                        tma_load_3d(sa, &maps.wd, k0, mb * kGemmBM, e, &full[stage], pol_w);
+                        tma_load_2d(sb, &maps.hr, k0, row, &full[stage], pol_h);
+                    }
+                    ++issued;
+                    if (++stage == kTcStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // no copy may still be landing in shared memory when the CTA exits
+            for (int n = issued > kTcStages ? issued - kTcStages : 0; n < issued; ++n)
+                mbar_wait(&full[n % kTcStages], (uint32_t)(n / kTcStages) & 1u, nullptr);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer
+        if (elect_one()) {
+            uint32_t stage = 0, phase = 0;
+            uint32_t acc = 0, acc_phase = 0;
+            bool stop = !mbar_wait(planbar, 0, abort_flag);
+            const int total = stop ? 0 : (has_shared + *n_slices) * n_mb;
+            const uint32_t idesc = idesc_bf16_f32(kGemmBM, kTcN);
+            for (int u = blockIdx.x; u < total && !stop; u += gridDim.x) {
+                const bool shared = u / n_mb < has_shared;
+                const int kblocks = ((shared ? a.I_s : a.I) + kGemmBK - 1) / kGemmBK;
+                if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag))
+                    break;
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem_base + acc * kTcN;
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, abort_flag)) {
+                        stop = true;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t a_addr = smem_u32(smem + stage * kTcStageBytes);
+                    const uint32_t b_addr = a_addr + kTcABytes;
+#pragma unroll
+                    for (int kk = 0; kk < kGemmBK / 16; ++kk)
+                        umma_bf16(d_tmem, smem_desc_sw128_kmajor(a_addr + kk * 32),
+                                  smem_desc_sw128_kmajor(b_addr + kk * 32), idesc,
+                                  (kb > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(&empty[stage]);  // frees the stage once these MMAs are done
+                    if (++stage == kTcStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (stop)
+                    break;
+                umma_commit(&tfull[acc]);
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+            // every MMA issued by this thread has completed before TMEM is freed
+            umma_commit(drain);
+            mbar_wait(drain, 0, nullptr);
+        }
+    } else {
+        // ------------------------------------------------ plan, then epilogue
+        const int ltid = (int)threadIdx.x - 64;
+        grid_dependency_wait();  // ids and weights may come from earlier kernels
+        build_stream_plan(P, a.ids, a.weights, a.T, a.top_k, a.E, ltid, 128, kTcBarPlan);
+        if (ltid == 0) {
+            int sl = 0;
+            for (int g = 0; g < P.n_groups; ++g) {
+                const int cnt = P.group_first[g + 1] - P.group_first[g];
+                for (int j0 = 0; j0 < cnt; j0 += kTcSlice) {
+                    slice_group[sl] = g;
+                    slice_j0[sl] = j0;
+                    ++sl;
+                }
+            }
+            *n_slices = sl;
+            mbar_arrive(planbar);  // release: the plan and the slice table are written
+        }
+        if (mbar_wait(planbar, 0, abort_flag)) {
+            const int q = warp & 3;  // TMEM lane quarter this warp may access
+            const int total = (has_shared + *n_slices) * n_mb;
+            uint32_t acc = 0, acc_phase = 0;
+            for (int u = blockIdx.x; u < total; u += gridDim.x) {
+                const int si = u / n_mb, mb = u - si * n_mb;
+                const bool shared = si < has_shared;
+                if (!mbar_wait(&tfull[acc], acc_phase, abort_flag))
+                    break;
+                tc_fence_after_sync();
+                uint32_t v[16];
+                tmem_load_16cols(tmem_base + ((uint32_t)(32 * q) << 16) + acc * kTcN, v);
+                tmem_load_wait();
+                const int row = mb * kGemmBM + 32 * q + lane;
+                if (row < a.H) {
+                    // column r + n holds the lo part of column r (n picks)
+                    const int slice = si - has_shared;
+                    const int g = shared ? 0 : slice_group[slice];
+                    const int p0 = shared ? 0 : P.group_first[g] + slice_j0[slice];
+                    const int n = shared ? a.T : min(kTcSlice, (int)P.group_first[g + 1] - p0);
+                    // lo[r] = column r + n, picked with constant register indices
+                    float lo[kTcSlice];
+#pragma unroll
+                    for (int r = 0; r < kTcSlice; ++r)
+                        lo[r] = 0.f;
+#pragma unroll
+                    for (int nn = 1; nn <= kTcSlice; ++nn)
+                        if (n == nn) {
+#pragma unroll
+                            for (int r = 0; r < nn; ++r)
+                                lo[r] = __uint_as_float(v[r + nn]);
+                        }
+#pragma unroll
+                    for (int r = 0; r < kTcSlice; ++r) {
+                        const float d = __uint_as_float(v[r]) + lo[r];
+                        if (r < n) {
+                            if (shared) {
+                                a.s[(size_t)r * a.H + row] = d;
+                            } else {
+                                const int pair = p0 + r;
+                                a.c[(size_t)P.sorted_src[pair] * a.H + row] = P.pair_weight[pair] * d;
+                            }
+                        }
                     }
                 }
                 tc_fence_before_sync();

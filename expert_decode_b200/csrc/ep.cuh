@@ -57,31 +57,45 @@ ep_combine_kernel(const float *__restrict__ partials, int64_t T, int H,
     grid_dependents_launch();
     grid_dependency_wait();  // the partials come from earlier kernels
     const int64_t t = blockIdx.y;
-    if (threadIdx.x == 0) {
+    if (threadIdx.x < 32) {
+        // lane j < top_k marks the band of pick j; the marks are OR-ed over the warp
+        const int j = (int)threadIdx.x;
         unsigned long long m = 0ull;
-        for (int j = 0; j < top_k; ++j) {
+        if (j < top_k) {
             const int32_t e = ids[t * top_k + j];
-            if (e < 0 || e >= E)
-                continue;
-            int r = 0;
-            while (r + 1 < R && bands.start[r + 1] <= e)
-                ++r;
-            m |= 1ull << r;
+            if (e >= 0 && e < E) {
+                int r = 0;
+                while (r + 1 < R && bands.start[r + 1] <= e)
+                    ++r;
+                m = 1ull << r;
+            }
         }
-        mask = m;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+            m |= __shfl_xor_sync(0xffffffffu, m, off);
+        if (j == 0)
+            mask = m;
     }
     __syncthreads();
     const int col = (int)blockIdx.x * kEpCombineThreads + (int)threadIdx.x;
     if (col >= H)
         return;
+    // the partials are loaded eight bands at a time before they are added, so
+    // that the loads' latencies overlap; the adds run in rank order
     float acc = 0.f;
     bool first = true;
-    for (int r = 0; r < R; ++r) {
-        if (!((mask >> r) & 1ull))
-            continue;
-        const float v = partials[((size_t)r * T + t) * H + col];
-        acc = first ? v : acc + v;
-        first = false;
+    for (int r0 = 0; r0 < R; r0 += 8) {
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (r0 + i < R && ((mask >> (r0 + i)) & 1ull))
+                v[i] = partials[((size_t)(r0 + i) * T + t) * H + col];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (r0 + i < R && ((mask >> (r0 + i)) & 1ull)) {
+                acc = first ? v[i] : acc + v[i];
+                first = false;
+            }
     }
     y[t * H + col] = shared != nullptr ? acc + shared[t * H + col] : acc;
 }

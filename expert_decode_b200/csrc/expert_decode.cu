@@ -169,6 +169,8 @@ ep_status device_info(const DeviceInfo **out) {
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, m));
         EP_CUDA_CHECK(cudaFuncSetAttribute(epk::stream_gate_up_tc_kernel,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, m));
+        EP_CUDA_CHECK(cudaFuncSetAttribute(epk::stream_down_tc_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, m));
         ep_status s = epk::grouped_set_attributes(m);
         if (s != EP_OK)
             return fail(s, "setting the grouped GEMM kernel attributes failed");
@@ -196,8 +198,9 @@ size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
 // ---------------------------------------------------------- workspace layout
 struct Workspace {
-    // streaming path (T <= 8)
-    size_t h_routed = 0, h_shared = 0;
+    // streaming path (T <= 8): fp32 h for the CUDA-core down projection, bf16
+    // hi/lo rows ([2 T k + 16][I], [16][I_s]) for the tensor-core one
+    size_t h_routed = 0, h_shared = 0, hb_routed = 0, hb_shared = 0;
     // tensor path
     epk::GroupedWorkspace grouped;
     size_t total = 0;
@@ -211,6 +214,10 @@ Workspace workspace_layout(int64_t T, int64_t H, int64_t E, int64_t k, int64_t I
         o = align256(o + (size_t)T * k * I * 4);
         w.h_shared = o;
         o = align256(o + (size_t)T * I_s * 4);
+        w.hb_routed = o;
+        o = align256(o + (size_t)(2 * T * k + 2 * epk::kTcSlice) * I * 2);
+        w.hb_shared = o;
+        o = align256(o + (size_t)2 * epk::kTcSlice * I_s * 2);
     }
     w.grouped = epk::grouped_workspace_layout(o, T, H, E, k, I, I_s);
     o = align256(w.grouped.end);
@@ -649,9 +656,51 @@ ep_status ffn_forward_impl(bool band_call, const void *x, ep_dtype x_dtype, int6
             ta.weights = weights;
             ta.h_routed = ga.h_routed;
             ta.h_shared = ga.h_shared;
-            KernelBracket kb0(st, 0);
-            EP_CUDA_CHECK(launch(epk::stream_gate_up_tc_kernel, gu_grid, epk::kTcThreads,
-                                 epk::TcSmem::alloc, st, tm, ta));
+            ta.hb_routed = reinterpret_cast<uint16_t *>(ws + W.hb_routed);
+            ta.hb_shared = I_s > 0 ? reinterpret_cast<uint16_t *>(ws + W.hb_shared) : nullptr;
+            // the down projection on the tensor cores too: W_down rows against
+            // the bf16 hi/lo slices of h, then the fold in combine_kernel
+            epk::DtMaps dm;
+            memset(&dm, 0, sizeof dm);
+            bool dm_ok = epk::DtSmem::alloc <= (uint32_t)d->smem_optin &&
+                         epk::map_3d(&dm.wd, w_down, I, H, E, epk::kGemmBM) &&
+                         epk::map_2d(&dm.hr, ta.hb_routed, I,
+                                     (uint64_t)(2 * T * top_k + 2 * epk::kTcSlice),
+                                     2 * epk::kTcSlice);
+            if (I_s > 0)
+                dm_ok = dm_ok && epk::map_2d(&dm.sd, ws_down, I_s, H, epk::kGemmBM) &&
+                        epk::map_2d(&dm.hs, ta.hb_shared, I_s, 2 * epk::kTcSlice,
+                                    2 * epk::kTcSlice);
+            if (!dm_ok)
+                return fail(EP_ECUDA, "moe_ffn_forward: encoding a down tensor map failed");
+            {
+                KernelBracket kb0(st, 0);
+                EP_CUDA_CHECK(launch(epk::stream_gate_up_tc_kernel, gu_grid, epk::kTcThreads,
+                                     epk::TcSmem::alloc, st, tm, ta));
+            }
+            epk::DtArgs dta;
+            dta.T = (int)T; dta.H = (int)H; dta.E = (int)E; dta.I = (int)I; dta.I_s = (int)I_s;
+            dta.top_k = top_k;
+            dta.ids = ids;
+            dta.weights = weights;
+            dta.c = reinterpret_cast<float *>(ws + W.grouped.c);
+            dta.s = reinterpret_cast<float *>(ws + W.grouped.s);
+            {
+                KernelBracket kb1(st, 1);
+                EP_CUDA_CHECK(launch(epk::stream_down_tc_kernel, gu_grid, epk::kTcThreads,
+                                     epk::DtSmem::alloc, st, dm, dta));
+            }
+            {
+                KernelBracket kb2(st, 2);
+                // 64-thread blocks: a few tokens still spread over most SMs
+                const dim3 cgrid((unsigned)T, (unsigned)((H / 4 + 63) / 64));
+                EP_CUDA_CHECK(launch(epk::combine_kernel, cgrid, 64, 0, st,
+                                     (const float *)dta.c,
+                                     (const float *)(I_s > 0 ? dta.s : nullptr), ids, (int64_t)T,
+                                     (int)H, (int)top_k, (int)E, y));
+            }
+            t_launches = 3;
+            return ok();
         } else {
             KernelBracket kb0(st, 0);
             if (x_dtype == EP_F32)

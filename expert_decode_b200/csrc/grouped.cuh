@@ -639,22 +639,33 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
                                                       const int32_t *__restrict__ ids, int64_t T,
                                                       int H, int top_k, int E,
                                                       float *__restrict__ y) {
+    __shared__ int pick_e[16];
     __shared__ int order[16];
     __shared__ int n_valid;
+    grid_dependency_wait();  // c and s come from the previous kernel (launched early or not)
     const int64_t t = blockIdx.x;
-    if (threadIdx.x == 0) {
-        int n = 0;
-        for (int j = 0; j < top_k; ++j) {
-            const int e = ids[t * top_k + j];
-            if (e < 0 || e >= E)
-                continue;
-            int pos = n++;
-            while (pos > 0 && ids[t * top_k + order[pos - 1]] > e) {
-                order[pos] = order[pos - 1];
-                --pos;
+    // the token's picks in ascending (expert id, slot): each valid pick's
+    // place is the number of valid picks before it in that order (blockDim.x
+    // >= top_k; the ids are read once, in parallel)
+    const int j = (int)threadIdx.x;
+    if (j < top_k)
+        pick_e[j] = ids[t * top_k + j];
+    __syncthreads();
+    if (j < top_k) {
+        const int e = pick_e[j];
+        if (e >= 0 && e < E) {
+            int r = 0;
+            for (int q = 0; q < top_k; ++q) {
+                const int f = pick_e[q];
+                r += f >= 0 && f < E && (f < e || (f == e && q < j));
             }
-            order[pos] = j;
+            order[r] = j;
         }
+    }
+    if (j == 0) {
+        int n = 0;
+        for (int q = 0; q < top_k; ++q)
+            n += pick_e[q] >= 0 && pick_e[q] < E;
         n_valid = n;
     }
     __syncthreads();

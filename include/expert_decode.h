@@ -252,15 +252,20 @@ ep_status moe_ep_combine(const float *partials, int64_t T, int64_t H, const int3
 /*
  * Which moe_ffn_forward path runs.  EP_DISPATCH_AUTO (the default) takes the
  * weight-streaming path for T <= 8 when its on-chip buffers fit, else the
- * tensor-core path.  Forcing a path that does not fit the sizes makes
+ * tensor-core path; inside the streaming path, the tensor-core kernels from
+ * 2 tokens with bf16 x, the CUDA-core kernels otherwise.  Forcing a path that does not fit the sizes makes
  * moe_ffn_forward return EP_EINVAL.  Process-wide; meant for tests and tuning.
  */
 typedef enum {
     EP_DISPATCH_AUTO = 0,
-    EP_DISPATCH_STREAMING = 1,      /* streaming path, gate/up kernel chosen as in AUTO */
+    EP_DISPATCH_STREAMING = 1,      /* streaming path, kernels chosen as in AUTO */
     EP_DISPATCH_TENSOR = 2,
-    EP_DISPATCH_STREAMING_TC = 3,   /* streaming path, gate/up on the tensor cores (bf16 x) */
-    EP_DISPATCH_STREAMING_SIMT = 4  /* streaming path, gate/up on the CUDA cores */
+    /* streaming path, gate/up and down on the tensor cores (bf16 x), then the
+       fold of the picks' contributions (three launches) */
+    EP_DISPATCH_STREAMING_TC = 3,
+    /* streaming path, gate/up on the CUDA cores and down with the fold (two
+       launches) */
+    EP_DISPATCH_STREAMING_SIMT = 4
 } ep_dispatch;
 ep_status ep_set_dispatch(ep_dispatch mode);
 
