@@ -1,7 +1,7 @@
 """The weight-streaming path (T <= 8) of moe_ffn_forward against the fp64 oracle,
 with the bit-identity the method promises: across runs and across band counts.
-Every test runs with the gate/up projection on the CUDA cores, on the tensor
-cores (bf16 activations only), and with the default choice of kernel."""
+Every test runs with the projections on the CUDA cores, on the tensor cores
+(bf16 activations only), and with the default choice of kernels."""
 import numpy as np
 import pytest
 import torch
@@ -18,10 +18,10 @@ WL = workloads.WORKLOADS
 TINY_BF16 = workloads.Workload("tiny_bf16", (4,), 256, 16, 4, 128, 128, "bf16", "none", (1, 2, 4))
 
 
-# streaming_simt: gate/up on the CUDA cores; streaming_tc: gate/up on the
-# tensor cores (bf16 activations only); streaming: the default choice (tensor
-# cores from 2 tokens with bf16 activations).  The down projection and its
-# fold run on the CUDA cores in every case.
+# streaming_simt: gate/up, then down with the fold, on the CUDA cores;
+# streaming_tc: gate/up and down on the tensor cores (bf16 activations only),
+# then the fold of the picks' contributions; streaming: the default choice
+# (tensor cores from 2 tokens with bf16 activations).
 @pytest.fixture(autouse=True, params=["streaming_simt", "streaming_tc", "streaming"])
 def gate_up(request):
     ed.ep_set_dispatch(request.param)
@@ -137,6 +137,22 @@ def test_repeated_expert_in_one_token(oracle_lib, gate_up, wl):
     ids[3, :] = ids[3, 1]          # token 3 picks one expert four times
     y = gpu_ffn(x, ids, w, W, ed.ep_plan(wl.E, 2))
     check_y(y, oracle_ffn(oracle_lib, x, ids, w, W), rel_tol=1e-4, what="repeated picks")
+
+
+# More than 8 picks of one expert (repeats within tokens): the tensor-core down
+# projection takes a group in slices of up to 8 picks (T = 3: 15 picks of
+# expert 3, two slices; T = 8: 40 picks, five slices).
+@pytest.mark.parametrize("T", [3, 8])
+def test_more_than_eight_picks_of_one_expert(oracle_lib, gate_up, T):
+    wl = workloads.Workload("many_picks", (T,), 256, 16, 8, 128, 128, "bf16", "none", (1,))
+    W, x, ids, w = _routed(oracle_lib, wl, T, seed=40 + T)
+    ids[:, :5] = 3
+    ids[0, 5:] = 7
+    y = gpu_ffn(x, ids, w, W, ed.ep_plan(wl.E, 4))
+    ed.ep_check_status()
+    check_y(y, oracle_ffn(oracle_lib, x, ids, w, W), rel_tol=1e-4,
+            what=f"{5 * T} picks of one expert")
+    assert torch.equal(gpu_ffn(x, ids, w, W, ed.ep_plan(wl.E, 1)), y), "bands=1 differs"
 
 
 @pytest.mark.parametrize("wl", [WL["tiny"], TINY_BF16], ids=["fp32_x", "bf16_x"])
