@@ -211,12 +211,39 @@ def kernel_cost(wl, T, n_distinct, tensor_path):
             "call_flops": call_flops, "n_experts": n_exp}
 
 
+def _code_only(text):
+    """C/C++/CUDA source with its comments removed and runs of white space
+    collapsed (string and character literals are kept as they are)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def source_digest():
+    """Digest of the kernel sources' code (comments excluded): the ncu counters
+    committed under profiles/ stand for the kernels while it matches."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "expert_decode_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(csrc, f), encoding="utf-8") as fh:
+            h.update(f.encode() + b"\0" + _code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -181,8 +181,8 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
     return p;
 }
 
-// Tiled TMA loads (no multicast).  The innermost coordinate c0 times the
-// element size must be a multiple of 16 bytes.
+// Tiled TMA loads, each into this CTA's own shared memory.  The innermost
+// coordinate c0 times the element size must be a multiple of 16 bytes.
 __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *map, int32_t c0,
                                             int32_t c1, uint64_t *bar, uint64_t policy) {
     asm volatile(

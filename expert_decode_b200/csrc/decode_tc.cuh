@@ -14,7 +14,7 @@
 // Persistent and warp specialised, one CTA per SM:
 //   warp 0     TMA producer: per 64-wide k block the A tile (two boxes of 64
 //              weight rows, 16 KB) and the x tile (16 rows, 2 KB) into a
-//              ring of kTcStages stages, 128-byte swizzle, no multicast: three
+//              ring of kTcStages stages, 128-byte swizzle, one CTA per copy: three
 //              copy instructions per stage, as few as the operands allow;
 //   warp 1     tcgen05.mma issuer (M = 128, N = 16, K = 16 per instruction),
 //              fp32 accumulators in TMEM, two of them so that the epilogue

@@ -24,7 +24,7 @@
 //                   plus the shared expert's output.
 //
 // The GEMMs are persistent and warp specialised: warp 0 issues TMA loads
-// (cp.async.bulk.tensor, 128-byte swizzle, no multicast) into a 4-stage
+// (cp.async.bulk.tensor, 128-byte swizzle, one CTA per copy) into a 4-stage
 // shared-memory ring, warp 1 issues tcgen05.mma with the fp32 accumulator in
 // tensor memory (two accumulators, so the epilogue of one tile overlaps the
 // MMAs of the next), and warps 2..5 drain the accumulator with tcgen05.ld.
