@@ -149,7 +149,6 @@ stream_gate_up_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
-    grid_dependents_launch();
     const uint32_t tmem_base = *tmem_holder;
 
     // tile u -> (group index gi, first unit m0); gi = 0 is the shared expert
@@ -263,6 +262,9 @@ stream_gate_up_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
         // ------------------------------------------------ plan, then epilogue
         const int ltid = (int)threadIdx.x - 64;
         grid_dependency_wait();  // ids and weights may come from the previous kernel
+        // the next kernel is let launch only once every CTA of this one has
+        // passed its wait, so that it may read the ids (and x) before its own
+        grid_dependents_launch();
         build_stream_plan(P, a.ids, a.weights, a.T, a.top_k, a.E, ltid, 128, kTcBarPlan);
         if (ltid == 0) {
             const int G = has_shared + P.n_groups;
@@ -460,12 +462,34 @@ stream_down_tc_kernel(const __grid_constant__ DtMaps maps, const DtArgs a) {
 
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer
+        // The plan comes from ids, which the kernel before the previous one
+        // wrote (the previous kernel lets this one launch only after its own
+        // wait), so the weights of the first kTcStages stages are requested
+        // before griddepcontrol.wait; their h boxes, written by the previous
+        // kernel, follow once it has completed.  A stage's full barrier takes
+        // the weight bytes by expect_tx and the h bytes with its one arrive.
         if (elect_one()) {
             const uint64_t pol_w = policy_evict_first();
             const uint64_t pol_h = policy_evict_last();
-            grid_dependency_wait();  // h comes from the previous kernel
             uint32_t stage = 0, phase = 0;
             int issued = 0;
+            bool waited = false;
+            int pend_row[kTcStages], pend_k0[kTcStages];  // h boxes not yet requested
+            auto load_h = [&](int st, int k0, int row) {
+                uint8_t *sb = smem + st * kTcStageBytes + kTcABytes;
+                if (row < 0)
+                    tma_load_2d(sb, &maps.hs, k0, 0, &full[st], pol_h);
+                else
+                    tma_load_2d(sb, &maps.hr, k0, row, &full[st], pol_h);
+            };
+            auto finish_wait = [&]() {
+                grid_dependency_wait();  // h comes from the previous kernel
+                waited = true;
+                for (int n = 0; n < issued; ++n) {
+                    mbar_arrive_expect_tx(&full[n], kTcBBytes);
+                    load_h(n, pend_k0[n], pend_row[n]);
+                }
+            };
             bool stop = !mbar_wait(planbar, 0, abort_flag);
             const int total = stop ? 0 : (has_shared + *n_slices) * n_mb;
             for (int u = blockIdx.x; u < total && !stop; u += gridDim.x) {
@@ -473,23 +497,32 @@ stream_down_tc_kernel(const __grid_constant__ DtMaps maps, const DtArgs a) {
                 const bool shared = si < has_shared;
                 const int slice = si - has_shared;
                 const int e = shared ? 0 : (int)P.group_expert[slice_group[slice]];
+                // h row of the slice's first pick (-1: the shared expert's rows)
+                const int row =
+                    shared ? -1 : 2 * ((int)P.group_first[slice_group[slice]] + slice_j0[slice]);
                 const int kblocks = ((shared ? a.I_s : a.I) + kGemmBK - 1) / kGemmBK;
                 for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!waited && issued == kTcStages)
+                        finish_wait();  // the ring is full: the stages need their h now
                     if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
                         stop = true;
                         break;
                     }
                     uint8_t *sa = smem + stage * kTcStageBytes;
-                    uint8_t *sb = sa + kTcABytes;
-                    mbar_arrive_expect_tx(&full[stage], kTcStageBytes);
                     const int k0 = kb * kGemmBK;
-                    if (shared) {
+                    if (waited)
+                        mbar_arrive_expect_tx(&full[stage], kTcStageBytes);
+                    else
+                        mbar_expect_tx(&full[stage], kTcABytes);
+                    if (shared)
                         tma_load_2d(sa, &maps.sd, k0, mb * kGemmBM, &full[stage], pol_w);
-                        tma_load_2d(sb, &maps.hs, k0, 0, &full[stage], pol_h);
-                    } else {
-                        const int row = 2 * ((int)P.group_first[slice_group[slice]] + slice_j0[slice]);
+                    else
                         tma_load_3d(sa, &maps.wd, k0, mb * kGemmBM, e, &full[stage], pol_w);
-                        tma_load_2d(sb, &maps.hr, k0, row, &full[stage], pol_h);
+                    if (waited) {
+                        load_h(stage, k0, row);
+                    } else {
+                        pend_k0[stage] = k0;
+                        pend_row[stage] = row;
                     }
                     ++issued;
                     if (++stage == kTcStages) {
@@ -498,6 +531,8 @@ stream_down_tc_kernel(const __grid_constant__ DtMaps maps, const DtArgs a) {
                     }
                 }
             }
+            if (!waited)
+                finish_wait();  // fewer stages than the ring holds, or none, or a stop
             // no copy may still be landing in shared memory when the CTA exits
             for (int n = issued > kTcStages ? issued - kTcStages : 0; n < issued; ++n)
                 mbar_wait(&full[n % kTcStages], (uint32_t)(n / kTcStages) & 1u, nullptr);
@@ -551,7 +586,9 @@ stream_down_tc_kernel(const __grid_constant__ DtMaps maps, const DtArgs a) {
     } else {
         // ------------------------------------------------ plan, then epilogue
         const int ltid = (int)threadIdx.x - 64;
-        grid_dependency_wait();  // ids and weights may come from earlier kernels
+        // ids and weights come from the kernel before the previous one, which
+        // has completed: the previous kernel let this one launch only after
+        // passing its own griddepcontrol.wait
         build_stream_plan(P, a.ids, a.weights, a.T, a.top_k, a.E, ltid, 128, kTcBarPlan);
         if (ltid == 0) {
             int sl = 0;
@@ -566,6 +603,7 @@ stream_down_tc_kernel(const __grid_constant__ DtMaps maps, const DtArgs a) {
             *n_slices = sl;
             mbar_arrive(planbar);  // release: the plan and the slice table are written
         }
+        grid_dependency_wait();  // before any output is written
         if (mbar_wait(planbar, 0, abort_flag)) {
             const int q = warp & 3;  // TMEM lane quarter this warp may access
             const int total = (has_shared + *n_slices) * n_mb;
