@@ -121,8 +121,9 @@ ep_status moe_route_sigmoid(const void *x, ep_dtype x_dtype, int64_t T, int64_t 
 /*
  * moe_ffn_workspace_size -- bytes of device workspace moe_ffn_forward needs
  * for these sizes (0 when T = 0).  The workspace holds the token grouping,
- * the grouped activations and the per-pick partial outputs; its contents on
- * entry do not matter.
+ * the grouped activations, the SwiGLU activations h (fp32, or bf16 hi/lo rows
+ * for the tensor-core down projection of T <= 8) and the per-pick partial
+ * outputs; its contents on entry do not matter.
  */
 size_t moe_ffn_workspace_size(int64_t T, int64_t H, int64_t E, int32_t top_k, int64_t I,
                               int64_t I_s);
