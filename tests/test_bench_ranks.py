@@ -61,3 +61,16 @@ def test_whole_job_throughput_over_two_gloo_ranks(tmp_path):
 def test_whole_job_throughput_single_rank():
     b = _bench()
     assert b.whole_job_throughput(130, 2.0) == (65.0, 2.0)
+
+
+def test_source_digest_ignores_comments_only():
+    """The digest that ties profiles/traffic.json to the kernels changes with the
+    code and not with comments or white space; literals are kept whole."""
+    b = _bench()
+    code = 'int f(int a) { return a + 1; } const char *s = "a // b /* c */";'
+    commented = ('// leading note\nint f(int a) {  /* inline */ return a + 1; }\n'
+                 'const char *s = "a // b /* c */";  // trailing\n')
+    assert b._code_only(code) == b._code_only(commented)
+    assert b._code_only(code) != b._code_only(code.replace("a + 1", "a + 2"))
+    assert '"a // b /* c */"' in b._code_only(commented)
+    assert b.source_digest() == b.source_digest()
