@@ -1,21 +1,22 @@
-// decode_tc.cuh -- gate/up of the weight-streaming (decode) path on the
-// tensor cores.
+// decode_tc.cuh -- gate/up and down projections of the weight-streaming
+// (decode, T <= 8) path on the tensor cores.
 //
-// Same contraction as stream_gate_up_kernel (h = silu(W_gate x) * (W_up x)
-// for every picked expert and the shared expert; fak note "GLM-5.2
-// multi-GPU", expertSwiGLU), laid out for tcgen05: a tile is 64 units of I,
-// i.e. 128 weight rows on the MMA's M side, the 64 W_gate rows over the 64
-// W_up rows of the same units (TensorFold #593's packGateUp operand), and all
-// T <= 8 tokens on its N side (N = 16; the tensor map zero-fills the rows
-// after T).  Every
-// tile therefore computes every token, and the epilogue keeps the tokens
-// that picked the tile's expert, so no activation gather is needed.
+// stream_gate_up_tc_kernel: the contraction of stream_gate_up_kernel
+// (h = silu(W_gate x) * (W_up x) for every picked expert and the shared
+// expert; fak note "GLM-5.2 multi-GPU", expertSwiGLU), laid out for tcgen05.
+// A tile is 64 units of I: 128 weight rows on the MMA's M side, the 64 W_gate
+// rows over the 64 W_up rows of the same units (TensorFold #593's packGateUp
+// operand), and all T <= 8 tokens on its N side (N = 16; the tensor map
+// zero-fills the rows after T).  Every tile therefore computes every token,
+// and the epilogue keeps the tokens that picked the tile's expert, so no
+// activation gather is needed.
 //
 // Persistent and warp specialised, one CTA per SM:
 //   warp 0     TMA producer: per 64-wide k block the A tile (two boxes of 64
 //              weight rows, 16 KB) and the x tile (16 rows, 2 KB) into a
-//              ring of kTcStages stages, 128-byte swizzle, one CTA per copy: three
-//              copy instructions per stage, as few as the operands allow;
+//              ring of kTcStages stages, 128-byte swizzle, each CTA loading
+//              its own copy: three copy instructions per stage, as few as the
+//              operands allow;
 //   warp 1     tcgen05.mma issuer (M = 128, N = 16, K = 16 per instruction),
 //              fp32 accumulators in TMEM, two of them so that the epilogue
 //              of one tile overlaps the MMAs of the next;
@@ -23,10 +24,12 @@
 //              drain each accumulator with tcgen05.ld: the warps of TMEM
 //              quarters 2 and 3 (up rows) pass their values through shared
 //              memory to those of quarters 0 and 1 (gate rows of the same
-//              units), which write h = silu(g) * u in fp32, in the layout the
-//              down kernel reads.
+//              units), which write h = silu(g) * u: as bf16 hi/lo rows for
+//              stream_down_tc_kernel, or in fp32 for stream_down_fold_kernel.
 // Tiles go round-robin over the CTAs: the shared expert's first, then each
 // routed group's in ascending expert id.
+//
+// stream_down_tc_kernel (below): the down projection with the same machinery.
 #pragma once
 
 #include "common.cuh"
