@@ -223,6 +223,10 @@ def ep_check_status(stream=None):
 
 
 def ep_set_dispatch(mode):
+    """Process-wide path choice: "auto", "tensor", "streaming" (kernels as in
+    auto), "streaming_tc" (gate/up and down on the tensor cores, then the
+    fold) or "streaming_simt" (gate/up, then down with the fold, on the CUDA
+    cores)."""
     _check(library().ep_set_dispatch(_DISPATCH[mode]))
 
 

@@ -1,11 +1,15 @@
 // streaming.cuh -- the weight-streaming path of the routed MoE FFN for 1..8
-// rows (decode).
+// rows (decode) on the CUDA cores: one token, fp32 activations, or a forced
+// choice (the tensor-core kernels of decode_tc.cuh take 2..8 tokens of bf16
+// activations by default).  The expert grouping (build_stream_plan) serves
+// both.
 //
 // Only the picked experts' weights are read, each exactly once for all the
 // tokens that picked it, with 1-D bulk copies (cp.async.bulk) into a ring of
 // shared-memory slots that a producer warp keeps full while consumer warps
-// compute on CUDA cores with packed fp32 FMAs (fma.rn.f32x2).  Products are bf16 x bf16 (or fp32 x bf16) folded in
-// fp32; the SwiGLU activations stay fp32 between the two projections.
+// compute with packed fp32 FMAs (fma.rn.f32x2).  Products are bf16 x bf16 (or
+// fp32 x bf16) folded in fp32; the SwiGLU activations stay fp32 between the
+// two projections.
 //
 // Two kernels:
 //  * stream_gate_up: per (picked expert, unit i of I) task, the dots of the
