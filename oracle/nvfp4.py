@@ -158,3 +158,16 @@ def nvfp4_quantize(w, tensor_scale=None):
     x = np.divide(blocks, denom, out=np.zeros_like(blocks), where=denom > 0)
     codes = e2m1_encode(x).reshape(rows, cols)
     return pack_nibbles(codes), scales, st
+
+
+def nvfp4_to_bf16_bits(packed, scales, tensor_scale):
+    """The dequantised weights as bf16 bit patterns (uint16), for the bf16
+    oracle.  Every value must be exact in bf16 (true for a power-of-two tensor
+    scale); anything else raises, since the bf16 oracle would then see other
+    weights than the format holds."""
+    w = nvfp4_dequantize(packed, scales, tensor_scale)
+    bits32 = w.astype(np.float32).view(np.uint32)
+    if not np.array_equal(w.astype(np.float32).astype(np.float64), w) or np.any(bits32 & 0xFFFF):
+        raise ValueError("dequantised weights are not exact in bf16")
+    return (bits32 >> 16).astype(np.uint16)
+

@@ -138,6 +138,18 @@ def pin_quantize_error_bound_and_bf16_exactness(m):
     assert np.array_equal(as_bf16, deq)
 
 
+def pin_bf16_bits_are_the_dequantised_weights(m):
+    rng = np.random.default_rng(9)
+    w = rng.normal(0, 0.02, (4, 64))
+    packed, scales, st = m.nvfp4_quantize(w)
+    bits = m.nvfp4_to_bf16_bits(packed, scales, st)
+    back = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(back, m.nvfp4_dequantize(packed, scales, st))
+    # a tensor scale that is not a power of two leaves values bf16 cannot hold
+    with pytest.raises(ValueError):
+        m.nvfp4_to_bf16_bits(packed, scales, st * 1.1)
+
+
 PINS = [pin_e4m3_decode_matches_torch_for_every_code,
         pin_e4m3_encode_matches_torch_rounding_including_ties,
         pin_e4m3_encode_saturates_above_448,
@@ -145,7 +157,8 @@ PINS = [pin_e4m3_decode_matches_torch_for_every_code,
         pin_e2m1_encode_is_round_to_nearest_even_with_saturation,
         pin_storage_nibble_order_and_block_layout,
         pin_quantize_round_trips_representable_blocks,
-        pin_quantize_error_bound_and_bf16_exactness]
+        pin_quantize_error_bound_and_bf16_exactness,
+        pin_bf16_bits_are_the_dequantised_weights]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__[4:] for p in PINS])
@@ -197,6 +210,6 @@ def test_pins_catch_planted_mistake(tmp_path, what, old, new):
     for pin in PINS:
         try:
             pin(mod)
-        except (AssertionError, ValueError, IndexError):
+        except (AssertionError, ValueError, IndexError, pytest.fail.Exception):
             caught.append(pin.__name__)
     assert caught, f"no pin catches: {what}"
