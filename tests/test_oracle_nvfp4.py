@@ -150,6 +150,20 @@ def pin_bf16_bits_are_the_dequantised_weights(m):
         m.nvfp4_to_bf16_bits(packed, scales, st * 1.1)
 
 
+def test_seeded_nvfp4_inputs_are_deterministic_and_exact_in_bf16():
+    import workloads
+    a = workloads.make_nvfp4_experts(2, 8, 64, seed=3)
+    b = workloads.make_nvfp4_experts(2, 8, 64, seed=3)
+    assert torch.equal(a["packed"], b["packed"]) and torch.equal(a["scales"], b["scales"])
+    assert a["packed"].shape == (2, 8, 32) and a["scales"].shape == (2, 8, 4)
+    for e in range(2):
+        bits = nvfp4.nvfp4_to_bf16_bits(a["packed"][e].numpy(), a["scales"][e].numpy(),
+                                        a["tensor_scale"])
+        w = nvfp4.nvfp4_dequantize(a["packed"][e].numpy(), a["scales"][e].numpy(),
+                                   a["tensor_scale"])
+        assert bits.shape == (8, 64) and np.all(np.abs(w) <= 6 * 3.75 * 2.0 ** -7)
+
+
 PINS = [pin_e4m3_decode_matches_torch_for_every_code,
         pin_e4m3_encode_matches_torch_rounding_including_ties,
         pin_e4m3_encode_saturates_above_448,

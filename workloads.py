@@ -111,6 +111,29 @@ def make_weights(w: Workload, device="cpu", seed=SEED_BASE, H=None, E=None, I=No
     return out
 
 
+# NVFP4 expert weights are drawn directly as stored bytes: element codes
+# uniform over all 16 FP4 codes (two per byte), block-scale bytes uniform over
+# the E4M3 codes of 0.5 .. 3.75 (0x30 .. 0x47), and a tensor scale of 2^-7, so
+# the weights lie within +-0.18.  Nothing is quantised here.
+NVFP4_SCALE_CODES = (0x30, 0x48)
+NVFP4_TENSOR_SCALE = 2.0 ** -7
+
+
+def make_nvfp4_experts(E: int, rows: int, cols: int, seed: int, device="cpu"):
+    """{"packed": [E, rows, cols / 2] uint8, "scales": [E, rows, cols / 16]
+    uint8, "tensor_scale": float} for one projection of E experts."""
+    if cols % 16:
+        raise ValueError("NVFP4 rows are whole blocks of 16")
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    packed = torch.randint(0, 256, (E, rows, cols // 2), generator=g, device=device,
+                           dtype=torch.int32).to(torch.uint8)
+    lo, hi = NVFP4_SCALE_CODES
+    scales = torch.randint(lo, hi, (E, rows, cols // 16), generator=g, device=device,
+                           dtype=torch.int32).to(torch.uint8)
+    return {"packed": packed, "scales": scales, "tensor_scale": NVFP4_TENSOR_SCALE}
+
+
 def make_x(w: Workload, T: int, device="cpu", seed=SEED_BASE, batch=0, H=None, x_dtype=None):
     """Activations for one batch; `batch` selects one of several distinct draws."""
     H = H or w.H
