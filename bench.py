@@ -12,6 +12,11 @@ events.  `value` = tokens / device time (CUDA events around each step, max over
 ranks); `e2e` repeats the measurement through the public API with the inputs
 copied from pinned host memory and y copied back inside the timed region.
 
+The default run also measures the prefill (T=512), load-imbalanced (T=2048)
+and large (T=4096) workloads, each with its own steps, and reports them under
+detail.configs: tokens/s, step time, the whole step's HBM and tensor-core
+fractions and the dominant kernel's roofline.
+
   python bench.py [--gpus N --steps K --warmup W] [--config decode|prefill|...]
   python bench.py --impl reference ...   # the fp64 CPU oracle on the host cores
 
@@ -41,6 +46,9 @@ METRIC = "routed MoE FFN tokens/s; decode HBM GB/s and prefill TFLOPS as % of B2
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 N_BATCHES = 16
 FLUSH_BYTES = 512 << 20
+DETAIL_CONFIGS = ("prefill", "imbalanced", "large")
+# a step shorter than this is graded against the burst GEMM peak
+SUSTAINED_AFTER_S = 1.0
 
 
 def whole_job_throughput(tokens, seconds, dist=None, device="cpu"):
@@ -57,7 +65,7 @@ def whole_job_throughput(tokens, seconds, dist=None, device="cpu"):
     return float(tokens_t.item()) / float(seconds_t.item()), float(seconds_t.item())
 
 
-def parse_args():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
@@ -68,6 +76,11 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=500)
     ap.add_argument("--graph-steps", type=int, default=200,
                     help="steps replayed from CUDA graphs (one graph per input batch); 0 skips")
+    ap.add_argument("--detail", default=None,
+                    help="comma-separated workloads measured after the headline one "
+                         "(default with --config decode: prefill,imbalanced,large; 'none' skips)")
+    ap.add_argument("--detail-steps", type=int, default=50,
+                    help="timed steps of each detail workload (at most --steps)")
     ap.add_argument("--experts", type=int, default=0,
                     help="profiling only: fewer experts (same H, I, top_k) to keep an ncu "
                          "capture to a few GB on the device")
@@ -76,7 +89,9 @@ def parse_args():
                     help="profiling only: run moe_route alone on the workload's router weights, "
                          "bias and activations (no expert weights on the device) and print its "
                          "per-call time; no bench line")
-    return ap.parse_args()
+    ap.add_argument("--reference-budget-s", type=float, default=150.0,
+                    help="wall-time budget of the reference arm's warm-up and timed steps")
+    return ap.parse_args(argv)
 
 
 def read_peaks():
@@ -88,19 +103,35 @@ def read_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 # --------------------------------------------------------------------- clocks
 class ClockSampler:
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+    """nvidia-smi read-only queries of this GPU's SM clock and throttle
+    reasons every 100 ms, each sample stamped with the host time."""
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, device):
         self.proc = None
         uuid = str(torch.cuda.get_device_properties(device).uuid)
         self.gpu = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
-        self.out = os.path.join("/tmp", f"clocks_{os.getpid()}.csv")
+        self.out = os.path.join("/tmp", f"clocks_{os.getpid()}_{id(self)}.csv")
 
-    def start(self):
+    def start(self, wait_first_s=5.0):
+        """Start sampling and wait (up to wait_first_s) for the first sample, so
+        that the region measured next is covered from its start."""
         try:
             self.fh = open(self.out, "w")
             self.proc = subprocess.Popen(
@@ -109,35 +140,61 @@ class ClockSampler:
                 stdout=self.fh, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
+            return
+        t0 = time.time()
+        while time.time() - t0 < wait_first_s and self.proc.poll() is None:
+            if os.path.getsize(self.out) > 0:
+                break
+            time.sleep(0.02)
 
-    def stop(self):
+    def _samples(self):
+        rows = []
+        for line in open(self.out):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                sm, mx = float(parts[1]), float(parts[2])
+            except ValueError:
+                continue
+            reasons = {n for n, v in zip(self.NAMES, parts[4:8]) if v.lower() == "active"}
+            rows.append((ts, sm, mx, reasons))
+        return rows
+
+    def stop(self, window=None, min_after_s=0.25):
+        """Stop and summarise.  window = (t0, t1) host times: the summary keeps
+        the samples taken in it, or, when the window is shorter than the
+        sampling period, the samples nearest to it on either side."""
         if self.proc is None:
             return None
+        if window is not None:
+            time.sleep(max(0.0, window[1] + min_after_s - time.time()))
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.fh.close()
-        sm, mx, reasons = [], [], set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for line in open(self.out):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 7:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx.append(float(parts[1]))
-            except ValueError:
-                continue
-            for name, val in zip(names, parts[3:7]):
-                if val.lower() == "active":
-                    reasons.add(name)
+        rows = self._samples()
         os.unlink(self.out)
-        if not sm:
+        if not rows:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
-                "reasons": sorted(reasons), "samples": len(sm)}
+        scope = "whole run"
+        if window is not None:
+            inside = [r for r in rows if window[0] <= r[0] <= window[1]]
+            if inside:
+                rows, scope = inside, "timed region"
+            else:
+                before = [r for r in rows if r[0] < window[0]][-1:]
+                after = [r for r in rows if r[0] > window[1]][:1]
+                if before or after:
+                    rows = before + after
+                    scope = "samples adjacent to the timed region (shorter than 100 ms)"
+        reasons = set().union(*(r[3] for r in rows))
+        return {"sm_mhz": statistics.median(r[1] for r in rows),
+                "sm_max_mhz": max(r[2] for r in rows), "reasons": sorted(reasons),
+                "samples": len(rows), "scope": scope}
 
 
 # ------------------------------------------------------------------ workload
@@ -261,105 +318,158 @@ def traffic_for(kernel, workload):
     return e.get("dram_bytes_per_launch")
 
 
+
+
 # ------------------------------------------------------------------- CPU legs
-def oracle_sample(layer, rows_per_T, threads, batches=1):
-    """Time the fp64 oracle on a bounded sample: route + monolith FFN of the
-    given rows of the first `batches` batches of each row count.  Returns
-    tokens, seconds (the host copies of the weights are not timed)."""
-    import oracle
-    o = oracle.load()
-    W = layer.W
-    wl = layer.wl
-    bias = None if W["bias"] is None else W["bias"].cpu().numpy()
-    wr = workloads.bits(W["w_router"])
-    sh = None if layer.shared is None else tuple(workloads.bits(t) for t in layer.shared)
-    tokens, seconds = 0, 0.0
-    for T, nrows, b in [(T, n, b) for T, n in rows_per_T.items() for b in range(batches)]:
-        x = layer.xs[T][b % len(layer.xs[T])][:nrows]
-        xh = workloads.bits(x)
-        t0 = time.perf_counter()
-        ids, w, _ = o.route(xh, wr, bias, wl.top_k, threads=min(threads, nrows))
-        seconds += time.perf_counter() - t0
-        used = sorted(set(int(e) for e in ids.ravel()))
-        mats = tuple({e: workloads.bits(W[k][e]) for e in used}
-                     for k in ("w_gate", "w_up", "w_down"))
-        t0 = time.perf_counter()
-        o.moe_ffn_monolith(xh, ids, w, *mats, wl.E, shared=sh, threads=min(threads, nrows))
-        seconds += time.perf_counter() - t0
-        tokens += nrows
-    return tokens, seconds
+class HostDecode:
+    """The oracle's view of a workload, drawn on the host from the same seeded
+    recipe (the host generator's numbers differ from the device generator's;
+    shapes, distributions and biases are the workload's).  Only the router,
+    the shared expert and the experts that the batches pick are drawn."""
+
+    def __init__(self, wl, n_batches=2, seed=workloads.SEED_BASE):
+        import oracle
+        self.o = oracle.load()
+        self.wl = wl
+        w_router, bias = workloads.make_router(wl, "cpu", seed)
+        self.wr = workloads.bits(w_router)
+        self.bias = None if bias is None else bias.numpy()
+        sh = workloads.make_shared(wl, "cpu", seed)
+        self.shared = None if sh is None else tuple(workloads.bits(t) for t in sh)
+        self.batches = [(T, workloads.bits(workloads.make_x(wl, T, "cpu", seed,
+                                                            batch=b + 100 * T)))
+                        for b in range(n_batches) for T in wl.T]
+        self.mats = ({}, {}, {})
+        self.seed = seed
+
+    def route(self, xh, threads):
+        return self.o.route(xh, self.wr, self.bias, self.wl.top_k, threads=threads)
+
+    def ensure(self, experts):
+        for e in experts:
+            if e not in self.mats[0]:
+                for m, which in zip(self.mats, ("w_gate", "w_up", "w_down")):
+                    m[e] = workloads.bits(workloads.make_expert(self.wl, which, e, "cpu",
+                                                                self.seed))
+
+    def ffn(self, xh, ids, w, threads):
+        return self.o.moe_ffn_monolith(xh, ids, w, *self.mats, self.wl.E, shared=self.shared,
+                                       threads=threads)
+
+
+def oracle_tokens(host, tokens, threads):
+    """Route + monolith FFN of the given tokens (rows of the host batches,
+    concatenated) in one oracle call each, OpenMP over tokens.  The experts'
+    host copies are drawn before the clock starts.  Returns seconds."""
+    xh = np.concatenate([x for _, x in host.batches], axis=0)[tokens]
+    ids, w, _ = host.route(xh, threads)
+    host.ensure(sorted(set(int(e) for e in ids.ravel())))
+    t0 = time.perf_counter()
+    ids, w, _ = host.route(xh, threads)
+    host.ffn(xh, ids, w, threads)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(wl):
+    """The oracle as it stands on all of this host's cores: the first two
+    batches of every row count in one route and one FFN call (OpenMP over the
+    tokens), and one token alone on one thread."""
+    host = HostDecode(wl, n_batches=2)
+    n_tok = sum(x.shape[0] for _, x in host.batches)
+    cores = os.cpu_count() or 1
+    threads = min(cores, n_tok)
+    sec = oracle_tokens(host, np.arange(n_tok), threads)
+    sec1 = oracle_tokens(host, np.arange(1), 1)
+    return {"value": n_tok / sec, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n_tok} tokens: the first 2 batches of each row count "
+                      f"({', '.join(f'T={T}' for T in wl.T)}), fp64 route + monolith FFN in "
+                      f"one call each, OpenMP over tokens; inputs drawn on the host from "
+                      f"the workload's recipe",
+            "host_cores": cores, "cpu_model": cpu_model(),
+            "one_thread": {"value": 1.0 / sec1, "unit": "tokens/s", "sample": "1 token"}}
 
 
 def run_reference(args, wl):
-    """The oracle arm: the fp64 CPU oracle, as it stands, on this host's cores.
+    """The reference arm: the fp64 CPU oracle, as it stands, on this host's
+    cores.  Nothing here loads the CUDA library or touches a GPU.
 
-    A token of the workload costs its routing plus top_k + 1 expert
-    evaluations (routed picks and the shared expert).  Each step makes one
-    oracle call over `cores` (token, expert) evaluations, which the oracle
-    runs in parallel (OpenMP over its rows); each evaluation counts as
-    1 / (top_k + 1) of a token, and routing is timed when a token is first
-    met.  That bounds a step to about one expert evaluation of wall time, so
-    that K + W steps finish within a few minutes."""
+    The work is the workload's own tokens: the decode step's batches (T = 1,
+    4 and 8, drawn on the host).  A token of the workload costs its routing
+    plus top_k + 1 expert evaluations (routed picks and the shared expert).
+    When W + K whole steps fit the wall-time budget, a step is the workload's
+    tokens in one route and one FFN call; otherwise a step is one oracle FFN
+    call over a bounded number n of (token, expert) evaluations, each counted
+    as 1 / (top_k + 1) token, with a token's routing timed when it is first
+    met; n = the host's cores (at most the workload's evaluations), which run
+    side by side in about one evaluation's time."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    import oracle
-    torch.cuda.set_device(0)
-    o = oracle.load()
-    layer = Layer(wl, "cuda:0", workloads.SEED_BASE)
+    host = HostDecode(wl, n_batches=1)
     cores = os.cpu_count() or 1
-    W = layer.W
-    T0 = wl.T[-1]
-    x = layer.xs[T0][0]
-    xh = workloads.bits(x)
-    bias = None if W["bias"] is None else W["bias"].cpu().numpy()
-    wr = workloads.bits(W["w_router"])
-    ids, w, _ = o.route(xh, wr, bias, wl.top_k, threads=min(cores, T0))
-    # the evaluations of the batch: (token, expert slot); the shared expert is
-    # appended to the expert table as entry E so one call can mix both kinds
-    evals = [(t, int(ids[t, j]), float(w[t, j])) for t in range(T0) for j in range(wl.top_k)]
-    if layer.shared is not None:
-        evals += [(t, wl.E, 1.0) for t in range(T0)]
-    per_token = wl.top_k + (1 if layer.shared is not None else 0)
-    used = sorted(set(e for _, e, _ in evals if e < wl.E))
-    tables = []
-    for kname, sname in (("w_gate", "ws_gate"), ("w_up", "ws_up"), ("w_down", "ws_down")):
-        t = {e: workloads.bits(W[kname][e]) for e in used}
-        if layer.shared is not None:
-            t[wl.E] = workloads.bits(W[sname])
-        tables.append(t)
-    n = min(cores, len(evals))
+    xh = np.concatenate([x for _, x in host.batches], axis=0)
+    n_tok = xh.shape[0]
+    ids, w, _ = host.route(xh, min(cores, n_tok))
+    host.ensure(sorted(set(int(e) for e in ids.ravel())))
+    per_token = wl.top_k + (1 if host.shared is not None else 0)
+    steps = args.warmup + args.steps
+    # one whole step, timed once, decides the form of the steps
+    t_whole = oracle_tokens(host, np.arange(n_tok), min(cores, n_tok))
+    if steps * t_whole <= args.reference_budget_s:
+        mode = "whole"
+        threads = min(cores, n_tok)
+        sample = (f"each step: the workload's {n_tok} tokens (one batch each of "
+                  f"{', '.join(f'T={T}' for T in wl.T)}) through one fp64 route and one "
+                  f"monolith FFN call, OpenMP over tokens")
+    else:
+        # n <= cores evaluations run side by side in about one evaluation's
+        # time, so every core takes one
+        mode = "evaluations"
+        n = min(cores, n_tok * per_token)
+        threads = n
+        sample = (f"each step: {n} (token, expert) evaluations of the workload's {n_tok} "
+                  f"tokens (one batch each of {', '.join(f'T={T}' for T in wl.T)}) in one "
+                  f"oracle FFN call (OpenMP over rows), each 1/{per_token} token, a token's "
+                  f"routing timed when it is first met")
+    evals = [(t, int(ids[t, j]), float(w[t, j])) for t in range(n_tok) for j in range(wl.top_k)]
+    if host.shared is not None:
+        evals += [(t, wl.E, 1.0) for t in range(n_tok)]
+        tables = tuple({**m, wl.E: s} for m, s in zip(host.mats, host.shared))
+    else:
+        tables = host.mats
     total_tok, total_s = 0.0, 0.0
     seen = set()
-    for i in range(args.warmup + args.steps):
-        batch = [evals[(i * n + q) % len(evals)] for q in range(n)]
-        rows = np.array([t for t, _, _ in batch])
-        new = sorted(set(rows.tolist()) - seen)
-        t0 = time.perf_counter()
-        if new:
-            o.route(xh[new], wr, bias, wl.top_k, threads=min(cores, len(new)))
-        o.moe_ffn_monolith(xh[rows], np.array([[e] for _, e, _ in batch], dtype=np.int32),
-                           np.array([[wt] for _, _, wt in batch]), *tables, wl.E + 1,
-                           threads=n)
-        sec = time.perf_counter() - t0
-        seen.update(new)
-        if len(seen) == T0:
-            seen = set()
+    for i in range(steps):
+        if mode == "whole":
+            sec = oracle_tokens(host, np.arange(n_tok), threads)
+            tok = float(n_tok)
+        else:
+            batch = [evals[(i * threads + q) % len(evals)] for q in range(threads)]
+            rows = np.array([t for t, _, _ in batch])
+            new = sorted(set(rows.tolist()) - seen)
+            t0 = time.perf_counter()
+            if new:
+                host.route(xh[new], min(cores, len(new)))
+            host.o.moe_ffn_monolith(xh[rows], np.array([[e] for _, e, _ in batch], dtype=np.int32),
+                                    np.array([[wt] for _, _, wt in batch]), *tables, wl.E + 1,
+                                    threads=threads)
+            sec = time.perf_counter() - t0
+            seen.update(new)
+            if len(seen) == n_tok:
+                seen = set()
+            tok = threads / per_token
         if i >= args.warmup:
-            total_tok += n / per_token
+            total_tok += tok
             total_s += sec
     value = total_tok / total_s
-    sample = (f"each step: {n} (token, expert) evaluations of the T={T0} batch in one oracle "
-              f"call (OpenMP over rows), routing when a token is first met; a token = "
-              f"{per_token} evaluations")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total_s / max(args.steps, 1), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.description, "bands": wl.bands[0]},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": n, "kind": "oracle",
-                         "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": sample, "host_cores": cores, "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -367,19 +477,11 @@ def run_reference(args, wl):
 
 
 # -------------------------------------------------------------------- our arm
-def run_ours(args, wl):
+def measure(args, wl, device, rank, dist, peaks, K, warmup, sampler=None, with_graph=True,
+            e2e_steps=0):
+    """Every measurement of one workload: the timed steps, the per-kernel and
+    per-call passes, CUDA-graph replay and the end-to-end pass."""
     import expert_decode_b200 as ed
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
-    dist = None
-    if world > 1:
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=device)
-    peaks, peak_src = read_peaks()
     layer = Layer(wl, device, workloads.SEED_BASE + 7919 * rank)
     Ts = wl.T
     tensor_path = {T: T > 8 for T in Ts}
@@ -388,8 +490,6 @@ def run_ours(args, wl):
     # per (T, batch): distinct experts picked (fixed for a given batch)
     n_batches = {T: len(layer.xs[T]) for T in Ts}
     distinct = {(T, b): layer.distinct_experts(T, b) for T in Ts for b in range(n_batches[T])}
-    dom = ("gate/up GEMM (tcgen05)" if any(tensor_path.values()) else
-           "decode gate/up (tcgen05 from 2 tokens with bf16 x, CUDA cores below)")
     dom_index = {T: (2 if tensor_path[T] else 0) for T in Ts}   # kernel j of the ffn call
 
     def step(i, prof=None):
@@ -403,42 +503,53 @@ def run_ours(args, wl):
             if prof is not None:
                 ed.ep_profile_events(None)
 
-    for i in range(args.warmup):
+    for i in range(warmup):
         flush.zero_()
         step(i)
     torch.cuda.synchronize()
     ed.ep_check_status()
 
-    K = args.steps
     ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     layer.launches = 0
-    sampler = ClockSampler(device) if rank == 0 else None
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
-    if sampler:
+    if sampler is not None:
         sampler.start()
-    t_wall = time.perf_counter()
+    t_wall0 = time.time()
     # an NVTX range marks the timed launches for a profiler's launch filter
     # (ncu --nvtx --nvtx-include timed/)
     torch.cuda.nvtx.range_push("timed")
     for i in range(K):
         flush.zero_()
         ev_s[i].record()
-        step(args.warmup + i)
+        step(warmup + i)
         ev_e[i].record()
     torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
-    t_wall = time.perf_counter() - t_wall
-    clocks = sampler.stop() if sampler else None
+    t_wall1 = time.time()
+    clocks = sampler.stop((t_wall0, t_wall1)) if sampler is not None else None
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
     ed.ep_check_status()
     launches = layer.launches
 
-    # second pass of K steps, each kernel bracketed by its own events, for the
+    # per-call pass: events around each row count's route + forward only, so
+    # the kernels inside a call keep their early (programmatic) launches
+    call_s = {T: [torch.cuda.Event(enable_timing=True) for _ in range(K)] for T in Ts}
+    call_e = {T: [torch.cuda.Event(enable_timing=True) for _ in range(K)] for T in Ts}
+    for i in range(K):
+        flush.zero_()
+        for T in Ts:
+            call_s[T][i].record()
+            layer.call(T, warmup + i)
+            layer.ffn(T, warmup + i)
+            call_e[T][i].record()
+    torch.cuda.synchronize()
+
+    # per-kernel pass: every kernel bracketed by its own events, for the
     # dominant kernel's duration (events between launches stop the early
     # launch of the next kernel, so the throughput above is taken without them)
     nk = 10
@@ -451,7 +562,7 @@ def run_ours(args, wl):
     torch.cuda.synchronize()
     for i in range(K):
         flush.zero_()
-        step(args.warmup + i, prof[i])
+        step(warmup + i, prof[i])
     torch.cuda.synchronize()
 
     step_ms = [ev_s[i].elapsed_time(ev_e[i]) for i in range(K)]
@@ -463,20 +574,28 @@ def run_ours(args, wl):
     per_T = {}
     for T in Ts:
         j = dom_index[T]
-        durs, byts, fl = [], 0.0, 0.0
+        durs, byts, fl, cbytes, cflops = [], 0.0, 0.0, 0.0, 0.0
         for i in range(K):
-            b = args.warmup + i
+            b = warmup + i
             c = kernel_cost(wl, T, distinct[(T, b % n_batches[T])], tensor_path[T])
             durs.append(prof[i][T][2 * j].elapsed_time(prof[i][T][2 * j + 1]) / 1e3)
             byts += c["gu_bytes"]
             fl += c["gu_flops"]
-            step_bytes += c["call_bytes"]
-            step_flops += c["call_flops"]
+            cbytes += c["call_bytes"]
+            cflops += c["call_flops"]
+        step_bytes += cbytes
+        step_flops += cflops
         dom_bytes += byts
         dom_flops += fl
         dom_s += sum(durs)
-        per_T[f"T={T}"] = {"dominant_kernel_us": 1e6 * sum(durs) / K,
-                           "dominant_kernel_GBps": byts / sum(durs) / 1e9}
+        call_sec = sum(call_s[T][i].elapsed_time(call_e[T][i]) for i in range(K)) / 1e3
+        per_T[f"T={T}"] = {
+            "call_us": 1e6 * call_sec / K,
+            "call_hbm_GBps": cbytes / call_sec / 1e9,
+            "call_hbm_frac": cbytes / call_sec / 1e9 / peaks["hbm_gbs"],
+            "call_bytes": cbytes / K,
+            "dominant_kernel_us": 1e6 * sum(durs) / K,
+            "dominant_kernel_GBps": byts / sum(durs) / 1e9}
         # mean duration of every kernel of the route and forward calls
         if tensor_path[T]:
             names = ["plan", "gather", "gate_up", "down", "combine"]
@@ -485,8 +604,8 @@ def run_ours(args, wl):
         else:
             names = ["gate_up", "down_fold"]
         kus = {}
-        for j, name in enumerate(names):
-            kus[name] = 1e3 * sum(prof[i][T][2 * j].elapsed_time(prof[i][T][2 * j + 1])
+        for jj, name in enumerate(names):
+            kus[name] = 1e3 * sum(prof[i][T][2 * jj].elapsed_time(prof[i][T][2 * jj + 1])
                                   for i in range(K)) / K
         kus["router"] = 1e3 * sum(prof[i][("route", T)][0].elapsed_time(prof[i][("route", T)][1])
                                   for i in range(K)) / K
@@ -494,10 +613,10 @@ def run_ours(args, wl):
 
     value, dev_s_max = whole_job_throughput(tokens_rank, dev_s, dist, device)
 
-    # roofline of the dominant kernel
+    # roofline of the dominant kernel: the burst GEMM peak for short steps
+    peak_tf_key = "bf16_tflops_sustained" if dev_s / K >= SUSTAINED_AFTER_S else "bf16_tflops"
+    peak_tf = peaks[peak_tf_key]
     t_hbm = dom_bytes / (peaks["hbm_gbs"] * 1e9)
-    # the kernel is timed inside a long run of steps: the sustained GEMM peak
-    peak_tf = peaks["bf16_tflops_sustained"]
     t_tc = dom_flops / (peak_tf * 1e12)
     if t_hbm >= t_tc:
         roof = {"bound": "hbm", "achieved": dom_bytes / dom_s / 1e9, "peak": peaks["hbm_gbs"],
@@ -509,13 +628,14 @@ def run_ours(args, wl):
     kname = "grouped_gemm_kernel<true>" if any(tensor_path.values()) else "decode_gate_up"
     roof["traffic"] = traffic_for(kname, wl.name)
     roof["kernel"] = kname
-    roof["peak_source"] = peak_src
+    roof["peak_source"] = "measured" if peaks.get("_source") == "measured" else "fallback"
+    roof["peak_key"] = "hbm_gbs" if roof["bound"] == "hbm" else peak_tf_key
 
     # the same steps replayed from CUDA graphs, one per input batch (the
     # kernels' launch attributes, programmatic dependent launch included, are
     # captured with them); the L2 flush stays outside the graphs
     graph = None
-    if args.graph_steps > 0:
+    if with_graph and args.graph_steps > 0:
         nb = min(len(layer.xs[T]) for T in Ts)
         graphs = []
         for b in range(nb):
@@ -524,7 +644,7 @@ def run_ours(args, wl):
                 step(b)
             graphs.append(g)
         torch.cuda.synchronize()
-        KG = args.graph_steps
+        KG = min(args.graph_steps, K) if wl.T[0] > 8 else args.graph_steps
         gs = [torch.cuda.Event(enable_timing=True) for _ in range(KG)]
         ge = [torch.cuda.Event(enable_timing=True) for _ in range(KG)]
         for i in range(KG):
@@ -541,8 +661,8 @@ def run_ours(args, wl):
 
     # e2e: inputs from pinned host memory, y back to pinned host, in the region
     e2e = None
-    if args.e2e_steps > 0:
-        KE = min(args.e2e_steps, K)
+    if e2e_steps > 0:
+        KE = e2e_steps
         hx = {T: [x.cpu().pin_memory() for x in layer.xs[T]] for T in Ts}
         dx = {T: torch.empty_like(layer.xs[T][0]) for T in Ts}
         hy = {T: torch.empty((T, wl.H), dtype=torch.float32).pin_memory() for T in Ts}
@@ -569,41 +689,103 @@ def run_ours(args, wl):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": KE,
                "l2": "not flushed"}
 
+    step_s = dev_s / K
+    out = {
+        "value": value, "ms_per_step": 1e3 * dev_s_max / K, "steps": K, "warmup": warmup,
+        "roofline": roof, "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
+        "per_T": per_T, "cuda_graph": graph,
+        "step_hbm_GBps": step_bytes / dev_s / 1e9,
+        "step_hbm_frac": step_bytes / dev_s / 1e9 / peaks["hbm_gbs"],
+        "step_tflops": step_flops / dev_s / 1e12,
+        "step_tensor_frac": step_flops / dev_s / 1e12 / peak_tf,
+        "step_tensor_peak_key": peak_tf_key,
+        "step_roofline_frac": max(step_bytes / (peaks["hbm_gbs"] * 1e9),
+                                  step_flops / (peak_tf * 1e12)) / step_s,
+        "wall_s": t_wall1 - t_wall0,
+    }
+    del layer, flush
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_ours(args, wl):
+    import expert_decode_b200 as ed  # noqa: F401  (the library must load)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+    peaks, peak_src = read_peaks()
+    peaks["_source"] = peak_src
+    K = args.steps
+    sampler = ClockSampler(device) if rank == 0 else None
+    head = measure(args, wl, device, rank, dist, peaks, K, args.warmup, sampler,
+                   e2e_steps=min(args.e2e_steps, K))
+
+    if args.detail is None:
+        detail_names = list(DETAIL_CONFIGS) if wl.name == "decode" else []
+    elif args.detail == "none":
+        detail_names = []
+    else:
+        detail_names = [n for n in args.detail.split(",") if n]
+    configs = {}
+    for name in detail_names:
+        dwl = workloads.WORKLOADS[name]
+        KD = max(1, min(args.detail_steps, K))
+        s2 = ClockSampler(device) if rank == 0 else None
+        r = measure(args, dwl, device, rank, dist, peaks, KD, max(3, min(args.warmup, 10)), s2,
+                    with_graph=False, e2e_steps=min(args.e2e_steps, KD))
+        per = r["per_T"][f"T={dwl.T[0]}"]
+        configs[name] = {
+            "workload": dwl.description, "bands": dwl.bands[0], "value": r["value"],
+            "unit": "tokens/s", "ms_per_step": r["ms_per_step"], "steps": KD,
+            "warmup": r["warmup"], "e2e": r["e2e"],
+            "step_hbm_frac": r["step_hbm_frac"], "step_tflops": r["step_tflops"],
+            "step_tensor_frac": r["step_tensor_frac"],
+            "step_tensor_peak_key": r["step_tensor_peak_key"],
+            "step_roofline_frac": r["step_roofline_frac"], "roofline": r["roofline"],
+            "kernels_us": per["kernels_us"], "call_us": per["call_us"], "clocks": r["clocks"]}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        threads = os.cpu_count() or 1
-        rows = {T: min(T, 8) for T in Ts}
-        tok, sec = oracle_sample(layer, rows, threads, batches=2)
-        cpu = {"value": tok / sec, "unit": "tokens/s", "cores": min(threads, max(rows.values())),
-               "kind": "oracle",
-               "sample": "first 2 batches of each row count ("
-                         + ", ".join(f"{n} of T={T}" for T, n in rows.items())
-                         + "), fp64 route + monolith FFN, OpenMP over tokens"}
+        cpu = cpu_baseline(wl)
 
     if dist is not None:
         dist.destroy_process_group()
     if rank != 0:
         return
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
-        "warmup": args.warmup, "ms_per_step": 1e3 * dev_s_max / K, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
         "config": {"workload": wl.description, "bands": wl.bands[0],
                    "l2": "flushed before every step (512 MiB write)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "batches": "16 distinct x batches per row count, cycled",
                    "roofline_timing": "dominant kernel timed in a second pass of K steps "
                                       "with events around each kernel"},
-        "roofline": roof,
+        "roofline": head["roofline"],
         "cpu_baseline": cpu,
-        "e2e": e2e,
-        "gpu_launches": launches,
-        "clocks": clocks,
-        "detail": {"per_T": per_T, "wall_s": t_wall, "cuda_graph": graph,
-                   "step_hbm_GBps": step_bytes / dev_s / 1e9,
-                   "step_hbm_frac": step_bytes / dev_s / 1e9 / peaks["hbm_gbs"],
-                   "step_tflops": step_flops / dev_s / 1e12,
-                   "dominant_kernel": dom},
+        "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"],
+        "clocks": head["clocks"],
+        "detail": {"per_T": head["per_T"], "wall_s": head["wall_s"],
+                   "cuda_graph": head["cuda_graph"],
+                   "step_hbm_GBps": head["step_hbm_GBps"],
+                   "step_hbm_frac": head["step_hbm_frac"],
+                   "step_tflops": head["step_tflops"],
+                   "step_tensor_frac": head["step_tensor_frac"],
+                   "peak_source": peak_src,
+                   "dominant_kernel": ("gate/up GEMM (tcgen05)" if wl.T[0] > 8 else
+                                       "decode gate/up (tcgen05 from 2 tokens with bf16 x, "
+                                       "CUDA cores below)"),
+                   "configs": configs},
     }
     print(json.dumps(line), flush=True)
 
@@ -613,10 +795,7 @@ def run_router_only(args, wl):
     import expert_decode_b200 as ed
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
-    w_router = workloads._bf16_normal((wl.E, wl.H), workloads.SEED_BASE + 1, device,
-                                      workloads.WEIGHT_STD)
-    bias = workloads.router_bias(wl.bias, wl.E)
-    bias = None if bias is None else bias.to(device)
+    w_router, bias = workloads.make_router(wl, device)
     for T in wl.T:
         x = workloads.make_x(wl, T, device=device)
         ids = torch.empty((T, wl.top_k), dtype=torch.int32, device=device)

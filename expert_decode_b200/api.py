@@ -29,6 +29,11 @@ class EPError(RuntimeError):
         self.code = code
 
 
+class WorkspaceLayout(ctypes.Structure):
+    _fields_ = [("bytes", ctypes.c_size_t), ("contrib_offset", ctypes.c_size_t),
+                ("shared_offset", ctypes.c_size_t)]
+
+
 class Plan(ctypes.Structure):
     _fields_ = [("num_experts", ctypes.c_int32), ("bands", ctypes.c_int32),
                 ("band_start", ctypes.c_int32 * (EP_MAX_BANDS + 1))]
@@ -56,6 +61,8 @@ def library():
                                               ctypes.c_float, P, P, P]
             lib.moe_ffn_workspace_size.argtypes = [I64, I64, I64, I32, I64, I64]
             lib.moe_ffn_workspace_size.restype = SZ
+            lib.moe_ffn_workspace_layout.argtypes = [I64, I64, I64, I32, I64, I64,
+                                                     ctypes.POINTER(WorkspaceLayout)]
             lib.moe_ffn_forward.argtypes = [P, ctypes.c_int, I64, I64, P, P, I32, P, P, P, I64,
                                             I64, P, P, P, I64, ctypes.POINTER(Plan), P, P, SZ, P]
             lib.moe_ffn_forward_noalloc.argtypes = [P, ctypes.c_int, I64, I64, P, P, I32, P, P,
@@ -68,6 +75,7 @@ def library():
             lib.ep_profile_events.argtypes = [P, I32]
             lib.ep_profile_events.restype = ctypes.c_int
             for fn in ("ep_plan", "moe_route", "moe_route_sigmoid", "moe_ffn_forward",
+                       "moe_ffn_workspace_layout",
                        "moe_ffn_forward_noalloc",
                        "ep_set_dispatch", "ep_check_status"):
                 getattr(lib, fn).restype = ctypes.c_int
@@ -156,6 +164,16 @@ def moe_route_sigmoid(x, w_router, bias, top_k, normalize=False, scale=1.0, ids=
 def moe_ffn_workspace_size(T, H, E, top_k, I, I_s):
     return int(library().moe_ffn_workspace_size(int(T), int(H), int(E), int(top_k), int(I),
                                                 int(I_s)))
+
+
+def moe_ffn_workspace_layout(T, H, E, top_k, I, I_s):
+    """Byte offsets, inside moe_ffn_forward's workspace, of the per-pick
+    contributions [T * top_k, H] fp32 and the shared expert's output [T, H]
+    fp32 that the tensor-core paths fold into y; returns a WorkspaceLayout."""
+    out = WorkspaceLayout()
+    _check(library().moe_ffn_workspace_layout(int(T), int(H), int(E), int(top_k), int(I),
+                                              int(I_s), ctypes.byref(out)))
+    return out
 
 
 def moe_ffn_forward(x, ids, weights, w_gate, w_up, w_down, shared, plan, y=None,

@@ -4,8 +4,8 @@
 // benchmark", "What landed": the experts are split into contiguous bands
 // (ExpertParallelPlan), every rank computes the partial FFN output of the
 // picks that fall in its band, and the partials are summed in rank order.
-// TensorFold #310's maintainer's reply: one fixed order of the sum however
-// the slices fall over ranks.
+// TensorFold #310's maintainer's reply: the sum is taken in one order that
+// does not depend on which rank holds which slice.
 //
 //  * ep_band_ids_kernel: a rank's view of the picks.  Ids inside its band
 //    [e_lo, e_hi) become band-local ids (e - e_lo, matching weights that hold

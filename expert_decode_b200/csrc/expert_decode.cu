@@ -524,6 +524,27 @@ extern "C" size_t moe_ffn_workspace_size(int64_t T, int64_t H, int64_t E, int32_
     return workspace_layout(T, H, E, top_k, I, I_s).total;
 }
 
+extern "C" ep_status moe_ffn_workspace_layout(int64_t T, int64_t H, int64_t E, int32_t top_k,
+                                             int64_t I, int64_t I_s, ep_workspace_layout_t *out) {
+    if (out == nullptr)
+        return fail(EP_EINVAL, "moe_ffn_workspace_layout: out is NULL");
+    if (T < 0 || T > kMaxT || T * (int64_t)std::max(top_k, 1) > kMaxPairs || H < 8 ||
+        H > kMaxH || H % 8 != 0 || E < 1 || E > kMaxE || top_k < 1 || top_k > kMaxTopK ||
+        top_k > E || I < 8 || I > kMaxI || I % 8 != 0 ||
+        (I_s != 0 && (I_s < 8 || I_s > kMaxI || I_s % 8 != 0)))
+        return fail(EP_EINVAL, "moe_ffn_workspace_layout: sizes out of range");
+    ep_workspace_layout_t l;
+    memset(&l, 0, sizeof l);
+    if (T > 0) {
+        const Workspace W = workspace_layout(T, H, E, top_k, I, I_s);
+        l.bytes = W.total;
+        l.contrib_offset = W.grouped.c;
+        l.shared_offset = W.grouped.s;
+    }
+    *out = l;
+    return ok();
+}
+
 namespace {
 
 // moe_ffn_forward's body.  band_call: a band partial (moe_ffn_partial), whose

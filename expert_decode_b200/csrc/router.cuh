@@ -1,8 +1,8 @@
 // router.cuh -- replicated softmax router with top-k and renormalisation.
 //
 // fak note "GLM-5.2 multi-GPU: expert-parallel sharding + the resident-fit
-// benchmark", "What landed": the router runs replicated and every rank picks
-// the same top-k.  Softmax over the logits, top_k by logit with ties to the
+// benchmark", "What landed": each rank holds a copy of the router and runs it
+// on the same rows, so the ranks agree on the picks.  Softmax over the logits, top_k by logit with ties to the
 // lower expert id, weights renormalised over the picked set.
 //
 // Two kernels, both launched as clusters of CTAs that split the experts and
@@ -190,7 +190,7 @@ __device__ void topk_softmax_warp(const double *lt, int E, int top_k, int32_t *i
     }
 }
 
-// Sigmoid router (the GLM variant: sigmoid + bias top-k, raw-score weights;
+// Sigmoid router (the GLM variant: sigmoid scores, a bias used in the selection only, weights from the unbiased scores;
 // TensorFold #593, "What exists now", glm_route.cu): the picks by key =
 // score + bias, weights = scale * score, or scale * score / (sum of the
 // picked scores) with normalize.

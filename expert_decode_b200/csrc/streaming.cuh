@@ -22,8 +22,8 @@
 //    picked experts in ascending (id, repeat) order, folding w * (W_down h)
 //    into one fp32 running sum per (feature, token); y = routed + shared.
 //    The walk is the bands in rank order with the carry passed along
-//    (TensorFold issue #310, maintainer's reply: one fixed sum order however
-//    the slices fall over ranks), so y does not depend on the plan; the
+//    (TensorFold issue #310, maintainer's reply: the order of the sums does
+//    not depend on where the slices live), so y does not depend on the plan; the
 //    shared expert enters after the routed sum (the GLM shared-expert wrapper
 //    of the fak note's gate table).
 //

@@ -2,8 +2,8 @@
  * expert_decode.h -- C ABI of the B200 (sm_100a) routed MoE FFN with an
  * expert-parallel band decomposition.
  *
- * The operation.  A replicated router picks the same top-k experts for every
- * rank; the experts are split into contiguous bands, one band per rank, and
+ * The operation.  Every rank runs one copy of the router on the same rows, so
+ * all ranks agree on the picked experts; the experts are split into contiguous bands, one band per rank, and
  * each band's SwiGLU experts contribute an [H] partial that is summed in rank
  * order (fak note "GLM-5.2 multi-GPU: expert-parallel sharding + the
  * resident-fit benchmark", section "What landed": ExpertParallelPlan, one
@@ -75,16 +75,22 @@ typedef struct {
 ep_status ep_plan(int32_t num_experts, int32_t bands, ep_plan_t *out);
 
 /*
- * moe_route -- the replicated router (fak note "GLM-5.2 multi-GPU", "What
- * landed": the router runs replicated and picks the same top-k).
+ * moe_route -- the router, one copy of which every rank runs on the same rows
+ * so that all ranks agree on the picks (fak note "GLM-5.2 multi-GPU", "What
+ * landed").
  *   l[t,e] = sum_h x[t,h] * W_router[e,h] + bias[e]
  *   p = softmax(l); S = the top_k experts by logit, ties to the lower id;
  *   weights[t,j] = p[S_j] / sum_{e in S} p[e]
  * ids[t,:] are written in descending weight order (equal weights: ascending
- * id).  The selection and the weights are decided on fp64 logits: logits are
- * first accumulated in fp32 with a proven error bound, and every expert that
- * could be in the top-k under that bound is recomputed in fp64 before the
- * pick, so the result equals the exact-arithmetic top-k up to fp64 rounding.
+ * id).  The pick is decided on compensated fp32 logits (Dot2, Ogita, Rump and
+ * Oishi 2005): every product is exact in fp32 and the running sum carries its
+ * own rounding error, so a logit is within about 1e-9 (relative to
+ * sum_h |x_h W_h|) of its exact value.  Up to 32 tokens every logit is formed
+ * that way; above, fp32 logits with a proven error bound come first and every
+ * expert that could still reach the top_k under that bound is recomputed by
+ * Dot2 before the pick.  The selection and its order therefore equal those of
+ * exact arithmetic, except between logits closer than the Dot2 bound; the
+ * weights carry that error plus one fp32 rounding.
  *
  *   x         device, [T, H], bf16 (EP_BF16) or fp32 (EP_F32)
  *   w_router  device, [E, H] bf16, one row per expert
@@ -99,9 +105,10 @@ ep_status moe_route(const void *x, ep_dtype x_dtype, int64_t T, int64_t H,
                     int32_t *ids, float *weights, void *stream);
 
 /*
- * moe_route_sigmoid -- the GLM router variant: "sigmoid + bias top-k,
- * raw-score weights" (TensorFold #593, a contributor's comment "What exists
- * now", glm_route.cu).  The page names the ingredients only; read as:
+ * moe_route_sigmoid -- the GLM router variant (TensorFold #593, a
+ * contributor's comment "What exists now", glm_route.cu), which the page
+ * describes only by its parts: a sigmoid score, a bias that takes part in
+ * the top-k choice, and weights taken from the unbiased scores.  Read as:
  *   l_e = sum_h x[t,h] W_router[e,h]       (no bias)
  *   s_e = 1 / (1 + exp(-l_e))              the score
  *   S   = top_k experts by s_e + bias[e]   (the bias moves the selection only),
@@ -110,8 +117,9 @@ ep_status moe_route(const void *x, ep_dtype x_dtype, int64_t T, int64_t H,
  *   weights[t,j] = scale * s_{S_j} / sum over S of s
  * ids written by descending s + bias.  Arguments, layouts, limits and errors
  * as moe_route, plus normalize (0 or 1) and scale (finite, > 0; else
- * EP_EINVAL).  The logits are compensated fp32 sums as in moe_route; the
- * scores and keys are formed from them in fp64.
+ * EP_EINVAL).  The logits are the compensated fp32 (Dot2) sums of moe_route,
+ * with the same candidate refinement above 32 tokens; the scores and keys
+ * are formed from them in fp64.
  */
 ep_status moe_route_sigmoid(const void *x, ep_dtype x_dtype, int64_t T, int64_t H,
                             const void *w_router, const float *bias, int64_t E, int32_t top_k,
@@ -129,17 +137,42 @@ size_t moe_ffn_workspace_size(int64_t T, int64_t H, int64_t E, int32_t top_k, in
                               int64_t I_s);
 
 /*
+ * moe_ffn_workspace_layout -- where moe_ffn_forward keeps, inside its
+ * workspace, the two results that its last step (the fold) reads, so that a
+ * caller can check that step on its own.  After a moe_ffn_forward call with
+ * these sizes that ran the grouped tensor-core path (T > 8) or the
+ * tensor-core streaming kernels (2 <= T <= 8 with bf16 x):
+ *   contrib  [T * top_k, H] fp32 at byte offset contrib_offset: row
+ *            t * top_k + j holds weights[t,j] * f_e(x[t]) of pick (t, j), as
+ *            rounded to fp32 (rows of skipped picks are not written);
+ *   shared   [T, H] fp32 at byte offset shared_offset: f_shared(x[t])
+ *            (written only when I_s > 0);
+ * and y[t] is the left fold of t's valid contrib rows in ascending (expert
+ * id, j), then + shared[t].  The CUDA-core streaming kernels (T = 1, or fp32
+ * x) fold on chip and write neither.  bytes = moe_ffn_workspace_size.  The
+ * sizes are checked as moe_ffn_forward checks them (EP_EINVAL), and T = 0
+ * gives an all-zero layout.
+ */
+typedef struct {
+    size_t bytes;
+    size_t contrib_offset;
+    size_t shared_offset;
+} ep_workspace_layout_t;
+ep_status moe_ffn_workspace_layout(int64_t T, int64_t H, int64_t E, int32_t top_k, int64_t I,
+                                   int64_t I_s, ep_workspace_layout_t *out);
+
+/*
  * moe_ffn_forward -- the routed MoE FFN with the shared expert.
  * For every token t and pick j (e = ids[t,j], w = weights[t,j]):
  *   f_e(x) = W_down[e] (silu(W_gate[e] x) * (W_up[e] x)),  silu(g) = g/(1+e^-g)
  *   (expertSwiGLU, fak note "GLM-5.2 multi-GPU", "What is not yet" update)
  *   y[t] = fold over the picks in ascending (expert id, j) of w * f_e(x[t]),
  *          then + f_shared(x[t]) when I_s > 0.
- * The fold runs band by band in rank order and passes its running sum from
- * one band to the next, so it is one fixed sum order whatever the plan
- * (TensorFold #310, maintainer's reply: every sum follows one fixed tree of
- * slices however the slices fall over ranks): y is bit-identical for every
- * plan and from run to run.
+ * The fold runs band by band in rank order and hands its running sum from
+ * one band to the next, so the order of the additions is the same for every
+ * plan (TensorFold #310, maintainer's reply: one sum order that does not
+ * depend on how the slices are placed on ranks): y is bit-identical for
+ * every plan and from run to run.
  *
  *   x        device, [T, H], bf16 or fp32
  *   ids      device, [T, top_k] int32 expert ids (any order, repeats allowed)
@@ -156,10 +189,15 @@ size_t moe_ffn_workspace_size(int64_t T, int64_t H, int64_t E, int32_t top_k, in
  * Limits: 0 <= T <= 65536, T * top_k <= 2^20; 8 <= H <= 16384; 1 <= E <= 1024;
  * 1 <= top_k <= min(E, 16); 8 <= I, I_s <= 16384 (I_s may be 0); H, I and
  * I_s multiples of 8.
- * Precision: bf16 products, fp32 accumulation.  Up to 8 rows the weights are
- * streamed by a CUDA-core path that keeps the SwiGLU activations in fp32;
- * above that, tensor-core tiles round the activations to bf16 between the
- * two projections.
+ * Precision: bf16 products, fp32 accumulation, fp32 routing weight applied
+ * to the down projection's fp32 result.  The SwiGLU activations h between the
+ * two projections are kept as follows:
+ *   - T = 1, or fp32 x, up to 8 rows: fp32 (CUDA-core streaming kernels);
+ *   - 2 <= T <= 8 with bf16 x: as the two bf16 parts hi = bf16(h) and
+ *     lo = bf16(h - hi), about 16 significant bits (tensor-core streaming
+ *     kernels);
+ *   - T > 8: rounded to bf16 once (grouped tensor-core GEMMs).
+ * x in fp32 is rounded to bf16 on the tensor-core paths.
  */
 ep_status moe_ffn_forward(const void *x, ep_dtype x_dtype, int64_t T, int64_t H,
                           const int32_t *ids, const float *weights, int32_t top_k,

@@ -29,7 +29,8 @@
  * notes: softmax router with renormalised top-k, ties to the lower expert id,
  * picks folded in ascending (expert id, slot), the shared expert added after
  * the routed sum, routed scaling factor 1.  The GLM router variant of the
- * tracker page (sigmoid + bias top-k, raw-score weights) is read as in
+ * tracker page (a sigmoid score, a bias in the selection, weights from the
+ * unbiased scores) is read as in
  * oracle_route_sigmoid below.
  */
 #include <math.h>
@@ -108,8 +109,8 @@ static int ranks_before(double la, int32_t ea, double lb, int32_t eb)
 }
 
 /*
- * The replicated router picks the same top-k on every rank [EP, "What
- * landed"].  For token t:
+ * Every rank runs its own copy of the router on the same rows and so gets the
+ * same picks [EP, "What landed"].  For token t:
  *   l_e = sum_h x[t,h] * W_r[e,h] + b_e                (sequential over h)
  *   p   = softmax(l), computed with the largest logit subtracted
  *   S   = the top_k experts by logit, ties to the lower id
@@ -193,8 +194,9 @@ int oracle_route(const void *x, int x_is_f32, int64_t T, int64_t H,
 
 /*
  * The GLM router variant [GATE page, a contributor's comment "What exists
- * now": glm_route.cu, "sigmoid + bias top-k, raw-score weights"].  The page
- * names only the three ingredients; they are read here as:
+ * now": glm_route.cu, described only as a sigmoid score, a bias in the top-k
+ * choice and weights from the unbiased scores].  The page names only these
+ * three ingredients; they are read here as:
  *   l_e = sum_h x[t,h] * W_r[e,h]          (sequential over h, no bias)
  *   s_e = 1 / (1 + exp(-l_e))              the expert's score
  *   k_e = s_e + b_e                        the bias moves the selection only

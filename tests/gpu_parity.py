@@ -97,6 +97,56 @@ def oracle_ffn(o, x, ids, weights, W, bands=None, rows=None, threads=8):
                                      threads=threads)
 
 
+def oracle_ffn_rows(o, x, ids, weights, W, rows, chunk=8, threads=8):
+    """oracle_ffn on the given rows, `chunk` rows per oracle call so that the
+    host copies of the experts they pick stay bounded (a few GB)."""
+    rows = np.asarray(rows)
+    parts = [oracle_ffn(o, x, ids, weights, W, rows=rows[i:i + chunk], threads=threads)
+             for i in range(0, len(rows), chunk)]
+    return np.concatenate(parts, axis=0)
+
+
+def spread_rows(ids, E, n_min=64, n_tile=256):
+    """Rows (tokens) that cover the grouped GEMMs' tiling of this batch:
+      * for the three most-picked experts, the first and last token of every
+        n_tile-row N tile of the expert's group (rows in (token, slot) order);
+      * for every group-size class of the activation boxes (1-32, 33-64,
+        65-128, 129-256, more), the first and last token of one expert of
+        that class, and of the least-picked expert present;
+      * the first and last tokens, and an even spread up to n_min rows."""
+    ids = np.asarray(ids)
+    T, k = ids.shape
+    flat = ids.reshape(-1)
+    groups = {}
+    for p, e in enumerate(flat.tolist()):
+        if 0 <= e < E:
+            groups.setdefault(e, []).append(p // k)
+    picked = {0, T - 1}
+    by_size = sorted(groups, key=lambda e: (-len(groups[e]), e))
+    for e in by_size[:3]:
+        toks = groups[e]
+        for n0 in range(0, len(toks), n_tile):
+            picked.add(toks[n0])
+            picked.add(toks[min(n0 + n_tile, len(toks)) - 1])
+    classes = [(1, 32), (33, 64), (65, 128), (129, 256), (257, 1 << 30)]
+    for lo, hi in classes:
+        for e in sorted(groups):
+            if lo <= len(groups[e]) <= hi:
+                picked.update((groups[e][0], groups[e][-1]))
+                break
+    if by_size:
+        last = by_size[-1]
+        picked.update((groups[last][0], groups[last][-1]))
+    step = max(1, T // n_min)
+    t = 0
+    while len(picked) < min(n_min, T):
+        picked.add(t % T)
+        t += step
+        if t >= T:
+            t = t % T + 1
+    return np.array(sorted(picked))
+
+
 def gpu_ffn(x, ids, weights, W, plan, **kw):
     y = ed.moe_ffn_forward(x, ids, weights, W["w_gate"], W["w_up"], W["w_down"], shared_of(W),
                            plan, **kw)

@@ -1,5 +1,5 @@
 """moe_route_sigmoid (the GLM router variant: sigmoid scores, the bias moves
-the selection only, raw-score weights) on the GPU against the fp64 oracle:
+the selection only, weights from the unbiased scores) on the GPU against the fp64 oracle:
 ids exact except where the oracle's own keys tie within 1e-6, weights within
 1e-6 of the oracle's (relative to the scale), run-to-run identical."""
 import ctypes

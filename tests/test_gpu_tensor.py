@@ -8,7 +8,8 @@ import torch
 
 import workloads
 import expert_decode_b200 as ed
-from gpu_parity import check_y, device_inputs, gpu_ffn, oracle_ffn, oracle_route
+from gpu_parity import (check_route, check_y, device_inputs, gpu_ffn, oracle_ffn,
+                        oracle_ffn_rows, oracle_route, spread_rows)
 
 pytestmark = pytest.mark.gpu
 WL = workloads.WORKLOADS
@@ -21,26 +22,28 @@ def tensor_dispatch():
     ed.ep_set_dispatch("auto")
 
 
-def _routed(o, wl, T, seed=workloads.SEED_BASE, batch=0, rows=None, **sizes):
+def _routed(o, wl, T, seed=workloads.SEED_BASE, batch=0, **sizes):
+    """GPU-routed inputs whose ids equal the oracle's; returns the GPU's ids and
+    weights (the forward's inputs) and the oracle's weights (the reference's)."""
     W, x = device_inputs(wl, T, seed=seed, batch=batch, **sizes)
     ids, w = ed.moe_route(x, W["w_router"], W["bias"], wl.top_k)
     torch.cuda.synchronize()
-    ids_ref, w_ref, _ = oracle_route(o, x, W, wl.top_k, rows=rows)
-    got = ids.cpu().numpy() if rows is None else ids.cpu().numpy()[rows]
-    assert np.array_equal(got, ids_ref)
-    return W, x, ids, w
+    ids_ref, w_ref, logits = oracle_route(o, x, W, wl.top_k)
+    assert check_route(ids, w, ids_ref, w_ref, logits) == 0
+    return W, x, ids, w, w_ref
 
 
 def test_tiny_tensor_path_all_bands(oracle_lib):
     wl = WL["tiny"]
-    W, x, ids, w = _routed(oracle_lib, wl, 24)
+    W, x, ids, w, w_ref = _routed(oracle_lib, wl, 24)
     ys = [gpu_ffn(x, ids, w, W, ed.ep_plan(wl.E, R)) for R in (1, 2, 4, 8)]
     ed.ep_check_status()
     assert ed.ep_last_launch_count() == 5
     for y in ys[1:]:
         assert torch.equal(y, ys[0])
-    check_y(ys[0], oracle_ffn(oracle_lib, x, ids, w, W), what="tiny T=24 tensor")
-    check_y(ys[0], oracle_ffn(oracle_lib, x, ids, w, W, bands=oracle_lib.expert_parallel_plan(16, 4)),
+    check_y(ys[0], oracle_ffn(oracle_lib, x, ids, w_ref, W), what="tiny T=24 tensor")
+    check_y(ys[0], oracle_ffn(oracle_lib, x, ids, w_ref, W,
+                             bands=oracle_lib.expert_parallel_plan(16, 4)),
             what="tiny T=24 tensor vs EP(4)")
 
 
@@ -48,17 +51,17 @@ def test_tiny_tensor_path_all_bands(oracle_lib):
 def test_ragged_multi_tile(oracle_lib, T):
     """H, I, I_s not multiples of the tile; groups of every size incl. > 256 rows."""
     wl = workloads.Workload("ragged", (T,), 200, 12, 6, 136, 72, "bf16", "none", (3,))
-    W, x, ids, w = _routed(oracle_lib, wl, T, seed=31)
+    W, x, ids, w, w_ref = _routed(oracle_lib, wl, T, seed=31)
     y = gpu_ffn(x, ids, w, W, ed.ep_plan(wl.E, 3))
     ed.ep_check_status()
-    check_y(y, oracle_ffn(oracle_lib, x, ids, w, W), what=f"ragged T={T}")
+    check_y(y, oracle_ffn(oracle_lib, x, ids, w_ref, W), what=f"ragged T={T}")
 
 
 def test_fp32_activations(oracle_lib):
     wl = workloads.Workload("f32", (40,), 256, 16, 4, 128, 128, "f32", "none", (2,))
-    W, x, ids, w = _routed(oracle_lib, wl, 40, seed=3)
+    W, x, ids, w, w_ref = _routed(oracle_lib, wl, 40, seed=3)
     y = gpu_ffn(x, ids, w, W, ed.ep_plan(wl.E, 2))
-    check_y(y, oracle_ffn(oracle_lib, x, ids, w, W), what="fp32 x tensor")
+    check_y(y, oracle_ffn(oracle_lib, x, ids, w_ref, W), what="fp32 x tensor")
 
 
 def test_hot_expert_many_tiles(oracle_lib):
@@ -76,20 +79,20 @@ def test_hot_expert_many_tiles(oracle_lib):
 
 def test_tensor_matches_streaming_within_tolerance(oracle_lib):
     wl = WL["decode"]
-    W, x, ids, w = _routed(oracle_lib, wl, 8, batch=2)
+    W, x, ids, w, w_ref = _routed(oracle_lib, wl, 8, batch=2)
     plan = ed.ep_plan(wl.E, 8)
     y_t = gpu_ffn(x, ids, w, W, plan)
     ed.ep_set_dispatch("streaming")
     y_s = gpu_ffn(x, ids, w, W, plan)
     ed.ep_set_dispatch("tensor")
-    ref = oracle_ffn(oracle_lib, x, ids, w, W)
+    ref = oracle_ffn(oracle_lib, x, ids, w_ref, W)
     check_y(y_t, ref, what="decode T=8 tensor")
     check_y(y_s, ref, rel_tol=1e-4, what="decode T=8 streaming")
 
 
 def test_repeated_and_bad_ids(oracle_lib):
     wl = WL["tiny"]
-    W, x, ids, w = _routed(oracle_lib, wl, 20, seed=14)
+    W, x, ids, w, w_ref = _routed(oracle_lib, wl, 20, seed=14)
     ed.ep_check_status()
     ids = ids.clone()
     ids[2, 1] = ids[2, 0]
@@ -97,35 +100,45 @@ def test_repeated_and_bad_ids(oracle_lib):
     y = gpu_ffn(x, ids, w, W, ed.ep_plan(wl.E, 4))
     with pytest.raises(ed.EPError):
         ed.ep_check_status()
-    ref_ids, ref_w = ids.clone(), w.clone()
+    ref_ids, ref_w = ids.clone(), w_ref.copy()
     ref_ids[5, 3] = 0
     ref_w[5, 3] = 0.0
     check_y(y, oracle_ffn(oracle_lib, x, ref_ids, ref_w, W), what="repeated / bad ids")
 
 
 # ------------------------------------------------------------ full-size workloads
-def _full(o, name, rows, bands):
+# At full size the oracle computes sampled rows only: at least 64, spread over
+# every N tile of the hottest experts, one expert of every activation-box
+# class and the least-picked expert (spread_rows).  The oracle routes those
+# rows itself; the GPU's ids must equal its ids there, and the FFN reference
+# takes the oracle's own ids and weights.
+def _full(o, name, bands):
     wl = WL[name]
     T = wl.T[0]
-    W, x, ids, w = _routed(o, wl, T, rows=rows)
+    W, x = device_inputs(wl, T)
+    ids, w = ed.moe_route(x, W["w_router"], W["bias"], wl.top_k)
     ys = [gpu_ffn(x, ids, w, W, ed.ep_plan(wl.E, R)) for R in bands]
     ed.ep_check_status()
     for y in ys[1:]:
         assert torch.equal(y, ys[0]), "band counts differ"
     assert torch.equal(gpu_ffn(x, ids, w, W, ed.ep_plan(wl.E, bands[0])), ys[0]), "runs differ"
-    ref = oracle_ffn(o, x, ids, w, W, rows=rows)
-    check_y(ys[0][rows], ref, what=f"{name} sampled rows")
+    rows = spread_rows(ids.cpu().numpy(), wl.E)
+    assert len(rows) >= 64
+    ids_ref, w_ref, logits = oracle_route(o, x, W, wl.top_k, rows=rows)
+    assert check_route(ids[rows], w[rows], ids_ref, w_ref, logits) == 0
+    ref = oracle_ffn_rows(o, x[rows], ids_ref, w_ref, W, np.arange(len(rows)))
+    check_y(ys[0][rows], ref, what=f"{name}: {len(rows)} sampled rows")
     return W, x, ids, w, ys[0]
 
 
 def test_prefill_full_size(oracle_lib):
-    _full(oracle_lib, "prefill", np.array([0, 1, 255, 511]), (4, 1, 2, 8))
+    _full(oracle_lib, "prefill", (4, 1, 2, 8))
 
 
 def test_imbalanced_full_size(oracle_lib):
-    W, x, ids, w, y = _full(oracle_lib, "imbalanced", np.r_[0:6, 1000:1004, 2042:2048], (4, 1))
+    W, x, ids, w, y = _full(oracle_lib, "imbalanced", (4, 1))
     assert int(ids.max()) < 16, "bias +8 on experts 0..15 must put every pick in band 0"
 
 
 def test_large_full_size(oracle_lib):
-    _full(oracle_lib, "large", np.array([0, 2047, 4095]), (8, 1))
+    _full(oracle_lib, "large", (8, 1))

@@ -47,6 +47,11 @@ def test_noalloc_matches_workspace_entry_point(T):
     y2 = torch.full((T, wl.H), float("nan"), dtype=torch.float32, device="cuda")
     _noalloc(x, ids, w, W, plan, y1)
     _noalloc(x, ids, w, W, plan, y2)
+    # the same kernels in the same order as the workspace entry point, so the
+    # same bits; a scratch area shared wrongly between steps or calls would
+    # show here first
+    assert torch.equal(y1, y_ref), f"noalloc T={T}: first call differs from moe_ffn_forward"
+    assert torch.equal(y2, y_ref), f"noalloc T={T}: second call differs from moe_ffn_forward"
     check_y(y1, ref, what=f"noalloc T={T} first call")
     check_y(y2, ref, what=f"noalloc T={T} second call")
 

@@ -67,12 +67,45 @@ def _bf16_normal(shape, seed, device, std):
     return _normal(shape, seed, device, std).to(torch.bfloat16)
 
 
+def _expert_seed(seed, e):
+    return seed * 1_000_003 + e
+
+
 def _expert_stack(E, rows, cols, seed, device):
     """[E, rows, cols] bf16, one seeded draw per expert (bounded temporaries)."""
     out = torch.empty((E, rows, cols), dtype=torch.bfloat16, device=device)
     for e in range(E):
-        out[e].copy_(_bf16_normal((rows, cols), seed * 1_000_003 + e, device, WEIGHT_STD))
+        out[e].copy_(_bf16_normal((rows, cols), _expert_seed(seed, e), device, WEIGHT_STD))
     return out
+
+
+# tensor index of each expert projection in make_weights' seed sequence
+_EXPERT_TENSORS = {"w_gate": 2, "w_up": 3, "w_down": 4}
+
+
+def make_expert(w: Workload, which: str, e: int, device="cpu", seed=SEED_BASE):
+    """One expert's matrix of make_weights (which = "w_gate", "w_up" or
+    "w_down"), drawn alone: the same values as make_weights(...)[which][e]
+    on the same device type."""
+    rows, cols = (w.I, w.H) if which in ("w_gate", "w_up") else (w.H, w.I)
+    return _bf16_normal((rows, cols), _expert_seed(seed + _EXPERT_TENSORS[which], e), device,
+                        WEIGHT_STD)
+
+
+def make_router(w: Workload, device="cpu", seed=SEED_BASE):
+    """(w_router, bias) of make_weights, without the experts."""
+    b = router_bias(w.bias, w.E)
+    return (_bf16_normal((w.E, w.H), seed + 1, device, WEIGHT_STD),
+            None if b is None else b.to(device))
+
+
+def make_shared(w: Workload, device="cpu", seed=SEED_BASE):
+    """(ws_gate, ws_up, ws_down) of make_weights, or None without a shared expert."""
+    if w.I_s == 0:
+        return None
+    return (_bf16_normal((w.I_s, w.H), seed + 5, device, WEIGHT_STD),
+            _bf16_normal((w.I_s, w.H), seed + 6, device, WEIGHT_STD),
+            _bf16_normal((w.H, w.I_s), seed + 7, device, WEIGHT_STD))
 
 
 def router_bias(kind: str, E: int) -> Optional[torch.Tensor]:
