@@ -89,6 +89,13 @@ def parse_args(argv=None):
                     help="profiling only: run moe_route alone on the workload's router weights, "
                          "bias and activations (no expert weights on the device) and print its "
                          "per-call time; no bench line")
+    ap.add_argument("--ep", action="store_true",
+                    help="expert parallel across the ranks: rank r holds band r of the experts "
+                         "(ep_plan(E, N)), every rank routes the same tokens, and the partials "
+                         "are exchanged by the rank-order reduce-scatter (strong scaling)")
+    ap.add_argument("--dispatch", default="auto",
+                    choices=("auto", "streaming", "tensor", "streaming_tc", "streaming_simt"),
+                    help="tuning: the path moe_ffn_forward takes (ep_set_dispatch)")
     ap.add_argument("--reference-budget-s", type=float, default=150.0,
                     help="wall-time budget of the reference arm's warm-up and timed steps")
     return ap.parse_args(argv)
@@ -709,7 +716,8 @@ def measure(args, wl, device, rank, dist, peaks, K, warmup, sampler=None, with_g
 
 
 def run_ours(args, wl):
-    import expert_decode_b200 as ed  # noqa: F401  (the library must load)
+    import expert_decode_b200 as ed  # the library must load
+    ed.ep_set_dispatch(args.dispatch)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -765,6 +773,7 @@ def run_ours(args, wl):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": wl.description, "bands": wl.bands[0],
+                   "dispatch": args.dispatch,
                    "l2": "flushed before every step (512 MiB write)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "batches": "16 distinct x batches per row count, cycled",
@@ -786,6 +795,88 @@ def run_ours(args, wl):
                                        "decode gate/up (tcgen05 from 2 tokens with bf16 x, "
                                        "CUDA cores below)"),
                    "configs": configs},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ep(args, wl):
+    """Band-resident expert parallelism across the ranks of one node: rank r
+    holds the experts of band r of ep_plan(E, N) only, every rank routes the
+    same batch, computes its band's partial, and the partials are folded in
+    rank order by the reduce-scatter exchange (expert_decode_b200.ep).  The
+    whole job processes each token once: value = tokens / slowest rank's
+    device time (strong scaling).  Collectives are NCCL's; the kernels read
+    this GPU's memory only."""
+    import expert_decode_b200 as ed
+    from expert_decode_b200 import ep
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+    plan = ed.ep_plan(wl.E, world)
+    lo, hi = plan.band_start[rank], plan.band_start[rank + 1]
+    band = tuple(torch.stack([workloads.make_expert(wl, which, e, device) for e in range(lo, hi)])
+                 for which in ("w_gate", "w_up", "w_down"))
+    w_router, bias = workloads.make_router(wl, device)
+    shared = workloads.make_shared(wl, device)
+    xs = {T: [workloads.make_x(wl, T, device=device, batch=b + 100 * T)
+              for b in range(N_BATCHES if T <= 8 else 2)] for T in wl.T}
+    flush = torch.empty(args.flush_mib << 20, dtype=torch.uint8, device=device)
+
+    def step(i):
+        for T in wl.T:
+            x = xs[T][i % len(xs[T])]
+            ids, w = ed.moe_route(x, w_router, bias, wl.top_k)
+            if dist is None:
+                ed.moe_ffn_forward(x, ids, w, *band, shared, plan)
+            else:
+                ep.ep_forward(x, ids, w, band, shared, plan, rank)
+
+    for i in range(args.warmup):
+        flush.zero_()
+        step(i)
+    torch.cuda.synchronize()
+    ed.ep_check_status()
+    K = args.steps
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.zero_()
+        ev_s[i].record()
+        step(args.warmup + i)
+        ev_e[i].record()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    ed.ep_check_status()
+    dev_s = sum(ev_s[i].elapsed_time(ev_e[i]) for i in range(K)) / 1e3
+    tokens = K * sum(wl.T)
+    if dist is not None:
+        t = torch.tensor([dev_s], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dev_s = float(t.item())
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": tokens / dev_s, "unit": "tokens/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": 1e3 * dev_s / K,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": wl.description, "bands": world,
+                   "parallelism": f"expert-parallel bands x{world} (rank-order reduce-scatter)",
+                   "l2": "flushed before every step (512 MiB write)"},
+        "roofline": None, "cpu_baseline": None, "e2e": None, "gpu_launches": None,
+        "clocks": None,
     }
     print(json.dumps(line), flush=True)
 
@@ -826,6 +917,8 @@ def main():
         run_reference(args, wl)
     elif args.router_only:
         run_router_only(args, wl)
+    elif args.ep:
+        run_ep(args, wl)
     else:
         run_ours(args, wl)
 

@@ -10,10 +10,18 @@ summed in rank order (TensorFold #310: one fixed order of that sum).
                    shared expert's output
   shared_expert    the shared expert's output alone (moe_ffn_forward with
                    every pick slot empty)
-  ep_forward       one rank's share of the layer: its partial, an all-gather
-                   of every rank's partial over a torch.distributed process
-                   group (NCCL between GPUs), the combine; every rank ends with
-                   the same y
+  ep_forward       one rank's share of the layer: its partial, then one of
+                   two exchanges over a torch.distributed process group (NCCL
+                   between GPUs), after which every rank holds the same y:
+                   "reduce_scatter" (default): rank j receives row slice j of
+                     every rank's partial (one all-to-all), folds them in rank
+                     order with the shared expert of its rows only, and the
+                     folded slices are all-gathered: 2 (R - 1) / R of a
+                     partial's bytes in and out per rank (TensorFold #310,
+                     maintainer's reply: the exact reduce-scatter in rank
+                     order);
+                   "all_gather": every rank gathers every partial and folds
+                     all rows itself: (R - 1) partials in per rank
 
 Argument marshalling only: every step runs in the library's kernels.
 """
@@ -109,26 +117,60 @@ class _Ops:
     shared = staticmethod(shared_expert)
 
 
-def ep_forward(x, ids, weights, band_experts, shared, plan, rank, group=None, ops=_Ops):
+def row_slices(T, ranks):
+    """Row offsets [ranks + 1] of the row slices of the reduce-scatter: whole
+    rows, as even as they go, the first T % ranks slices one row longer (the
+    share rule of ep_plan, applied to rows; a slice may be empty)."""
+    base, extra = divmod(int(T), int(ranks))
+    out = [0]
+    for j in range(ranks):
+        out.append(out[-1] + base + (1 if j < extra else 0))
+    return out
+
+
+def ep_forward(x, ids, weights, band_experts, shared, plan, rank, group=None, ops=_Ops,
+               exchange="reduce_scatter"):
     """One rank's share of the expert-parallel layer.
 
     band_experts = (w_gate, w_up, w_down) of this rank's band; shared =
     (ws_gate, ws_up, ws_down) replicated on every rank, or None.  The partials
-    of all ranks are gathered in rank order over `group` (torch.distributed),
-    so every rank returns the same y.
+    are exchanged over `group` (torch.distributed) and folded in rank order,
+    so every rank returns the same y [T, H], bit for bit the same whichever
+    exchange runs (each row's fold is the same additions in the same order).
     """
     import torch.distributed as dist
     w_gate, w_up, w_down = band_experts
-    part = ops.partial(x, ids, weights, w_gate, w_up, w_down, plan, rank)
+    part = ops.partial(x, ids, weights, w_gate, w_up, w_down, plan, rank).contiguous()
     world = dist.get_world_size(group)
     if world != plan.bands:
         raise ValueError(f"{world} ranks for a plan of {plan.bands} bands")
-    slots = [torch.empty_like(part) for _ in range(world)]
-    dist.all_gather(slots, part.contiguous(), group=group)
-    gathered = torch.stack(slots)  # rank r's partial at r
-    s = None if shared is None else ops.shared(x, *shared)
-    return ops.combine(gathered, ids, plan, s)
+    T, H = part.shape
+    if exchange == "all_gather":
+        slots = [torch.empty_like(part) for _ in range(world)]
+        dist.all_gather(slots, part, group=group)
+        gathered = torch.stack(slots)  # rank r's partial at r
+        s = None if shared is None else ops.shared(x, *shared)
+        return ops.combine(gathered, ids, plan, s)
+    if exchange != "reduce_scatter":
+        raise ValueError(f"unknown exchange {exchange!r}")
+    # row slice j of every rank's partial to rank j, in rank order
+    rs = row_slices(T, world)
+    sizes = [rs[j + 1] - rs[j] for j in range(world)]
+    lo, hi = rs[rank], rs[rank + 1]
+    mine = torch.empty((world * sizes[rank], H), dtype=part.dtype, device=part.device)
+    dist.all_to_all_single(mine, part, output_split_sizes=[sizes[rank]] * world,
+                           input_split_sizes=sizes, group=group)
+    s = None if shared is None else ops.shared(x[lo:hi], *shared)
+    y_mine = ops.combine(mine.view(world, sizes[rank], H), ids[lo:hi].contiguous(), plan, s)
+    # the folded slices to every rank (padded to the longest slice)
+    pad = max(sizes)
+    send = torch.zeros((pad, H), dtype=part.dtype, device=part.device)
+    send[:sizes[rank]] = y_mine
+    every = torch.empty((world * pad, H), dtype=part.dtype, device=part.device)
+    dist.all_gather_into_tensor(every, send, group=group)
+    every = every.view(world, pad, H)
+    return torch.cat([every[j, :sizes[j]] for j in range(world)], dim=0)
 
 
 __all__ = ["EP_ID_NONE", "moe_ffn_partial_workspace_size", "moe_ffn_partial", "moe_ep_combine",
-           "shared_expert", "ep_forward", "EPError", "EP_OK"]
+           "shared_expert", "ep_forward", "row_slices", "EPError", "EP_OK"]
