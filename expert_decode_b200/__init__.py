@@ -7,10 +7,10 @@ nothing here falls back to the CPU.
 """
 from .api import (  # noqa: F401
     EP_OK, EP_EINVAL, EP_EDIM, EP_EBADID, EP_ENOMEM, EP_ECUDA, EP_ETIMEOUT,
-    EPError, Plan, WorkspaceLayout, ep_plan, moe_route, moe_route_sigmoid,
+    EPError, Plan, WorkspaceLayout, ep_plan, moe_route, moe_route_logits, moe_route_sigmoid,
     moe_ffn_workspace_size, moe_ffn_workspace_layout,
     moe_ffn_forward,
     moe_ffn_forward_noalloc,
-    ep_check_status, ep_set_dispatch, ep_last_launch_count, ep_profile_events, library,
+    ep_check_status, ep_set_dispatch, ep_set_router, ep_last_launch_count, ep_profile_events, library,
     library_path,
 )

@@ -15,7 +15,8 @@ import torch
 EP_OK, EP_EINVAL, EP_EDIM, EP_EBADID, EP_ENOMEM, EP_ECUDA, EP_ETIMEOUT = range(7)
 EP_BF16, EP_F32 = 0, 1
 EP_MAX_BANDS = 64
-_DISPATCH = {"auto": 0, "streaming": 1, "tensor": 2, "streaming_tc": 3, "streaming_simt": 4}
+_DISPATCH = {"auto": 0, "streaming": 1, "tensor": 2, "streaming_tc": 3, "streaming_simt": 4,
+             "tensor_m128": 5, "tensor_m256": 6}
 _NAMES = {0: "EP_OK", 1: "EP_EINVAL", 2: "EP_EDIM", 3: "EP_EBADID", 4: "EP_ENOMEM",
           5: "EP_ECUDA", 6: "EP_ETIMEOUT"}
 
@@ -31,7 +32,8 @@ class EPError(RuntimeError):
 
 class WorkspaceLayout(ctypes.Structure):
     _fields_ = [("bytes", ctypes.c_size_t), ("contrib_offset", ctypes.c_size_t),
-                ("shared_offset", ctypes.c_size_t)]
+                ("shared_offset", ctypes.c_size_t), ("group_offset_offset", ctypes.c_size_t),
+                ("perm_offset", ctypes.c_size_t)]
 
 
 class Plan(ctypes.Structure):
@@ -57,6 +59,7 @@ def library():
             P, I64, I32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
             lib.ep_plan.argtypes = [I32, I32, ctypes.POINTER(Plan)]
             lib.moe_route.argtypes = [P, ctypes.c_int, I64, I64, P, P, I64, I32, P, P, P]
+            lib.moe_route_logits.argtypes = [P, ctypes.c_int, I64, I64, P, P, I64, P, P, P]
             lib.moe_route_sigmoid.argtypes = [P, ctypes.c_int, I64, I64, P, P, I64, I32, I32,
                                               ctypes.c_float, P, P, P]
             lib.moe_ffn_workspace_size.argtypes = [I64, I64, I64, I32, I64, I64]
@@ -69,15 +72,17 @@ def library():
                                                     P, I64, I64, P, P, P, I64,
                                                     ctypes.POINTER(Plan), P, P]
             lib.ep_set_dispatch.argtypes = [ctypes.c_int]
+            lib.ep_set_router.argtypes = [ctypes.c_int]
             lib.ep_check_status.argtypes = [P]
             lib.ep_last_error.restype = ctypes.c_char_p
             lib.ep_last_launch_count.restype = I32
             lib.ep_profile_events.argtypes = [P, I32]
             lib.ep_profile_events.restype = ctypes.c_int
-            for fn in ("ep_plan", "moe_route", "moe_route_sigmoid", "moe_ffn_forward",
+            for fn in ("ep_plan", "moe_route", "moe_route_logits", "moe_route_sigmoid",
+                       "moe_ffn_forward",
                        "moe_ffn_workspace_layout",
                        "moe_ffn_forward_noalloc",
-                       "ep_set_dispatch", "ep_check_status"):
+                       "ep_set_dispatch", "ep_set_router", "ep_check_status"):
                 getattr(lib, fn).restype = ctypes.c_int
             _lib = lib
         return _lib
@@ -139,6 +144,21 @@ def moe_route(x, w_router, bias, top_k, ids=None, weights=None, stream=None):
     _check(library().moe_route(_ptr(x), _dtype(x), T, H, _ptr(w_router), _ptr(bias), E,
                                int(top_k), _ptr(ids), _ptr(weights), _stream(stream)))
     return ids, weights
+
+
+def moe_route_logits(x, w_router, bias, stream=None):
+    """(logits, bounds) [T, E] fp32: the router's fp32 logits above 32 tokens
+    and the bound of each one's error (inspection)."""
+    _dense(x, "x", ndim=2)
+    _dense(w_router, "w_router", torch.bfloat16, 2)
+    _dense(bias, "bias", torch.float32, 1)
+    T, H = x.shape
+    E = w_router.shape[0]
+    logits = torch.empty((T, E), dtype=torch.float32, device=x.device)
+    bounds = torch.empty((T, E), dtype=torch.float32, device=x.device)
+    _check(library().moe_route_logits(_ptr(x), _dtype(x), T, H, _ptr(w_router), _ptr(bias), E,
+                                      _ptr(logits), _ptr(bounds), _stream(stream)))
+    return logits, bounds
 
 
 def moe_route_sigmoid(x, w_router, bias, top_k, normalize=False, scale=1.0, ids=None,
@@ -246,6 +266,15 @@ def ep_set_dispatch(mode):
     fold) or "streaming_simt" (gate/up, then down with the fold, on the CUDA
     cores)."""
     _check(library().ep_set_dispatch(_DISPATCH[mode]))
+
+
+_ROUTER = {"auto": 0, "tiled": 1, "tensor": 2}
+
+
+def ep_set_router(mode):
+    """Process-wide router choice above 32 tokens: "auto", "tiled" (CUDA-core
+    fp32 logits) or "tensor" (tcgen05 logits)."""
+    _check(library().ep_set_router(_ROUTER[mode]))
 
 
 def ep_last_launch_count():

@@ -177,9 +177,36 @@ __device__ __forceinline__ void bulk_g2s(void *smem_dst, const void *gsrc, uint3
         : "memory");
 }
 
+// Bulk prefetch of global memory into L2 (no shared memory, no completion
+// to wait for).  Address and size multiples of 16 bytes.
+__device__ __forceinline__ void prefetch_l2_bulk(const void *gsrc, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gsrc), "r"(bytes)
+                 : "memory");
+}
+
+// This CTA's share (1/gridDim.x, in 16-byte units) of `bytes` bytes at p,
+// prefetched into L2 in pieces of at most 64 KB.
+__device__ __forceinline__ void prefetch_l2_share(const void *p, size_t bytes) {
+    if (p == nullptr || bytes == 0)
+        return;
+    const size_t units = bytes / 16, per = (units + gridDim.x - 1) / gridDim.x;
+    size_t u0 = per * blockIdx.x, u1 = u0 + per < units ? u0 + per : units;
+    const uint8_t *b = static_cast<const uint8_t *>(p);
+    for (; u0 < u1; u0 += 4096) {
+        const size_t n = (u1 - u0 < 4096 ? u1 - u0 : 4096);
+        prefetch_l2_bulk(b + u0 * 16, (uint32_t)(n * 16));
+    }
+}
+
 __device__ __forceinline__ uint64_t policy_evict_first() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ uint64_t policy_evict_normal() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
     return p;
 }
 

@@ -27,7 +27,8 @@
 //              units), which write h = silu(g) * u: as bf16 hi/lo rows for
 //              stream_down_tc_kernel, or in fp32 for stream_down_fold_kernel.
 // Tiles go round-robin over the CTAs: the shared expert's first, then each
-// routed group's in ascending expert id.
+// routed group's in ascending expert id.  While it waits for the router,
+// each CTA prefetches a share of the shared expert's three matrices into L2.
 //
 // stream_down_tc_kernel (below): the down projection with the same machinery.
 #pragma once
@@ -59,6 +60,10 @@ struct TcArgs {
     int T, H, E, I, I_s, top_k;
     const int32_t *ids;
     const float *weights;
+    // the shared expert's weights (no routing decides them), prefetched into
+    // L2 while the kernel waits for the router: Ws_gate, Ws_up, Ws_down
+    const void *pf[3];
+    size_t pf_bytes[3];
     float *h_routed;  // [pairs, I] in plan order
     float *h_shared;  // [T, I_s]
     // When set, h goes out instead as bf16 hi/lo pairs for the tensor-core
@@ -144,6 +149,8 @@ stream_gate_up_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
         prefetch_tensormap(&maps.wg);
         prefetch_tensormap(&maps.wu);
         prefetch_tensormap(&maps.x);
+        for (int i = 0; i < 3; ++i)
+            prefetch_l2_share(a.pf[i], a.pf_bytes[i]);
     }
     if (warp == 1) {
         tmem_alloc(tmem_holder, kTcTmemCols);

@@ -20,6 +20,7 @@
 #include "grouped.cuh"
 #include "decode_tc.cuh"
 #include "ep.cuh"
+#include "router_tc.cuh"
 
 namespace {
 
@@ -42,6 +43,7 @@ struct KernelBracket {
     }
 };
 std::atomic<int> g_dispatch{EP_DISPATCH_AUTO};
+std::atomic<int> g_router{EP_ROUTER_AUTO};
 
 ep_status fail(ep_status s, const char *fmt, ...) {
     va_list ap;
@@ -159,6 +161,10 @@ ep_status device_info(const DeviceInfo **out) {
         EPK_RD_ATTR(false, 1, true); EPK_RD_ATTR(false, 2, true);
         EPK_RD_ATTR(true, 1, true); EPK_RD_ATTR(true, 2, true);
 #undef EPK_RD_ATTR
+        EP_CUDA_CHECK(cudaFuncSetAttribute(epk::router_tc_kernel<false>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, m));
+        EP_CUDA_CHECK(cudaFuncSetAttribute(epk::router_tc_kernel<true>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, m));
         EP_CUDA_CHECK(cudaFuncSetAttribute(epk::stream_gate_up_kernel<false, false>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, m));
         EP_CUDA_CHECK(cudaFuncSetAttribute(epk::stream_gate_up_kernel<false, true>,
@@ -188,6 +194,10 @@ constexpr int64_t kMaxI = 16384;
 constexpr int kMaxTopK = 16;
 // the decode path's gate/up runs on the tensor cores from this many tokens
 constexpr int64_t kTcMinT = 2;
+
+
+// GEMM tile height of the tensor path by default: 1 = 128 weight rows, 2 = 256
+constexpr int kGemmMhAuto = 1;
 // moe_route computes every logit by Dot2 up to this many tokens
 constexpr int64_t kRouterDot2MaxT = 32;
 // Shared memory the streaming kernels may take, leaving the rest of the
@@ -309,9 +319,16 @@ extern "C" ep_status ep_plan(int32_t num_experts, int32_t bands, ep_plan_t *out)
 }
 
 extern "C" ep_status ep_set_dispatch(ep_dispatch mode) {
-    if ((int)mode < (int)EP_DISPATCH_AUTO || (int)mode > (int)EP_DISPATCH_STREAMING_SIMT)
+    if ((int)mode < (int)EP_DISPATCH_AUTO || (int)mode > (int)EP_DISPATCH_TENSOR_M256)
         return fail(EP_EINVAL, "ep_set_dispatch: unknown mode %d", (int)mode);
     g_dispatch.store((int)mode);
+    return ok();
+}
+
+extern "C" ep_status ep_set_router(ep_router_mode mode) {
+    if ((int)mode < (int)EP_ROUTER_AUTO || (int)mode > (int)EP_ROUTER_TENSOR)
+        return fail(EP_EINVAL, "ep_set_router: unknown mode %d", (int)mode);
+    g_router.store((int)mode);
     return ok();
 }
 
@@ -382,12 +399,24 @@ int max_active_clusters(const void *fn, int csize, uint32_t smem) {
     return n;
 }
 
+// The tensor-core router takes batches of more than 32 tokens with bf16
+// activations, at most 256 experts and at least two 64-wide blocks of H (so
+// that every CTA of its cluster has a slice); the tiled fp32 router the rest.
+bool tc_router_fits(const DeviceInfo &d, ep_dtype x_dtype, int64_t H, int64_t E) {
+    if (x_dtype != EP_BF16 || E > epk::kRcMaxE || H < 2 * epk::kGemmBK)
+        return false;
+    const int MT = (int)((E + epk::kGemmBM - 1) / epk::kGemmBM);
+    return epk::rc_smem_layout(MT, (int)E, epk::kRcMinCK).alloc <= (uint32_t)d.smem_optin &&
+           epk::tensor_map_encoder() != nullptr;
+}
+
 // Both routers: sig selects the sigmoid variant (normalize, scale used only
 // there); `who` names the entry point in error messages.
 ep_status route_impl(const char *who, bool sig, const void *x, ep_dtype x_dtype, int64_t T,
                      int64_t H, const void *w_router, const float *bias, int64_t E,
                      int32_t top_k, int32_t normalize, float scale, int32_t *ids,
-                     float *weights, void *stream) {
+                     float *weights, void *stream, float *dump_logit = nullptr,
+                     float *dump_bound = nullptr) {
     if (x_dtype != EP_BF16 && x_dtype != EP_F32)
         return fail(EP_EINVAL, "%s: unknown x dtype %d", who, (int)x_dtype);
     if (T < 0 || T > kMaxT)
@@ -405,19 +434,27 @@ ep_status route_impl(const char *who, bool sig, const void *x, ep_dtype x_dtype,
         t_launches = 0;
         return ok();
     }
-    if (x == nullptr || w_router == nullptr || ids == nullptr || weights == nullptr)
+    const bool dump = dump_logit != nullptr;
+    if (x == nullptr || w_router == nullptr || (!dump && (ids == nullptr || weights == nullptr)) ||
+        (dump && dump_bound == nullptr))
         return fail(EP_EINVAL, "%s: NULL x, w_router, ids or weights", who);
     if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(ids, 4) || !aligned(weights, 4) ||
-        (bias != nullptr && !aligned(bias, 4)))
+        (bias != nullptr && !aligned(bias, 4)) || !aligned(dump_logit, 4) ||
+        !aligned(dump_bound, 4))
         return fail(EP_EINVAL, "%s: misaligned pointer (x, w_router need 16 bytes)", who);
     const DeviceInfo *d = nullptr;
     ep_status s = device_info(&d);
     if (s != EP_OK)
         return s;
+    const int router_mode = g_router.load();
+    if (router_mode == EP_ROUTER_TENSOR && T > kRouterDot2MaxT &&
+        !tc_router_fits(*d, x_dtype, H, E))
+        return fail(EP_EINVAL, "%s: the tensor-core router takes bf16 x, E <= %d and H >= %d",
+                    who, epk::kRcMaxE, 2 * epk::kGemmBK);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const uint16_t *wr = static_cast<const uint16_t *>(w_router);
     KernelBracket kb0(st, 0);
-    if (T <= kRouterDot2MaxT) {
+    if (T <= kRouterDot2MaxT && !dump) {
         // small batches: every logit by Dot2, one cluster per token while
         // the clusters fit on the SMs at once, else two tokens per cluster
         const int64_t max_clusters = std::max(1, d->sm_count / epk::kRouterCluster);
@@ -442,6 +479,31 @@ ep_status route_impl(const char *who, bool sig, const void *x, ep_dtype x_dtype,
         }
 #undef EPK_RD
         EP_CUDA_CHECK(e);
+    } else if (router_mode != EP_ROUTER_TILED && tc_router_fits(*d, x_dtype, H, E)) {
+        // larger batches of bf16 activations: logits on the tensor cores, a
+        // cluster of CK CTAs per 64 tokens, Dot2 for the candidates
+        const int MT = (int)((E + epk::kGemmBM - 1) / epk::kGemmBM);
+        const int64_t tiles = (T + epk::kRcNT - 1) / epk::kRcNT;
+        const int nkb = (int)((H + epk::kGemmBK - 1) / epk::kGemmBK);
+        int CK = (int)std::max<int64_t>(epk::kRcMinCK,
+                                        std::min<int64_t>(epk::kRcMaxCK, d->sm_count / tiles));
+        CK = std::min(CK, nkb);
+        const epk::RcSmem L = epk::rc_smem_layout(MT, (int)E, CK);
+        epk::RcMaps maps;
+        memset(&maps, 0, sizeof maps);
+        if (!epk::map_2d(&maps.w, w_router, (uint64_t)H, (uint64_t)E, epk::kGemmBM) ||
+            !epk::map_2d(&maps.x, x, (uint64_t)H, (uint64_t)T, epk::kRcNT))
+            return fail(EP_ECUDA, "%s: encoding the router's tensor maps failed", who);
+        const dim3 grid((unsigned)CK, (unsigned)tiles);
+        const uint16_t *xb = static_cast<const uint16_t *>(x);
+        const cudaError_t e =
+            sig ? launch_cluster(epk::router_tc_kernel<true>, grid, epk::kRcThreads, L.alloc, st,
+                                 (unsigned)CK, maps, xb, T, (int)H, wr, bias, (int)E, top_k, ids,
+                                 weights, CK, normalize, scale, dump_logit, dump_bound)
+                : launch_cluster(epk::router_tc_kernel<false>, grid, epk::kRcThreads, L.alloc, st,
+                                 (unsigned)CK, maps, xb, T, (int)H, wr, bias, (int)E, top_k, ids,
+                                 weights, CK, normalize, scale, dump_logit, dump_bound);
+        EP_CUDA_CHECK(e);
     } else {
         // larger batches: register-tiled fp32 logits, Dot2 for the candidates
         const int BT = epk::rt_block_tokens((int)E);
@@ -451,7 +513,7 @@ ep_status route_impl(const char *who, bool sig, const void *x, ep_dtype x_dtype,
                         (long long)E, L.total);
         // the kernel for this activation type, block size and router
         using TiledFn = void (*)(const void *, int64_t, int, const uint16_t *, const float *, int,
-                                 int, int32_t *, float *, int, int, int, float);
+                                 int, int32_t *, float *, int, int, int, float, float *, float *);
         TiledFn fn;
         {
             const bool f = x_dtype == EP_F32;
@@ -489,7 +551,8 @@ ep_status route_impl(const char *who, bool sig, const void *x, ep_dtype x_dtype,
         const dim3 grid((unsigned)(CE * CK), (unsigned)blocks);
         const cudaError_t e = launch_cluster(fn, grid, epk::kRtThreads, L.total, st,
                                              (unsigned)(CE * CK), x, T, (int)H, wr, bias, (int)E,
-                                             top_k, ids, weights, CE, CK, normalize, scale);
+                                             top_k, ids, weights, CE, CK, normalize, scale,
+                                             dump_logit, dump_bound);
         EP_CUDA_CHECK(e);
     }
     t_launches = 1;
@@ -503,6 +566,16 @@ extern "C" ep_status moe_route(const void *x, ep_dtype x_dtype, int64_t T, int64
                                int32_t top_k, int32_t *ids, float *weights, void *stream) {
     return route_impl("moe_route", false, x, x_dtype, T, H, w_router, bias, E, top_k, 0, 1.0f,
                       ids, weights, stream);
+}
+
+extern "C" ep_status moe_route_logits(const void *x, ep_dtype x_dtype, int64_t T, int64_t H,
+                                      const void *w_router, const float *bias, int64_t E,
+                                      float *logits, float *bounds, void *stream) {
+    if (logits == nullptr || bounds == nullptr)
+        return fail(EP_EINVAL, "moe_route_logits: NULL logits or bounds");
+    return route_impl("moe_route_logits", false, x, x_dtype, T, H, w_router, bias, E,
+                      (int32_t)std::min<int64_t>(E, 1), 0, 1.0f, nullptr, nullptr, stream,
+                      logits, bounds);
 }
 
 extern "C" ep_status moe_route_sigmoid(const void *x, ep_dtype x_dtype, int64_t T, int64_t H,
@@ -540,6 +613,8 @@ extern "C" ep_status moe_ffn_workspace_layout(int64_t T, int64_t H, int64_t E, i
         l.bytes = W.total;
         l.contrib_offset = W.grouped.c;
         l.shared_offset = W.grouped.s;
+        l.group_offset_offset = W.grouped.group_offset;
+        l.perm_offset = W.grouped.perm_pair;
     }
     *out = l;
     return ok();
@@ -624,7 +699,8 @@ ep_status ffn_forward_impl(bool band_call, const void *x, ep_dtype x_dtype, int6
         if (!sp.fits)
             return fail(EP_EINVAL, "moe_ffn_forward: the streaming path does not fit these sizes");
         use_streaming = true;
-    } else if (mode == EP_DISPATCH_TENSOR) {
+    } else if (mode == EP_DISPATCH_TENSOR || mode == EP_DISPATCH_TENSOR_M128 ||
+               mode == EP_DISPATCH_TENSOR_M256) {
         use_streaming = false;
     } else {
         use_streaming = sp.fits;
@@ -679,6 +755,12 @@ ep_status ffn_forward_impl(bool band_call, const void *x, ep_dtype x_dtype, int6
             ta.h_shared = ga.h_shared;
             ta.hb_routed = reinterpret_cast<uint16_t *>(ws + W.hb_routed);
             ta.hb_shared = I_s > 0 ? reinterpret_cast<uint16_t *>(ws + W.hb_shared) : nullptr;
+            ta.pf[0] = ws_gate;
+            ta.pf[1] = ws_up;
+            ta.pf[2] = ws_down;
+            for (int i = 0; i < 3; ++i)
+                ta.pf_bytes[i] = I_s > 0 ? (size_t)I_s * H * 2 : 0;
+
             // the down projection on the tensor cores too: W_down rows against
             // the bf16 hi/lo slices of h, then the fold in combine_kernel
             epk::DtMaps dm;
@@ -765,6 +847,8 @@ ep_status ffn_forward_impl(bool band_call, const void *x, ep_dtype x_dtype, int6
     g.y = y;
     g.sm_count = d->sm_count;
     g.smem_optin = d->smem_optin;
+    g.pdl = pdl_enabled();
+    g.mh = mode == EP_DISPATCH_TENSOR_M256 ? 2 : (mode == EP_DISPATCH_TENSOR_M128 ? 1 : kGemmMhAuto);
     int launches = 0;
     char why[256] = "";
     s = epk::grouped_forward(g, W.grouped, ws, st, &launches, why, sizeof why,

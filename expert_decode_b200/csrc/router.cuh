@@ -172,13 +172,11 @@ __device__ void topk_select_warp(const double *v, int E, int top_k, int &pick_e,
     }
 }
 
-// Softmax router: the picks by logit, weights = softmax over the picked set.
-__device__ void topk_softmax_warp(const double *lt, int E, int top_k, int32_t *ids_row,
-                                  float *w_row) {
+// Softmax weights of a token's picks (lane r < top_k holds the r-th pick's
+// id and logit): softmax over the picked set, summed in pick order.
+__device__ void softmax_finish_warp(int pick_e, double pick_v, int top_k, int32_t *ids_row,
+                                    float *w_row) {
     const int lane = (int)lane_id();
-    int pick_e;
-    double pick_v;
-    topk_select_warp(lt, E, top_k, pick_e, pick_v);
     const double top = __shfl_sync(0xffffffffu, pick_v, 0);
     const double ev = lane < top_k ? exp(pick_v - top) : 0.0;
     double sum = 0.0;
@@ -190,16 +188,22 @@ __device__ void topk_softmax_warp(const double *lt, int E, int top_k, int32_t *i
     }
 }
 
+// Softmax router: the picks by logit, weights = softmax over the picked set.
+__device__ void topk_softmax_warp(const double *lt, int E, int top_k, int32_t *ids_row,
+                                  float *w_row) {
+    int pick_e;
+    double pick_v;
+    topk_select_warp(lt, E, top_k, pick_e, pick_v);
+    softmax_finish_warp(pick_e, pick_v, top_k, ids_row, w_row);
+}
+
 // Sigmoid router (the GLM variant: sigmoid scores, a bias used in the selection only, weights from the unbiased scores;
 // TensorFold #593, "What exists now", glm_route.cu): the picks by key =
 // score + bias, weights = scale * score, or scale * score / (sum of the
 // picked scores) with normalize.
-__device__ void topk_sigmoid_warp(const double *key, const double *score, int E, int top_k,
-                                  int normalize, float scale, int32_t *ids_row, float *w_row) {
+__device__ void sigmoid_finish_warp(const double *score, int pick_e, int top_k, int normalize,
+                                    float scale, int32_t *ids_row, float *w_row) {
     const int lane = (int)lane_id();
-    int pick_e;
-    double pick_v;
-    topk_select_warp(key, E, top_k, pick_e, pick_v);
     const double sc = lane < top_k ? score[pick_e] : 0.0;
     double sum = 0.0;
     for (int j = 0; j < top_k; ++j)
@@ -208,6 +212,14 @@ __device__ void topk_sigmoid_warp(const double *key, const double *score, int E,
         ids_row[lane] = pick_e;
         w_row[lane] = (float)((double)scale * (normalize ? sc / sum : sc));
     }
+}
+
+__device__ void topk_sigmoid_warp(const double *key, const double *score, int E, int top_k,
+                                  int normalize, float scale, int32_t *ids_row, float *w_row) {
+    int pick_e;
+    double pick_v;
+    topk_select_warp(key, E, top_k, pick_e, pick_v);
+    sigmoid_finish_warp(score, pick_e, top_k, normalize, scale, ids_row, w_row);
 }
 
 __device__ __forceinline__ double sigmoid_f64(double l) { return 1.0 / (1.0 + exp(-l)); }
@@ -225,8 +237,13 @@ constexpr int kRdWarps = kRdThreads / 32;
 constexpr int kRdMaxTB = 2;
 
 struct RdSmem {
-    uint32_t x, vals, logit, total;
+    uint32_t x, vals, logit, keys, sel, total;
 };
+
+// Up to this many experts the small-batch router picks by a parallel rank
+// count (every (token, expert) key counts the keys above it); above, one
+// warp per token selects the top_k in top_k rounds.
+constexpr int kRdRankMaxE = 256;
 
 __host__ __device__ inline RdSmem rd_smem_layout(int tb_max, int H, int E) {
     RdSmem s;
@@ -237,6 +254,8 @@ __host__ __device__ inline RdSmem rd_smem_layout(int tb_max, int H, int E) {
     // score (sigmoid)
     s.vals = o;  o = align_up_u32(o + 2u * tb_max * per_cta * 8, 16);
     s.logit = o; o = align_up_u32(o + 2u * tb_max * E * 8, 16);
+    s.keys = o;  o = align_up_u32(o + (uint32_t)tb_max * E * 8, 16);
+    s.sel = o;   o = align_up_u32(o + (uint32_t)tb_max * 16 * 4, 16);
     s.total = o;
     return s;
 }
@@ -365,7 +384,43 @@ router_dot2_kernel(const void *__restrict__ x, int64_t T, int H,
         }
     }
     cluster_sync();  // all logits are in CTA 0
-    if (rank != 0 || warp >= tb)
+    if (rank != 0)
+        return;
+    if (E <= kRdRankMaxE) {
+        // the pick by rank: key (value, id) ranks r among the token's keys when
+        // r keys are above it; ranks below top_k are the picks, in order
+        unsigned long long *keys = reinterpret_cast<unsigned long long *>(smem + L.keys);
+        int *sel = reinterpret_cast<int *>(smem + L.sel);
+        for (int i = threadIdx.x; i < tb * E; i += kRdThreads) {
+            const int t = i / E, e = i - t * E;
+            keys[i] = topk_key(logit[t * E + e], e);
+        }
+        __syncthreads();
+        for (int i = threadIdx.x; i < tb * E; i += kRdThreads) {
+            const int t = i / E;
+            const unsigned long long k = keys[i];
+            const unsigned long long *kt = keys + t * E;
+            int r = 0;
+            for (int f = 0; f < E; ++f)
+                r += kt[f] > k ? 1 : 0;
+            if (r < top_k)
+                sel[t * 16 + r] = i - t * E;
+        }
+        __syncthreads();
+        if (warp >= tb)
+            return;
+        const int pick_e = lane < top_k ? sel[warp * 16 + lane] : 0;
+        if constexpr (SIG) {
+            sigmoid_finish_warp(logit + (TB + warp) * E, pick_e, top_k, normalize, scale,
+                                ids + (t0 + warp) * top_k, weights + (t0 + warp) * top_k);
+        } else {
+            const double pick_v = lane < top_k ? logit[warp * E + pick_e] : 0.0;
+            softmax_finish_warp(pick_e, pick_v, top_k, ids + (t0 + warp) * top_k,
+                                weights + (t0 + warp) * top_k);
+        }
+        return;
+    }
+    if (warp >= tb)
         return;
     if constexpr (SIG)
         topk_sigmoid_warp(logit + warp * E, logit + (TB + warp) * E, E, top_k, normalize, scale,
@@ -466,12 +521,258 @@ __device__ double logit_dot2_global(const void *xrow, const uint16_t *__restrict
     return acc;
 }
 
+// Dot2 logits of up to NC experts for one token (one warp): the token's
+// activation chunks are loaded once per round and the experts' weight chunks
+// beside them, so that NC rows are in flight at once instead of one.  Lane
+// results are combined as in logit_dot2_global; out[i] (all lanes) includes
+// the bias when bias is not NULL.
+template <bool XF32, int NC>
+__device__ void logit_dot2_multi(const void *xrow, const uint16_t *__restrict__ w_router,
+                                 const float *__restrict__ bias, int H, const int *es, int n,
+                                 double (&out)[NC]) {
+    constexpr int U = 8;
+    const int lane = (int)lane_id();
+    const int nck = H >> 3;
+    float2 s[NC], c[NC];
+#pragma unroll
+    for (int i = 0; i < NC; ++i) {
+        s[i] = make_float2(0.f, 0.f);
+        c[i] = make_float2(0.f, 0.f);
+    }
+    const uint4 *wrow[NC];
+#pragma unroll
+    for (int i = 0; i < NC; ++i)
+        wrow[i] = reinterpret_cast<const uint4 *>(w_router + (size_t)es[i < n ? i : 0] * H);
+    for (int base = 0; base < nck; base += 32 * U) {
+        uint4 wv[NC][U], xv[U][XF32 ? 2 : 1];
+#pragma unroll
+        for (int q = 0; q < U; ++q) {
+            const int ch = base + lane + 32 * q;
+            const bool ok = ch < nck;
+#pragma unroll
+            for (int h = 0; h < (XF32 ? 2 : 1); ++h)
+                xv[q][h] = ok ? reinterpret_cast<const uint4 *>(xrow)[(XF32 ? 2 : 1) * ch + h]
+                              : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int i = 0; i < NC; ++i)
+                wv[i][q] = (ok && i < n) ? wrow[i][ch] : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int q = 0; q < U; ++q) {
+            float2 xp[4];
+            if constexpr (XF32) {
+                xp[0] = make_float2(__uint_as_float(xv[q][0].x), __uint_as_float(xv[q][0].y));
+                xp[1] = make_float2(__uint_as_float(xv[q][0].z), __uint_as_float(xv[q][0].w));
+                xp[2] = make_float2(__uint_as_float(xv[q][1].x), __uint_as_float(xv[q][1].y));
+                xp[3] = make_float2(__uint_as_float(xv[q][1].z), __uint_as_float(xv[q][1].w));
+            } else {
+                xp[0] = bf16x2_to_f2(xv[q][0].x); xp[1] = bf16x2_to_f2(xv[q][0].y);
+                xp[2] = bf16x2_to_f2(xv[q][0].z); xp[3] = bf16x2_to_f2(xv[q][0].w);
+            }
+#pragma unroll
+            for (int i = 0; i < NC; ++i) {
+                float2 wp[4], wn[4];
+                dot2_unpack_w(wv[i][q], wp, wn);
+                dot2_chunk<XF32>(wp, wn, xp, s[i], c[i]);  // zero chunks add exact zeros
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < NC; ++i) {
+        double acc = dot2_warp_total(s[i], c[i]);
+        if (bias != nullptr && i < n)
+            acc += (double)bias[es[i]];
+        out[i] = acc;
+    }
+}
+
+// The pick of the tokens a CTA owns, shared by the routers that first form
+// fp32 logits with an error bound (router_tiled_kernel, router_tc_kernel).
+// Owned token j (0 <= j < n_local) is token t0 + tbase + tstride j of the
+// batch; logit [n_local][E] (the selection key for the sigmoid variant) is in
+// shared memory and bound_at(j, e) gives the bound of its error.  For every
+// owned token: its candidates (every expert whose exact value could reach the
+// k-th largest under the bounds), their Dot2 logits (one warp per candidate),
+// the pick on those values and the weights.  More than max_cand candidates
+// (a degenerate input) take a slower path over every expert that clears the
+// threshold, in ascending id.
+template <bool XF32, bool SIG, int NWARPS, typename BoundAt>
+__device__ void router_pick_owned(int n_local, int tbase, int tstride, int64_t t0, const void *x,
+                                  int H, const uint16_t *__restrict__ w_router,
+                                  const float *__restrict__ bias, int E, int top_k,
+                                  int32_t *__restrict__ ids, float *__restrict__ weights,
+                                  int normalize, float scale, const float *logit, int *ncand,
+                                  int *cand, double *cval, double *cscore, int max_cand,
+                                  BoundAt bound_at) {
+    constexpr int XB = XF32 ? 4 : 2;
+    const int warp = (int)(threadIdx.x >> 5), lane = (int)lane_id();
+    // candidates per owned token (one warp each): every expert whose exact
+    // logit could reach the k-th largest under the bounds
+    for (int j = warp; j < n_local; j += NWARPS) {
+        const float *lt = logit + j * E;
+        const float vk = kth_logit(lt, E, top_k);
+        float dmax = 0.f;
+        for (int e = lane; e < E; e += 32)
+            dmax = fmaxf(dmax, bound_at(j, e));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+            dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, off));
+        const double thr = (double)vk - 2.0 * (double)dmax * 1.0001;
+        int count = 0;
+        for (int i = 0; i < (E + 31) / 32; ++i) {
+            const int e = lane + 32 * i;
+            const bool c = e < E && (double)lt[e] >= thr;
+            const uint32_t m = __ballot_sync(0xffffffffu, c);
+            const int pos = count + __popc(m & ((1u << lane) - 1u));
+            if (c && pos < max_cand)
+                cand[j * max_cand + pos] = e;
+            count += __popc(m);
+        }
+        if (lane == 0)
+            ncand[j] = count;
+    }
+    __syncthreads();
+
+    // Dot2 logits of the owned tokens' candidates, spread over the warps in
+    // groups of up to NG candidates of one token (one warp refines a group
+    // at once: its rows stream side by side)
+    {
+        constexpr int NG = XF32 ? 2 : 4;
+        int mine = 0;
+        for (int j = 0; j < n_local; ++j) {
+            const int t = tbase + tstride * j;
+            const int nc = ncand[j] <= max_cand ? ncand[j] : 0;
+            const uint8_t *xrow = reinterpret_cast<const uint8_t *>(x) + (size_t)(t0 + t) * H * XB;
+            for (int c0 = 0; c0 < nc; c0 += NG) {
+                if ((mine++ % NWARPS) != warp)
+                    continue;
+                const int n = nc - c0 < NG ? nc - c0 : NG;
+                const int *es = cand + j * max_cand + c0;
+                double v[NG];
+                logit_dot2_multi<XF32, NG>(xrow, w_router, SIG ? nullptr : bias, H, es, n, v);
+                if (lane == 0) {
+                    for (int i = 0; i < n; ++i) {
+                        if (SIG) {
+                            const double sc = sigmoid_f64(v[i]);
+                            cval[j * max_cand + c0 + i] =
+                                sc + (bias != nullptr ? (double)bias[es[i]] : 0.0);
+                            cscore[j * max_cand + c0 + i] = sc;
+                        } else {
+                            cval[j * max_cand + c0 + i] = v[i];
+                        }
+                    }
+                }
+            }
+        }
+    }
+    __syncthreads();
+
+    // pick top_k on the refined values of each owned token, weigh, write
+    for (int j = warp; j < n_local; j += NWARPS) {
+        const int t = tbase + tstride * j;
+        const int nc = ncand[j];
+        double bv_list = 0.0, top = 0.0, bs_list = 0.0;  // lane r: the r-th pick's value, score
+        int be_list = 0;
+        if (nc <= max_cand) {
+            uint32_t chosen = 0;
+            for (int r = 0; r < top_k; ++r) {
+                double bv = -INFINITY;
+                int be = 0x7fffffff, bi = -1;
+                for (int i = 0; i < (max_cand + 31) / 32; ++i) {
+                    const int ci = lane + 32 * i;
+                    if (ci < nc && !((chosen >> i) & 1u)) {
+                        const double v = cval[j * max_cand + ci];
+                        const int e = cand[j * max_cand + ci];
+                        if (v > bv || (v == bv && e < be)) { bv = v; be = e; bi = ci; }
+                    }
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    const double ov = __shfl_xor_sync(0xffffffffu, bv, off);
+                    const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+                    const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+                    if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; bi = oi; }
+                }
+                if (bi >= 0 && (bi & 31) == lane)
+                    chosen |= 1u << (bi >> 5);
+                if (r == 0)
+                    top = bv;
+                if (lane == r) {
+                    bv_list = bv;
+                    be_list = be;
+                    if (SIG && bi >= 0)
+                        bs_list = cscore[j * max_cand + bi];
+                }
+            }
+        } else {
+            // degenerate input: every candidate in ascending id through a
+            // sorted top_k list kept in registers of lanes 0..top_k-1
+            const float *lt = logit + j * E;
+            float dmax = 0.f;
+            for (int e = lane; e < E; e += 32)
+                dmax = fmaxf(dmax, bound_at(j, e));
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1)
+                dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, off));
+            const double thr = (double)kth_logit(lt, E, top_k) - 2.0 * (double)dmax * 1.0001;
+            const uint8_t *xrow = reinterpret_cast<const uint8_t *>(x) + (size_t)(t0 + t) * H * XB;
+            double lv = -INFINITY;  // lane j holds the j-th best so far
+            double ls = 0.0;        // and its score (sigmoid)
+            int li = 0x7fffffff;
+            for (int e = 0; e < E; ++e) {
+                if ((double)lt[e] < thr)
+                    continue;
+                double v, sc = 0.0;
+                if (SIG) {
+                    sc = sigmoid_f64(logit_dot2_global<XF32>(xrow, w_router, nullptr, H, e));
+                    v = sc + (bias != nullptr ? (double)bias[e] : 0.0);
+                } else {
+                    v = logit_dot2_global<XF32>(xrow, w_router, bias, H, e);
+                }
+                // insert: lanes whose value ranks below v shift down by one
+                const bool below = !(lv > v || (lv == v && li < e));
+                const uint32_t m = __ballot_sync(0xffffffffu, below && lane < top_k);
+                const int pos = m ? __ffs(m) - 1 : top_k;
+                const double pv = __shfl_up_sync(0xffffffffu, lv, 1);
+                const double ps = __shfl_up_sync(0xffffffffu, ls, 1);
+                const int pi = __shfl_up_sync(0xffffffffu, li, 1);
+                if (lane < top_k && pos < top_k) {
+                    if (lane == pos) { lv = v; ls = sc; li = e; }
+                    else if (lane > pos) { lv = pv; ls = ps; li = pi; }
+                }
+            }
+            top = __shfl_sync(0xffffffffu, lv, 0);
+            bv_list = lv;
+            bs_list = ls;
+            be_list = li;
+        }
+        double wv;
+        if (SIG) {
+            double ssum = 0.0;
+            for (int jj = 0; jj < top_k; ++jj)
+                ssum += __shfl_sync(0xffffffffu, lane < top_k ? bs_list : 0.0, jj);
+            wv = (double)scale * (normalize ? bs_list / ssum : bs_list);
+        } else {
+            const double ev = lane < top_k ? exp(bv_list - top) : 0.0;
+            double ssum = 0.0;
+            for (int jj = 0; jj < top_k; ++jj)
+                ssum += __shfl_sync(0xffffffffu, ev, jj);
+            wv = ev / ssum;
+        }
+        if (lane < top_k) {
+            ids[(t0 + t) * top_k + lane] = be_list;
+            weights[(t0 + t) * top_k + lane] = (float)wv;
+        }
+    }
+}
+
 template <bool XF32, int TM, bool SIG>
 __global__ void __launch_bounds__(kRtThreads, 1)
 router_tiled_kernel(const void *__restrict__ x, int64_t T, int H,
                     const uint16_t *__restrict__ w_router, const float *__restrict__ bias, int E,
                     int top_k, int32_t *__restrict__ ids, float *__restrict__ weights, int CE,
-                    int CK, int normalize, float scale) {
+                    int CK, int normalize, float scale, float *__restrict__ dump_logit,
+                    float *__restrict__ dump_bound) {
     constexpr int BT = 8 * TM;             // tokens per cluster
     constexpr int XB = XF32 ? 4 : 2;
     constexpr int LD = kRtBK + kRtPad;     // padded row of a k-tile, in floats
@@ -706,159 +1007,20 @@ router_tiled_kernel(const void *__restrict__ x, int64_t T, int H,
     }
     cluster_sync();  // every token's logits and bounds are with its owner; no
                      // shared memory of another CTA is used after this point
-
-    // candidates per owned token (one warp each): every expert whose exact
-    // logit could reach the k-th largest under the bounds
-    for (int j = warp; j < n_local; j += kRtThreads / 32) {
-        const float *lt = logit + j * E;
-        const float *bt = bound + j * E;
-        const float vk = kth_logit(lt, E, top_k);
-        float dmax = 0.f;
-        for (int e = lane; e < E; e += 32)
-            dmax = fmaxf(dmax, bt[e]);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
-            dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, off));
-        const double thr = (double)vk - 2.0 * (double)dmax * 1.0001;
-        int count = 0;
-        for (int i = 0; i < (E + 31) / 32; ++i) {
-            const int e = lane + 32 * i;
-            const bool c = e < E && (double)lt[e] >= thr;
-            const uint32_t m = __ballot_sync(0xffffffffu, c);
-            const int pos = count + __popc(m & ((1u << lane) - 1u));
-            if (c && pos < kRouterMaxCand)
-                cand[j * kRouterMaxCand + pos] = e;
-            count += __popc(m);
+    if (dump_logit != nullptr) {
+        // inspection (moe_route_logits): the fp32 logits and their bounds
+        for (int idx = tid; idx < n_local * E; idx += kRtThreads) {
+            const int j = idx / E, e = idx - j * E;
+            const int64_t t = t0 + (int)rank + NC * j;
+            dump_logit[t * E + e] = logit[j * E + e];
+            dump_bound[t * E + e] = bound[j * E + e];
         }
-        if (lane == 0)
-            ncand[j] = count;
+        return;
     }
-    __syncthreads();
-
-    // Dot2 logits of the owned tokens' candidates, spread over the warps
-    {
-        int mine = 0;
-        for (int j = 0; j < n_local; ++j) {
-            const int t = (int)rank + NC * j;
-            const int nc = ncand[j] <= kRouterMaxCand ? ncand[j] : 0;
-            const uint8_t *xrow = reinterpret_cast<const uint8_t *>(x) + (size_t)(t0 + t) * H * XB;
-            for (int ci = 0; ci < nc; ++ci) {
-                if ((mine++ % (kRtThreads / 32)) != warp)
-                    continue;
-                const int e = cand[j * kRouterMaxCand + ci];
-                if (SIG) {
-                    const double sc = sigmoid_f64(logit_dot2_global<XF32>(xrow, w_router, nullptr, H, e));
-                    if (lane == 0) {
-                        cval[j * kRouterMaxCand + ci] = sc + (bias != nullptr ? (double)bias[e] : 0.0);
-                        cscore[j * kRouterMaxCand + ci] = sc;
-                    }
-                } else {
-                    const double v = logit_dot2_global<XF32>(xrow, w_router, bias, H, e);
-                    if (lane == 0)
-                        cval[j * kRouterMaxCand + ci] = v;
-                }
-            }
-        }
-    }
-    __syncthreads();
-
-    // pick top_k on the refined values of each owned token, weigh, write
-    for (int j = warp; j < n_local; j += kRtThreads / 32) {
-        const int t = (int)rank + NC * j;
-        const int nc = ncand[j];
-        double bv_list = 0.0, top = 0.0, bs_list = 0.0;  // lane r: the r-th pick's value, score
-        int be_list = 0;
-        if (nc <= kRouterMaxCand) {
-            uint32_t chosen = 0;
-            for (int r = 0; r < top_k; ++r) {
-                double bv = -INFINITY;
-                int be = 0x7fffffff, bi = -1;
-                for (int i = 0; i < 2; ++i) {
-                    const int ci = lane + 32 * i;
-                    if (ci < nc && !((chosen >> i) & 1u)) {
-                        const double v = cval[j * kRouterMaxCand + ci];
-                        const int e = cand[j * kRouterMaxCand + ci];
-                        if (v > bv || (v == bv && e < be)) { bv = v; be = e; bi = ci; }
-                    }
-                }
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) {
-                    const double ov = __shfl_xor_sync(0xffffffffu, bv, off);
-                    const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-                    const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-                    if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; bi = oi; }
-                }
-                if (bi >= 0 && (bi & 31) == lane)
-                    chosen |= 1u << (bi >> 5);
-                if (r == 0)
-                    top = bv;
-                if (lane == r) {
-                    bv_list = bv;
-                    be_list = be;
-                    if (SIG && bi >= 0)
-                        bs_list = cscore[j * kRouterMaxCand + bi];
-                }
-            }
-        } else {
-            // degenerate input: every candidate in ascending id through a
-            // sorted top_k list kept in registers of lanes 0..top_k-1
-            const float *lt = logit + j * E;
-            float dmax = 0.f;
-            for (int e = lane; e < E; e += 32)
-                dmax = fmaxf(dmax, bound[j * E + e]);
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1)
-                dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, off));
-            const double thr = (double)kth_logit(lt, E, top_k) - 2.0 * (double)dmax * 1.0001;
-            const uint8_t *xrow = reinterpret_cast<const uint8_t *>(x) + (size_t)(t0 + t) * H * XB;
-            double lv = -INFINITY;  // lane j holds the j-th best so far
-            double ls = 0.0;        // and its score (sigmoid)
-            int li = 0x7fffffff;
-            for (int e = 0; e < E; ++e) {
-                if ((double)lt[e] < thr)
-                    continue;
-                double v, sc = 0.0;
-                if (SIG) {
-                    sc = sigmoid_f64(logit_dot2_global<XF32>(xrow, w_router, nullptr, H, e));
-                    v = sc + (bias != nullptr ? (double)bias[e] : 0.0);
-                } else {
-                    v = logit_dot2_global<XF32>(xrow, w_router, bias, H, e);
-                }
-                // insert: lanes whose value ranks below v shift down by one
-                const bool below = !(lv > v || (lv == v && li < e));
-                const uint32_t m = __ballot_sync(0xffffffffu, below && lane < top_k);
-                const int pos = m ? __ffs(m) - 1 : top_k;
-                const double pv = __shfl_up_sync(0xffffffffu, lv, 1);
-                const double ps = __shfl_up_sync(0xffffffffu, ls, 1);
-                const int pi = __shfl_up_sync(0xffffffffu, li, 1);
-                if (lane < top_k && pos < top_k) {
-                    if (lane == pos) { lv = v; ls = sc; li = e; }
-                    else if (lane > pos) { lv = pv; ls = ps; li = pi; }
-                }
-            }
-            top = __shfl_sync(0xffffffffu, lv, 0);
-            bv_list = lv;
-            bs_list = ls;
-            be_list = li;
-        }
-        double wv;
-        if (SIG) {
-            double ssum = 0.0;
-            for (int jj = 0; jj < top_k; ++jj)
-                ssum += __shfl_sync(0xffffffffu, lane < top_k ? bs_list : 0.0, jj);
-            wv = (double)scale * (normalize ? bs_list / ssum : bs_list);
-        } else {
-            const double ev = lane < top_k ? exp(bv_list - top) : 0.0;
-            double ssum = 0.0;
-            for (int jj = 0; jj < top_k; ++jj)
-                ssum += __shfl_sync(0xffffffffu, ev, jj);
-            wv = ev / ssum;
-        }
-        if (lane < top_k) {
-            ids[(t0 + t) * top_k + lane] = be_list;
-            weights[(t0 + t) * top_k + lane] = (float)wv;
-        }
-    }
+    router_pick_owned<XF32, SIG, kRtThreads / 32>(
+        n_local, (int)rank, NC, t0, x, H, w_router, bias, E, top_k, ids, weights, normalize,
+        scale, logit, ncand, cand, cval, cscore, kRouterMaxCand,
+        [&](int j, int e) { return bound[j * E + e]; });
 }
 
 }  // namespace epk

@@ -1,0 +1,348 @@
+// router_tc.cuh -- the router for batches of more than 32 tokens of bf16
+// activations (E <= 256) with its logits on the tensor cores.
+//
+// The same operation as router_tiled_kernel (fak note "GLM-5.2 multi-GPU",
+// "What landed": every rank runs the router on the same rows), with the
+// logit contraction l = W_router x moved from fp32 CUDA-core FMAs to tcgen05:
+//
+//  * A cluster of CK CTAs (2 <= CK <= 8) takes a tile of 64 tokens; CTA k of
+//    the cluster contracts the k-th of CK slices of H.  Warp 0 issues TMA
+//    loads (128-byte swizzle, each CTA its own copy) of the router weights,
+//    one 128-expert box per MMA M tile (MT = 1 or 2), and of the 64 token
+//    rows; warp 1 issues tcgen05.mma (M = 128 experts, N = 64 tokens) into
+//    fp32 TMEM accumulators; warps 2..7 add up, from the same shared-memory
+//    stages, each expert's and each token's sum of squares over the slice
+//    (a row's sum does not depend on the swizzle's order of its chunks).
+//  * Warps 2..5 drain the accumulators (tcgen05.ld) into a [token][expert]
+//    tile; the CK partial tiles are added in ascending slice order over
+//    distributed shared memory by the CTA that owns the token (CK owners per
+//    tile, 64 / CK tokens each), which also forms its error bound.
+//  * The owner then picks as router_tiled_kernel does (router_pick_owned):
+//    every expert that could reach the k-th largest under the bounds is
+//    recomputed by Dot2 and the pick and the weights are made on those
+//    values, so the result is that of the other routers.
+//
+// Error bound of a tensor-core logit.  The products x_h w_h of bf16 values
+// are exact in fp32; only the accumulation rounds.  The tensor core's fp32
+// accumulation order and rounding are not specified, so the bound assumes
+// little: each MMA instruction (16 products added to the accumulator) may
+// err by up to 2^-19 of the magnitudes it adds (|acc| + sum |p|), which
+// covers aligning 17 operands to the largest and truncating each to 25 bits,
+// and a final rounding.  Over n instructions along one accumulator that is at
+// most 2 n 2^-19 S, S = sum_h |x_h w_h| <= ||x|| ||w||; the CK partials are
+// then added in fp32 ((CK + 2) u S more, u = 2^-24) and the bias (u |l|).
+// A test checks the tensor core's actual error against this bound.
+#pragma once
+
+#include "common.cuh"
+#include "grouped.cuh"
+#include "router.cuh"
+
+namespace epk {
+
+constexpr int kRcNT = 64;         // tokens per tile: the MMA's N
+constexpr int kRcThreads = 256;
+constexpr int kRcMaxE = 256;      // two 128-expert M tiles at most
+constexpr int kRcMaxCand = 32;    // refined candidates per token
+constexpr int kRcMinCK = 2;
+constexpr int kRcMaxCK = 8;
+constexpr uint32_t kRcWBox = kGemmBM * kGemmBK * 2;  // 128 experts x 64 of H, 16 KB
+constexpr uint32_t kRcXBox = kRcNT * kGemmBK * 2;    // 64 tokens x 64 of H, 8 KB
+constexpr int kRcNormWarps = 6;                      // warps 2..7
+
+struct RcMaps {
+    CUtensorMap w;  // W_router [E, H]: box 64 x 128
+    CUtensorMap x;  // x [T, H]: box 64 x 64
+};
+
+// Shared memory: the stage ring, later reused for the partial tile, the
+// norms, and the owned tokens' logits, bounds and candidates.
+struct RcSmem {
+    uint32_t stage_bytes, stages, ring;            // ring = stages * stage_bytes
+    uint32_t part, xsq, wsq;                       // read by the cluster's other CTAs
+    uint32_t logit, bound, xn, wn, ncand, cand, cval, cscore, end;  // this CTA's only
+    uint32_t bars, total, alloc;
+};
+
+__host__ __device__ inline RcSmem rc_smem_layout(int MT, int E, int CK) {
+    RcSmem s;
+    s.stage_bytes = MT * kRcWBox + kRcXBox;
+    s.stages = 200u * 1024u / s.stage_bytes;
+    if (s.stages > 8)
+        s.stages = 8;
+    s.ring = s.stages * s.stage_bytes;
+    const uint32_t own = (kRcNT + CK - 1) / CK;  // tokens a CTA owns at most
+    uint32_t o = 0;
+    s.part = o;   o = align_up_u32(o + (uint32_t)kRcNT * E * 4, 16);
+    s.xsq = o;    o = align_up_u32(o + (uint32_t)kRcNT * 4, 16);
+    s.wsq = o;    o = align_up_u32(o + (uint32_t)E * 4, 16);
+    s.logit = o;  o = align_up_u32(o + own * E * 4, 16);
+    s.bound = o;  o = align_up_u32(o + own * E * 4, 16);
+    s.xn = o;     o = align_up_u32(o + own * 4, 16);
+    s.wn = o;     o = align_up_u32(o + (uint32_t)E * 4, 16);
+    s.ncand = o;  o = align_up_u32(o + own * 4, 16);
+    s.cand = o;   o = align_up_u32(o + own * kRcMaxCand * 4, 16);
+    s.cval = o;   o = align_up_u32(o + own * kRcMaxCand * 8, 16);
+    s.cscore = o; o = align_up_u32(o + own * kRcMaxCand * 8, 16);
+    s.end = o;
+    s.bars = align_up_u32(s.ring > s.end ? s.ring : s.end, 1024);
+    // full[S], empty[S], tdone; tmem holder, abort flag
+    s.total = s.bars + (2 * s.stages + 1) * 8 + 16;
+    s.alloc = s.total + 1024;
+    return s;
+}
+
+template <bool SIG>
+__global__ void __launch_bounds__(kRcThreads, 1)
+router_tc_kernel(const __grid_constant__ RcMaps maps, const uint16_t *__restrict__ x,
+                 int64_t T, int H, const uint16_t *__restrict__ w_router,
+                 const float *__restrict__ bias, int E, int top_k, int32_t *__restrict__ ids,
+                 float *__restrict__ weights, int CK, int normalize, float scale,
+                 float *__restrict__ dump_logit, float *__restrict__ dump_bound) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int MT = (E + kGemmBM - 1) / kGemmBM;
+    const RcSmem L = rc_smem_layout(MT, E, CK);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bars);
+    uint64_t *empty = full + L.stages;
+    uint64_t *tdone = empty + L.stages;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(tdone + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tdone + 1) + 2;
+    float *part = reinterpret_cast<float *>(smem + L.part);    // [64][E]
+    float *xsq = reinterpret_cast<float *>(smem + L.xsq);      // [64]
+    float *wsq = reinterpret_cast<float *>(smem + L.wsq);      // [E]
+    float *logit = reinterpret_cast<float *>(smem + L.logit);  // [own][E]
+    float *bound = reinterpret_cast<float *>(smem + L.bound);  // [own][E]
+    float *xn = reinterpret_cast<float *>(smem + L.xn);        // [own] ||x_t||
+    float *wn = reinterpret_cast<float *>(smem + L.wn);        // [E] ||w_e||
+    int *ncand = reinterpret_cast<int *>(smem + L.ncand);
+    int *cand = reinterpret_cast<int *>(smem + L.cand);
+    double *cval = reinterpret_cast<double *>(smem + L.cval);
+    double *cscore = reinterpret_cast<double *>(smem + L.cscore);
+
+    const int warp = (int)(threadIdx.x >> 5), lane = (int)lane_id();
+    const uint32_t rank = cluster_ctarank();
+    const int64_t t0 = (int64_t)blockIdx.y * kRcNT;
+    const int tb = (T - t0 < (int64_t)kRcNT) ? (int)(T - t0) : kRcNT;
+    const int nkb = (H + kGemmBK - 1) / kGemmBK;
+    const int kb_lo = nkb * (int)rank / CK, kb_hi = nkb * ((int)rank + 1) / CK;
+    const uint32_t tcols = MT * kRcNT <= 64 ? 64u : 128u;
+
+    if (warp == 0 && lane == 0) {
+        for (uint32_t s = 0; s < L.stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1 + kRcNormWarps);
+        }
+        mbar_init(tdone, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tensormap(&maps.w);
+        prefetch_tensormap(&maps.x);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, tcols);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_holder;
+    grid_dependents_launch();
+    // x may come from the previous kernel, which may also still read the ids
+    // and weights this call overwrites
+    grid_dependency_wait();
+
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer
+        if (elect_one()) {
+            const uint64_t pol = policy_evict_last();  // every tile rereads W
+            uint32_t stage = 0, phase = 0;
+            int issued = 0;
+            for (int kb = kb_lo; kb < kb_hi; ++kb) {
+                if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag))
+                    break;
+                uint8_t *sa = smem + stage * L.stage_bytes;
+                mbar_arrive_expect_tx(&full[stage], L.stage_bytes);
+                const int k0 = kb * kGemmBK;
+                for (int m = 0; m < MT; ++m)
+                    tma_load_2d(sa + m * kRcWBox, &maps.w, k0, m * kGemmBM, &full[stage], pol);
+                tma_load_2d(sa + MT * kRcWBox, &maps.x, k0, (int32_t)t0, &full[stage], pol);
+                ++issued;
+                if (++stage == L.stages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            // no copy may still be landing in shared memory when the stages
+            // are reused below
+            for (int n = issued > (int)L.stages ? issued - (int)L.stages : 0; n < issued; ++n)
+                mbar_wait(&full[n % L.stages], (uint32_t)(n / L.stages) & 1u, nullptr);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer
+        if (elect_one()) {
+            uint32_t stage = 0, phase = 0;
+            const uint32_t idesc = idesc_bf16_f32(kGemmBM, kRcNT);
+            for (int kb = kb_lo; kb < kb_hi; ++kb) {
+                if (!mbar_wait(&full[stage], phase, abort_flag))
+                    break;
+                tc_fence_after_sync();
+                const uint32_t a0 = smem_u32(smem + stage * L.stage_bytes);
+                const uint32_t b0 = a0 + MT * kRcWBox;
+                for (int m = 0; m < MT; ++m)
+#pragma unroll
+                    for (int kk = 0; kk < kGemmBK / 16; ++kk)
+                        umma_bf16(tmem_base + m * kRcNT,
+                                  smem_desc_sw128_kmajor(a0 + m * kRcWBox + kk * 32),
+                                  smem_desc_sw128_kmajor(b0 + kk * 32), idesc,
+                                  (kb > kb_lo || kk > 0) ? 1u : 0u);
+                umma_commit(&empty[stage]);
+                if (++stage == L.stages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            umma_commit(tdone);  // every MMA of the slice has completed
+        }
+    } else {
+        // ---------------------------------- sums of squares from the stages
+        const int nt = (int)threadIdx.x - 64;  // 0 .. 191
+        const int rows = MT * kGemmBM + kRcNT;
+        float2 sq[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        uint32_t stage = 0, phase = 0;
+        for (int kb = kb_lo; kb < kb_hi; ++kb) {
+            if (!mbar_wait(&full[stage], phase, abort_flag))
+                break;
+            const uint8_t *sa = smem + stage * L.stage_bytes;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int r = nt + i * (kRcThreads - 64);
+                if (r < rows) {
+                    // row r of the stage: W rows of tile r / 128, then x rows
+                    const uint4 *row = reinterpret_cast<const uint4 *>(
+                        sa + (r < MT * kGemmBM ? (r / kGemmBM) * kRcWBox + (r % kGemmBM) * 128
+                                               : MT * kRcWBox + (r - MT * kGemmBM) * 128));
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint4 v = row[c];
+                        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int h = 0; h < 4; ++h) {
+                            const float2 f = bf16x2_to_f2(w4[h]);
+                            sq[i] = ffma2(f, f, sq[i]);
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&empty[stage]);
+            if (++stage == L.stages) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+        // the partial tile out of TMEM: warps 2..5 hold lane quarters 2, 3, 0, 1
+        const bool have = mbar_wait(tdone, 0, abort_flag);
+        __syncwarp();
+        // the stages are free once every MMA and every copy has completed;
+        // the producer's final waits and tdone cover both
+        named_sync(1, kRcThreads - 64);
+        if (have && warp < 6) {
+            tc_fence_after_sync();
+            const int q = warp & 3;
+            for (int m = 0; m < MT; ++m) {
+                const int e = m * kGemmBM + 32 * q + lane;
+                for (int c0 = 0; c0 < kRcNT; c0 += 32) {
+                    uint32_t v[32];
+                    tmem_load_32cols(tmem_base + ((uint32_t)(32 * q) << 16) + m * kRcNT + c0, v);
+                    tmem_load_wait();
+                    if (e < E) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            part[(c0 + j) * E + e] = __uint_as_float(v[j]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int r = nt + i * (kRcThreads - 64);
+            if (r < MT * kGemmBM) {
+                if (r < E)
+                    wsq[r] = sq[i].x + sq[i].y;
+            } else if (r < rows) {
+                xsq[r - MT * kGemmBM] = sq[i].x + sq[i].y;
+            }
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem_base, tcols);
+    }
+    cluster_sync();  // every CTA's partial tile and norms are in place
+
+    // The owner of tokens [64 rank / CK, 64 (rank + 1) / CK) adds the CK
+    // partials of each (token, expert) in ascending slice order, then its
+    // bound: 1.5 (gam ||x|| ||w|| + u |l|) with gam for the longest slice.
+    const int own_lo = kRcNT * (int)rank / CK, own_hi = kRcNT * ((int)rank + 1) / CK;
+    const int n_local = max(0, min(own_hi, tb) - own_lo);
+    for (int i = threadIdx.x; i < E + n_local; i += kRcThreads) {
+        float s2 = 0.f;
+        for (int r = 0; r < CK; ++r)
+            s2 += ld_cluster_f32(map_shared_rank(i < E ? wsq + i : xsq + own_lo + (i - E),
+                                                 (uint32_t)r));
+        if (i < E)
+            wn[i] = sqrtf(s2);
+        else
+            xn[i - E] = sqrtf(s2);
+    }
+    __syncthreads();
+    {
+        const float u = 5.9604644775390625e-8f;  // 2^-24
+        const float n_instr = (float)(4 * ((nkb + CK - 1) / CK));
+        const float gam = 2.0f * n_instr * 1.9073486328125e-6f + (float)(CK + 2) * u;  // 2^-19
+        for (int idx = threadIdx.x; idx < n_local * E; idx += kRcThreads) {
+            const int j = idx / E, e = idx - j * E;
+            const int t = own_lo + j;
+            float sum = 0.f;
+            for (int r = 0; r < CK; ++r)
+                sum += ld_cluster_f32(map_shared_rank(part + t * E + e, (uint32_t)r));
+            const float b = bias != nullptr ? bias[e] : 0.f;
+            float l, d;
+            if (SIG) {
+                // key = sigmoid(l) + b; the sigmoid's slope is at most 1/4, and
+                // 4e-7 (1 + |key|) covers its fp32 evaluation and the sum
+                const float d_l = 1.5f * (gam * xn[j] * wn[e] + u * fabsf(sum)) + 1e-30f;
+                l = 1.0f / (1.0f + expf(-sum)) + b;
+                d = 0.25f * d_l + 4e-7f * (1.0f + fabsf(l));
+            } else {
+                l = sum + b;
+                d = 1.5f * (gam * xn[j] * wn[e] + u * fabsf(l)) + 1e-30f;
+            }
+            logit[j * E + e] = l;
+            bound[j * E + e] = d;
+        }
+    }
+    cluster_sync();  // no shared memory of another CTA is read after this point
+    if (dump_logit != nullptr) {
+        // inspection (moe_route_logits): the fp32 logits and their bounds
+        for (int idx = threadIdx.x; idx < n_local * E; idx += kRcThreads) {
+            const int j = idx / E, e = idx - j * E;
+            const int64_t t = t0 + own_lo + j;
+            dump_logit[t * E + e] = logit[j * E + e];
+            dump_bound[t * E + e] = bound[j * E + e];
+        }
+        return;
+    }
+
+    router_pick_owned<false, SIG, kRcThreads / 32>(
+        n_local, own_lo, 1, t0, x, H, w_router, bias, E, top_k, ids, weights, normalize, scale,
+        logit, ncand, cand, cval, cscore, kRcMaxCand,
+        [&](int j, int e) { return bound[j * E + e]; });
+}
+
+}  // namespace epk

@@ -105,6 +105,19 @@ ep_status moe_route(const void *x, ep_dtype x_dtype, int64_t T, int64_t H,
                     int32_t *ids, float *weights, void *stream);
 
 /*
+ * moe_route_logits -- for inspection: the fp32 logits (with the bias) that
+ * moe_route forms above 32 tokens before it refines its candidates, and the
+ * bound of each one's error, |logits[t,e] - exact l[t,e]| <= bounds[t,e],
+ * on which the selection of those candidates relies.  The router chosen by
+ * ep_set_router runs (for any T >= 1); nothing is picked.
+ *   logits, bounds  device, [T, E] fp32 (outputs)
+ * Other arguments, limits and errors as moe_route.
+ */
+ep_status moe_route_logits(const void *x, ep_dtype x_dtype, int64_t T, int64_t H,
+                           const void *w_router, const float *bias, int64_t E, float *logits,
+                           float *bounds, void *stream);
+
+/*
  * moe_route_sigmoid -- the GLM router variant (TensorFold #593, a
  * contributor's comment "What exists now", glm_route.cu), which the page
  * describes only by its parts: a sigmoid score, a bias that takes part in
@@ -149,14 +162,24 @@ size_t moe_ffn_workspace_size(int64_t T, int64_t H, int64_t E, int32_t top_k, in
  *            (written only when I_s > 0);
  * and y[t] is the left fold of t's valid contrib rows in ascending (expert
  * id, j), then + shared[t].  The CUDA-core streaming kernels (T = 1, or fp32
- * x) fold on chip and write neither.  bytes = moe_ffn_workspace_size.  The
- * sizes are checked as moe_ffn_forward checks them (EP_EINVAL), and T = 0
- * gives an all-zero layout.
+ * x) fold on chip and write neither.  After a call on the grouped path
+ * (T > 8) the workspace also holds the grouping of the picks by expert:
+ *   group_offset  [E + 2] int32 at group_offset_offset: the picks of expert
+ *            e are rows [group_offset[e], group_offset[e+1]) of the grouped
+ *            order; group_offset[E] = the number of valid picks,
+ *            group_offset[E+1] = T * top_k;
+ *   perm     [T * top_k] int32 at perm_offset: row r of the grouped order is
+ *            pick perm[r] = t * top_k + j; inside an expert the picks keep
+ *            their (t, j) order (a stable sort by expert id).
+ * bytes = moe_ffn_workspace_size.  The sizes are checked as moe_ffn_forward
+ * checks them (EP_EINVAL), and T = 0 gives an all-zero layout.
  */
 typedef struct {
     size_t bytes;
     size_t contrib_offset;
     size_t shared_offset;
+    size_t group_offset_offset;
+    size_t perm_offset;
 } ep_workspace_layout_t;
 ep_status moe_ffn_workspace_layout(int64_t T, int64_t H, int64_t E, int32_t top_k, int64_t I,
                                    int64_t I_s, ep_workspace_layout_t *out);
@@ -292,7 +315,8 @@ ep_status moe_ep_combine(const float *partials, int64_t T, int64_t H, const int3
  * Which moe_ffn_forward path runs.  EP_DISPATCH_AUTO (the default) takes the
  * weight-streaming path for T <= 8 when its on-chip buffers fit, else the
  * tensor-core path; inside the streaming path, the tensor-core kernels from
- * 2 tokens with bf16 x, the CUDA-core kernels otherwise.  Forcing a path that does not fit the sizes makes
+ * 2 tokens with bf16 x, the CUDA-core kernels otherwise; on the tensor path,
+ * GEMM tiles of 128 weight rows.  Forcing a path that does not fit the sizes makes
  * moe_ffn_forward return EP_EINVAL.  Process-wide; meant for tests and tuning.
  */
 typedef enum {
@@ -304,9 +328,32 @@ typedef enum {
     EP_DISPATCH_STREAMING_TC = 3,
     /* streaming path, gate/up on the CUDA cores and down with the fold (two
        launches) */
-    EP_DISPATCH_STREAMING_SIMT = 4
+    EP_DISPATCH_STREAMING_SIMT = 4,
+    /* tensor path with GEMM tiles of 128 weight rows (two accumulators, the
+       epilogue of one tile beside the MMAs of the next) */
+    EP_DISPATCH_TENSOR_M128 = 5,
+    /* tensor path with GEMM tiles of 256 weight rows (two 128-row halves on
+       one activation tile, one accumulator) */
+    EP_DISPATCH_TENSOR_M256 = 6
 } ep_dispatch;
 ep_status ep_set_dispatch(ep_dispatch mode);
+
+/*
+ * Which router moe_route and moe_route_sigmoid run for more than 32 tokens
+ * (up to 32 tokens every logit is a Dot2 sum on the CUDA cores).
+ * EP_ROUTER_AUTO (the default) takes the tensor-core router where it fits
+ * (bf16 x, E <= 256, H >= 128), else the CUDA-core one.  Both form fp32
+ * logits with an error bound and refine every expert that could reach the
+ * top_k by Dot2, so they give the same ids and the same weights.  Forcing
+ * EP_ROUTER_TENSOR where it does not fit makes those calls return EP_EINVAL.
+ * Process-wide; meant for tests and tuning.
+ */
+typedef enum {
+    EP_ROUTER_AUTO = 0,
+    EP_ROUTER_TILED = 1,   /* register-tiled fp32 logits on the CUDA cores */
+    EP_ROUTER_TENSOR = 2   /* fp32 logits on the tensor cores (tcgen05) */
+} ep_router_mode;
+ep_status ep_set_router(ep_router_mode mode);
 
 /*
  * Launch mode.  Kernels are launched with programmatic dependent launch: a

@@ -33,7 +33,7 @@ from gpu_parity import device_inputs, oracle_route, shared_of
 
 pytestmark = pytest.mark.gpu
 
-PATHS = ["streaming_simt", "streaming_tc", "tensor"]
+PATHS = ["streaming_simt", "streaming_tc", "tensor_m128", "tensor_m256"]
 
 
 @pytest.fixture(autouse=True)
@@ -186,9 +186,12 @@ def _workspace_fold(x, ids, w, W, plan, path):
 
 @pytest.mark.parametrize("name,T,path", [("decode", 4, "streaming_tc"),
                                          ("decode", 8, "streaming_tc"),
-                                         ("decode", 8, "tensor"),
-                                         ("prefill", 512, "tensor"),
-                                         ("imbalanced", 2048, "tensor")])
+                                         ("decode", 8, "tensor_m128"),
+                                         ("decode", 8, "tensor_m256"),
+                                         ("prefill", 512, "tensor_m128"),
+                                         ("prefill", 512, "tensor_m256"),
+                                         ("imbalanced", 2048, "tensor_m128"),
+                                         ("imbalanced", 2048, "tensor_m256")])
 def test_y_is_the_host_fold_of_the_dumped_contributions(oracle_lib, name, T, path):
     wl = workloads.WORKLOADS[name]
     W, x = device_inputs(wl, T, batch=4)
@@ -199,3 +202,40 @@ def test_y_is_the_host_fold_of_the_dumped_contributions(oracle_lib, name, T, pat
         assert np.array_equal(ids.cpu().numpy(), ids_ref)
     y, want = _workspace_fold(x, ids, w, W, ed.ep_plan(wl.E, wl.bands[0]), path)
     assert np.array_equal(y.view(np.uint32), want.view(np.uint32)), (name, T, path)
+
+
+@pytest.mark.parametrize("name,T,seed", [("prefill", 512, 1000), ("large", 4096, 1000),
+                                         ("tiny", 300, 7)])
+def test_grouping_is_a_stable_sort_by_expert(name, T, seed):
+    """The grouped path's plan (group_plan_kernel: warp histograms, scans,
+    stable scatter) against a host stable sort of the picks by expert id, bit
+    for bit, with some empty, repeated and out-of-range ids mixed in."""
+    wl = workloads.WORKLOADS[name]
+    W, x = device_inputs(wl, T, seed=seed)
+    ids, w = ed.moe_route(x, W["w_router"], W["bias"], wl.top_k)
+    ids = ids.clone()
+    ids[3, 0] = ep.EP_ID_NONE
+    ids[5, 1] = ids[5, 0]
+    ids[T - 1, wl.top_k - 1] = wl.E + 4
+    E, k = wl.E, wl.top_k
+    I, I_s = wl.I, wl.I_s
+    lay = ed.moe_ffn_workspace_layout(T, wl.H, E, k, I, I_s)
+    ws = torch.empty(lay.bytes, dtype=torch.uint8, device="cuda")
+    ed.ep_set_dispatch("tensor")
+    ed.moe_ffn_forward(x, ids, w, W["w_gate"], W["w_up"], W["w_down"], shared_of(W),
+                       ed.ep_plan(E, 1), workspace=ws)
+    torch.cuda.synchronize()
+    with pytest.raises(ed.EPError):   # the out-of-range id is reported
+        ed.ep_check_status()
+    wsh = ws.cpu().numpy()
+    go = wsh[lay.group_offset_offset:lay.group_offset_offset + (E + 2) * 4].view(np.int32)
+    P = T * k
+    perm = wsh[lay.perm_offset:lay.perm_offset + P * 4].view(np.int32)
+    flat = ids.cpu().numpy().reshape(-1)
+    valid = [p for p in range(P) if 0 <= flat[p] < E]
+    want = sorted(valid, key=lambda p: (int(flat[p]), p))   # stable by expert id
+    counts = np.bincount(flat[valid], minlength=E)
+    want_go = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    assert np.array_equal(go[:E + 1], want_go)
+    assert go[E + 1] == P
+    assert np.array_equal(perm[:len(valid)], np.array(want, dtype=np.int32))

@@ -16,6 +16,14 @@ pytestmark = pytest.mark.gpu
 WL = workloads.WORKLOADS
 
 
+# above 32 tokens: the CUDA-core (tiled) and the tensor-core logits
+@pytest.fixture(params=["tiled", "tensor"])
+def router(request):
+    ed.ep_set_router(request.param)
+    yield request.param
+    ed.ep_set_router("auto")
+
+
 def _route_and_check(o, wl, T, normalize=False, scale=1.0, rows=None, seed=workloads.SEED_BASE,
                      **sizes):
     W, x = device_inputs(wl, T, seed=seed, **sizes)
@@ -46,16 +54,16 @@ def test_sigmoid_small_batches_with_bias(oracle_lib, T, x_dtype):
 
 
 @pytest.mark.parametrize("T", [40, 200])
-def test_sigmoid_tiled_odd_sizes(oracle_lib, T):
+def test_sigmoid_tiled_odd_sizes(oracle_lib, router, T):
     wl = workloads.Workload("sig_tiled", (T,), 200, 37, 5, 16, 0, "bf16", "zipf1.1", (1,))
     _route_and_check(oracle_lib, wl, T, normalize=True, seed=7)
 
 
-def test_sigmoid_prefill_full(oracle_lib):
+def test_sigmoid_prefill_full(oracle_lib, router):
     _route_and_check(oracle_lib, WL["prefill"], 512)
 
 
-def test_sigmoid_imbalanced_bias_selects_only(oracle_lib):
+def test_sigmoid_imbalanced_bias_selects_only(oracle_lib, router):
     """+8 on experts 0..15 puts every pick there, but the weights stay the raw
     sigmoid scores (no 8 in them)."""
     wl = WL["imbalanced"]
@@ -67,7 +75,7 @@ def test_sigmoid_imbalanced_bias_selects_only(oracle_lib):
     _route_and_check(oracle_lib, wl, 2048)
 
 
-def test_sigmoid_large_sampled(oracle_lib):
+def test_sigmoid_large_sampled(oracle_lib, router):
     T = 4096
     rows = np.r_[0:16, 16:T - 16:61, T - 16:T]
     _route_and_check(oracle_lib, WL["large"], T, rows=rows)

@@ -15,10 +15,12 @@ pytestmark = pytest.mark.gpu
 WL = workloads.WORKLOADS
 
 
-@pytest.fixture(autouse=True)
-def tensor_dispatch():
-    ed.ep_set_dispatch("tensor")
-    yield
+# Every test runs with GEMM tiles of 128 weight rows (two accumulators) and of
+# 256 (two 128-row halves on one activation tile, one accumulator).
+@pytest.fixture(autouse=True, params=["tensor_m128", "tensor_m256"])
+def tensor_dispatch(request):
+    ed.ep_set_dispatch(request.param)
+    yield request.param
     ed.ep_set_dispatch("auto")
 
 
@@ -77,14 +79,15 @@ def test_hot_expert_many_tiles(oracle_lib):
     check_y(y[rows], ref, what="hot expert")
 
 
-def test_tensor_matches_streaming_within_tolerance(oracle_lib):
+def test_tensor_matches_streaming_within_tolerance(oracle_lib, tensor_dispatch):
     wl = WL["decode"]
     W, x, ids, w, w_ref = _routed(oracle_lib, wl, 8, batch=2)
     plan = ed.ep_plan(wl.E, 8)
     y_t = gpu_ffn(x, ids, w, W, plan)
+    mode = tensor_dispatch
     ed.ep_set_dispatch("streaming")
     y_s = gpu_ffn(x, ids, w, W, plan)
-    ed.ep_set_dispatch("tensor")
+    ed.ep_set_dispatch(mode)
     ref = oracle_ffn(oracle_lib, x, ids, w_ref, W)
     check_y(y_t, ref, what="decode T=8 tensor")
     check_y(y_s, ref, rel_tol=1e-4, what="decode T=8 streaming")
