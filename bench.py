@@ -94,8 +94,7 @@ def parse_args(argv=None):
                          "(ep_plan(E, N)), every rank routes the same tokens, and the partials "
                          "are exchanged by the rank-order reduce-scatter (strong scaling)")
     ap.add_argument("--dispatch", default="auto",
-                    choices=("auto", "streaming", "tensor", "streaming_tc", "streaming_simt",
-                             "tensor_m128", "tensor_m256"),
+                    choices=("auto", "streaming", "tensor", "streaming_tc", "streaming_simt"),
                     help="tuning: the path moe_ffn_forward takes (ep_set_dispatch)")
     ap.add_argument("--reference-budget-s", type=float, default=150.0,
                     help="wall-time budget of the reference arm's warm-up and timed steps")

@@ -15,8 +15,7 @@ import torch
 EP_OK, EP_EINVAL, EP_EDIM, EP_EBADID, EP_ENOMEM, EP_ECUDA, EP_ETIMEOUT = range(7)
 EP_BF16, EP_F32 = 0, 1
 EP_MAX_BANDS = 64
-_DISPATCH = {"auto": 0, "streaming": 1, "tensor": 2, "streaming_tc": 3, "streaming_simt": 4,
-             "tensor_m128": 5, "tensor_m256": 6}
+_DISPATCH = {"auto": 0, "streaming": 1, "tensor": 2, "streaming_tc": 3, "streaming_simt": 4}
 _NAMES = {0: "EP_OK", 1: "EP_EINVAL", 2: "EP_EDIM", 3: "EP_EBADID", 4: "EP_ENOMEM",
           5: "EP_ECUDA", 6: "EP_ETIMEOUT"}
 

@@ -21,6 +21,7 @@
 #include "decode_tc.cuh"
 #include "ep.cuh"
 #include "router_tc.cuh"
+#include "decode_fp4.cuh"
 
 namespace {
 
@@ -161,6 +162,10 @@ ep_status device_info(const DeviceInfo **out) {
         EPK_RD_ATTR(false, 1, true); EPK_RD_ATTR(false, 2, true);
         EPK_RD_ATTR(true, 1, true); EPK_RD_ATTR(true, 2, true);
 #undef EPK_RD_ATTR
+        EP_CUDA_CHECK(cudaFuncSetAttribute(epk::stream_gate_up_fp4_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, m));
+        EP_CUDA_CHECK(cudaFuncSetAttribute(epk::stream_down_fp4_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, m));
         EP_CUDA_CHECK(cudaFuncSetAttribute(epk::router_tc_kernel<false>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, m));
         EP_CUDA_CHECK(cudaFuncSetAttribute(epk::router_tc_kernel<true>,
@@ -196,8 +201,6 @@ constexpr int kMaxTopK = 16;
 constexpr int64_t kTcMinT = 2;
 
 
-// GEMM tile height of the tensor path by default: 1 = 128 weight rows, 2 = 256
-constexpr int kGemmMhAuto = 1;
 // moe_route computes every logit by Dot2 up to this many tokens
 constexpr int64_t kRouterDot2MaxT = 32;
 // Shared memory the streaming kernels may take, leaving the rest of the
@@ -319,7 +322,7 @@ extern "C" ep_status ep_plan(int32_t num_experts, int32_t bands, ep_plan_t *out)
 }
 
 extern "C" ep_status ep_set_dispatch(ep_dispatch mode) {
-    if ((int)mode < (int)EP_DISPATCH_AUTO || (int)mode > (int)EP_DISPATCH_TENSOR_M256)
+    if ((int)mode < (int)EP_DISPATCH_AUTO || (int)mode > (int)EP_DISPATCH_STREAMING_SIMT)
         return fail(EP_EINVAL, "ep_set_dispatch: unknown mode %d", (int)mode);
     g_dispatch.store((int)mode);
     return ok();
@@ -699,8 +702,7 @@ ep_status ffn_forward_impl(bool band_call, const void *x, ep_dtype x_dtype, int6
         if (!sp.fits)
             return fail(EP_EINVAL, "moe_ffn_forward: the streaming path does not fit these sizes");
         use_streaming = true;
-    } else if (mode == EP_DISPATCH_TENSOR || mode == EP_DISPATCH_TENSOR_M128 ||
-               mode == EP_DISPATCH_TENSOR_M256) {
+    } else if (mode == EP_DISPATCH_TENSOR) {
         use_streaming = false;
     } else {
         use_streaming = sp.fits;
@@ -848,7 +850,6 @@ ep_status ffn_forward_impl(bool band_call, const void *x, ep_dtype x_dtype, int6
     g.sm_count = d->sm_count;
     g.smem_optin = d->smem_optin;
     g.pdl = pdl_enabled();
-    g.mh = mode == EP_DISPATCH_TENSOR_M256 ? 2 : (mode == EP_DISPATCH_TENSOR_M128 ? 1 : kGemmMhAuto);
     int launches = 0;
     char why[256] = "";
     s = epk::grouped_forward(g, W.grouped, ws, st, &launches, why, sizeof why,
@@ -871,6 +872,172 @@ extern "C" ep_status moe_ffn_forward(const void *x, ep_dtype x_dtype, int64_t T,
     return ffn_forward_impl(false, x, x_dtype, T, H, ids, weights, top_k, w_gate, w_up, w_down,
                             E, I, ws_gate, ws_up, ws_down, I_s, plan, y, workspace,
                             workspace_bytes, stream);
+}
+
+// ============================================================ NVFP4 decode
+namespace {
+
+struct Fp4Workspace {
+    size_t x16 = 0, hb = 0, hs = 0, c = 0, s = 0, total = 0;
+};
+
+Fp4Workspace fp4_workspace_layout(int64_t T, int64_t H, int64_t k, int64_t I, int64_t I_s) {
+    Fp4Workspace w;
+    size_t o = 0;
+    w.x16 = o; o = align256(o + (size_t)T * H * 2);
+    w.hb = o;  o = align256(o + (size_t)(2 * T * k + 2 * epk::kTcSlice) * I * 2);
+    w.hs = o;  o = align256(o + (size_t)2 * epk::kTcSlice * std::max<int64_t>(I_s, 64) * 2);
+    w.c = o;   o = align256(o + (size_t)T * k * H * 4);
+    w.s = o;   o = align256(o + (size_t)T * H * 4);
+    w.total = o;
+    return w;
+}
+
+bool fp4_mat_ok(const ep_nvfp4_t *m) {
+    return m != nullptr && m->codes != nullptr && m->scales != nullptr && aligned(m->codes, 16) &&
+           aligned(m->scales, 4) && std::isfinite(m->tensor_scale);
+}
+
+}  // namespace
+
+extern "C" size_t moe_ffn_nvfp4_workspace_size(int64_t T, int64_t H, int64_t E, int32_t top_k,
+                                               int64_t I, int64_t I_s) {
+    if (T <= 0 || H <= 0 || E <= 0 || top_k <= 0 || I <= 0 || I_s < 0)
+        return 0;
+    return fp4_workspace_layout(T, H, top_k, I, I_s).total;
+}
+
+extern "C" ep_status moe_ffn_forward_nvfp4(const void *x, int64_t T, int64_t H,
+                                           const int32_t *ids, const float *weights,
+                                           int32_t top_k, const ep_nvfp4_t *w_gate,
+                                           const ep_nvfp4_t *w_up, const ep_nvfp4_t *w_down,
+                                           int64_t E, int64_t I, const ep_nvfp4_t *ws_gate,
+                                           const ep_nvfp4_t *ws_up, const ep_nvfp4_t *ws_down,
+                                           int64_t I_s, const ep_plan_t *plan, float *y,
+                                           void *workspace, size_t workspace_bytes,
+                                           void *stream) {
+    const char *who = "moe_ffn_forward_nvfp4";
+    if (plan == nullptr)
+        return fail(EP_EINVAL, "%s: plan is NULL", who);
+    if (plan->num_experts != E)
+        return fail(EP_EDIM, "%s: plan covers %d experts, E = %lld", who, plan->num_experts,
+                    (long long)E);
+    if (plan->bands < 1 || plan->bands > EP_MAX_BANDS || plan->bands > E ||
+        plan->band_start[0] != 0 || plan->band_start[plan->bands] != E)
+        return fail(EP_EINVAL, "%s: plan is not a partition of [0, E)", who);
+    for (int r = 0; r < plan->bands; ++r)
+        if (plan->band_start[r + 1] <= plan->band_start[r])
+            return fail(EP_EINVAL, "%s: band %d of the plan is empty or reversed", who, r);
+    if (T < 0 || T > epk::kStreamMaxT)
+        return fail(EP_EINVAL, "%s: T = %lld outside [0, %d]", who, (long long)T,
+                    epk::kStreamMaxT);
+    auto dim_ok = [](int64_t v) { return v >= 64 && v <= kMaxH && v % 64 == 0; };
+    if (!dim_ok(H) || !dim_ok(I) || (I_s != 0 && !dim_ok(I_s)))
+        return fail(EP_EINVAL, "%s: H, I and I_s must be multiples of 64 in [64, %lld]", who,
+                    (long long)kMaxH);
+    if (E < 1 || E > kMaxE)
+        return fail(EP_EINVAL, "%s: E = %lld outside [1, %lld]", who, (long long)E,
+                    (long long)kMaxE);
+    if (top_k < 1 || top_k > kMaxTopK || top_k > E)
+        return fail(EP_EINVAL, "%s: top_k = %d outside [1, min(E, %d)]", who, top_k, kMaxTopK);
+    if (T == 0) {
+        t_launches = 0;
+        return ok();
+    }
+    if (x == nullptr || ids == nullptr || weights == nullptr || y == nullptr ||
+        !fp4_mat_ok(w_gate) || !fp4_mat_ok(w_up) || !fp4_mat_ok(w_down))
+        return fail(EP_EINVAL, "%s: a required pointer is NULL or misaligned", who);
+    if ((I_s > 0) != (ws_gate != nullptr) || (I_s > 0) != (ws_up != nullptr) ||
+        (I_s > 0) != (ws_down != nullptr) ||
+        (I_s > 0 && (!fp4_mat_ok(ws_gate) || !fp4_mat_ok(ws_up) || !fp4_mat_ok(ws_down))))
+        return fail(EP_EINVAL, "%s: shared-expert matrices must all be given iff I_s > 0", who);
+    if (!aligned(x, 16) || !aligned(y, 16) || !aligned(ids, 4) || !aligned(weights, 4))
+        return fail(EP_EINVAL, "%s: misaligned x, y, ids or weights", who);
+    const Fp4Workspace W = fp4_workspace_layout(T, H, top_k, I, I_s);
+    if (workspace == nullptr || workspace_bytes < W.total)
+        return fail(EP_ENOMEM, "%s: workspace of %zu bytes, %zu needed", who, workspace_bytes,
+                    W.total);
+    if (!aligned(workspace, 256))
+        return fail(EP_EINVAL, "%s: workspace not 256-byte aligned", who);
+    const DeviceInfo *d = nullptr;
+    ep_status s = device_info(&d);
+    if (s != EP_OK)
+        return s;
+    if (epk::F4Smem::alloc > (uint32_t)d->smem_optin ||
+        epk::F4DnSmem::alloc > (uint32_t)d->smem_optin || epk::tensor_map_encoder() == nullptr)
+        return fail(EP_ECUDA, "%s: this device cannot run the NVFP4 kernels", who);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint16_t *x16 = reinterpret_cast<uint16_t *>(ws + W.x16);
+    uint16_t *hb = reinterpret_cast<uint16_t *>(ws + W.hb);
+    uint16_t *hs = reinterpret_cast<uint16_t *>(ws + W.hs);
+    float *c = reinterpret_cast<float *>(ws + W.c);
+    float *sh = reinterpret_cast<float *>(ws + W.s);
+
+    epk::F4GuMaps gm;
+    memset(&gm, 0, sizeof gm);
+    bool okm = epk::map_codes(&gm.cg, w_gate->codes, H, I, E, epk::kGateUpRows) &&
+               epk::map_codes(&gm.cu, w_up->codes, H, I, E, epk::kGateUpRows) &&
+               epk::map_f16(&gm.x, x16, H, T, epk::kTcN);
+    if (I_s > 0)
+        okm = okm && epk::map_codes(&gm.sg, ws_gate->codes, H, I_s, 1, epk::kGateUpRows) &&
+              epk::map_codes(&gm.su, ws_up->codes, H, I_s, 1, epk::kGateUpRows);
+    epk::F4DnMaps dm;
+    memset(&dm, 0, sizeof dm);
+    okm = okm && epk::map_codes(&dm.cd, w_down->codes, I, H, E, epk::kGemmBM) &&
+          epk::map_f16(&dm.hr, hb, I, (uint64_t)(2 * T * top_k + 2 * epk::kTcSlice),
+                       2 * epk::kTcSlice);
+    if (I_s > 0)
+        okm = okm && epk::map_codes(&dm.sd, ws_down->codes, I_s, H, 1, epk::kGemmBM) &&
+              epk::map_f16(&dm.hs, hs, I_s, 2 * epk::kTcSlice, 2 * epk::kTcSlice);
+    if (!okm)
+        return fail(EP_ECUDA, "%s: encoding a tensor map failed", who);
+
+    auto mat = [](const ep_nvfp4_t *m, int64_t rows, int64_t cols) {
+        epk::F4Mat f;
+        f.scales = m == nullptr ? nullptr : static_cast<const uint8_t *>(m->scales);
+        f.ts = m == nullptr ? 0.f : m->tensor_scale;
+        f.rows = rows;
+        f.cols = cols;
+        return f;
+    };
+    const dim3 grid((unsigned)d->sm_count);
+    {
+        KernelBracket kb0(st, 0);
+        const int64_t n = T * H;
+        EP_CUDA_CHECK(launch(epk::to_f16_kernel, dim3((unsigned)((n + 255) / 256)), 256, 0, st,
+                             static_cast<const uint16_t *>(x), n, x16));
+    }
+    epk::F4GuArgs ga;
+    ga.T = (int)T; ga.H = (int)H; ga.E = (int)E; ga.I = (int)I; ga.I_s = (int)I_s;
+    ga.top_k = top_k; ga.ids = ids; ga.weights = weights;
+    ga.wg = mat(w_gate, I, H); ga.wu = mat(w_up, I, H);
+    ga.sg = mat(ws_gate, I_s, H); ga.su = mat(ws_up, I_s, H);
+    ga.hb_routed = hb; ga.hb_shared = I_s > 0 ? hs : nullptr;
+    {
+        KernelBracket kb1(st, 1);
+        EP_CUDA_CHECK(launch(epk::stream_gate_up_fp4_kernel, grid, epk::kF4Threads,
+                             epk::F4Smem::alloc, st, gm, ga));
+    }
+    epk::F4DnArgs da;
+    da.T = (int)T; da.H = (int)H; da.E = (int)E; da.I = (int)I; da.I_s = (int)I_s;
+    da.top_k = top_k; da.ids = ids; da.weights = weights;
+    da.wd = mat(w_down, H, I); da.sd = mat(ws_down, H, I_s);
+    da.c = c; da.s = sh;
+    {
+        KernelBracket kb2(st, 2);
+        EP_CUDA_CHECK(launch(epk::stream_down_fp4_kernel, grid, epk::kF4Threads,
+                             epk::F4DnSmem::alloc, st, dm, da));
+    }
+    {
+        KernelBracket kb3(st, 3);
+        const dim3 cgrid((unsigned)T, (unsigned)((H / 4 + 63) / 64));
+        EP_CUDA_CHECK(launch(epk::combine_kernel, cgrid, 64, 0, st, (const float *)c,
+                             (const float *)(I_s > 0 ? sh : nullptr), ids, (int64_t)T, (int)H,
+                             (int)top_k, (int)E, y));
+    }
+    t_launches = 4;
+    return ok();
 }
 
 // ======================================================== expert parallel

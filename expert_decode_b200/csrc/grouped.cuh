@@ -127,7 +127,6 @@ struct PlanArgs {
     const int32_t *ids;
     int64_t T, P;
     int top_k, E, H, I, I_s;
-    int mh;                 // 128-row halves per GEMM tile (grouped_gemm_kernel's MH)
     int32_t *group_offset;  // [E + 2]: routed row offsets, [E] = valid picks, [E+1] = P
     int32_t *perm_pair;     // [P]: permuted row -> pick index t * top_k + j
     int32_t *units_gu;      // [G + 1] exclusive prefix of gate/up tiles per group
@@ -233,9 +232,8 @@ __global__ void __launch_bounds__(kPlanThreads, 1) group_plan_kernel(const PlanA
                 const int64_t rows = g < E ? total[g] : a.T;
                 const int nb = (int)((rows + kGemmBN - 1) / kGemmBN);
                 const int m_rows = g < E ? a.I : a.I_s;
-                const int gu_rows = a.mh * kGateUpRows, dn_rows = a.mh * kGemmBM;
-                gu[q] = nb * ((m_rows + gu_rows - 1) / gu_rows);
-                dn[q] = nb * ((a.H + dn_rows - 1) / dn_rows);
+                gu[q] = nb * ((m_rows + kGateUpRows - 1) / kGateUpRows);
+                dn[q] = nb * ((a.H + kGemmBM - 1) / kGemmBM);
             }
         }
         const int all_gu = block_exclusive_scan2(gu[0], gu[1], wsum);
@@ -323,25 +321,8 @@ struct GemmParams {
     int b_rows[kBoxLevels], bs_rows[kBoxLevels];  // box heights of maps.b and maps.b_shared
 };
 
-// A tile of the grouped GEMMs is MH halves of 128 weight rows (the MMA's M
-// side) against up to 256 of the expert's rows (N).  MH = 2 puts two halves
-// on one shared activation tile: a 64 KB stage carries 8.4 MFLOP instead of
-// 4.2 MFLOP per 48 KB, so the same bytes in flight keep the tensor pipe busy
-// longer, and every activation tile is read from L2 half as often; the cost
-// is a single accumulator (the two halves fill the 512 TMEM columns), so a
-// tile's MMAs wait for the previous tile's epilogue.
-template <int MH>
-struct GemmCfg {
-    static constexpr int stages = MH == 1 ? kGemmStages : 3;
-    static constexpr uint32_t a_bytes = MH * kTileABytes;
-    static constexpr uint32_t stage_bytes = a_bytes + kTileBBytes;
-    static constexpr int n_acc = MH == 1 ? 2 : 1;           // accumulators in TMEM
-    static constexpr uint32_t acc_cols = MH * kGemmBN;      // columns of one accumulator
-};
-
-template <int MH>
 struct GemmSmem {
-    static constexpr uint32_t bars = GemmCfg<MH>::stages * GemmCfg<MH>::stage_bytes;
+    static constexpr uint32_t bars = kGemmStages * kStageBytes;
     static constexpr uint32_t misc = bars + 256;
     static constexpr uint32_t units = misc + 64;
     static constexpr uint32_t offsets = units + kMaxGroups * 4 + 4;
@@ -351,12 +332,11 @@ struct GemmSmem {
     static constexpr uint32_t alloc = total + 1024;  // room to align the base to 1024
 };
 
-template <bool GATE_UP, int MH>
+template <bool GATE_UP>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
-    using Cfg = GemmCfg<MH>;
-    using Smem = GemmSmem<MH>;
-    constexpr int S = Cfg::stages;
+    using Smem = GemmSmem;
+    constexpr int S = kGemmStages;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -466,31 +446,26 @@ grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
                         stop = true;
                         break;
                     }
-                    uint8_t *sa = smem + stage * Cfg::stage_bytes;
-                    uint8_t *sb = sa + Cfg::a_bytes;
-                    mbar_arrive_expect_tx(&full[stage], Cfg::a_bytes + b_bytes);
+                    uint8_t *sa = smem + stage * kStageBytes;
+                    uint8_t *sb = sa + kTileABytes;
+                    mbar_arrive_expect_tx(&full[stage], kTileABytes + b_bytes);
                     const int k0 = kb * kGemmBK;
-#pragma unroll
-                    for (int h = 0; h < MH; ++h) {
-                        uint8_t *sh = sa + h * kTileABytes;
-                        if (GATE_UP) {
-                            // half h, rows 0..63: W_gate of its 64 units, 64..127: W_up
-                            const int row = (mb * MH + h) * kGateUpRows;
-                            uint8_t *sh_up = sh + kGateUpRows * kGemmBK * 2;
-                            if (shared) {
-                                tma_load_2d(sh, &maps.a_shared, k0, row, &full[stage], pol_w);
-                                tma_load_2d(sh_up, &maps.a2_shared, k0, row, &full[stage], pol_w);
-                            } else {
-                                tma_load_3d(sh, &maps.a, k0, row, g, &full[stage], pol_w);
-                                tma_load_3d(sh_up, &maps.a2, k0, row, g, &full[stage], pol_w);
-                            }
+                    if (GATE_UP) {
+                        // rows 0..63: W_gate of the tile's 64 units, 64..127: W_up
+                        const int row = mb * kGateUpRows;
+                        uint8_t *sa_up = sa + kGateUpRows * kGemmBK * 2;
+                        if (shared) {
+                            tma_load_2d(sa, &maps.a_shared, k0, row, &full[stage], pol_w);
+                            tma_load_2d(sa_up, &maps.a2_shared, k0, row, &full[stage], pol_w);
                         } else {
-                            const int row = (mb * MH + h) * kGemmBM;
-                            if (shared)
-                                tma_load_2d(sh, &maps.a_shared, k0, row, &full[stage], pol_w);
-                            else
-                                tma_load_3d(sh, &maps.a, k0, row, g, &full[stage], pol_w);
+                            tma_load_3d(sa, &maps.a, k0, row, g, &full[stage], pol_w);
+                            tma_load_3d(sa_up, &maps.a2, k0, row, g, &full[stage], pol_w);
                         }
+                    } else {
+                        if (shared)
+                            tma_load_2d(sa, &maps.a_shared, k0, mb * kGemmBM, &full[stage], pol_w);
+                        else
+                            tma_load_3d(sa, &maps.a, k0, mb * kGemmBM, g, &full[stage], pol_w);
                     }
                     tma_load_2d(sb, bmap, k0, brow, &full[stage], pol_x);
                     ++issued;
@@ -521,7 +496,7 @@ grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
                 if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag))
                     break;
                 tc_fence_after_sync();
-                const uint32_t d_tmem = tmem_base + acc * Cfg::acc_cols;
+                const uint32_t d_tmem = tmem_base + acc * kGemmBN;
                 const int kblocks = (K + kGemmBK - 1) / kGemmBK;
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait(&full[stage], phase, abort_flag)) {
@@ -529,16 +504,13 @@ grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
                         break;
                     }
                     tc_fence_after_sync();
-                    const uint32_t a_addr = smem_u32(smem + stage * Cfg::stage_bytes);
-                    const uint32_t b_addr = a_addr + Cfg::a_bytes;
+                    const uint32_t a_addr = smem_u32(smem + stage * kStageBytes);
+                    const uint32_t b_addr = a_addr + kTileABytes;
 #pragma unroll
-                    for (int h = 0; h < MH; ++h)
-#pragma unroll
-                        for (int kk = 0; kk < kGemmBK / 16; ++kk)
-                            umma_bf16(d_tmem + h * kGemmBN,
-                                      smem_desc_sw128_kmajor(a_addr + h * kTileABytes + kk * 32),
-                                      smem_desc_sw128_kmajor(b_addr + kk * 32), idesc,
-                                      (kb > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < kGemmBK / 16; ++kk)
+                        umma_bf16(d_tmem, smem_desc_sw128_kmajor(a_addr + kk * 32),
+                                  smem_desc_sw128_kmajor(b_addr + kk * 32), idesc,
+                                  (kb > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&empty[stage]);  // frees the slot once these MMAs are done
                     if (++stage == S) {
                         stage = 0;
@@ -548,7 +520,7 @@ grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
                 if (stop)
                     break;
                 umma_commit(&tfull[acc]);
-                if (++acc == Cfg::n_acc) {
+                if (++acc == 2) {
                     acc = 0;
                     acc_phase ^= 1u;
                 }
@@ -562,12 +534,11 @@ grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         int *col_pick = reinterpret_cast<int *>(smem + Smem::colmeta) + (warp - 2) * 2 * kGemmBN;
         float *col_w = reinterpret_cast<float *>(col_pick + kGemmBN);
-        // gate/up: in each half, quarters 0, 1 hold the gate rows of units
-        // 0..31, 32..63 and quarters 2, 3 the up rows of the same units; the
-        // two warps of a pair (same units) swap half their columns through
-        // the colmeta area, which gate/up does not otherwise use: xg = gate
-        // values of columns 16..31, xu = up values of columns 0..15, each
-        // [16][32 lanes]
+        // gate/up: quarters 0, 1 hold the gate rows of units 0..31, 32..63 and
+        // quarters 2, 3 the up rows of the same units; the two warps of a pair
+        // (same units) swap half their columns through the colmeta area, which
+        // gate/up does not otherwise use: xg = gate values of columns 16..31,
+        // xu = up values of columns 0..15, each [16][32 lanes]
         const bool gate_warp = q < 2;
         const int pair = q & 1;
         float *xg = reinterpret_cast<float *>(smem + Smem::colmeta) + pair * 2 * 16 * 32;
@@ -597,64 +568,60 @@ grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
             if (!ok)
                 break;
             tc_fence_after_sync();
-#pragma unroll 1
-            for (int h = 0; h < MH; ++h) {
-                const uint32_t t_row = tmem_base + ((uint32_t)(32 * q) << 16) +
-                                       acc * Cfg::acc_cols + h * kGemmBN;
-                for (int c0 = 0; c0 < n_valid; c0 += 32) {
-                    uint32_t v[32];
-                    tmem_load_32cols(t_row + (uint32_t)c0, v);
-                    tmem_load_wait();
-                    if (GATE_UP) {
-                        // lane = unit; the gate warp finishes columns 0..15 of the
-                        // chunk, the up warp columns 16..31
-                        const int M = shared ? p.I_s : p.I;
-                        const int unit = (mb * MH + h) * kGateUpRows + 32 * pair + lane;
-                        uint16_t *hrow_base = shared ? p.h_shared_out : p.h_out;
-                        const int ld = shared ? p.I_s : p.I;
-                        const int64_t row0 = (shared ? 0 : offsets[g]) + n0 + c0;
-                        if (gate_warp) {
+            const uint32_t t_row = tmem_base + ((uint32_t)(32 * q) << 16) + acc * kGemmBN;
+            for (int c0 = 0; c0 < n_valid; c0 += 32) {
+                uint32_t v[32];
+                tmem_load_32cols(t_row + (uint32_t)c0, v);
+                tmem_load_wait();
+                if (GATE_UP) {
+                    // lane = unit; the gate warp finishes columns 0..15 of the
+                    // chunk, the up warp columns 16..31
+                    const int M = shared ? p.I_s : p.I;
+                    const int unit = mb * kGateUpRows + 32 * pair + lane;
+                    uint16_t *hrow_base = shared ? p.h_shared_out : p.h_out;
+                    const int ld = shared ? p.I_s : p.I;
+                    const int64_t row0 = (shared ? 0 : offsets[g]) + n0 + c0;
+                    if (gate_warp) {
 #pragma unroll
-                            for (int j = 0; j < 16; ++j)
-                                xg[j * 32 + lane] = __uint_as_float(v[16 + j]);
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 16; ++j)
-                                xu[j * 32 + lane] = __uint_as_float(v[j]);
-                        }
-                        named_sync(1 + pair, 64);
-                        if (gate_warp) {
-#pragma unroll
-                            for (int j = 0; j < 16; ++j) {
-                                const int col = c0 + j;
-                                if (col < n_valid && unit < M)
-                                    hrow_base[(size_t)(row0 + j) * ld + unit] = f32_to_bf16_rne(
-                                        silu_f32(__uint_as_float(v[j])) * xu[j * 32 + lane]);
-                            }
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 16; ++j) {
-                                const int col = c0 + 16 + j;
-                                if (col < n_valid && unit < M)
-                                    hrow_base[(size_t)(row0 + 16 + j) * ld + unit] = f32_to_bf16_rne(
-                                        silu_f32(xg[j * 32 + lane]) * __uint_as_float(v[16 + j]));
-                            }
-                        }
-                        named_sync(1 + pair, 64);  // the buffers are free for the next chunk
+                        for (int j = 0; j < 16; ++j)
+                            xg[j * 32 + lane] = __uint_as_float(v[16 + j]);
                     } else {
-                        const int row = (mb * MH + h) * kGemmBM + 32 * q + lane;
-                        if (row < p.H) {
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) {
-                                const int col = c0 + j;
-                                if (col < n_valid) {
-                                    const float d = __uint_as_float(v[j]);
-                                    if (shared) {
-                                        p.s_out[(size_t)(n0 + col) * p.H + row] = d;
-                                    } else {
-                                        const int pick = col_pick[col];
-                                        p.c_out[(size_t)pick * p.H + row] = col_w[col] * d;
-                                    }
+                        for (int j = 0; j < 16; ++j)
+                            xu[j * 32 + lane] = __uint_as_float(v[j]);
+                    }
+                    named_sync(1 + pair, 64);
+                    if (gate_warp) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int col = c0 + j;
+                            if (col < n_valid && unit < M)
+                                hrow_base[(size_t)(row0 + j) * ld + unit] = f32_to_bf16_rne(
+                                    silu_f32(__uint_as_float(v[j])) * xu[j * 32 + lane]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int col = c0 + 16 + j;
+                            if (col < n_valid && unit < M)
+                                hrow_base[(size_t)(row0 + 16 + j) * ld + unit] = f32_to_bf16_rne(
+                                    silu_f32(xg[j * 32 + lane]) * __uint_as_float(v[16 + j]));
+                        }
+                    }
+                    named_sync(1 + pair, 64);  // the buffers are free for the next chunk
+                } else {
+                    const int row = mb * kGemmBM + 32 * q + lane;
+                    if (row < p.H) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int col = c0 + j;
+                            if (col < n_valid) {
+                                const float d = __uint_as_float(v[j]);
+                                if (shared) {
+                                    p.s_out[(size_t)(n0 + col) * p.H + row] = d;
+                                } else {
+                                    const int pick = col_pick[col];
+                                    p.c_out[(size_t)pick * p.H + row] = col_w[col] * d;
                                 }
                             }
                         }
@@ -665,7 +632,7 @@ grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(&tempty[acc]);
-            if (++acc == Cfg::n_acc) {
+            if (++acc == 2) {
                 acc = 0;
                 acc_phase ^= 1u;
             }
@@ -750,7 +717,6 @@ struct GroupedArgs {
     float *y;
     int sm_count, smem_optin;
     bool pdl;  // launch as programmatic dependents
-    int mh;    // 128-row halves per GEMM tile: 1 or 2
 };
 
 inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -823,16 +789,10 @@ inline ep_status grouped_set_attributes(int smem_optin) {
     if (cudaFuncSetAttribute(group_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem_optin) != cudaSuccess)
         return EP_ECUDA;
-    if (cudaFuncSetAttribute(grouped_gemm_kernel<true, 1>,
+    if (cudaFuncSetAttribute(grouped_gemm_kernel<true>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem_optin) != cudaSuccess ||
-        cudaFuncSetAttribute(grouped_gemm_kernel<false, 1>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem_optin) != cudaSuccess ||
-        cudaFuncSetAttribute(grouped_gemm_kernel<true, 2>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem_optin) != cudaSuccess ||
-        cudaFuncSetAttribute(grouped_gemm_kernel<false, 2>,
+        cudaFuncSetAttribute(grouped_gemm_kernel<false>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem_optin) != cudaSuccess)
         return EP_ECUDA;
@@ -870,7 +830,7 @@ inline ep_status grouped_forward(const GroupedArgs &g, const GroupedWorkspace &W
     const int k = g.top_k;
     const int64_t P = T * k;
     const int G = (int)E + (I_s > 0 ? 1 : 0);
-    const uint32_t gemm_smem = g.mh == 2 ? GemmSmem<2>::alloc : GemmSmem<1>::alloc;
+    const uint32_t gemm_smem = GemmSmem::alloc;
     if (gemm_smem > (uint32_t)g.smem_optin || plan_smem_bytes(E) > (size_t)g.smem_optin) {
         snprintf(why, why_len, "not enough shared memory per block for the tensor path");
         return EP_EINVAL;
@@ -892,7 +852,7 @@ inline ep_status grouped_forward(const GroupedArgs &g, const GroupedWorkspace &W
     // 1. plan
     PlanArgs pa;
     pa.ids = g.ids; pa.T = T; pa.P = P; pa.top_k = k; pa.E = (int)E; pa.H = (int)H;
-    pa.I = (int)I; pa.I_s = (int)I_s; pa.mh = g.mh;
+    pa.I = (int)I; pa.I_s = (int)I_s;
     pa.group_offset = group_offset; pa.perm_pair = perm_pair;
     pa.units_gu = units_gu; pa.units_dn = units_dn;
     bracket_event(ev, n_ev, 0, st);
@@ -941,11 +901,8 @@ inline ep_status grouped_forward(const GroupedArgs &g, const GroupedWorkspace &W
     gp.h_out = h_perm; gp.h_shared_out = h_shared; gp.I = (int)I; gp.I_s = (int)I_s;
     gp.c_out = c; gp.s_out = s; gp.H = (int)H;
     bracket_event(ev, n_ev, 4, st);
-    const cudaError_t e_gu =
-        g.mh == 2 ? grouped_launch(g.pdl, grouped_gemm_kernel<true, 2>, dim3(g.sm_count),
-                                   dim3(kGemmThreads), gemm_smem, st, gm, gp)
-                  : grouped_launch(g.pdl, grouped_gemm_kernel<true, 1>, dim3(g.sm_count),
-                                   dim3(kGemmThreads), gemm_smem, st, gm, gp);
+    const cudaError_t e_gu = grouped_launch(g.pdl, grouped_gemm_kernel<true>, dim3(g.sm_count),
+                                            dim3(kGemmThreads), gemm_smem, st, gm, gp);
     bracket_event(ev, n_ev, 5, st);
     if (e_gu != cudaSuccess) {
         snprintf(why, why_len, "gate/up GEMM launch failed");
@@ -965,11 +922,8 @@ inline ep_status grouped_forward(const GroupedArgs &g, const GroupedWorkspace &W
     gp.m_routed = (int)H; gp.m_shared = (int)H; gp.k_routed = (int)I; gp.k_shared = (int)I_s;
     gp.units = units_dn;
     bracket_event(ev, n_ev, 6, st);
-    const cudaError_t e_dn =
-        g.mh == 2 ? grouped_launch(g.pdl, grouped_gemm_kernel<false, 2>, dim3(g.sm_count),
-                                   dim3(kGemmThreads), gemm_smem, st, gm, gp)
-                  : grouped_launch(g.pdl, grouped_gemm_kernel<false, 1>, dim3(g.sm_count),
-                                   dim3(kGemmThreads), gemm_smem, st, gm, gp);
+    const cudaError_t e_dn = grouped_launch(g.pdl, grouped_gemm_kernel<false>, dim3(g.sm_count),
+                                            dim3(kGemmThreads), gemm_smem, st, gm, gp);
     bracket_event(ev, n_ev, 7, st);
     if (e_dn != cudaSuccess) {
         snprintf(why, why_len, "down GEMM launch failed");

@@ -207,31 +207,36 @@ router_tc_kernel(const __grid_constant__ RcMaps maps, const uint16_t *__restrict
         }
     } else {
         // ---------------------------------- sums of squares from the stages
-        const int nt = (int)threadIdx.x - 64;  // 0 .. 191
+        // The stage's rows (the W tiles' rows, then the token rows) are 128
+        // bytes each and contiguous (the swizzle only permutes the chunks of
+        // a row), so a warp reads four rows at once, lane l taking chunk
+        // l % 8 of row l / 8: 512 contiguous bytes, free of bank conflicts.
+        // Row quad g (rows 4g .. 4g + 3) goes to norm warp g mod 6; a lane
+        // keeps one partial sum per quad it reads, and the eight lanes of a
+        // row add theirs at the end.
+        constexpr int kMaxQuads = (2 * kGemmBM + kRcNT) / 4 / kRcNormWarps + 1;  // 14
+        const int nw = warp - 2;  // 0 .. 5
         const int rows = MT * kGemmBM + kRcNT;
-        float2 sq[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        const int quads = rows / 4;
+        float2 sq[kMaxQuads];
+#pragma unroll
+        for (int i = 0; i < kMaxQuads; ++i)
+            sq[i] = make_float2(0.f, 0.f);
         uint32_t stage = 0, phase = 0;
         for (int kb = kb_lo; kb < kb_hi; ++kb) {
             if (!mbar_wait(&full[stage], phase, abort_flag))
                 break;
-            const uint8_t *sa = smem + stage * L.stage_bytes;
+            const uint4 *sa = reinterpret_cast<const uint4 *>(smem + stage * L.stage_bytes);
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const int r = nt + i * (kRcThreads - 64);
-                if (r < rows) {
-                    // row r of the stage: W rows of tile r / 128, then x rows
-                    const uint4 *row = reinterpret_cast<const uint4 *>(
-                        sa + (r < MT * kGemmBM ? (r / kGemmBM) * kRcWBox + (r % kGemmBM) * 128
-                                               : MT * kRcWBox + (r - MT * kGemmBM) * 128));
+            for (int i = 0; i < kMaxQuads; ++i) {
+                const int g = nw + kRcNormWarps * i;
+                if (g < quads) {
+                    const uint4 v = sa[g * 32 + lane];  // rows 4g.., 16-byte chunk lane
+                    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const uint4 v = row[c];
-                        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                        for (int h = 0; h < 4; ++h) {
-                            const float2 f = bf16x2_to_f2(w4[h]);
-                            sq[i] = ffma2(f, f, sq[i]);
-                        }
+                    for (int h = 0; h < 4; ++h) {
+                        const float2 f = bf16x2_to_f2(w4[h]);
+                        sq[i] = ffma2(f, f, sq[i]);
                     }
                 }
             }
@@ -266,14 +271,22 @@ router_tc_kernel(const __grid_constant__ RcMaps maps, const uint16_t *__restrict
                 }
             }
         }
+        // a row's eight chunks sit in lanes 8 (l / 8) .. 8 (l / 8) + 7
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const int r = nt + i * (kRcThreads - 64);
-            if (r < MT * kGemmBM) {
-                if (r < E)
-                    wsq[r] = sq[i].x + sq[i].y;
-            } else if (r < rows) {
-                xsq[r - MT * kGemmBM] = sq[i].x + sq[i].y;
+        for (int i = 0; i < kMaxQuads; ++i) {
+            float v = sq[i].x + sq[i].y;
+            v += __shfl_xor_sync(0xffffffffu, v, 1);
+            v += __shfl_xor_sync(0xffffffffu, v, 2);
+            v += __shfl_xor_sync(0xffffffffu, v, 4);
+            const int g = nw + kRcNormWarps * i;
+            const int r = 4 * g + (lane >> 3);
+            if (g < quads && (lane & 7) == 0) {
+                if (r < MT * kGemmBM) {
+                    if (r < E)
+                        wsq[r] = v;
+                } else {
+                    xsq[r - MT * kGemmBM] = v;
+                }
             }
         }
     }

@@ -262,6 +262,53 @@ ep_status moe_ffn_forward_noalloc(const void *x, ep_dtype x_dtype, int64_t T, in
                                   int64_t I_s, const ep_plan_t *plan, float *y, void *stream);
 
 /*
+ * NVFP4 expert weights (TensorFold #593, "Checkpoint formats on that
+ * family": NVIDIA's NVFP4 checkpoint used as stored, 4-bit weights against
+ * 16-bit activations).  The page names the format only; this library takes
+ * NVIDIA's public definition: FP4 E2M1 elements (magnitudes 0, 0.5, 1, 1.5,
+ * 2, 3, 4, 6), one FP8 E4M3 block scale per 16 consecutive elements of a row
+ * along the reduction dimension, one fp32 scale per tensor; a weight is
+ * tensor_scale x block scale x element.
+ *   codes   device, [mats][rows][cols / 2] bytes, 16-byte aligned: element
+ *           2i of a row in the low nibble of byte i, 2i + 1 in the high one
+ *   scales  device, [mats][rows][cols / 16] bytes (E4M3), 4-byte aligned
+ * mats = E for the routed experts, 1 for the shared expert.
+ */
+typedef struct {
+    const void *codes;
+    const void *scales;
+    float tensor_scale;
+} ep_nvfp4_t;
+
+/*
+ * moe_ffn_nvfp4_workspace_size -- device workspace moe_ffn_forward_nvfp4
+ * needs (0 when T = 0).
+ *
+ * moe_ffn_forward_nvfp4 -- moe_ffn_forward for decode batches (1 <= T <= 8)
+ * with every expert matrix (routed and shared) in NVFP4: W_gate, W_up
+ * [E][I][H], W_down [E][H][I]; Ws_gate, Ws_up [I_s][H], Ws_down [H][I_s].
+ * Same operation, same fold order (ascending (expert id, j), then the
+ * shared expert), bit-identical for every plan and from run to run.  The
+ * weights stream as stored (4.5 bits each) and are dequantised on chip to
+ * fp16 (exact); the products run on the tensor cores with fp16 operands and
+ * fp32 accumulation: x is rounded to fp16 (exact for bf16 values of
+ * magnitude 2^-14 .. 65504) and h passes between the projections as an fp16
+ * hi/lo pair (about 22 significant bits).  The tensor scale multiplies the
+ * fp32 accumulator.  x must be bf16 (EP_EINVAL otherwise).
+ * Limits: 1 <= T <= 8 (0 is a no-op); H, I and I_s (when not 0) multiples of
+ * 64 in [64, 16384]; 1 <= E <= 1024; 1 <= top_k <= min(E, 16).  Errors and
+ * the other arguments as moe_ffn_forward.
+ */
+size_t moe_ffn_nvfp4_workspace_size(int64_t T, int64_t H, int64_t E, int32_t top_k, int64_t I,
+                                    int64_t I_s);
+ep_status moe_ffn_forward_nvfp4(const void *x, int64_t T, int64_t H, const int32_t *ids,
+                                const float *weights, int32_t top_k, const ep_nvfp4_t *w_gate,
+                                const ep_nvfp4_t *w_up, const ep_nvfp4_t *w_down, int64_t E,
+                                int64_t I, const ep_nvfp4_t *ws_gate, const ep_nvfp4_t *ws_up,
+                                const ep_nvfp4_t *ws_down, int64_t I_s, const ep_plan_t *plan,
+                                float *y, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * EP_ID_NONE -- an empty pick slot.  A pick whose id is EP_ID_NONE is skipped
  * by every call that takes ids and is not reported as a bad id (any other id
  * outside [0, E) is skipped and reported).
@@ -315,8 +362,7 @@ ep_status moe_ep_combine(const float *partials, int64_t T, int64_t H, const int3
  * Which moe_ffn_forward path runs.  EP_DISPATCH_AUTO (the default) takes the
  * weight-streaming path for T <= 8 when its on-chip buffers fit, else the
  * tensor-core path; inside the streaming path, the tensor-core kernels from
- * 2 tokens with bf16 x, the CUDA-core kernels otherwise; on the tensor path,
- * GEMM tiles of 128 weight rows.  Forcing a path that does not fit the sizes makes
+ * 2 tokens with bf16 x, the CUDA-core kernels otherwise.  Forcing a path that does not fit the sizes makes
  * moe_ffn_forward return EP_EINVAL.  Process-wide; meant for tests and tuning.
  */
 typedef enum {
@@ -328,13 +374,7 @@ typedef enum {
     EP_DISPATCH_STREAMING_TC = 3,
     /* streaming path, gate/up on the CUDA cores and down with the fold (two
        launches) */
-    EP_DISPATCH_STREAMING_SIMT = 4,
-    /* tensor path with GEMM tiles of 128 weight rows (two accumulators, the
-       epilogue of one tile beside the MMAs of the next) */
-    EP_DISPATCH_TENSOR_M128 = 5,
-    /* tensor path with GEMM tiles of 256 weight rows (two 128-row halves on
-       one activation tile, one accumulator) */
-    EP_DISPATCH_TENSOR_M256 = 6
+    EP_DISPATCH_STREAMING_SIMT = 4
 } ep_dispatch;
 ep_status ep_set_dispatch(ep_dispatch mode);
 

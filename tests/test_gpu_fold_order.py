@@ -33,7 +33,7 @@ from gpu_parity import device_inputs, oracle_route, shared_of
 
 pytestmark = pytest.mark.gpu
 
-PATHS = ["streaming_simt", "streaming_tc", "tensor_m128", "tensor_m256"]
+PATHS = ["streaming_simt", "streaming_tc", "tensor"]
 
 
 @pytest.fixture(autouse=True)
@@ -186,12 +186,9 @@ def _workspace_fold(x, ids, w, W, plan, path):
 
 @pytest.mark.parametrize("name,T,path", [("decode", 4, "streaming_tc"),
                                          ("decode", 8, "streaming_tc"),
-                                         ("decode", 8, "tensor_m128"),
-                                         ("decode", 8, "tensor_m256"),
-                                         ("prefill", 512, "tensor_m128"),
-                                         ("prefill", 512, "tensor_m256"),
-                                         ("imbalanced", 2048, "tensor_m128"),
-                                         ("imbalanced", 2048, "tensor_m256")])
+                                         ("decode", 8, "tensor"),
+                                         ("prefill", 512, "tensor"),
+                                         ("imbalanced", 2048, "tensor")])
 def test_y_is_the_host_fold_of_the_dumped_contributions(oracle_lib, name, T, path):
     wl = workloads.WORKLOADS[name]
     W, x = device_inputs(wl, T, batch=4)

@@ -15,12 +15,10 @@ pytestmark = pytest.mark.gpu
 WL = workloads.WORKLOADS
 
 
-# Every test runs with GEMM tiles of 128 weight rows (two accumulators) and of
-# 256 (two 128-row halves on one activation tile, one accumulator).
-@pytest.fixture(autouse=True, params=["tensor_m128", "tensor_m256"])
-def tensor_dispatch(request):
-    ed.ep_set_dispatch(request.param)
-    yield request.param
+@pytest.fixture(autouse=True)
+def tensor_dispatch():
+    ed.ep_set_dispatch("tensor")
+    yield "tensor"
     ed.ep_set_dispatch("auto")
 
 
