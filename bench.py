@@ -715,6 +715,141 @@ def measure(args, wl, device, rank, dist, peaks, K, warmup, sampler=None, with_g
     return out
 
 
+def nvfp4_cost(wl, T, n_distinct):
+    """Algorithmic bytes of one NVFP4 decode call: the picked experts' and the
+    shared expert's codes (half a byte per weight) and block scales (one byte
+    per 16 weights) read once, the activations and h at their stored widths
+    (fp16 hi/lo for h), the contributions and y in fp32.  Returns the gate/up
+    kernel's bytes and the call's (router included)."""
+    H, I, I_s, k = wl.H, wl.I, wl.I_s, wl.top_k
+    per_w = 0.5 + 1.0 / 16
+    w_gu = (n_distinct * 2 * H * I + 2 * H * I_s) * per_w
+    w_dn = (n_distinct * H * I + H * I_s) * per_w
+    P = T * k
+    h_bytes = (P * I + T * I_s) * 2 * 2
+    gu_bytes = w_gu + T * H * 2 + h_bytes
+    call_bytes = (wl.E * H * 2 + T * H * 2 + T * k * 8) + w_gu + w_dn + T * H * 4
+    return gu_bytes, call_bytes
+
+
+def measure_nvfp4(args, wl, device, peaks, K, warmup):
+    """The decode workload with every expert matrix in NVFP4 (moe_ffn_forward_nvfp4
+    after the same bf16 router): tokens/s over the row counts, per-call and
+    per-kernel times, and the gate/up kernel's roofline at the stored bytes."""
+    import expert_decode_b200 as ed
+    seed = workloads.SEED_BASE
+    mats = [workloads.make_nvfp4_experts(wl.E, rows, cols, seed + 11 + j, device=device)
+            for j, (rows, cols) in enumerate(((wl.I, wl.H), (wl.I, wl.H), (wl.H, wl.I)))]
+    shared = tuple({"packed": m["packed"][0], "scales": m["scales"][0],
+                    "tensor_scale": m["tensor_scale"]}
+                   for m in (workloads.make_nvfp4_experts(1, rows, cols, seed + 14 + j, device)
+                             for j, (rows, cols) in enumerate(((wl.I_s, wl.H), (wl.I_s, wl.H),
+                                                               (wl.H, wl.I_s)))))
+    w_router, bias = workloads.make_router(wl, device)
+    plan = ed.ep_plan(wl.E, wl.bands[0])
+    Ts = wl.T
+    xs = {T: [workloads.make_x(wl, T, device=device, seed=seed, batch=b + 100 * T)
+              for b in range(N_BATCHES)] for T in Ts}
+    ids = {T: torch.empty((T, wl.top_k), dtype=torch.int32, device=device) for T in Ts}
+    wts = {T: torch.empty((T, wl.top_k), dtype=torch.float32, device=device) for T in Ts}
+    ys = {T: torch.empty((T, wl.H), dtype=torch.float32, device=device) for T in Ts}
+    ws = torch.empty(max(ed.moe_ffn_nvfp4_workspace_size(T, wl.H, wl.E, wl.top_k, wl.I, wl.I_s)
+                         for T in Ts), dtype=torch.uint8, device=device)
+    flush = torch.empty(args.flush_mib << 20, dtype=torch.uint8, device=device)
+    launches = [0]
+
+    def call(T, i, prof=None):
+        x = xs[T][i % N_BATCHES]
+        if prof is not None:
+            ed.ep_profile_events(prof[("route", T)])
+        ed.moe_route(x, w_router, bias, wl.top_k, ids=ids[T], weights=wts[T])
+        launches[0] += ed.ep_last_launch_count()
+        if prof is not None:
+            ed.ep_profile_events(prof[T])
+        ed.moe_ffn_forward_nvfp4(x, ids[T], wts[T], *mats, shared, plan, y=ys[T], workspace=ws)
+        launches[0] += ed.ep_last_launch_count()
+        if prof is not None:
+            ed.ep_profile_events(None)
+
+    for i in range(warmup):
+        flush.zero_()
+        for T in Ts:
+            call(T, i)
+    torch.cuda.synchronize()
+    ed.ep_check_status()
+    distinct = {}
+    for T in Ts:
+        for b in range(N_BATCHES):
+            call(T, b)
+            torch.cuda.synchronize()
+            distinct[(T, b)] = int(torch.unique(ids[T]).numel())
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    call_s = {T: [torch.cuda.Event(enable_timing=True) for _ in range(K)] for T in Ts}
+    call_e = {T: [torch.cuda.Event(enable_timing=True) for _ in range(K)] for T in Ts}
+    launches[0] = 0
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.zero_()
+        ev_s[i].record()
+        for T in Ts:
+            call_s[T][i].record()
+            call(T, warmup + i)
+            call_e[T][i].record()
+        ev_e[i].record()
+    torch.cuda.synchronize()
+    ed.ep_check_status()
+    n_launch = launches[0]
+    nk = 4
+    prof = [{key: [torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)]
+             for key in list(Ts) + [("route", T) for T in Ts]} for _ in range(K)]
+    for p in prof:
+        for evs in p.values():
+            for e in evs:
+                e.record()
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.zero_()
+        for T in Ts:
+            call(T, warmup + i, prof[i])
+    torch.cuda.synchronize()
+    dev_s = sum(ev_s[i].elapsed_time(ev_e[i]) for i in range(K)) / 1e3
+    per_T = {}
+    gu_b = gu_s = 0.0
+    for T in Ts:
+        names = ["to_f16", "gate_up", "down", "combine"]
+        kus = {nm: 1e3 * sum(prof[i][T][2 * j].elapsed_time(prof[i][T][2 * j + 1])
+                             for i in range(K)) / K for j, nm in enumerate(names)}
+        kus["router"] = 1e3 * sum(prof[i][("route", T)][0].elapsed_time(prof[i][("route", T)][1])
+                                  for i in range(K)) / K
+        costs = [nvfp4_cost(wl, T, distinct[(T, (warmup + i) % N_BATCHES)]) for i in range(K)]
+        call_sec = sum(call_s[T][i].elapsed_time(call_e[T][i]) for i in range(K)) / 1e3
+        cb = sum(c[1] for c in costs)
+        gb = sum(c[0] for c in costs)
+        gs = sum(prof[i][T][2].elapsed_time(prof[i][T][3]) for i in range(K)) / 1e3
+        gu_b += gb
+        gu_s += gs
+        per_T[f"T={T}"] = {"call_us": 1e6 * call_sec / K, "call_bytes": cb / K,
+                           "call_hbm_GBps": cb / call_sec / 1e9,
+                           "call_hbm_frac": cb / call_sec / 1e9 / peaks["hbm_gbs"],
+                           "gate_up_GBps": gb / gs / 1e9,
+                           "kernels_us": {k: round(v, 2) for k, v in kus.items()}}
+    achieved = gu_b / gu_s / 1e9
+    roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "kernel": "stream_gate_up_fp4_kernel",
+            "traffic": traffic_for("stream_gate_up_fp4_kernel", "decode_nvfp4"),
+            "peak_source": "measured" if peaks.get("_source") == "measured" else "fallback",
+            "bytes": "codes 0.5 B + block scales 1/16 B per weight, x fp16, h fp16 hi/lo"}
+    out = {"workload": wl.description + ", every expert matrix NVFP4 (E2M1 codes, E4M3 "
+                                        "scales per 16, fp32 tensor scale)",
+           "value": K * sum(Ts) / dev_s, "unit": "tokens/s", "ms_per_step": 1e3 * dev_s / K,
+           "steps": K, "warmup": warmup, "gpu_launches": n_launch, "roofline": roof,
+           "per_T": per_T}
+    del mats, shared, flush, ws
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, wl):
     import expert_decode_b200 as ed  # the library must load
     ed.ep_set_dispatch(args.dispatch)
@@ -758,6 +893,11 @@ def run_ours(args, wl):
             "step_tensor_peak_key": r["step_tensor_peak_key"],
             "step_roofline_frac": r["step_roofline_frac"], "roofline": r["roofline"],
             "kernels_us": per["kernels_us"], "call_us": per["call_us"], "clocks": r["clocks"]}
+
+    if wl.name == "decode" and args.detail != "none":
+        KD = max(1, min(args.detail_steps, K))
+        configs["decode_nvfp4"] = measure_nvfp4(args, wl, device, peaks, KD,
+                                                max(3, min(args.warmup, 10)))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

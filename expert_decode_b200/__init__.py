@@ -11,6 +11,7 @@ from .api import (  # noqa: F401
     moe_ffn_workspace_size, moe_ffn_workspace_layout,
     moe_ffn_forward,
     moe_ffn_forward_noalloc,
+    NvFp4, moe_ffn_nvfp4_workspace_size, moe_ffn_forward_nvfp4,
     ep_check_status, ep_set_dispatch, ep_set_router, ep_last_launch_count, ep_profile_events, library,
     library_path,
 )

@@ -35,6 +35,12 @@ class WorkspaceLayout(ctypes.Structure):
                 ("perm_offset", ctypes.c_size_t)]
 
 
+class NvFp4(ctypes.Structure):
+    """ep_nvfp4_t: codes and block scales on the device, one fp32 tensor scale."""
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("tensor_scale", ctypes.c_float)]
+
+
 class Plan(ctypes.Structure):
     _fields_ = [("num_experts", ctypes.c_int32), ("bands", ctypes.c_int32),
                 ("band_start", ctypes.c_int32 * (EP_MAX_BANDS + 1))]
@@ -70,6 +76,12 @@ def library():
             lib.moe_ffn_forward_noalloc.argtypes = [P, ctypes.c_int, I64, I64, P, P, I32, P, P,
                                                     P, I64, I64, P, P, P, I64,
                                                     ctypes.POINTER(Plan), P, P]
+            F4 = ctypes.POINTER(NvFp4)
+            lib.moe_ffn_nvfp4_workspace_size.argtypes = [I64, I64, I64, I32, I64, I64]
+            lib.moe_ffn_nvfp4_workspace_size.restype = SZ
+            lib.moe_ffn_forward_nvfp4.argtypes = [P, I64, I64, P, P, I32, F4, F4, F4, I64, I64,
+                                                  F4, F4, F4, I64, ctypes.POINTER(Plan), P, P,
+                                                  SZ, P]
             lib.ep_set_dispatch.argtypes = [ctypes.c_int]
             lib.ep_set_router.argtypes = [ctypes.c_int]
             lib.ep_check_status.argtypes = [P]
@@ -80,7 +92,7 @@ def library():
             for fn in ("ep_plan", "moe_route", "moe_route_logits", "moe_route_sigmoid",
                        "moe_ffn_forward",
                        "moe_ffn_workspace_layout",
-                       "moe_ffn_forward_noalloc",
+                       "moe_ffn_forward_noalloc", "moe_ffn_forward_nvfp4",
                        "ep_set_dispatch", "ep_set_router", "ep_check_status"):
                 getattr(lib, fn).restype = ctypes.c_int
             _lib = lib
@@ -252,6 +264,60 @@ def moe_ffn_forward_noalloc(x, ids, weights, w_gate, w_up, w_down, shared, plan,
         _ptr(x), _dtype(x), T, H, _ptr(ids), _ptr(weights), ids.shape[1], _ptr(w_gate),
         _ptr(w_up), _ptr(w_down), E, I, _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), I_s,
         ctypes.byref(plan), _ptr(y), _stream(stream)))
+    return y
+
+
+def _nvfp4(m, name, mats, rows, cols):
+    """m = {"packed": uint8 [mats,] rows, cols / 2; "scales": uint8 [mats,]
+    rows, cols / 16; "tensor_scale": float} -> NvFp4 (keeps no reference)."""
+    packed, scales = m["packed"], m["scales"]
+    lead = (mats,) if mats is not None else ()
+    for what, t, shape in (("packed", packed, lead + (rows, cols // 2)),
+                           ("scales", scales, lead + (rows, cols // 16))):
+        _dense(t, f"{name}.{what}", torch.uint8)
+        if tuple(t.shape) != shape:
+            raise ValueError(f"{name}.{what} must be {shape}, got {tuple(t.shape)}")
+    return NvFp4(packed.data_ptr(), scales.data_ptr(), float(m["tensor_scale"]))
+
+
+def moe_ffn_nvfp4_workspace_size(T, H, E, top_k, I, I_s):
+    return int(library().moe_ffn_nvfp4_workspace_size(int(T), int(H), int(E), int(top_k),
+                                                      int(I), int(I_s)))
+
+
+def moe_ffn_forward_nvfp4(x, ids, weights, w_gate, w_up, w_down, shared, plan, y=None,
+                          workspace=None, stream=None):
+    """y [T, H] fp32 of the routed MoE FFN for a decode batch (T <= 8) with
+    NVFP4 experts.  w_gate, w_up: {"packed" [E, I, H/2], "scales" [E, I, H/16],
+    "tensor_scale"}; w_down: [E, H, I/2], [E, H, I/16]; shared = (ws_gate,
+    ws_up, ws_down) of the same form without the expert dimension, or None."""
+    _dense(x, "x", torch.bfloat16, 2)
+    _dense(ids, "ids", torch.int32, 2)
+    _dense(weights, "weights", torch.float32, 2)
+    T, H = x.shape
+    top_k = ids.shape[1]
+    E, I = w_gate["packed"].shape[0], w_gate["packed"].shape[1]
+    g, u, d = (_nvfp4(w_gate, "w_gate", E, I, H), _nvfp4(w_up, "w_up", E, I, H),
+               _nvfp4(w_down, "w_down", E, H, I))
+    if shared is not None:
+        I_s = shared[0]["packed"].shape[0]
+        sg, su, sd = (_nvfp4(shared[0], "ws_gate", None, I_s, H),
+                      _nvfp4(shared[1], "ws_up", None, I_s, H),
+                      _nvfp4(shared[2], "ws_down", None, H, I_s))
+        sp = [ctypes.byref(sg), ctypes.byref(su), ctypes.byref(sd)]
+    else:
+        I_s = 0
+        sp = [None, None, None]
+    if y is None:
+        y = torch.empty((T, H), dtype=torch.float32, device=x.device)
+    _dense(y, "y", torch.float32, 2)
+    need = moe_ffn_nvfp4_workspace_size(T, H, E, top_k, I, I_s)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    _check(library().moe_ffn_forward_nvfp4(
+        _ptr(x), T, H, _ptr(ids), _ptr(weights), top_k, ctypes.byref(g), ctypes.byref(u),
+        ctypes.byref(d), E, I, *sp, I_s, ctypes.byref(plan), _ptr(y), _ptr(workspace),
+        workspace.numel(), _stream(stream)))
     return y
 
 

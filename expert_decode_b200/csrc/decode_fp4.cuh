@@ -10,21 +10,26 @@
 //
 // Streaming the weights as stored cuts the bytes a decode call reads to
 // 4.5 bits per weight.  The two kernels are those of decode_tc.cuh with a
-// dequantising stage between the copy and the MMA:
+// dequantising step between the copy and the MMA:
 //
-//   warp 0     TMA: per 64-wide k block the raw codes of the tile's 128 rows
-//              (32 bytes each) and the 16-bit activation (or h) tile;
-//   warps 6-9  dequantise: thread r takes row r's 64 codes (cvt of E2M1
-//              pairs to fp16 pairs, exact), multiplies them by the row's four
-//              block scales (E4M3 to fp16, exact: every product has at most 6
-//              significant bits and lies in fp16's normal range) and writes
-//              the row into the stage's fp16 A tile in the 128-byte swizzled
-//              K-major layout the MMA reads;
-//   warp 1     tcgen05.mma kind::f16 with fp16 A and B, fp32 accumulators in
-//              TMEM;
-//   warps 2-5  the epilogue of decode_tc.cuh, with the tensor scale applied
-//              to the fp32 accumulator first (an exact power of two for the
-//              usual per-tensor scales).
+//   warp 0      TMA: per 256-wide k stage the raw codes of the tile's 128
+//               rows (128 bytes each, 128-byte swizzled) and the stage's four
+//               16-bit activation (or h) boxes;
+//   warps 6-13  dequantise, 64-wide k block by k block, into a ring of fp16
+//               A tiles: thread (r, half) takes 32 codes of row r (cvt of
+//               E2M1 pairs to fp16 pairs, exact), multiplies them by their
+//               two block scales (E4M3 to fp16, exact: every product has at
+//               most 6 significant bits and lies in fp16's range) and writes
+//               them in the 128-byte swizzled K-major layout the MMA reads;
+//   warp 1      tcgen05.mma kind::f16 with fp16 A and B, fp32 accumulators in
+//               TMEM, one A tile of the ring per k block;
+//   warps 2-5   the epilogue of decode_tc.cuh, with the tensor scale applied
+//               to the fp32 accumulator first.
+//
+// At 4.5 bits per weight a stage of 64-wide k blocks holds too few bytes to
+// keep HBM busy: the 256-wide stage puts 16 KB of codes per stage and 96 KB
+// per SM in flight, in 128-byte rows, while the 16 KB A tiles cycle through
+// a ring of their own.
 //
 // The activations enter as fp16: x is converted once per call (exact for
 // bf16 values of magnitude 2^-14 .. 65504, which covers activations in
@@ -41,15 +46,22 @@
 
 namespace epk {
 
-constexpr int kF4Stages = 8;
-constexpr int kF4Threads = 320;                           // warps 0..9
-constexpr uint32_t kF4ABytes = kGemmBM * kGemmBK * 2;    // dequantised fp16 A, 16 KB
-constexpr uint32_t kF4CodeBytes = kGemmBM * kGemmBK / 2; // 128 rows x 32 code bytes, 4 KB
-constexpr uint32_t kF4BBytes = kTcN * kGemmBK * 2;       // 16 fp16 rows, 2 KB
-constexpr uint32_t kF4CodeOff = kF4ABytes;
-constexpr uint32_t kF4BOff = kF4ABytes + kF4CodeBytes;   // 20 KB, 1024-aligned
-constexpr uint32_t kF4StageBytes = kF4ABytes + kF4CodeBytes + kF4BBytes;  // 22 KB
-constexpr int kF4DeqWarp0 = 6;
+constexpr int kF4KS = 256;                               // k extent of one stage
+constexpr int kF4Sub = kF4KS / kGemmBK;                  // 64-wide k blocks per stage
+constexpr int kF4Stages = 6;
+constexpr int kF4ASlots = 4;
+constexpr int kF4Threads = 448;                          // warps 0..13
+constexpr uint32_t kF4CodeBytes = kGemmBM * kF4KS / 2;   // 128 rows x 128 code bytes, 16 KB
+constexpr uint32_t kF4BBox = kTcN * kGemmBK * 2;         // 16 fp16 rows x 64, 2 KB
+constexpr uint32_t kF4BOff = kF4CodeBytes;               // four B boxes after the codes
+constexpr uint32_t kF4StageBytes = kF4CodeBytes + kF4Sub * kF4BBox;   // 24 KB
+constexpr uint32_t kF4ABytes = kGemmBM * kGemmBK * 2;    // one fp16 A tile, 16 KB
+constexpr uint32_t kF4AOff = kF4Stages * kF4StageBytes;  // the A ring after the stages
+constexpr uint32_t kF4Bars = kF4AOff + kF4ASlots * kF4ABytes;
+// full[S], empty[S], afull[A], aempty[A], tfull[2], tempty[2], drain, planbar
+constexpr uint32_t kF4Misc = kF4Bars + (2 * kF4Stages + 2 * kF4ASlots + 6) * 8;
+constexpr int kF4DeqWarp0 = 6;                           // warps 6..13 dequantise
+constexpr int kF4DeqWarps = 8;
 
 // Instruction descriptor: fp16 A and B, fp32 D, both operands K-major.
 __host__ __device__ constexpr uint32_t idesc_f16_f32(uint32_t M, uint32_t N) {
@@ -90,32 +102,230 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Row r of a stage: its 64 codes (32 bytes at codes + 32 r) times its four
-// block scales (s4: the scale bytes of k block kb, scales 4 kb .. 4 kb + 3
-// of the row) into row r of the fp16 A tile, 128-byte swizzled: 16-byte
-// chunk j of the row at position j ^ (r mod 8).
-__device__ __forceinline__ void dequant_row(const uint8_t *codes, uint32_t s4, uint8_t *a_tile,
-                                            int r) {
-    const uint4 c0 = reinterpret_cast<const uint4 *>(codes + 32 * r)[0];
-    const uint4 c1 = reinterpret_cast<const uint4 *>(codes + 32 * r)[1];
-    const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-    const uint32_t s01 = e4m3x2_to_f16x2(s4 & 0xffffu), s23 = e4m3x2_to_f16x2(s4 >> 16);
+// k block `sub` of a stage, half h of row r: 32 codes (chunk 2 sub + h of
+// the row's 128 code bytes, which the copy stored 128-byte swizzled at
+// position (2 sub + h) ^ (r mod 8)) times their two block scales (bytes 2h,
+// 2h + 1 of s4, the row's four scale bytes of this k block) into row r of an
+// fp16 A tile, 128-byte swizzled: chunk j of the row (elements 8j .. 8j + 7)
+// at position j ^ (r mod 8).  Eight consecutive lanes take eight
+// consecutive rows with one h (dequant_row_of), so the eight 16-byte chunks
+// each of them reads or writes fall in eight distinct bank groups.
+__device__ __forceinline__ void dequant_half(const uint8_t *codes, int sub, uint32_t s4,
+                                             uint8_t *a_tile, int r, int h) {
+    const uint4 c =
+        reinterpret_cast<const uint4 *>(codes + 128 * r)[(2 * sub + h) ^ (r & 7)];
+    const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+    const uint32_t s2 = e4m3x2_to_f16x2(h ? (s4 >> 16) : (s4 & 0xffffu));
     // each block scale broadcast to both halves of an fp16 pair
-    const uint32_t sb[4] = {__byte_perm(s01, 0, 0x1010), __byte_perm(s01, 0, 0x3232),
-                            __byte_perm(s23, 0, 0x1010), __byte_perm(s23, 0, 0x3232)};
+    const uint32_t sb[2] = {__byte_perm(s2, 0, 0x1010), __byte_perm(s2, 0, 0x3232)};
     uint4 *row = reinterpret_cast<uint4 *>(a_tile + 128 * r);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {  // chunk j: elements 8 j .. 8 j + 7, code word j
-        const uint32_t w = cw[j];
-        const uint32_t s = sb[j >> 1];  // 16 elements per block: two chunks
+    for (int jj = 0; jj < 4; ++jj) {  // chunk 4h + jj: code word jj, block jj / 2
+        const uint32_t w = cw[jj];
+        const uint32_t sc = sb[jj >> 1];
         uint4 out;
-        out.x = hmul2_u32(e2m1x2_to_f16x2(w & 0xffu), s);
-        out.y = hmul2_u32(e2m1x2_to_f16x2((w >> 8) & 0xffu), s);
-        out.z = hmul2_u32(e2m1x2_to_f16x2((w >> 16) & 0xffu), s);
-        out.w = hmul2_u32(e2m1x2_to_f16x2(w >> 24), s);
-        row[j ^ (r & 7)] = out;
+        out.x = hmul2_u32(e2m1x2_to_f16x2(w & 0xffu), sc);
+        out.y = hmul2_u32(e2m1x2_to_f16x2((w >> 8) & 0xffu), sc);
+        out.z = hmul2_u32(e2m1x2_to_f16x2((w >> 16) & 0xffu), sc);
+        out.w = hmul2_u32(e2m1x2_to_f16x2(w >> 24), sc);
+        row[(4 * h + jj) ^ (r & 7)] = out;
     }
 }
+
+// The row and half a dequantiser thread takes (d = 0..255 over warps 6..13):
+// warp d / 32 owns rows 16 (d / 32) .. + 15; lanes 0-7 / 8-15 take rows 0-7
+// with h = 0 / 1, lanes 16-23 / 24-31 rows 8-15.
+__device__ __forceinline__ void dequant_row_of(int d, int &r, int &h) {
+    const int l = d & 31;
+    r = 16 * (d >> 5) + (l & 7) + 8 * (l >> 4);
+    h = (l >> 3) & 1;
+}
+
+// Scale rows past a matrix read this zero row instead.
+constexpr int kF4MaxKBlocks = 16384 / kGemmBK;  // reduction dims up to 16384
+__device__ const uint32_t kZeroScales[kF4MaxKBlocks] = {};
+
+// One stage as a dequantiser sees it: its k blocks' scale words (this
+// thread's row) and how many of its four k blocks exist.
+struct F4StageScales {
+    uint32_t s[kF4Sub];
+    int n_sub;
+};
+
+// The stages one dequantiser thread consumes, in order of (tile, stage).
+// row_of(u, p, kbn) gives tile u's scale row (left at the zero row past the
+// matrix) and its count of 64-wide k blocks; fetch() loads the next stage's
+// scale words (each index clamped into the row: no branch around a load).
+template <class RowOf>
+struct ScaleCursor {
+    int u, ks, kbn, total, step;
+    const uint32_t *p;
+    RowOf row_of;
+
+    __device__ __forceinline__ ScaleCursor(int u0, int total_, int step_, RowOf f)
+        : u(u0), ks(0), kbn(1), total(total_), step(step_), p(kZeroScales), row_of(f) {
+        if (u < total)
+            row_of(u, p, kbn);
+    }
+    __device__ __forceinline__ F4StageScales fetch() {
+        F4StageScales o;
+        const int kb0 = ks * kF4Sub;
+#pragma unroll
+        for (int i = 0; i < kF4Sub; ++i)
+            o.s[i] = __ldg(p + min(kb0 + i, kbn - 1));
+        o.n_sub = min(kF4Sub, kbn - kb0);
+        if (kb0 + kF4Sub >= kbn) {
+            ks = 0;
+            u += step;
+            p = kZeroScales;
+            kbn = 1;
+            if (u < total)
+                row_of(u, p, kbn);
+        } else {
+            ++ks;
+        }
+        return o;
+    }
+};
+
+// Stages of a tile whose reduction spans kbn 64-wide k blocks.
+__device__ __forceinline__ int f4_stages_of(int kbn) { return (kbn + kF4Sub - 1) / kF4Sub; }
+
+// The dequantisers' loop over the n_stages stages this CTA consumes: wait for
+// a stage's codes, then per k block wait for a free A tile, write this
+// thread's half-row and release the tile to the MMA.  Each stage's scales are
+// loaded kScaleAhead stages before their use; the loop is unrolled by that
+// distance so each stays in its registers from load to use.
+constexpr int kScaleAhead = 2;
+
+template <class RowOf>
+__device__ __forceinline__ void dequant_stages(uint8_t *smem, uint64_t *full, uint64_t *afull,
+                                               uint64_t *aempty, volatile int *abort_flag,
+                                               int n_stages, ScaleCursor<RowOf> &cur, int r,
+                                               int h, int lane) {
+    F4StageScales q[kScaleAhead];
+#pragma unroll
+    for (int j = 0; j < kScaleAhead; ++j)
+        q[j] = cur.fetch();
+    uint32_t stage = 0, phase = 0, slot = 0, aphase = 0;
+    for (int n0 = 0; n0 < n_stages; n0 += kScaleAhead) {
+#pragma unroll
+        for (int j = 0; j < kScaleAhead; ++j) {
+            if (n0 + j < n_stages) {
+                if (!mbar_wait(&full[stage], phase, abort_flag))
+                    return;
+                const uint8_t *codes = smem + stage * kF4StageBytes;
+#pragma unroll
+                for (int sub = 0; sub < kF4Sub; ++sub) {
+                    if (sub < q[j].n_sub) {
+                        if (!mbar_wait(&aempty[slot], aphase ^ 1u, abort_flag))
+                            return;
+                        dequant_half(codes, sub, q[j].s[sub], smem + kF4AOff + slot * kF4ABytes,
+                                     r, h);
+                        fence_proxy_async_smem();  // the MMA reads the tile through the async proxy
+                        __syncwarp();
+                        if (lane == 0)
+                            mbar_arrive(&afull[slot]);
+                        if (++slot == kF4ASlots) {
+                            slot = 0;
+                            aphase ^= 1u;
+                        }
+                    }
+                }
+                q[j] = cur.fetch();
+                if (++stage == kF4Stages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+    }
+}
+
+// The MMA issuer's loop, common to both kernels: per tile one accumulator
+// (of two in TMEM), per stage its k blocks, each from the next A tile of the
+// ring and the stage's B box of that k block.
+template <class KbnOf>
+__device__ __forceinline__ void f4_mma_loop(uint8_t *smem, uint64_t *full, uint64_t *empty,
+                                            uint64_t *afull, uint64_t *aempty, uint64_t *tfull,
+                                            uint64_t *tempty, volatile int *abort_flag,
+                                            uint32_t tmem_base, int total, KbnOf kbn_of) {
+    uint32_t stage = 0, phase = 0, slot = 0, aphase = 0;
+    uint32_t acc = 0, acc_phase = 0;
+    const uint32_t idesc = idesc_f16_f32(kGemmBM, kTcN);
+    for (int u = blockIdx.x; u < total; u += gridDim.x) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag))
+            return;
+        tc_fence_after_sync();
+        const uint32_t d_tmem = tmem_base + acc * kTcN;
+        const int kbn = kbn_of(u);
+        const int n_st = f4_stages_of(kbn);
+        for (int ks = 0; ks < n_st; ++ks) {
+            if (!mbar_wait(&full[stage], phase, abort_flag))
+                return;
+            const uint32_t b_base = smem_u32(smem + stage * kF4StageBytes + kF4BOff);
+            const int n_sub = min(kF4Sub, kbn - ks * kF4Sub);
+            for (int sub = 0; sub < n_sub; ++sub) {
+                if (!mbar_wait(&afull[slot], aphase, abort_flag))
+                    return;
+                tc_fence_after_sync();
+                const uint32_t a_addr = smem_u32(smem + kF4AOff + slot * kF4ABytes);
+                const uint32_t b_addr = b_base + sub * kF4BBox;
+#pragma unroll
+                for (int kk = 0; kk < kGemmBK / 16; ++kk)
+                    umma_bf16(d_tmem, smem_desc_sw128_kmajor(a_addr + kk * 32),
+                              smem_desc_sw128_kmajor(b_addr + kk * 32), idesc,
+                              (ks > 0 || sub > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(&aempty[slot]);
+                if (++slot == kF4ASlots) {
+                    slot = 0;
+                    aphase ^= 1u;
+                }
+            }
+            umma_commit(&empty[stage]);
+            if (++stage == kF4Stages) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+        umma_commit(&tfull[acc]);
+        if (++acc == 2) {
+            acc = 0;
+            acc_phase ^= 1u;
+        }
+    }
+}
+
+// Barrier set of both kernels, at kF4Bars.
+struct F4Bars {
+    uint64_t *full, *empty, *afull, *aempty, *tfull, *tempty, *drain, *planbar;
+    __device__ __forceinline__ explicit F4Bars(uint8_t *smem) {
+        full = reinterpret_cast<uint64_t *>(smem + kF4Bars);
+        empty = full + kF4Stages;
+        afull = empty + kF4Stages;
+        aempty = afull + kF4ASlots;
+        tfull = aempty + kF4ASlots;
+        tempty = tfull + 2;
+        drain = tempty + 2;
+        planbar = drain + 1;
+    }
+    __device__ __forceinline__ void init() const {
+        for (int s = 0; s < kF4Stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int s = 0; s < kF4ASlots; ++s) {
+            mbar_init(&afull[s], kF4DeqWarps);
+            mbar_init(&aempty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 4);
+        }
+        mbar_init(drain, 1);
+        mbar_init(planbar, 1);
+    }
+};
 
 // h as fp16 hi/lo: hi = fp16(h), lo = fp16(h - hi).
 __device__ __forceinline__ void store_hi_lo_f16(uint16_t *hi_p, uint16_t *lo_p, float h) {
@@ -125,10 +335,12 @@ __device__ __forceinline__ void store_hi_lo_f16(uint16_t *hi_p, uint16_t *lo_p, 
 }
 
 // ------------------------------------------------------------------ gate/up
+// Tiles as in decode_tc.cuh: 64 units of one expert's W_gate (A rows 0..63)
+// and the same units of W_up (rows 64..127) against the 16 token rows of x.
 struct F4GuMaps {
-    CUtensorMap cg, cu;  // routed W_gate / W_up codes [E, I, H/2] u8: box 32 x 64 x 1
-    CUtensorMap sg, su;  // shared codes [I_s, H/2] u8: box 32 x 64
-    CUtensorMap x;       // x fp16 [T, H]: box 64 x 16
+    CUtensorMap cg, cu;  // routed W_gate / W_up codes [E, I, H/2] u8: box 128 x 64 x 1, SW128
+    CUtensorMap sg, su;  // shared codes [I_s, H/2] u8: box 128 x 64, SW128
+    CUtensorMap x;       // x fp16 [T, H]: box 64 x 16, SW128
 };
 
 struct F4GuArgs {
@@ -141,9 +353,7 @@ struct F4GuArgs {
 };
 
 struct F4Smem {
-    static constexpr uint32_t bars = kF4Stages * kF4StageBytes;
-    // full[S], deq[S], empty[S], tfull[2], tempty[2], drain, planbar; holder, abort
-    static constexpr uint32_t misc = bars + (3 * kF4Stages + 6) * 8;
+    static constexpr uint32_t misc = kF4Misc;  // tmem holder, abort flag
     static constexpr uint32_t tile_first = misc + 16;
     static constexpr uint32_t row_first = tile_first + (kTcMaxGroups + 1) * 4;
     static constexpr uint32_t xchg = (row_first + kTcMaxGroups * 4 + 15) / 16 * 16;
@@ -157,13 +367,7 @@ stream_gate_up_fp4_kernel(const __grid_constant__ F4GuMaps maps, const F4GuArgs 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + F4Smem::bars);
-    uint64_t *deq = full + kF4Stages;
-    uint64_t *empty = deq + kF4Stages;
-    uint64_t *tfull = empty + kF4Stages;
-    uint64_t *tempty = tfull + 2;
-    uint64_t *drain = tempty + 2;
-    uint64_t *planbar = drain + 1;
+    const F4Bars B(smem);
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + F4Smem::misc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + F4Smem::misc + 8);
     int *tile_first = reinterpret_cast<int *>(smem + F4Smem::tile_first);
@@ -176,17 +380,7 @@ stream_gate_up_fp4_kernel(const __grid_constant__ F4GuMaps maps, const F4GuArgs 
     const int has_shared = a.I_s > 0 ? 1 : 0;
 
     if (warp == 0 && lane == 0) {
-        for (int s = 0; s < kF4Stages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&deq[s], 4);
-            mbar_init(&empty[s], 1);
-        }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 4);
-        }
-        mbar_init(drain, 1);
-        mbar_init(planbar, 1);
+        B.init();
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tensormap(&maps.cg);
@@ -216,6 +410,7 @@ stream_gate_up_fp4_kernel(const __grid_constant__ F4GuMaps maps, const F4GuArgs 
         m0 = (u - tile_first[gi]) * kGateUpRows;
     };
     const int kblocks = (a.H + kGemmBK - 1) / kGemmBK;
+    const int n_st = f4_stages_of(kblocks);
 
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer
@@ -225,31 +420,34 @@ stream_gate_up_fp4_kernel(const __grid_constant__ F4GuMaps maps, const F4GuArgs 
             grid_dependency_wait();  // x16 comes from the previous kernel
             uint32_t stage = 0, phase = 0;
             int issued = 0;
-            bool stop = !mbar_wait(planbar, 0, abort_flag);
+            bool stop = !mbar_wait(B.planbar, 0, abort_flag);
             const int total = stop ? 0 : tile_first[has_shared + P.n_groups];
             for (int u = blockIdx.x; u < total && !stop; u += gridDim.x) {
                 int gi, m0;
                 decode(u, gi, m0);
                 const bool shared = gi < has_shared;
                 const int e = shared ? 0 : (int)P.group_expert[gi - has_shared];
-                for (int kb = 0; kb < kblocks; ++kb) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+                for (int ks = 0; ks < n_st; ++ks) {
+                    if (!mbar_wait(&B.empty[stage], phase ^ 1u, abort_flag)) {
                         stop = true;
                         break;
                     }
                     uint8_t *st = smem + stage * kF4StageBytes;
-                    mbar_arrive_expect_tx(&full[stage], kF4CodeBytes + kF4BBytes);
-                    const int kc = kb * (kGemmBK / 2);  // byte column of the codes
+                    const int n_sub = min(kF4Sub, kblocks - ks * kF4Sub);
+                    mbar_arrive_expect_tx(&B.full[stage], kF4CodeBytes + n_sub * kF4BBox);
+                    const int kc = ks * (kF4KS / 2);  // byte column of the codes
                     // rows 0..63: W_gate codes of the tile's units, 64..127: W_up
-                    uint8_t *cg = st + kF4CodeOff, *cu = cg + kF4CodeBytes / 2;
+                    uint8_t *cg = st, *cu = st + kF4CodeBytes / 2;
                     if (shared) {
-                        tma_load_2d(cg, &maps.sg, kc, m0, &full[stage], pol_w);
-                        tma_load_2d(cu, &maps.su, kc, m0, &full[stage], pol_w);
+                        tma_load_2d(cg, &maps.sg, kc, m0, &B.full[stage], pol_w);
+                        tma_load_2d(cu, &maps.su, kc, m0, &B.full[stage], pol_w);
                     } else {
-                        tma_load_3d(cg, &maps.cg, kc, m0, e, &full[stage], pol_w);
-                        tma_load_3d(cu, &maps.cu, kc, m0, e, &full[stage], pol_w);
+                        tma_load_3d(cg, &maps.cg, kc, m0, e, &B.full[stage], pol_w);
+                        tma_load_3d(cu, &maps.cu, kc, m0, e, &B.full[stage], pol_w);
                     }
-                    tma_load_2d(st + kF4BOff, &maps.x, kb * kGemmBK, 0, &full[stage], pol_x);
+                    for (int sub = 0; sub < n_sub; ++sub)
+                        tma_load_2d(st + kF4BOff + sub * kF4BBox, &maps.x,
+                                    (ks * kF4Sub + sub) * kGemmBK, 0, &B.full[stage], pol_x);
                     ++issued;
                     if (++stage == kF4Stages) {
                         stage = 0;
@@ -258,88 +456,44 @@ stream_gate_up_fp4_kernel(const __grid_constant__ F4GuMaps maps, const F4GuArgs 
                 }
             }
             for (int n = issued > kF4Stages ? issued - kF4Stages : 0; n < issued; ++n)
-                mbar_wait(&full[n % kF4Stages], (uint32_t)(n / kF4Stages) & 1u, nullptr);
+                mbar_wait(&B.full[n % kF4Stages], (uint32_t)(n / kF4Stages) & 1u, nullptr);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer
         if (elect_one()) {
-            uint32_t stage = 0, phase = 0;
-            uint32_t acc = 0, acc_phase = 0;
-            bool stop = !mbar_wait(planbar, 0, abort_flag);
-            const int total = stop ? 0 : tile_first[has_shared + P.n_groups];
-            const uint32_t idesc = idesc_f16_f32(kGemmBM, kTcN);
-            for (int u = blockIdx.x; u < total && !stop; u += gridDim.x) {
-                if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag))
-                    break;
-                tc_fence_after_sync();
-                const uint32_t d_tmem = tmem_base + acc * kTcN;
-                for (int kb = 0; kb < kblocks; ++kb) {
-                    if (!mbar_wait(&deq[stage], phase, abort_flag)) {
-                        stop = true;
-                        break;
-                    }
-                    tc_fence_after_sync();
-                    const uint32_t a_addr = smem_u32(smem + stage * kF4StageBytes);
-                    const uint32_t b_addr = a_addr + kF4BOff;
-#pragma unroll
-                    for (int kk = 0; kk < kGemmBK / 16; ++kk)
-                        umma_bf16(d_tmem, smem_desc_sw128_kmajor(a_addr + kk * 32),
-                                  smem_desc_sw128_kmajor(b_addr + kk * 32), idesc,
-                                  (kb > 0 || kk > 0) ? 1u : 0u);
-                    umma_commit(&empty[stage]);
-                    if (++stage == kF4Stages) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
-                }
-                if (stop)
-                    break;
-                umma_commit(&tfull[acc]);
-                if (++acc == 2) {
-                    acc = 0;
-                    acc_phase ^= 1u;
-                }
-            }
-            umma_commit(drain);
-            mbar_wait(drain, 0, nullptr);
+            const bool planned = mbar_wait(B.planbar, 0, abort_flag);
+            const int total = planned ? tile_first[has_shared + P.n_groups] : 0;
+            f4_mma_loop(smem, B.full, B.empty, B.afull, B.aempty, B.tfull, B.tempty, abort_flag,
+                        tmem_base, total, [&](int) { return kblocks; });
+            umma_commit(B.drain);
+            mbar_wait(B.drain, 0, nullptr);
         }
     } else if (warp >= kF4DeqWarp0) {
         // ---------------------------------------------------- dequantisers
-        const int r = (int)threadIdx.x - 32 * kF4DeqWarp0;  // 0..127: row of the A tile
-        const bool planned = mbar_wait(planbar, 0, abort_flag);
+        int r, h;  // row of the A tile, half of it
+        dequant_row_of((int)threadIdx.x - 32 * kF4DeqWarp0, r, h);
+        const bool planned = mbar_wait(B.planbar, 0, abort_flag);
         const int total = planned ? tile_first[has_shared + P.n_groups] : 0;
-        uint32_t stage = 0, phase = 0;
-        bool stop = false;
-        for (int u = blockIdx.x; u < total && !stop; u += gridDim.x) {
+        // the row's unit and its scale row (zeros past the matrix)
+        auto row_of = [&](int u, const uint32_t *&p, int &kbn) {
             int gi, m0;
             decode(u, gi, m0);
             const bool shared = gi < has_shared;
             const int e = shared ? 0 : (int)P.group_expert[gi - has_shared];
-            // the row's unit and its scales row (zero past the matrix)
             const bool up = r >= kGateUpRows;
             const int unit = m0 + (r & (kGateUpRows - 1));
             const F4Mat &m = shared ? (up ? a.su : a.sg) : (up ? a.wu : a.wg);
-            const bool in = unit < m.rows;
-            const uint32_t *srow = reinterpret_cast<const uint32_t *>(
-                m.scales + ((size_t)e * m.rows + (in ? unit : 0)) * (size_t)(m.cols / 16));
-            for (int kb = 0; kb < kblocks; ++kb) {
-                if (!mbar_wait(&full[stage], phase, abort_flag)) {
-                    stop = true;
-                    break;
-                }
-                uint8_t *st = smem + stage * kF4StageBytes;
-                const uint32_t s4 = in ? __ldg(srow + kb) : 0u;
-                dequant_row(st + kF4CodeOff, s4, st, r);
-                fence_proxy_async_smem();  // the MMA reads the tile through the async proxy
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(&deq[stage]);
-                if (++stage == kF4Stages) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
-            }
-        }
+            if (unit < m.rows)
+                p = reinterpret_cast<const uint32_t *>(
+                    m.scales + ((size_t)e * m.rows + unit) * (size_t)(m.cols / 16));
+            kbn = kblocks;
+        };
+        const int mine = (int)blockIdx.x < total
+                             ? (total - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x
+                             : 0;
+        ScaleCursor<decltype(row_of)> cur((int)blockIdx.x, total, (int)gridDim.x, row_of);
+        dequant_stages(smem, B.full, B.afull, B.aempty, abort_flag, mine * n_st, cur, r, h,
+                       lane);
     } else {
         // ------------------------------------------------ plan, then epilogue
         const int ltid = (int)threadIdx.x - 64;
@@ -357,10 +511,10 @@ stream_gate_up_fp4_kernel(const __grid_constant__ F4GuMaps maps, const F4GuArgs 
             tile_first[G] = t;
             for (int g = 0; g < P.n_groups; ++g)
                 row_first[g] = 2 * P.group_first[g];
-            mbar_arrive(planbar);
+            mbar_arrive(B.planbar);
         }
         const bool planned =
-            named_count(kTcBarPlan, 128, mbar_wait(planbar, 0, abort_flag)) == 128;
+            named_count(kTcBarPlan, 128, mbar_wait(B.planbar, 0, abort_flag)) == 128;
         if (planned) {
             const int q = warp & 3;
             const bool gate_warp = q < 2;
@@ -371,7 +525,7 @@ stream_gate_up_fp4_kernel(const __grid_constant__ F4GuMaps maps, const F4GuArgs 
                 int gi, m0;
                 decode(u, gi, m0);
                 const bool shared = gi < has_shared;
-                const bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag);
+                const bool ok = mbar_wait(&B.tfull[acc], acc_phase, abort_flag);
                 if (named_count(kTcBarPair + pair, 64, ok) != 64)
                     break;
                 tc_fence_after_sync();
@@ -393,10 +547,10 @@ stream_gate_up_fp4_kernel(const __grid_constant__ F4GuMaps maps, const F4GuArgs 
 #pragma unroll
                     for (int t = 0; t < kStreamMaxT; ++t)
                         if (t < a.T && unit < a.I_s) {
-                            const float h =
+                            const float hv =
                                 silu_f32(ts * __uint_as_float(v[t])) * xb[t * 32 + lane];
                             store_hi_lo_f16(a.hb_shared + (size_t)t * a.I_s + unit,
-                                            a.hb_shared + (size_t)(a.T + t) * a.I_s + unit, h);
+                                            a.hb_shared + (size_t)(a.T + t) * a.I_s + unit, hv);
                         }
                 } else if (gate_warp) {
                     const int g = gi - has_shared;
@@ -404,25 +558,25 @@ stream_gate_up_fp4_kernel(const __grid_constant__ F4GuMaps maps, const F4GuArgs 
                     const int cnt = P.group_first[g + 1] - first;
                     for (int j = 0; j < cnt; ++j) {
                         const int tok = P.pair_token[first + j];
-                        float mine = 0.f;
+                        float mv = 0.f;
 #pragma unroll
                         for (int t = 0; t < kStreamMaxT; ++t)
-                            mine = t == tok ? __uint_as_float(v[t]) : mine;
+                            mv = t == tok ? __uint_as_float(v[t]) : mv;
                         if (unit < a.I) {
-                            const float h = silu_f32(ts * mine) * xb[tok * 32 + lane];
+                            const float hv = silu_f32(ts * mv) * xb[tok * 32 + lane];
                             const int j0 = j / kTcSlice * kTcSlice;
                             const int n = min(kTcSlice, cnt - j0);
                             const size_t b = (size_t)row_first[g] + 2 * j0;
                             uint16_t *hb = a.hb_routed + unit;
                             store_hi_lo_f16(hb + (b + (j - j0)) * a.I,
-                                            hb + (b + n + (j - j0)) * a.I, h);
+                                            hb + (b + n + (j - j0)) * a.I, hv);
                         }
                     }
                 }
                 tc_fence_before_sync();
                 __syncwarp();
                 if (lane == 0)
-                    mbar_arrive(&tempty[acc]);
+                    mbar_arrive(&B.tempty[acc]);
                 if (++acc == 2) {
                     acc = 0;
                     acc_phase ^= 1u;
@@ -439,11 +593,13 @@ stream_gate_up_fp4_kernel(const __grid_constant__ F4GuMaps maps, const F4GuArgs 
 }
 
 // --------------------------------------------------------------------- down
+// Tiles as in decode_tc.cuh: 128 rows of W_down against one slice of <= 8
+// picks of one expert (h as fp16 hi/lo rows), or against the shared h.
 struct F4DnMaps {
-    CUtensorMap cd;  // routed W_down codes [E, H, I/2] u8: box 32 x 128 x 1
-    CUtensorMap sd;  // shared W_down codes [H, I_s/2] u8: box 32 x 128
-    CUtensorMap hr;  // routed h fp16 hi/lo rows [2 pairs + 16, I]: box 64 x 16
-    CUtensorMap hs;  // shared h fp16 [16, I_s]: box 64 x 16
+    CUtensorMap cd;  // routed W_down codes [E, H, I/2] u8: box 128 x 128 x 1, SW128
+    CUtensorMap sd;  // shared W_down codes [H, I_s/2] u8: box 128 x 128, SW128
+    CUtensorMap hr;  // routed h fp16 hi/lo rows [2 pairs + 16, I]: box 64 x 16, SW128
+    CUtensorMap hs;  // shared h fp16 [16, I_s]: box 64 x 16, SW128
 };
 
 struct F4DnArgs {
@@ -456,8 +612,7 @@ struct F4DnArgs {
 };
 
 struct F4DnSmem {
-    static constexpr uint32_t bars = kF4Stages * kF4StageBytes;
-    static constexpr uint32_t misc = bars + (3 * kF4Stages + 6) * 8;
+    static constexpr uint32_t misc = kF4Misc;
     static constexpr uint32_t slice_group = misc + 16;
     static constexpr uint32_t slice_j0 = slice_group + kStreamMaxPairs * 4;
     static constexpr uint32_t n_slices = slice_j0 + kStreamMaxPairs * 4;
@@ -471,13 +626,7 @@ stream_down_fp4_kernel(const __grid_constant__ F4DnMaps maps, const F4DnArgs a) 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + F4DnSmem::bars);
-    uint64_t *deq = full + kF4Stages;
-    uint64_t *empty = deq + kF4Stages;
-    uint64_t *tfull = empty + kF4Stages;
-    uint64_t *tempty = tfull + 2;
-    uint64_t *drain = tempty + 2;
-    uint64_t *planbar = drain + 1;
+    const F4Bars B(smem);
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + F4DnSmem::misc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + F4DnSmem::misc + 8);
     int *slice_group = reinterpret_cast<int *>(smem + F4DnSmem::slice_group);
@@ -489,19 +638,12 @@ stream_down_fp4_kernel(const __grid_constant__ F4DnMaps maps, const F4DnArgs a) 
     const int lane = (int)lane_id();
     const int has_shared = a.I_s > 0 ? 1 : 0;
     const int n_mb = (a.H + kGemmBM - 1) / kGemmBM;
+    const int kb_routed = (a.I + kGemmBK - 1) / kGemmBK;
+    const int kb_shared = (a.I_s + kGemmBK - 1) / kGemmBK;
+    auto kbn_of = [&](int u) { return u / n_mb < has_shared ? kb_shared : kb_routed; };
 
     if (warp == 0 && lane == 0) {
-        for (int s = 0; s < kF4Stages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&deq[s], 4);
-            mbar_init(&empty[s], 1);
-        }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 4);
-        }
-        mbar_init(drain, 1);
-        mbar_init(planbar, 1);
+        B.init();
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tensormap(&maps.cd);
@@ -525,7 +667,7 @@ stream_down_fp4_kernel(const __grid_constant__ F4DnMaps maps, const F4DnArgs a) 
             grid_dependency_wait();  // h comes from the previous kernel
             uint32_t stage = 0, phase = 0;
             int issued = 0;
-            bool stop = !mbar_wait(planbar, 0, abort_flag);
+            bool stop = !mbar_wait(B.planbar, 0, abort_flag);
             const int total = stop ? 0 : (has_shared + *n_slices) * n_mb;
             for (int u = blockIdx.x; u < total && !stop; u += gridDim.x) {
                 const int si = u / n_mb, mb = u - si * n_mb;
@@ -533,24 +675,25 @@ stream_down_fp4_kernel(const __grid_constant__ F4DnMaps maps, const F4DnArgs a) 
                 const int slice = si - has_shared;
                 const int e = shared ? 0 : (int)P.group_expert[slice_group[slice]];
                 const int row =
-                    shared ? -1 : 2 * ((int)P.group_first[slice_group[slice]] + slice_j0[slice]);
-                const int kblocks = ((shared ? a.I_s : a.I) + kGemmBK - 1) / kGemmBK;
-                for (int kb = 0; kb < kblocks; ++kb) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+                    shared ? 0 : 2 * ((int)P.group_first[slice_group[slice]] + slice_j0[slice]);
+                const int kbn = kbn_of(u);
+                const int n_st = f4_stages_of(kbn);
+                for (int ks = 0; ks < n_st; ++ks) {
+                    if (!mbar_wait(&B.empty[stage], phase ^ 1u, abort_flag)) {
                         stop = true;
                         break;
                     }
                     uint8_t *st = smem + stage * kF4StageBytes;
-                    mbar_arrive_expect_tx(&full[stage], kF4CodeBytes + kF4BBytes);
-                    const int kc = kb * (kGemmBK / 2);
-                    if (shared) {
-                        tma_load_2d(st + kF4CodeOff, &maps.sd, kc, mb * kGemmBM, &full[stage], pol_w);
-                        tma_load_2d(st + kF4BOff, &maps.hs, kb * kGemmBK, 0, &full[stage], pol_h);
-                    } else {
-                        tma_load_3d(st + kF4CodeOff, &maps.cd, kc, mb * kGemmBM, e, &full[stage],
-                                    pol_w);
-                        tma_load_2d(st + kF4BOff, &maps.hr, kb * kGemmBK, row, &full[stage], pol_h);
-                    }
+                    const int n_sub = min(kF4Sub, kbn - ks * kF4Sub);
+                    mbar_arrive_expect_tx(&B.full[stage], kF4CodeBytes + n_sub * kF4BBox);
+                    const int kc = ks * (kF4KS / 2);
+                    if (shared)
+                        tma_load_2d(st, &maps.sd, kc, mb * kGemmBM, &B.full[stage], pol_w);
+                    else
+                        tma_load_3d(st, &maps.cd, kc, mb * kGemmBM, e, &B.full[stage], pol_w);
+                    for (int sub = 0; sub < n_sub; ++sub)
+                        tma_load_2d(st + kF4BOff + sub * kF4BBox, shared ? &maps.hs : &maps.hr,
+                                    (ks * kF4Sub + sub) * kGemmBK, row, &B.full[stage], pol_h);
                     ++issued;
                     if (++stage == kF4Stages) {
                         stage = 0;
@@ -559,88 +702,40 @@ stream_down_fp4_kernel(const __grid_constant__ F4DnMaps maps, const F4DnArgs a) 
                 }
             }
             for (int n = issued > kF4Stages ? issued - kF4Stages : 0; n < issued; ++n)
-                mbar_wait(&full[n % kF4Stages], (uint32_t)(n / kF4Stages) & 1u, nullptr);
+                mbar_wait(&B.full[n % kF4Stages], (uint32_t)(n / kF4Stages) & 1u, nullptr);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer
         if (elect_one()) {
-            uint32_t stage = 0, phase = 0;
-            uint32_t acc = 0, acc_phase = 0;
-            bool stop = !mbar_wait(planbar, 0, abort_flag);
-            const int total = stop ? 0 : (has_shared + *n_slices) * n_mb;
-            const uint32_t idesc = idesc_f16_f32(kGemmBM, kTcN);
-            for (int u = blockIdx.x; u < total && !stop; u += gridDim.x) {
-                const bool shared = u / n_mb < has_shared;
-                const int kblocks = ((shared ? a.I_s : a.I) + kGemmBK - 1) / kGemmBK;
-                if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag))
-                    break;
-                tc_fence_after_sync();
-                const uint32_t d_tmem = tmem_base + acc * kTcN;
-                for (int kb = 0; kb < kblocks; ++kb) {
-                    if (!mbar_wait(&deq[stage], phase, abort_flag)) {
-                        stop = true;
-                        break;
-                    }
-                    tc_fence_after_sync();
-                    const uint32_t a_addr = smem_u32(smem + stage * kF4StageBytes);
-                    const uint32_t b_addr = a_addr + kF4BOff;
-#pragma unroll
-                    for (int kk = 0; kk < kGemmBK / 16; ++kk)
-                        umma_bf16(d_tmem, smem_desc_sw128_kmajor(a_addr + kk * 32),
-                                  smem_desc_sw128_kmajor(b_addr + kk * 32), idesc,
-                                  (kb > 0 || kk > 0) ? 1u : 0u);
-                    umma_commit(&empty[stage]);
-                    if (++stage == kF4Stages) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
-                }
-                if (stop)
-                    break;
-                umma_commit(&tfull[acc]);
-                if (++acc == 2) {
-                    acc = 0;
-                    acc_phase ^= 1u;
-                }
-            }
-            umma_commit(drain);
-            mbar_wait(drain, 0, nullptr);
+            const bool planned = mbar_wait(B.planbar, 0, abort_flag);
+            const int total = planned ? (has_shared + *n_slices) * n_mb : 0;
+            f4_mma_loop(smem, B.full, B.empty, B.afull, B.aempty, B.tfull, B.tempty, abort_flag,
+                        tmem_base, total, kbn_of);
+            umma_commit(B.drain);
+            mbar_wait(B.drain, 0, nullptr);
         }
     } else if (warp >= kF4DeqWarp0) {
         // ---------------------------------------------------- dequantisers
-        const int r = (int)threadIdx.x - 32 * kF4DeqWarp0;  // row of the 128-row tile
-        const bool planned = mbar_wait(planbar, 0, abort_flag);
+        int r, h;  // row of the 128-row tile, half of it
+        dequant_row_of((int)threadIdx.x - 32 * kF4DeqWarp0, r, h);
+        const bool planned = mbar_wait(B.planbar, 0, abort_flag);
         const int total = planned ? (has_shared + *n_slices) * n_mb : 0;
-        uint32_t stage = 0, phase = 0;
-        bool stop = false;
-        for (int u = blockIdx.x; u < total && !stop; u += gridDim.x) {
+        auto row_of = [&](int u, const uint32_t *&p, int &kbn) {
             const int si = u / n_mb, mb = u - si * n_mb;
             const bool shared = si < has_shared;
             const int e = shared ? 0 : (int)P.group_expert[slice_group[si - has_shared]];
             const F4Mat &m = shared ? a.sd : a.wd;
             const int hrow = mb * kGemmBM + r;
-            const bool in = hrow < m.rows;
-            const uint32_t *srow = reinterpret_cast<const uint32_t *>(
-                m.scales + ((size_t)e * m.rows + (in ? hrow : 0)) * (size_t)(m.cols / 16));
-            const int kblocks = ((int)m.cols + kGemmBK - 1) / kGemmBK;
-            for (int kb = 0; kb < kblocks; ++kb) {
-                if (!mbar_wait(&full[stage], phase, abort_flag)) {
-                    stop = true;
-                    break;
-                }
-                uint8_t *st = smem + stage * kF4StageBytes;
-                const uint32_t s4 = in ? __ldg(srow + kb) : 0u;
-                dequant_row(st + kF4CodeOff, s4, st, r);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(&deq[stage]);
-                if (++stage == kF4Stages) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
-            }
-        }
+            if (hrow < m.rows)
+                p = reinterpret_cast<const uint32_t *>(
+                    m.scales + ((size_t)e * m.rows + hrow) * (size_t)(m.cols / 16));
+            kbn = kbn_of(u);
+        };
+        int n_stages = 0;
+        for (int u = blockIdx.x; u < total; u += gridDim.x)
+            n_stages += f4_stages_of(kbn_of(u));
+        ScaleCursor<decltype(row_of)> cur((int)blockIdx.x, total, (int)gridDim.x, row_of);
+        dequant_stages(smem, B.full, B.afull, B.aempty, abort_flag, n_stages, cur, r, h, lane);
     } else {
         // ------------------------------------------------ plan, then epilogue
         const int ltid = (int)threadIdx.x - 64;
@@ -656,17 +751,17 @@ stream_down_fp4_kernel(const __grid_constant__ F4DnMaps maps, const F4DnArgs a) 
                 }
             }
             *n_slices = sl;
-            mbar_arrive(planbar);
+            mbar_arrive(B.planbar);
         }
         grid_dependency_wait();  // before any output is written
-        if (mbar_wait(planbar, 0, abort_flag)) {
+        if (mbar_wait(B.planbar, 0, abort_flag)) {
             const int q = warp & 3;
             const int total = (has_shared + *n_slices) * n_mb;
             uint32_t acc = 0, acc_phase = 0;
             for (int u = blockIdx.x; u < total; u += gridDim.x) {
                 const int si = u / n_mb, mb = u - si * n_mb;
                 const bool shared = si < has_shared;
-                if (!mbar_wait(&tfull[acc], acc_phase, abort_flag))
+                if (!mbar_wait(&B.tfull[acc], acc_phase, abort_flag))
                     break;
                 tc_fence_after_sync();
                 uint32_t v[16];
@@ -681,25 +776,25 @@ stream_down_fp4_kernel(const __grid_constant__ F4DnMaps maps, const F4DnArgs a) 
                     const int n = shared ? a.T : min(kTcSlice, (int)P.group_first[g + 1] - p0);
                     float lo[kTcSlice];
 #pragma unroll
-                    for (int r = 0; r < kTcSlice; ++r)
-                        lo[r] = 0.f;
+                    for (int i = 0; i < kTcSlice; ++i)
+                        lo[i] = 0.f;
 #pragma unroll
                     for (int nn = 1; nn <= kTcSlice; ++nn)
                         if (n == nn) {
 #pragma unroll
-                            for (int r = 0; r < nn; ++r)
-                                lo[r] = __uint_as_float(v[r + nn]);
+                            for (int i = 0; i < nn; ++i)
+                                lo[i] = __uint_as_float(v[i + nn]);
                         }
 #pragma unroll
-                    for (int r = 0; r < kTcSlice; ++r) {
-                        const float d = ts * (__uint_as_float(v[r]) + lo[r]);
-                        if (r < n) {
+                    for (int i = 0; i < kTcSlice; ++i) {
+                        const float dv = ts * (__uint_as_float(v[i]) + lo[i]);
+                        if (i < n) {
                             if (shared) {
-                                a.s[(size_t)r * a.H + row] = d;
+                                a.s[(size_t)i * a.H + row] = dv;
                             } else {
-                                const int pair = p0 + r;
+                                const int pair = p0 + i;
                                 a.c[(size_t)P.sorted_src[pair] * a.H + row] =
-                                    P.pair_weight[pair] * d;
+                                    P.pair_weight[pair] * dv;
                             }
                         }
                     }
@@ -707,7 +802,7 @@ stream_down_fp4_kernel(const __grid_constant__ F4DnMaps maps, const F4DnArgs a) 
                 tc_fence_before_sync();
                 __syncwarp();
                 if (lane == 0)
-                    mbar_arrive(&tempty[acc]);
+                    mbar_arrive(&B.tempty[acc]);
                 if (++acc == 2) {
                     acc = 0;
                     acc_phase ^= 1u;
@@ -743,14 +838,14 @@ inline bool make_map_typed(CUtensorMap *m, const void *base, int rank, const uin
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Codes of `mats` matrices of [rows][cols] NVFP4 elements: 32-byte (64
-// element) by box_rows boxes, no swizzle (the dequantisers read them).
+// Codes of `mats` matrices of [rows][cols] NVFP4 elements: 128-byte (one
+// stage's 256 elements) by box_rows boxes, 128-byte swizzled.
 inline bool map_codes(CUtensorMap *m, const void *codes, uint64_t cols, uint64_t rows,
                       uint64_t mats, uint32_t box_rows) {
     const uint64_t dims[3] = {cols / 2, rows, mats};
     const uint64_t strides[2] = {cols / 2, rows * cols / 2};
-    return make_map_typed(m, codes, mats > 1 ? 3 : 2, dims, strides, kGemmBK / 2, box_rows,
-                          CU_TENSOR_MAP_DATA_TYPE_UINT8, CU_TENSOR_MAP_SWIZZLE_NONE);
+    return make_map_typed(m, codes, mats > 1 ? 3 : 2, dims, strides, kF4KS / 2, box_rows,
+                          CU_TENSOR_MAP_DATA_TYPE_UINT8, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // fp16 [rows][cols]: 64 x box_rows boxes, 128-byte swizzle (an MMA operand).
