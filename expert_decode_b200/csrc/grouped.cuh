@@ -23,11 +23,14 @@
 //                   passed along, one fixed order whatever the plan -- then
 //                   plus the shared expert's output.
 //
-// The GEMMs are persistent and warp specialised: warp 0 issues TMA loads
-// (cp.async.bulk.tensor, 128-byte swizzle, one CTA per copy) into a 4-stage
-// shared-memory ring, warp 1 issues tcgen05.mma with the fp32 accumulator in
-// tensor memory (two accumulators, so the epilogue of one tile overlaps the
-// MMAs of the next), and warps 2..5 drain the accumulator with tcgen05.ld.
+// The GEMMs are persistent and warp specialised: warp 0 issues the weight
+// tiles' TMA loads (cp.async.bulk.tensor, 128-byte swizzle, one CTA per copy)
+// into a 6-stage ring of 16 KB and warp 6 the activation tiles' into a
+// 3-stage ring of 32 KB, so that a tile with few rows (whose weights are most
+// of its bytes) keeps 96 KB of weights in flight; warp 1 issues tcgen05.mma
+// with the fp32 accumulator in tensor memory (two accumulators, so the
+// epilogue of one tile overlaps the MMAs of the next), and warps 2..5 drain
+// the accumulator with tcgen05.ld.
 // Weights sit on the MMA's M side (128 rows) and the expert's tokens on the
 // N side (16..256), so a tile is never padded to 128 tokens.
 #pragma once
@@ -42,8 +45,10 @@ namespace epk {
 constexpr int kGemmBM = 128;
 constexpr int kGemmBN = 256;
 constexpr int kGemmBK = 64;
-constexpr int kGemmStages = 4;
-constexpr int kGemmThreads = 192;
+constexpr int kGemmAStages = 6;   // weight tiles
+constexpr int kGemmBStages = 3;   // activation tiles
+constexpr int kGemmThreads = 224;
+constexpr int kGemmWarpB = 6;     // the activation-tile producer
 constexpr int kGateUpRows = 64;  // units of I per gate/up tile (64 gate + 64 up rows)
 // The activation tile is one box per stage, of the smallest of these heights
 // (capped at the tensor's rows rounded up to 32) that covers the tile's rows:
@@ -52,7 +57,8 @@ constexpr int kBoxLevels = 4;
 constexpr int kBoxRowsB[kBoxLevels] = {32, 64, 128, 256};
 constexpr uint32_t kTileABytes = kGemmBM * kGemmBK * 2;
 constexpr uint32_t kTileBBytes = kGemmBN * kGemmBK * 2;
-constexpr uint32_t kStageBytes = kTileABytes + kTileBBytes;
+constexpr uint32_t kRingBOff = kGemmAStages * kTileABytes;
+constexpr uint32_t kRingBytes = kRingBOff + kGemmBStages * kTileBBytes;
 constexpr int kTmemCols = 2 * kGemmBN;
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanWarps = kPlanThreads / 32;
@@ -322,13 +328,13 @@ struct GemmParams {
 };
 
 struct GemmSmem {
-    static constexpr uint32_t bars = kGemmStages * kStageBytes;
+    static constexpr uint32_t bars = kRingBytes;
     static constexpr uint32_t misc = bars + 256;
     static constexpr uint32_t units = misc + 64;
     static constexpr uint32_t offsets = units + kMaxGroups * 4 + 4;
-    // per epilogue warp: the tile's pick index and routing weight per column
-    static constexpr uint32_t colmeta = (offsets + (kMaxGroups + 2) * 4 + 15) / 16 * 16;
-    static constexpr uint32_t total = colmeta + 4 * kGemmBN * 8;
+    // gate/up: the column exchange of the two epilogue warp pairs, 2 x 2 x [16][32]
+    static constexpr uint32_t xchg = (offsets + (kMaxGroups + 2) * 4 + 15) / 16 * 16;
+    static constexpr uint32_t total = xchg + 2 * 2 * 16 * 32 * 4;
     static constexpr uint32_t alloc = total + 1024;  // room to align the base to 1024
 };
 
@@ -336,13 +342,15 @@ template <bool GATE_UP>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
     using Smem = GemmSmem;
-    constexpr int S = kGemmStages;
+    constexpr int SA = kGemmAStages, SB = kGemmBStages;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + Smem::bars);
-    uint64_t *empty = full + S;
-    uint64_t *tfull = empty + S;
+    uint64_t *full_a = reinterpret_cast<uint64_t *>(smem + Smem::bars);
+    uint64_t *empty_a = full_a + SA;
+    uint64_t *full_b = empty_a + SA;
+    uint64_t *empty_b = full_b + SB;
+    uint64_t *tfull = empty_b + SB;
     uint64_t *tempty = tfull + 2;
     uint64_t *drain = tempty + 2;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + Smem::misc);
@@ -355,9 +363,13 @@ grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
     const int G = p.G;
 
     if (warp == 0 && lane == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+        for (int s = 0; s < SA; ++s) {
+            mbar_init(&full_a[s], 1);
+            mbar_init(&empty_a[s], 1);
+        }
+        for (int s = 0; s < SB; ++s) {
+            mbar_init(&full_b[s], 1);
+            mbar_init(&empty_b[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
@@ -408,7 +420,7 @@ grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
     };
 
     if (warp == 0) {
-        // ------------------------------------------------------ TMA producer
+        // -------------------------------------------- TMA producer: weights
         if (elect_one()) {
             // a weight tile read by one n block streams through L2 once; one
             // read by several (an expert with more than 256 rows, whose n
@@ -416,7 +428,6 @@ grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
             // at normal priority so that the other n blocks find it there
             const uint64_t pol_once = policy_evict_first();
             const uint64_t pol_again = policy_evict_normal();
-            const uint64_t pol_x = policy_evict_last();
             uint32_t stage = 0, phase = 0;
             int issued = 0;
             bool stop = false;
@@ -424,6 +435,56 @@ grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
                 int g, mb, nb, rows, n_blocks;
                 decode(u, g, mb, nb, rows, n_blocks);
                 const uint64_t pol_w = n_blocks > 1 ? pol_again : pol_once;
+                const bool shared = g >= p.E;
+                const int K = shared ? p.k_shared : p.k_routed;
+                const int kblocks = (K + kGemmBK - 1) / kGemmBK;
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(&empty_a[stage], phase ^ 1u, abort_flag)) {
+                        stop = true;
+                        break;
+                    }
+                    uint8_t *sa = smem + stage * kTileABytes;
+                    mbar_arrive_expect_tx(&full_a[stage], kTileABytes);
+                    const int k0 = kb * kGemmBK;
+                    if (GATE_UP) {
+                        // rows 0..63: W_gate of the tile's 64 units, 64..127: W_up
+                        const int row = mb * kGateUpRows;
+                        uint8_t *sa_up = sa + kGateUpRows * kGemmBK * 2;
+                        if (shared) {
+                            tma_load_2d(sa, &maps.a_shared, k0, row, &full_a[stage], pol_w);
+                            tma_load_2d(sa_up, &maps.a2_shared, k0, row, &full_a[stage], pol_w);
+                        } else {
+                            tma_load_3d(sa, &maps.a, k0, row, g, &full_a[stage], pol_w);
+                            tma_load_3d(sa_up, &maps.a2, k0, row, g, &full_a[stage], pol_w);
+                        }
+                    } else {
+                        if (shared)
+                            tma_load_2d(sa, &maps.a_shared, k0, mb * kGemmBM, &full_a[stage],
+                                        pol_w);
+                        else
+                            tma_load_3d(sa, &maps.a, k0, mb * kGemmBM, g, &full_a[stage], pol_w);
+                    }
+                    ++issued;
+                    if (++stage == SA) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // no copy may still be landing in shared memory when the CTA exits
+            for (int n = issued > SA ? issued - SA : 0; n < issued; ++n)
+                mbar_wait(&full_a[n % SA], (uint32_t)(n / SA) & 1u, nullptr);
+        }
+    } else if (warp == kGemmWarpB) {
+        // ---------------------------------------- TMA producer: activations
+        if (elect_one()) {
+            const uint64_t pol_x = policy_evict_last();
+            uint32_t stage = 0, phase = 0;
+            int issued = 0;
+            bool stop = false;
+            for (int u = blockIdx.x; u < total_units && !stop; u += gridDim.x) {
+                int g, mb, nb, rows, n_blocks;
+                decode(u, g, mb, nb, rows, n_blocks);
                 const bool shared = g >= p.E;
                 const int K = shared ? p.k_shared : p.k_routed;
                 const int n0 = nb * kGemmBN;
@@ -442,47 +503,27 @@ grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
                 const uint32_t b_bytes = (uint32_t)box_rows[lvl] * kGemmBK * 2;
                 const int kblocks = (K + kGemmBK - 1) / kGemmBK;
                 for (int kb = 0; kb < kblocks; ++kb) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+                    if (!mbar_wait(&empty_b[stage], phase ^ 1u, abort_flag)) {
                         stop = true;
                         break;
                     }
-                    uint8_t *sa = smem + stage * kStageBytes;
-                    uint8_t *sb = sa + kTileABytes;
-                    mbar_arrive_expect_tx(&full[stage], kTileABytes + b_bytes);
-                    const int k0 = kb * kGemmBK;
-                    if (GATE_UP) {
-                        // rows 0..63: W_gate of the tile's 64 units, 64..127: W_up
-                        const int row = mb * kGateUpRows;
-                        uint8_t *sa_up = sa + kGateUpRows * kGemmBK * 2;
-                        if (shared) {
-                            tma_load_2d(sa, &maps.a_shared, k0, row, &full[stage], pol_w);
-                            tma_load_2d(sa_up, &maps.a2_shared, k0, row, &full[stage], pol_w);
-                        } else {
-                            tma_load_3d(sa, &maps.a, k0, row, g, &full[stage], pol_w);
-                            tma_load_3d(sa_up, &maps.a2, k0, row, g, &full[stage], pol_w);
-                        }
-                    } else {
-                        if (shared)
-                            tma_load_2d(sa, &maps.a_shared, k0, mb * kGemmBM, &full[stage], pol_w);
-                        else
-                            tma_load_3d(sa, &maps.a, k0, mb * kGemmBM, g, &full[stage], pol_w);
-                    }
-                    tma_load_2d(sb, bmap, k0, brow, &full[stage], pol_x);
+                    uint8_t *sb = smem + kRingBOff + stage * kTileBBytes;
+                    mbar_arrive_expect_tx(&full_b[stage], b_bytes);
+                    tma_load_2d(sb, bmap, kb * kGemmBK, brow, &full_b[stage], pol_x);
                     ++issued;
-                    if (++stage == S) {
+                    if (++stage == SB) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
             }
-            // no copy may still be landing in shared memory when the CTA exits
-            for (int n = issued > S ? issued - S : 0; n < issued; ++n)
-                mbar_wait(&full[n % S], (uint32_t)(n / S) & 1u, nullptr);
+            for (int n = issued > SB ? issued - SB : 0; n < issued; ++n)
+                mbar_wait(&full_b[n % SB], (uint32_t)(n / SB) & 1u, nullptr);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer
         if (elect_one()) {
-            uint32_t stage = 0, phase = 0;
+            uint32_t sa = 0, pa = 0, sb = 0, pb = 0;
             uint32_t acc = 0, acc_phase = 0;
             bool stop = false;
             for (int u = blockIdx.x; u < total_units && !stop; u += gridDim.x) {
@@ -499,22 +540,29 @@ grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
                 const uint32_t d_tmem = tmem_base + acc * kGemmBN;
                 const int kblocks = (K + kGemmBK - 1) / kGemmBK;
                 for (int kb = 0; kb < kblocks; ++kb) {
-                    if (!mbar_wait(&full[stage], phase, abort_flag)) {
+                    if (!mbar_wait(&full_a[sa], pa, abort_flag) ||
+                        !mbar_wait(&full_b[sb], pb, abort_flag)) {
                         stop = true;
                         break;
                     }
                     tc_fence_after_sync();
-                    const uint32_t a_addr = smem_u32(smem + stage * kStageBytes);
-                    const uint32_t b_addr = a_addr + kTileABytes;
+                    const uint32_t a_addr = smem_u32(smem + sa * kTileABytes);
+                    const uint32_t b_addr = smem_u32(smem + kRingBOff + sb * kTileBBytes);
 #pragma unroll
                     for (int kk = 0; kk < kGemmBK / 16; ++kk)
                         umma_bf16(d_tmem, smem_desc_sw128_kmajor(a_addr + kk * 32),
                                   smem_desc_sw128_kmajor(b_addr + kk * 32), idesc,
                                   (kb > 0 || kk > 0) ? 1u : 0u);
-                    umma_commit(&empty[stage]);  // frees the slot once these MMAs are done
-                    if (++stage == S) {
-                        stage = 0;
-                        phase ^= 1u;
+                    // each frees its slot once these MMAs are done
+                    umma_commit(&empty_a[sa]);
+                    umma_commit(&empty_b[sb]);
+                    if (++sa == SA) {
+                        sa = 0;
+                        pa ^= 1u;
+                    }
+                    if (++sb == SB) {
+                        sb = 0;
+                        pb ^= 1u;
                     }
                 }
                 if (stop)
@@ -529,19 +577,17 @@ grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
             umma_commit(drain);
             mbar_wait(drain, 0, nullptr);
         }
-    } else {
+    } else if (warp >= 2 && warp < 6) {
         // ------------------------------------------------------ epilogue
         const int q = warp & 3;  // TMEM lane quarter this warp may access
-        int *col_pick = reinterpret_cast<int *>(smem + Smem::colmeta) + (warp - 2) * 2 * kGemmBN;
-        float *col_w = reinterpret_cast<float *>(col_pick + kGemmBN);
         // gate/up: quarters 0, 1 hold the gate rows of units 0..31, 32..63 and
         // quarters 2, 3 the up rows of the same units; the two warps of a pair
-        // (same units) swap half their columns through the colmeta area, which
-        // gate/up does not otherwise use: xg = gate values of columns 16..31,
-        // xu = up values of columns 0..15, each [16][32 lanes]
+        // (same units) swap half their columns through shared memory:
+        // xg = gate values of columns 16..31, xu = up values of columns 0..15,
+        // each [16][32 lanes]
         const bool gate_warp = q < 2;
         const int pair = q & 1;
-        float *xg = reinterpret_cast<float *>(smem + Smem::colmeta) + pair * 2 * 16 * 32;
+        float *xg = reinterpret_cast<float *>(smem + Smem::xchg) + pair * 2 * 16 * 32;
         float *xu = xg + 16 * 32;
         uint32_t acc = 0, acc_phase = 0;
         for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
@@ -550,15 +596,25 @@ grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
             const bool shared = g >= p.E;
             const int n0 = nb * kGemmBN;
             const int n_valid = min(kGemmBN, rows - n0);
+            // down: the pick index and routing weight of column 32 c + lane in
+            // mp[c], mw[c], loaded while the accumulator fills and handed to the
+            // other lanes by shuffles, so that no load waits behind a store
+            int mp[kGemmBN / 32];
+            float mw[kGemmBN / 32];
+#pragma unroll
+            for (int c = 0; c < kGemmBN / 32; ++c) {
+                mp[c] = 0;
+                mw[c] = 0.f;
+            }
             if (!GATE_UP && !shared) {
-                // this tile's pick index and routing weight per column, loaded by
-                // the warp's lanes in parallel while the accumulator fills
-                for (int col = lane; col < n_valid; col += 32) {
-                    const int pick = p.perm_pair[offsets[g] + n0 + col];
-                    col_pick[col] = pick;
-                    col_w[col] = p.weights[pick];
-                }
-                __syncwarp();
+#pragma unroll
+                for (int c = 0; c < kGemmBN / 32; ++c)
+                    if (32 * c + lane < n_valid)
+                        mp[c] = p.perm_pair[offsets[g] + n0 + 32 * c + lane];
+#pragma unroll
+                for (int c = 0; c < kGemmBN / 32; ++c)
+                    if (32 * c + lane < n_valid)
+                        mw[c] = p.weights[mp[c]];
             }
             bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag);
             // the two warps of a pair leave together or not at all (their
@@ -569,7 +625,11 @@ grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
                 break;
             tc_fence_after_sync();
             const uint32_t t_row = tmem_base + ((uint32_t)(32 * q) << 16) + acc * kGemmBN;
-            for (int c0 = 0; c0 < n_valid; c0 += 32) {
+#pragma unroll
+            for (int c = 0; c < kGemmBN / 32; ++c) {
+                const int c0 = 32 * c;
+                if (c0 >= n_valid)
+                    break;
                 uint32_t v[32];
                 tmem_load_32cols(t_row + (uint32_t)c0, v);
                 tmem_load_wait();
@@ -591,38 +651,68 @@ grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
                             xu[j * 32 + lane] = __uint_as_float(v[j]);
                     }
                     named_sync(1 + pair, 64);
-                    if (gate_warp) {
+                    // the partner's half, into registers before any store
+                    float xo[16];
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int col = c0 + j;
-                            if (col < n_valid && unit < M)
-                                hrow_base[(size_t)(row0 + j) * ld + unit] = f32_to_bf16_rne(
-                                    silu_f32(__uint_as_float(v[j])) * xu[j * 32 + lane]);
-                        }
-                    } else {
+                    for (int j = 0; j < 16; ++j)
+                        xo[j] = gate_warp ? xu[j * 32 + lane] : xg[j * 32 + lane];
+                    named_sync(1 + pair, 64);  // the buffers are free for the next chunk
+                    const int cb = gate_warp ? 0 : 16;
+                    uint16_t *dst = hrow_base + (size_t)(row0 + cb) * ld + unit;
+                    // whole half-chunks store without a test per column
+                    if (unit < M) {
+                        if (c0 + cb + 16 <= n_valid) {
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int col = c0 + 16 + j;
-                            if (col < n_valid && unit < M)
-                                hrow_base[(size_t)(row0 + 16 + j) * ld + unit] = f32_to_bf16_rne(
-                                    silu_f32(xg[j * 32 + lane]) * __uint_as_float(v[16 + j]));
+                            for (int j = 0; j < 16; ++j) {
+                                const float gv = gate_warp ? __uint_as_float(v[j]) : xo[j];
+                                const float uv = gate_warp ? xo[j] : __uint_as_float(v[16 + j]);
+                                dst[(size_t)j * ld] = f32_to_bf16_rne(silu_fast_f32(gv) * uv);
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) {
+                                const float gv = gate_warp ? __uint_as_float(v[j]) : xo[j];
+                                const float uv = gate_warp ? xo[j] : __uint_as_float(v[16 + j]);
+                                if (c0 + cb + j < n_valid)
+                                    dst[(size_t)j * ld] = f32_to_bf16_rne(silu_fast_f32(gv) * uv);
+                            }
                         }
                     }
-                    named_sync(1 + pair, 64);  // the buffers are free for the next chunk
                 } else {
                     const int row = mb * kGemmBM + 32 * q + lane;
-                    if (row < p.H) {
+                    // whole chunks store without a test per column; the pick
+                    // metadata of column c0 + j comes from lane j
+                    float wv[32];
+                    int pk[32];
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const int col = c0 + j;
-                            if (col < n_valid) {
-                                const float d = __uint_as_float(v[j]);
-                                if (shared) {
-                                    p.s_out[(size_t)(n0 + col) * p.H + row] = d;
-                                } else {
-                                    const int pick = col_pick[col];
-                                    p.c_out[(size_t)pick * p.H + row] = col_w[col] * d;
-                                }
+                    for (int j = 0; j < 32; ++j) {
+                        pk[j] = __shfl_sync(0xffffffffu, mp[c], j);
+                        wv[j] = __shfl_sync(0xffffffffu, mw[c], j);
+                    }
+                    if (row < p.H) {
+                        if (shared) {
+                            float *dst = p.s_out + (size_t)(n0 + c0) * p.H + row;
+                            if (c0 + 32 <= n_valid) {
+#pragma unroll
+                                for (int j = 0; j < 32; ++j)
+                                    dst[(size_t)j * p.H] = __uint_as_float(v[j]);
+                            } else {
+#pragma unroll
+                                for (int j = 0; j < 32; ++j)
+                                    if (c0 + j < n_valid)
+                                        dst[(size_t)j * p.H] = __uint_as_float(v[j]);
+                            }
+                        } else {
+                            float *dst = p.c_out + row;
+                            if (c0 + 32 <= n_valid) {
+#pragma unroll
+                                for (int j = 0; j < 32; ++j)
+                                    dst[(size_t)pk[j] * p.H] = wv[j] * __uint_as_float(v[j]);
+                            } else {
+#pragma unroll
+                                for (int j = 0; j < 32; ++j)
+                                    if (c0 + j < n_valid)
+                                        dst[(size_t)pk[j] * p.H] = wv[j] * __uint_as_float(v[j]);
                             }
                         }
                     }
