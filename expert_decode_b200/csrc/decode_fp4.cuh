@@ -14,22 +14,25 @@
 //
 //   warp 0      TMA: per 256-wide k stage the raw codes of the tile's 128
 //               rows (128 bytes each, 128-byte swizzled) and the stage's four
-//               16-bit activation (or h) boxes;
+//               16-bit activation (or h) boxes, into an 8-stage ring;
 //   warps 6-13  dequantise, 64-wide k block by k block, into a ring of fp16
-//               A tiles: thread (r, half) takes 32 codes of row r (cvt of
-//               E2M1 pairs to fp16 pairs, exact), multiplies them by their
-//               two block scales (E4M3 to fp16, exact: every product has at
-//               most 6 significant bits and lies in fp16's range) and writes
-//               them in the 128-byte swizzled K-major layout the MMA reads;
-//   warp 1      tcgen05.mma kind::f16 with fp16 A and B, fp32 accumulators in
-//               TMEM, one A tile of the ring per k block;
+//               A tiles held in tensor memory: thread (row, half) takes 32
+//               codes of its row (cvt of E2M1 pairs to fp16 pairs, exact),
+//               multiplies them by their two block scales (E4M3 to fp16,
+//               exact: every product has at most 6 significant bits and lies
+//               in fp16's range) and stores the 16 fp16 pairs to its row's
+//               TMEM lane with tcgen05.st;
+//   warp 1      tcgen05.mma kind::f16 with A from tensor memory and B (fp16)
+//               from shared memory, fp32 accumulators in TMEM;
 //   warps 2-5   the epilogue of decode_tc.cuh, with the tensor scale applied
 //               to the fp32 accumulator first.
 //
-// At 4.5 bits per weight a stage of 64-wide k blocks holds too few bytes to
-// keep HBM busy: the 256-wide stage puts 16 KB of codes per stage and 96 KB
-// per SM in flight, in 128-byte rows, while the 16 KB A tiles cycle through
-// a ring of their own.
+// The A tiles live in tensor memory rather than shared memory for two
+// reasons.  A tile is released only when the MMAs reading it complete, and
+// that latency must be covered by tiles already dequantised: tensor memory
+// holds fifteen 64-wide A tiles (480 of its 512 columns) where shared memory
+// could spare four.  And shared memory then carries only the codes and the
+// activations, whose 24 KB stages keep 192 KB of codes in flight per SM.
 //
 // The activations enter as fp16: x is converted once per call (exact for
 // bf16 values of magnitude 2^-14 .. 65504, which covers activations in
@@ -48,16 +51,19 @@ namespace epk {
 
 constexpr int kF4KS = 256;                               // k extent of one stage
 constexpr int kF4Sub = kF4KS / kGemmBK;                  // 64-wide k blocks per stage
-constexpr int kF4Stages = 6;
-constexpr int kF4ASlots = 4;
+constexpr int kF4Stages = 8;
+constexpr int kF4ASlots = 15;                            // A tiles in TMEM
 constexpr int kF4Threads = 448;                          // warps 0..13
 constexpr uint32_t kF4CodeBytes = kGemmBM * kF4KS / 2;   // 128 rows x 128 code bytes, 16 KB
 constexpr uint32_t kF4BBox = kTcN * kGemmBK * 2;         // 16 fp16 rows x 64, 2 KB
 constexpr uint32_t kF4BOff = kF4CodeBytes;               // four B boxes after the codes
 constexpr uint32_t kF4StageBytes = kF4CodeBytes + kF4Sub * kF4BBox;   // 24 KB
-constexpr uint32_t kF4ABytes = kGemmBM * kGemmBK * 2;    // one fp16 A tile, 16 KB
-constexpr uint32_t kF4AOff = kF4Stages * kF4StageBytes;  // the A ring after the stages
-constexpr uint32_t kF4Bars = kF4AOff + kF4ASlots * kF4ABytes;
+constexpr uint32_t kF4Bars = kF4Stages * kF4StageBytes;
+// tensor memory: two accumulators of kTcN columns, then the A ring, 32
+// columns (64 fp16 of k, two per 32-bit column) per tile
+constexpr uint32_t kF4TmemCols = 512;
+constexpr uint32_t kF4ACol0 = 2 * kTcN;
+constexpr uint32_t kF4ACols = kGemmBK / 2;
 // full[S], empty[S], afull[A], aempty[A], tfull[2], tempty[2], drain, planbar
 constexpr uint32_t kF4Misc = kF4Bars + (2 * kF4Stages + 2 * kF4ASlots + 6) * 8;
 constexpr int kF4DeqWarp0 = 6;                           // warps 6..13 dequantise
@@ -102,43 +108,62 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// k block `sub` of a stage, half h of row r: 32 codes (chunk 2 sub + h of
-// the row's 128 code bytes, which the copy stored 128-byte swizzled at
-// position (2 sub + h) ^ (r mod 8)) times their two block scales (bytes 2h,
-// 2h + 1 of s4, the row's four scale bytes of this k block) into row r of an
-// fp16 A tile, 128-byte swizzled: chunk j of the row (elements 8j .. 8j + 7)
-// at position j ^ (r mod 8).  Eight consecutive lanes take eight
-// consecutive rows with one h (dequant_row_of), so the eight 16-byte chunks
-// each of them reads or writes fall in eight distinct bank groups.
-__device__ __forceinline__ void dequant_half(const uint8_t *codes, int sub, uint32_t s4,
-                                             uint8_t *a_tile, int r, int h) {
+__device__ __forceinline__ void tmem_store_16cols(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_store_wait() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// One MMA with A (M x 16 of k) from tensor memory and B from shared memory.
+__device__ __forceinline__ void umma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// k block `sub` of a stage, half h of row r: 32 codes (chunk 2 sub + h of the
+// row's 128 code bytes, which the copy stored 128-byte swizzled at position
+// (2 sub + h) ^ (r mod 8)) times their two block scales (bytes 2h, 2h + 1 of
+// s4, the row's four scale bytes of this k block), as 16 fp16 pairs in the
+// order of k (element 2i in the low half of pair i).  A warp takes 32
+// consecutive rows: each eight lanes read eight distinct bank groups.
+__device__ __forceinline__ void dequant_half(const uint8_t *codes, int sub, uint32_t s4, int r,
+                                             int h, uint32_t (&out)[16]) {
     const uint4 c =
         reinterpret_cast<const uint4 *>(codes + 128 * r)[(2 * sub + h) ^ (r & 7)];
     const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
     const uint32_t s2 = e4m3x2_to_f16x2(h ? (s4 >> 16) : (s4 & 0xffffu));
     // each block scale broadcast to both halves of an fp16 pair
     const uint32_t sb[2] = {__byte_perm(s2, 0, 0x1010), __byte_perm(s2, 0, 0x3232)};
-    uint4 *row = reinterpret_cast<uint4 *>(a_tile + 128 * r);
 #pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {  // chunk 4h + jj: code word jj, block jj / 2
+    for (int jj = 0; jj < 4; ++jj) {  // code word jj: elements 8 jj .. 8 jj + 7, block jj / 2
         const uint32_t w = cw[jj];
         const uint32_t sc = sb[jj >> 1];
-        uint4 out;
-        out.x = hmul2_u32(e2m1x2_to_f16x2(w & 0xffu), sc);
-        out.y = hmul2_u32(e2m1x2_to_f16x2((w >> 8) & 0xffu), sc);
-        out.z = hmul2_u32(e2m1x2_to_f16x2((w >> 16) & 0xffu), sc);
-        out.w = hmul2_u32(e2m1x2_to_f16x2(w >> 24), sc);
-        row[(4 * h + jj) ^ (r & 7)] = out;
+        out[4 * jj + 0] = hmul2_u32(e2m1x2_to_f16x2(w & 0xffu), sc);
+        out[4 * jj + 1] = hmul2_u32(e2m1x2_to_f16x2((w >> 8) & 0xffu), sc);
+        out[4 * jj + 2] = hmul2_u32(e2m1x2_to_f16x2((w >> 16) & 0xffu), sc);
+        out[4 * jj + 3] = hmul2_u32(e2m1x2_to_f16x2(w >> 24), sc);
     }
 }
 
-// The row and half a dequantiser thread takes (d = 0..255 over warps 6..13):
-// warp d / 32 owns rows 16 (d / 32) .. + 15; lanes 0-7 / 8-15 take rows 0-7
-// with h = 0 / 1, lanes 16-23 / 24-31 rows 8-15.
-__device__ __forceinline__ void dequant_row_of(int d, int &r, int &h) {
-    const int l = d & 31;
-    r = 16 * (d >> 5) + (l & 7) + 8 * (l >> 4);
-    h = (l >> 3) & 1;
+// The row and half a dequantiser warp takes: warps 6..13; a warp may store
+// only to its lane quarter of tensor memory (warp mod 4), so warp w takes
+// rows 32 (w mod 4) + lane, half (w - 6) / 4 of each k block.
+__device__ __forceinline__ void dequant_row_of(int warp, int lane, int &r, int &h) {
+    r = 32 * (warp & 3) + lane;
+    h = (warp - kF4DeqWarp0) >> 2;
 }
 
 // Scale rows past a matrix read this zero row instead.
@@ -202,11 +227,13 @@ template <class RowOf>
 __device__ __forceinline__ void dequant_stages(uint8_t *smem, uint64_t *full, uint64_t *afull,
                                                uint64_t *aempty, volatile int *abort_flag,
                                                int n_stages, ScaleCursor<RowOf> &cur, int r,
-                                               int h, int lane) {
+                                               int h, int lane, uint32_t tmem_base) {
     F4StageScales q[kScaleAhead];
 #pragma unroll
     for (int j = 0; j < kScaleAhead; ++j)
         q[j] = cur.fetch();
+    // this warp's lane quarter and k half of every A tile
+    const uint32_t t_own = tmem_base + ((uint32_t)(r & ~31) << 16) + kF4ACol0 + 16u * (uint32_t)h;
     uint32_t stage = 0, phase = 0, slot = 0, aphase = 0;
     for (int n0 = 0; n0 < n_stages; n0 += kScaleAhead) {
 #pragma unroll
@@ -218,11 +245,14 @@ __device__ __forceinline__ void dequant_stages(uint8_t *smem, uint64_t *full, ui
 #pragma unroll
                 for (int sub = 0; sub < kF4Sub; ++sub) {
                     if (sub < q[j].n_sub) {
+                        uint32_t v[16];
+                        dequant_half(codes, sub, q[j].s[sub], r, h, v);
                         if (!mbar_wait(&aempty[slot], aphase ^ 1u, abort_flag))
                             return;
-                        dequant_half(codes, sub, q[j].s[sub], smem + kF4AOff + slot * kF4ABytes,
-                                     r, h);
-                        fence_proxy_async_smem();  // the MMA reads the tile through the async proxy
+                        tc_fence_after_sync();
+                        tmem_store_16cols(t_own + slot * kF4ACols, v);
+                        tmem_store_wait();
+                        tc_fence_before_sync();  // the MMA reads the tile after the arrive
                         __syncwarp();
                         if (lane == 0)
                             mbar_arrive(&afull[slot]);
@@ -269,13 +299,13 @@ __device__ __forceinline__ void f4_mma_loop(uint8_t *smem, uint64_t *full, uint6
                 if (!mbar_wait(&afull[slot], aphase, abort_flag))
                     return;
                 tc_fence_after_sync();
-                const uint32_t a_addr = smem_u32(smem + kF4AOff + slot * kF4ABytes);
+                const uint32_t a_tmem = tmem_base + kF4ACol0 + slot * kF4ACols;
                 const uint32_t b_addr = b_base + sub * kF4BBox;
 #pragma unroll
-                for (int kk = 0; kk < kGemmBK / 16; ++kk)
-                    umma_bf16(d_tmem, smem_desc_sw128_kmajor(a_addr + kk * 32),
-                              smem_desc_sw128_kmajor(b_addr + kk * 32), idesc,
-                              (ks > 0 || sub > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < kGemmBK / 16; ++kk)  // 16 of k: 8 columns of A
+                    umma_f16_tmem_a(d_tmem, a_tmem + 8 * kk,
+                                    smem_desc_sw128_kmajor(b_addr + kk * 32), idesc,
+                                    (ks > 0 || sub > 0 || kk > 0) ? 1u : 0u);
                 umma_commit(&aempty[slot]);
                 if (++slot == kF4ASlots) {
                     slot = 0;
@@ -388,7 +418,7 @@ stream_gate_up_fp4_kernel(const __grid_constant__ F4GuMaps maps, const F4GuArgs 
         prefetch_tensormap(&maps.x);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_holder, kTcTmemCols);
+        tmem_alloc(tmem_holder, kF4TmemCols);
         tmem_relinquish();
     }
     tc_fence_before_sync();
@@ -470,8 +500,8 @@ stream_gate_up_fp4_kernel(const __grid_constant__ F4GuMaps maps, const F4GuArgs 
         }
     } else if (warp >= kF4DeqWarp0) {
         // ---------------------------------------------------- dequantisers
-        int r, h;  // row of the A tile, half of it
-        dequant_row_of((int)threadIdx.x - 32 * kF4DeqWarp0, r, h);
+        int r, h;  // row of the A tile, half of its k block
+        dequant_row_of(warp, lane, r, h);
         const bool planned = mbar_wait(B.planbar, 0, abort_flag);
         const int total = planned ? tile_first[has_shared + P.n_groups] : 0;
         // the row's unit and its scale row (zeros past the matrix)
@@ -493,7 +523,7 @@ stream_gate_up_fp4_kernel(const __grid_constant__ F4GuMaps maps, const F4GuArgs 
                              : 0;
         ScaleCursor<decltype(row_of)> cur((int)blockIdx.x, total, (int)gridDim.x, row_of);
         dequant_stages(smem, B.full, B.afull, B.aempty, abort_flag, mine * n_st, cur, r, h,
-                       lane);
+                       lane, tmem_base);
     } else {
         // ------------------------------------------------ plan, then epilogue
         const int ltid = (int)threadIdx.x - 64;
@@ -588,7 +618,7 @@ stream_gate_up_fp4_kernel(const __grid_constant__ F4GuMaps maps, const F4GuArgs 
     __syncthreads();
     if (warp == 1) {
         tc_fence_after_sync();
-        tmem_dealloc(tmem_base, kTcTmemCols);
+        tmem_dealloc(tmem_base, kF4TmemCols);
     }
 }
 
@@ -650,7 +680,7 @@ stream_down_fp4_kernel(const __grid_constant__ F4DnMaps maps, const F4DnArgs a) 
         prefetch_tensormap(&maps.hr);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_holder, kTcTmemCols);
+        tmem_alloc(tmem_holder, kF4TmemCols);
         tmem_relinquish();
     }
     tc_fence_before_sync();
@@ -716,8 +746,8 @@ stream_down_fp4_kernel(const __grid_constant__ F4DnMaps maps, const F4DnArgs a) 
         }
     } else if (warp >= kF4DeqWarp0) {
         // ---------------------------------------------------- dequantisers
-        int r, h;  // row of the 128-row tile, half of it
-        dequant_row_of((int)threadIdx.x - 32 * kF4DeqWarp0, r, h);
+        int r, h;  // row of the 128-row tile, half of its k block
+        dequant_row_of(warp, lane, r, h);
         const bool planned = mbar_wait(B.planbar, 0, abort_flag);
         const int total = planned ? (has_shared + *n_slices) * n_mb : 0;
         auto row_of = [&](int u, const uint32_t *&p, int &kbn) {
@@ -735,7 +765,8 @@ stream_down_fp4_kernel(const __grid_constant__ F4DnMaps maps, const F4DnArgs a) 
         for (int u = blockIdx.x; u < total; u += gridDim.x)
             n_stages += f4_stages_of(kbn_of(u));
         ScaleCursor<decltype(row_of)> cur((int)blockIdx.x, total, (int)gridDim.x, row_of);
-        dequant_stages(smem, B.full, B.afull, B.aempty, abort_flag, n_stages, cur, r, h, lane);
+        dequant_stages(smem, B.full, B.afull, B.aempty, abort_flag, n_stages, cur, r, h, lane,
+                       tmem_base);
     } else {
         // ------------------------------------------------ plan, then epilogue
         const int ltid = (int)threadIdx.x - 64;
@@ -814,7 +845,7 @@ stream_down_fp4_kernel(const __grid_constant__ F4DnMaps maps, const F4DnArgs a) 
     __syncthreads();
     if (warp == 1) {
         tc_fence_after_sync();
-        tmem_dealloc(tmem_base, kTcTmemCols);
+        tmem_dealloc(tmem_base, kF4TmemCols);
     }
 }
 
