@@ -84,11 +84,16 @@ struct F4Mat {
     int64_t rows, cols;  // per matrix
 };
 
-__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
-    uint32_t d;
-    asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
-        : "=r"(d) : "r"(byte));
-    return d;
+// The eight E2M1 codes of a 32-bit word as four fp16 pairs: byte k (elements
+// 2k, 2k + 1) into d[k].  The word is split into its four bytes by one
+// vector move, which the conversions take directly (measured 1.7x the
+// conversion rate of a shift and mask per byte).
+__device__ __forceinline__ void e2m1x8_to_f16x2x4(uint32_t w, uint32_t (&d)[4]) {
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(w));
 }
 
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
@@ -149,12 +154,12 @@ __device__ __forceinline__ void dequant_half(const uint8_t *codes, int sub, uint
     const uint32_t sb[2] = {__byte_perm(s2, 0, 0x1010), __byte_perm(s2, 0, 0x3232)};
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj) {  // code word jj: elements 8 jj .. 8 jj + 7, block jj / 2
-        const uint32_t w = cw[jj];
+        uint32_t d[4];
+        e2m1x8_to_f16x2x4(cw[jj], d);
         const uint32_t sc = sb[jj >> 1];
-        out[4 * jj + 0] = hmul2_u32(e2m1x2_to_f16x2(w & 0xffu), sc);
-        out[4 * jj + 1] = hmul2_u32(e2m1x2_to_f16x2((w >> 8) & 0xffu), sc);
-        out[4 * jj + 2] = hmul2_u32(e2m1x2_to_f16x2((w >> 16) & 0xffu), sc);
-        out[4 * jj + 3] = hmul2_u32(e2m1x2_to_f16x2(w >> 24), sc);
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+            out[4 * jj + m] = hmul2_u32(d[m], sc);
     }
 }
 
