@@ -3,9 +3,9 @@
 //  1. group_plan    (one CTA): the picks grouped by expert with a warp-level
 //                   histogram (__match_any_sync) and prefix scans; a stable
 //                   scatter keeps each expert's rows in (token, slot) order.
-//                   This is the batched expert dispatch of the fak note
-//                   "GLM-5.2 multi-GPU" (hostBatchedGLMExperts: run each
-//                   expert once over the rows that picked it).
+//                   The fak note "GLM-5.2 multi-GPU" batches its expert
+//                   dispatch the same way (hostBatchedGLMExperts: each
+//                   expert runs once over the rows that picked it).
 //  2. gather_rows:  the picked activation rows, expert by expert, as bf16,
 //                   followed by every token's row for the shared expert.
 //  3. grouped GEMM, gate/up: per (expert, 64 units of I, up to 256 rows) tile

@@ -59,7 +59,7 @@ typedef enum { EP_BF16 = 0, EP_F32 = 1 } ep_dtype;
  * landed").  Band sizes follow the shard rule of TensorFold issue #310
  * ("GLM-5.3-Flash on CUDA over three ranks (--tp 3)", MiaAI-Lab's proposal,
  * shares.py): whole experts, as even as they go, the first E % bands bands
- * taking one more (largest remainder, ties to the lower rank).
+ * taking one more (largest remainder; of equal remainders the lower rank wins).
  */
 typedef struct {
     int32_t num_experts;

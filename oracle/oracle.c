@@ -19,7 +19,7 @@
  *  [TP3]  TensorFold issue #310 "GLM-5.3-Flash on CUDA over three ranks
  *         (--tp 3)", the share rule (whole units, the first units % world
  *         ranks take one more) and the maintainer's reply (largest remainder,
- *         ties to the lower rank; one fixed sum order).
+ *         equal remainders to the lower rank; one fixed sum order).
  *  [GATE] TensorFold issue #593 "GLM-5.3-Flash and full GLM-5.3 on the native
  *         CUDA engine (tracker)", "The gate" (an FP64 reference per
  *         projection class).
