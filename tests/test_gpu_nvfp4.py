@@ -206,3 +206,22 @@ def test_limits():
         ed.moe_ffn_forward_nvfp4(x, ids, w, g, u, d, shared, plan, workspace=ws[:need - 1])
     assert err.value.code == ed.EP_ENOMEM
     ed.ep_check_status()
+
+
+def test_longest_rows_and_empty_slots(oracle_lib):
+    """H = 16384, the longest rows (256 block-scale words per row, 64 stages per
+    tile), against I = 64 (one k block, a quarter stage), and EP_ID_NONE slots,
+    which contribute nothing and are not reported."""
+    T, H, E, k, I, I_s = 3, 16384, 4, 2, 64, 64
+    x, ids, w, mats = _case(oracle_lib, T, H, E, k, I, I_s, seed=16)
+    ids = ids.clone()
+    ids[1, 1] = -(2 ** 31)  # EP_ID_NONE
+    g, u, d, shared = mats
+    y = ed.moe_ffn_forward_nvfp4(x, ids, w, g, u, d, shared, ed.ep_plan(E, 2))
+    torch.cuda.synchronize()
+    ed.ep_check_status()
+    ref_ids, ref_w = ids.cpu().numpy().copy(), w.cpu().double().numpy().copy()
+    ref_ids[1, 1] = 0
+    ref_w[1, 1] = 0.0
+    check_y(y, oracle_ffn(oracle_lib, x, ref_ids, ref_w, _oracle_weights(*mats)),
+            rel_tol=REL_TOL, what="nvfp4 H=16384 I=64")
