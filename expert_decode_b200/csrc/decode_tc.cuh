@@ -41,7 +41,7 @@ namespace epk {
 
 constexpr int kTcN = 16;                                   // MMA N: tokens, zero rows after T
 constexpr int kTcStages = 10;
-constexpr int kTcThreads = 192;
+constexpr int kTcThreads = 224;  // warp 6: the gate/up kernel's group publisher
 constexpr uint32_t kTcABytes = kGemmBM * kGemmBK * 2;      // 64 gate + 64 up rows, 16 KB
 constexpr uint32_t kTcBBytes = kTcN * kGemmBK * 2;         // 16 token rows, 2 KB
 constexpr uint32_t kTcStageBytes = kTcABytes + kTcBBytes;  // 18 KB, a multiple of 1024
@@ -74,9 +74,46 @@ struct TcArgs {
     // in hb_shared [16][I_s] (hi in rows 0..T-1, lo in T..2T-1).
     uint16_t *hb_routed;
     uint16_t *hb_shared;
+    // When set, one word per group (the shared expert first, then the routed
+    // groups in plan order) counting the gate warps that have written their
+    // tile's h, for stream_down_tc_kernel of the same call (group_done_add)
+    unsigned long long *grp_done;
+    unsigned long long epoch;  // this call's number, 1 .. 2^48 - 1
 };
 
 constexpr int kTcSlice = 8;  // picks per slice of the bf16 hi/lo activations
+
+// Per-group completion words between the two decode kernels of a call.  The
+// word holds the call's epoch in its high 48 bits and the number of the
+// group's gate/up tiles done in its low 16, so a word left by an earlier call
+// (or never written) counts as zero without any reset: the first add of a
+// call replaces it.  The gate/up kernel adds one per tile once its h stores
+// are fenced; the down kernel starts a group's slices when the word reads
+// (epoch, the group's tile count).
+// Called by one thread after a __threadfence that follows the tile's h
+// stores (seen through a barrier): the fence is cumulative over them.
+__device__ __forceinline__ void group_done_add(unsigned long long *w, unsigned long long epoch) {
+    unsigned long long old = *reinterpret_cast<volatile unsigned long long *>(w);
+    for (int tries = 0; tries < (1 << 20); ++tries) {
+        const unsigned long long nw = (old >> 16) == epoch ? old + 1 : (epoch << 16) | 1ull;
+        const unsigned long long got = atomicCAS(w, old, nw);
+        if (got == old)
+            return;
+        old = got;
+    }
+    flag_status(kStatusTimeout);
+}
+
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// The count a group reaches: its gate/up tiles (`width` units of I, 64 per tile).
+__host__ __device__ inline int group_done_target(int width) {
+    return (width + kGateUpRows - 1) / kGateUpRows;
+}
 
 // h as the two bf16 parts hi = bf16(h), lo = bf16(h - hi): together they
 // carry h to about 16 significant bits, so that a bf16 x bf16 contraction of
@@ -90,8 +127,9 @@ __device__ __forceinline__ void store_hi_lo(uint16_t *hi_p, uint16_t *lo_p, floa
 struct TcSmem {
     static constexpr uint32_t stages = 0;
     static constexpr uint32_t bars = kTcStages * kTcStageBytes;
-    // full[S], empty[S], tfull[2], tempty[2], drain, planbar; tmem holder, abort flag
-    static constexpr uint32_t misc = bars + (2 * kTcStages + 6) * 8;
+    // full[S], empty[S], tfull[2], tempty[2], drain, planbar, hdone[2],
+    // hfree[2]; tmem holder, abort flag
+    static constexpr uint32_t misc = bars + (2 * kTcStages + 10) * 8;
     static constexpr uint32_t tile_first = misc + 16;  // [kTcMaxGroups + 1]
     static constexpr uint32_t row_first = tile_first + (kTcMaxGroups + 1) * 4;  // [kTcMaxGroups]
     // up values handed to the gate warps: [pair][accumulator][token][lane]
@@ -122,6 +160,8 @@ stream_gate_up_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     uint64_t *tempty = tfull + 2;
     uint64_t *drain = tempty + 2;
     uint64_t *planbar = drain + 1;
+    uint64_t *hdone = planbar + 1;  // [2]: both gate warps have stored a tile's h
+    uint64_t *hfree = hdone + 2;    // [2]: the publisher has taken hdone's phase
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + TcSmem::misc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + TcSmem::misc + 8);
     int *tile_first = reinterpret_cast<int *>(smem + TcSmem::tile_first);
@@ -144,6 +184,10 @@ stream_gate_up_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
         }
         mbar_init(drain, 1);
         mbar_init(planbar, 1);
+        mbar_init(&hdone[0], 2);
+        mbar_init(&hdone[1], 2);
+        mbar_init(&hfree[0], 1);
+        mbar_init(&hfree[1], 1);
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tensormap(&maps.wg);
@@ -268,6 +312,30 @@ stream_gate_up_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
             umma_commit(drain);
             mbar_wait(drain, 0, nullptr);
         }
+    } else if (warp == 6) {
+        // ---------------------------------------------------- group publisher
+        // After both gate warps have stored a tile's h (hdone), a gpu-scope
+        // fence (cumulative over those stores, seen through the barrier) and
+        // the group's count; kept off the epilogue, where the fence's wait
+        // would hold both warps of a pair.
+        if (a.grp_done != nullptr && elect_one()) {
+            const bool planned = mbar_wait(planbar, 0, abort_flag);
+            const int total = planned ? tile_first[has_shared + P.n_groups] : 0;
+            uint32_t acc = 0, acc_phase = 0;
+            for (int u = blockIdx.x; u < total; u += gridDim.x) {
+                int gi, m0;
+                decode(u, gi, m0);
+                if (!mbar_wait(&hdone[acc], acc_phase, abort_flag))
+                    break;
+                mbar_arrive(&hfree[acc]);  // the gate warps may arrive on it again
+                __threadfence();
+                group_done_add(&a.grp_done[gi], a.epoch);
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+        }
     } else {
         // ------------------------------------------------ plan, then epilogue
         const int ltid = (int)threadIdx.x - 64;
@@ -360,9 +428,16 @@ stream_gate_up_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
                     }
                 }
                 tc_fence_before_sync();
-                __syncwarp();
-                if (lane == 0)
+                __syncwarp();  // the warp's h stores before lane 0's arrive
+                if (lane == 0) {
                     mbar_arrive(&tempty[acc]);
+                    // the publisher has taken this barrier's previous phase
+                    // (it runs far ahead of the tiles: this wait normally
+                    // returns at once)
+                    if (gate_warp && a.grp_done != nullptr &&
+                        mbar_wait(&hfree[acc], acc_phase ^ 1u, abort_flag))
+                        mbar_arrive(&hdone[acc]);
+                }
                 if (++acc == 2) {
                     acc = 0;
                     acc_phase ^= 1u;
@@ -403,6 +478,10 @@ struct DtArgs {
     const float *weights;
     float *c;  // [T * top_k, H]: weighted contribution of pick t * top_k + j
     float *s;  // [T, H]: the shared expert's output
+    // the gate/up kernel's per-group completion words and the call's epoch;
+    // without them the kernel waits for the whole gate/up kernel instead
+    const unsigned long long *grp_done;
+    unsigned long long epoch;
 };
 
 struct DtSmem {
@@ -478,7 +557,79 @@ stream_down_tc_kernel(const __grid_constant__ DtMaps maps, const DtArgs a) {
         // before griddepcontrol.wait; their h boxes, written by the previous
         // kernel, follow once it has completed.  A stage's full barrier takes
         // the weight bytes by expect_tx and the h bytes with its one arrive.
-        if (elect_one()) {
+        if (a.grp_done != nullptr && elect_one()) {
+            // Each slice starts once its group's gate/up tiles have published
+            // their h (group_done_add): the slices of groups finished early
+            // stream while the gate/up kernel's last tiles still run.
+            const uint64_t pol_w = policy_evict_first();
+            const uint64_t pol_h = policy_evict_last();
+            uint32_t stage = 0, phase = 0;
+            int issued = 0, ready_group = -1;
+            bool stop = !mbar_wait(planbar, 0, abort_flag);
+            const int total = stop ? 0 : (has_shared + *n_slices) * n_mb;
+            auto group_ready = [&](int gidx, int width) -> bool {
+                const unsigned long long want =
+                    (a.epoch << 16) | (unsigned long long)group_done_target(width);
+                if (ld_acquire_u64(&a.grp_done[gidx]) == want)
+                    return true;
+                const uint64_t t0 = global_timer_ns();
+                for (uint32_t spin = 1;; ++spin) {
+                    if (ld_acquire_u64(&a.grp_done[gidx]) == want)
+                        return true;
+                    if (*abort_flag)
+                        return false;
+                    if ((spin & 255u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
+                        *abort_flag = 1;
+                        flag_status(kStatusTimeout);
+                        return false;
+                    }
+                }
+            };
+            for (int u = blockIdx.x; u < total && !stop; u += gridDim.x) {
+                const int si = u / n_mb, mb = u - si * n_mb;
+                const bool shared = si < has_shared;
+                const int slice = si - has_shared;
+                const int g = shared ? 0 : slice_group[slice];
+                const int gidx = shared ? 0 : has_shared + g;
+                const int e = shared ? 0 : (int)P.group_expert[g];
+                const int row = shared ? -1 : 2 * ((int)P.group_first[g] + slice_j0[slice]);
+                const int kblocks = ((shared ? a.I_s : a.I) + kGemmBK - 1) / kGemmBK;
+                if (gidx != ready_group) {
+                    if (!group_ready(gidx, shared ? a.I_s : a.I)) {
+                        stop = true;
+                        break;
+                    }
+                    // the h boxes are read by the copy engine (async proxy)
+                    asm volatile("fence.proxy.async.global;" ::: "memory");
+                    ready_group = gidx;
+                }
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+                        stop = true;
+                        break;
+                    }
+                    uint8_t *sa = smem + stage * kTcStageBytes;
+                    uint8_t *sb = sa + kTcABytes;
+                    const int k0 = kb * kGemmBK;
+                    mbar_arrive_expect_tx(&full[stage], kTcStageBytes);
+                    if (shared) {
+                        tma_load_2d(sa, &maps.sd, k0, mb * kGemmBM, &full[stage], pol_w);
+                        tma_load_2d(sb, &maps.hs, k0, 0, &full[stage], pol_h);
+                    } else {
+                        tma_load_3d(sa, &maps.wd, k0, mb * kGemmBM, e, &full[stage], pol_w);
+                        tma_load_2d(sb, &maps.hr, k0, row, &full[stage], pol_h);
+                    }
+                    ++issued;
+                    if (++stage == kTcStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // no copy may still be landing in shared memory when the CTA exits
+            for (int n = issued > kTcStages ? issued - kTcStages : 0; n < issued; ++n)
+                mbar_wait(&full[n % kTcStages], (uint32_t)(n / kTcStages) & 1u, nullptr);
+        } else if (a.grp_done == nullptr && elect_one()) {
             const uint64_t pol_w = policy_evict_first();
             const uint64_t pol_h = policy_evict_last();
             uint32_t stage = 0, phase = 0;
@@ -593,7 +744,7 @@ stream_down_tc_kernel(const __grid_constant__ DtMaps maps, const DtArgs a) {
             umma_commit(drain);
             mbar_wait(drain, 0, nullptr);
         }
-    } else {
+    } else if (warp < 6) {
         // ------------------------------------------------ plan, then epilogue
         const int ltid = (int)threadIdx.x - 64;
         // ids and weights come from the kernel before the previous one, which
@@ -613,7 +764,12 @@ stream_down_tc_kernel(const __grid_constant__ DtMaps maps, const DtArgs a) {
             *n_slices = sl;
             mbar_arrive(planbar);  // release: the plan and the slice table are written
         }
-        grid_dependency_wait();  // before any output is written
+        // Without the completion words, nothing is written before the gate/up
+        // kernel has completed.  With them, the outputs c and s are read only
+        // by the next kernel, and their earlier readers (the previous call's)
+        // completed before this call's router did.
+        if (a.grp_done == nullptr)
+            grid_dependency_wait();
         if (mbar_wait(planbar, 0, abort_flag)) {
             const int q = warp & 3;  // TMEM lane quarter this warp may access
             const int total = (has_shared + *n_slices) * n_mb;

@@ -214,6 +214,7 @@ struct Workspace {
     // streaming path (T <= 8): fp32 h for the CUDA-core down projection, bf16
     // hi/lo rows ([2 T k + 16][I], [16][I_s]) for the tensor-core one
     size_t h_routed = 0, h_shared = 0, hb_routed = 0, hb_shared = 0;
+    size_t grp_done = 0;  // per-group completion words between the decode kernels
     // tensor path
     epk::GroupedWorkspace grouped;
     size_t total = 0;
@@ -231,6 +232,8 @@ Workspace workspace_layout(int64_t T, int64_t H, int64_t E, int64_t k, int64_t I
         o = align256(o + (size_t)(2 * T * k + 2 * epk::kTcSlice) * I * 2);
         w.hb_shared = o;
         o = align256(o + (size_t)2 * epk::kTcSlice * I_s * 2);
+        w.grp_done = o;
+        o = align256(o + (size_t)8 * epk::kTcMaxGroups);
     }
     w.grouped = epk::grouped_workspace_layout(o, T, H, E, k, I, I_s);
     o = align256(w.grouped.end);
@@ -757,6 +760,13 @@ ep_status ffn_forward_impl(bool band_call, const void *x, ep_dtype x_dtype, int6
             ta.h_shared = ga.h_shared;
             ta.hb_routed = reinterpret_cast<uint16_t *>(ws + W.hb_routed);
             ta.hb_shared = I_s > 0 ? reinterpret_cast<uint16_t *>(ws + W.hb_shared) : nullptr;
+            // the call's epoch for the group completion words (1 .. 2^48 - 1)
+            static std::atomic<unsigned long long> epoch_counter{0};
+            unsigned long long epoch = 0;
+            while (epoch == 0)
+                epoch = (epoch_counter.fetch_add(1) + 1) & ((1ull << 48) - 1);
+            ta.grp_done = reinterpret_cast<unsigned long long *>(ws + W.grp_done);
+            ta.epoch = epoch;
             ta.pf[0] = ws_gate;
             ta.pf[1] = ws_up;
             ta.pf[2] = ws_down;
@@ -790,6 +800,8 @@ ep_status ffn_forward_impl(bool band_call, const void *x, ep_dtype x_dtype, int6
             dta.weights = weights;
             dta.c = reinterpret_cast<float *>(ws + W.grouped.c);
             dta.s = reinterpret_cast<float *>(ws + W.grouped.s);
+            dta.grp_done = ta.grp_done;
+            dta.epoch = ta.epoch;
             {
                 KernelBracket kb1(st, 1);
                 EP_CUDA_CHECK(launch(epk::stream_down_tc_kernel, gu_grid, epk::kTcThreads,
