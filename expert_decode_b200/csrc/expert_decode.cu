@@ -220,6 +220,16 @@ struct Workspace {
     size_t total = 0;
 };
 
+// A call's number for the decode kernels' group completion words: 1 .. 2^48 - 1,
+// never twice in a row on the same workspace.
+unsigned long long next_epoch() {
+    static std::atomic<unsigned long long> counter{0};
+    unsigned long long e = 0;
+    while (e == 0)
+        e = (counter.fetch_add(1) + 1) & ((1ull << 48) - 1);
+    return e;
+}
+
 Workspace workspace_layout(int64_t T, int64_t H, int64_t E, int64_t k, int64_t I, int64_t I_s) {
     Workspace w;
     size_t o = 0;
@@ -760,13 +770,8 @@ ep_status ffn_forward_impl(bool band_call, const void *x, ep_dtype x_dtype, int6
             ta.h_shared = ga.h_shared;
             ta.hb_routed = reinterpret_cast<uint16_t *>(ws + W.hb_routed);
             ta.hb_shared = I_s > 0 ? reinterpret_cast<uint16_t *>(ws + W.hb_shared) : nullptr;
-            // the call's epoch for the group completion words (1 .. 2^48 - 1)
-            static std::atomic<unsigned long long> epoch_counter{0};
-            unsigned long long epoch = 0;
-            while (epoch == 0)
-                epoch = (epoch_counter.fetch_add(1) + 1) & ((1ull << 48) - 1);
             ta.grp_done = reinterpret_cast<unsigned long long *>(ws + W.grp_done);
-            ta.epoch = epoch;
+            ta.epoch = next_epoch();
             ta.pf[0] = ws_gate;
             ta.pf[1] = ws_up;
             ta.pf[2] = ws_down;
