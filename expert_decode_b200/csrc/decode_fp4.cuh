@@ -389,9 +389,7 @@ struct F4GuArgs {
 
 struct F4Smem {
     static constexpr uint32_t misc = kF4Misc;  // tmem holder, abort flag
-    static constexpr uint32_t tile_first = misc + 16;
-    static constexpr uint32_t row_first = tile_first + (kTcMaxGroups + 1) * 4;
-    static constexpr uint32_t xchg = (row_first + kTcMaxGroups * 4 + 15) / 16 * 16;
+    static constexpr uint32_t xchg = (misc + 16 + 15) / 16 * 16;
     static constexpr uint32_t plan = (xchg + 2 * 2 * kStreamMaxT * 32 * 4 + 127) / 128 * 128;
     static constexpr uint32_t total = plan + (uint32_t)sizeof(StreamPlan);
     static constexpr uint32_t alloc = total + 1024;
@@ -405,8 +403,6 @@ stream_gate_up_fp4_kernel(const __grid_constant__ F4GuMaps maps, const F4GuArgs 
     const F4Bars B(smem);
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + F4Smem::misc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + F4Smem::misc + 8);
-    int *tile_first = reinterpret_cast<int *>(smem + F4Smem::tile_first);
-    int *row_first = reinterpret_cast<int *>(smem + F4Smem::row_first);
     float *xchg = reinterpret_cast<float *>(smem + F4Smem::xchg);
     StreamPlan &P = *reinterpret_cast<StreamPlan *>(smem + F4Smem::plan);
 
@@ -431,18 +427,20 @@ stream_gate_up_fp4_kernel(const __grid_constant__ F4GuMaps maps, const F4GuArgs 
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_holder;
 
+    // tiles of kGateUpRows units: the shared expert's first, then each routed
+    // group's, every routed group being I units wide
+    const int tiles_s = has_shared ? (a.I_s + kGateUpRows - 1) / kGateUpRows : 0;
+    const int tiles_r = (a.I + kGateUpRows - 1) / kGateUpRows;
+    auto n_tiles = [&]() { return tiles_s + P.n_groups * tiles_r; };
     auto decode = [&](int u, int &gi, int &m0) {
-        const int G = has_shared + P.n_groups;
-        int lo = 0, hi = G - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (tile_first[mid] <= u)
-                lo = mid;
-            else
-                hi = mid - 1;
+        if (u < tiles_s) {
+            gi = 0;
+            m0 = u * kGateUpRows;
+        } else {
+            const int v = u - tiles_s, g = v / tiles_r;
+            gi = has_shared + g;
+            m0 = (v - g * tiles_r) * kGateUpRows;
         }
-        gi = lo;
-        m0 = (u - tile_first[gi]) * kGateUpRows;
     };
     const int kblocks = (a.H + kGemmBK - 1) / kGemmBK;
     const int n_st = f4_stages_of(kblocks);
@@ -456,7 +454,7 @@ stream_gate_up_fp4_kernel(const __grid_constant__ F4GuMaps maps, const F4GuArgs 
             uint32_t stage = 0, phase = 0;
             int issued = 0;
             bool stop = !mbar_wait(B.planbar, 0, abort_flag);
-            const int total = stop ? 0 : tile_first[has_shared + P.n_groups];
+            const int total = stop ? 0 : n_tiles();
             for (int u = blockIdx.x; u < total && !stop; u += gridDim.x) {
                 int gi, m0;
                 decode(u, gi, m0);
@@ -497,7 +495,7 @@ stream_gate_up_fp4_kernel(const __grid_constant__ F4GuMaps maps, const F4GuArgs 
         // ------------------------------------------------------ MMA issuer
         if (elect_one()) {
             const bool planned = mbar_wait(B.planbar, 0, abort_flag);
-            const int total = planned ? tile_first[has_shared + P.n_groups] : 0;
+            const int total = planned ? n_tiles() : 0;
             f4_mma_loop(smem, B.full, B.empty, B.afull, B.aempty, B.tfull, B.tempty, abort_flag,
                         tmem_base, total, [&](int) { return kblocks; });
             umma_commit(B.drain);
@@ -508,7 +506,7 @@ stream_gate_up_fp4_kernel(const __grid_constant__ F4GuMaps maps, const F4GuArgs 
         int r, h;  // row of the A tile, half of its k block
         dequant_row_of(warp, lane, r, h);
         const bool planned = mbar_wait(B.planbar, 0, abort_flag);
-        const int total = planned ? tile_first[has_shared + P.n_groups] : 0;
+        const int total = planned ? n_tiles() : 0;
         // the row's unit and its scale row (zeros past the matrix)
         auto row_of = [&](int u, const uint32_t *&p, int &kbn) {
             int gi, m0;
@@ -535,26 +533,15 @@ stream_gate_up_fp4_kernel(const __grid_constant__ F4GuMaps maps, const F4GuArgs 
         grid_dependency_wait();  // ids and weights may come from the previous kernel
         grid_dependents_launch();
         build_stream_plan(P, a.ids, a.weights, a.T, a.top_k, a.E, ltid, 128, kTcBarPlan);
-        if (ltid == 0) {
-            const int G = has_shared + P.n_groups;
-            int t = 0;
-            for (int gi = 0; gi < G; ++gi) {
-                tile_first[gi] = t;
-                const int width = gi < has_shared ? a.I_s : a.I;
-                t += (width + kGateUpRows - 1) / kGateUpRows;
-            }
-            tile_first[G] = t;
-            for (int g = 0; g < P.n_groups; ++g)
-                row_first[g] = 2 * P.group_first[g];
-            mbar_arrive(B.planbar);
-        }
+        if (ltid == 0)
+            mbar_arrive(B.planbar);  // release: the plan is written
         const bool planned =
             named_count(kTcBarPlan, 128, mbar_wait(B.planbar, 0, abort_flag)) == 128;
         if (planned) {
             const int q = warp & 3;
             const bool gate_warp = q < 2;
             const int pair = q & 1;
-            const int total = tile_first[has_shared + P.n_groups];
+            const int total = n_tiles();
             uint32_t acc = 0, acc_phase = 0;
             for (int u = blockIdx.x; u < total; u += gridDim.x) {
                 int gi, m0;
@@ -601,7 +588,7 @@ stream_gate_up_fp4_kernel(const __grid_constant__ F4GuMaps maps, const F4GuArgs 
                             const float hv = silu_f32(ts * mv) * xb[tok * 32 + lane];
                             const int j0 = j / kTcSlice * kTcSlice;
                             const int n = min(kTcSlice, cnt - j0);
-                            const size_t b = (size_t)row_first[g] + 2 * j0;
+                            const size_t b = 2 * (size_t)first + 2 * j0;  // 2 rows (hi, lo) per pick
                             uint16_t *hb = a.hb_routed + unit;
                             store_hi_lo_f16(hb + (b + (j - j0)) * a.I,
                                             hb + (b + n + (j - j0)) * a.I, hv);

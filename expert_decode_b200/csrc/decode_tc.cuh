@@ -130,10 +130,8 @@ struct TcSmem {
     // full[S], empty[S], tfull[2], tempty[2], drain, planbar, hdone[2],
     // hfree[2]; tmem holder, abort flag
     static constexpr uint32_t misc = bars + (2 * kTcStages + 10) * 8;
-    static constexpr uint32_t tile_first = misc + 16;  // [kTcMaxGroups + 1]
-    static constexpr uint32_t row_first = tile_first + (kTcMaxGroups + 1) * 4;  // [kTcMaxGroups]
     // up values handed to the gate warps: [pair][accumulator][token][lane]
-    static constexpr uint32_t xchg = (row_first + kTcMaxGroups * 4 + 15) / 16 * 16;
+    static constexpr uint32_t xchg = (misc + 16 + 15) / 16 * 16;
     static constexpr uint32_t plan = (xchg + 2 * 2 * kStreamMaxT * 32 * 4 + 127) / 128 * 128;
     static constexpr uint32_t total = plan + (uint32_t)sizeof(StreamPlan);
     static constexpr uint32_t alloc = total + 1024;  // room to align the base to 1024
@@ -164,8 +162,6 @@ stream_gate_up_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     uint64_t *hfree = hdone + 2;    // [2]: the publisher has taken hdone's phase
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + TcSmem::misc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + TcSmem::misc + 8);
-    int *tile_first = reinterpret_cast<int *>(smem + TcSmem::tile_first);
-    int *row_first = reinterpret_cast<int *>(smem + TcSmem::row_first);  // per routed group
     float *xchg = reinterpret_cast<float *>(smem + TcSmem::xchg);
     StreamPlan &P = *reinterpret_cast<StreamPlan *>(smem + TcSmem::plan);
 
@@ -205,20 +201,21 @@ stream_gate_up_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_holder;
 
-    // tile u -> (group index gi, first unit m0); gi = 0 is the shared expert
-    // when there is one
+    // tile u -> (group index gi, first unit m0): tiles of kGateUpRows units,
+    // the shared expert's first (gi = 0, when there is one), then each routed
+    // group's, every routed group being I units wide
+    const int tiles_s = has_shared ? (a.I_s + kGateUpRows - 1) / kGateUpRows : 0;
+    const int tiles_r = (a.I + kGateUpRows - 1) / kGateUpRows;
+    auto n_tiles = [&]() { return tiles_s + P.n_groups * tiles_r; };
     auto decode = [&](int u, int &gi, int &m0) {
-        const int G = has_shared + P.n_groups;
-        int lo = 0, hi = G - 1;
-        while (lo < hi) {  // largest gi with tile_first[gi] <= u
-            const int mid = (lo + hi + 1) >> 1;
-            if (tile_first[mid] <= u)
-                lo = mid;
-            else
-                hi = mid - 1;
+        if (u < tiles_s) {
+            gi = 0;
+            m0 = u * kGateUpRows;
+        } else {
+            const int v = u - tiles_s, g = v / tiles_r;
+            gi = has_shared + g;
+            m0 = (v - g * tiles_r) * kGateUpRows;
         }
-        gi = lo;
-        m0 = (u - tile_first[gi]) * kGateUpRows;
     };
 
     if (warp == 0) {
@@ -230,7 +227,7 @@ stream_gate_up_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
             uint32_t stage = 0, phase = 0;
             int issued = 0;
             bool stop = !mbar_wait(planbar, 0, abort_flag);
-            const int total = stop ? 0 : tile_first[has_shared + P.n_groups];
+            const int total = stop ? 0 : n_tiles();
             const int kblocks = (a.H + kGemmBK - 1) / kGemmBK;
             for (int u = blockIdx.x; u < total && !stop; u += gridDim.x) {
                 int gi, m0;
@@ -273,7 +270,7 @@ stream_gate_up_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
             uint32_t stage = 0, phase = 0;
             uint32_t acc = 0, acc_phase = 0;
             bool stop = !mbar_wait(planbar, 0, abort_flag);
-            const int total = stop ? 0 : tile_first[has_shared + P.n_groups];
+            const int total = stop ? 0 : n_tiles();
             const int kblocks = (a.H + kGemmBK - 1) / kGemmBK;
             const uint32_t idesc = idesc_bf16_f32(kGemmBM, kTcN);
             for (int u = blockIdx.x; u < total && !stop; u += gridDim.x) {
@@ -320,7 +317,7 @@ stream_gate_up_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
         // would hold both warps of a pair.
         if (a.grp_done != nullptr && elect_one()) {
             const bool planned = mbar_wait(planbar, 0, abort_flag);
-            const int total = planned ? tile_first[has_shared + P.n_groups] : 0;
+            const int total = planned ? n_tiles() : 0;
             uint32_t acc = 0, acc_phase = 0;
             for (int u = blockIdx.x; u < total; u += gridDim.x) {
                 int gi, m0;
@@ -344,19 +341,8 @@ stream_gate_up_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
         // passed its wait, so that it may read the ids (and x) before its own
         grid_dependents_launch();
         build_stream_plan(P, a.ids, a.weights, a.T, a.top_k, a.E, ltid, 128, kTcBarPlan);
-        if (ltid == 0) {
-            const int G = has_shared + P.n_groups;
-            int t = 0;
-            for (int gi = 0; gi < G; ++gi) {
-                tile_first[gi] = t;
-                const int width = gi < has_shared ? a.I_s : a.I;
-                t += (width + kGateUpRows - 1) / kGateUpRows;
-            }
-            tile_first[G] = t;
-            for (int g = 0; g < P.n_groups; ++g)
-                row_first[g] = 2 * P.group_first[g];  // 2 rows (hi, lo) per pick
-            mbar_arrive(planbar);  // release: the plan and the tile tables are written
-        }
+        if (ltid == 0)
+            mbar_arrive(planbar);  // release: the plan is written
         // the planning warps agree on the plan wait, so the pairs below either
         // all enter the tile loop or none does
         const bool planned =
@@ -366,7 +352,7 @@ stream_gate_up_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
             // quarters 0, 1: gate rows of units 0..31, 32..63; 2, 3: their up rows
             const bool gate_warp = q < 2;
             const int pair = q & 1;
-            const int total = tile_first[has_shared + P.n_groups];
+            const int total = n_tiles();
             uint32_t acc = 0, acc_phase = 0;
             for (int u = blockIdx.x; u < total; u += gridDim.x) {
                 int gi, m0;
@@ -417,7 +403,7 @@ stream_gate_up_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
                             if (a.hb_routed != nullptr) {
                                 const int j0 = j / kTcSlice * kTcSlice;
                                 const int n = min(kTcSlice, cnt - j0);
-                                const size_t b = (size_t)row_first[g] + 2 * j0;
+                                const size_t b = 2 * (size_t)first + 2 * j0;  // 2 rows (hi, lo) per pick
                                 uint16_t *hb = a.hb_routed + unit;
                                 store_hi_lo(hb + (b + (j - j0)) * a.I,
                                             hb + (b + n + (j - j0)) * a.I, h);

@@ -62,14 +62,19 @@ struct StreamPlan {
 
 // Built from ids (<= 128 picks) by `nthr` (>= 128) threads with local ids
 // ltid, synchronised on named barrier `bar`; sort key (expert, repeat, token).
+// Each valid pick finds its rank and whether it is its token's first pick in
+// one pass over the keys, and writes its own row of the sorted tables.
 __device__ void build_stream_plan(StreamPlan &P, const int32_t *__restrict__ ids,
                                   const float *__restrict__ weights, int T, int k, int E,
                                   int ltid, uint32_t nthr, uint32_t bar) {
     const int np = T * k;
-    int key = 0x7fffffff;
+    int key = 0x7fffffff, t = 0;
+    float w = 0.f;
     if (ltid < np) {
         const int e = ids[ltid];
-        const int t = ltid / k, j = ltid - t * k;
+        w = weights[ltid];  // in flight with the id
+        t = ltid / k;
+        const int j = ltid - t * k;
         if (e >= 0 && e < E) {
             int rep = 0;
             for (int q = 0; q < j; ++q)
@@ -81,13 +86,27 @@ __device__ void build_stream_plan(StreamPlan &P, const int32_t *__restrict__ ids
     }
     if (ltid < kStreamMaxPairs)
         P.keys[ltid] = key;
-    const int nvalid = named_count(bar, nthr, ltid < np && key != 0x7fffffff);
-    if (ltid < np && key != 0x7fffffff) {
+    if (ltid < T)
+        P.token_has_pick[ltid] = 0;
+    const bool valid = ltid < np && key != 0x7fffffff;
+    const int nvalid = named_count(bar, nthr, valid);
+    if (valid) {
         int r = 0;
-        for (int q = 0; q < np; ++q)
-            r += P.keys[q] < key;
+        bool first = true;  // no smaller key of the same token
+#pragma unroll 4
+        for (int q = 0; q < np; ++q) {
+            const int kq = P.keys[q];
+            const bool below = kq < key;
+            r += below;
+            first &= !(below && kq % kStreamMaxT == t);
+        }
         P.sorted_key[r] = key;
         P.sorted_src[r] = ltid;
+        P.pair_token[r] = (int8_t)t;
+        P.pair_weight[r] = w;
+        P.pair_is_first[r] = first;
+        if (first)
+            P.token_has_pick[t] = 1;
     }
     named_sync(bar, nthr);
     if (ltid < 32) {
@@ -110,22 +129,6 @@ __device__ void build_stream_plan(StreamPlan &P, const int32_t *__restrict__ ids
             P.group_first[base] = (int16_t)nvalid;
             P.n_pairs = nvalid;
         }
-    }
-    if (ltid < nvalid) {
-        const int src = P.sorted_src[ltid];
-        const int t = src / k;
-        P.pair_token[ltid] = (int8_t)t;
-        P.pair_weight[ltid] = weights[src];
-        bool first = true;
-        for (int q = 0; q < ltid; ++q)
-            first &= (P.sorted_key[q] % kStreamMaxT) != t;
-        P.pair_is_first[ltid] = first;
-    }
-    if (ltid < T) {
-        bool has = false;
-        for (int q = 0; q < nvalid; ++q)
-            has |= (P.sorted_key[q] % kStreamMaxT) == ltid;
-        P.token_has_pick[ltid] = has;
     }
     named_sync(bar, nthr);
 }
