@@ -360,6 +360,13 @@ __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
                  "barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+// The shared::cluster address, in CTA `rank` of the cluster, of this CTA's
+// shared-memory address `addr`.
+__device__ __forceinline__ uint32_t remote_shared(uint32_t addr, uint32_t rank) {
+    uint32_t out;
+    asm("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(addr), "r"(rank));
+    return out;
+}
 // Address of the same shared variable in CTA `rank` of the cluster.
 __device__ __forceinline__ uint32_t map_shared_rank(const void *p, uint32_t rank) {
     uint32_t out;

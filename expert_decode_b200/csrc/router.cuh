@@ -33,10 +33,50 @@ __device__ __forceinline__ void unpack_w8(uint4 v, float (&wf)[8]) {
     wf[4] = bf16_lo(v.z); wf[5] = bf16_hi(v.z); wf[6] = bf16_lo(v.w); wf[7] = bf16_hi(v.w);
 }
 
-// Index of the k-th largest fp32 logit of one token (ties to the lower id),
-// computed by a warp; `chosen` keeps the picked lanes' bits.
+// The k-th largest fp32 logit of one token (counted with multiplicity; NaN
+// never counts), computed by a warp.  Up to 256 experts the logits sit in
+// registers as order-preserving 32-bit keys (NaN and empty slots 0): each
+// round takes the warp's largest key and how many lanes' keys equal it by two
+// warp reductions, and clears them, until top_k are counted.  Above 256 the
+// logits are re-read each round.
+__device__ __forceinline__ uint32_t order_key(float v) {
+    const uint32_t b = __float_as_uint(v);
+    return v != v ? 0u : ((b & 0x80000000u) ? ~b : (b | 0x80000000u));
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
 __device__ float kth_logit(const float *lt, int E, int top_k) {
     const int lane = (int)lane_id();
+    if (E <= 256) {
+        uint32_t key[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int e = lane + 32 * i;
+            key[i] = e < E ? order_key(lt[e]) : 0u;
+        }
+        int counted = 0;
+        for (int r = 0; r < top_k; ++r) {
+            uint32_t m = key[0];
+#pragma unroll
+            for (int i = 1; i < 8; ++i)
+                m = max(m, key[i]);
+            m = __reduce_max_sync(0xffffffffu, m);
+            if (m == 0u)
+                return -INFINITY;  // fewer than top_k orderable logits
+            uint32_t c = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                c += key[i] == m ? 1u : 0u;
+                key[i] = key[i] == m ? 0u : key[i];
+            }
+            counted += (int)__reduce_add_sync(0xffffffffu, c);
+            if (counted >= top_k)
+                return key_value(m);
+        }
+        return -INFINITY;
+    }
     const int per_lane = (E + 31) / 32;  // <= 32
     uint32_t chosen = 0;
     float vk = -INFINITY;
@@ -614,14 +654,15 @@ __device__ void router_pick_owned(int n_local, int tbase, int tstride, int64_t t
         float dmax = 0.f;
         for (int e = lane; e < E; e += 32)
             dmax = fmaxf(dmax, bound_at(j, e));
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
-            dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, off));
-        const double thr = (double)vk - 2.0 * (double)dmax * 1.0001;
+        // bounds are positive (or NaN, dropped by fmaxf): their bits order as integers
+        dmax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(dmax)));
+        // the largest float not above the threshold: the same experts pass,
+        // and at most those equal to it besides
+        const float thr = __double2float_rd((double)vk - 2.0 * (double)dmax * 1.0001);
         int count = 0;
         for (int i = 0; i < (E + 31) / 32; ++i) {
             const int e = lane + 32 * i;
-            const bool c = e < E && (double)lt[e] >= thr;
+            const bool c = e < E && lt[e] >= thr;
             const uint32_t m = __ballot_sync(0xffffffffu, c);
             const int pos = count + __popc(m & ((1u << lane) - 1u));
             if (c && pos < max_cand)
@@ -635,7 +676,8 @@ __device__ void router_pick_owned(int n_local, int tbase, int tstride, int64_t t
 
     // Dot2 logits of the owned tokens' candidates, spread over the warps in
     // groups of up to NG candidates of one token (one warp refines a group
-    // at once: its rows stream side by side)
+    // at once: its rows stream side by side; a short group's missing rows
+    // add zeros, cheaper than more code variants in the instruction cache)
     {
         constexpr int NG = XF32 ? 2 : 4;
         int mine = 0;
@@ -673,7 +715,44 @@ __device__ void router_pick_owned(int n_local, int tbase, int tstride, int64_t t
         const int nc = ncand[j];
         double bv_list = 0.0, top = 0.0, bs_list = 0.0;  // lane r: the r-th pick's value, score
         int be_list = 0;
-        if (nc <= max_cand) {
+        if (nc <= 32 && nc <= max_cand) {
+            // lane ci holds candidate ci; its rank among the orderable ones
+            // (larger value first, ties to the lower id; NaN never picked)
+            // sends it to slot rank of the token's lists
+            const int base = j * max_cand;
+            const bool ok0 = lane < nc;
+            const double v = ok0 ? cval[base + lane] : 0.0;
+            const int e = ok0 ? cand[base + lane] : 0x7fffffff;
+            const double sc = (SIG && ok0) ? cscore[base + lane] : 0.0;
+            const bool ok = ok0 && v == v;
+            int rank = 0;
+            for (int q = 0; q < nc; ++q) {
+                const double ov = __shfl_sync(0xffffffffu, v, q);
+                const int oe = __shfl_sync(0xffffffffu, e, q);
+                rank += (ov > v || (ov == v && oe < e)) ? 1 : 0;  // NaN ov: false
+            }
+            const int n_ok = __popc(__ballot_sync(0xffffffffu, ok));
+            __syncwarp();
+            if (ok && rank < top_k) {
+                cval[base + rank] = v;
+                cand[base + rank] = e;
+                if (SIG)
+                    cscore[base + rank] = sc;
+            }
+            __syncwarp();
+            if (lane < top_k) {
+                if (lane < n_ok) {
+                    bv_list = cval[base + lane];
+                    be_list = cand[base + lane];
+                    if (SIG)
+                        bs_list = cscore[base + lane];
+                } else {
+                    bv_list = -INFINITY;
+                    be_list = 0x7fffffff;
+                }
+            }
+            top = __shfl_sync(0xffffffffu, bv_list, 0);
+        } else if (nc <= max_cand) {
             uint32_t chosen = 0;
             for (int r = 0; r < top_k; ++r) {
                 double bv = -INFINITY;

@@ -13,10 +13,12 @@
 //    fp32 TMEM accumulators; warps 2..7 add up, from the same shared-memory
 //    stages, each expert's and each token's sum of squares over the slice
 //    (a row's sum does not depend on the swizzle's order of its chunks).
-//  * Warps 2..5 drain the accumulators (tcgen05.ld) into a [token][expert]
-//    tile; the CK partial tiles are added in ascending slice order over
-//    distributed shared memory by the CTA that owns the token (CK owners per
-//    tile, 64 / CK tokens each), which also forms its error bound.
+//  * Once every CTA of the cluster has finished its slice, warps 2..5 drain
+//    the accumulators (tcgen05.ld) and push each token's partial row, and
+//    every CTA its sums of squares, into the shared memory of the CTA that
+//    owns the token (CK owners per tile, 64 / CK tokens each; stores over
+//    distributed shared memory, no remote loads).  The owner adds the CK
+//    partials in ascending slice order and forms the error bounds.
 //  * The owner then picks as router_tiled_kernel does (router_pick_owned):
 //    every expert that could reach the k-th largest under the bounds is
 //    recomputed by Dot2 and the pick and the weights are made on those
@@ -55,13 +57,16 @@ struct RcMaps {
     CUtensorMap x;  // x [T, H]: box 64 x 64
 };
 
-// Shared memory: the stage ring, later reused for the partial tile, the
-// norms, and the owned tokens' logits, bounds and candidates.
+// Shared memory: the stage ring, later reused for the partials pushed to
+// this CTA by the cluster (its owned tokens' rows from every slice, and every
+// slice's sums of squares), then the owned tokens' logits and bounds (in place
+// of slices 0 and 1) and candidates.  The row sums of squares of this CTA's
+// own slice wait beyond the ring (nsq) until the ring may be written.
 struct RcSmem {
     uint32_t stage_bytes, stages, ring;            // ring = stages * stage_bytes
-    uint32_t part, xsq, wsq;                       // read by the cluster's other CTAs
-    uint32_t logit, bound, xn, wn, ncand, cand, cval, cscore, end;  // this CTA's only
-    uint32_t bars, total, alloc;
+    uint32_t recv, wsq, xsq;                       // written by the cluster's CTAs
+    uint32_t xn, wn, ncand, cand, cval, cscore, end;  // this CTA's only
+    uint32_t bars, nsq, pbase, total, alloc;
 };
 
 __host__ __device__ inline RcSmem rc_smem_layout(int MT, int E, int CK) {
@@ -73,11 +78,9 @@ __host__ __device__ inline RcSmem rc_smem_layout(int MT, int E, int CK) {
     s.ring = s.stages * s.stage_bytes;
     const uint32_t own = (kRcNT + CK - 1) / CK;  // tokens a CTA owns at most
     uint32_t o = 0;
-    s.part = o;   o = align_up_u32(o + (uint32_t)kRcNT * E * 4, 16);
-    s.xsq = o;    o = align_up_u32(o + (uint32_t)kRcNT * 4, 16);
-    s.wsq = o;    o = align_up_u32(o + (uint32_t)E * 4, 16);
-    s.logit = o;  o = align_up_u32(o + own * E * 4, 16);
-    s.bound = o;  o = align_up_u32(o + own * E * 4, 16);
+    s.recv = o;   o = align_up_u32(o + (uint32_t)CK * own * E * 4, 16);  // [CK][own][E]
+    s.wsq = o;    o = align_up_u32(o + (uint32_t)CK * E * 4, 16);        // [CK][E]
+    s.xsq = o;    o = align_up_u32(o + (uint32_t)CK * own * 4, 16);      // [CK][own]
     s.xn = o;     o = align_up_u32(o + own * 4, 16);
     s.wn = o;     o = align_up_u32(o + (uint32_t)E * 4, 16);
     s.ncand = o;  o = align_up_u32(o + own * 4, 16);
@@ -87,7 +90,9 @@ __host__ __device__ inline RcSmem rc_smem_layout(int MT, int E, int CK) {
     s.end = o;
     s.bars = align_up_u32(s.ring > s.end ? s.ring : s.end, 1024);
     // full[S], empty[S], tdone; tmem holder, abort flag
-    s.total = s.bars + (2 * s.stages + 1) * 8 + 16;
+    s.nsq = align_up_u32(s.bars + (2 * s.stages + 1) * 8 + 16, 16);
+    s.pbase = s.nsq + (uint32_t)(MT * kGemmBM + kRcNT) * 4;  // nsq: [MT 128 + 64]
+    s.total = s.pbase + kRcMaxCK * 4;
     s.alloc = s.total + 1024;
     return s;
 }
@@ -109,11 +114,11 @@ router_tc_kernel(const __grid_constant__ RcMaps maps, const uint16_t *__restrict
     uint64_t *tdone = empty + L.stages;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(tdone + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tdone + 1) + 2;
-    float *part = reinterpret_cast<float *>(smem + L.part);    // [64][E]
-    float *xsq = reinterpret_cast<float *>(smem + L.xsq);      // [64]
-    float *wsq = reinterpret_cast<float *>(smem + L.wsq);      // [E]
-    float *logit = reinterpret_cast<float *>(smem + L.logit);  // [own][E]
-    float *bound = reinterpret_cast<float *>(smem + L.bound);  // [own][E]
+    float *recv = reinterpret_cast<float *>(smem + L.recv);    // [CK][own][E]
+    float *wsq = reinterpret_cast<float *>(smem + L.wsq);      // [CK][E]
+    float *xsq = reinterpret_cast<float *>(smem + L.xsq);      // [CK][own]
+    float *nsq = reinterpret_cast<float *>(smem + L.nsq);      // [MT 128 + 64]
+    uint32_t *pbase = reinterpret_cast<uint32_t *>(smem + L.pbase);  // [CK]
     float *xn = reinterpret_cast<float *>(smem + L.xn);        // [own] ||x_t||
     float *wn = reinterpret_cast<float *>(smem + L.wn);        // [E] ||w_e||
     int *ncand = reinterpret_cast<int *>(smem + L.ncand);
@@ -128,7 +133,18 @@ router_tc_kernel(const __grid_constant__ RcMaps maps, const uint16_t *__restrict
     const int nkb = (H + kGemmBK - 1) / kGemmBK;
     const int kb_lo = nkb * (int)rank / CK, kb_hi = nkb * ((int)rank + 1) / CK;
     const uint32_t tcols = MT * kRcNT <= 64 ? 64u : 128u;
+    const int own = (kRcNT + CK - 1) / CK;
+    float *logit = recv;            // [own][E], in place of slice 0's rows
+    float *bound = recv + own * E;  // [own][E], in place of slice 1's rows
+    bool have = false;              // the partial tile is in TMEM (warps 2..7)
 
+    if (warp == 0 && lane < CK) {
+        // where this CTA's rows of owner `lane` begin there, less the owner's
+        // first token's rows (so that token t of the tile adds t E floats)
+        const int lo = kRcNT * lane / CK;
+        pbase[lane] = remote_shared(smem_u32(recv) + (uint32_t)(rank * own * E) * 4, (uint32_t)lane) -
+                      (uint32_t)(lo * E) * 4;
+    }
     if (warp == 0 && lane == 0) {
         for (uint32_t s = 0; s < L.stages; ++s) {
             mbar_init(&full[s], 1);
@@ -248,29 +264,7 @@ router_tc_kernel(const __grid_constant__ RcMaps maps, const uint16_t *__restrict
                 phase ^= 1u;
             }
         }
-        // the partial tile out of TMEM: warps 2..5 hold lane quarters 2, 3, 0, 1
-        const bool have = mbar_wait(tdone, 0, abort_flag);
-        __syncwarp();
-        // the stages are free once every MMA and every copy has completed;
-        // the producer's final waits and tdone cover both
-        named_sync(1, kRcThreads - 64);
-        if (have && warp < 6) {
-            tc_fence_after_sync();
-            const int q = warp & 3;
-            for (int m = 0; m < MT; ++m) {
-                const int e = m * kGemmBM + 32 * q + lane;
-                for (int c0 = 0; c0 < kRcNT; c0 += 32) {
-                    uint32_t v[32];
-                    tmem_load_32cols(tmem_base + ((uint32_t)(32 * q) << 16) + m * kRcNT + c0, v);
-                    tmem_load_wait();
-                    if (e < E) {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            part[(c0 + j) * E + e] = __uint_as_float(v[j]);
-                    }
-                }
-            }
-        }
+        have = __all_sync(0xffffffffu, mbar_wait(tdone, 0, abort_flag));
         // a row's eight chunks sit in lanes 8 (l / 8) .. 8 (l / 8) + 7
 #pragma unroll
         for (int i = 0; i < kMaxQuads; ++i) {
@@ -279,15 +273,54 @@ router_tc_kernel(const __grid_constant__ RcMaps maps, const uint16_t *__restrict
             v += __shfl_xor_sync(0xffffffffu, v, 2);
             v += __shfl_xor_sync(0xffffffffu, v, 4);
             const int g = nw + kRcNormWarps * i;
-            const int r = 4 * g + (lane >> 3);
-            if (g < quads && (lane & 7) == 0) {
-                if (r < MT * kGemmBM) {
-                    if (r < E)
-                        wsq[r] = v;
-                } else {
-                    xsq[r - MT * kGemmBM] = v;
+            if (g < quads && (lane & 7) == 0)
+                nsq[4 * g + (lane >> 3)] = v;
+        }
+    }
+    // this CTA's stages are free (every copy landed, every MMA completed,
+    // every norm read done); after the cluster barrier every CTA's are, and
+    // the partials are pushed to the CTAs that own their tokens
+    tc_fence_before_sync();
+    __syncthreads();
+    cluster_sync();
+    tc_fence_after_sync();
+    // the owner of token t of the tile and t's row there
+    static_assert(kRcNT == 64, "owner_of divides by 64");
+    auto owner_of = [&](int t) { return (t * CK + CK - 1) >> 6; };
+    if (have && warp >= 2 && warp < 6) {
+        // warps 2..5 hold TMEM lane quarters 2, 3, 0, 1: expert e's partials
+        // of 32 tokens per load, each sent to row (rank, t - lo) of t's owner
+        const int q = warp & 3;
+        for (int m = 0; m < MT; ++m) {
+            const int e = m * kGemmBM + 32 * q + lane;
+            for (int c0 = 0; c0 < kRcNT; c0 += 32) {
+                uint32_t v[32];
+                tmem_load_32cols(tmem_base + ((uint32_t)(32 * q) << 16) + m * kRcNT + c0, v);
+                tmem_load_wait();
+                if (e < E) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int t = c0 + j;
+                        st_cluster_f32(pbase[owner_of(t)] + (uint32_t)(t * E + e) * 4,
+                                       __uint_as_float(v[j]));
+                    }
                 }
             }
+        }
+    }
+    // this slice's sums of squares: every expert's to every CTA, every
+    // token's to its owner
+    for (int i = threadIdx.x; i < E + kRcNT; i += kRcThreads) {
+        if (i < E) {
+            const float v = nsq[i];
+            const uint32_t addr = smem_u32(wsq + rank * E + i);
+            for (int o = 0; o < CK; ++o)
+                st_cluster_f32(remote_shared(addr, (uint32_t)o), v);
+        } else {
+            const int t = i - E, o = owner_of(t);
+            const int tl = t - kRcNT * o / CK;
+            st_cluster_f32(remote_shared(smem_u32(xsq + rank * own + tl), (uint32_t)o),
+                           nsq[MT * kGemmBM + t]);
         }
     }
     tc_fence_before_sync();
@@ -296,7 +329,7 @@ router_tc_kernel(const __grid_constant__ RcMaps maps, const uint16_t *__restrict
         tc_fence_after_sync();
         tmem_dealloc(tmem_base, tcols);
     }
-    cluster_sync();  // every CTA's partial tile and norms are in place
+    cluster_sync();  // every push has landed; no CTA's shared memory is written by another after this
 
     // The owner of tokens [64 rank / CK, 64 (rank + 1) / CK) adds the CK
     // partials of each (token, expert) in ascending slice order, then its
@@ -306,8 +339,7 @@ router_tc_kernel(const __grid_constant__ RcMaps maps, const uint16_t *__restrict
     for (int i = threadIdx.x; i < E + n_local; i += kRcThreads) {
         float s2 = 0.f;
         for (int r = 0; r < CK; ++r)
-            s2 += ld_cluster_f32(map_shared_rank(i < E ? wsq + i : xsq + own_lo + (i - E),
-                                                 (uint32_t)r));
+            s2 += i < E ? wsq[r * E + i] : xsq[r * own + (i - E)];
         if (i < E)
             wn[i] = sqrtf(s2);
         else
@@ -318,13 +350,14 @@ router_tc_kernel(const __grid_constant__ RcMaps maps, const uint16_t *__restrict
         const float u = 5.9604644775390625e-8f;  // 2^-24
         const float n_instr = (float)(4 * ((nkb + CK - 1) / CK));
         const float gam = 2.0f * n_instr * 1.9073486328125e-6f + (float)(CK + 2) * u;  // 2^-19
-        for (int idx = threadIdx.x; idx < n_local * E; idx += kRcThreads) {
-            const int j = idx / E, e = idx - j * E;
-            const int t = own_lo + j;
+        // thread (j0, e) takes tokens j0, j0 + js, ... of expert e
+        const int js = kRcThreads / E;  // >= 1: E <= 256
+        const int e = (int)threadIdx.x % E, j0 = (int)threadIdx.x / E;
+        const float b = (bias != nullptr && j0 < js) ? bias[e] : 0.f;
+        for (int j = j0 < js ? j0 : n_local; j < n_local; j += js) {
             float sum = 0.f;
             for (int r = 0; r < CK; ++r)
-                sum += ld_cluster_f32(map_shared_rank(part + t * E + e, (uint32_t)r));
-            const float b = bias != nullptr ? bias[e] : 0.f;
+                sum += recv[(r * own + j) * E + e];
             float l, d;
             if (SIG) {
                 // key = sigmoid(l) + b; the sigmoid's slope is at most 1/4, and
@@ -336,11 +369,11 @@ router_tc_kernel(const __grid_constant__ RcMaps maps, const uint16_t *__restrict
                 l = sum + b;
                 d = 1.5f * (gam * xn[j] * wn[e] + u * fabsf(l)) + 1e-30f;
             }
-            logit[j * E + e] = l;
-            bound[j * E + e] = d;
+            logit[j * E + e] = l;  // the element just read of slice 0
+            bound[j * E + e] = d;  // and of slice 1
         }
     }
-    cluster_sync();  // no shared memory of another CTA is read after this point
+    __syncthreads();
     if (dump_logit != nullptr) {
         // inspection (moe_route_logits): the fp32 logits and their bounds
         for (int idx = threadIdx.x; idx < n_local * E; idx += kRcThreads) {
