@@ -65,7 +65,7 @@ constexpr int kPlanWarps = kPlanThreads / 32;
 constexpr int kMaxGroups = 1025;
 
 struct GroupedWorkspace {
-    size_t group_offset = 0, perm_pair = 0, units_gu = 0, units_dn = 0;
+    size_t group_offset = 0, perm_pair = 0, units_gu = 0, units_dn = 0, chunk_count = 0;
     size_t x_perm = 0, h_perm = 0, h_shared = 0, c = 0, s = 0;
     size_t end = 0;
 };
@@ -81,6 +81,7 @@ inline GroupedWorkspace grouped_workspace_layout(size_t base, int64_t T, int64_t
     w.perm_pair = o;    o = g_align256(o + P * 4);
     w.units_gu = o;     o = g_align256(o + (size_t)(E + 2) * 4);
     w.units_dn = o;     o = g_align256(o + (size_t)(E + 2) * 4);
+    w.chunk_count = o;  o = g_align256(o + (P + kPlanThreads - 1) / kPlanThreads * (size_t)E * 4);
     w.x_perm = o;       o = g_align256(o + (P + (size_t)T) * H * 2);
     w.h_perm = o;       o = g_align256(o + P * I * 2);
     w.h_shared = o;     o = g_align256(o + (size_t)T * I_s * 2);
@@ -129,6 +130,12 @@ __device__ int block_exclusive_scan2(int &v0, int &v1, int *warp_sums) {
 }
 
 // ------------------------------------------------------------- group plan
+// The picks are grouped by expert in two launches over chunks of
+// kPlanThreads picks, one CTA per chunk: group_count_kernel counts each
+// chunk's picks per expert; group_plan_kernel then gives every CTA its
+// chunk's first row in each expert's group (the experts before it, plus the
+// same expert's picks in earlier chunks) and scatters the chunk stably, so
+// the grouped order is a stable sort of the picks by expert id.
 struct PlanArgs {
     const int32_t *ids;
     int64_t T, P;
@@ -137,12 +144,39 @@ struct PlanArgs {
     int32_t *perm_pair;     // [P]: permuted row -> pick index t * top_k + j
     int32_t *units_gu;      // [G + 1] exclusive prefix of gate/up tiles per group
     int32_t *units_dn;      // [G + 1] same for the down projection
+    int32_t *chunk_count;   // [chunks][E]: valid picks of expert e in chunk c
 };
+
+__global__ void __launch_bounds__(kPlanThreads, 1) group_count_kernel(const PlanArgs a) {
+    extern __shared__ __align__(16) int hist[];  // [E]
+    grid_dependents_launch();
+    grid_dependency_wait();  // ids come from the router
+    const int E = a.E, lane = threadIdx.x & 31;
+    for (int e = threadIdx.x; e < E; e += kPlanThreads)
+        hist[e] = 0;
+    __syncthreads();
+    const int64_t p = (int64_t)blockIdx.x * kPlanThreads + threadIdx.x;
+    int e = -1;
+    bool valid = false;
+    if (p < a.P) {
+        e = a.ids[p];
+        valid = e >= 0 && e < E;
+        if (!valid && e != kIdNone)
+            flag_status(kStatusBadId);
+    }
+    const int key = valid ? e : -(lane + 2);
+    const uint32_t m = __match_any_sync(0xffffffffu, key);
+    if (valid && lane == __ffs(m) - 1)
+        atomicAdd(&hist[e], __popc(m));
+    __syncthreads();
+    for (int f = threadIdx.x; f < E; f += kPlanThreads)
+        a.chunk_count[(size_t)blockIdx.x * E + f] = hist[f];
+}
 
 __global__ void __launch_bounds__(kPlanThreads, 1) group_plan_kernel(const PlanArgs a) {
     extern __shared__ __align__(1024) uint8_t smem[];
     grid_dependents_launch();
-    grid_dependency_wait();  // ids come from the router; the workspace from earlier kernels
+    grid_dependency_wait();  // the chunk counts come from group_count_kernel
     int *cnt = reinterpret_cast<int *>(smem);            // [kPlanWarps][E]
     int *total = cnt + kPlanWarps * a.E;                 // [E]
     int *goff = total + a.E;                             // [E]
@@ -150,64 +184,77 @@ __global__ void __launch_bounds__(kPlanThreads, 1) group_plan_kernel(const PlanA
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int E = a.E;
     const int64_t P = a.P;
-    const int64_t per_warp = (((P + kPlanWarps - 1) / kPlanWarps) + 31) / 32 * 32;
-    const int64_t p_lo = (int64_t)warp * per_warp;
-    const int64_t p_hi = min(P, p_lo + per_warp);
+    const int chunk = (int)blockIdx.x, n_chunks = (int)gridDim.x;
+    // this chunk's picks, 32 per warp, in pick order
+    const int64_t p_lo = (int64_t)chunk * kPlanThreads + 32 * warp;
+    const int64_t p_hi = min(P, p_lo + 32);
 
     for (int i = tid; i < kPlanWarps * E; i += kPlanThreads)
         cnt[i] = 0;
+    // every expert's total, and its picks in the chunks before this one
+    // (summed in chunk order)
+    for (int e = tid; e < E; e += kPlanThreads) {
+        int all = 0, before = 0;
+        for (int c = 0; c < n_chunks; ++c) {
+            const int v = a.chunk_count[(size_t)c * E + e];
+            before += c < chunk ? v : 0;
+            all += v;
+        }
+        total[e] = all;
+        goff[e] = before;
+    }
     __syncthreads();
-    // pass 1: per-warp histogram of the picks, in pick order
-    for (int64_t base = p_lo; base < p_hi; base += 32) {
-        const int64_t p = base + lane;
+    // per-warp histogram of the chunk's picks
+    {
+        const int64_t p = p_lo + lane;
         int e = -1;
         bool valid = false;
         if (p < p_hi) {
             e = a.ids[p];
             valid = e >= 0 && e < E;
-            if (!valid && e != kIdNone)
-                flag_status(kStatusBadId);
         }
         const int key = valid ? e : -(lane + 2);
         const uint32_t m = __match_any_sync(0xffffffffu, key);
         if (valid && lane == __ffs(m) - 1)
-            cnt[warp * E + e] += __popc(m);
+            cnt[warp * E + e] = __popc(m);
     }
-    __syncthreads();
-    for (int e = tid; e < E; e += kPlanThreads) {
-        int run = 0;
-        for (int w = 0; w < kPlanWarps; ++w) {
-            const int c = cnt[w * E + e];
-            cnt[w * E + e] = run;
-            run += c;
-        }
-        total[e] = run;
-    }
-    __syncthreads();
     // exclusive scan of the per-expert totals (E <= 1024 <= 2 * threads)
     {
         int v0 = 2 * tid < E ? total[2 * tid] : 0;
         int v1 = 2 * tid + 1 < E ? total[2 * tid + 1] : 0;
         const int all = block_exclusive_scan2(v0, v1, wsum);
+        // each expert's first row for this chunk: its group's start plus the
+        // earlier chunks' picks of it
         if (2 * tid < E)
-            goff[2 * tid] = v0;
+            goff[2 * tid] += v0;
         if (2 * tid + 1 < E)
-            goff[2 * tid + 1] = v1;
-        if (tid == 0) {
+            goff[2 * tid + 1] += v1;
+        if (chunk == 0 && tid == 0) {
             a.group_offset[E] = all;
             a.group_offset[E + 1] = (int)P;
         }
+        if (chunk == 0) {
+            if (2 * tid < E)
+                a.group_offset[2 * tid] = v0;
+            if (2 * tid + 1 < E)
+                a.group_offset[2 * tid + 1] = v1;
+        }
     }
     __syncthreads();
+    // each warp's first row per expert: the chunk's start plus the earlier
+    // warps' picks of it
     for (int e = tid; e < E; e += kPlanThreads) {
-        a.group_offset[e] = goff[e];
-        for (int w = 0; w < kPlanWarps; ++w)
-            cnt[w * E + e] += goff[e];
+        int run = goff[e];
+        for (int w = 0; w < kPlanWarps; ++w) {
+            const int c = cnt[w * E + e];
+            cnt[w * E + e] = run;
+            run += c;
+        }
     }
     __syncthreads();
-    // pass 2: stable scatter, same order as pass 1
-    for (int64_t base = p_lo; base < p_hi; base += 32) {
-        const int64_t p = base + lane;
+    // stable scatter: lane order inside a warp, warp order inside the chunk
+    {
+        const int64_t p = p_lo + lane;
         int e = -1;
         bool valid = false;
         if (p < p_hi) {
@@ -216,17 +263,11 @@ __global__ void __launch_bounds__(kPlanThreads, 1) group_plan_kernel(const PlanA
         }
         const int key = valid ? e : -(lane + 2);
         const uint32_t m = __match_any_sync(0xffffffffu, key);
-        int pos = 0;
         if (valid)
-            pos = cnt[warp * E + e] + __popc(m & ((1u << lane) - 1u));
-        __syncwarp();
-        if (valid) {
-            a.perm_pair[pos] = (int32_t)p;
-            if (lane == __ffs(m) - 1)
-                cnt[warp * E + e] += __popc(m);
-        }
-        __syncwarp();
+            a.perm_pair[cnt[warp * E + e] + __popc(m & ((1u << lane) - 1u))] = (int32_t)p;
     }
+    if (chunk != 0)
+        return;
     // tiles per group: routed groups, then the shared expert (all T rows)
     const int G = E + (a.I_s > 0 ? 1 : 0);
     {
@@ -945,10 +986,14 @@ inline ep_status grouped_forward(const GroupedArgs &g, const GroupedWorkspace &W
     pa.I = (int)I; pa.I_s = (int)I_s;
     pa.group_offset = group_offset; pa.perm_pair = perm_pair;
     pa.units_gu = units_gu; pa.units_dn = units_dn;
+    pa.chunk_count = reinterpret_cast<int32_t *>(ws + W.chunk_count);
+    const unsigned n_chunks = (unsigned)((P + kPlanThreads - 1) / kPlanThreads);
     bracket_event(ev, n_ev, 0, st);
-    const cudaError_t e_plan =
-        grouped_launch(g.pdl, group_plan_kernel, dim3(1), dim3(kPlanThreads), plan_smem_bytes(E),
-                       st, pa);
+    cudaError_t e_plan = grouped_launch(g.pdl, group_count_kernel, dim3(n_chunks),
+                                        dim3(kPlanThreads), (size_t)E * 4, st, pa);
+    if (e_plan == cudaSuccess)
+        e_plan = grouped_launch(g.pdl, group_plan_kernel, dim3(n_chunks), dim3(kPlanThreads),
+                                plan_smem_bytes(E), st, pa);
     bracket_event(ev, n_ev, 1, st);
     if (e_plan != cudaSuccess) {
         snprintf(why, why_len, "group_plan launch failed");
@@ -1032,7 +1077,7 @@ inline ep_status grouped_forward(const GroupedArgs &g, const GroupedWorkspace &W
             return EP_ECUDA;
         }
     }
-    *launches = 5;
+    *launches = 6;
     return EP_OK;
 }
 

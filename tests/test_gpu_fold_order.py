@@ -204,7 +204,7 @@ def test_y_is_the_host_fold_of_the_dumped_contributions(oracle_lib, name, T, pat
 @pytest.mark.parametrize("name,T,seed", [("prefill", 512, 1000), ("large", 4096, 1000),
                                          ("tiny", 300, 7)])
 def test_grouping_is_a_stable_sort_by_expert(name, T, seed):
-    """The grouped path's plan (group_plan_kernel: warp histograms, scans,
+    """The grouped path's plan (group_count_kernel, group_plan_kernel: chunk counts,
     stable scatter) against a host stable sort of the picks by expert id, bit
     for bit, with some empty, repeated and out-of-range ids mixed in."""
     wl = workloads.WORKLOADS[name]
