@@ -788,7 +788,6 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
     __shared__ int pick_e[16];
     __shared__ int order[16];
     __shared__ int n_valid;
-    grid_dependency_wait();  // c and s come from the previous kernel (launched early or not)
     const int64_t t = blockIdx.x;
     // the token's picks in ascending (expert id, slot): each valid pick's
     // place is the number of valid picks before it in that order (blockDim.x
@@ -815,6 +814,11 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
         n_valid = n;
     }
     __syncthreads();
+    // The ids were written before the previous kernel began (every kernel
+    // that launches this one early has passed its own wait on its
+    // predecessor, back to the router), so the order above was formed while
+    // the previous kernel ran; c and s come from that kernel.
+    grid_dependency_wait();
     const int h4 = blockIdx.y * blockDim.x + threadIdx.x;  // float4 column
     if (h4 * 4 >= H)
         return;
