@@ -25,8 +25,8 @@
  *         projection class).
  *
  * Readings where the pages are silent (router nonlinearity, tie-break, fold
- * order, where the shared expert enters) are the ones listed in the design
- * notes: softmax router with renormalised top-k, ties to the lower expert id,
+ * order, where the shared expert enters): softmax router with renormalised
+ * top-k, ties to the lower expert id,
  * picks folded in ascending (expert id, slot), the shared expert added after
  * the routed sum, routed scaling factor 1.  The GLM router variant of the
  * tracker page (a sigmoid score, a bias in the selection, weights from the
