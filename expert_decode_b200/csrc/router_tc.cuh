@@ -282,7 +282,10 @@ router_tc_kernel(const __grid_constant__ RcMaps maps, const uint16_t *__restrict
     // the partials are pushed to the CTAs that own their tokens
     tc_fence_before_sync();
     __syncthreads();
-    cluster_sync();
+    // an execution barrier only: what it orders (the copies into the stages
+    // and the MMAs reading them) has completed, as the mbarriers showed
+    cluster_arrive_relaxed();
+    cluster_wait();
     tc_fence_after_sync();
     // the owner of token t of the tile and t's row there
     static_assert(kRcNT == 64, "owner_of divides by 64");
