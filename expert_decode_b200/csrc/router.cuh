@@ -103,6 +103,52 @@ __device__ float kth_logit(const float *lt, int E, int top_k) {
     return vk;
 }
 
+// The k-th largest logits of two tokens at once (E <= 256), as kth_logit
+// computes each: the two selections interleave, so that each round's warp
+// reductions of one token overlap those of the other.
+__device__ void kth_logit2(const float *la, const float *lb, int E, int top_k, float &va,
+                           float &vb) {
+    const int lane = (int)lane_id();
+    uint32_t ka[8], kb[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int e = lane + 32 * i;
+        ka[i] = e < E ? order_key(la[e]) : 0u;
+        kb[i] = e < E ? order_key(lb[e]) : 0u;
+    }
+    int ca = 0, cb = 0;
+    bool da = false, db = false;
+    va = vb = -INFINITY;
+    for (int r = 0; r < top_k && !(da && db); ++r) {
+        uint32_t ma = ka[0], mb = kb[0];
+#pragma unroll
+        for (int i = 1; i < 8; ++i) {
+            ma = max(ma, ka[i]);
+            mb = max(mb, kb[i]);
+        }
+        ma = __reduce_max_sync(0xffffffffu, ma);
+        mb = __reduce_max_sync(0xffffffffu, mb);
+        uint32_t na = 0, nb = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            na += ka[i] == ma ? 1u : 0u;
+            ka[i] = ka[i] == ma ? 0u : ka[i];
+            nb += kb[i] == mb ? 1u : 0u;
+            kb[i] = kb[i] == mb ? 0u : kb[i];
+        }
+        ca += (int)__reduce_add_sync(0xffffffffu, na);
+        cb += (int)__reduce_add_sync(0xffffffffu, nb);
+        if (!da && (ma == 0u || ca >= top_k)) {
+            da = true;
+            va = ma == 0u ? -INFINITY : key_value(ma);
+        }
+        if (!db && (mb == 0u || cb >= top_k)) {
+            db = true;
+            vb = mb == 0u ? -INFINITY : key_value(mb);
+        }
+    }
+}
+
 // ------------------------------------------------------ compensated logits
 // A logit is a dot product of H terms x_h w_h.  With bf16 activations every
 // product is exact in fp32 (8 + 8 significant bits); with fp32 activations
@@ -647,10 +693,19 @@ __device__ void router_pick_owned(int n_local, int tbase, int tstride, int64_t t
     constexpr int XB = XF32 ? 4 : 2;
     const int warp = (int)(threadIdx.x >> 5), lane = (int)lane_id();
     // candidates per owned token (one warp each): every expert whose exact
-    // logit could reach the k-th largest under the bounds
+    // logit could reach the k-th largest under the bounds.  A warp's tokens
+    // j and j + NWARPS find their k-th logits together.
+    float vk_next = 0.f;
     for (int j = warp; j < n_local; j += NWARPS) {
         const float *lt = logit + j * E;
-        const float vk = kth_logit(lt, E, top_k);
+        float vk;
+        if (E <= 256 && ((j - warp) / NWARPS) % 2 == 1) {
+            vk = vk_next;  // found with the previous token's
+        } else if (E <= 256 && j + NWARPS < n_local) {
+            kth_logit2(lt, logit + (j + NWARPS) * E, E, top_k, vk, vk_next);
+        } else {
+            vk = kth_logit(lt, E, top_k);
+        }
         float dmax = 0.f;
         for (int e = lane; e < E; e += 32)
             dmax = fmaxf(dmax, bound_at(j, e));
