@@ -202,12 +202,16 @@ def test_y_is_the_host_fold_of_the_dumped_contributions(oracle_lib, name, T, pat
 
 
 @pytest.mark.parametrize("name,T,seed", [("prefill", 512, 1000), ("large", 4096, 1000),
-                                         ("tiny", 300, 7)])
+                                         ("tiny", 300, 7), ("many_experts", 333, 5)])
 def test_grouping_is_a_stable_sort_by_expert(name, T, seed):
     """The grouped path's plan (group_count_kernel, group_plan_kernel: chunk counts,
     stable scatter) against a host stable sort of the picks by expert id, bit
     for bit, with some empty, repeated and out-of-range ids mixed in."""
-    wl = workloads.WORKLOADS[name]
+    # many_experts: 1000 experts, top_k 7, so that T k = 2331 picks fall in
+    # three chunks of the plan (the last one ragged) over an expert count that
+    # is no power of two
+    wl = (workloads.Workload("many_experts", (T,), 128, 1000, 7, 64, 64, "bf16", "none", (1,))
+          if name == "many_experts" else workloads.WORKLOADS[name])
     W, x = device_inputs(wl, T, seed=seed)
     ids, w = ed.moe_route(x, W["w_router"], W["bias"], wl.top_k)
     ids = ids.clone()
