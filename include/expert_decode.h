@@ -421,7 +421,9 @@ int32_t ep_last_launch_count(void);
  * every kernel that a later moe_route / moe_ffn_forward call on this host
  * thread launches is bracketed on the call's stream by
  * cudaEventRecord(events[2j]) and cudaEventRecord(events[2j+1]), j counting
- * the kernels of that one call (kernels past n_events / 2 are not bracketed).
+ * the kernels of that one call (kernels past n_events / 2 are not bracketed;
+ * on the tensor-core path the two kernels of the grouping plan share one
+ * bracket, j = 0, so its brackets are plan, gather, gate/up, down, combine).
  * `events` are cudaEvent_t handles the caller created and owns; the array is
  * read at each call, so the caller may change its contents between calls.
  * Pass NULL (or n_events = 0) to stop.  EP_EINVAL for n_events < 0.
