@@ -10,7 +10,7 @@
 //    loads (128-byte swizzle, each CTA its own copy) of the router weights,
 //    one 128-expert box per MMA M tile (MT = 1 or 2), and of the 64 token
 //    rows; warp 1 issues tcgen05.mma (M = 128 experts, N = 64 tokens) into
-//    fp32 TMEM accumulators; warps 2..7 add up, from the same shared-memory
+//    fp32 TMEM accumulators; warps 2..15 add up, from the same shared-memory
 //    stages, each expert's and each token's sum of squares over the slice
 //    (a row's sum does not depend on the swizzle's order of its chunks).
 //  * Once every CTA of the cluster has finished its slice, warps 2..5 drain
@@ -43,14 +43,14 @@
 namespace epk {
 
 constexpr int kRcNT = 64;         // tokens per tile: the MMA's N
-constexpr int kRcThreads = 256;
+constexpr int kRcThreads = 512;
 constexpr int kRcMaxE = 256;      // two 128-expert M tiles at most
 constexpr int kRcMaxCand = 32;    // refined candidates per token
 constexpr int kRcMinCK = 2;
 constexpr int kRcMaxCK = 8;
 constexpr uint32_t kRcWBox = kGemmBM * kGemmBK * 2;  // 128 experts x 64 of H, 16 KB
 constexpr uint32_t kRcXBox = kRcNT * kGemmBK * 2;    // 64 tokens x 64 of H, 8 KB
-constexpr int kRcNormWarps = 6;                      // warps 2..7
+constexpr int kRcNormWarps = 14;                     // warps 2..15
 
 struct RcMaps {
     CUtensorMap w;  // W_router [E, H]: box 64 x 128
@@ -136,7 +136,7 @@ router_tc_kernel(const __grid_constant__ RcMaps maps, const uint16_t *__restrict
     const int own = (kRcNT + CK - 1) / CK;
     float *logit = recv;            // [own][E], in place of slice 0's rows
     float *bound = recv + own * E;  // [own][E], in place of slice 1's rows
-    bool have = false;              // the partial tile is in TMEM (warps 2..7)
+    bool have = false;              // the partial tile is in TMEM (warps 2..15)
 
     if (warp == 0 && lane < CK) {
         // where this CTA's rows of owner `lane` begin there, less the owner's
@@ -227,11 +227,11 @@ router_tc_kernel(const __grid_constant__ RcMaps maps, const uint16_t *__restrict
         // bytes each and contiguous (the swizzle only permutes the chunks of
         // a row), so a warp reads four rows at once, lane l taking chunk
         // l % 8 of row l / 8: 512 contiguous bytes, free of bank conflicts.
-        // Row quad g (rows 4g .. 4g + 3) goes to norm warp g mod 6; a lane
+        // Row quad g (rows 4g .. 4g + 3) goes to norm warp g mod 14; a lane
         // keeps one partial sum per quad it reads, and the eight lanes of a
         // row add theirs at the end.
-        constexpr int kMaxQuads = (2 * kGemmBM + kRcNT) / 4 / kRcNormWarps + 1;  // 14
-        const int nw = warp - 2;  // 0 .. 5
+        constexpr int kMaxQuads = (2 * kGemmBM + kRcNT) / 4 / kRcNormWarps + 1;
+        const int nw = warp - 2;  // 0 .. 13
         const int rows = MT * kGemmBM + kRcNT;
         const int quads = rows / 4;
         float2 sq[kMaxQuads];
