@@ -271,15 +271,22 @@ StreamingPlan streaming_fit(const DeviceInfo &d, int64_t T, int64_t H, int xb, i
     // is widened when it takes at most 64 KB
     p.xs_f32 = xb == 4 || T * H * 4 <= 64 * 1024;
     const int xsb = p.xs_f32 ? 4 : 2;
+    // The gate/up kernel keeps x in shared memory and reads nothing else
+    // through L1, so its ring may take all the shared memory there is.  Each
+    // slot has a single consumer warp: the slot count is the largest that
+    // fits and has at least six consumers (12: six, 16: eight), else the
+    // largest that fits with its most consumers (gate_up_consumers).
+    const size_t gu_budget = (size_t)d.smem_optin;
     int slots = epk::kGUMaxSlots;
-    while (slots >= 2 && epk::gate_up_smem_layout((int)T, (int)H, xsb, slots).total > budget)
+    while (slots >= 2 && epk::gate_up_smem_layout((int)T, (int)H, xsb, slots).total > gu_budget)
         --slots;
     if (slots < 2)
         return p;
-    // each gate/up slot has a single consumer warp: 8 warps share 8 or 16
-    // slots, and fewer slots than warps leave the extra warps idle
-    if (slots >= epk::kGUConsumerWarps)
-        slots = slots / epk::kGUConsumerWarps * epk::kGUConsumerWarps;
+    for (int s = slots; s >= 6; --s)
+        if (epk::gate_up_consumers(s) >= 6) {
+            slots = s;
+            break;
+        }
     p.gu_slots = slots;
     p.gu_smem = epk::gate_up_smem_layout((int)T, (int)H, xsb, slots).total;
     const int64_t I_max = std::max(I, I_s);

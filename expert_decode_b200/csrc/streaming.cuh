@@ -341,6 +341,15 @@ struct StreamGateUpArgs {
     float *h_shared;  // [T, I_s]
 };
 
+// Consumer warps of the gate/up kernel for NS slots: the most, up to
+// kGUConsumerWarps, that divide NS (task n goes to warp n % A and slot n % NS).
+__host__ __device__ inline int gate_up_consumers(int NS) {
+    for (int a = kGUConsumerWarps; a > 1; --a)
+        if (NS % a == 0)
+            return a;
+    return 1;
+}
+
 struct GateUpSmem {
     size_t plan, x, slots, bars, total;
 };
@@ -482,8 +491,8 @@ __global__ void __launch_bounds__(kGUThreads, 1) stream_gate_up_kernel(const Str
     // slot's phases in order.  (Were a slot shared by two warps, one could
     // wait for phase k + 1 while phase k is still in flight, and the parity
     // test would pass at once on the stale phase.)
-    // (the host sizes NS as 2..7, 8 or 16)
-    const int A = NS < kGUConsumerWarps ? NS : kGUConsumerWarps;
+    // (the host sizes NS so that such an A of several warps exists)
+    const int A = gate_up_consumers(NS);
     const int nck = H >> 3;
     const size_t xrow_bytes = (size_t)H * XSB;
     for (int n = w; w < A && n < ntask; n += A) {
