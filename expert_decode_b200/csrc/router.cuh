@@ -323,12 +323,12 @@ constexpr int kRdWarps = kRdThreads / 32;
 constexpr int kRdMaxTB = 2;
 
 struct RdSmem {
-    uint32_t x, vals, logit, keys, sel, total;
+    uint32_t x, vals, logit, total;
 };
 
-// Up to this many experts the small-batch router picks by a parallel rank
-// count (every (token, expert) key counts the keys above it); above, one
-// warp per token selects the top_k in top_k rounds.
+// Up to this many experts the small-batch router picks with the token's keys
+// in registers, two warp reductions a round; above, one warp per token
+// selects the top_k in top_k rounds of shuffles over shared memory.
 constexpr int kRdRankMaxE = 256;
 
 __host__ __device__ inline RdSmem rd_smem_layout(int tb_max, int H, int E) {
@@ -340,8 +340,6 @@ __host__ __device__ inline RdSmem rd_smem_layout(int tb_max, int H, int E) {
     // score (sigmoid)
     s.vals = o;  o = align_up_u32(o + 2u * tb_max * per_cta * 8, 16);
     s.logit = o; o = align_up_u32(o + 2u * tb_max * E * 8, 16);
-    s.keys = o;  o = align_up_u32(o + (uint32_t)tb_max * E * 8, 16);
-    s.sel = o;   o = align_up_u32(o + (uint32_t)tb_max * 16 * 4, 16);
     s.total = o;
     return s;
 }
@@ -473,34 +471,40 @@ router_dot2_kernel(const void *__restrict__ x, int64_t T, int H,
     if (rank != 0)
         return;
     if (E <= kRdRankMaxE) {
-        // the pick by rank: key (value, id) ranks r among the token's keys when
-        // r keys are above it; ranks below top_k are the picks, in order
-        unsigned long long *keys = reinterpret_cast<unsigned long long *>(smem + L.keys);
-        int *sel = reinterpret_cast<int *>(smem + L.sel);
-        for (int i = threadIdx.x; i < tb * E; i += kRdThreads) {
-            const int t = i / E, e = i - t * E;
-            keys[i] = topk_key(logit[t * E + e], e);
-        }
-        __syncthreads();
-        for (int i = threadIdx.x; i < tb * E; i += kRdThreads) {
-            const int t = i / E;
-            const unsigned long long k = keys[i];
-            const unsigned long long *kt = keys + t * E;
-            int r = 0;
-            for (int f = 0; f < E; ++f)
-                r += kt[f] > k ? 1 : 0;
-            if (r < top_k)
-                sel[t * 16 + r] = i - t * E;
-        }
-        __syncthreads();
+        // the pick by warp reductions: warp t holds token t's keys (value,
+        // id) in registers, eight per lane, and round r takes the largest
+        // (its high half by one reduction, then its low half among the lanes
+        // whose largest key shares that high half), which lane r keeps
         if (warp >= tb)
             return;
-        const int pick_e = lane < top_k ? sel[warp * 16 + lane] : 0;
+        const double *lt = logit + warp * E;
+        unsigned long long key[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int e = lane + 32 * i;
+            key[i] = e < E ? topk_key(lt[e], e) : 0ull;
+        }
+        int pick_e = 0;
+        for (int r = 0; r < top_k; ++r) {
+            unsigned long long m = key[0];
+#pragma unroll
+            for (int i = 1; i < 8; ++i)
+                m = key[i] > m ? key[i] : m;
+            const uint32_t hi = __reduce_max_sync(0xffffffffu, (uint32_t)(m >> 32));
+            const uint32_t lo =
+                __reduce_max_sync(0xffffffffu, (uint32_t)(m >> 32) == hi ? (uint32_t)m : 0u);
+            const unsigned long long best = ((unsigned long long)hi << 32) | lo;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                key[i] = key[i] == best ? 0ull : key[i];
+            if (lane == r)
+                pick_e = 1023 - (int)(lo & 0x3ffu);
+        }
         if constexpr (SIG) {
             sigmoid_finish_warp(logit + (TB + warp) * E, pick_e, top_k, normalize, scale,
                                 ids + (t0 + warp) * top_k, weights + (t0 + warp) * top_k);
         } else {
-            const double pick_v = lane < top_k ? logit[warp * E + pick_e] : 0.0;
+            const double pick_v = lane < top_k ? lt[pick_e] : 0.0;
             softmax_finish_warp(pick_e, pick_v, top_k, ids + (t0 + warp) * top_k,
                                 weights + (t0 + warp) * top_k);
         }
